@@ -1,0 +1,494 @@
+"""Oracle for one ALoDLM denoising step: a plain, slow CPU statement of the method.
+
+TEST INFRASTRUCTURE.  Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline /
+reference leg of ``bench.py`` may import or run this module.  The CUDA library never
+does, and this module imports nothing of it.
+
+Sources are the pages collected on ALoDLM.  Citations name the page and its section:
+
+* [digest]  "ALoDLM: Adaptively Looped Diffusion Language Models" (paper digest page).
+    - section "Core method" (核心方法): Prelude / Recurrent Core / Coda; each loop the
+      Core updates the state, the Coda reads out r^(s); r^(s) feeds the LMHead
+      (distribution, entropy commit H <= tau) and the ExitGate
+      lambda = sigmoid(ExitGate(sg[r])); the loop ends once the mean cumulative halt of
+      the unresolved positions reaches q, and s = K forces the exit.
+    - same section, Eq. 3: h_i^(s) = Emb(y_i) for a committed position, else h~_i^(s).
+    - section "Method steps" (方法步骤详情), Algorithm 1 steps (1)-(5).
+    - section "Technical novelty" (技术新颖性): depth-aware KV cache (matching depth first,
+      deepest available as fallback); the 8B path executes 10 + 4 x (16 + 10) = 114 layers.
+    - section "Prerequisites" (前置知识), KV-cache paragraph: the same physical layer gives
+      different KV at different loop depths.
+    - section "Limitations" (局限与改进): L + (K-1) m = 84 logical KV buffers for the 8B.
+    - section "Results" (实验结果): greedy decoding.
+* [summary] tokendh.com lay summary: two heads (token guess, "think again?"), committed
+  tokens become context, unresolved positions keep their internal state.
+
+Where the pages are silent the oracle takes these readings (each is also a reading
+of the CUDA library, stated in its header):
+
+* Layers are pre-norm Qwen3 decoder layers: RMSNorm, QKV, per-head RMSNorm of q and k,
+  rotate-half RoPE (base 1e6), softmax attention with grouped KV heads, output
+  projection, residual; RMSNorm, SwiGLU MLP, residual.
+* Prefill attention over the prefix is causal.  The block attends to every prefix
+  position and to every block position (bidirectional); the prefix never sees the block.
+* Positions: prefix 0..P-1, block P..P+N-1.
+* The Coda KV of the prefix is one set, computed from each position's exit-depth state.
+* Token choice is argmax (lowest id on ties); entropy is in nats over the full vocab.
+* "Emb" is the input embedding, unscaled.  The ExitGate is Linear(H -> 1) with bias,
+  applied to r^(s) (after the final RMSNorm).
+* Two commit rules (they differ on the role of the halting threshold):
+    PAPER      commit {i in U : H_i <= tau}; stop when U is empty, when the mean of a
+               over the remaining U reaches q (``lam``), or at s = K; if nothing was
+               committed in the whole step, commit the single lowest-entropy position
+               of the last loop (lowest index on ties); the rest stay [MASK].
+    PER_TOKEN  commit {i in U : H_i <= tau or a_i >= lam}, and all of U at s = K;
+               stop when U is empty.
+* a is updated for every i in U before the commit test; committed rows keep being
+  processed by Core and Coda in later loops with input Emb(y_i); block positions that
+  hold a given (non-mask) id are never in U and carry h~ like unresolved ones.
+
+Precision: ``precision="fp64"`` computes everything in float64 from the given weights.
+``precision="bf16"`` takes the decisions in the CUDA kernels' precision: every matrix
+weight and every operand of a matrix product (normed activations, q/k/v, attention
+probabilities, attention output, SwiGLU output, the readout state fed to the LM head)
+is rounded to bfloat16 (nearest, ties to even) at the point where the kernels round it;
+accumulation stays float64.  ``dtype=np.float32`` trades accuracy for speed at the
+Qwen3 shapes.
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, List, Optional
+
+import numpy as np
+
+RULE_PAPER = 0
+RULE_PER_TOKEN = 1
+
+
+# ----------------------------------------------------------------------------------
+# primitives
+# ----------------------------------------------------------------------------------
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Nearest bfloat16 value of x (via float32, ties to even), in x's float type."""
+    x = np.asarray(x)
+    f = np.ascontiguousarray(x, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return u.astype(np.uint32).view(np.float32).astype(x.dtype)
+
+
+def rmsnorm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) * g over the last axis."""
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * g
+
+
+def rope_cos_sin(positions: np.ndarray, head_dim: int, base: float, dtype) -> tuple:
+    """Rotary angles pos * base^(-2j/hd), j = 0..hd/2-1 (computed in float64)."""
+    j = np.arange(head_dim // 2, dtype=np.float64)
+    inv_freq = base ** (-2.0 * j / head_dim)
+    ang = positions.astype(np.float64)[:, None] * inv_freq[None, :]
+    return np.cos(ang).astype(dtype), np.sin(ang).astype(dtype)
+
+
+def apply_rope(x: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
+    """Rotate-half RoPE. x: [T, heads, hd]; cos/sin: [T, hd/2]."""
+    half = x.shape[-1] // 2
+    x1, x2 = x[..., :half], x[..., half:]
+    c, s = cos[:, None, :], sin[:, None, :]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def silu(x: np.ndarray) -> np.ndarray:
+    return x / (1.0 + np.exp(-x))
+
+
+def sigmoid(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, visible: np.ndarray,
+              bf16: bool) -> np.ndarray:
+    """softmax(q k^T / sqrt(hd)) v per query head; query head h reads KV head h // (nq/nkv).
+
+    q: [Tq, nq, hd]; k, v: [Tk, nkv, hd]; visible: [Tq, Tk] bool.
+    With bf16, the probabilities enter the value product rounded to bfloat16 while the
+    normaliser is the sum of the unrounded ones (the kernels' precision).
+    """
+    Tq, nq, hd = q.shape
+    nkv = k.shape[1]
+    group = nq // nkv
+    out = np.zeros((Tq, nq, hd), dtype=q.dtype)
+    scale = 1.0 / math.sqrt(hd)
+    for h in range(nq):
+        kh = h // group
+        s = (q[:, h, :] @ k[:, kh, :].T) * scale
+        s = np.where(visible, s, -np.inf)
+        s = s - s.max(axis=-1, keepdims=True)
+        p = np.exp(s)
+        denom = p.sum(axis=-1, keepdims=True)
+        pv = round_bf16(p) if bf16 else p
+        out[:, h, :] = (pv @ v[:, kh, :]) / denom
+    return out
+
+
+# ----------------------------------------------------------------------------------
+# the model
+# ----------------------------------------------------------------------------------
+
+class Oracle:
+    """ALoDLM inference, one sequence at a time, in plain NumPy.
+
+    cfg: dict with hidden, n_q_heads, n_kv_heads, head_dim, inter, vocab, n_prelude,
+    n_core, n_coda, k_max, rope_base, rms_eps, qk_norm, mask_id.
+    weights: {"embed" [V,H], "lm_head" [V,H], "final_norm" [H], "exit_w" [H],
+    "exit_b" float, "layers": list (model order) of {"attn_norm", "q", "k", "v", "o",
+    "q_norm", "k_norm", "mlp_norm", "gate", "up", "down"}} as float arrays
+    (row-major [out, in]).
+    """
+
+    def __init__(self, cfg: dict, weights: dict, precision: str = "fp64", dtype=np.float64):
+        assert precision in ("fp64", "bf16")
+        self.cfg = dict(cfg)
+        self.W = weights
+        self.bf16 = precision == "bf16"
+        self.dt = dtype
+        self.layer_execs = 0          # layer applications in the last denoise_step (per sequence, summed)
+        self._layer_cache: Dict[int, dict] = {}
+        n_params = sum(int(np.prod(np.shape(v))) for lw in self._layer_list() for v in lw.values())
+        self._cache_layers = n_params < 200_000_000
+        self.kv = None
+
+    # --- weights ------------------------------------------------------------------
+
+    def _layer_list(self):
+        L = self.W["layers"]
+        return L if isinstance(L, list) else [L[i] for i in sorted(L)]
+
+    def _mat(self, a):
+        a = np.asarray(a, dtype=self.dt)
+        return round_bf16(a) if self.bf16 else a
+
+    def _vec(self, a):
+        # norm gains and the ExitGate weight are float32 in the kernels: no bf16 rounding
+        return np.asarray(np.asarray(a, dtype=np.float32), dtype=self.dt)
+
+    def layer_weights(self, idx: int) -> dict:
+        if idx in self._layer_cache:
+            return self._layer_cache[idx]
+        src = self.W["layers"][idx]
+        lw = {k: (self._vec(v) if np.ndim(v) == 1 else self._mat(v)) for k, v in src.items()}
+        if self._cache_layers:
+            self._layer_cache[idx] = lw
+        return lw
+
+    def _global(self, key):
+        if ("g", key) not in self._layer_cache:
+            v = self.W[key]
+            self._layer_cache[("g", key)] = self._vec(v) if np.ndim(v) == 1 else self._mat(v)
+        return self._layer_cache[("g", key)]
+
+    def _act(self, x):
+        return round_bf16(x) if self.bf16 else x
+
+    # --- slots of the depth-aware KV cache ---------------------------------------------
+    # [digest] "Technical novelty" and "Prerequisites": a shared Core layer produces a
+    # different KV at every loop depth, so the cache keeps one buffer per (Core layer,
+    # depth) beside one per Prelude and per Coda layer.
+
+    def n_kv_slots(self, k_max: Optional[int] = None) -> int:
+        c = self.cfg
+        K = c["k_max"] if k_max is None else k_max
+        return c["n_prelude"] + K * c["n_core"] + c["n_coda"]
+
+    def core_layer_index(self, j: int) -> int:
+        return self.cfg["n_prelude"] + j
+
+    def coda_layer_index(self, j: int) -> int:
+        return self.cfg["n_prelude"] + self.cfg["n_core"] + j
+
+    # --- one decoder layer -------------------------------------------------------------
+
+    def qkv(self, lw: dict, h: np.ndarray, positions: np.ndarray):
+        """Normed input -> (q, k, v) after the per-head norms and RoPE."""
+        c = self.cfg
+        nq, nkv, hd = c["n_q_heads"], c["n_kv_heads"], c["head_dim"]
+        x = self._act(rmsnorm(h, lw["attn_norm"], c["rms_eps"]))
+        q = (x @ lw["q"].T).reshape(-1, nq, hd)
+        k = (x @ lw["k"].T).reshape(-1, nkv, hd)
+        v = (x @ lw["v"].T).reshape(-1, nkv, hd)
+        if c["qk_norm"]:
+            q = rmsnorm(q, lw["q_norm"], c["rms_eps"])
+            k = rmsnorm(k, lw["k_norm"], c["rms_eps"])
+        cos, sin = rope_cos_sin(positions, hd, c["rope_base"], self.dt)
+        q = apply_rope(q, cos, sin)
+        k = apply_rope(k, cos, sin)
+        return self._act(q), self._act(k), self._act(v)
+
+    def finish_layer(self, lw: dict, h: np.ndarray, q, k_all, v_all, visible) -> np.ndarray:
+        """Attention over (k_all, v_all), output projection, residual, SwiGLU MLP, residual."""
+        c = self.cfg
+        o = attention(q, k_all, v_all, visible, self.bf16)
+        o = self._act(o.reshape(o.shape[0], -1))
+        h = h + o @ lw["o"].T
+        x = self._act(rmsnorm(h, lw["mlp_norm"], c["rms_eps"]))
+        a = self._act(silu(x @ lw["gate"].T) * (x @ lw["up"].T))
+        return h + a @ lw["down"].T
+
+    # --- prefill: the depth-aware KV cache ---------------------------------------------
+
+    def prefill(self, prefix_ids: np.ndarray, exit_depth: Optional[np.ndarray] = None) -> dict:
+        """Build the depth-aware KV cache of the prefix.
+
+        [digest] "Technical novelty"/"Prerequisites": each prefix position is served at the
+        matching loop depth, falling back to the deepest depth it reached.  Position j with
+        exit depth e_j runs the Core e_j times; for depth d > e_j its Core KV is its depth-e_j
+        KV.  Keys at Core depth d are therefore read at depth min(d, e_k).  The Coda runs
+        once, on each position's depth-e_j state.  Attention is causal over the prefix.
+
+        Stores self.kv[b][("prelude", l) | ("core", c, d) | ("coda", j)] = (K, V), each
+        [P, nkv, hd]; returns it.
+        """
+        c = self.cfg
+        K = c["k_max"]
+        prefix_ids = np.asarray(prefix_ids)
+        B, P = prefix_ids.shape
+        if exit_depth is None:
+            exit_depth = np.full((B, P), K, dtype=np.int64)
+        exit_depth = np.asarray(exit_depth)
+        assert exit_depth.min() >= 1 and exit_depth.max() <= K
+        emb = self._global("embed")
+        pos = np.arange(P)
+        causal = pos[None, :] <= pos[:, None]
+        self.kv = []
+        for b in range(B):
+            kv = {}
+            h = emb[prefix_ids[b]].astype(self.dt)
+            for l in range(c["n_prelude"]):
+                lw = self.layer_weights(l)
+                q, k, v = self.qkv(lw, h, pos)
+                kv[("prelude", l)] = (k, v)
+                h = self.finish_layer(lw, h, q, k, v, causal)
+            e = exit_depth[b]
+            h_exit = h.copy()
+            for d in range(1, K + 1):
+                act = np.nonzero(e >= d)[0]
+                for j in range(c["n_core"]):
+                    lw = self.layer_weights(self.core_layer_index(j))
+                    if d == 1:
+                        k_d = np.zeros((P, c["n_kv_heads"], c["head_dim"]), dtype=self.dt)
+                        v_d = np.zeros_like(k_d)
+                    else:
+                        # positions that stopped before depth d keep their deepest KV
+                        k_d, v_d = (x.copy() for x in kv[("core", j, d - 1)])
+                    kv[("core", j, d)] = (k_d, v_d)
+                    if len(act) == 0:
+                        continue
+                    q, k, v = self.qkv(lw, h[act], pos[act])
+                    k_d[act], v_d[act] = k, v
+                    h[act] = self.finish_layer(lw, h[act], q, k_d, v_d, causal[act])
+                h_exit[e == d] = h[e == d]
+            h = h_exit
+            for j in range(c["n_coda"]):
+                lw = self.layer_weights(self.coda_layer_index(j))
+                q, k, v = self.qkv(lw, h, pos)
+                kv[("coda", j)] = (k, v)
+                h = self.finish_layer(lw, h, q, k, v, causal)
+            self.kv.append(kv)
+        self.prefix_len = P
+        return self.kv
+
+    # --- one layer over the block against the cached prefix ----------------------------
+
+    def block_layer(self, b: int, key, lw: dict, h: np.ndarray) -> np.ndarray:
+        """The block attends to every cached prefix position (slot ``key``) and to itself."""
+        P = self.prefix_len
+        N = h.shape[0]
+        pos = P + np.arange(N)
+        q, k, v = self.qkv(lw, h, pos)
+        kp, vp = self.kv[b][key]
+        k_all = np.concatenate([kp, k], axis=0)
+        v_all = np.concatenate([vp, v], axis=0)
+        visible = np.ones((N, P + N), dtype=bool)
+        self.layer_execs += 1
+        return self.finish_layer(lw, h, q, k_all, v_all, visible)
+
+    def readout(self, r: np.ndarray):
+        """LMHead and ExitGate on readout states r [n, H].
+
+        [digest] "Core method": p_i = softmax(LMHead(r_i)); entropy H_i = -sum p log p (nats);
+        lambda_i = sigmoid(ExitGate(r_i)).  Returns (H, y = argmax, lam, z = logits).
+        """
+        W = self._global("lm_head")
+        z = self._act(r) @ W.T
+        m = z.max(axis=-1, keepdims=True)
+        logZ = m + np.log(np.exp(z - m).sum(axis=-1, keepdims=True))
+        logp = z - logZ
+        p = np.exp(logp)
+        H = -(p * logp).sum(axis=-1)
+        y = np.argmax(z, axis=-1)
+        g = r @ self._global("exit_w") + float(self.W["exit_b"])
+        return H, y, sigmoid(g), z
+
+    def merge(self, committed: np.ndarray, tok: np.ndarray, h_tilde: np.ndarray) -> np.ndarray:
+        """[digest] Eq. 3: h_i^(s) = Emb(y_i) for a committed position, h~_i^(s) otherwise."""
+        emb = self._global("embed")
+        return np.where(committed[:, None], emb[tok], h_tilde)
+
+    # --- the denoising step --------------------------------------------------------------
+
+    def denoise_step(self, block_ids: np.ndarray, tau: float, lam: float, k_max: int,
+                     rule: int = RULE_PAPER, follow: Optional[dict] = None, band: float = 1e-3,
+                     logit_rows: Optional[List[tuple]] = None) -> dict:
+        """One denoising step, [digest] "Method steps" Algorithm 1 (1)-(5) and Eq. 3.
+
+        block_ids [B, N]; positions holding mask_id form U.  ``lam`` is the halting
+        threshold (q in the pages).  ``follow`` (optional) holds another run's decisions
+        {"tokens" [B,N], "exit_depth" [B,N], "loops_run" [B]}: at a decision whose deciding
+        value lies within ``band`` of its threshold (or whose top-two gap is below ``band``),
+        the oracle takes that run's decision and records it in "followed"; band=inf follows
+        every decision.  ``logit_rows``: (b, s, i) triples whose logits are returned.
+
+        Returns tokens, exit_depth, entropy/halt/cum_halt [B,K,N] (NaN where not computed),
+        loops_run [B], active_rows [K], readout_rows [K]; per sequence b, lists of
+        [loops, N, H] arrays: r (readout states r^(s)), h_in (loop inputs h^(s-1)) and
+        h_tilde (Core outputs); logits {(b,s,i): z}, followed, committed_per_step [B].
+        """
+        c = self.cfg
+        assert self.kv is not None, "prefill first"
+        assert 1 <= k_max <= c["k_max"]
+        block_ids = np.asarray(block_ids)
+        B, N = block_ids.shape
+        K = k_max
+        mask_id = c["mask_id"]
+        emb = self._global("embed")
+        nan = np.full((B, K, N), np.nan)
+        out = dict(tokens=block_ids.astype(np.int64).copy(), exit_depth=np.zeros((B, N), np.int64),
+                   entropy=nan.copy(), halt=nan.copy(), cum_halt=nan.copy(),
+                   loops_run=np.zeros(B, np.int64), active_rows=np.zeros(K, np.int64),
+                   readout_rows=np.zeros(K, np.int64), r=[], h_in=[], h_tilde=[], logits={}, followed=[],
+                   committed_per_step=np.zeros(B, np.int64))
+        want_logits = set(logit_rows or [])
+        self.layer_execs = 0
+
+        def near(x, thr):
+            return follow is not None and abs(float(x) - float(thr)) < band
+
+        for b in range(B):
+            # (1) U = masked positions; h^(0) = Prelude(x); a = 0; C = empty
+            U = block_ids[b] == mask_id
+            tok = block_ids[b].astype(np.int64).copy()
+            committed = np.zeros(N, dtype=bool)
+            a = np.zeros(N, dtype=self.dt)
+            h = emb[block_ids[b]].astype(self.dt)
+            for l in range(c["n_prelude"]):
+                h = self.block_layer(b, ("prelude", l), self.layer_weights(l), h)
+            rs, h_ins, h_tildes = [], [], []
+            n_committed = 0
+            last_H = None
+            s_last = 0
+            for s in range(1, K + 1):
+                s_last = s
+                out["active_rows"][s - 1] += N
+                # (2) h~ = Core(h^(s-1)) against prefix Core KV at depth s; r = Coda(h~)
+                h_ins.append(h)
+                ht = h
+                for j in range(c["n_core"]):
+                    ht = self.block_layer(b, ("core", j, s), self.layer_weights(self.core_layer_index(j)), ht)
+                h_tildes.append(ht)
+                hc = ht
+                for j in range(c["n_coda"]):
+                    hc = self.block_layer(b, ("coda", j), self.layer_weights(self.coda_layer_index(j)), hc)
+                r = rmsnorm(hc, self._global("final_norm"), c["rms_eps"])
+                rs.append(r)
+                idx = np.nonzero(U)[0]
+                out["readout_rows"][s - 1] += len(idx)
+                H, y, lmb, z = self.readout(r[idx])
+                for t, i in enumerate(idx):
+                    if (b, s, int(i)) in want_logits:
+                        out["logits"][(b, s, int(i))] = z[t]
+                # (4) cumulative halting a <- a + (1 - a) lambda, for every i in U
+                a[idx] = a[idx] + (1.0 - a[idx]) * lmb
+                out["entropy"][b, s - 1, idx] = H
+                out["halt"][b, s - 1, idx] = lmb
+                out["cum_halt"][b, s - 1, idx] = a[idx]
+                last_H = dict(zip(idx.tolist(), H.tolist()))
+                # greedy token choice, lowest id on ties
+                y = y.astype(np.int64).copy()
+                if follow is not None:
+                    for t in range(len(idx)):
+                        top2 = np.partition(z[t], -2)[-2:]
+                        if top2[1] - top2[0] < band:
+                            i = int(idx[t])
+                            if follow["exit_depth"][b, i] == s:
+                                out["followed"].append(dict(b=b, s=s, i=i, kind="argmax",
+                                                            margin=float(top2[1] - top2[0])))
+                                y[t] = int(follow["tokens"][b, i])
+                # (3) commit set B^(s)
+                commit = np.zeros(len(idx), dtype=bool)
+                for t, i in enumerate(idx):
+                    ent_ok = H[t] <= tau
+                    if rule == RULE_PAPER:
+                        dec = ent_ok
+                        is_near = near(H[t], tau)
+                        margin = H[t] - tau
+                    else:
+                        halt_ok = a[i] >= lam
+                        dec = ent_ok or halt_ok or s == K
+                        is_near = s < K and (near(H[t], tau) or near(a[i], lam))
+                        margin = min(abs(H[t] - tau), abs(a[i] - lam))
+                    if is_near:
+                        gpu = bool(follow["exit_depth"][b, i] == s)
+                        out["followed"].append(dict(b=b, s=s, i=int(i), kind="commit",
+                                                    margin=float(margin), own=bool(dec), taken=gpu))
+                        dec = gpu
+                    commit[t] = dec
+                ci = idx[commit]
+                tok[ci] = y[commit]
+                out["exit_depth"][b, ci] = s
+                U[ci] = False
+                committed[ci] = True
+                n_committed += len(ci)
+                h = self.merge(committed, tok, ht)
+                # (4) halting
+                if not U.any():
+                    break
+                if rule == RULE_PAPER:
+                    mean_a = float(np.mean(a[U]))
+                    stop = mean_a >= lam
+                    if near(mean_a, lam):
+                        gpu = bool(follow["loops_run"][b] == s)
+                        out["followed"].append(dict(b=b, s=s, i=-1, kind="halt",
+                                                    margin=float(mean_a - lam), own=stop, taken=gpu))
+                        stop = gpu
+                    if stop:
+                        break
+            # (5) forced progress: nothing committed in this step -> lowest entropy of the last loop
+            if rule == RULE_PAPER and n_committed == 0 and U.any():
+                cand = sorted(last_H.items(), key=lambda kv: (kv[1], kv[0]))
+                i_star = cand[0][0]
+                if follow is not None and len(cand) > 1 and cand[1][1] - cand[0][1] < band:
+                    gpu_i = [i for i in last_H if follow["exit_depth"][b, i] == s_last]
+                    out["followed"].append(dict(b=b, s=s_last, i=int(i_star), kind="forced",
+                                                margin=float(cand[1][1] - cand[0][1])))
+                    if gpu_i:
+                        i_star = gpu_i[0]
+                z_star = self.readout(rs[-1][[i_star]])[3][0]
+                y_star = int(np.argmax(z_star))
+                if follow is not None and follow["exit_depth"][b, i_star] == s_last:
+                    top2 = np.partition(z_star, -2)[-2:]
+                    if top2[1] - top2[0] < band:
+                        y_star = int(follow["tokens"][b, i_star])
+                tok[i_star] = y_star
+                out["exit_depth"][b, i_star] = s_last
+                U[i_star] = False
+                n_committed = 1
+            out["tokens"][b] = tok
+            out["loops_run"][b] = s_last
+            out["committed_per_step"][b] = n_committed
+            out["r"].append(np.stack(rs))
+            out["h_in"].append(np.stack(h_ins))
+            out["h_tilde"].append(np.stack(h_tildes))
+        return out
