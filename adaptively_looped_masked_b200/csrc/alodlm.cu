@@ -1,0 +1,949 @@
+// alodlm.cu — host side of the ALoDLM denoising-step library: the C ABI declared in
+// include/alodlm.h, weight packing, the depth-aware KV arena, the prefill schedule and the
+// looped denoising step.  Every step of the path runs in the kernels of this directory;
+// the host only sizes launches and reads a 16-byte loop-control word per loop.
+#include "../../include/alodlm.h"
+
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "attention.cuh"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "kernels.cuh"
+
+namespace {
+
+constexpr int NUM_SMS_HINT = 148;
+constexpr int PREFILL_ROWS = 16384;         // rows of one prefill group (sequences x P)
+constexpr size_t SPLITK_WS_FLOATS = 32u << 20;  // split-K partials (128 MB)
+constexpr size_t ATTN_WS_FLOATS = 16u << 20;    // split-KV partials (64 MB)
+
+enum KClass { KC_GEMM = 0, KC_ATTN, KC_RGEMM, KC_RCOMB, KC_NORM, KC_QKV, KC_COMMIT, KC_OTHER };
+const char *kclass_names[ALODLM_N_KCLASS] = {"gemm", "attention", "readout_gemm", "readout_combine",
+                                             "norm", "qkv_rope", "commit", "other"};
+
+std::mutex g_err_mu;
+std::string g_create_err;
+
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------------------------
+// TMA descriptors (driver entry point fetched through the runtime)
+// ---------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2D bf16 tensor [rows, inner] row-major, box [box_rows, 64], 128-byte swizzle, zero OOB fill
+bool make_tmap(CUtensorMap *map, const void *ptr, int inner, int rows, int box_rows) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)inner * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// one-time per device: opt the big-shared-memory kernels in
+template <int BN, int EPI>
+void set_gemm_attr() {
+    cudaFuncSetAttribute(gemm::gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)gemm::Cfg<BN>::SMEM);
+}
+bool init_kernel_attrs() {
+    static bool done[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return false;
+    if (done[dev]) return true;
+    set_gemm_attr<32, gemm::EPI_F32>();
+    set_gemm_attr<32, gemm::EPI_ADD>();
+    set_gemm_attr<32, gemm::EPI_SWIGLU>();
+    set_gemm_attr<64, gemm::EPI_F32>();
+    set_gemm_attr<64, gemm::EPI_ADD>();
+    set_gemm_attr<64, gemm::EPI_SWIGLU>();
+    set_gemm_attr<128, gemm::EPI_F32>();
+    set_gemm_attr<128, gemm::EPI_ADD>();
+    set_gemm_attr<128, gemm::EPI_SWIGLU>();
+    set_gemm_attr<256, gemm::EPI_F32>();
+    set_gemm_attr<256, gemm::EPI_ADD>();
+    set_gemm_attr<256, gemm::EPI_SWIGLU>();
+    set_gemm_attr<256, gemm::EPI_READOUT>();
+    cudaFuncSetAttribute(attn::attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 5 * 64 * 64 * 2);
+    cudaFuncSetAttribute(attn::attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 5 * 64 * 128 * 2);
+    done[dev] = cudaGetLastError() == cudaSuccess;
+    return done[dev];
+}
+
+int pick_bn(int M) { return M <= 32 ? 32 : (M <= 64 ? 64 : (M <= 128 ? 128 : 256)); }
+
+struct GemmShape {
+    int bn, splits, kps, k_tiles;
+};
+
+// Tile/split choice: enough CTAs to cover the SMs (memory-bound small-M launches), at least
+// four k-tiles per split, partials within the workspace.
+GemmShape plan_gemm(int M, int Nw, int K, size_t ws_floats) {
+    GemmShape g;
+    g.bn = pick_bn(M);
+    g.k_tiles = cdiv(K, gemm::BK);
+    const int tiles = cdiv(Nw, gemm::BM) * cdiv(M, g.bn);
+    const int per_sm = g.bn <= 64 ? 2 : 1;
+    int splits = (NUM_SMS_HINT * per_sm) / tiles;
+    splits = std::max(1, std::min(splits, g.k_tiles / 4));
+    while (splits > 1 && (size_t)splits * M * Nw > ws_floats) --splits;
+    g.kps = cdiv(g.k_tiles, splits);
+    g.splits = cdiv(g.k_tiles, g.kps);
+    return g;
+}
+
+template <int BN, int EPI>
+void launch_gemm_bn(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int rowsB, int k_tiles, int kps,
+                    int splits, int a_fastest, const gemm::EpiParams &ep, int *err, cudaStream_t st) {
+    dim3 grid;
+    const int ta = cdiv(rowsA, gemm::BM), tb = cdiv(rowsB, BN);
+    grid = a_fastest ? dim3(ta, tb, splits) : dim3(tb, ta, splits);
+    gemm::gemm_tc_kernel<BN, EPI><<<grid, 192, gemm::Cfg<BN>::SMEM, st>>>(tA, tB, rowsA, rowsB, k_tiles, kps,
+                                                                           a_fastest, ep, err);
+}
+
+template <int EPI>
+void launch_gemm_epi(int bn, const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int rowsB, int k_tiles, int kps,
+                     int splits, int a_fastest, const gemm::EpiParams &ep, int *err, cudaStream_t st) {
+    switch (bn) {
+        case 32: launch_gemm_bn<32, EPI>(tA, tB, rowsA, rowsB, k_tiles, kps, splits, a_fastest, ep, err, st); break;
+        case 64: launch_gemm_bn<64, EPI>(tA, tB, rowsA, rowsB, k_tiles, kps, splits, a_fastest, ep, err, st); break;
+        case 128: launch_gemm_bn<128, EPI>(tA, tB, rowsA, rowsB, k_tiles, kps, splits, a_fastest, ep, err, st); break;
+        default: launch_gemm_bn<256, EPI>(tA, tB, rowsA, rowsB, k_tiles, kps, splits, a_fastest, ep, err, st); break;
+    }
+}
+
+void launch_splitk_reduce(int epi, const float *ws, int splits, long long sstride, int rowsA, int rowsB,
+                          const gemm::EpiParams &ep, cudaStream_t st) {
+    const long long total = (long long)rowsA * rowsB;
+    const int blocks = (int)std::min<long long>((total + 255) / 256, 148 * 8);
+    if (epi == gemm::EPI_ADD)
+        gemm::splitk_reduce_kernel<gemm::EPI_ADD><<<blocks, 256, 0, st>>>(ws, splits, sstride, rowsA, rowsB, ep);
+    else if (epi == gemm::EPI_SWIGLU)
+        gemm::splitk_reduce_kernel<gemm::EPI_SWIGLU><<<blocks, 256, 0, st>>>(ws, splits, sstride, rowsA, rowsB, ep);
+    else
+        gemm::splitk_reduce_kernel<gemm::EPI_F32><<<blocks, 256, 0, st>>>(ws, splits, sstride, rowsA, rowsB, ep);
+}
+
+struct LayerDev {
+    bf16 *wqkv = nullptr, *wo = nullptr, *wgu = nullptr, *wd = nullptr;
+    float *attn_norm = nullptr, *mlp_norm = nullptr, *q_norm = nullptr, *k_norm = nullptr;
+    CUtensorMap tm_qkv, tm_o, tm_gu, tm_d;
+};
+
+struct TimedLaunch {
+    int cls;
+    cudaEvent_t e0, e1;
+};
+
+}  // namespace
+
+// ---------------------------------------------------------------------------------
+// the handle
+// ---------------------------------------------------------------------------------
+struct alodlm {
+    alodlm_cfg cfg;
+    cudaStream_t stream = nullptr;
+    int device = 0;
+    std::string err;
+    std::vector<void *> allocs;
+    size_t alloc_bytes = 0;
+
+    // model
+    int H = 0, nq = 0, nkv = 0, hd = 0, I = 0, V = 0, L = 0, n_qkv = 0;
+    bf16 *embed = nullptr, *lm_head = nullptr;
+    float *final_norm = nullptr, *exit_w = nullptr;
+    float exit_b = 0.f;
+    std::vector<LayerDev> layers;
+    CUtensorMap tm_lm;
+
+    // depth-aware KV arena: [slot][b][kvh][pos][hd]
+    bf16 *kv_k = nullptr, *kv_v = nullptr;
+    int n_slots = 0, pos_stride = 0;
+    long long head_stride = 0, seq_stride = 0, slot_elems = 0;
+    float2 *rope = nullptr;
+
+    // prefill state
+    int B = 0, P = 0, last_N = 0;
+    bool prefilled = false;
+    int *exit_dev = nullptr;
+    int *iota = nullptr;
+
+    // activation scratch (rows_cap rows)
+    int rows_cap = 0, step_rows_cap = 0;
+    float *hbuf[2] = {nullptr, nullptr}, *hc = nullptr, *hexit = nullptr, *qkv = nullptr;
+    bf16 *xn = nullptr, *qb = nullptr, *attn_out = nullptr, *act = nullptr;
+    float *ws = nullptr, *aws_o = nullptr, *aws_ml = nullptr;
+
+    // readout
+    int R_cap = 0, n_vt = 0;
+    bf16 *rb = nullptr;
+    float *lam_rr = nullptr;
+    float4 *part = nullptr;
+    int *ridx = nullptr, *rr_b = nullptr, *rr_i = nullptr;
+    CUtensorMap tm_rb;
+
+    // step state
+    unsigned char *U = nullptr;
+    float *a = nullptr, *cur_H = nullptr;
+    int *cur_y = nullptr, *cont = nullptr, *ncommit = nullptr;
+    int *seq_of[2] = {nullptr, nullptr}, *old_slot = nullptr;
+    int *counts = nullptr, *counts_host = nullptr, *d_err = nullptr;
+
+    // debug copies [K][maxB][maxN][H]
+    float *dbg[3] = {nullptr, nullptr, nullptr};
+
+    // activation tensor maps by (pointer, inner, rows, box rows)
+    std::map<std::tuple<const void *, int, int, int>, CUtensorMap> tmcache;
+
+    // launch accounting
+    int launches = 0;
+    bool timing = false;
+    std::vector<cudaEvent_t> ev_pool;
+    size_t ev_next = 0;
+    std::vector<TimedLaunch> timed;
+    double cls_bytes[ALODLM_N_KCLASS] = {0}, cls_flops[ALODLM_N_KCLASS] = {0};
+    int cls_launches[ALODLM_N_KCLASS] = {0};
+    cudaEvent_t pending_e0 = nullptr;
+};
+
+namespace {
+
+int fail(alodlm *h, int code, const std::string &msg) {
+    if (h)
+        h->err = msg;
+    else {
+        std::lock_guard<std::mutex> lk(g_err_mu);
+        g_create_err = msg;
+    }
+    return code;
+}
+
+int cuda_fail(alodlm *h, cudaError_t e, const char *what) {
+    return fail(h, ALODLM_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+template <typename T>
+int dalloc(alodlm *h, T **p, size_t count) {
+    const size_t bytes = std::max<size_t>(count * sizeof(T), 256);
+    if (h->cfg.mem_limit_bytes && h->alloc_bytes + bytes > h->cfg.mem_limit_bytes)
+        return fail(h, ALODLM_ENOMEM, "allocation would pass cfg.mem_limit_bytes");
+    void *q = nullptr;
+    cudaError_t e = cudaMalloc(&q, bytes);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(h, ALODLM_ENOMEM, std::string("cudaMalloc: ") + cudaGetErrorString(e));
+    }
+    h->allocs.push_back(q);
+    h->alloc_bytes += bytes;
+    *p = static_cast<T *>(q);
+    return ALODLM_OK;
+}
+
+// launch bookkeeping: count, optional CUDA-event timing per kernel class, algorithmic work
+void kbegin(alodlm *h) {
+    if (!h->timing) return;
+    if (h->ev_next + 2 > h->ev_pool.size()) {
+        for (int i = 0; i < 64; ++i) {
+            cudaEvent_t e;
+            cudaEventCreate(&e);
+            h->ev_pool.push_back(e);
+        }
+    }
+    h->pending_e0 = h->ev_pool[h->ev_next++];
+    cudaEventRecord(h->pending_e0, h->stream);
+}
+void kend(alodlm *h, int cls, double bytes, double flops) {
+    h->launches++;
+    h->cls_bytes[cls] += bytes;
+    h->cls_flops[cls] += flops;
+    h->cls_launches[cls]++;
+    if (!h->timing) return;
+    cudaEvent_t e1 = h->ev_pool[h->ev_next++];
+    cudaEventRecord(e1, h->stream);
+    h->timed.push_back({cls, h->pending_e0, e1});
+}
+void reset_stats(alodlm *h) {
+    h->launches = 0;
+    h->ev_next = 0;
+    h->timed.clear();
+    for (int c = 0; c < ALODLM_N_KCLASS; ++c) {
+        h->cls_bytes[c] = h->cls_flops[c] = 0;
+        h->cls_launches[c] = 0;
+    }
+}
+
+#define LAUNCH(cls, bytes, flops, ...)   \
+    do {                                 \
+        kbegin(h);                       \
+        __VA_ARGS__;                     \
+        kend(h, cls, (bytes), (flops));  \
+    } while (0)
+
+const CUtensorMap *act_map(alodlm *h, const void *ptr, int inner, int rows, int box_rows) {
+    auto key = std::make_tuple(ptr, inner, rows, box_rows);
+    auto it = h->tmcache.find(key);
+    if (it != h->tmcache.end()) return &it->second;
+    CUtensorMap m;
+    if (!make_tmap(&m, ptr, inner, rows, box_rows)) return nullptr;
+    return &(h->tmcache[key] = m);
+}
+
+// C = act[M, K] x W[Nw, K]^T with a fused epilogue (weights on the MMA's M side)
+int linear(alodlm *h, const CUtensorMap &tmW, int Nw, const bf16 *actp, int M, int K, int epi, float *out, int ldo,
+           bf16 *act_out, int ld_act) {
+    GemmShape g = plan_gemm(M, Nw, K, SPLITK_WS_FLOATS);
+    const CUtensorMap *tB = act_map(h, actp, K, h->rows_cap, g.bn);
+    if (!tB) return fail(h, ALODLM_ECUDA, "cuTensorMapEncodeTiled failed (activation)");
+    const double bytes = 2.0 * Nw * K + 2.0 * M * K +
+                         (epi == gemm::EPI_ADD ? 8.0 : (epi == gemm::EPI_SWIGLU ? 1.0 : 4.0)) * M * Nw;
+    const double flops = 2.0 * M * Nw * K;
+    gemm::EpiParams ep{};
+    if (g.splits == 1) {
+        ep.out = out;
+        ep.ldo = ldo;
+        ep.split_stride = 0;
+        ep.act = act_out;
+        ep.ld_act = ld_act;
+        switch (epi) {
+            case gemm::EPI_F32:
+                LAUNCH(KC_GEMM, bytes, flops,
+                       launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, 1, 0, ep, h->d_err,
+                                                      h->stream));
+                break;
+            case gemm::EPI_ADD:
+                LAUNCH(KC_GEMM, bytes, flops,
+                       launch_gemm_epi<gemm::EPI_ADD>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, 1, 0, ep, h->d_err,
+                                                      h->stream));
+                break;
+            default:
+                LAUNCH(KC_GEMM, bytes, flops,
+                       launch_gemm_epi<gemm::EPI_SWIGLU>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, 1, 0, ep, h->d_err,
+                                                         h->stream));
+                break;
+        }
+    } else {
+        ep.out = h->ws;
+        ep.ldo = Nw;
+        ep.split_stride = (long long)M * Nw;
+        LAUNCH(KC_GEMM, bytes, flops,
+               launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, h->d_err,
+                                              h->stream));
+        gemm::EpiParams ep2{};
+        ep2.out = out;
+        ep2.ldo = ldo;
+        ep2.act = act_out;
+        ep2.ld_act = ld_act;
+        LAUNCH(KC_GEMM, 0.0, 0.0,
+               launch_splitk_reduce(epi, h->ws, g.splits, (long long)M * Nw, Nw, M, ep2, h->stream));
+    }
+    return ALODLM_OK;
+}
+
+// attention of M rows (n_seq sequences x rows_per_seq) against slot `slot`, keys [0, kv_len)
+int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_len, int causal) {
+    attn::Params p{};
+    p.q = h->qb;
+    p.q_ld = h->nq * h->hd;
+    p.kc = h->kv_k + (long long)slot * h->slot_elems;
+    p.vc = h->kv_v + (long long)slot * h->slot_elems;
+    p.seq_stride = h->seq_stride;
+    p.head_stride = h->head_stride;
+    p.map = map;
+    p.G = h->nq / h->nkv;
+    p.nq = h->nq;
+    p.kv_len = kv_len;
+    p.causal = causal;
+    p.out = h->attn_out;
+    p.out_ld = h->nq * h->hd;
+    p.ws_o = h->aws_o;
+    p.ws_ml = h->aws_ml;
+    p.m_rows = M;
+    p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)h->hd));
+    const int Tq = map.rows_per_seq;
+    const int qtiles = cdiv(p.G * Tq, 64);
+    const int base = qtiles * h->nkv * n_seq;
+    const int ktiles = cdiv(kv_len, 64);
+    int splits = 1;
+    if (!causal) {
+        splits = std::max(1, std::min(ktiles, cdiv(2 * NUM_SMS_HINT, base)));
+        while (splits > 1 && (size_t)splits * M * h->nq * (h->hd + 2) > ATTN_WS_FLOATS) --splits;
+    }
+    const int kps_tiles = cdiv(ktiles, splits);
+    splits = cdiv(ktiles, kps_tiles);
+    p.n_splits = splits;
+    p.keys_per_split = kps_tiles * 64;
+    dim3 grid(qtiles, h->nkv * splits, n_seq);
+    const double kvb = 4.0 * n_seq * h->nkv * (double)kv_len * h->hd;
+    const double bytes = kvb + 4.0 * M * h->nq * h->hd;
+    const double flops = 4.0 * M * h->nq * (double)kv_len * h->hd * (causal ? 0.5 : 1.0);
+    if (h->hd == 128)
+        LAUNCH(KC_ATTN, bytes, flops, (attn::attn_kernel<128><<<grid, 128, 5 * 64 * 128 * 2, h->stream>>>(p)));
+    else
+        LAUNCH(KC_ATTN, bytes, flops, (attn::attn_kernel<64><<<grid, 128, 5 * 64 * 64 * 2, h->stream>>>(p)));
+    if (splits > 1) {
+        dim3 g2(M, h->nq);
+        if (h->hd == 128)
+            LAUNCH(KC_ATTN, 0.0, 0.0,
+                   (attn::attn_combine_kernel<128><<<g2, 64, 0, h->stream>>>(h->aws_o, h->aws_ml, splits, M, h->nq,
+                                                                            h->attn_out, h->nq * h->hd)));
+        else
+            LAUNCH(KC_ATTN, 0.0, 0.0,
+                   (attn::attn_combine_kernel<64><<<g2, 64, 0, h->stream>>>(h->aws_o, h->aws_ml, splits, M, h->nq,
+                                                                           h->attn_out, h->nq * h->hd)));
+    }
+    return ALODLM_OK;
+}
+
+int slot_prelude(const alodlm *h, int l) { return l; }
+int slot_core(const alodlm *h, int c, int d) { return h->cfg.n_prelude + (d - 1) * h->cfg.n_core + c; }
+int slot_coda(const alodlm *h, int j) { return h->cfg.n_prelude + h->cfg.k_max * h->cfg.n_core + j; }
+
+struct Fallback {
+    int P, b0, nb, depth, src_slot;
+};
+
+// one pre-norm Qwen3 decoder layer over M rows, residual stream `x` updated in place
+int run_layer(alodlm *h, int li, int slot, int M, const RowMap &map, int n_seq, int kv_len, int causal, float *x,
+              const Fallback *fb) {
+    const LayerDev &Lw = h->layers[li];
+    const int H = h->H, qd = h->nq * h->hd;
+    int rc;
+    LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
+           (k::rmsnorm_kernel<<<M, 256, 0, h->stream>>>(x, Lw.attn_norm, h->xn, H, h->cfg.rms_eps)));
+    if ((rc = linear(h, Lw.tm_qkv, h->n_qkv, h->xn, M, H, gemm::EPI_F32, h->qkv, h->n_qkv, nullptr, 0))) return rc;
+    bf16 *kc = h->kv_k + (long long)slot * h->slot_elems, *vc = h->kv_v + (long long)slot * h->slot_elems;
+    LAUNCH(KC_QKV, 6.0 * M * h->n_qkv, 0.0,
+           (k::qkv_post_kernel<<<M, 256, 0, h->stream>>>(h->qkv, h->nq, h->nkv, h->hd, Lw.q_norm, Lw.k_norm,
+                                                          h->cfg.qk_norm, h->cfg.rms_eps, h->rope, map, h->qb, kc, vc,
+                                                          h->seq_stride, h->head_stride)));
+    if (fb) {
+        const long long so = (long long)fb->src_slot * h->slot_elems;
+        LAUNCH(KC_OTHER, 8.0 * fb->nb * h->nkv * fb->P * h->hd, 0.0,
+               (k::kv_fallback_kernel<<<dim3(fb->nb, h->nkv), 256, 0, h->stream>>>(
+                   h->exit_dev, fb->P, fb->b0, fb->depth, h->kv_k + so, h->kv_v + so, kc, vc, h->seq_stride,
+                   h->head_stride, h->hd)));
+    }
+    if ((rc = attention(h, slot, M, map, n_seq, kv_len, causal))) return rc;
+    if ((rc = linear(h, Lw.tm_o, H, h->attn_out, M, qd, gemm::EPI_ADD, x, H, nullptr, 0))) return rc;
+    LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
+           (k::rmsnorm_kernel<<<M, 256, 0, h->stream>>>(x, Lw.mlp_norm, h->xn, H, h->cfg.rms_eps)));
+    if ((rc = linear(h, Lw.tm_gu, 2 * h->I, h->xn, M, H, gemm::EPI_SWIGLU, nullptr, 0, h->act, h->I))) return rc;
+    if ((rc = linear(h, Lw.tm_d, H, h->act, M, h->I, gemm::EPI_ADD, x, H, nullptr, 0))) return rc;
+    return ALODLM_OK;
+}
+
+int check_launch(alodlm *h, const char *what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(h, e, what);
+    return ALODLM_OK;
+}
+
+int validate_cfg(const alodlm_cfg *c, std::string &why) {
+    auto bad = [&](const char *m) {
+        why = m;
+        return ALODLM_EINVAL;
+    };
+    if (c->hidden < 64 || c->hidden % 16) return bad("hidden must be >= 64 and a multiple of 16");
+    if (c->head_dim != 64 && c->head_dim != 128) return bad("head_dim must be 64 or 128");
+    if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads)
+        return bad("n_q_heads must be a positive multiple of n_kv_heads");
+    if (c->inter < 16 || c->inter % 16) return bad("inter must be a positive multiple of 16");
+    if (c->vocab < 2) return bad("vocab must be >= 2");
+    if (c->n_core < 1 || c->n_prelude < 0 || c->n_coda < 0) return bad("layer counts out of range");
+    if (c->k_max < 1 || c->k_max > 64) return bad("k_max must be in 1..64");
+    if (c->max_batch < 1 || c->max_batch > 1024) return bad("max_batch must be in 1..1024");
+    if (c->max_block < 1 || c->max_block > 1024) return bad("max_block must be in 1..1024");
+    if ((long long)c->max_batch * c->max_block > 65536) return bad("max_batch * max_block must be <= 65536");
+    if (c->max_prefix < 1) return bad("max_prefix must be >= 1");
+    if (c->mask_id < 0 || c->mask_id >= c->vocab) return bad("mask_id out of range");
+    if (!(c->rms_eps > 0.f) || !(c->rope_base > 1.f)) return bad("rms_eps/rope_base out of range");
+    return ALODLM_OK;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------------
+// ABI
+// ---------------------------------------------------------------------------------
+extern "C" {
+
+const char *alodlm_kernel_class_name(int k) {
+    return (k >= 0 && k < ALODLM_N_KCLASS) ? kclass_names[k] : "";
+}
+
+const char *alodlm_last_error(const alodlm_t *h) {
+    if (h) return h->err.c_str();
+    std::lock_guard<std::mutex> lk(g_err_mu);
+    return g_create_err.c_str();
+}
+
+void alodlm_destroy(alodlm_t *h) {
+    if (!h) return;
+    cudaStreamSynchronize(h->stream);
+    for (void *p : h->allocs) cudaFree(p);
+    for (auto e : h->ev_pool) cudaEventDestroy(e);
+    if (h->counts_host) cudaFreeHost(h->counts_host);
+    delete h;
+}
+
+int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, alodlm_t **out) {
+    if (out) *out = nullptr;
+    if (!cfg || !w || !out || !w->layers || !w->embed || !w->lm_head || !w->final_norm || !w->exit_w)
+        return fail(nullptr, ALODLM_EINVAL, "null argument");
+    std::string why;
+    if (validate_cfg(cfg, why)) return fail(nullptr, ALODLM_EINVAL, why);
+    if (w->matrix_dtype != ALODLM_DTYPE_BF16 && w->matrix_dtype != ALODLM_DTYPE_F32)
+        return fail(nullptr, ALODLM_EINVAL, "matrix_dtype must be ALODLM_DTYPE_BF16 or ALODLM_DTYPE_F32");
+    const int L = cfg->n_prelude + cfg->n_core + cfg->n_coda;
+    for (int l = 0; l < L; ++l) {
+        const alodlm_layer_w &lw = w->layers[l];
+        if (!lw.attn_norm || !lw.q || !lw.k || !lw.v || !lw.o || !lw.mlp_norm || !lw.gate || !lw.up || !lw.down ||
+            (cfg->qk_norm && (!lw.q_norm || !lw.k_norm)))
+            return fail(nullptr, ALODLM_EINVAL, "null layer weight pointer");
+    }
+    if (!get_encode_fn()) return fail(nullptr, ALODLM_ECUDA, "cuTensorMapEncodeTiled unavailable");
+    if (!init_kernel_attrs()) return fail(nullptr, ALODLM_ECUDA, "cudaFuncSetAttribute failed");
+
+    alodlm *h = new alodlm();
+    h->cfg = *cfg;
+    h->stream = static_cast<cudaStream_t>(stream);
+    cudaGetDevice(&h->device);
+    h->H = cfg->hidden;
+    h->nq = cfg->n_q_heads;
+    h->nkv = cfg->n_kv_heads;
+    h->hd = cfg->head_dim;
+    h->I = cfg->inter;
+    h->V = cfg->vocab;
+    h->L = L;
+    h->n_qkv = (h->nq + 2 * h->nkv) * h->hd;
+    const int H = h->H, qd = h->nq * h->hd;
+    const int f32 = w->matrix_dtype == ALODLM_DTYPE_F32;
+    int rc = ALODLM_OK;
+    auto cleanup = [&](int code) {
+        std::string msg = h->err;
+        alodlm_destroy(h);
+        fail(nullptr, code, msg);
+        return code;
+    };
+
+    // ---- weights: pack to bf16, rows padded to multiples of 128 with zeros ----
+    auto pack = [&](bf16 **dst, int rows_pad, int cols, const void *src, int src_rows) -> int {
+        int r;
+        if ((r = dalloc(h, dst, (size_t)rows_pad * cols))) return r;
+        cudaMemsetAsync(*dst, 0, (size_t)rows_pad * cols * 2, h->stream);
+        k::pack_rows_kernel<<<src_rows, 256, 0, h->stream>>>(src, f32, cols, nullptr, src_rows, cols, *dst, cols);
+        return check_launch(h, "pack_rows_kernel");
+    };
+    auto copy_vec = [&](float **dst, const void *src, int n) -> int {
+        int r;
+        if ((r = dalloc(h, dst, n))) return r;
+        cudaMemcpyAsync(*dst, src, n * sizeof(float), cudaMemcpyDeviceToDevice, h->stream);
+        return ALODLM_OK;
+    };
+    if ((rc = pack(&h->embed, h->V, H, w->embed, h->V))) return cleanup(rc);
+    if ((rc = pack(&h->lm_head, round_up(h->V, 256), H, w->lm_head, h->V))) return cleanup(rc);
+    if ((rc = copy_vec(&h->final_norm, w->final_norm, H))) return cleanup(rc);
+    if ((rc = copy_vec(&h->exit_w, w->exit_w, H))) return cleanup(rc);
+    h->exit_b = w->exit_b;
+    if (!make_tmap(&h->tm_lm, h->lm_head, H, round_up(h->V, 256), 256)) {
+        h->err = "cuTensorMapEncodeTiled failed (lm_head)";
+        return cleanup(ALODLM_ECUDA);
+    }
+    h->layers.resize(L);
+    for (int l = 0; l < L; ++l) {
+        const alodlm_layer_w &lw = w->layers[l];
+        LayerDev &d = h->layers[l];
+        // fused QKV: rows [q; k; v]
+        if ((rc = dalloc(h, &d.wqkv, (size_t)round_up(h->n_qkv, 128) * H))) return cleanup(rc);
+        cudaMemsetAsync(d.wqkv, 0, (size_t)round_up(h->n_qkv, 128) * H * 2, h->stream);
+        k::pack_rows_kernel<<<qd, 256, 0, h->stream>>>(lw.q, f32, H, nullptr, qd, H, d.wqkv, H);
+        k::pack_rows_kernel<<<h->nkv * h->hd, 256, 0, h->stream>>>(lw.k, f32, H, nullptr, h->nkv * h->hd, H,
+                                                                   d.wqkv + (size_t)qd * H, H);
+        k::pack_rows_kernel<<<h->nkv * h->hd, 256, 0, h->stream>>>(
+            lw.v, f32, H, nullptr, h->nkv * h->hd, H, d.wqkv + (size_t)(qd + h->nkv * h->hd) * H, H);
+        if ((rc = check_launch(h, "pack qkv"))) return cleanup(rc);
+        if ((rc = pack(&d.wo, round_up(H, 128), qd, lw.o, H))) return cleanup(rc);
+        if ((rc = dalloc(h, &d.wgu, (size_t)round_up(2 * h->I, 128) * H))) return cleanup(rc);
+        cudaMemsetAsync(d.wgu, 0, (size_t)round_up(2 * h->I, 128) * H * 2, h->stream);
+        k::pack_gate_up_kernel<<<2 * h->I, 256, 0, h->stream>>>(lw.gate, lw.up, f32, h->I, H, d.wgu);
+        if ((rc = check_launch(h, "pack gate/up"))) return cleanup(rc);
+        if ((rc = pack(&d.wd, round_up(H, 128), h->I, lw.down, H))) return cleanup(rc);
+        if ((rc = copy_vec(&d.attn_norm, lw.attn_norm, H))) return cleanup(rc);
+        if ((rc = copy_vec(&d.mlp_norm, lw.mlp_norm, H))) return cleanup(rc);
+        if (cfg->qk_norm) {
+            if ((rc = copy_vec(&d.q_norm, lw.q_norm, h->hd))) return cleanup(rc);
+            if ((rc = copy_vec(&d.k_norm, lw.k_norm, h->hd))) return cleanup(rc);
+        }
+        bool ok = make_tmap(&d.tm_qkv, d.wqkv, H, round_up(h->n_qkv, 128), 128) &&
+                  make_tmap(&d.tm_o, d.wo, qd, round_up(H, 128), 128) &&
+                  make_tmap(&d.tm_gu, d.wgu, H, round_up(2 * h->I, 128), 128) &&
+                  make_tmap(&d.tm_d, d.wd, h->I, round_up(H, 128), 128);
+        if (!ok) {
+            h->err = "cuTensorMapEncodeTiled failed (layer weights)";
+            return cleanup(ALODLM_ECUDA);
+        }
+    }
+
+    // ---- depth-aware KV arena ----
+    h->n_slots = cfg->n_prelude + cfg->k_max * cfg->n_core + cfg->n_coda;
+    h->pos_stride = cfg->max_prefix + cfg->max_block;
+    h->head_stride = (long long)h->pos_stride * h->hd;
+    h->seq_stride = h->head_stride * h->nkv;
+    h->slot_elems = h->seq_stride * cfg->max_batch;
+    if ((rc = dalloc(h, &h->kv_k, (size_t)h->slot_elems * h->n_slots))) return cleanup(rc);
+    if ((rc = dalloc(h, &h->kv_v, (size_t)h->slot_elems * h->n_slots))) return cleanup(rc);
+    if ((rc = dalloc(h, &h->rope, (size_t)h->pos_stride * (h->hd / 2)))) return cleanup(rc);
+    {
+        const long long n = (long long)h->pos_stride * (h->hd / 2);
+        k::rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, h->stream>>>(h->rope, h->pos_stride, h->hd / 2,
+                                                                                (double)cfg->rope_base);
+        if ((rc = check_launch(h, "rope_table_kernel"))) return cleanup(rc);
+    }
+
+    // ---- scratch ----
+    const int g_max = std::max(1, std::min(cfg->max_batch, PREFILL_ROWS / std::max(1, cfg->max_prefix)));
+    h->step_rows_cap = cfg->max_batch * cfg->max_block;
+    h->rows_cap = round_up(std::max(h->step_rows_cap, g_max * cfg->max_prefix), 256);
+    const size_t R = h->rows_cap;
+    if ((rc = dalloc(h, &h->hbuf[0], R * H)) || (rc = dalloc(h, &h->hbuf[1], R * H)) ||
+        (rc = dalloc(h, &h->hc, R * H)) || (rc = dalloc(h, &h->hexit, R * H)) ||
+        (rc = dalloc(h, &h->qkv, R * h->n_qkv)) || (rc = dalloc(h, &h->xn, R * H)) ||
+        (rc = dalloc(h, &h->qb, R * qd)) || (rc = dalloc(h, &h->attn_out, R * qd)) ||
+        (rc = dalloc(h, &h->act, R * h->I)) || (rc = dalloc(h, &h->ws, SPLITK_WS_FLOATS)) ||
+        (rc = dalloc(h, &h->aws_o, ATTN_WS_FLOATS)) ||
+        (rc = dalloc(h, &h->aws_ml, ATTN_WS_FLOATS / 16)))
+        return cleanup(rc);
+    // zero the activation buffers once so rows past the live ones never hold NaN patterns
+    cudaMemsetAsync(h->xn, 0, R * H * 2, h->stream);
+    cudaMemsetAsync(h->attn_out, 0, R * qd * 2, h->stream);
+    cudaMemsetAsync(h->act, 0, R * h->I * 2, h->stream);
+
+    h->R_cap = round_up(h->step_rows_cap, 128);
+    h->n_vt = cdiv(h->V, 256);
+    if ((rc = dalloc(h, &h->rb, (size_t)h->R_cap * H)) || (rc = dalloc(h, &h->lam_rr, h->R_cap)) ||
+        (rc = dalloc(h, &h->part, (size_t)h->R_cap * h->n_vt)) || (rc = dalloc(h, &h->ridx, h->step_rows_cap)) ||
+        (rc = dalloc(h, &h->rr_b, h->R_cap)) || (rc = dalloc(h, &h->rr_i, h->R_cap)))
+        return cleanup(rc);
+    cudaMemsetAsync(h->rb, 0, (size_t)h->R_cap * H * 2, h->stream);
+    if (!make_tmap(&h->tm_rb, h->rb, H, h->R_cap, 128)) {
+        h->err = "cuTensorMapEncodeTiled failed (readout rows)";
+        return cleanup(ALODLM_ECUDA);
+    }
+    const size_t BN_ = (size_t)cfg->max_batch * cfg->max_block;
+    if ((rc = dalloc(h, &h->U, BN_)) || (rc = dalloc(h, &h->a, BN_)) || (rc = dalloc(h, &h->cur_H, BN_)) ||
+        (rc = dalloc(h, &h->cur_y, BN_)) || (rc = dalloc(h, &h->cont, cfg->max_batch)) ||
+        (rc = dalloc(h, &h->ncommit, cfg->max_batch)) || (rc = dalloc(h, &h->seq_of[0], cfg->max_batch)) ||
+        (rc = dalloc(h, &h->seq_of[1], cfg->max_batch)) || (rc = dalloc(h, &h->old_slot, cfg->max_batch)) ||
+        (rc = dalloc(h, &h->counts, 4)) || (rc = dalloc(h, &h->d_err, 1)) || (rc = dalloc(h, &h->iota, cfg->max_batch)) ||
+        (rc = dalloc(h, &h->exit_dev, (size_t)cfg->max_batch * cfg->max_prefix)))
+        return cleanup(rc);
+    {
+        std::vector<int> io(cfg->max_batch);
+        for (int i = 0; i < cfg->max_batch; ++i) io[i] = i;
+        cudaMemcpyAsync(h->iota, io.data(), io.size() * sizeof(int), cudaMemcpyHostToDevice, h->stream);
+        cudaMemsetAsync(h->d_err, 0, sizeof(int), h->stream);
+    }
+    if (cfg->debug_dump) {
+        for (int i = 0; i < 3; ++i)
+            if ((rc = dalloc(h, &h->dbg[i], (size_t)cfg->k_max * BN_ * H))) return cleanup(rc);
+    }
+    if (cudaMallocHost(&h->counts_host, 4 * sizeof(int)) != cudaSuccess) {
+        h->err = "cudaMallocHost failed";
+        return cleanup(ALODLM_ENOMEM);
+    }
+    cudaError_t e = cudaStreamSynchronize(h->stream);
+    if (e != cudaSuccess) {
+        cuda_fail(h, e, "create");
+        return cleanup(ALODLM_ECUDA);
+    }
+    *out = h;
+    return ALODLM_OK;
+}
+
+int alodlm_set_timing(alodlm_t *h, int on) {
+    if (!h) return ALODLM_EINVAL;
+    h->timing = on != 0;
+    return ALODLM_OK;
+}
+
+int alodlm_sync(alodlm_t *h) {
+    if (!h) return ALODLM_EINVAL;
+    cudaError_t e = cudaStreamSynchronize(h->stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "sync");
+    int dev_err = 0;
+    e = cudaMemcpy(&dev_err, h->d_err, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(h, e, "sync: read error word");
+    if (dev_err) {
+        cudaMemset(h->d_err, 0, sizeof(int));
+        if (dev_err & DEVERR_TIMEOUT) return fail(h, ALODLM_ETIMEOUT, "a bounded device wait timed out");
+        return fail(h, ALODLM_EDEVICE, "a kernel flagged an out-of-range value (token id or exit depth)");
+    }
+    return ALODLM_OK;
+}
+
+int alodlm_prefill(alodlm_t *h, const int32_t *prefix_ids, int B, int P, const int32_t *exit_depth) {
+    if (!h || !prefix_ids) return fail(h, ALODLM_EINVAL, "null argument");
+    const alodlm_cfg &c = h->cfg;
+    if (B < 1 || B > c.max_batch || P < 1 || P > c.max_prefix)
+        return fail(h, ALODLM_EINVAL, "prefill: B or P out of range");
+    reset_stats(h);
+    h->prefilled = false;
+    if (exit_depth)
+        cudaMemcpyAsync(h->exit_dev, exit_depth, (size_t)B * P * sizeof(int), cudaMemcpyDeviceToDevice, h->stream);
+    const int g = std::max(1, std::min(B, h->rows_cap / P));
+    int rc;
+    for (int b0 = 0; b0 < B; b0 += g) {
+        const int nb = std::min(g, B - b0), M = nb * P;
+        RowMap map{h->iota + b0, P, 0};
+        float *x = h->hbuf[0];
+        LAUNCH(KC_OTHER, 6.0 * M * h->H, 0.0,
+               (k::embed_kernel<<<M, 256, 0, h->stream>>>(prefix_ids, P, map, h->embed, h->V, h->H, x, h->d_err)));
+        for (int l = 0; l < c.n_prelude; ++l)
+            if ((rc = run_layer(h, l, slot_prelude(h, l), M, map, nb, P, 1, x, nullptr))) return rc;
+        for (int d = 1; d <= c.k_max; ++d) {
+            for (int cc = 0; cc < c.n_core; ++cc) {
+                Fallback fb{P, b0, nb, d, d > 1 ? slot_core(h, cc, d - 1) : 0};
+                const bool use_fb = exit_depth && d > 1;
+                if ((rc = run_layer(h, c.n_prelude + cc, slot_core(h, cc, d), M, map, nb, P, 1, x,
+                                    use_fb ? &fb : nullptr)))
+                    return rc;
+            }
+            if (exit_depth)
+                LAUNCH(KC_OTHER, 8.0 * M * h->H / c.k_max, 0.0,
+                       (k::capture_exit_kernel<<<M, 256, 0, h->stream>>>(h->exit_dev, P, b0, d, x, h->hexit, h->H)));
+        }
+        if (exit_depth) x = h->hexit;
+        for (int j = 0; j < c.n_coda; ++j)
+            if ((rc = run_layer(h, c.n_prelude + c.n_core + j, slot_coda(h, j), M, map, nb, P, 1, x, nullptr)))
+                return rc;
+        if ((rc = check_launch(h, "prefill"))) return rc;
+    }
+    h->B = B;
+    h->P = P;
+    h->prefilled = true;
+    return ALODLM_OK;
+}
+
+int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda, int k_max,
+                        int rule, const alodlm_step_out *out) {
+    if (!h || !block_ids || !out || !out->tokens || !out->exit_depth || !out->entropy || !out->halt ||
+        !out->cum_halt || !out->loops_run || !out->active_rows || !out->readout_rows)
+        return fail(h, ALODLM_EINVAL, "null argument");
+    const alodlm_cfg &c = h->cfg;
+    if (!h->prefilled) return fail(h, ALODLM_ESTATE, "denoise_step before prefill");
+    if (B != h->B) return fail(h, ALODLM_ESTATE, "batch differs from the prefill's");
+    if (N < 1 || N > c.max_block) return fail(h, ALODLM_EINVAL, "N out of range");
+    if (k_max < 1 || k_max > c.k_max) return fail(h, ALODLM_EINVAL, "k_max out of range");
+    if (rule != ALODLM_RULE_PAPER && rule != ALODLM_RULE_PER_TOKEN) return fail(h, ALODLM_EINVAL, "unknown rule");
+    if (std::isnan(tau_H) || std::isnan(lambda)) return fail(h, ALODLM_EINVAL, "tau_H/lambda is NaN");
+    reset_stats(h);
+    const int H = h->H, P = h->P;
+    const int K = k_max;
+    h->last_N = N;
+    k::StepState st;
+    st.tokens = out->tokens;
+    st.exit_depth = out->exit_depth;
+    st.tr_H = out->entropy;
+    st.tr_lam = out->halt;
+    st.tr_a = out->cum_halt;
+    st.loops_run = out->loops_run;
+    st.active_rows = out->active_rows;
+    st.readout_rows = out->readout_rows;
+    st.U = h->U;
+    st.a = h->a;
+    st.cur_H = h->cur_H;
+    st.cur_y = h->cur_y;
+    st.cont = h->cont;
+    st.n_commit = h->ncommit;
+
+    int cur = 0, hi = 0, rc;
+    const long long BNt = (long long)B * N;
+    LAUNCH(KC_COMMIT, 16.0 * BNt, 0.0,
+           (k::step_init_kernel<<<(unsigned)std::min<long long>((BNt + 255) / 256, 1024), 256, 0, h->stream>>>(
+               block_ids, B, N, K, c.mask_id, st)));
+    LAUNCH(KC_COMMIT, 8.0 * BNt, 0.0,
+           (k::plan_kernel<<<1, 1024, 0, h->stream>>>(B, h->iota, N, h->cont, h->U, h->seq_of[0], h->old_slot,
+                                                      h->ridx, h->rr_b, h->rr_i, h->counts, 1, K, out->active_rows,
+                                                      out->readout_rows, h->d_err)));
+    cudaMemcpyAsync(h->counts_host, h->counts, 4 * sizeof(int), cudaMemcpyDeviceToHost, h->stream);
+
+    int n_act = B;
+    RowMap map{h->seq_of[0], N, P};
+    int M = n_act * N;
+    float *x = h->hbuf[hi];
+    LAUNCH(KC_OTHER, 6.0 * M * H, 0.0,
+           (k::embed_kernel<<<M, 256, 0, h->stream>>>(block_ids, N, map, h->embed, h->V, H, x, h->d_err)));
+    for (int l = 0; l < c.n_prelude; ++l)
+        if ((rc = run_layer(h, l, slot_prelude(h, l), M, map, n_act, P + N, 0, x, nullptr))) return rc;
+
+    cudaError_t e = cudaStreamSynchronize(h->stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "step: first loop plan");
+    int R = h->counts_host[1];
+    if (h->counts_host[2]) return alodlm_sync(h);
+
+    for (int s = 1; s <= K; ++s) {
+        map.seq_of = h->seq_of[cur];
+        M = n_act * N;
+        x = h->hbuf[hi];
+        const long long dbg_off = (long long)(s - 1) * c.max_batch * c.max_block * H;
+        if (c.debug_dump)
+            LAUNCH(KC_OTHER, 0.0, 0.0,
+                   (k::dump_rows_kernel<<<M, 256, 0, h->stream>>>(x, map, H, h->dbg[0] + dbg_off)));
+        for (int cc = 0; cc < c.n_core; ++cc)
+            if ((rc = run_layer(h, c.n_prelude + cc, slot_core(h, cc, s), M, map, n_act, P + N, 0, x, nullptr)))
+                return rc;
+        if (c.debug_dump)
+            LAUNCH(KC_OTHER, 0.0, 0.0,
+                   (k::dump_rows_kernel<<<M, 256, 0, h->stream>>>(x, map, H, h->dbg[1] + dbg_off)));
+        cudaMemcpyAsync(h->hc, x, (size_t)M * H * sizeof(float), cudaMemcpyDeviceToDevice, h->stream);
+        for (int j = 0; j < c.n_coda; ++j)
+            if ((rc = run_layer(h, c.n_prelude + c.n_core + j, slot_coda(h, j), M, map, n_act, P + N, 0, h->hc,
+                                nullptr)))
+                return rc;
+        LAUNCH(KC_NORM, 4.0 * M * H + 2.0 * R * H, 0.0,
+               (k::final_norm_kernel<<<M, 256, 0, h->stream>>>(h->hc, h->final_norm, h->exit_w, h->exit_b, H,
+                                                               c.rms_eps, map, h->ridx, h->rb, h->lam_rr,
+                                                               c.debug_dump ? h->dbg[2] + dbg_off : nullptr)));
+        if (R > 0) {
+            gemm::EpiParams ep{};
+            ep.partials = h->part;
+            ep.n_btiles = h->n_vt;
+            const double bytes = 2.0 * h->V * H + 2.0 * R * H + 16.0 * R * h->n_vt;
+            LAUNCH(KC_RGEMM, bytes, 2.0 * R * h->V * (double)H,
+                   launch_gemm_bn<256, gemm::EPI_READOUT>(h->tm_rb, h->tm_lm, R, h->V, cdiv(H, gemm::BK),
+                                                          cdiv(H, gemm::BK), 1, 1, ep, h->d_err, h->stream));
+            LAUNCH(KC_RCOMB, 16.0 * R * h->n_vt, 0.0,
+                   (k::readout_combine_kernel<<<cdiv(R, 8), 256, 0, h->stream>>>(
+                       h->part, h->n_vt, R, h->rr_b, h->rr_i, h->lam_rr, N, K, s, h->a, h->cur_H, h->cur_y,
+                       out->entropy, out->halt, out->cum_halt)));
+        }
+        LAUNCH(KC_COMMIT, 16.0 * M + 0.0, 0.0,
+               (k::commit_kernel<<<n_act, 256, 0, h->stream>>>(map, s, K, rule, tau_H, lambda, h->embed, H, x, st)));
+        LAUNCH(KC_COMMIT, 8.0 * M, 0.0,
+               (k::plan_kernel<<<1, 1024, 0, h->stream>>>(n_act, h->seq_of[cur], N, h->cont, h->U,
+                                                          h->seq_of[cur ^ 1], h->old_slot, h->ridx, h->rr_b, h->rr_i,
+                                                          h->counts, s + 1, K, out->active_rows, out->readout_rows,
+                                                          h->d_err)));
+        cudaMemcpyAsync(h->counts_host, h->counts, 4 * sizeof(int), cudaMemcpyDeviceToHost, h->stream);
+        e = cudaStreamSynchronize(h->stream);
+        if (e != cudaSuccess) return cuda_fail(h, e, "step: loop control");
+        if ((rc = check_launch(h, "step"))) return rc;
+        if (h->counts_host[2]) return alodlm_sync(h);
+        const int n_next = h->counts_host[0];
+        R = h->counts_host[1];
+        if (n_next == 0) break;
+        if (n_next != n_act) {
+            LAUNCH(KC_COMMIT, 8.0 * n_next * N * H, 0.0,
+                   (k::gather_rows_kernel<<<n_next * N, 256, 0, h->stream>>>(x, h->hbuf[hi ^ 1], h->old_slot, N, H)));
+            hi ^= 1;
+        }
+        cur ^= 1;
+        n_act = n_next;
+    }
+    return check_launch(h, "step end");
+}
+
+int alodlm_debug_state(alodlm_t *h, int which, int loop, float *dst) {
+    if (!h || !dst) return ALODLM_EINVAL;
+    if (!h->cfg.debug_dump) return fail(h, ALODLM_EINVAL, "debug_dump is off");
+    if (which < 0 || which > 2 || loop < 1 || loop > h->cfg.k_max || h->last_N < 1)
+        return fail(h, ALODLM_EINVAL, "debug_state: out of range or no step yet");
+    const float *src = h->dbg[which] + (size_t)(loop - 1) * h->cfg.max_batch * h->cfg.max_block * h->H;
+    cudaError_t e = cudaMemcpyAsync(dst, src, (size_t)h->B * h->last_N * h->H * sizeof(float),
+                                    cudaMemcpyDeviceToDevice, h->stream);
+    return e == cudaSuccess ? ALODLM_OK : cuda_fail(h, e, "debug_state");
+}
+
+int alodlm_kv_slot(alodlm_t *h, int which, int slot, int b, int n_pos, void *dst) {
+    if (!h || !dst || which < 0 || which > 1 || slot < 0 || slot >= h->n_slots || b < 0 ||
+        b >= h->cfg.max_batch || n_pos < 1 || n_pos > h->pos_stride)
+        return h ? fail(h, ALODLM_EINVAL, "kv_slot: out of range") : ALODLM_EINVAL;
+    const bf16 *base = (which ? h->kv_v : h->kv_k) + (long long)slot * h->slot_elems + (long long)b * h->seq_stride;
+    cudaError_t e = cudaMemcpy2DAsync(dst, (size_t)n_pos * h->hd * 2, base, (size_t)h->head_stride * 2,
+                                      (size_t)n_pos * h->hd * 2, h->nkv, cudaMemcpyDeviceToDevice, h->stream);
+    return e == cudaSuccess ? ALODLM_OK : cuda_fail(h, e, "kv_slot");
+}
+
+int alodlm_step_stats(const alodlm_t *hc, int *kernel_launches, double *times_ms, int *launches, double *bytes,
+                      double *flops) {
+    alodlm *h = const_cast<alodlm *>(hc);
+    if (!h) return ALODLM_EINVAL;
+    if (kernel_launches) *kernel_launches = h->launches;
+    for (int c = 0; c < ALODLM_N_KCLASS; ++c) {
+        if (times_ms) times_ms[c] = 0.0;
+        if (launches) launches[c] = h->cls_launches[c];
+        if (bytes) bytes[c] = h->cls_bytes[c];
+        if (flops) flops[c] = h->cls_flops[c];
+    }
+    if (times_ms && !h->timed.empty()) {
+        cudaError_t e = cudaStreamSynchronize(h->stream);
+        if (e != cudaSuccess) return cuda_fail(h, e, "stats");
+        for (const auto &t : h->timed) {
+            float ms = 0.f;
+            cudaEventElapsedTime(&ms, t.e0, t.e1);
+            times_ms[t.cls] += ms;
+        }
+    }
+    return ALODLM_OK;
+}
+
+int alodlm_gemm_bf16(const void *A, const void *W, float *C, int M, int N, int K, float *workspace,
+                     size_t workspace_bytes, void *stream) {
+    if (!A || !W || !C || !workspace || workspace_bytes < 256 || M < 1 || N < 1 || K < 8 || K % 8)
+        return ALODLM_EINVAL;
+    if (!get_encode_fn() || !init_kernel_attrs()) return ALODLM_ECUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // first 256 bytes: the device status word; the rest: split-K partials
+    int *err = reinterpret_cast<int *>(workspace);
+    float *parts = workspace + 64;
+    const size_t part_floats = (workspace_bytes - 256) / sizeof(float);
+    GemmShape g = plan_gemm(M, N, K, part_floats);
+    CUtensorMap tW, tA;
+    if (!make_tmap(&tW, W, K, N, gemm::BM) || !make_tmap(&tA, A, K, M, g.bn)) return ALODLM_ECUDA;
+    gemm::EpiParams ep{};
+    if (g.splits == 1) {
+        ep.out = C;
+        ep.ldo = N;
+        launch_gemm_epi<gemm::EPI_F32>(g.bn, tW, tA, N, M, g.k_tiles, g.kps, 1, 0, ep, err, st);
+    } else {
+        ep.out = parts;
+        ep.ldo = N;
+        ep.split_stride = (long long)M * N;
+        launch_gemm_epi<gemm::EPI_F32>(g.bn, tW, tA, N, M, g.k_tiles, g.kps, g.splits, 0, ep, err, st);
+        gemm::EpiParams ep2{};
+        ep2.out = C;
+        ep2.ldo = N;
+        launch_splitk_reduce(gemm::EPI_F32, parts, g.splits, (long long)M * N, N, M, ep2, st);
+    }
+    return cudaGetLastError() == cudaSuccess ? ALODLM_OK : ALODLM_ECUDA;
+}
+
+}  // extern "C"

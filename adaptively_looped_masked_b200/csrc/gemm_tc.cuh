@@ -1,0 +1,248 @@
+// gemm_tc.cuh — bf16 GEMM on the fifth-generation tensor core (tcgen05 + TMEM + TMA).
+//
+// D[a, b] = sum_k A[a, k] * B[b, k], both operands K-major bf16 in global memory, f32
+// accumulation in tensor memory.  One CTA computes one 128 x BN tile (128 rows of A = the
+// MMA's M side, BN rows of B = its N side) over a range of K (split-K):
+//   warp 0      one thread issues TMA loads of A and B k-tiles (64 wide, 128-byte swizzle)
+//               into a ring of STAGES shared-memory slots,
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, K=16) per
+//               16-wide k step and releases each slot with tcgen05.commit,
+//   warps 2-5   epilogue: tcgen05.ld the accumulator (thread = one A row, registers =
+//               its BN columns) and apply the fused epilogue.
+//
+// For the decoder's linear layers A is the weight (output features on TMEM lanes) and B
+// the activation rows (swap-AB): a 32-row step still fills the 128-row MMA, and the
+// epilogue writes consecutive features from consecutive lanes (coalesced).  For the LM-head
+// readout A is the readout rows and B the vocabulary, so each thread owns one row's logits
+// and reduces them without shuffles; the logits never leave the SM.
+#pragma once
+#include "common.cuh"
+
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+
+enum Epi { EPI_F32 = 0, EPI_ADD = 1, EPI_SWIGLU = 2, EPI_READOUT = 3 };
+
+struct EpiParams {
+    float *out;           // EPI_F32 / EPI_ADD: out[b_row * ldo + a_row] (+ split * split_stride)
+    int ldo;
+    long long split_stride;
+    bf16 *act;            // EPI_SWIGLU: act[b_row * ld_act + feature]
+    int ld_act;
+    float4 *partials;     // EPI_READOUT: partials[a_row * n_btiles + b_tile] = (max, sum e, sum e*d, argmax)
+    int n_btiles;
+};
+
+template <int BN>
+struct Cfg {
+    static constexpr int STAGES = (BN <= 64) ? 4 : (BN == 128 ? 5 : 4);
+    static constexpr uint32_t A_BYTES = BM * BK * 2;
+    static constexpr uint32_t B_BYTES = BN * BK * 2;
+    static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr uint32_t TMEM_COLS = BN;  // power of two >= 32
+    static constexpr size_t SMEM = 1024 /*align slack*/ + (size_t)STAGES * STAGE_BYTES + 256;
+};
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int rowsA,
+                   int rowsB, int k_tiles, int kt_per_split, int a_fastest, EpiParams ep, int *err) {
+    using C = Cfg<BN>;
+    constexpr int STAGES = C::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * C::STAGE_BYTES);
+    uint64_t *empty = full + STAGES;
+    uint64_t *accum = empty + STAGES;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int a_tile = a_fastest ? blockIdx.x : blockIdx.y;
+    const int b_tile = a_fastest ? blockIdx.y : blockIdx.x;
+    const int split = blockIdx.z;
+    const int kt0 = split * kt_per_split;
+    const int nkt = min(k_tiles, kt0 + kt_per_split) - kt0;  // >= 1 by construction on the host
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        mbar_init(accum, 1);
+        fence_mbarrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int it = 0; it < nkt; ++it) {
+                const int s = it % STAGES;
+                const uint32_t use = (uint32_t)(it / STAGES);
+                if (!mbar_wait(empty + s, (use & 1u) ^ 1u, err)) break;
+                mbar_arrive_expect_tx(full + s, C::STAGE_BYTES);
+                uint8_t *sa = smem + s * C::STAGE_BYTES;
+                const int kx = (kt0 + it) * BK;
+                tma_load_2d(sa, &tmA, full + s, kx, a_tile * BM);
+                tma_load_2d(sa + C::A_BYTES, &tmB, full + s, kx, b_tile * BN);
+                issued = it + 1;
+            }
+            // make sure no copy into shared memory is still in flight when the CTA exits
+            for (int it = max(0, issued - STAGES); it < issued; ++it)
+                mbar_wait(full + (it % STAGES), (uint32_t)(it / STAGES) & 1u, err);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16(BM, BN);
+            for (int it = 0; it < nkt; ++it) {
+                const int s = it % STAGES;
+                if (!mbar_wait(full + s, (uint32_t)(it / STAGES) & 1u, err)) break;
+                tc_fence_after();
+                const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+                const uint64_t da = umma_sdesc_sw128(sa);
+                const uint64_t db = umma_sdesc_sw128(sa + C::A_BYTES);
+#pragma unroll
+                for (int k = 0; k < BK / 16; ++k)  // 16 bf16 = 32 bytes = 2 descriptor units per k step
+                    umma_f16(tmem_base, da + 2 * k, db + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
+                umma_commit(empty + s);
+            }
+            umma_commit(accum);
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5) ----------------
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const bool ready = mbar_wait(accum, 0, err);
+        tc_fence_after();
+        const int a_row = a_tile * BM + q * 32 + lane;
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
+        const int b0 = b_tile * BN;
+        if (ready) {
+            if constexpr (EPI == EPI_F32 || EPI == EPI_ADD) {
+                float *out = ep.out + (long long)split * ep.split_stride;
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    if (b0 + c0 >= rowsB) break;  // warp-uniform
+                    float v[16];
+                    tmem_ld16(taddr + c0, v);
+                    if (a_row < rowsA) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int br = b0 + c0 + j;
+                            if (br < rowsB) {
+                                float *p = out + (long long)br * ep.ldo + a_row;
+                                if constexpr (EPI == EPI_ADD)
+                                    *p += v[j];
+                                else
+                                    *p = v[j];
+                            }
+                        }
+                    }
+                }
+            } else if constexpr (EPI == EPI_SWIGLU) {
+                // weight rows interleaved in groups of 32: 16 gate rows then the 16 up rows of
+                // the same features, so lane l < 16 holds gate and lane l + 16 holds up
+                const int feat = (a_row >> 5) * 16 + (lane & 15);
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    if (b0 + c0 >= rowsB) break;
+                    float v[16];
+                    tmem_ld16(taddr + c0, v);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float up = __shfl_xor_sync(0xffffffffu, v[j], 16);
+                        const int br = b0 + c0 + j;
+                        if (lane < 16 && a_row < rowsA && br < rowsB)
+                            ep.act[(long long)br * ep.ld_act + feat] = __float2bfloat16_rn(silu_f(v[j]) * up);
+                    }
+                }
+            } else {  // EPI_READOUT: this thread's row of logits over BN vocabulary entries
+                float best = -INFINITY;
+                int best_idx = b0;
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    if (b0 + c0 >= rowsB) break;
+                    float v[16];
+                    tmem_ld16(taddr + c0, v);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int vid = b0 + c0 + j;
+                        if (vid < rowsB && v[j] > best) {  // strict: lowest id wins ties
+                            best = v[j];
+                            best_idx = vid;
+                        }
+                    }
+                }
+                float se = 0.f, sed = 0.f;
+                const float LOG2E = 1.4426950408889634f;
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    if (b0 + c0 >= rowsB) break;
+                    float v[16];
+                    tmem_ld16(taddr + c0, v);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        if (b0 + c0 + j < rowsB) {
+                            const float d = v[j] - best;
+                            const float e = exp2f(d * LOG2E);
+                            se += e;
+                            sed = fmaf(e, d, sed);
+                        }
+                    }
+                }
+                if (a_row < rowsA)
+                    ep.partials[(long long)a_row * ep.n_btiles + b_tile] =
+                        make_float4(best, se, sed, __int_as_float(best_idx));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// Fixed-order sum of split-K partials ws[split][b_row][a_row] followed by the epilogue.
+template <int EPI>
+__global__ void splitk_reduce_kernel(const float *__restrict__ ws, int splits, long long split_stride, int rowsA,
+                                     int rowsB, EpiParams ep) {
+    if constexpr (EPI == EPI_SWIGLU) {
+        const int n_feat = rowsA / 2;
+        const long long total = (long long)rowsB * n_feat;
+        for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+             idx += (long long)gridDim.x * blockDim.x) {
+            const int br = (int)(idx / n_feat), f = (int)(idx % n_feat);
+            const int rg = (f >> 4) * 32 + (f & 15), ru = rg + 16;
+            float g = 0.f, u = 0.f;
+            for (int s = 0; s < splits; ++s) {
+                const float *p = ws + s * split_stride + (long long)br * rowsA;
+                g += p[rg];
+                u += p[ru];
+            }
+            ep.act[(long long)br * ep.ld_act + f] = __float2bfloat16_rn(silu_f(g) * u);
+        }
+    } else {
+        const long long total = (long long)rowsB * rowsA;
+        for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+             idx += (long long)gridDim.x * blockDim.x) {
+            const int br = (int)(idx / rowsA), ar = (int)(idx % rowsA);
+            float acc = 0.f;
+            for (int s = 0; s < splits; ++s) acc += ws[s * split_stride + idx];
+            float *p = ep.out + (long long)br * ep.ldo + ar;
+            if constexpr (EPI == EPI_ADD)
+                *p += acc;
+            else
+                *p = acc;
+        }
+    }
+}
+
+}  // namespace gemm

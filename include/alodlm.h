@@ -1,0 +1,199 @@
+/*
+ * alodlm.h — C ABI of the ALoDLM denoising-step library (libalodlm.so), sm_100a only.
+ *
+ * One denoising step of an adaptively looped masked diffusion LM ("ALoDLM: Adaptively
+ * Looped Diffusion Language Models", paper digest page, sections "Core method",
+ * "Method steps" (Algorithm 1) and Eq. 3).  The model is a Qwen3-style decoder cut into
+ * a Prelude, a weight-shared Recurrent Core that is looped per token, and a Coda; after
+ * each loop the Coda's readout r^(s) feeds an LM head (vocab distribution, entropy,
+ * argmax) and an ExitGate (halting probability).  Confident positions commit their
+ * argmax token, whose embedding re-enters the loop as discrete context (Eq. 3); the
+ * others carry their latent state into the next loop, up to K.  A depth-aware KV cache
+ * serves the prefix at the matching loop depth, falling back to the deepest depth the
+ * position reached (section "Technical novelty").
+ *
+ * Conventions for every entry point:
+ *   - Returns ALODLM_OK (0) or a negative ALODLM_E* code; nothing aborts or exits and no
+ *     exception crosses the ABI.  alodlm_last_error() gives a one-line reason.
+ *   - "device" pointers are CUDA device memory of the handle's device, "host" pointers
+ *     are ordinary host memory.  The caller owns every buffer it passes in; the handle
+ *     owns the packed weights, the KV arena and all scratch.
+ *   - Work is enqueued on the handle's stream; calls return before the GPU finishes
+ *     unless stated otherwise.  alodlm_sync() waits and reports device-side errors.
+ *   - A handle is not thread-safe: one host thread at a time.
+ */
+#ifndef ALODLM_H
+#define ALODLM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define ALODLM_OK 0
+#define ALODLM_EINVAL (-1)   /* bad argument: null pointer, size out of range, unsupported shape */
+#define ALODLM_ENOMEM (-2)   /* device allocation failed or would pass cfg.mem_limit_bytes */
+#define ALODLM_ECUDA (-3)    /* a CUDA runtime/driver call failed (text in last_error) */
+#define ALODLM_EDEVICE (-4)  /* a kernel flagged an inconsistency (bounds, bad id) */
+#define ALODLM_ETIMEOUT (-5) /* a bounded device-side wait gave up; the step's outputs are invalid */
+#define ALODLM_ESTATE (-6)   /* call out of order (step before prefill, batch differs from prefill) */
+
+/* commit rules (the pages and the benchmark spec differ on the halting threshold) */
+#define ALODLM_RULE_PAPER 0     /* commit H <= tau; stop when mean a over U >= lambda (the pages' q),
+                                   or U empty, or s = K; if nothing committed in the step, commit
+                                   the lowest-entropy position of the last loop */
+#define ALODLM_RULE_PER_TOKEN 1 /* commit H <= tau or a_i >= lambda, and all of U at s = K */
+
+/* storage type of weight matrices handed to alodlm_create */
+#define ALODLM_DTYPE_BF16 0
+#define ALODLM_DTYPE_F32 1
+
+#if defined(__GNUC__)
+#define ALODLM_API __attribute__((visibility("default")))
+#else
+#define ALODLM_API
+#endif
+
+typedef struct alodlm alodlm_t; /* opaque handle */
+
+/* Model and capacity.  Supported: head_dim 64 or 128; hidden, n_q_heads*head_dim and inter
+ * multiples of 16; n_q_heads a multiple of n_kv_heads; n_core >= 1 (n_prelude, n_coda >= 0);
+ * 1 <= k_max <= 64; max_block <= 1024; max_batch <= 1024. */
+typedef struct {
+    int hidden, n_q_heads, n_kv_heads, head_dim, inter, vocab;
+    int n_prelude, n_core, n_coda;
+    int k_max;                          /* deepest loop the KV arena holds (prefill builds 1..k_max) */
+    int max_batch, max_prefix, max_block;
+    float rope_base;                    /* 1e6 for Qwen3 */
+    float rms_eps;                      /* 1e-6 */
+    int mask_id;                        /* [MASK] token id (vocab-1 in the synthetic configs) */
+    int qk_norm;                        /* 1: per-head RMSNorm of q and k (Qwen3) */
+    size_t mem_limit_bytes;             /* 0 = no limit; otherwise create fails with ENOMEM beyond it */
+    int debug_dump;                     /* 1: keep per-loop copies of h^(s-1), h~^(s), r^(s) (parity checks) */
+} alodlm_cfg;
+
+/* One decoder layer: device pointers, row-major [out, in].  Matrices in weights.matrix_dtype,
+ * gains always float32.  q [nq*hd, H], k/v [nkv*hd, H], o [H, nq*hd], gate/up [I, H],
+ * down [H, I]; attn_norm/mlp_norm [H], q_norm/k_norm [hd]. */
+typedef struct {
+    const void *attn_norm, *q, *k, *v, *o, *q_norm, *k_norm, *mlp_norm, *gate, *up, *down;
+} alodlm_layer_w;
+
+typedef struct {
+    int matrix_dtype;             /* ALODLM_DTYPE_BF16 or ALODLM_DTYPE_F32 (rounded to bf16, nearest-even) */
+    const void *embed;            /* device [vocab, hidden], the input embedding Emb */
+    const void *lm_head;          /* device [vocab, hidden] */
+    const float *final_norm;      /* device [hidden] */
+    const float *exit_w;          /* device [hidden], ExitGate weight */
+    float exit_b;                 /* ExitGate bias */
+    const alodlm_layer_w *layers; /* host array, n_prelude + n_core + n_coda entries in model order */
+} alodlm_weights;
+
+/* Outputs of one step, all caller-owned DEVICE buffers. K below is the step's k_max. */
+typedef struct {
+    int32_t *tokens;      /* [B,N] committed token, the given id at non-mask positions, mask_id if uncommitted */
+    int32_t *exit_depth;  /* [B,N] loop s (1..K) at which the position committed, 0 if not */
+    float *entropy;       /* [B,K,N] H_i^(s) in nats for i in U at loop s, NaN elsewhere */
+    float *halt;          /* [B,K,N] lambda_i^(s), NaN elsewhere */
+    float *cum_halt;      /* [B,K,N] a_i^(s) after the loop-s update, NaN elsewhere */
+    int32_t *loops_run;   /* [B] loops the sequence ran in this step */
+    int32_t *active_rows; /* [K] block rows run through Core/Coda at loop s (sequences still looping x N) */
+    int32_t *readout_rows;/* [K] rows read out (|U| summed over looping sequences) at loop s */
+} alodlm_step_out;
+
+/* Create a handle on the current CUDA device.
+ * [digest "Core method"]: Prelude = layers [0, n_prelude), Core = next n_core (weight-shared,
+ * looped), Coda = last n_coda.  The weights are read during the call only (packed to bf16
+ * into handle-owned memory: fused QKV, gate/up interleaved); the caller may free them after.
+ * Allocates the depth-aware KV arena: (n_prelude + k_max*n_core + n_coda) slots of
+ * max_batch x n_kv_heads x (max_prefix + max_block) x head_dim, K and V, bf16.
+ * stream: a cudaStream_t (NULL = legacy default stream).
+ * Errors: EINVAL (shape/null), ENOMEM, ECUDA.  On error *out is NULL and the text is in
+ * alodlm_last_error(NULL). */
+ALODLM_API int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *weights, void *stream, alodlm_t **out);
+
+/* Build the depth-aware KV cache of the prefix.
+ * [digest "Technical novelty", "Prerequisites"]: prefix position j with exit depth e_j runs
+ * the Core e_j times; its Core KV at depth d > e_j is its depth-e_j KV (written at prefill
+ * time, so a step reads one dense slot per depth); the Coda runs once on the depth-e_j state.
+ * Prefix attention is causal; positions are 0..P-1.
+ * prefix_ids: device int32 [B,P], ids in [0, vocab).  exit_depth: device int32 [B,P] in
+ * 1..k_max, or NULL for k_max everywhere.  1 <= B <= max_batch, 1 <= P <= max_prefix.
+ * Replaces any previous prefill.  Errors: EINVAL, ECUDA, EDEVICE (id out of range). */
+ALODLM_API int alodlm_prefill(alodlm_t *h, const int32_t *prefix_ids, int B, int P, const int32_t *exit_depth);
+
+/* One denoising step over a block of N positions per sequence (positions P..P+N-1).
+ * [digest "Method steps", Algorithm 1 (1)-(5); Eq. 3]:
+ *   U = mask positions; h^(0) = Prelude(Emb(block)); for s = 1..k_max:
+ *   h~ = Core(h^(s-1)) against prefix Core KV at depth s; r = RMSNorm_f(Coda(h~));
+ *   for i in U: H_i (entropy, nats), y_i (argmax, lowest id on ties), lambda_i =
+ *   sigmoid(w.r_i + b), a_i += (1 - a_i) lambda_i; commit per `rule`; h^(s) = Emb(y) on
+ *   committed rows, h~ elsewhere; stop per `rule`.  The block attends to the whole prefix
+ *   and to itself (bidirectional).  Sequences that stop leave the batch (rows compacted);
+ *   the readout runs on U rows only; logits never reach global memory.
+ * block_ids: device int32 [B,N]; B must equal the prefill's B; 1 <= N <= max_block;
+ * 1 <= k_max <= cfg.k_max; rule = ALODLM_RULE_*.  lambda is the halting threshold.
+ * Asynchronous except for one 16-byte device-to-host read per loop (loop control).
+ * Errors: EINVAL, ESTATE, ECUDA, ETIMEOUT, EDEVICE. */
+ALODLM_API int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda,
+                        int k_max, int rule, const alodlm_step_out *out);
+
+/* Wait for the handle's stream; returns ETIMEOUT/EDEVICE if a kernel raised the device error
+ * word since the last call (the word is then cleared), ECUDA on a CUDA error. */
+ALODLM_API int alodlm_sync(alodlm_t *h);
+
+/* Free everything the handle owns (synchronises first).  NULL is a no-op. */
+ALODLM_API void alodlm_destroy(alodlm_t *h);
+
+/* Last error text of the handle (or of the last failed create when h is NULL).  Valid until the
+ * next call on the same handle. */
+ALODLM_API const char *alodlm_last_error(const alodlm_t *h);
+
+/* Debug copies (cfg.debug_dump = 1): copy the last step's float32 [B, N, hidden] state of loop
+ * `loop` (1-based) into the caller's device buffer dst (enqueued on the handle's stream):
+ * which = 0 loop input h^(s-1), 1 Core output h~^(s), 2 readout state r^(s) (after the final
+ * RMSNorm).  Rows of sequences that had stopped before `loop` hold stale data.
+ * EINVAL without debug_dump, before a step, or out of range. */
+ALODLM_API int alodlm_debug_state(alodlm_t *h, int which, int loop, float *dst);
+
+/* Copy K (which = 0) or V (1) of KV slot `slot` for sequence b, positions [0, n_pos), into the
+ * caller's device buffer dst laid out bf16 [n_kv_heads, n_pos, head_dim] (handle's stream).
+ * Slots: Prelude layer l -> l; Core layer c at depth d (1-based) -> n_prelude + (d-1)*n_core + c;
+ * Coda layer j -> n_prelude + k_max*n_core + j.  Positions P..P+N-1 hold the last step's block
+ * K/V of the last loop that wrote the slot.  For parity checks.  EINVAL out of range. */
+ALODLM_API int alodlm_kv_slot(alodlm_t *h, int which, int slot, int b, int n_pos, void *dst);
+
+/* Counters of the last denoise step: kernels launched, loops run (max over the batch) and,
+ * if timing was enabled, per kernel class the summed device time (ms) and launch count and the
+ * algorithmic bytes and flops (see alodlm_kernel_class_name).  times/launches/bytes/flops may be
+ * NULL; each is an array of ALODLM_N_KCLASS entries. */
+#define ALODLM_N_KCLASS 8
+ALODLM_API int alodlm_step_stats(const alodlm_t *h, int *kernel_launches, double *times_ms, int *launches,
+                      double *bytes, double *flops);
+/* 1: time every kernel class with CUDA events on the handle's stream during the next steps
+ * (adds event records between launches); 0: off (default). */
+ALODLM_API int alodlm_set_timing(alodlm_t *h, int on);
+/* Name of kernel class k (0 <= k < ALODLM_N_KCLASS): "gemm", "attention", "readout_gemm",
+ * "readout_combine", "norm", "qkv_rope", "commit", "other". */
+ALODLM_API const char *alodlm_kernel_class_name(int k);
+
+/* Plain bf16 GEMM through the library's tcgen05 kernel: C[m, n] = sum_k A[m, k] * W[n, k],
+ * A device bf16 [M, K], W device bf16 [N, K] (both row-major, K-major), C device float32
+ * [M, N].  K a multiple of 8 (16-byte rows for TMA), M, N >= 1, all pointers 16-byte aligned.
+ * workspace: caller-owned device scratch of workspace_bytes >= 256 bytes.  Its first 4 bytes
+ * are the device status word: the caller zeroes it before the call; non-zero afterwards
+ * means a bounded wait inside the kernel timed out and C is invalid.  The remaining bytes
+ * hold split-K partials (too small for the split the heuristic picks = fewer splits); the
+ * sum over splits runs in a fixed order, so results are deterministic.  Runs on `stream` of
+ * the current device and allocates nothing.  For kernel-level tests and benchmarks.
+ * Errors: EINVAL, ECUDA. */
+ALODLM_API int alodlm_gemm_bf16(const void *A, const void *W, float *C, int M, int N, int K, float *workspace,
+                     size_t workspace_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ALODLM_H */

@@ -1,0 +1,215 @@
+"""GPU parity: the CUDA library (through the C ABI) against the CPU oracle on the same
+seeded inputs.
+
+Decisions (tokens, commit masks, exit depths, loops) must match the oracle run in the
+kernels' precision exactly, except where the oracle's deciding value lies within 1e-3 of
+its threshold (those it takes from the GPU, and they are counted).  Continuous values
+(readout and hidden states, entropies, halting) must match the float64 oracle, which
+follows the GPU's decisions, within 2e-2 relative (states) and 1e-2 (entropy, halting).
+"""
+import numpy as np
+import pytest
+import torch
+
+from synth import WORKLOADS, make_exit_depths, make_block_ids
+from tests.gpu_util import (BAND, STATE_REL_TOL, Case, compare_decisions, compare_values, follow_of,
+                            row_rel_err)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    c = Case("tiny", 1, 48, 16, 4)
+    c.prefill()
+    return c
+
+
+@pytest.fixture(scope="module")
+def mid():
+    c = Case("mid", 3, 75, 20, 5)
+    c.prefill()
+    return c
+
+
+def _gemm_ref(A, W):
+    return (A.double() @ W.double().T).float()
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 64), (16, 200, 256), (32, 384, 880), (33, 1376, 256), (100, 512, 320),
+                                   (128, 256, 4096), (300, 640, 768), (2048, 512, 1024), (20, 6144, 4096)])
+def test_gemm_tcgen05_against_fp64(M, N, K):
+    import adaptively_looped_masked_b200 as alo
+    g = torch.Generator(device="cuda").manual_seed(M * 7 + N)
+    A = torch.randn((M, K), device="cuda", generator=g).to(torch.bfloat16)
+    W = torch.randn((N, K), device="cuda", generator=g).to(torch.bfloat16)
+    for ws_size in (64, 64 + 16 * M * N):  # without and with split-K room
+        ws = torch.zeros(ws_size, dtype=torch.float32, device="cuda")
+        C = alo.gemm_bf16(A, W, workspace=ws)
+        torch.cuda.synchronize()
+        assert int(ws[:1].view(torch.int32).item()) == 0
+        ref = _gemm_ref(A, W)
+        err = (C - ref).abs().max().item() / ref.abs().max().item()
+        assert err < 1e-5, (M, N, K, ws_size, err)
+
+
+def _check_prefill_kv(case, oracle, b_list, slots):
+    """KV arena slots against the oracle's cache (bf16 values, rows of hd)."""
+    m = case.m
+    for b in b_list:
+        for key, slot in slots:
+            for which in (0, 1):
+                gpu = case.handle.kv_slot(which, slot, b, case.prefix).float().cpu().numpy()  # [nkv, P, hd]
+                ref = oracle.kv[b][key][which].transpose(1, 0, 2)
+                rel = row_rel_err(gpu, ref)
+                assert rel.max() < 2e-2, (b, key, which, rel.max())
+
+
+def _slots(case):
+    m, K = case.m, case.k_max
+    out = [(("prelude", l), l) for l in range(m.n_prelude)]
+    out += [(("core", c, d), m.n_prelude + (d - 1) * m.n_core + c) for d in range(1, K + 1) for c in range(m.n_core)]
+    out += [(("coda", j), m.n_prelude + K * m.n_core + j) for j in range(m.n_coda)]
+    return out
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_prefill_kv_matches_oracle(name, tiny, mid):
+    case = tiny if name == "tiny" else mid
+    o = case.oracle("bf16")
+    o.prefill(case.prefix_ids)
+    _check_prefill_kv(case, o, range(case.batch), _slots(case))
+
+
+def test_prefill_mixed_exit_depths_fallback():
+    case = Case("mid", 2, 75, 20, 5)
+    e = make_exit_depths(2, 75, 5, seed=2)
+    case.prefill(e)
+    o = case.oracle("bf16")
+    o.prefill(case.prefix_ids, e)
+    _check_prefill_kv(case, o, range(2), _slots(case))
+    # write-time fallback: positions with e_j < d hold exactly their depth-e_j KV
+    m = case.m
+    for b in range(2):
+        for c in range(m.n_core):
+            for d in range(2, 6):
+                kd = case.handle.kv_slot(0, m.n_prelude + (d - 1) * m.n_core + c, b, 75).cpu()
+                for dd in range(1, d):
+                    sel = torch.tensor(e[b] == dd)
+                    ke = case.handle.kv_slot(0, m.n_prelude + (dd - 1) * m.n_core + c, b, 75).cpu()
+                    assert torch.equal(kd[:, sel], ke[:, sel])
+
+
+def _step_parity(case, tau, lam, rule, block_ids=None, k_max=None):
+    K = case.k_max if k_max is None else k_max
+    blk = case.block_ids if block_ids is None else block_ids
+    gpu = case.step(tau, lam, k_max=K, rule=rule, block_ids=blk)
+    ob = case.oracle("bf16")
+    ob.prefill(case.prefix_ids)
+    ref = ob.denoise_step(blk, tau, lam, K, rule, follow=follow_of(gpu), band=BAND)
+    compare_decisions(gpu, ref)
+    compare_values(gpu, ref)
+    followed = [f for f in ref["followed"] if f["kind"] != "argmax" or True]
+    # float64 oracle on the GPU's decisions: continuous values
+    of = case.oracle("fp64")
+    of.prefill(case.prefix_ids)
+    ref64 = of.denoise_step(blk, tau, lam, K, rule, follow=follow_of(gpu), band=np.inf)
+    compare_decisions(gpu, ref64)
+    dH = compare_values(gpu, ref64)
+    for b in range(case.batch):
+        for s in range(1, int(gpu["loops_run"][b]) + 1):
+            for which, key in ((0, "h_in"), (1, "h_tilde"), (2, "r")):
+                st = case.handle.debug_state(which, s)[b].cpu().numpy()
+                rel = row_rel_err(st, ref64[key][b][s - 1])
+                assert rel.max() <= STATE_REL_TOL, (key, b, s, rel.max())
+    return len([f for f in ref["followed"] if f["kind"] in ("commit", "halt", "forced")]), dH
+
+
+@pytest.mark.parametrize("tau", [0.1, 0.6, 0.9])
+@pytest.mark.parametrize("lam", [0.1, 0.9])
+@pytest.mark.parametrize("rule", [0, 1])
+def test_step_parity_tiny(tiny, tau, lam, rule):
+    n_followed, dH = _step_parity(tiny, tau, lam, rule)
+    print(f"tiny tau={tau} lam={lam} rule={rule}: followed {n_followed}, max |dH| vs fp64 {dH:.2e}")
+
+
+@pytest.mark.parametrize("tau", [0.1, 0.6, 0.9])
+@pytest.mark.parametrize("lam", [0.1, 0.9])
+@pytest.mark.parametrize("rule", [0, 1])
+def test_step_parity_mid(mid, tau, lam, rule):
+    n_followed, dH = _step_parity(mid, tau, lam, rule)
+    print(f"mid tau={tau} lam={lam} rule={rule}: followed {n_followed}, max |dH| vs fp64 {dH:.2e}")
+
+
+def test_step_edge_cases(mid):
+    # k_max below the arena's depth, given (non-mask) ids in the block, a block shorter than max_block
+    blk = make_block_ids(mid.m, 3, 20, n_given=4, seed=9)
+    _step_parity(mid, 0.6, 0.9, 0, block_ids=blk, k_max=3)
+    _step_parity(mid, 0.6, 0.5, 1, block_ids=blk[:, :11].copy(), k_max=2)
+    # commits disabled (PAPER): all loops run, one forced commit per sequence
+    _step_parity(mid, -1.0, 2.0, 0)
+    # everything commits at loop 1
+    _step_parity(mid, 1e9, 0.5, 0)
+    # a block without any [MASK]: nothing to read out, every sequence stops after loop 1
+    full = make_block_ids(mid.m, 3, 20, n_given=20, seed=4)
+    gpu = mid.step(0.6, 0.5, rule=0, block_ids=full)
+    np.testing.assert_array_equal(gpu["tokens"], full)
+    assert (gpu["exit_depth"] == 0).all() and (gpu["loops_run"] == 1).all()
+    assert np.isnan(gpu["entropy"]).all()
+
+
+def test_step_is_deterministic(mid):
+    a = mid.step(0.6, 0.9, rule=0)
+    b = mid.step(0.6, 0.9, rule=0)
+    for k in a:
+        np.testing.assert_array_equal(np.nan_to_num(a[k], nan=-7.0), np.nan_to_num(b[k], nan=-7.0))
+    r1 = mid.handle.debug_state(2, 1).cpu()
+    mid.step(0.6, 0.9, rule=0)
+    assert torch.equal(r1, mid.handle.debug_state(2, 1).cpu())
+
+
+def test_full_core_model_without_prelude_or_coda():
+    case = Case("tiny_fullcore", 1, 48, 16, 3)
+    case.prefill()
+    _step_parity(case, 0.6, 0.5, 0)
+    _step_parity(case, 0.6, 0.5, 1)
+
+
+def test_state_and_argument_errors():
+    import adaptively_looped_masked_b200 as alo
+    case = Case("tiny", 2, 48, 16, 4, debug=False)
+    blk = torch.tensor(case.block_ids, device="cuda")
+    with pytest.raises(alo.AlodlmError) as e:
+        case.handle.denoise_step(blk, 0.5, 0.5, 4)
+    assert e.value.code == -6  # ESTATE: no prefill
+    case.prefill()
+    with pytest.raises(alo.AlodlmError) as e:
+        case.handle.denoise_step(blk[:1], 0.5, 0.5, 4)
+    assert e.value.code == -6  # batch differs
+    with pytest.raises(alo.AlodlmError) as e:
+        case.handle.denoise_step(blk, 0.5, 0.5, 5)
+    assert e.value.code == -1  # k_max above the arena's depth
+    with pytest.raises(alo.AlodlmError) as e:
+        case.handle.denoise_step(torch.zeros((2, 17), dtype=torch.int32, device="cuda"), 0.5, 0.5, 4)
+    assert e.value.code == -1  # N above max_block
+    bad = blk.clone()
+    bad[0, 0] = 10 ** 6  # token id out of range: flagged by the embedding gather, reported as EDEVICE
+    with pytest.raises(alo.AlodlmError) as e:
+        case.handle.denoise_step(bad, 0.5, 0.5, 4)
+        case.handle.sync()
+    assert e.value.code == -4
+    case.handle.sync()  # the error word was cleared; the handle stays usable
+    out = case.step(0.6, 0.9)
+    assert (out["exit_depth"] >= 0).all()
+
+
+def test_memory_limit_gives_enomem():
+    import adaptively_looped_masked_b200 as alo
+    from synth import MODELS
+    from tests.gpu_util import _to_cuda
+    from synth import make_weights
+    m = MODELS["tiny"]
+    w = _to_cuda(make_weights(m))
+    with pytest.raises(alo.AlodlmError) as e:
+        alo.Handle(m, w, k_max=4, max_batch=1, max_prefix=48, max_block=16, mem_limit_bytes=1 << 20)
+    assert e.value.code == -2
