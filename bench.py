@@ -1,0 +1,444 @@
+"""Benchmark: committed tokens/s per ALoDLM denoising step on Qwen3-8B-shaped synthetic models.
+
+One "step" is one call of alodlm_denoise_step over one batch: Prelude over the block, the
+looped Core/Coda with the fused readout and commit/merge, until every sequence halts.
+The prefix KV cache is built once (prefill, untimed).  Weights are seeded random bf16 and
+inputs are seeded random prefix ids with an all-[MASK] block (no datasets or trained
+weights exist here; they stand in for the paper's GSM8K decoding).
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload qwen3-8b-bs32] [--impl reference]
+
+Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs its own replica on its
+own batch (sequences are independent; no collective on the data path), value = all ranks'
+committed tokens / max-over-ranks time ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import MODELS, WORKLOADS, make_weights, make_prefix_ids, make_block_ids, make_exit_depths  # noqa: E402
+
+METRIC = "committed tokens/s per denoise step (8B-shape bf16, bs 1/32); % of roofline"
+FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"]))), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------------
+# distributed plumbing
+# ------------------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def all_max(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def all_sum(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("swp", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        loaded = [r["sm"] for r in rows if r["power"] > 200.0] or [r["sm"] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------
+# algorithmic work of a step (roofline)
+# ------------------------------------------------------------------------------------
+
+def layer_params(m):
+    return (m.hidden * m.n_q_heads * m.head_dim * 2 + 2 * m.hidden * m.n_kv_heads * m.head_dim
+            + 3 * m.hidden * m.inter)
+
+
+def step_roofline(m, B, P, N, active_rows, readout_rows, peaks):
+    """T_roof = T_prelude + sum over loops of max(F_s / P_peak, Bytes_s / BW)."""
+    p = layer_params(m)
+    H, V = m.hidden, m.vocab
+    CD = m.n_core + m.n_coda
+    kv_bytes_per_layer_seq = 2 * 2 * m.n_kv_heads * (P + N) * m.head_dim
+    BW = peaks["hbm_gbs"] * 1e9
+    PK = peaks["bf16_tflops_sustained"] * 1e12
+    rows0 = B * N
+    f_pre = 2.0 * rows0 * m.n_prelude * p + 4.0 * rows0 * (P + N) * m.n_q_heads * m.head_dim * m.n_prelude
+    b_pre = 2.0 * p * m.n_prelude + B * m.n_prelude * kv_bytes_per_layer_seq
+    t = max(f_pre / PK, b_pre / BW)
+    total_f, total_b = f_pre, b_pre
+    for rows, R in zip(active_rows, readout_rows):
+        if rows <= 0:
+            continue
+        n_seq = rows // N
+        f = 2.0 * rows * CD * p + 2.0 * R * V * H + 4.0 * rows * (P + N) * m.n_q_heads * m.head_dim * CD
+        by = 2.0 * p * CD + 2.0 * V * H + n_seq * CD * kv_bytes_per_layer_seq
+        t += max(f / PK, by / BW)
+        total_f += f
+        total_b += by
+    return t, total_f, total_b
+
+
+# ------------------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample
+# ------------------------------------------------------------------------------------
+
+def cpu_sample(m, wl, loops_per_seq, commits_per_step, w_dev, budget_s=20.0):
+    """Time the oracle (as it stands) on one sequence: one Core layer over the block against a
+    prefix-sized KV context and one readout of the block; scale to a whole step of the
+    workload using the loops the GPU ran."""
+    from oracle import Oracle
+    from synth import weights_to_numpy
+    from tests.helpers import oracle_cfg
+    li = m.n_prelude  # first Core layer
+    wh = weights_to_numpy(w_dev, layers=[li])
+    o = Oracle(oracle_cfg(m, wl.k_max), {**wh, "layers": {li: wh["layers"][li]}}, precision="fp64")
+    rng = np.random.default_rng(0)
+    P, N = wl.prefix, wl.block
+    kvshape = (P, m.n_kv_heads, m.head_dim)
+    o.kv = [{("core", 0, 1): (rng.standard_normal(kvshape) * 0.5, rng.standard_normal(kvshape) * 0.5)}]
+    o.prefix_len = P
+    h = rng.standard_normal((N, m.hidden)) * 0.02
+    lw = o.layer_weights(li)
+    t0 = time.perf_counter()
+    n_layer = 0
+    while True:
+        o.block_layer(0, ("core", 0, 1), lw, h)
+        n_layer += 1
+        if time.perf_counter() - t0 > budget_s / 2 or n_layer >= 3:
+            break
+    t_layer = (time.perf_counter() - t0) / n_layer
+    o._global("lm_head")
+    t1 = time.perf_counter()
+    o.readout(h)
+    t_read = time.perf_counter() - t1
+    CD = m.n_core + m.n_coda
+    per_seq = [m.n_prelude * t_layer + L * (CD * t_layer + t_read) for L in loops_per_seq]
+    t_step = float(sum(per_seq))
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        nt = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if nt:
+            cores = int(nt[0])
+    except Exception:
+        pass
+    return dict(value=commits_per_step / t_step, unit="tokens/s", cores=cores, kind="oracle",
+                sample=(f"oracle float64, one sequence: one Core layer over the {N}-row block against a "
+                        f"{P}-position KV context ({t_layer:.2f} s) and one {m.vocab}-vocab readout of the block "
+                        f"({t_read:.2f} s), scaled to the step's {sum(loops_per_seq)} sequence-loops "
+                        f"(P_l + loops x (C + D) layers + loops readouts per sequence): {t_step:.1f} s per step"),
+                seconds_per_step=t_step)
+
+
+# ------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------
+
+def run_ours(args, world, rank, local):
+    import adaptively_looped_masked_b200 as alo
+    wl = WORKLOADS[args.workload]
+    m = MODELS[wl.model]
+    peaks, peaks_src = load_peaks()
+    stream = torch.cuda.Stream()
+    w = make_weights(m, seed=0, device="cuda")
+    handle = alo.Handle(m, w, k_max=wl.k_max, max_batch=wl.batch, max_prefix=wl.prefix, max_block=wl.block,
+                        stream=stream)
+    keep_w = w if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    del w
+    torch.cuda.empty_cache()
+    prefix = torch.tensor(make_prefix_ids(m, wl.batch, wl.prefix, seed=1 + rank), device="cuda")
+    exit_depth = None
+    if wl.mixed_exit_depths:
+        exit_depth = torch.tensor(make_exit_depths(wl.batch, wl.prefix, wl.k_max, seed=2 + rank), device="cuda")
+    t0 = time.time()
+    handle.prefill(prefix, exit_depth)
+    handle.sync()
+    prefill_s = time.time() - t0
+    block_np = make_block_ids(m, wl.batch, wl.block)
+    block = torch.tensor(block_np, device="cuda")
+    out = handle.alloc_outputs(wl.batch, wl.block, wl.k_max)
+    tau, lam, rule = args.tau, args.lam, args.rule
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            handle.denoise_step(block, tau, lam, wl.k_max, rule, out=out)
+        handle.sync()
+        commits = int((out["exit_depth"] > 0).sum().item())
+        loops = out["loops_run"].cpu().tolist()
+        active_rows = out["active_rows"].cpu().tolist()
+        readout_rows = out["readout_rows"].cpu().tolist()
+
+        # ---- timed region (device events on the handle's stream) ----
+        clocks = ClockSampler(local)
+        clocks.start()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            handle.denoise_step(block, tau, lam, wl.k_max, rule, out=out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        clk = clocks.stop()
+        handle.sync()
+        ms = e0.elapsed_time(e1)
+        launches_per_step = handle.step_stats()["launches"]
+        commits_last = int((out["exit_depth"] > 0).sum().item())
+        assert commits_last == commits, "the step is deterministic: every timed step commits the same tokens"
+
+        # ---- per-kernel-class device time (separate pass with event records between launches) ----
+        handle.set_timing(True)
+        prof_steps = max(1, min(args.steps, 5))
+        cls_ms, cls_n, cls_b, cls_f = {}, {}, {}, {}
+        for _ in range(prof_steps):
+            handle.denoise_step(block, tau, lam, wl.k_max, rule, out=out)
+            st = handle.step_stats()
+            for k_, v in st["classes"].items():
+                cls_ms[k_] = cls_ms.get(k_, 0.0) + v["ms"]
+                cls_n[k_] = cls_n.get(k_, 0) + v["launches"]
+                cls_b[k_] = cls_b.get(k_, 0.0) + v["bytes"]
+                cls_f[k_] = cls_f.get(k_, 0.0) + v["flops"]
+        handle.set_timing(False)
+
+        # ---- end to end through the public API with host buffers ----
+        ids_host = torch.tensor(block_np).pin_memory()
+        host_out = {k_: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k_, v in out.items()}
+        dev_ids = torch.empty_like(block)
+        h2d = ids_host.numel() * 4
+        d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+        barrier(world)
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            dev_ids.copy_(ids_host, non_blocking=True)
+            handle.denoise_step(dev_ids, tau, lam, wl.k_max, rule, out=out)
+            for k_, v in out.items():
+                host_out[k_].copy_(v, non_blocking=True)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = f0.elapsed_time(f1)
+
+    max_ms = all_max(ms, world)
+    max_e2e = all_max(e2e_ms, world)
+    total_commits = all_sum(float(commits) * args.steps, world)
+    value = total_commits / (max_ms / 1e3)
+    e2e_value = total_commits / (max_e2e / 1e3)
+    ms_step = max_ms / args.steps
+
+    # roofline of the dominant kernel class
+    dom = max(cls_ms, key=lambda k_: cls_ms[k_])
+    g_ms = cls_ms["gemm"] / prof_steps
+    g_launch = cls_n["gemm"] / prof_steps
+    g_b = cls_b["gemm"] / prof_steps
+    g_f = cls_f["gemm"] / prof_steps
+    t_roof, F_step, B_step = step_roofline(m, wl.batch, wl.prefix, wl.block, active_rows, readout_rows, peaks)
+    tensor_bound = (F_step / (peaks["bf16_tflops_sustained"] * 1e12)) > (B_step / (peaks["hbm_gbs"] * 1e9))
+    if tensor_bound:
+        achieved = g_f / (g_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = dict(bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s", frac=achieved / peak,
+                    traffic=None)
+    else:
+        achieved = g_b / (g_ms / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = dict(bound="hbm", achieved=achieved, peak=peak, unit="GB/s", frac=achieved / peak, traffic=None)
+    roof.update(kernel="gemm (tcgen05 linear layers, incl. split-K reduce)", peak_source=peaks_src,
+                launches_per_step=g_launch, ms_per_step=g_ms,
+                algorithmic_per_launch=(g_f / g_launch if tensor_bound else g_b / g_launch),
+                algorithmic_unit=("flop" if tensor_bound else "byte"))
+    kernel_share = {k_: round(v / max(sum(cls_ms.values()), 1e-9), 4) for k_, v in cls_ms.items()}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded random bf16 weights, random prefix ids, "
+                                                      "all-[MASK] block)",
+        "config": {"workload": args.workload, "model": wl.model, "batch_per_gpu": wl.batch, "prefix": wl.prefix,
+                   "block": wl.block, "k_max": wl.k_max, "tau_H": tau, "lambda": lam,
+                   "rule": ["paper", "per_token"][rule], "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (weights 16 GB + KV arena)"},
+        "roofline": roof,
+        "step_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_step,
+                          "bound": "tensor" if tensor_bound else "hbm", "flops": F_step, "bytes": B_step},
+        "committed_per_step": commits, "loops_run": loops, "active_rows": active_rows,
+        "readout_rows": readout_rows, "per_sequence_tokens_per_s": value / (wl.batch * world),
+        "gpu_launches": launches_per_step * args.steps, "kernel_time_share": kernel_share,
+        "dominant_kernel_class": dom, "prefill_s": prefill_s,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_sample(m, wl, loops, commits, keep_w)
+        line["cpu_baseline"] = {k_: cb[k_] for k_ in ("value", "unit", "cores", "kind", "sample")}
+    if args.secondary and world == 1:
+        line["secondary"] = args.secondary_result
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    handle.close()
+
+
+# ------------------------------------------------------------------------------------
+# reference arm: the CPU oracle, as it stands, on bounded samples of the same workload
+# ------------------------------------------------------------------------------------
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    m = MODELS[wl.model]
+    # one Core layer of weights on the host is all the sample needs
+    w = make_weights(m, seed=0, device="cuda" if torch.cuda.is_available() else "cpu")
+    # the GPU arm's loop count is not known here: take every sequence to loop 2 times and
+    # commit the whole block (an optimistic bound for the CPU side)
+    loops = [2] * wl.batch
+    commits = wl.batch * wl.block
+    vals = []
+    t_all = time.perf_counter()
+    for i in range(args.warmup + args.steps):
+        cb = cpu_sample(m, wl, loops, commits, w, budget_s=4.0)
+        if i >= args.warmup:
+            vals.append(cb)
+    elapsed = time.perf_counter() - t_all
+    value = statistics.median(v["value"] for v in vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": statistics.median(v["seconds_per_step"] for v in vals) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": args.workload, "model": wl.model, "batch": wl.batch,
+                                            "prefix": wl.prefix, "block": wl.block, "k_max": wl.k_max},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": vals[0]["cores"], "kind": "oracle",
+                             "sample": vals[0]["sample"] + "; loops per sequence assumed 2, whole block committed"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_s": elapsed}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qwen3-8b-bs32", choices=sorted(WORKLOADS))
+    ap.add_argument("--tau", type=float, default=0.6)
+    ap.add_argument("--lam", type=float, default=0.5)
+    ap.add_argument("--rule", type=int, default=0, choices=[0, 1])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.secondary = None
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -135,6 +135,73 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, visible: np.ndarray,
 
 
 # ----------------------------------------------------------------------------------
+# decisions of one loop ([digest] "Method steps" (3)-(5))
+# ----------------------------------------------------------------------------------
+
+def commit_set(H: np.ndarray, a: np.ndarray, s: int, K: int, rule: int, tau: float, lam: float) -> np.ndarray:
+    """Commit mask over the unresolved positions of loop s.
+
+    PAPER: H <= tau (step (3)).  PER_TOKEN: H <= tau, or a >= lam, or the last loop."""
+    if rule == RULE_PAPER:
+        return H <= tau
+    return (H <= tau) | (a >= lam) | (s == K)
+
+
+def halts(n_left: int, mean_a_left: float, s: int, K: int, rule: int, lam: float) -> bool:
+    """Step (4): the loop ends when nothing is unresolved, at s = K, or (PAPER) when the mean
+    cumulative halt of the unresolved positions reaches the threshold."""
+    if n_left == 0 or s == K:
+        return True
+    return rule == RULE_PAPER and mean_a_left >= lam
+
+
+def forced_pick(H_by_pos: Dict[int, float]) -> int:
+    """Step (5): the lowest-entropy unresolved position (lowest index on ties)."""
+    return min(H_by_pos.items(), key=lambda kv: (kv[1], kv[0]))[0]
+
+
+def replay_decisions(block_ids: np.ndarray, mask_id: int, entropy: np.ndarray, cum_halt: np.ndarray,
+                     token_at, tau: float, lam: float, K: int, rule: int, mean_band: float = 1e-5) -> dict:
+    """Re-take every decision of a step from given per-loop traces (entropy and cumulative
+    halt [B,K,N], NaN outside U) with the rules above, in float32 like the traces.
+    token_at(b, s, i) gives the token a position committing at loop s takes.  Returns
+    tokens, exit_depth, loops_run and the near-threshold halting decisions it could not fix."""
+    B, N = block_ids.shape
+    tau32, lam32 = np.float32(tau), np.float32(lam)
+    tokens = block_ids.astype(np.int64).copy()
+    exit_depth = np.zeros((B, N), np.int64)
+    loops = np.zeros(B, np.int64)
+    ambiguous = []
+    for b in range(B):
+        U = block_ids[b] == mask_id
+        n_commit = 0
+        s_last = 1
+        for s in range(1, K + 1):
+            s_last = s
+            idx = np.nonzero(U)[0]
+            H = entropy[b, s - 1, idx].astype(np.float32)
+            a = cum_halt[b, s - 1, idx].astype(np.float32)
+            c = commit_set(H, a, s, K, rule, tau32, lam32)
+            for i in idx[c]:
+                tokens[b, i] = token_at(b, s, int(i))
+                exit_depth[b, i] = s
+            U[idx[c]] = False
+            n_commit += int(c.sum())
+            left = np.nonzero(U)[0]
+            mean_a = float(np.mean(cum_halt[b, s - 1, left].astype(np.float64))) if len(left) else 0.0
+            if len(left) and rule == RULE_PAPER and abs(mean_a - float(lam32)) < mean_band:
+                ambiguous.append((b, s))
+            if halts(len(left), np.float32(mean_a), s, K, rule, lam32):
+                break
+        if rule == RULE_PAPER and n_commit == 0 and U.any():
+            i = forced_pick({int(i): float(entropy[b, s_last - 1, i]) for i in np.nonzero(U)[0]})
+            tokens[b, i] = token_at(b, s_last, i)
+            exit_depth[b, i] = s_last
+        loops[b] = s_last
+    return dict(tokens=tokens, exit_depth=exit_depth, loops_run=loops, ambiguous=ambiguous)
+
+
+# ----------------------------------------------------------------------------------
 # the model
 # ----------------------------------------------------------------------------------
 
@@ -427,16 +494,13 @@ class Oracle:
                                                             margin=float(top2[1] - top2[0])))
                                 y[t] = int(follow["tokens"][b, i])
                 # (3) commit set B^(s)
-                commit = np.zeros(len(idx), dtype=bool)
+                commit = commit_set(H, a[idx], s, K, rule, tau, lam)
                 for t, i in enumerate(idx):
-                    ent_ok = H[t] <= tau
+                    dec = bool(commit[t])
                     if rule == RULE_PAPER:
-                        dec = ent_ok
                         is_near = near(H[t], tau)
                         margin = H[t] - tau
                     else:
-                        halt_ok = a[i] >= lam
-                        dec = ent_ok or halt_ok or s == K
                         is_near = s < K and (near(H[t], tau) or near(a[i], lam))
                         margin = min(abs(H[t] - tau), abs(a[i] - lam))
                     if is_near:
@@ -453,22 +517,19 @@ class Oracle:
                 n_committed += len(ci)
                 h = self.merge(committed, tok, ht)
                 # (4) halting
-                if not U.any():
+                mean_a = float(np.mean(a[U])) if U.any() else 0.0
+                stop = halts(int(U.sum()), mean_a, s, K, rule, lam)
+                if rule == RULE_PAPER and U.any() and s < K and near(mean_a, lam):
+                    gpu = bool(follow["loops_run"][b] == s)
+                    out["followed"].append(dict(b=b, s=s, i=-1, kind="halt",
+                                                margin=float(mean_a - lam), own=stop, taken=gpu))
+                    stop = gpu
+                if stop:
                     break
-                if rule == RULE_PAPER:
-                    mean_a = float(np.mean(a[U]))
-                    stop = mean_a >= lam
-                    if near(mean_a, lam):
-                        gpu = bool(follow["loops_run"][b] == s)
-                        out["followed"].append(dict(b=b, s=s, i=-1, kind="halt",
-                                                    margin=float(mean_a - lam), own=stop, taken=gpu))
-                        stop = gpu
-                    if stop:
-                        break
             # (5) forced progress: nothing committed in this step -> lowest entropy of the last loop
             if rule == RULE_PAPER and n_committed == 0 and U.any():
                 cand = sorted(last_H.items(), key=lambda kv: (kv[1], kv[0]))
-                i_star = cand[0][0]
+                i_star = forced_pick(last_H)
                 if follow is not None and len(cand) > 1 and cand[1][1] - cand[0][1] < band:
                     gpu_i = [i for i in last_H if follow["exit_depth"][b, i] == s_last]
                     out["followed"].append(dict(b=b, s=s_last, i=int(i_star), kind="forced",

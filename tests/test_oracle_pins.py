@@ -561,3 +561,19 @@ def test_planted_merge_keeps_latent(monkeypatch):
     monkeypatch.setattr(om.Oracle, "merge", bad)
     with pytest.raises(AssertionError):
         test_merge_follows_eq3()
+
+
+@pytest.mark.parametrize("rule", [RULE_PAPER, RULE_PER_TOKEN])
+def test_replay_of_own_traces_reproduces_decisions(rule):
+    """The decision rules re-taken from a run's traces give that run's decisions."""
+    shape = MODELS["mid"]
+    o, _ = build(shape, 5)
+    o.prefill(make_prefix_ids(shape, 3, 30))
+    block = make_block_ids(shape, 3, 12, n_given=2)
+    for tau, lam in ((0.1, 0.1), (0.6, 0.9), (0.9, 0.5), (-1.0, 2.0)):
+        out = o.denoise_step(block, tau, lam, 5, rule)
+        rep = om.replay_decisions(block, shape.mask_id, out["entropy"], out["cum_halt"],
+                                  lambda b, s, i: int(out["tokens"][b, i]), tau, lam, 5, rule)
+        np.testing.assert_array_equal(rep["exit_depth"], out["exit_depth"])
+        np.testing.assert_array_equal(rep["tokens"], out["tokens"])
+        np.testing.assert_array_equal(rep["loops_run"], out["loops_run"])
