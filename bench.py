@@ -415,6 +415,35 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_kernel_gemm(args):
+    """Micro-benchmark of the tcgen05 GEMM alone (alodlm_gemm_bf16): C[M,N] = A[M,K] W[N,K]^T."""
+    import adaptively_looped_masked_b200 as alo
+    M, N, K = (int(x) for x in args.shape.split(","))
+    torch.cuda.set_device(0)
+    g = torch.Generator(device="cuda").manual_seed(0)
+    A = torch.randn((M, K), device="cuda", generator=g).to(torch.bfloat16)
+    W = torch.randn((N, K), device="cuda", generator=g).to(torch.bfloat16)
+    C = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(64 + 8 * M * N, dtype=torch.float32, device="cuda")
+    peaks, src = load_peaks()
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        alo.gemm_bf16(A, W, out=C, workspace=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        alo.gemm_bf16(A, W, out=C, workspace=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    by = 2.0 * N * K + 2.0 * M * K + 4.0 * M * N
+    fl = 2.0 * M * N * K
+    print(json.dumps({"kernel": "gemm_bf16", "M": M, "N": N, "K": K, "ms": ms, "GB/s": by / ms / 1e6,
+                      "TFLOP/s": fl / ms / 1e9, "hbm_frac": by / ms / 1e6 / peaks["hbm_gbs"],
+                      "tensor_frac": fl / ms / 1e9 / peaks["bf16_tflops"], "peak_source": src}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -426,7 +455,13 @@ def main():
     ap.add_argument("--lam", type=float, default=0.5)
     ap.add_argument("--rule", type=int, default=0, choices=[0, 1])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", default=None, choices=["gemm"],
+                    help="micro-benchmark one kernel instead of the step")
+    ap.add_argument("--shape", default="32,24576,4096", help="M,N,K for --kernel gemm")
     args = ap.parse_args()
+    if args.kernel == "gemm":
+        run_kernel_gemm(args)
+        return
     args.secondary = None
     world, rank, local = dist_setup(args.gpus)
     try:
