@@ -83,11 +83,13 @@ def lib() -> ctypes.CDLL:
                                         ctypes.POINTER(ci), ctypes.POINTER(ctypes.c_double),
                                         ctypes.POINTER(ctypes.c_double)]
         L.alodlm_set_timing.argtypes = [vp, ci]
+        L.alodlm_set_graphs.argtypes = [vp, ci]
         L.alodlm_kernel_class_name.argtypes = [ci]
         L.alodlm_kernel_class_name.restype = ctypes.c_char_p
         L.alodlm_gemm_bf16.argtypes = [vp, vp, vp, ci, ci, ci, vp, csz, vp]
         for f in ("alodlm_create", "alodlm_prefill", "alodlm_denoise_step", "alodlm_sync", "alodlm_debug_state",
-                  "alodlm_kv_slot", "alodlm_step_stats", "alodlm_set_timing", "alodlm_gemm_bf16"):
+                  "alodlm_kv_slot", "alodlm_step_stats", "alodlm_set_timing", "alodlm_set_graphs",
+                  "alodlm_gemm_bf16"):
             getattr(L, f).restype = ci
         _lib = L
     return _lib
@@ -165,6 +167,18 @@ class Handle:
         self.B = None
         self.N = None
 
+    def _order_in(self):
+        """The handle's stream waits for work already queued on torch's current stream."""
+        cur = torch.cuda.current_stream()
+        if cur != self.stream:
+            self.stream.wait_stream(cur)
+
+    def _order_out(self):
+        """torch's current stream waits for the handle's stream (results visible to later ops)."""
+        cur = torch.cuda.current_stream()
+        if cur != self.stream:
+            cur.wait_stream(self.stream)
+
     def _check(self, rc: int, what: str):
         if rc:
             raise AlodlmError(rc, f"{what}: {lib().alodlm_last_error(self._h).decode()}")
@@ -185,7 +199,9 @@ class Handle:
         ids = prefix_ids.to(torch.int32).contiguous()
         e = None if exit_depth is None else exit_depth.to(torch.int32).contiguous()
         self._keep = (ids, e)
+        self._order_in()
         self._check(lib().alodlm_prefill(self._h, _ptr(ids), B, P, _ptr(e)), "prefill")
+        self._order_out()
         self.B, self.P = B, P
 
     def alloc_outputs(self, B: int, N: int, k_max: int, device=None) -> dict:
@@ -206,8 +222,10 @@ class Handle:
         if out is None:
             out = self.alloc_outputs(B, N, k_max)
         so = StepOut(**{k: _ptr(v) for k, v in out.items()})
+        self._order_in()
         self._check(lib().alodlm_denoise_step(self._h, _ptr(block_ids), B, N, float(tau_H), float(lam), k_max,
                                               rule, ctypes.byref(so)), "denoise_step")
+        self._order_out()
         self.N = N
         return out
 
@@ -216,17 +234,24 @@ class Handle:
 
     def debug_state(self, which: int, loop: int) -> torch.Tensor:
         dst = torch.empty((self.B, self.N, self.shape.hidden), dtype=torch.float32, device="cuda")
+        self._order_in()
         self._check(lib().alodlm_debug_state(self._h, which, loop, _ptr(dst)), "debug_state")
+        self._order_out()
         return dst
 
     def kv_slot(self, which: int, slot: int, b: int, n_pos: int) -> torch.Tensor:
         s = self.shape
         dst = torch.empty((s.n_kv_heads, n_pos, s.head_dim), dtype=torch.bfloat16, device="cuda")
+        self._order_in()
         self._check(lib().alodlm_kv_slot(self._h, which, slot, b, n_pos, _ptr(dst)), "kv_slot")
+        self._order_out()
         return dst
 
     def set_timing(self, on: bool):
         self._check(lib().alodlm_set_timing(self._h, int(on)), "set_timing")
+
+    def set_graphs(self, on: bool):
+        self._check(lib().alodlm_set_graphs(self._h, int(on)), "set_graphs")
 
     def step_stats(self) -> dict:
         n = ctypes.c_int()

@@ -121,12 +121,13 @@ GemmShape plan_gemm(int M, int Nw, int K, size_t ws_floats) {
 
 template <int BN, int EPI>
 void launch_gemm_bn(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int rowsB, int k_tiles, int kps,
-                    int splits, int a_fastest, const gemm::EpiParams &ep, int *err, cudaStream_t st) {
+                    int splits, int a_fastest, const gemm::EpiParams &ep, int *err, cudaStream_t st,
+                    const int *rowsA_dyn = nullptr) {
     dim3 grid;
     const int ta = cdiv(rowsA, gemm::BM), tb = cdiv(rowsB, BN);
     grid = a_fastest ? dim3(ta, tb, splits) : dim3(tb, ta, splits);
-    gemm::gemm_tc_kernel<BN, EPI><<<grid, 192, gemm::Cfg<BN>::SMEM, st>>>(tA, tB, rowsA, rowsB, k_tiles, kps,
-                                                                           a_fastest, ep, err);
+    gemm::gemm_tc_kernel<BN, EPI><<<grid, 192, gemm::Cfg<BN>::SMEM, st>>>(tA, tB, rowsA, rowsB, rowsA_dyn, k_tiles,
+                                                                           kps, a_fastest, ep, err);
 }
 
 template <int EPI>
@@ -161,6 +162,23 @@ struct LayerDev {
 struct TimedLaunch {
     int cls;
     cudaEvent_t e0, e1;
+};
+
+struct GraphKey {
+    int s, n_act, cur, hi, N, K, rule;
+    float tau, lam;
+    const void *p0, *p1, *p2, *p3, *p4, *p5, *p6, *p7;
+    bool operator==(const GraphKey &o) const {
+        return s == o.s && n_act == o.n_act && cur == o.cur && hi == o.hi && N == o.N && K == o.K &&
+               rule == o.rule && tau == o.tau && lam == o.lam && p0 == o.p0 && p1 == o.p1 && p2 == o.p2 &&
+               p3 == o.p3 && p4 == o.p4 && p5 == o.p5 && p6 == o.p6 && p7 == o.p7;
+    }
+};
+
+struct LoopGraph {
+    GraphKey key;
+    cudaGraphExec_t exec;
+    int n_kernels;
 };
 
 }  // namespace
@@ -223,6 +241,10 @@ struct alodlm {
     // activation tensor maps by (pointer, inner, rows, box rows)
     std::map<std::tuple<const void *, int, int, int>, CUtensorMap> tmcache;
 
+    // CUDA graphs of the loop body
+    bool use_graphs = true;
+    std::vector<LoopGraph> graphs;
+
     // launch accounting
     int launches = 0;
     bool timing = false;
@@ -248,6 +270,11 @@ int fail(alodlm *h, int code, const std::string &msg) {
 
 int cuda_fail(alodlm *h, cudaError_t e, const char *what) {
     return fail(h, ALODLM_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+void clear_graphs(alodlm *h) {
+    for (auto &g : h->graphs) cudaGraphExecDestroy(g.exec);
+    h->graphs.clear();
 }
 
 template <typename T>
@@ -508,6 +535,7 @@ const char *alodlm_last_error(const alodlm_t *h) {
 void alodlm_destroy(alodlm_t *h) {
     if (!h) return;
     cudaStreamSynchronize(h->stream);
+    clear_graphs(h);
     for (void *p : h->allocs) cudaFree(p);
     for (auto e : h->ev_pool) cudaEventDestroy(e);
     if (h->counts_host) cudaFreeHost(h->counts_host);
@@ -793,8 +821,6 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
            (k::plan_kernel<<<1, 1024, 0, h->stream>>>(B, h->iota, N, h->cont, h->U, h->seq_of[0], h->old_slot,
                                                       h->ridx, h->rr_b, h->rr_i, h->counts, 1, K, out->active_rows,
                                                       out->readout_rows, h->d_err)));
-    cudaMemcpyAsync(h->counts_host, h->counts, 4 * sizeof(int), cudaMemcpyDeviceToHost, h->stream);
-
     int n_act = B;
     RowMap map{h->seq_of[0], N, P};
     int M = n_act * N;
@@ -804,63 +830,106 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
     for (int l = 0; l < c.n_prelude; ++l)
         if ((rc = run_layer(h, l, slot_prelude(h, l), M, map, n_act, P + N, 0, x, nullptr))) return rc;
 
-    cudaError_t e = cudaStreamSynchronize(h->stream);
-    if (e != cudaSuccess) return cuda_fail(h, e, "step: first loop plan");
-    int R = h->counts_host[1];
-    if (h->counts_host[2]) return alodlm_sync(h);
-
-    for (int s = 1; s <= K; ++s) {
-        map.seq_of = h->seq_of[cur];
-        M = n_act * N;
-        x = h->hbuf[hi];
+    // One loop: Core, Coda, readout over the U rows (their count is read on the device, the
+    // grids are sized for every row of the looping sequences), commit/merge and the plan of the
+    // next loop, then the 16-byte control word to the host.  With a capture-capable stream the
+    // loop is recorded once per (loop, looping sequences, buffer parity, outputs, thresholds)
+    // as a CUDA graph and replayed.
+    auto enqueue_loop = [&](int s, int n_act_, int cur_, int hi_) -> int {
+        RowMap mp{h->seq_of[cur_], N, P};
+        const int Ml = n_act_ * N;
+        float *xl = h->hbuf[hi_];
         const long long dbg_off = (long long)(s - 1) * c.max_batch * c.max_block * H;
+        int r;
         if (c.debug_dump)
             LAUNCH(KC_OTHER, 0.0, 0.0,
-                   (k::dump_rows_kernel<<<M, 256, 0, h->stream>>>(x, map, H, h->dbg[0] + dbg_off)));
+                   (k::dump_rows_kernel<<<Ml, 256, 0, h->stream>>>(xl, mp, H, h->dbg[0] + dbg_off)));
         for (int cc = 0; cc < c.n_core; ++cc)
-            if ((rc = run_layer(h, c.n_prelude + cc, slot_core(h, cc, s), M, map, n_act, P + N, 0, x, nullptr)))
-                return rc;
+            if ((r = run_layer(h, c.n_prelude + cc, slot_core(h, cc, s), Ml, mp, n_act_, P + N, 0, xl, nullptr)))
+                return r;
         if (c.debug_dump)
             LAUNCH(KC_OTHER, 0.0, 0.0,
-                   (k::dump_rows_kernel<<<M, 256, 0, h->stream>>>(x, map, H, h->dbg[1] + dbg_off)));
-        cudaMemcpyAsync(h->hc, x, (size_t)M * H * sizeof(float), cudaMemcpyDeviceToDevice, h->stream);
+                   (k::dump_rows_kernel<<<Ml, 256, 0, h->stream>>>(xl, mp, H, h->dbg[1] + dbg_off)));
+        cudaMemcpyAsync(h->hc, xl, (size_t)Ml * H * sizeof(float), cudaMemcpyDeviceToDevice, h->stream);
         for (int j = 0; j < c.n_coda; ++j)
-            if ((rc = run_layer(h, c.n_prelude + c.n_core + j, slot_coda(h, j), M, map, n_act, P + N, 0, h->hc,
-                                nullptr)))
-                return rc;
-        LAUNCH(KC_NORM, 4.0 * M * H + 2.0 * R * H, 0.0,
-               (k::final_norm_kernel<<<M, 256, 0, h->stream>>>(h->hc, h->final_norm, h->exit_w, h->exit_b, H,
-                                                               c.rms_eps, map, h->ridx, h->rb, h->lam_rr,
-                                                               c.debug_dump ? h->dbg[2] + dbg_off : nullptr)));
-        if (R > 0) {
+            if ((r = run_layer(h, c.n_prelude + c.n_core + j, slot_coda(h, j), Ml, mp, n_act_, P + N, 0, h->hc,
+                               nullptr)))
+                return r;
+        LAUNCH(KC_NORM, 4.0 * Ml * H + 2.0 * Ml * H, 0.0,
+               (k::final_norm_kernel<<<Ml, 256, 0, h->stream>>>(h->hc, h->final_norm, h->exit_w, h->exit_b, H,
+                                                                c.rms_eps, mp, h->ridx, h->rb, h->lam_rr,
+                                                                c.debug_dump ? h->dbg[2] + dbg_off : nullptr)));
+        {
             gemm::EpiParams ep{};
             ep.partials = h->part;
             ep.n_btiles = h->n_vt;
-            const double bytes = 2.0 * h->V * H + 2.0 * R * H + 16.0 * R * h->n_vt;
-            LAUNCH(KC_RGEMM, bytes, 2.0 * R * h->V * (double)H,
-                   launch_gemm_bn<256, gemm::EPI_READOUT>(h->tm_rb, h->tm_lm, R, h->V, cdiv(H, gemm::BK),
-                                                          cdiv(H, gemm::BK), 1, 1, ep, h->d_err, h->stream));
-            LAUNCH(KC_RCOMB, 16.0 * R * h->n_vt, 0.0,
-                   (k::readout_combine_kernel<<<cdiv(R, 8), 256, 0, h->stream>>>(
-                       h->part, h->n_vt, R, h->rr_b, h->rr_i, h->lam_rr, N, K, s, h->a, h->cur_H, h->cur_y,
-                       out->entropy, out->halt, out->cum_halt)));
+            const double R_est = Ml;  // upper bound on the readout rows (exact counts are on the device)
+            const double bytes = 2.0 * h->V * H + 2.0 * R_est * H + 16.0 * R_est * h->n_vt;
+            LAUNCH(KC_RGEMM, bytes, 2.0 * R_est * h->V * (double)H,
+                   launch_gemm_bn<256, gemm::EPI_READOUT>(h->tm_rb, h->tm_lm, Ml, h->V, cdiv(H, gemm::BK),
+                                                          cdiv(H, gemm::BK), 1, 1, ep, h->d_err, h->stream,
+                                                          h->counts + 1));
+            LAUNCH(KC_RCOMB, 16.0 * R_est * h->n_vt, 0.0,
+                   (k::readout_combine_kernel<<<cdiv(Ml, 8), 256, 0, h->stream>>>(
+                       h->part, h->n_vt, h->counts + 1, h->rr_b, h->rr_i, h->lam_rr, N, K, s, h->a, h->cur_H,
+                       h->cur_y, out->entropy, out->halt, out->cum_halt)));
         }
-        LAUNCH(KC_COMMIT, 16.0 * M + 0.0, 0.0,
-               (k::commit_kernel<<<n_act, 256, 0, h->stream>>>(map, s, K, rule, tau_H, lambda, h->embed, H, x, st)));
-        LAUNCH(KC_COMMIT, 8.0 * M, 0.0,
-               (k::plan_kernel<<<1, 1024, 0, h->stream>>>(n_act, h->seq_of[cur], N, h->cont, h->U,
-                                                          h->seq_of[cur ^ 1], h->old_slot, h->ridx, h->rr_b, h->rr_i,
-                                                          h->counts, s + 1, K, out->active_rows, out->readout_rows,
-                                                          h->d_err)));
+        LAUNCH(KC_COMMIT, 16.0 * Ml, 0.0,
+               (k::commit_kernel<<<n_act_, 256, 0, h->stream>>>(mp, s, K, rule, tau_H, lambda, h->embed, H, xl,
+                                                               st)));
+        LAUNCH(KC_COMMIT, 8.0 * Ml, 0.0,
+               (k::plan_kernel<<<1, 1024, 0, h->stream>>>(n_act_, h->seq_of[cur_], N, h->cont, h->U,
+                                                          h->seq_of[cur_ ^ 1], h->old_slot, h->ridx, h->rr_b,
+                                                          h->rr_i, h->counts, s + 1, K, out->active_rows,
+                                                          out->readout_rows, h->d_err)));
         cudaMemcpyAsync(h->counts_host, h->counts, 4 * sizeof(int), cudaMemcpyDeviceToHost, h->stream);
-        e = cudaStreamSynchronize(h->stream);
+        return ALODLM_OK;
+    };
+
+    const bool graphs = h->use_graphs && !h->timing && h->stream != nullptr && h->stream != cudaStreamLegacy &&
+                        h->stream != cudaStreamPerThread;
+    for (int s = 1; s <= K; ++s) {
+        if (graphs) {
+            const GraphKey key{s, n_act, cur, hi, N, K, rule, tau_H, lambda, out->tokens, out->exit_depth,
+                               out->entropy, out->halt, out->cum_halt, out->loops_run, out->active_rows,
+                               out->readout_rows};
+            cudaGraphExec_t exec = nullptr;
+            for (auto &g : h->graphs)
+                if (g.key == key) exec = g.exec;
+            if (!exec) {
+                if (h->graphs.size() >= 512) clear_graphs(h);
+                const int launches_before = h->launches;
+                cudaError_t e = cudaStreamBeginCapture(h->stream, cudaStreamCaptureModeThreadLocal);
+                if (e != cudaSuccess) return cuda_fail(h, e, "graph capture begin");
+                rc = enqueue_loop(s, n_act, cur, hi);
+                cudaGraph_t graph = nullptr;
+                e = cudaStreamEndCapture(h->stream, &graph);
+                if (rc) {
+                    if (graph) cudaGraphDestroy(graph);
+                    return rc;
+                }
+                if (e != cudaSuccess) return cuda_fail(h, e, "graph capture end");
+                e = cudaGraphInstantiate(&exec, graph, 0);
+                cudaGraphDestroy(graph);
+                if (e != cudaSuccess) return cuda_fail(h, e, "graph instantiate");
+                h->graphs.push_back({key, exec, h->launches - launches_before});
+            } else {
+                for (auto &g : h->graphs)
+                    if (g.exec == exec) h->launches += g.n_kernels;
+            }
+            cudaError_t e = cudaGraphLaunch(exec, h->stream);
+            if (e != cudaSuccess) return cuda_fail(h, e, "graph launch");
+        } else {
+            if ((rc = enqueue_loop(s, n_act, cur, hi))) return rc;
+        }
+        cudaError_t e = cudaStreamSynchronize(h->stream);
         if (e != cudaSuccess) return cuda_fail(h, e, "step: loop control");
         if ((rc = check_launch(h, "step"))) return rc;
         if (h->counts_host[2]) return alodlm_sync(h);
         const int n_next = h->counts_host[0];
-        R = h->counts_host[1];
         if (n_next == 0) break;
         if (n_next != n_act) {
+            x = h->hbuf[hi];
             LAUNCH(KC_COMMIT, 8.0 * n_next * N * H, 0.0,
                    (k::gather_rows_kernel<<<n_next * N, 256, 0, h->stream>>>(x, h->hbuf[hi ^ 1], h->old_slot, N, H)));
             hi ^= 1;
@@ -869,6 +938,13 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
         n_act = n_next;
     }
     return check_launch(h, "step end");
+}
+
+int alodlm_set_graphs(alodlm_t *h, int on) {
+    if (!h) return ALODLM_EINVAL;
+    h->use_graphs = on != 0;
+    if (!h->use_graphs) clear_graphs(h);
+    return ALODLM_OK;
 }
 
 int alodlm_debug_state(alodlm_t *h, int which, int loop, float *dst) {

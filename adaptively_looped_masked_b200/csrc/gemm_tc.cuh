@@ -48,7 +48,8 @@ struct Cfg {
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int rowsA,
-                   int rowsB, int k_tiles, int kt_per_split, int a_fastest, EpiParams ep, int *err) {
+                   int rowsB, const int *rowsA_dyn, int k_tiles, int kt_per_split, int a_fastest, EpiParams ep,
+                   int *err) {
     using C = Cfg<BN>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -61,6 +62,11 @@ __global__ void __launch_bounds__(192, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int a_tile = a_fastest ? blockIdx.x : blockIdx.y;
     const int b_tile = a_fastest ? blockIdx.y : blockIdx.x;
+    if (rowsA_dyn) {  // row count known only on the device (grid sized for the maximum)
+        const int live = *rowsA_dyn;
+        if (a_tile * BM >= live) return;
+        rowsA = min(rowsA, live);
+    }
     const int split = blockIdx.z;
     const int kt0 = split * kt_per_split;
     const int nkt = min(k_tiles, kt0 + kt_per_split) - kt0;  // >= 1 by construction on the host
@@ -242,6 +248,223 @@ __global__ void splitk_reduce_kernel(const float *__restrict__ ws, int splits, l
             else
                 *p = acc;
         }
+    }
+}
+
+}  // namespace gemm
+
+namespace gemm {
+
+// ---------------------------------------------------------------------------------
+// Stream-K variant for few activation rows (one BN-row tile covers them all): a grid of at
+// most one CTA per SM walks a contiguous, equal share of the (weight tile, k-tile) units, so
+// every SM streams the same number of weight bytes.  The accumulator is double-buffered in
+// TMEM (the epilogue of one tile overlaps the MMAs of the next).  A tile whose k range is
+// split across CTAs is finished by the CTA that completes last: it sums the partials in
+// segment order (deterministic, independent of arrival order) and applies the epilogue.
+// ---------------------------------------------------------------------------------
+template <int BN>
+struct SkCfg {
+    static constexpr int STAGES = 8;
+    static constexpr uint32_t A_BYTES = BM * BK * 2;
+    static constexpr uint32_t B_BYTES = BN * BK * 2;
+    static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr uint32_t TMEM_COLS = 2 * BN;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+};
+
+template <int EPI, int BN>
+__device__ __forceinline__ void sk_epilogue(const float (&acc)[BN], int a_row, int lane, int rowsA, int rowsB,
+                                            const EpiParams &ep) {
+    if constexpr (EPI == EPI_SWIGLU) {
+        const int feat = (a_row >> 5) * 16 + (lane & 15);
+#pragma unroll
+        for (int j = 0; j < BN; ++j) {
+            const float up = __shfl_xor_sync(0xffffffffu, acc[j], 16);
+            if (lane < 16 && a_row < rowsA && j < rowsB)
+                ep.act[(long long)j * ep.ld_act + feat] = __float2bfloat16_rn(silu_f(acc[j]) * up);
+        }
+    } else {
+        if (a_row < rowsA) {
+#pragma unroll
+            for (int j = 0; j < BN; ++j) {
+                if (j < rowsB) {
+                    float *p = ep.out + (long long)j * ep.ldo + a_row;
+                    if constexpr (EPI == EPI_ADD)
+                        *p += acc[j];
+                    else
+                        *p = acc[j];
+                }
+            }
+        }
+    }
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_sk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int rowsA,
+                   int rowsB, int k_tiles, int n_tiles, int upc, EpiParams ep, float *ws, int max_seg, int *counters,
+                   int *err) {
+    using C = SkCfg<BN>;
+    constexpr int STAGES = C::STAGES;
+    const long long total = (long long)n_tiles * k_tiles;
+    const long long u0 = (long long)blockIdx.x * upc;
+    const long long u1 = min(total, u0 + upc);
+    if (u0 >= u1) return;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * C::STAGE_BYTES);
+    uint64_t *empty = full + STAGES;
+    uint64_t *tfull = empty + STAGES;  // [2] accumulator buffer ready
+    uint64_t *tempty = tfull + 2;      // [2] accumulator buffer drained
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    int *last_flag = reinterpret_cast<int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull + b, 1);
+            mbar_init(tempty + b, 4);
+        }
+        fence_mbarrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol_w = l2_policy_evict_first();
+            int issued = 0;
+            for (long long u = u0; u < u1; ++u) {
+                const int it = (int)(u - u0);
+                const int s = it % STAGES;
+                if (!mbar_wait(empty + s, ((uint32_t)(it / STAGES) & 1u) ^ 1u, err)) break;
+                const int tile = (int)(u / k_tiles), kt = (int)(u % k_tiles);
+                mbar_arrive_expect_tx(full + s, C::STAGE_BYTES);
+                uint8_t *sa = smem + s * C::STAGE_BYTES;
+                tma_load_2d_hint(sa, &tmA, full + s, kt * BK, tile * BM, pol_w);
+                tma_load_2d(sa + C::A_BYTES, &tmB, full + s, kt * BK, 0);
+                issued = it + 1;
+            }
+            for (int it = max(0, issued - STAGES); it < issued; ++it)
+                mbar_wait(full + (it % STAGES), (uint32_t)(it / STAGES) & 1u, err);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16(BM, BN);
+            int seg = 0;
+            bool ok = true;
+            for (long long u = u0; u < u1 && ok; ++u) {
+                const int it = (int)(u - u0);
+                const int s = it % STAGES;
+                const int kt = (int)(u % k_tiles);
+                const bool first = (u == u0) || kt == 0;
+                const int buf = seg & 1;
+                if (first && !mbar_wait(tempty + buf, ((uint32_t)(seg >> 1) & 1u) ^ 1u, err)) break;
+                if (!mbar_wait(full + s, (uint32_t)(it / STAGES) & 1u, err)) break;
+                tc_fence_after();
+                const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+                const uint64_t da = umma_sdesc_sw128(sa);
+                const uint64_t db = umma_sdesc_sw128(sa + C::A_BYTES);
+#pragma unroll
+                for (int k = 0; k < BK / 16; ++k)
+                    umma_f16(tmem_base + buf * BN, da + 2 * k, db + 2 * k, idesc, (first && k == 0) ? 0u : 1u);
+                umma_commit(empty + s);
+                if (u + 1 == u1 || kt == k_tiles - 1) {
+                    umma_commit(tfull + buf);
+                    ++seg;
+                }
+            }
+            (void)ok;
+        }
+    } else {
+        const int q = warp & 3;
+        const int ep_tid = threadIdx.x - 64;  // 0..127
+        int seg = 0;
+        long long u = u0;
+        while (u < u1) {
+            const int tile = (int)(u / k_tiles);
+            const int kt_begin = (int)(u % k_tiles);
+            const long long tile_end = (long long)(tile + 1) * k_tiles;
+            const long long seg_end = min(u1, tile_end);
+            const int buf = seg & 1;
+            const bool ready = mbar_wait(tfull + buf, (uint32_t)(seg >> 1) & 1u, err);
+            tc_fence_after();
+            float acc[BN];
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
+#pragma unroll
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                float v[16];
+                tmem_ld16(taddr + c0, v);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) acc[c0 + j] = v[j];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty + buf);
+            if (!ready) break;
+            const int a_row = tile * BM + q * 32 + lane;
+            if (kt_begin == 0 && seg_end == tile_end) {
+                sk_epilogue<EPI, BN>(acc, a_row, lane, rowsA, rowsB, ep);
+            } else {
+                const int c_first = (int)(((long long)tile * k_tiles) / upc);
+                const int c_last = (int)((tile_end - 1) / upc);
+                const int nseg = c_last - c_first + 1;
+                const int myseg = (int)blockIdx.x - c_first;
+                float *mine = ws + (((long long)tile * max_seg + myseg) * BM + q * 32 + lane) * BN;
+#pragma unroll
+                for (int j = 0; j < BN; j += 4)
+                    *reinterpret_cast<float4 *>(mine + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                __threadfence();
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (ep_tid == 0) {
+                    const int prev = atomicAdd(counters + tile, 1);
+                    *last_flag = (prev == nseg - 1);
+                    if (prev == nseg - 1) counters[tile] = 0;  // every segment has arrived: re-arm
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (*last_flag) {
+                    __threadfence();
+                    float sum[BN];
+#pragma unroll
+                    for (int j = 0; j < BN; ++j) sum[j] = 0.f;
+                    for (int sg = 0; sg < nseg; ++sg) {
+                        const float *p = ws + (((long long)tile * max_seg + sg) * BM + q * 32 + lane) * BN;
+#pragma unroll
+                        for (int j = 0; j < BN; j += 4) {
+                            const float4 v = __ldcg(reinterpret_cast<const float4 *>(p + j));
+                            sum[j] += v.x;
+                            sum[j + 1] += v.y;
+                            sum[j + 2] += v.z;
+                            sum[j + 3] += v.w;
+                        }
+                    }
+                    sk_epilogue<EPI, BN>(sum, a_row, lane, rowsA, rowsB, ep);
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");  // last_flag is reused by the next segment
+            }
+            ++seg;
+            u = seg_end;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
 }
 

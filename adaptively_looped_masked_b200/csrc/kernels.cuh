@@ -235,12 +235,12 @@ __device__ __forceinline__ Stat merge_stat(Stat a, Stat b) {
 // One warp per readout row: merge the per-vocab-tile (max, sum e^(z-max), sum e^(z-max)(z-max),
 // argmax) in a fixed order -> entropy H = log S - T/S (nats) and argmax; then the cumulative
 // halt a <- a + (1 - a) lambda and the traces.
-__global__ void readout_combine_kernel(const float4 *part, int n_vt, int R, const int *rr_b, const int *rr_i,
-                                       const float *lam_rr, int N, int Kstep, int s, float *a_state, float *cur_H,
-                                       int *cur_y, float *tr_H, float *tr_lam, float *tr_a) {
+__global__ void readout_combine_kernel(const float4 *part, int n_vt, const int *R_dev, const int *rr_b,
+                                       const int *rr_i, const float *lam_rr, int N, int Kstep, int s, float *a_state,
+                                       float *cur_H, int *cur_y, float *tr_H, float *tr_lam, float *tr_a) {
     const int rr = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (rr >= R) return;
+    if (rr >= *R_dev) return;
     const float4 *p = part + (long long)rr * n_vt;
     Stat acc = {-INFINITY, 0.f, 0.f, 0x7fffffff};
     bool have = false;

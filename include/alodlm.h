@@ -176,6 +176,11 @@ ALODLM_API int alodlm_step_stats(const alodlm_t *h, int *kernel_launches, double
 /* 1: time every kernel class with CUDA events on the handle's stream during the next steps
  * (adds event records between launches); 0: off (default). */
 ALODLM_API int alodlm_set_timing(alodlm_t *h, int on);
+/* 1 (default): record each loop of a step as a CUDA graph on first use and replay it (needs a
+ * stream other than the legacy/per-thread default stream; timing mode launches directly);
+ * 0: launch every kernel directly and drop the recorded graphs. */
+ALODLM_API int alodlm_set_graphs(alodlm_t *h, int on);
+
 /* Name of kernel class k (0 <= k < ALODLM_N_KCLASS): "gemm", "attention", "readout_gemm",
  * "readout_combine", "norm", "qkv_rope", "commit", "other". */
 ALODLM_API const char *alodlm_kernel_class_name(int k);

@@ -25,8 +25,9 @@ class Case:
         self.w_dev = make_weights(self.m, seed=seed, device="cuda" if big else "cpu")
         if not big:
             self.w_dev = _to_cuda(self.w_dev)
+        self.stream = stream if stream is not None else torch.cuda.Stream()
         self.handle = alo.Handle(self.m, self.w_dev, k_max=k_max, max_batch=batch, max_prefix=prefix,
-                                 max_block=block, debug_dump=debug, stream=stream)
+                                 max_block=block, debug_dump=debug, stream=self.stream)
         self.prefix_ids = make_prefix_ids(self.m, batch, prefix)
         self.block_ids = make_block_ids(self.m, batch, block)
         self._w_host = None
