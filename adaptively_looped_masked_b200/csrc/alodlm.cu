@@ -26,6 +26,8 @@ constexpr int NUM_SMS_HINT = 148;
 constexpr int PREFILL_ROWS = 16384;         // rows of one prefill group (sequences x P)
 constexpr size_t SPLITK_WS_FLOATS = 32u << 20;  // split-K partials (128 MB)
 constexpr size_t ATTN_WS_FLOATS = 16u << 20;    // split-KV partials (64 MB)
+constexpr int SK_COUNTERS = 4096;               // stream-K tile counters
+constexpr int ATTN_COUNTERS = 16384;            // split-KV merge counters
 
 enum KClass { KC_GEMM = 0, KC_ATTN, KC_RGEMM, KC_RCOMB, KC_NORM, KC_QKV, KC_COMMIT, KC_OTHER };
 const char *kclass_names[ALODLM_N_KCLASS] = {"gemm", "attention", "readout_gemm", "readout_combine",
@@ -72,6 +74,11 @@ void set_gemm_attr() {
     cudaFuncSetAttribute(gemm::gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)gemm::Cfg<BN>::SMEM);
 }
+template <int BN, int EPI>
+void set_sk_attr() {
+    cudaFuncSetAttribute(gemm::gemm_sk_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)gemm::SkCfg<BN>::SMEM);
+}
 bool init_kernel_attrs() {
     static bool done[64] = {false};
     int dev = 0;
@@ -91,6 +98,12 @@ bool init_kernel_attrs() {
     set_gemm_attr<256, gemm::EPI_ADD>();
     set_gemm_attr<256, gemm::EPI_SWIGLU>();
     set_gemm_attr<256, gemm::EPI_READOUT>();
+    set_sk_attr<32, gemm::EPI_F32>();
+    set_sk_attr<32, gemm::EPI_ADD>();
+    set_sk_attr<32, gemm::EPI_SWIGLU>();
+    set_sk_attr<64, gemm::EPI_F32>();
+    set_sk_attr<64, gemm::EPI_ADD>();
+    set_sk_attr<64, gemm::EPI_SWIGLU>();
     cudaFuncSetAttribute(attn::attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 5 * 64 * 64 * 2);
     cudaFuncSetAttribute(attn::attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 5 * 64 * 128 * 2);
     done[dev] = cudaGetLastError() == cudaSuccess;
@@ -151,6 +164,105 @@ void launch_splitk_reduce(int epi, const float *ws, int splits, long long sstrid
         gemm::splitk_reduce_kernel<gemm::EPI_SWIGLU><<<blocks, 256, 0, st>>>(ws, splits, sstride, rowsA, rowsB, ep);
     else
         gemm::splitk_reduce_kernel<gemm::EPI_F32><<<blocks, 256, 0, st>>>(ws, splits, sstride, rowsA, rowsB, ep);
+}
+
+// Where a GEMM may put its scratch: split-K / stream-K partials, stream-K tile counters
+// (zero between launches; every launch leaves them zero), the device error word.
+struct GemmEnv {
+    float *ws;
+    size_t ws_floats;
+    int *counters;
+    int n_counters;
+    int *err;
+    cudaStream_t st;
+    int num_sms;
+};
+
+struct SkPlan {
+    int bn, grid, upc, max_seg, n_tiles, k_tiles;
+};
+
+// Stream-K partition: at most one CTA per SM, equal numbers of (weight tile, k-tile) units.
+SkPlan plan_sk(int M, int Nw, int K, int num_sms) {
+    SkPlan p;
+    p.bn = M <= 32 ? 32 : 64;
+    p.k_tiles = cdiv(K, gemm::BK);
+    p.n_tiles = cdiv(Nw, gemm::BM);
+    const long long total = (long long)p.n_tiles * p.k_tiles;
+    const int grid0 = (int)std::min<long long>(num_sms, total);
+    p.upc = (int)((total + grid0 - 1) / grid0);
+    p.grid = (int)((total + p.upc - 1) / p.upc);
+    p.max_seg = 1;
+    for (int t = 0; t < p.n_tiles; ++t) {
+        const long long a = (long long)t * p.k_tiles, b = (long long)(t + 1) * p.k_tiles - 1;
+        p.max_seg = std::max(p.max_seg, (int)(b / p.upc - a / p.upc + 1));
+    }
+    return p;
+}
+
+template <int BN, int EPI>
+void launch_sk_bn(const SkPlan &p, const CUtensorMap &tW, const CUtensorMap &tB, int Nw, int M,
+                  const gemm::EpiParams &ep, const GemmEnv &env) {
+    gemm::gemm_sk_kernel<BN, EPI><<<p.grid, 192, gemm::SkCfg<BN>::SMEM, env.st>>>(
+        tW, tB, Nw, M, p.k_tiles, p.n_tiles, p.upc, ep, env.ws, p.max_seg, env.counters, env.err);
+}
+
+template <int EPI>
+void launch_sk(const SkPlan &p, const CUtensorMap &tW, const CUtensorMap &tB, int Nw, int M,
+               const gemm::EpiParams &ep, const GemmEnv &env) {
+    if (p.bn == 32)
+        launch_sk_bn<32, EPI>(p, tW, tB, Nw, M, ep, env);
+    else
+        launch_sk_bn<64, EPI>(p, tW, tB, Nw, M, ep, env);
+}
+
+// out = act[M, K] x W[Nw, K]^T with epilogue `epi`.  Few rows (<= 64): stream-K kernel with the
+// split reduction fused; more rows: one CTA per 128 x BN tile, split-K with a fixed-order
+// reduce only when the tiles do not fill the SMs.  map_for_bn(bn) returns the activation's
+// tensor map with BN-row boxes.  Returns the number of kernels launched, or -1 (tensor map
+// failure).
+template <typename MapFn>
+int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_bn, int M, int K, int epi, float *out,
+             int ldo, bf16 *act_out, int ld_act) {
+    gemm::EpiParams ep{};
+    ep.out = out;
+    ep.ldo = ldo;
+    ep.act = act_out;
+    ep.ld_act = ld_act;
+    if (M <= 64) {
+        const SkPlan p = plan_sk(M, Nw, K, env.num_sms);
+        if (p.n_tiles <= env.n_counters && (size_t)p.n_tiles * p.max_seg * gemm::BM * p.bn <= env.ws_floats) {
+            const CUtensorMap *tB = map_for_bn(p.bn);
+            if (!tB) return -1;
+            if (epi == gemm::EPI_F32)
+                launch_sk<gemm::EPI_F32>(p, tmW, *tB, Nw, M, ep, env);
+            else if (epi == gemm::EPI_ADD)
+                launch_sk<gemm::EPI_ADD>(p, tmW, *tB, Nw, M, ep, env);
+            else
+                launch_sk<gemm::EPI_SWIGLU>(p, tmW, *tB, Nw, M, ep, env);
+            return 1;
+        }
+    }
+    GemmShape g = plan_gemm(M, Nw, K, env.ws_floats);
+    const CUtensorMap *tB = map_for_bn(g.bn);
+    if (!tB) return -1;
+    if (g.splits == 1) {
+        if (epi == gemm::EPI_F32)
+            launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, 1, 0, ep, env.err, env.st);
+        else if (epi == gemm::EPI_ADD)
+            launch_gemm_epi<gemm::EPI_ADD>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, 1, 0, ep, env.err, env.st);
+        else
+            launch_gemm_epi<gemm::EPI_SWIGLU>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, 1, 0, ep, env.err, env.st);
+        return 1;
+    } else {
+        gemm::EpiParams ep1{};
+        ep1.out = env.ws;
+        ep1.ldo = Nw;
+        ep1.split_stride = (long long)M * Nw;
+        launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep1, env.err, env.st);
+        launch_splitk_reduce(epi, env.ws, g.splits, (long long)M * Nw, Nw, M, ep, env.st);
+        return 2;
+    }
 }
 
 struct LayerDev {
@@ -219,6 +331,9 @@ struct alodlm {
     float *hbuf[2] = {nullptr, nullptr}, *hc = nullptr, *hexit = nullptr, *qkv = nullptr;
     bf16 *xn = nullptr, *qb = nullptr, *attn_out = nullptr, *act = nullptr;
     float *ws = nullptr, *aws_o = nullptr, *aws_ml = nullptr;
+    int *sk_counters = nullptr, *attn_counters = nullptr;
+    int norm_threads = 256;  // one float4 per thread per row where possible
+    int num_sms = 148;
 
     // readout
     int R_cap = 0, n_vt = 0;
@@ -346,51 +461,15 @@ const CUtensorMap *act_map(alodlm *h, const void *ptr, int inner, int rows, int 
 // C = act[M, K] x W[Nw, K]^T with a fused epilogue (weights on the MMA's M side)
 int linear(alodlm *h, const CUtensorMap &tmW, int Nw, const bf16 *actp, int M, int K, int epi, float *out, int ldo,
            bf16 *act_out, int ld_act) {
-    GemmShape g = plan_gemm(M, Nw, K, SPLITK_WS_FLOATS);
-    const CUtensorMap *tB = act_map(h, actp, K, h->rows_cap, g.bn);
-    if (!tB) return fail(h, ALODLM_ECUDA, "cuTensorMapEncodeTiled failed (activation)");
     const double bytes = 2.0 * Nw * K + 2.0 * M * K +
                          (epi == gemm::EPI_ADD ? 8.0 : (epi == gemm::EPI_SWIGLU ? 1.0 : 4.0)) * M * Nw;
     const double flops = 2.0 * M * Nw * K;
-    gemm::EpiParams ep{};
-    if (g.splits == 1) {
-        ep.out = out;
-        ep.ldo = ldo;
-        ep.split_stride = 0;
-        ep.act = act_out;
-        ep.ld_act = ld_act;
-        switch (epi) {
-            case gemm::EPI_F32:
-                LAUNCH(KC_GEMM, bytes, flops,
-                       launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, 1, 0, ep, h->d_err,
-                                                      h->stream));
-                break;
-            case gemm::EPI_ADD:
-                LAUNCH(KC_GEMM, bytes, flops,
-                       launch_gemm_epi<gemm::EPI_ADD>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, 1, 0, ep, h->d_err,
-                                                      h->stream));
-                break;
-            default:
-                LAUNCH(KC_GEMM, bytes, flops,
-                       launch_gemm_epi<gemm::EPI_SWIGLU>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, 1, 0, ep, h->d_err,
-                                                         h->stream));
-                break;
-        }
-    } else {
-        ep.out = h->ws;
-        ep.ldo = Nw;
-        ep.split_stride = (long long)M * Nw;
-        LAUNCH(KC_GEMM, bytes, flops,
-               launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, h->d_err,
-                                              h->stream));
-        gemm::EpiParams ep2{};
-        ep2.out = out;
-        ep2.ldo = ldo;
-        ep2.act = act_out;
-        ep2.ld_act = ld_act;
-        LAUNCH(KC_GEMM, 0.0, 0.0,
-               launch_splitk_reduce(epi, h->ws, g.splits, (long long)M * Nw, Nw, M, ep2, h->stream));
-    }
+    const GemmEnv env{h->ws, SPLITK_WS_FLOATS, h->sk_counters, SK_COUNTERS, h->d_err, h->stream, h->num_sms};
+    auto map_for_bn = [&](int bn) { return act_map(h, actp, K, h->rows_cap, bn); };
+    int n = 0;
+    LAUNCH(KC_GEMM, bytes, flops, n = run_gemm(env, tmW, Nw, map_for_bn, M, K, epi, out, ldo, act_out, ld_act));
+    if (n < 0) return fail(h, ALODLM_ECUDA, "cuTensorMapEncodeTiled failed (activation)");
+    h->launches += n - 1;
     return ALODLM_OK;
 }
 
@@ -412,6 +491,7 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
     p.out_ld = h->nq * h->hd;
     p.ws_o = h->aws_o;
     p.ws_ml = h->aws_ml;
+    p.counters = h->attn_counters;
     p.m_rows = M;
     p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)h->hd));
     const int Tq = map.rows_per_seq;
@@ -420,8 +500,11 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
     const int ktiles = cdiv(kv_len, 64);
     int splits = 1;
     if (!causal) {
-        splits = std::max(1, std::min(ktiles, cdiv(2 * NUM_SMS_HINT, base)));
-        while (splits > 1 && (size_t)splits * M * h->nq * (h->hd + 2) > ATTN_WS_FLOATS) --splits;
+        // enough CTAs to cover the SMs, but at least 4 key tiles per split
+        splits = std::max(1, std::min(ktiles / 4, cdiv(h->num_sms, base)));
+        while (splits > 1 && ((size_t)splits * M * h->nq * (h->hd + 2) > ATTN_WS_FLOATS ||
+                              (size_t)base > ATTN_COUNTERS))
+            --splits;
     }
     const int kps_tiles = cdiv(ktiles, splits);
     splits = cdiv(ktiles, kps_tiles);
@@ -435,17 +518,6 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
         LAUNCH(KC_ATTN, bytes, flops, (attn::attn_kernel<128><<<grid, 128, 5 * 64 * 128 * 2, h->stream>>>(p)));
     else
         LAUNCH(KC_ATTN, bytes, flops, (attn::attn_kernel<64><<<grid, 128, 5 * 64 * 64 * 2, h->stream>>>(p)));
-    if (splits > 1) {
-        dim3 g2(M, h->nq);
-        if (h->hd == 128)
-            LAUNCH(KC_ATTN, 0.0, 0.0,
-                   (attn::attn_combine_kernel<128><<<g2, 64, 0, h->stream>>>(h->aws_o, h->aws_ml, splits, M, h->nq,
-                                                                            h->attn_out, h->nq * h->hd)));
-        else
-            LAUNCH(KC_ATTN, 0.0, 0.0,
-                   (attn::attn_combine_kernel<64><<<g2, 64, 0, h->stream>>>(h->aws_o, h->aws_ml, splits, M, h->nq,
-                                                                           h->attn_out, h->nq * h->hd)));
-    }
     return ALODLM_OK;
 }
 
@@ -464,11 +536,11 @@ int run_layer(alodlm *h, int li, int slot, int M, const RowMap &map, int n_seq, 
     const int H = h->H, qd = h->nq * h->hd;
     int rc;
     LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
-           (k::rmsnorm_kernel<<<M, 256, 0, h->stream>>>(x, Lw.attn_norm, h->xn, H, h->cfg.rms_eps)));
+           (k::rmsnorm_kernel<<<M, h->norm_threads, 0, h->stream>>>(x, Lw.attn_norm, h->xn, H, h->cfg.rms_eps)));
     if ((rc = linear(h, Lw.tm_qkv, h->n_qkv, h->xn, M, H, gemm::EPI_F32, h->qkv, h->n_qkv, nullptr, 0))) return rc;
     bf16 *kc = h->kv_k + (long long)slot * h->slot_elems, *vc = h->kv_v + (long long)slot * h->slot_elems;
     LAUNCH(KC_QKV, 6.0 * M * h->n_qkv, 0.0,
-           (k::qkv_post_kernel<<<M, 256, 0, h->stream>>>(h->qkv, h->nq, h->nkv, h->hd, Lw.q_norm, Lw.k_norm,
+           (k::qkv_post_kernel<<<dim3(M, cdiv(h->nq + 2 * h->nkv, 8)), 256, 0, h->stream>>>(h->qkv, h->nq, h->nkv, h->hd, Lw.q_norm, Lw.k_norm,
                                                           h->cfg.qk_norm, h->cfg.rms_eps, h->rope, map, h->qb, kc, vc,
                                                           h->seq_stride, h->head_stride)));
     if (fb) {
@@ -481,7 +553,7 @@ int run_layer(alodlm *h, int li, int slot, int M, const RowMap &map, int n_seq, 
     if ((rc = attention(h, slot, M, map, n_seq, kv_len, causal))) return rc;
     if ((rc = linear(h, Lw.tm_o, H, h->attn_out, M, qd, gemm::EPI_ADD, x, H, nullptr, 0))) return rc;
     LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
-           (k::rmsnorm_kernel<<<M, 256, 0, h->stream>>>(x, Lw.mlp_norm, h->xn, H, h->cfg.rms_eps)));
+           (k::rmsnorm_kernel<<<M, h->norm_threads, 0, h->stream>>>(x, Lw.mlp_norm, h->xn, H, h->cfg.rms_eps)));
     if ((rc = linear(h, Lw.tm_gu, 2 * h->I, h->xn, M, H, gemm::EPI_SWIGLU, nullptr, 0, h->act, h->I))) return rc;
     if ((rc = linear(h, Lw.tm_d, H, h->act, M, h->I, gemm::EPI_ADD, x, H, nullptr, 0))) return rc;
     return ALODLM_OK;
@@ -564,6 +636,8 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
     h->cfg = *cfg;
     h->stream = static_cast<cudaStream_t>(stream);
     cudaGetDevice(&h->device);
+    cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+    h->norm_threads = std::max(32, std::min(1024, round_up(cfg->hidden / 4, 32)));
     h->H = cfg->hidden;
     h->nq = cfg->n_q_heads;
     h->nkv = cfg->n_kv_heads;
@@ -667,8 +741,11 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
         (rc = dalloc(h, &h->qb, R * qd)) || (rc = dalloc(h, &h->attn_out, R * qd)) ||
         (rc = dalloc(h, &h->act, R * h->I)) || (rc = dalloc(h, &h->ws, SPLITK_WS_FLOATS)) ||
         (rc = dalloc(h, &h->aws_o, ATTN_WS_FLOATS)) ||
-        (rc = dalloc(h, &h->aws_ml, ATTN_WS_FLOATS / 16)))
+        (rc = dalloc(h, &h->aws_ml, ATTN_WS_FLOATS / 16)) || (rc = dalloc(h, &h->sk_counters, SK_COUNTERS)) ||
+        (rc = dalloc(h, &h->attn_counters, ATTN_COUNTERS)))
         return cleanup(rc);
+    cudaMemsetAsync(h->sk_counters, 0, SK_COUNTERS * sizeof(int), h->stream);
+    cudaMemsetAsync(h->attn_counters, 0, ATTN_COUNTERS * sizeof(int), h->stream);
     // zero the activation buffers once so rows past the live ones never hold NaN patterns
     cudaMemsetAsync(h->xn, 0, R * H * 2, h->stream);
     cudaMemsetAsync(h->attn_out, 0, R * qd * 2, h->stream);
@@ -996,29 +1073,32 @@ int alodlm_gemm_bf16(const void *A, const void *W, float *C, int M, int N, int K
     if (!A || !W || !C || !workspace || workspace_bytes < 256 || M < 1 || N < 1 || K < 8 || K % 8)
         return ALODLM_EINVAL;
     if (!get_encode_fn() || !init_kernel_attrs()) return ALODLM_ECUDA;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // first 256 bytes: the device status word; the rest: split-K partials
-    int *err = reinterpret_cast<int *>(workspace);
-    float *parts = workspace + 64;
-    const size_t part_floats = (workspace_bytes - 256) / sizeof(float);
-    GemmShape g = plan_gemm(M, N, K, part_floats);
-    CUtensorMap tW, tA;
-    if (!make_tmap(&tW, W, K, N, gemm::BM) || !make_tmap(&tA, A, K, M, g.bn)) return ALODLM_ECUDA;
-    gemm::EpiParams ep{};
-    if (g.splits == 1) {
-        ep.out = C;
-        ep.ldo = N;
-        launch_gemm_epi<gemm::EPI_F32>(g.bn, tW, tA, N, M, g.k_tiles, g.kps, 1, 0, ep, err, st);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // workspace: [status word | 63 spare floats | tile counters | partials]
+    const size_t total_floats = workspace_bytes / sizeof(float);
+    const int n_tiles = cdiv(N, gemm::BM);
+    const size_t counter_floats = (size_t)cdiv(n_tiles, 64) * 64;
+    GemmEnv env{};
+    env.err = reinterpret_cast<int *>(workspace);
+    env.st = static_cast<cudaStream_t>(stream);
+    env.num_sms = sms;
+    if (total_floats >= 64 + counter_floats) {
+        env.counters = reinterpret_cast<int *>(workspace + 64);
+        env.n_counters = (int)counter_floats;
+        env.ws = workspace + 64 + counter_floats;
+        env.ws_floats = total_floats - 64 - counter_floats;
     } else {
-        ep.out = parts;
-        ep.ldo = N;
-        ep.split_stride = (long long)M * N;
-        launch_gemm_epi<gemm::EPI_F32>(g.bn, tW, tA, N, M, g.k_tiles, g.kps, g.splits, 0, ep, err, st);
-        gemm::EpiParams ep2{};
-        ep2.out = C;
-        ep2.ldo = N;
-        launch_splitk_reduce(gemm::EPI_F32, parts, g.splits, (long long)M * N, N, M, ep2, st);
+        env.counters = nullptr;
+        env.n_counters = 0;
+        env.ws = workspace + 64;
+        env.ws_floats = 0;
     }
+    CUtensorMap tW, tA;
+    if (!make_tmap(&tW, W, K, N, gemm::BM)) return ALODLM_ECUDA;
+    auto map_for_bn = [&](int bn) -> const CUtensorMap * { return make_tmap(&tA, A, K, M, bn) ? &tA : nullptr; };
+    if (run_gemm(env, tW, N, map_for_bn, M, K, gemm::EPI_F32, C, N, nullptr, 0) < 0) return ALODLM_ECUDA;
     return cudaGetLastError() == cudaSuccess ? ALODLM_OK : ALODLM_ECUDA;
 }
 

@@ -5,8 +5,8 @@
 // share every K/V tile load.  K/V tiles of 64 keys are staged in shared memory with
 // cp.async (double-buffered, zero-filled past the last key, XOR-swizzled 16-byte chunks);
 // QK^T and PV run on mma.sync (bf16 in, f32 accumulate) with an online softmax in the
-// exp2 domain.  With n_splits > 1 the keys are split across CTAs (flash-decoding) and a
-// combine kernel merges the partial (max, sum, O) triples in a fixed order.
+// exp2 domain.  With n_splits > 1 the keys are split across CTAs (flash-decoding); the CTA
+// that finishes a query tile last merges the partial (max, sum, O) triples in split order.
 #pragma once
 #include "common.cuh"
 
@@ -23,6 +23,7 @@ struct Params {
     bf16 *out;                     // out[m * out_ld + h * HD + d] (n_splits == 1)
     int out_ld;
     float *ws_o, *ws_ml;           // partials (n_splits > 1): [split][m][h][HD] and [split][m][h][2]
+    int *counters;                 // per (sequence, kv head, query tile): splits done (left at zero)
     int m_rows;                    // rows of the whole launch (for partial indexing)
     float scale_log2;              // log2(e) / sqrt(HD)
 };
@@ -268,28 +269,46 @@ __global__ void __launch_bounds__(128) attn_kernel(Params p) {
             }
         }
     }
-}
+    if (p.n_splits == 1) return;
 
-// merge split partials in split order: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s
-template <int HD>
-__global__ void attn_combine_kernel(const float *__restrict__ ws_o, const float *__restrict__ ws_ml, int n_splits,
-                                    int m_rows, int nq, bf16 *out, int out_ld) {
-    const int m = blockIdx.x, h = blockIdx.y;
-    float M = -INFINITY;
-    for (int s = 0; s < n_splits; ++s) M = fmaxf(M, ws_ml[(((long long)s * m_rows + m) * nq + h) * 2]);
-    float L = 0.f;
-    for (int s = 0; s < n_splits; ++s) {
-        const long long row = ((long long)s * m_rows + m) * nq + h;
-        L += exp2f(ws_ml[row * 2] - M) * ws_ml[row * 2 + 1];
+    // The CTA that finishes a (sequence, kv head, query tile) last merges the split partials in
+    // split order: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s (deterministic).
+    __shared__ int last;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        int *cnt = p.counters + ((long long)j * gridDim.y / p.n_splits + kvh) * gridDim.x + blockIdx.x;
+        const int prev = atomicAdd(cnt, 1);
+        last = prev == p.n_splits - 1;
+        if (last) *cnt = 0;
     }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    for (int d = threadIdx.x; d < HD; d += blockDim.x) {
-        float acc = 0.f;
-        for (int s = 0; s < n_splits; ++s) {
-            const long long row = ((long long)s * m_rows + m) * nq + h;
-            acc += exp2f(ws_ml[row * 2] - M) * ws_o[row * HD + d];
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    const int rows_here = min(64, rows_packed - r0);
+    for (int idx = tid; idx < rows_here * (HD / 4); idx += 128) {
+        const int rl = idx / (HD / 4), d = (idx % (HD / 4)) * 4;
+        const int rp = r0 + rl;
+        const int t = rp / p.G, h = kvh * p.G + rp % p.G;
+        const int m = j * Tq + t;
+        float M = -INFINITY;
+        for (int s = 0; s < p.n_splits; ++s)
+            M = fmaxf(M, __ldcg(p.ws_ml + (((long long)s * p.m_rows + m) * p.nq + h) * 2));
+        float L = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        for (int s = 0; s < p.n_splits; ++s) {
+            const long long row = ((long long)s * p.m_rows + m) * p.nq + h;
+            const float w = exp2f(__ldcg(p.ws_ml + row * 2) - M);
+            L += w * __ldcg(p.ws_ml + row * 2 + 1);
+            const float4 o4 = __ldcg(reinterpret_cast<const float4 *>(p.ws_o + row * HD + d));
+            a0 += w * o4.x;
+            a1 += w * o4.y;
+            a2 += w * o4.z;
+            a3 += w * o4.w;
         }
-        out[(long long)m * out_ld + h * HD + d] = __float2bfloat16_rn(acc * inv);
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        bf16 *dst = p.out + (long long)m * p.out_ld + h * HD + d;
+        *reinterpret_cast<__nv_bfloat162 *>(dst) = __floats2bfloat162_rn(a0 * inv, a1 * inv);
+        *reinterpret_cast<__nv_bfloat162 *>(dst + 2) = __floats2bfloat162_rn(a2 * inv, a3 * inv);
     }
 }
 

@@ -113,7 +113,8 @@ __global__ void qkv_post_kernel(const float *qkv, int nq, int nkv, int hd, const
     const int half = hd >> 1;
     const int n_heads = nq + 2 * nkv;
     const float *row = qkv + (long long)m * n_heads * hd;
-    for (int hh = warp; hh < n_heads; hh += nw) {
+    // blockIdx.y selects a group of nw heads: one warp per (row, head)
+    for (int hh = blockIdx.y * nw + warp; hh < min(n_heads, (int)(blockIdx.y + 1) * nw); hh += nw) {
         float x[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)
@@ -411,14 +412,21 @@ __global__ void commit_kernel(RowMap map, int s, int Kstep, int rule, float tau,
         }
     }
     if (!stop) {
-        // Eq. 3: committed rows re-enter as Emb(y); unresolved and given rows keep h~
-        for (int i = 0; i < N; ++i) {
-            if (st.exit_depth[base + i] == 0) continue;  // uniform across the block
+        // Eq. 3: committed rows re-enter as Emb(y); unresolved and given rows keep h~.
+        // One warp per row, rows spread over the warps.
+        const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
+        for (int i = w; i < N; i += nw) {
+            if (st.exit_depth[base + i] == 0) continue;
             const bf16 *src = emb + (long long)st.tokens[base + i] * H;
             float *dst = h + ((long long)jj * N + i) * H;
-            for (int c = threadIdx.x * 2; c < H; c += blockDim.x * 2)
-                *reinterpret_cast<float2 *>(dst + c) =
-                    __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(src + c));
+            for (int c = l * 8; c < H; c += 32 * 8) {
+                const uint4 raw = *reinterpret_cast<const uint4 *>(src + c);
+                const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+                const float2 f0 = __bfloat1622float2(p2[0]), f1 = __bfloat1622float2(p2[1]);
+                const float2 f2 = __bfloat1622float2(p2[2]), f3 = __bfloat1622float2(p2[3]);
+                *reinterpret_cast<float4 *>(dst + c) = make_float4(f0.x, f0.y, f1.x, f1.y);
+                *reinterpret_cast<float4 *>(dst + c + 4) = make_float4(f2.x, f2.y, f3.x, f3.y);
+            }
         }
     }
 }

@@ -188,12 +188,13 @@ ALODLM_API const char *alodlm_kernel_class_name(int k);
 /* Plain bf16 GEMM through the library's tcgen05 kernel: C[m, n] = sum_k A[m, k] * W[n, k],
  * A device bf16 [M, K], W device bf16 [N, K] (both row-major, K-major), C device float32
  * [M, N].  K a multiple of 8 (16-byte rows for TMA), M, N >= 1, all pointers 16-byte aligned.
- * workspace: caller-owned device scratch of workspace_bytes >= 256 bytes.  Its first 4 bytes
- * are the device status word: the caller zeroes it before the call; non-zero afterwards
- * means a bounded wait inside the kernel timed out and C is invalid.  The remaining bytes
- * hold split-K partials (too small for the split the heuristic picks = fewer splits); the
- * sum over splits runs in a fixed order, so results are deterministic.  Runs on `stream` of
- * the current device and allocates nothing.  For kernel-level tests and benchmarks.
+ * workspace: caller-owned device scratch of workspace_bytes >= 256 bytes, zeroed by the caller
+ * before its first use (calls leave it ready for the next one).  Its first 4 bytes are the
+ * device status word (non-zero after a call means a bounded wait inside the kernel timed out
+ * and C is invalid; the caller clears it); then come per-tile counters and split partials.
+ * With too little room for the split the heuristic picks, fewer splits are used.  Partial
+ * sums are added in a fixed order, so results are deterministic.  Runs on `stream` of the
+ * current device and allocates nothing.  For kernel-level tests and benchmarks.
  * Errors: EINVAL, ECUDA. */
 ALODLM_API int alodlm_gemm_bf16(const void *A, const void *W, float *C, int M, int N, int K, float *workspace,
                      size_t workspace_bytes, void *stream);
