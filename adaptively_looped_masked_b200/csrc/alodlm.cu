@@ -22,6 +22,13 @@
 
 namespace {
 
+#ifndef ALODLM_SK_ENABLE
+#define ALODLM_SK_ENABLE 1
+#endif
+#ifndef ALODLM_SK_CTAS_PER_SM
+#define ALODLM_SK_CTAS_PER_SM 1
+#endif
+
 constexpr int NUM_SMS_HINT = 148;
 constexpr int PREFILL_ROWS = 16384;         // rows of one prefill group (sequences x P)
 constexpr size_t SPLITK_WS_FLOATS = 32u << 20;  // split-K partials (128 MB)
@@ -229,8 +236,8 @@ int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_b
     ep.ldo = ldo;
     ep.act = act_out;
     ep.ld_act = ld_act;
-    if (M <= 64) {
-        const SkPlan p = plan_sk(M, Nw, K, env.num_sms);
+    if (M <= 64 && ALODLM_SK_ENABLE) {
+        const SkPlan p = plan_sk(M, Nw, K, env.num_sms * ALODLM_SK_CTAS_PER_SM);
         if (p.n_tiles <= env.n_counters && (size_t)p.n_tiles * p.max_seg * gemm::BM * p.bn <= env.ws_floats) {
             const CUtensorMap *tB = map_for_bn(p.bn);
             if (!tB) return -1;

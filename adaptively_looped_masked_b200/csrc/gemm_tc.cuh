@@ -263,9 +263,16 @@ namespace gemm {
 // split across CTAs is finished by the CTA that completes last: it sums the partials in
 // segment order (deterministic, independent of arrival order) and applies the epilogue.
 // ---------------------------------------------------------------------------------
+#ifndef ALODLM_SK_STAGES
+#define ALODLM_SK_STAGES 8
+#endif
+#ifndef ALODLM_SK_EVICT_FIRST
+#define ALODLM_SK_EVICT_FIRST 1
+#endif
+
 template <int BN>
 struct SkCfg {
-    static constexpr int STAGES = 8;
+    static constexpr int STAGES = ALODLM_SK_STAGES;
     static constexpr uint32_t A_BYTES = BM * BK * 2;
     static constexpr uint32_t B_BYTES = BN * BK * 2;
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
@@ -355,7 +362,10 @@ __global__ void __launch_bounds__(192, 1)
                 const int tile = (int)(u / k_tiles), kt = (int)(u % k_tiles);
                 mbar_arrive_expect_tx(full + s, C::STAGE_BYTES);
                 uint8_t *sa = smem + s * C::STAGE_BYTES;
-                tma_load_2d_hint(sa, &tmA, full + s, kt * BK, tile * BM, pol_w);
+                if (ALODLM_SK_EVICT_FIRST)
+                    tma_load_2d_hint(sa, &tmA, full + s, kt * BK, tile * BM, pol_w);
+                else
+                    tma_load_2d(sa, &tmA, full + s, kt * BK, tile * BM);
                 tma_load_2d(sa + C::A_BYTES, &tmB, full + s, kt * BK, 0);
                 issued = it + 1;
             }
