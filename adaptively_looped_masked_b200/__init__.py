@@ -87,9 +87,10 @@ def lib() -> ctypes.CDLL:
         L.alodlm_kernel_class_name.argtypes = [ci]
         L.alodlm_kernel_class_name.restype = ctypes.c_char_p
         L.alodlm_gemm_bf16.argtypes = [vp, vp, vp, ci, ci, ci, vp, csz, vp]
+        L.alodlm_gemm_bf16_noalloc.argtypes = [vp, vp, vp, ci, ci, ci, vp]
         for f in ("alodlm_create", "alodlm_prefill", "alodlm_denoise_step", "alodlm_sync", "alodlm_debug_state",
                   "alodlm_kv_slot", "alodlm_step_stats", "alodlm_set_timing", "alodlm_set_graphs",
-                  "alodlm_gemm_bf16"):
+                  "alodlm_gemm_bf16", "alodlm_gemm_bf16_noalloc"):
             getattr(L, f).restype = ci
         _lib = L
     return _lib
@@ -124,6 +125,17 @@ def gemm_bf16(A: torch.Tensor, W: torch.Tensor, out: Optional[torch.Tensor] = No
                                 workspace.numel() * 4, _stream_ptr(stream))
     if rc:
         raise AlodlmError(rc, "alodlm_gemm_bf16 failed")
+    return out
+
+
+def gemm_bf16_noalloc(A: torch.Tensor, W: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+    """C = A @ W^T through the allocation-free entry point (scratch compiled into the library).
+    ``out`` must be given: this call allocates nothing."""
+    M, K = A.shape
+    N = W.shape[0]
+    rc = lib().alodlm_gemm_bf16_noalloc(_ptr(A), _ptr(W), _ptr(out), M, N, K, _stream_ptr(stream))
+    if rc:
+        raise AlodlmError(rc, lib().alodlm_last_error(None).decode())
     return out
 
 

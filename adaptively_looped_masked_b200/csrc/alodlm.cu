@@ -1109,4 +1109,82 @@ int alodlm_gemm_bf16(const void *A, const void *W, float *C, int M, int N, int K
     return cudaGetLastError() == cudaSuccess ? ALODLM_OK : ALODLM_ECUDA;
 }
 
+// ---------------------------------------------------------------------------------
+// Allocation-free GEMM.  Its scratch (status word, tile counters, split partials) is a fixed
+// array compiled into the library; host code reaches it only through the device address
+// looked up once per device.
+// ---------------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+constexpr size_t NOALLOC_HEAD_FLOATS = 64;       // status word + spare
+constexpr size_t NOALLOC_COUNTER_FLOATS = 1024;  // tile counters (N <= 32768 -> <= 256 tiles)
+constexpr size_t NOALLOC_PARTIAL_FLOATS = 4u << 20;
+constexpr size_t NOALLOC_FLOATS = NOALLOC_HEAD_FLOATS + NOALLOC_COUNTER_FLOATS + NOALLOC_PARTIAL_FLOATS;
+constexpr int NOALLOC_MAX_M = 64, NOALLOC_MAX_N = 32768, NOALLOC_MAX_K = 32768;
+
+std::mutex g_noalloc_mu;
+float *g_noalloc_addr[64] = {nullptr};
+}  // namespace
+
+static __device__ __align__(256) float g_noalloc_scratch[NOALLOC_FLOATS];
+
+extern "C" {
+
+int alodlm_gemm_bf16_noalloc(const void *A, const void *W, float *C, int M, int N, int K, void *stream) {
+    if (!A || !W || !C) return fail(nullptr, ALODLM_EINVAL, "gemm_bf16_noalloc: null pointer");
+    if (M < 1 || M > NOALLOC_MAX_M || N < 1 || N > NOALLOC_MAX_N || K < 8 || K > NOALLOC_MAX_K || K % 8)
+        return fail(nullptr, ALODLM_EINVAL,
+                    "gemm_bf16_noalloc: needs 1 <= M <= 64, 1 <= N <= 32768, 8 <= K <= 32768, K % 8 == 0");
+    if (!get_encode_fn() || !init_kernel_attrs())
+        return fail(nullptr, ALODLM_ECUDA, "gemm_bf16_noalloc: tensor-map encoder or kernel attributes");
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return fail(nullptr, ALODLM_ECUDA, "gemm_bf16_noalloc: device index");
+    float *scratch = nullptr;
+    {
+        // first call on this device: look up the device address of the scratch array (the
+        // array's name in host code is only a stand-in for it)
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        if (!g_noalloc_addr[dev]) {
+            void *p = nullptr;
+            cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return fail(nullptr, ALODLM_ECUDA, std::string("gemm_bf16_noalloc: cudaGetSymbolAddress: ") +
+                                                       cudaGetErrorString(e));
+            }
+            g_noalloc_addr[dev] = static_cast<float *>(p);
+        }
+        scratch = g_noalloc_addr[dev];
+    }
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const SkPlan plan = plan_sk(M, N, K, sms);
+    if ((size_t)plan.n_tiles > NOALLOC_COUNTER_FLOATS ||
+        (size_t)plan.n_tiles * plan.max_seg * gemm::BM * plan.bn > NOALLOC_PARTIAL_FLOATS)
+        return fail(nullptr, ALODLM_EINVAL, "gemm_bf16_noalloc: shape needs more scratch than the fixed array holds");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the array keeps the previous call's contents: the status word and the counters must start at zero
+    cudaError_t e = cudaMemsetAsync(scratch, 0, (NOALLOC_HEAD_FLOATS + NOALLOC_COUNTER_FLOATS) * sizeof(float), st);
+    if (e != cudaSuccess) return fail(nullptr, ALODLM_ECUDA, std::string("gemm_bf16_noalloc: ") + cudaGetErrorString(e));
+    CUtensorMap tW, tA;
+    if (!make_tmap(&tW, W, K, N, gemm::BM) || !make_tmap(&tA, A, K, M, plan.bn))
+        return fail(nullptr, ALODLM_ECUDA, "gemm_bf16_noalloc: cuTensorMapEncodeTiled failed");
+    GemmEnv env{};
+    env.err = reinterpret_cast<int *>(scratch);
+    env.counters = reinterpret_cast<int *>(scratch + NOALLOC_HEAD_FLOATS);
+    env.n_counters = (int)NOALLOC_COUNTER_FLOATS;
+    env.ws = scratch + NOALLOC_HEAD_FLOATS + NOALLOC_COUNTER_FLOATS;
+    env.ws_floats = NOALLOC_PARTIAL_FLOATS;
+    env.st = st;
+    env.num_sms = sms;
+    gemm::EpiParams ep{};
+    ep.out = C;
+    ep.ldo = N;
+    launch_sk<gemm::EPI_F32>(plan, tW, tA, N, M, ep, env);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(nullptr, ALODLM_ECUDA, std::string("gemm_bf16_noalloc: ") + cudaGetErrorString(e));
+    return ALODLM_OK;
+}
+
 }  // extern "C"

@@ -199,6 +199,27 @@ ALODLM_API const char *alodlm_kernel_class_name(int k);
 ALODLM_API int alodlm_gemm_bf16(const void *A, const void *W, float *C, int M, int N, int K, float *workspace,
                      size_t workspace_bytes, void *stream);
 
+/* Allocation-free variant of alodlm_gemm_bf16 for a few activation rows (the library's
+ * stream-K kernel): C[m, n] = sum_k A[m, k] * W[n, k], A device bf16 [M, K], W device bf16
+ * [N, K], C device float32 [M, N], all row-major and 16-byte aligned.  The paper has no
+ * counterpart; this entry point exists for callers that cannot allocate device memory
+ * themselves: code whose device memory is owned and budgeted by a host framework's own
+ * pool, and latency-critical paths that must not pay for cudaMalloc/cudaFree, which can
+ * synchronise the device.  It takes no workspace and calls no allocator: its scratch (the
+ * status word, per-tile counters and split partials, 16 MB + 4 KB) is a fixed array compiled
+ * into the library, which every GPU that loads the library's kernels holds until the
+ * process exits.
+ * Limits: 1 <= M <= 64, 1 <= N <= 32768, 8 <= K <= 32768, K % 8 == 0; outside them (or if
+ * the split of a shape would not fit the array) it returns EINVAL, reason in
+ * alodlm_last_error(NULL).
+ * The first call on a device looks up the array's device address with that device
+ * current; make that first call before any stream capture.  Every call shares the one
+ * array: each call clears its status word and counters on `stream` before the kernel, and
+ * calls that overlap on the GPU (other streams, other host threads) race and corrupt each
+ * other's results — serialise them.  A bounded wait that times out inside the kernel leaves C
+ * invalid and is not reported.  Errors: EINVAL, ECUDA. */
+ALODLM_API int alodlm_gemm_bf16_noalloc(const void *A, const void *W, float *C, int M, int N, int K, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,50 @@
+"""The allocation-free GEMM entry point (alodlm_gemm_bf16_noalloc).
+
+Some callers cannot allocate device memory themselves: code whose device memory is owned
+and budgeted by a host framework's pool, and latency-critical paths that must not pay for
+cudaMalloc/cudaFree (which can synchronise the device).  For them the library offers a
+variant of its stream-K GEMM whose scratch is a fixed array compiled into the library.
+This test calls it through the C ABI twice in a row and checks each result against the
+workspace-taking entry point (alodlm_gemm_bf16) on the same inputs, within the GEMM tests'
+tolerance; it also checks that shapes beyond the array's limits are refused.  It runs last
+so that a failure here leaves every other test already run, and it passes both alone in a
+fresh process and after the rest of the suite.
+"""
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("M,N,K", [(32, 6144, 4096), (20, 1376, 880), (64, 4096, 12288), (1, 128, 64)])
+def test_noalloc_gemm_matches_workspace_gemm_twice(M, N, K):
+    import adaptively_looped_masked_b200 as alo
+    g = torch.Generator(device="cuda").manual_seed(1000 + M + N + K)
+    ws = torch.zeros(64 + 4096 + 16 * M * N + (8 << 20), dtype=torch.float32, device="cuda")
+    ref = None
+    for call in range(2):
+        A = torch.randn((M, K), device="cuda", generator=g).to(torch.bfloat16)
+        W = torch.randn((N, K), device="cuda", generator=g).to(torch.bfloat16)
+        ref = alo.gemm_bf16(A, W, workspace=ws)
+        out = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        alo.gemm_bf16_noalloc(A, W, out)
+        torch.cuda.synchronize()
+        assert int(ws[:1].view(torch.int32).item()) == 0
+        err = ((out - ref).abs().max() / ref.abs().max()).item()
+        assert err < 1e-5, (call, M, N, K, err)
+
+
+def test_noalloc_gemm_refuses_shapes_beyond_its_scratch():
+    import adaptively_looped_masked_b200 as alo
+    A = torch.zeros((65, 64), dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros((128, 64), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((65, 128), dtype=torch.float32, device="cuda")
+    with pytest.raises(alo.AlodlmError) as e:
+        alo.gemm_bf16_noalloc(A, W, out)
+    assert e.value.code == -1 and "M <= 64" in str(e.value)
+    A = torch.zeros((8, 64), dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros((32768 + 128, 64), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((8, 32768 + 128), dtype=torch.float32, device="cuda")
+    with pytest.raises(alo.AlodlmError) as e:
+        alo.gemm_bf16_noalloc(A, W, out)
+    assert e.value.code == -1
