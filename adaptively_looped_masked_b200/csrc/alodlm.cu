@@ -22,14 +22,40 @@
 
 namespace {
 
-#ifndef ALODLM_SK_ENABLE
-#define ALODLM_SK_ENABLE 1
+// The step's linear layers use the per-tile kernel at every row count: on B200 it streams
+// the weights faster than the stream-K kernel at 32-64 rows (0.77 vs 0.65 of the measured
+// HBM bandwidth on the 24576 x 4096 gate/up shape).  The GEMM entry points use stream-K for
+// up to 64 rows.
+#ifndef ALODLM_STEP_STREAM_K
+#define ALODLM_STEP_STREAM_K 0
 #endif
 #ifndef ALODLM_SK_CTAS_PER_SM
 #define ALODLM_SK_CTAS_PER_SM 1
 #endif
 
+#ifndef ALODLM_PDL
+#define ALODLM_PDL 1
+#endif
+
 constexpr int NUM_SMS_HINT = 148;
+
+// Launch with programmatic stream serialisation (the kernel may start while its predecessor
+// on the stream finishes; the kernels order themselves with pdl_wait()).  Not on the legacy
+// default stream.
+template <typename... KArgs, typename... Args>
+void klaunch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (ALODLM_PDL && st != nullptr && st != cudaStreamLegacy && st != cudaStreamPerThread) ? 1 : 0;
+    cudaLaunchKernelEx(&cfg, kern, args...);
+}
 constexpr int PREFILL_ROWS = 16384;         // rows of one prefill group (sequences x P)
 constexpr size_t SPLITK_WS_FLOATS = 32u << 20;  // split-K partials (128 MB)
 constexpr size_t ATTN_WS_FLOATS = 16u << 20;    // split-KV partials (64 MB)
@@ -146,7 +172,7 @@ void launch_gemm_bn(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int
     dim3 grid;
     const int ta = cdiv(rowsA, gemm::BM), tb = cdiv(rowsB, BN);
     grid = a_fastest ? dim3(ta, tb, splits) : dim3(tb, ta, splits);
-    gemm::gemm_tc_kernel<BN, EPI><<<grid, 192, gemm::Cfg<BN>::SMEM, st>>>(tA, tB, rowsA, rowsB, rowsA_dyn, k_tiles,
+    klaunch(gemm::gemm_tc_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM, st, tA, tB, rowsA, rowsB, rowsA_dyn, k_tiles,
                                                                            kps, a_fastest, ep, err);
 }
 
@@ -166,11 +192,11 @@ void launch_splitk_reduce(int epi, const float *ws, int splits, long long sstrid
     const long long total = (long long)rowsA * rowsB;
     const int blocks = (int)std::min<long long>((total + 255) / 256, 148 * 8);
     if (epi == gemm::EPI_ADD)
-        gemm::splitk_reduce_kernel<gemm::EPI_ADD><<<blocks, 256, 0, st>>>(ws, splits, sstride, rowsA, rowsB, ep);
+        klaunch(gemm::splitk_reduce_kernel<gemm::EPI_ADD>, blocks, 256, 0, st, ws, splits, sstride, rowsA, rowsB, ep);
     else if (epi == gemm::EPI_SWIGLU)
-        gemm::splitk_reduce_kernel<gemm::EPI_SWIGLU><<<blocks, 256, 0, st>>>(ws, splits, sstride, rowsA, rowsB, ep);
+        klaunch(gemm::splitk_reduce_kernel<gemm::EPI_SWIGLU>, blocks, 256, 0, st, ws, splits, sstride, rowsA, rowsB, ep);
     else
-        gemm::splitk_reduce_kernel<gemm::EPI_F32><<<blocks, 256, 0, st>>>(ws, splits, sstride, rowsA, rowsB, ep);
+        klaunch(gemm::splitk_reduce_kernel<gemm::EPI_F32>, blocks, 256, 0, st, ws, splits, sstride, rowsA, rowsB, ep);
 }
 
 // Where a GEMM may put its scratch: split-K / stream-K partials, stream-K tile counters
@@ -210,7 +236,7 @@ SkPlan plan_sk(int M, int Nw, int K, int num_sms) {
 template <int BN, int EPI>
 void launch_sk_bn(const SkPlan &p, const CUtensorMap &tW, const CUtensorMap &tB, int Nw, int M,
                   const gemm::EpiParams &ep, const GemmEnv &env) {
-    gemm::gemm_sk_kernel<BN, EPI><<<p.grid, 192, gemm::SkCfg<BN>::SMEM, env.st>>>(
+    klaunch(gemm::gemm_sk_kernel<BN, EPI>, p.grid, 192, gemm::SkCfg<BN>::SMEM, env.st, 
         tW, tB, Nw, M, p.k_tiles, p.n_tiles, p.upc, ep, env.ws, p.max_seg, env.counters, env.err);
 }
 
@@ -230,13 +256,13 @@ void launch_sk(const SkPlan &p, const CUtensorMap &tW, const CUtensorMap &tB, in
 // failure).
 template <typename MapFn>
 int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_bn, int M, int K, int epi, float *out,
-             int ldo, bf16 *act_out, int ld_act) {
+             int ldo, bf16 *act_out, int ld_act, bool stream_k) {
     gemm::EpiParams ep{};
     ep.out = out;
     ep.ldo = ldo;
     ep.act = act_out;
     ep.ld_act = ld_act;
-    if (M <= 64 && ALODLM_SK_ENABLE) {
+    if (M <= 64 && stream_k) {
         const SkPlan p = plan_sk(M, Nw, K, env.num_sms * ALODLM_SK_CTAS_PER_SM);
         if (p.n_tiles <= env.n_counters && (size_t)p.n_tiles * p.max_seg * gemm::BM * p.bn <= env.ws_floats) {
             const CUtensorMap *tB = map_for_bn(p.bn);
@@ -358,7 +384,7 @@ struct alodlm {
     int *counts = nullptr, *counts_host = nullptr, *d_err = nullptr;
 
     // debug copies [K][maxB][maxN][H]
-    float *dbg[3] = {nullptr, nullptr, nullptr};
+    float *dbg[4] = {nullptr, nullptr, nullptr, nullptr};
 
     // activation tensor maps by (pointer, inner, rows, box rows)
     std::map<std::tuple<const void *, int, int, int>, CUtensorMap> tmcache;
@@ -474,7 +500,8 @@ int linear(alodlm *h, const CUtensorMap &tmW, int Nw, const bf16 *actp, int M, i
     const GemmEnv env{h->ws, SPLITK_WS_FLOATS, h->sk_counters, SK_COUNTERS, h->d_err, h->stream, h->num_sms};
     auto map_for_bn = [&](int bn) { return act_map(h, actp, K, h->rows_cap, bn); };
     int n = 0;
-    LAUNCH(KC_GEMM, bytes, flops, n = run_gemm(env, tmW, Nw, map_for_bn, M, K, epi, out, ldo, act_out, ld_act));
+    LAUNCH(KC_GEMM, bytes, flops,
+           n = run_gemm(env, tmW, Nw, map_for_bn, M, K, epi, out, ldo, act_out, ld_act, ALODLM_STEP_STREAM_K != 0));
     if (n < 0) return fail(h, ALODLM_ECUDA, "cuTensorMapEncodeTiled failed (activation)");
     h->launches += n - 1;
     return ALODLM_OK;
@@ -522,9 +549,9 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
     const double bytes = kvb + 4.0 * M * h->nq * h->hd;
     const double flops = 4.0 * M * h->nq * (double)kv_len * h->hd * (causal ? 0.5 : 1.0);
     if (h->hd == 128)
-        LAUNCH(KC_ATTN, bytes, flops, (attn::attn_kernel<128><<<grid, 128, 5 * 64 * 128 * 2, h->stream>>>(p)));
+        LAUNCH(KC_ATTN, bytes, flops, (klaunch(attn::attn_kernel<128>, grid, 128, 5 * 64 * 128 * 2, h->stream, p)));
     else
-        LAUNCH(KC_ATTN, bytes, flops, (attn::attn_kernel<64><<<grid, 128, 5 * 64 * 64 * 2, h->stream>>>(p)));
+        LAUNCH(KC_ATTN, bytes, flops, (klaunch(attn::attn_kernel<64>, grid, 128, 5 * 64 * 64 * 2, h->stream, p)));
     return ALODLM_OK;
 }
 
@@ -543,24 +570,24 @@ int run_layer(alodlm *h, int li, int slot, int M, const RowMap &map, int n_seq, 
     const int H = h->H, qd = h->nq * h->hd;
     int rc;
     LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
-           (k::rmsnorm_kernel<<<M, h->norm_threads, 0, h->stream>>>(x, Lw.attn_norm, h->xn, H, h->cfg.rms_eps)));
+           (klaunch(k::rmsnorm_kernel, M, h->norm_threads, 0, h->stream, x, Lw.attn_norm, h->xn, H, h->cfg.rms_eps)));
     if ((rc = linear(h, Lw.tm_qkv, h->n_qkv, h->xn, M, H, gemm::EPI_F32, h->qkv, h->n_qkv, nullptr, 0))) return rc;
     bf16 *kc = h->kv_k + (long long)slot * h->slot_elems, *vc = h->kv_v + (long long)slot * h->slot_elems;
     LAUNCH(KC_QKV, 6.0 * M * h->n_qkv, 0.0,
-           (k::qkv_post_kernel<<<dim3(M, cdiv(h->nq + 2 * h->nkv, 8)), 256, 0, h->stream>>>(h->qkv, h->nq, h->nkv, h->hd, Lw.q_norm, Lw.k_norm,
+           (klaunch(k::qkv_post_kernel, dim3(M, cdiv(h->nq + 2 * h->nkv, 8)), 256, 0, h->stream, h->qkv, h->nq, h->nkv, h->hd, Lw.q_norm, Lw.k_norm,
                                                           h->cfg.qk_norm, h->cfg.rms_eps, h->rope, map, h->qb, kc, vc,
                                                           h->seq_stride, h->head_stride)));
     if (fb) {
         const long long so = (long long)fb->src_slot * h->slot_elems;
         LAUNCH(KC_OTHER, 8.0 * fb->nb * h->nkv * fb->P * h->hd, 0.0,
-               (k::kv_fallback_kernel<<<dim3(fb->nb, h->nkv), 256, 0, h->stream>>>(
+               (klaunch(k::kv_fallback_kernel, dim3(fb->nb, h->nkv), 256, 0, h->stream, 
                    h->exit_dev, fb->P, fb->b0, fb->depth, h->kv_k + so, h->kv_v + so, kc, vc, h->seq_stride,
                    h->head_stride, h->hd)));
     }
     if ((rc = attention(h, slot, M, map, n_seq, kv_len, causal))) return rc;
     if ((rc = linear(h, Lw.tm_o, H, h->attn_out, M, qd, gemm::EPI_ADD, x, H, nullptr, 0))) return rc;
     LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
-           (k::rmsnorm_kernel<<<M, h->norm_threads, 0, h->stream>>>(x, Lw.mlp_norm, h->xn, H, h->cfg.rms_eps)));
+           (klaunch(k::rmsnorm_kernel, M, h->norm_threads, 0, h->stream, x, Lw.mlp_norm, h->xn, H, h->cfg.rms_eps)));
     if ((rc = linear(h, Lw.tm_gu, 2 * h->I, h->xn, M, H, gemm::EPI_SWIGLU, nullptr, 0, h->act, h->I))) return rc;
     if ((rc = linear(h, Lw.tm_d, H, h->act, M, h->I, gemm::EPI_ADD, x, H, nullptr, 0))) return rc;
     return ALODLM_OK;
@@ -784,7 +811,7 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
         cudaMemsetAsync(h->d_err, 0, sizeof(int), h->stream);
     }
     if (cfg->debug_dump) {
-        for (int i = 0; i < 3; ++i)
+        for (int i = 0; i < 4; ++i)
             if ((rc = dalloc(h, &h->dbg[i], (size_t)cfg->k_max * BN_ * H))) return cleanup(rc);
     }
     if (cudaMallocHost(&h->counts_host, 4 * sizeof(int)) != cudaSuccess) {
@@ -837,7 +864,7 @@ int alodlm_prefill(alodlm_t *h, const int32_t *prefix_ids, int B, int P, const i
         RowMap map{h->iota + b0, P, 0};
         float *x = h->hbuf[0];
         LAUNCH(KC_OTHER, 6.0 * M * h->H, 0.0,
-               (k::embed_kernel<<<M, 256, 0, h->stream>>>(prefix_ids, P, map, h->embed, h->V, h->H, x, h->d_err)));
+               (klaunch(k::embed_kernel, M, 256, 0, h->stream, prefix_ids, P, map, h->embed, h->V, h->H, x, h->d_err)));
         for (int l = 0; l < c.n_prelude; ++l)
             if ((rc = run_layer(h, l, slot_prelude(h, l), M, map, nb, P, 1, x, nullptr))) return rc;
         for (int d = 1; d <= c.k_max; ++d) {
@@ -850,7 +877,7 @@ int alodlm_prefill(alodlm_t *h, const int32_t *prefix_ids, int B, int P, const i
             }
             if (exit_depth)
                 LAUNCH(KC_OTHER, 8.0 * M * h->H / c.k_max, 0.0,
-                       (k::capture_exit_kernel<<<M, 256, 0, h->stream>>>(h->exit_dev, P, b0, d, x, h->hexit, h->H)));
+                       (klaunch(k::capture_exit_kernel, M, 256, 0, h->stream, h->exit_dev, P, b0, d, x, h->hexit, h->H)));
         }
         if (exit_depth) x = h->hexit;
         for (int j = 0; j < c.n_coda; ++j)
@@ -899,10 +926,10 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
     int cur = 0, hi = 0, rc;
     const long long BNt = (long long)B * N;
     LAUNCH(KC_COMMIT, 16.0 * BNt, 0.0,
-           (k::step_init_kernel<<<(unsigned)std::min<long long>((BNt + 255) / 256, 1024), 256, 0, h->stream>>>(
+           (klaunch(k::step_init_kernel, (unsigned)std::min<long long>((BNt + 255) / 256, 1024), 256, 0, h->stream, 
                block_ids, B, N, K, c.mask_id, st)));
     LAUNCH(KC_COMMIT, 8.0 * BNt, 0.0,
-           (k::plan_kernel<<<1, 1024, 0, h->stream>>>(B, h->iota, N, h->cont, h->U, h->seq_of[0], h->old_slot,
+           (klaunch(k::plan_kernel, 1, 1024, 0, h->stream, B, h->iota, N, h->cont, h->U, h->seq_of[0], h->old_slot,
                                                       h->ridx, h->rr_b, h->rr_i, h->counts, 1, K, out->active_rows,
                                                       out->readout_rows, h->d_err)));
     int n_act = B;
@@ -910,7 +937,7 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
     int M = n_act * N;
     float *x = h->hbuf[hi];
     LAUNCH(KC_OTHER, 6.0 * M * H, 0.0,
-           (k::embed_kernel<<<M, 256, 0, h->stream>>>(block_ids, N, map, h->embed, h->V, H, x, h->d_err)));
+           (klaunch(k::embed_kernel, M, 256, 0, h->stream, block_ids, N, map, h->embed, h->V, H, x, h->d_err)));
     for (int l = 0; l < c.n_prelude; ++l)
         if ((rc = run_layer(h, l, slot_prelude(h, l), M, map, n_act, P + N, 0, x, nullptr))) return rc;
 
@@ -927,20 +954,24 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
         int r;
         if (c.debug_dump)
             LAUNCH(KC_OTHER, 0.0, 0.0,
-                   (k::dump_rows_kernel<<<Ml, 256, 0, h->stream>>>(xl, mp, H, h->dbg[0] + dbg_off)));
-        for (int cc = 0; cc < c.n_core; ++cc)
+                   (klaunch(k::dump_rows_kernel, Ml, 256, 0, h->stream, xl, mp, H, h->dbg[0] + dbg_off)));
+        for (int cc = 0; cc < c.n_core; ++cc) {
             if ((r = run_layer(h, c.n_prelude + cc, slot_core(h, cc, s), Ml, mp, n_act_, P + N, 0, xl, nullptr)))
                 return r;
+            if (cc == 0 && c.debug_dump)
+                LAUNCH(KC_OTHER, 0.0, 0.0,
+                       (klaunch(k::dump_rows_kernel, Ml, 256, 0, h->stream, xl, mp, H, h->dbg[3] + dbg_off)));
+        }
         if (c.debug_dump)
             LAUNCH(KC_OTHER, 0.0, 0.0,
-                   (k::dump_rows_kernel<<<Ml, 256, 0, h->stream>>>(xl, mp, H, h->dbg[1] + dbg_off)));
+                   (klaunch(k::dump_rows_kernel, Ml, 256, 0, h->stream, xl, mp, H, h->dbg[1] + dbg_off)));
         cudaMemcpyAsync(h->hc, xl, (size_t)Ml * H * sizeof(float), cudaMemcpyDeviceToDevice, h->stream);
         for (int j = 0; j < c.n_coda; ++j)
             if ((r = run_layer(h, c.n_prelude + c.n_core + j, slot_coda(h, j), Ml, mp, n_act_, P + N, 0, h->hc,
                                nullptr)))
                 return r;
         LAUNCH(KC_NORM, 4.0 * Ml * H + 2.0 * Ml * H, 0.0,
-               (k::final_norm_kernel<<<Ml, 256, 0, h->stream>>>(h->hc, h->final_norm, h->exit_w, h->exit_b, H,
+               (klaunch(k::final_norm_kernel, Ml, 256, 0, h->stream, h->hc, h->final_norm, h->exit_w, h->exit_b, H,
                                                                 c.rms_eps, mp, h->ridx, h->rb, h->lam_rr,
                                                                 c.debug_dump ? h->dbg[2] + dbg_off : nullptr)));
         {
@@ -954,15 +985,15 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
                                                           cdiv(H, gemm::BK), 1, 1, ep, h->d_err, h->stream,
                                                           h->counts + 1));
             LAUNCH(KC_RCOMB, 16.0 * R_est * h->n_vt, 0.0,
-                   (k::readout_combine_kernel<<<cdiv(Ml, 8), 256, 0, h->stream>>>(
+                   (klaunch(k::readout_combine_kernel, cdiv(Ml, 8), 256, 0, h->stream, 
                        h->part, h->n_vt, h->counts + 1, h->rr_b, h->rr_i, h->lam_rr, N, K, s, h->a, h->cur_H,
                        h->cur_y, out->entropy, out->halt, out->cum_halt)));
         }
         LAUNCH(KC_COMMIT, 16.0 * Ml, 0.0,
-               (k::commit_kernel<<<n_act_, 256, 0, h->stream>>>(mp, s, K, rule, tau_H, lambda, h->embed, H, xl,
+               (klaunch(k::commit_kernel, n_act_, 256, 0, h->stream, mp, s, K, rule, tau_H, lambda, h->embed, H, xl,
                                                                st)));
         LAUNCH(KC_COMMIT, 8.0 * Ml, 0.0,
-               (k::plan_kernel<<<1, 1024, 0, h->stream>>>(n_act_, h->seq_of[cur_], N, h->cont, h->U,
+               (klaunch(k::plan_kernel, 1, 1024, 0, h->stream, n_act_, h->seq_of[cur_], N, h->cont, h->U,
                                                           h->seq_of[cur_ ^ 1], h->old_slot, h->ridx, h->rr_b,
                                                           h->rr_i, h->counts, s + 1, K, out->active_rows,
                                                           out->readout_rows, h->d_err)));
@@ -1015,7 +1046,7 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
         if (n_next != n_act) {
             x = h->hbuf[hi];
             LAUNCH(KC_COMMIT, 8.0 * n_next * N * H, 0.0,
-                   (k::gather_rows_kernel<<<n_next * N, 256, 0, h->stream>>>(x, h->hbuf[hi ^ 1], h->old_slot, N, H)));
+                   (klaunch(k::gather_rows_kernel, n_next * N, 256, 0, h->stream, x, h->hbuf[hi ^ 1], h->old_slot, N, H)));
             hi ^= 1;
         }
         cur ^= 1;
@@ -1034,7 +1065,7 @@ int alodlm_set_graphs(alodlm_t *h, int on) {
 int alodlm_debug_state(alodlm_t *h, int which, int loop, float *dst) {
     if (!h || !dst) return ALODLM_EINVAL;
     if (!h->cfg.debug_dump) return fail(h, ALODLM_EINVAL, "debug_dump is off");
-    if (which < 0 || which > 2 || loop < 1 || loop > h->cfg.k_max || h->last_N < 1)
+    if (which < 0 || which > 3 || loop < 1 || loop > h->cfg.k_max || h->last_N < 1)
         return fail(h, ALODLM_EINVAL, "debug_state: out of range or no step yet");
     const float *src = h->dbg[which] + (size_t)(loop - 1) * h->cfg.max_batch * h->cfg.max_block * h->H;
     cudaError_t e = cudaMemcpyAsync(dst, src, (size_t)h->B * h->last_N * h->H * sizeof(float),
@@ -1105,7 +1136,7 @@ int alodlm_gemm_bf16(const void *A, const void *W, float *C, int M, int N, int K
     CUtensorMap tW, tA;
     if (!make_tmap(&tW, W, K, N, gemm::BM)) return ALODLM_ECUDA;
     auto map_for_bn = [&](int bn) -> const CUtensorMap * { return make_tmap(&tA, A, K, M, bn) ? &tA : nullptr; };
-    if (run_gemm(env, tW, N, map_for_bn, M, K, gemm::EPI_F32, C, N, nullptr, 0) < 0) return ALODLM_ECUDA;
+    if (run_gemm(env, tW, N, map_for_bn, M, K, gemm::EPI_F32, C, N, nullptr, 0, true) < 0) return ALODLM_ECUDA;
     return cudaGetLastError() == cudaSuccess ? ALODLM_OK : ALODLM_ECUDA;
 }
 

@@ -36,6 +36,14 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
+// Programmatic dependent launch: kernels of a step are launched so that a kernel's CTAs may
+// start while its predecessor finishes.  pdl_wait() blocks until the predecessor grid has
+// completed and its writes are visible (a no-op without the launch attribute); every kernel
+// calls it before touching memory that a predecessor writes or reads.  pdl_trigger() lets
+// the successor's CTAs be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------------

@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(192, 1)
     const int a_tile = a_fastest ? blockIdx.x : blockIdx.y;
     const int b_tile = a_fastest ? blockIdx.y : blockIdx.x;
     if (rowsA_dyn) {  // row count known only on the device (grid sized for the maximum)
+        pdl_wait();
         const int live = *rowsA_dyn;
         if (a_tile * BM >= live) return;
         rowsA = min(rowsA, live);
@@ -89,11 +90,24 @@ __global__ void __launch_bounds__(192, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_trigger();
 
     if (warp == 0) {
         if (lane == 0) {
-            int issued = 0;
-            for (int it = 0; it < nkt; ++it) {
+            // The A operand of the linear layers is a weight, which no kernel writes: its first
+            // stages are requested before waiting for the predecessor kernel, so the pipeline
+            // fills while the predecessor drains.  The readout's A operand is produced by the
+            // predecessor (rowsA_dyn set): then everything waits.
+            const int pre = rowsA_dyn ? 0 : min(nkt, STAGES);
+            for (int it = 0; it < pre; ++it) {
+                mbar_arrive_expect_tx(full + it, C::STAGE_BYTES);
+                tma_load_2d(smem + it * C::STAGE_BYTES, &tmA, full + it, (kt0 + it) * BK, a_tile * BM);
+            }
+            pdl_wait();
+            for (int it = 0; it < pre; ++it)
+                tma_load_2d(smem + it * C::STAGE_BYTES + C::A_BYTES, &tmB, full + it, (kt0 + it) * BK, b_tile * BN);
+            int issued = pre;
+            for (int it = pre; it < nkt; ++it) {
                 const int s = it % STAGES;
                 const uint32_t use = (uint32_t)(it / STAGES);
                 if (!mbar_wait(empty + s, (use & 1u) ^ 1u, err)) break;
@@ -128,6 +142,7 @@ __global__ void __launch_bounds__(192, 1)
     } else {
         // ---------------- epilogue (warps 2..5) ----------------
         const int q = warp & 3;  // TMEM lane quarter this warp may access
+        pdl_wait();
         const bool ready = mbar_wait(accum, 0, err);
         tc_fence_after();
         const int a_row = a_tile * BM + q * 32 + lane;
@@ -220,6 +235,8 @@ __global__ void __launch_bounds__(192, 1)
 template <int EPI>
 __global__ void splitk_reduce_kernel(const float *__restrict__ ws, int splits, long long split_stride, int rowsA,
                                      int rowsB, EpiParams ep) {
+    pdl_wait();
+    pdl_trigger();
     if constexpr (EPI == EPI_SWIGLU) {
         const int n_feat = rowsA / 2;
         const long long total = (long long)rowsB * n_feat;
@@ -350,6 +367,8 @@ __global__ void __launch_bounds__(192, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         if (lane == 0) {

@@ -62,6 +62,8 @@ __global__ void rope_table_kernel(float2 *rope, int n_pos, int half, double base
 // h[m, :] = Emb[ids[b, t], :] (bf16 -> f32)
 __global__ void embed_kernel(const int *ids, int ids_ld, RowMap map, const bf16 *emb, int vocab, int H, float *h,
                              int *err) {
+    pdl_wait();
+    pdl_trigger();
     const int m = blockIdx.x;
     const int jj = m / map.rows_per_seq, t = m % map.rows_per_seq;
     const int b = map.seq_of[jj];
@@ -80,6 +82,8 @@ __global__ void embed_kernel(const int *ids, int ids_ld, RowMap map, const bf16 
 
 // y[m, :] = bf16(x[m, :] / sqrt(mean(x^2) + eps) * g)
 __global__ void rmsnorm_kernel(const float *x, const float *g, bf16 *y, int H, float eps) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float red[32];
     const long long m = blockIdx.x;
     const float4 *xr = reinterpret_cast<const float4 *>(x + m * H);
@@ -104,6 +108,8 @@ __global__ void rmsnorm_kernel(const float *x, const float *g, bf16 *y, int H, f
 __global__ void qkv_post_kernel(const float *qkv, int nq, int nkv, int hd, const float *qn, const float *kn,
                                 int qk_norm, float eps, const float2 *rope, RowMap map, bf16 *q_out, bf16 *kc,
                                 bf16 *vc, long long seq_stride, long long head_stride) {
+    pdl_wait();
+    pdl_trigger();
     const int m = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const int jj = m / map.rows_per_seq, t = m % map.rows_per_seq;
@@ -162,6 +168,8 @@ __global__ void qkv_post_kernel(const float *qkv, int nq, int nkv, int hd, const
 __global__ void kv_fallback_kernel(const int *exit_depth, int P, int b0, int depth, const bf16 *src_k,
                                    const bf16 *src_v, bf16 *dst_k, bf16 *dst_v, long long seq_stride,
                                    long long head_stride, int hd) {
+    pdl_wait();
+    pdl_trigger();
     const int b = b0 + blockIdx.x, kvh = blockIdx.y;
     const long long base = (long long)b * seq_stride + (long long)kvh * head_stride;
     const int chunks = hd / 8;
@@ -177,6 +185,8 @@ __global__ void kv_fallback_kernel(const int *exit_depth, int P, int b0, int dep
 // h_exit[m] = h[m] for prefix rows whose exit depth equals `depth`
 __global__ void capture_exit_kernel(const int *exit_depth, int P, int b0, int depth, const float *h, float *h_exit,
                                     int H) {
+    pdl_wait();
+    pdl_trigger();
     const int m = blockIdx.x;
     const int b = b0 + m / P, pos = m % P;
     if (exit_depth[(long long)b * P + pos] != depth) return;
@@ -194,6 +204,8 @@ __global__ void capture_exit_kernel(const int *exit_depth, int P, int b0, int de
 // r is also stored at [b, i].
 __global__ void final_norm_kernel(const float *hc, const float *g, const float *exit_w, float exit_b, int H, float eps,
                                   RowMap map, const int *ridx, bf16 *rb, float *lam_rr, float *dbg_r) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float red[32];
     const int m = blockIdx.x;
     const int rr = ridx[m];
@@ -239,6 +251,8 @@ __device__ __forceinline__ Stat merge_stat(Stat a, Stat b) {
 __global__ void readout_combine_kernel(const float4 *part, int n_vt, const int *R_dev, const int *rr_b,
                                        const int *rr_i, const float *lam_rr, int N, int Kstep, int s, float *a_state,
                                        float *cur_H, int *cur_y, float *tr_H, float *tr_lam, float *tr_a) {
+    pdl_wait();
+    pdl_trigger();
     const int rr = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (rr >= *R_dev) return;
@@ -301,6 +315,8 @@ struct StepState {
 };
 
 __global__ void step_init_kernel(const int *block_ids, int B, int N, int Kstep, int mask_id, StepState st) {
+    pdl_wait();
+    pdl_trigger();
     const long long total = (long long)B * N;
     const float qnan = __int_as_float(0x7fc00000);
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
@@ -334,6 +350,8 @@ __global__ void step_init_kernel(const int *block_ids, int B, int N, int Kstep, 
 // commit, and the Eq. 3 merge of committed rows into the loop state h.
 __global__ void commit_kernel(RowMap map, int s, int Kstep, int rule, float tau, float lam, const bf16 *emb, int H,
                               float *h, StepState st) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float red[32];
     __shared__ int red_i[32];
     const int jj = blockIdx.x;
@@ -437,6 +455,8 @@ __global__ void commit_kernel(RowMap map, int s, int Kstep, int rule, float tau,
 __global__ void plan_kernel(int n_cur, const int *seq_cur, int N, const int *cont, const unsigned char *U,
                             int *seq_next, int *old_slot, int *ridx, int *rr_b, int *rr_i, int *counts, int s_next,
                             int Kstep, int *active_rows, int *readout_rows, const int *err) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int n_next;
     __shared__ int scan[1024];
     __shared__ int carry;
@@ -496,6 +516,8 @@ __global__ void plan_kernel(int n_cur, const int *seq_cur, int N, const int *con
 
 // dst rows of the next loop's compact layout from the current layout
 __global__ void gather_rows_kernel(const float *src, float *dst, const int *old_slot, int N, int H) {
+    pdl_wait();
+    pdl_trigger();
     const int m = blockIdx.x;
     const int jn = m / N, i = m % N;
     const float4 *s = reinterpret_cast<const float4 *>(src + ((long long)old_slot[jn] * N + i) * H);
@@ -505,6 +527,8 @@ __global__ void gather_rows_kernel(const float *src, float *dst, const int *old_
 
 // debug copy of compact rows to [b, i] order
 __global__ void dump_rows_kernel(const float *src, RowMap map, int H, float *dst) {
+    pdl_wait();
+    pdl_trigger();
     const int m = blockIdx.x;
     const int N = map.rows_per_seq;
     const int b = map.seq_of[m / N], i = m % N;

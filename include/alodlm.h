@@ -155,7 +155,7 @@ ALODLM_API const char *alodlm_last_error(const alodlm_t *h);
 /* Debug copies (cfg.debug_dump = 1): copy the last step's float32 [B, N, hidden] state of loop
  * `loop` (1-based) into the caller's device buffer dst (enqueued on the handle's stream):
  * which = 0 loop input h^(s-1), 1 Core output h~^(s), 2 readout state r^(s) (after the final
- * RMSNorm).  Rows of sequences that had stopped before `loop` hold stale data.
+ * RMSNorm), 3 output of the first Core layer at loop s.  Rows of sequences that had stopped before `loop` hold stale data.
  * EINVAL without debug_dump, before a step, or out of range. */
 ALODLM_API int alodlm_debug_state(alodlm_t *h, int which, int loop, float *dst);
 
