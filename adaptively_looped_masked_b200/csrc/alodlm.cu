@@ -143,7 +143,15 @@ bool init_kernel_attrs() {
     return done[dev];
 }
 
-int pick_bn(int M) { return M <= 32 ? 32 : (M <= 64 ? 64 : (M <= 128 ? 128 : 256)); }
+// Activation rows per tile: the smallest of 32/64/128 that covers them up to 128 rows; above,
+// 256-row tiles only once they still give at least one tile per SM (fewer, fatter tiles
+// leave SMs idle on mid-sized row counts).
+int pick_bn(int M, int Nw) {
+    if (M <= 32) return 32;
+    if (M <= 64) return 64;
+    if (M <= 128) return 128;
+    return (cdiv(Nw, 128) * cdiv(M, 256) >= NUM_SMS_HINT) ? 256 : 128;
+}
 
 struct GemmShape {
     int bn, splits, kps, k_tiles;
@@ -153,7 +161,7 @@ struct GemmShape {
 // four k-tiles per split, partials within the workspace.
 GemmShape plan_gemm(int M, int Nw, int K, size_t ws_floats) {
     GemmShape g;
-    g.bn = pick_bn(M);
+    g.bn = pick_bn(M, Nw);
     g.k_tiles = cdiv(K, gemm::BK);
     const int tiles = cdiv(Nw, gemm::BM) * cdiv(M, g.bn);
     const int per_sm = g.bn <= 64 ? 2 : 1;
@@ -185,18 +193,6 @@ void launch_gemm_epi(int bn, const CUtensorMap &tA, const CUtensorMap &tB, int r
         case 128: launch_gemm_bn<128, EPI>(tA, tB, rowsA, rowsB, k_tiles, kps, splits, a_fastest, ep, err, st); break;
         default: launch_gemm_bn<256, EPI>(tA, tB, rowsA, rowsB, k_tiles, kps, splits, a_fastest, ep, err, st); break;
     }
-}
-
-void launch_splitk_reduce(int epi, const float *ws, int splits, long long sstride, int rowsA, int rowsB,
-                          const gemm::EpiParams &ep, cudaStream_t st) {
-    const long long total = (long long)rowsA * rowsB;
-    const int blocks = (int)std::min<long long>((total + 255) / 256, 148 * 8);
-    if (epi == gemm::EPI_ADD)
-        klaunch(gemm::splitk_reduce_kernel<gemm::EPI_ADD>, blocks, 256, 0, st, ws, splits, sstride, rowsA, rowsB, ep);
-    else if (epi == gemm::EPI_SWIGLU)
-        klaunch(gemm::splitk_reduce_kernel<gemm::EPI_SWIGLU>, blocks, 256, 0, st, ws, splits, sstride, rowsA, rowsB, ep);
-    else
-        klaunch(gemm::splitk_reduce_kernel<gemm::EPI_F32>, blocks, 256, 0, st, ws, splits, sstride, rowsA, rowsB, ep);
 }
 
 // Where a GEMM may put its scratch: split-K / stream-K partials, stream-K tile counters
@@ -249,9 +245,9 @@ void launch_sk(const SkPlan &p, const CUtensorMap &tW, const CUtensorMap &tB, in
         launch_sk_bn<64, EPI>(p, tW, tB, Nw, M, ep, env);
 }
 
-// out = act[M, K] x W[Nw, K]^T with epilogue `epi`.  Few rows (<= 64): stream-K kernel with the
-// split reduction fused; more rows: one CTA per 128 x BN tile, split-K with a fixed-order
-// reduce only when the tiles do not fill the SMs.  map_for_bn(bn) returns the activation's
+// out = act[M, K] x W[Nw, K]^T with epilogue `epi`.  Stream-K kernel (few rows, when asked) or
+// one CTA per 128 x BN tile with split-K when the tiles do not fill the SMs; split partials are
+// added in split order by the CTA that completes a tile last.  map_for_bn(bn) returns the activation's
 // tensor map with BN-row boxes.  Returns the number of kernels launched, or -1 (tensor map
 // failure).
 template <typename MapFn>
@@ -277,25 +273,22 @@ int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_b
         }
     }
     GemmShape g = plan_gemm(M, Nw, K, env.ws_floats);
+    if (g.splits > 1 && cdiv(Nw, gemm::BM) * cdiv(M, g.bn) > env.n_counters) {
+        g.splits = 1;
+        g.kps = g.k_tiles;
+    }
     const CUtensorMap *tB = map_for_bn(g.bn);
     if (!tB) return -1;
-    if (g.splits == 1) {
-        if (epi == gemm::EPI_F32)
-            launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, 1, 0, ep, env.err, env.st);
-        else if (epi == gemm::EPI_ADD)
-            launch_gemm_epi<gemm::EPI_ADD>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, 1, 0, ep, env.err, env.st);
-        else
-            launch_gemm_epi<gemm::EPI_SWIGLU>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, 1, 0, ep, env.err, env.st);
-        return 1;
-    } else {
-        gemm::EpiParams ep1{};
-        ep1.out = env.ws;
-        ep1.ldo = Nw;
-        ep1.split_stride = (long long)M * Nw;
-        launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep1, env.err, env.st);
-        launch_splitk_reduce(epi, env.ws, g.splits, (long long)M * Nw, Nw, M, ep, env.st);
-        return 2;
-    }
+    ep.ws = env.ws;
+    ep.counters = env.counters;
+    ep.split_stride = (long long)M * Nw;
+    if (epi == gemm::EPI_F32)
+        launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, env.err, env.st);
+    else if (epi == gemm::EPI_ADD)
+        launch_gemm_epi<gemm::EPI_ADD>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, env.err, env.st);
+    else
+        launch_gemm_epi<gemm::EPI_SWIGLU>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, env.err, env.st);
+    return 1;
 }
 
 struct LayerDev {
@@ -534,8 +527,8 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
     const int ktiles = cdiv(kv_len, 64);
     int splits = 1;
     if (!causal) {
-        // enough CTAs to cover the SMs, but at least 4 key tiles per split
-        splits = std::max(1, std::min(ktiles / 4, cdiv(h->num_sms, base)));
+        // enough CTAs to cover the SMs, but at least 2 key tiles per split
+        splits = std::max(1, std::min(ktiles / 2, cdiv(h->num_sms, base)));
         while (splits > 1 && ((size_t)splits * M * h->nq * (h->hd + 2) > ATTN_WS_FLOATS ||
                               (size_t)base > ATTN_COUNTERS))
             --splits;

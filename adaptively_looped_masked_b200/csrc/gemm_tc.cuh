@@ -26,9 +26,11 @@ constexpr int BK = 64;
 enum Epi { EPI_F32 = 0, EPI_ADD = 1, EPI_SWIGLU = 2, EPI_READOUT = 3 };
 
 struct EpiParams {
-    float *out;           // EPI_F32 / EPI_ADD: out[b_row * ldo + a_row] (+ split * split_stride)
+    float *out;           // EPI_F32 / EPI_ADD: out[b_row * ldo + a_row]
     int ldo;
     long long split_stride;
+    float *ws;            // split-K (gridDim.z > 1): partials ws[split * split_stride + b_row * rowsA + a_row]
+    int *counters;        // split-K: per output tile, splits done (left at zero)
     bf16 *act;            // EPI_SWIGLU: act[b_row * ld_act + feature]
     int ld_act;
     float4 *partials;     // EPI_READOUT: partials[a_row * n_btiles + b_tile] = (max, sum e, sum e*d, argmax)
@@ -149,18 +151,26 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
         const int b0 = b_tile * BN;
         if (ready) {
-            if constexpr (EPI == EPI_F32 || EPI == EPI_ADD) {
-                float *out = ep.out + (long long)split * ep.split_stride;
-                for (int c0 = 0; c0 < BN; c0 += 16) {
-                    if (b0 + c0 >= rowsB) break;  // warp-uniform
-                    float v[16];
-                    tmem_ld16(taddr + c0, v);
-                    if (a_row < rowsA) {
+            if constexpr (EPI == EPI_F32 || EPI == EPI_ADD || EPI == EPI_SWIGLU) {
+                // final epilogue of one 16-column chunk (warp-uniform: SwiGLU shuffles lanes)
+                auto apply = [&](int c0, const float (&v)[16]) {
+                    if constexpr (EPI == EPI_SWIGLU) {
+                        // weight rows interleaved in groups of 32: 16 gate rows then the 16 up rows
+                        // of the same features, so lane l < 16 holds gate and lane l + 16 holds up
+                        const int feat = (a_row >> 5) * 16 + (lane & 15);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float up = __shfl_xor_sync(0xffffffffu, v[j], 16);
+                            const int br = b0 + c0 + j;
+                            if (lane < 16 && a_row < rowsA && br < rowsB)
+                                ep.act[(long long)br * ep.ld_act + feat] = __float2bfloat16_rn(silu_f(v[j]) * up);
+                        }
+                    } else if (a_row < rowsA) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int br = b0 + c0 + j;
                             if (br < rowsB) {
-                                float *p = out + (long long)br * ep.ldo + a_row;
+                                float *p = ep.out + (long long)br * ep.ldo + a_row;
                                 if constexpr (EPI == EPI_ADD)
                                     *p += v[j];
                                 else
@@ -168,21 +178,57 @@ __global__ void __launch_bounds__(192, 1)
                             }
                         }
                     }
-                }
-            } else if constexpr (EPI == EPI_SWIGLU) {
-                // weight rows interleaved in groups of 32: 16 gate rows then the 16 up rows of
-                // the same features, so lane l < 16 holds gate and lane l + 16 holds up
-                const int feat = (a_row >> 5) * 16 + (lane & 15);
-                for (int c0 = 0; c0 < BN; c0 += 16) {
-                    if (b0 + c0 >= rowsB) break;
-                    float v[16];
-                    tmem_ld16(taddr + c0, v);
+                };
+                if (gridDim.z == 1) {
+                    for (int c0 = 0; c0 < BN; c0 += 16) {
+                        if (b0 + c0 >= rowsB) break;  // warp-uniform
+                        float v[16];
+                        tmem_ld16(taddr + c0, v);
+                        apply(c0, v);
+                    }
+                } else {
+                    // split-K: store this split's partial tile; the CTA that completes the tile last
+                    // adds the partials in split order (deterministic) and applies the epilogue
+                    float *mine = ep.ws + (long long)split * ep.split_stride;
+                    for (int c0 = 0; c0 < BN; c0 += 16) {
+                        if (b0 + c0 >= rowsB) break;
+                        float v[16];
+                        tmem_ld16(taddr + c0, v);
+                        if (a_row < rowsA) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float up = __shfl_xor_sync(0xffffffffu, v[j], 16);
-                        const int br = b0 + c0 + j;
-                        if (lane < 16 && a_row < rowsA && br < rowsB)
-                            ep.act[(long long)br * ep.ld_act + feat] = __float2bfloat16_rn(silu_f(v[j]) * up);
+                            for (int j = 0; j < 16; ++j)
+                                if (b0 + c0 + j < rowsB) mine[(long long)(b0 + c0 + j) * rowsA + a_row] = v[j];
+                        }
+                    }
+                    __threadfence();
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    __shared__ int last_split;
+                    if (threadIdx.x == 64) {
+                        const int n_btiles = a_fastest ? gridDim.y : gridDim.x;
+                        int *cnt = ep.counters + a_tile * n_btiles + b_tile;
+                        const int prev = atomicAdd(cnt, 1);
+                        last_split = prev == (int)gridDim.z - 1;
+                        if (last_split) *cnt = 0;
+                    }
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    if (last_split) {
+                        __threadfence();
+                        for (int c0 = 0; c0 < BN; c0 += 16) {
+                            if (b0 + c0 >= rowsB) break;
+                            float v[16];
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) v[j] = 0.f;
+                            if (a_row < rowsA) {
+                                for (int sp = 0; sp < (int)gridDim.z; ++sp) {
+                                    const float *src = ep.ws + (long long)sp * ep.split_stride;
+#pragma unroll
+                                    for (int j = 0; j < 16; ++j)
+                                        if (b0 + c0 + j < rowsB)
+                                            v[j] += __ldcg(src + (long long)(b0 + c0 + j) * rowsA + a_row);
+                                }
+                            }
+                            apply(c0, v);
+                        }
                     }
                 }
             } else {  // EPI_READOUT: this thread's row of logits over BN vocabulary entries
@@ -228,43 +274,6 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
-    }
-}
-
-// Fixed-order sum of split-K partials ws[split][b_row][a_row] followed by the epilogue.
-template <int EPI>
-__global__ void splitk_reduce_kernel(const float *__restrict__ ws, int splits, long long split_stride, int rowsA,
-                                     int rowsB, EpiParams ep) {
-    pdl_wait();
-    pdl_trigger();
-    if constexpr (EPI == EPI_SWIGLU) {
-        const int n_feat = rowsA / 2;
-        const long long total = (long long)rowsB * n_feat;
-        for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
-             idx += (long long)gridDim.x * blockDim.x) {
-            const int br = (int)(idx / n_feat), f = (int)(idx % n_feat);
-            const int rg = (f >> 4) * 32 + (f & 15), ru = rg + 16;
-            float g = 0.f, u = 0.f;
-            for (int s = 0; s < splits; ++s) {
-                const float *p = ws + s * split_stride + (long long)br * rowsA;
-                g += p[rg];
-                u += p[ru];
-            }
-            ep.act[(long long)br * ep.ld_act + f] = __float2bfloat16_rn(silu_f(g) * u);
-        }
-    } else {
-        const long long total = (long long)rowsB * rowsA;
-        for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
-             idx += (long long)gridDim.x * blockDim.x) {
-            const int br = (int)(idx / rowsA), ar = (int)(idx % rowsA);
-            float acc = 0.f;
-            for (int s = 0; s < splits; ++s) acc += ws[s * split_stride + idx];
-            float *p = ep.out + (long long)br * ep.ldo + ar;
-            if constexpr (EPI == EPI_ADD)
-                *p += acc;
-            else
-                *p = acc;
-        }
     }
 }
 
