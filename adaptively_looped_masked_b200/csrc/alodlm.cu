@@ -16,6 +16,7 @@
 #include <vector>
 
 #include "attention.cuh"
+#include "attention_tc.cuh"
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
@@ -54,6 +55,27 @@ void klaunch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStr
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = (ALODLM_PDL && st != nullptr && st != cudaStreamLegacy && st != cudaStreamPerThread) ? 1 : 0;
+    cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// The same with a thread-block cluster of (1, 1, cluster_z) CTAs.
+template <typename... KArgs, typename... Args>
+void klaunch_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_z,
+                     Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = cluster_z;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (ALODLM_PDL && st != nullptr && st != cudaStreamLegacy && st != cudaStreamPerThread) ? 2 : 1;
     cudaLaunchKernelEx(&cfg, kern, args...);
 }
 constexpr int PREFILL_ROWS = 16384;         // rows of one prefill group (sequences x P)
@@ -138,6 +160,7 @@ bool init_kernel_attrs() {
     set_sk_attr<64, gemm::EPI_ADD>();
     set_sk_attr<64, gemm::EPI_SWIGLU>();
     cudaFuncSetAttribute(attn::attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 5 * 64 * 64 * 2);
+    cudaFuncSetAttribute(attn_tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_tc::SMEM);
     cudaFuncSetAttribute(attn::attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 5 * 64 * 128 * 2);
     done[dev] = cudaGetLastError() == cudaSuccess;
     return done[dev];
@@ -158,16 +181,16 @@ struct GemmShape {
 };
 
 // Tile/split choice: enough CTAs to cover the SMs (memory-bound small-M launches), at least
-// four k-tiles per split, partials within the workspace.
-GemmShape plan_gemm(int M, int Nw, int K, size_t ws_floats) {
+// four k-tiles per split, at most 8 splits (one cluster).
+GemmShape plan_gemm(int M, int Nw, int K) {
     GemmShape g;
     g.bn = pick_bn(M, Nw);
     g.k_tiles = cdiv(K, gemm::BK);
     const int tiles = cdiv(Nw, gemm::BM) * cdiv(M, g.bn);
     const int per_sm = g.bn <= 64 ? 2 : 1;
     int splits = (NUM_SMS_HINT * per_sm) / tiles;
-    splits = std::max(1, std::min(splits, g.k_tiles / 4));
-    while (splits > 1 && (size_t)splits * M * Nw > ws_floats) --splits;
+    // splits form one cluster (portable size <= 8); at least 4 k-tiles each
+    splits = std::max(1, std::min(std::min(splits, 8), g.k_tiles / 4));
     g.kps = cdiv(g.k_tiles, splits);
     g.splits = cdiv(g.k_tiles, g.kps);
     return g;
@@ -180,6 +203,10 @@ void launch_gemm_bn(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int
     dim3 grid;
     const int ta = cdiv(rowsA, gemm::BM), tb = cdiv(rowsB, BN);
     grid = a_fastest ? dim3(ta, tb, splits) : dim3(tb, ta, splits);
+    if (splits > 1)
+        klaunch_cluster(gemm::gemm_tc_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM, st, splits, tA, tB, rowsA,
+                        rowsB, rowsA_dyn, k_tiles, kps, a_fastest, ep, err);
+    else
     klaunch(gemm::gemm_tc_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM, st, tA, tB, rowsA, rowsB, rowsA_dyn, k_tiles,
                                                                            kps, a_fastest, ep, err);
 }
@@ -272,16 +299,9 @@ int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_b
             return 1;
         }
     }
-    GemmShape g = plan_gemm(M, Nw, K, env.ws_floats);
-    if (g.splits > 1 && cdiv(Nw, gemm::BM) * cdiv(M, g.bn) > env.n_counters) {
-        g.splits = 1;
-        g.kps = g.k_tiles;
-    }
+    GemmShape g = plan_gemm(M, Nw, K);
     const CUtensorMap *tB = map_for_bn(g.bn);
     if (!tB) return -1;
-    ep.ws = env.ws;
-    ep.counters = env.counters;
-    ep.split_stride = (long long)M * Nw;
     if (epi == gemm::EPI_F32)
         launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, env.err, env.st);
     else if (epi == gemm::EPI_ADD)
@@ -345,6 +365,8 @@ struct alodlm {
     int n_slots = 0, pos_stride = 0;
     long long head_stride = 0, seq_stride = 0, slot_elems = 0;
     float2 *rope = nullptr;
+    bool tc_attn = false;            // tcgen05 attention for the step (head_dim 128)
+    CUtensorMap tm_q, tm_kv_k, tm_kv_v;
 
     // prefill state
     int B = 0, P = 0, last_N = 0;
@@ -502,6 +524,64 @@ int linear(alodlm *h, const CUtensorMap &tmW, int Nw, const bf16 *actp, int M, i
 
 // attention of M rows (n_seq sequences x rows_per_seq) against slot `slot`, keys [0, kv_len)
 int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_len, int causal) {
+    if (!causal && h->tc_attn) {
+        attn_tc::Params p{};
+        p.G = h->nq / h->nkv;
+        p.RP = p.G * map.rows_per_seq;
+        p.nkv = h->nkv;
+        p.nq = h->nq;
+        p.Tq = map.rows_per_seq;
+        p.kv_len = kv_len;
+        p.slot = slot;
+        p.max_batch = h->cfg.max_batch;
+        p.pos_stride = h->pos_stride;
+        p.seq_of = map.seq_of;
+        p.out = h->attn_out;
+        p.out_ld = h->nq * h->hd;
+        p.m_rows = M;
+        p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)h->hd));
+        p.err = h->d_err;
+        const int qtiles = cdiv(p.RP, attn_tc::BQ);
+        const int base = qtiles * h->nkv * n_seq;
+        const int ktiles = cdiv(kv_len, attn_tc::BKV);
+        // splits of a query tile form one cluster (<= 8 CTAs, a power of two so that they
+        // share the 128 rows evenly), at least 2 key tiles each
+        int splits = std::max(1, std::min(std::min(ktiles / 2, cdiv(h->num_sms, base)), 8));
+        while (splits & (splits - 1)) --splits;
+        int kps = cdiv(ktiles, splits);
+        while (splits > 1 && cdiv(ktiles, kps) < splits) {  // every rank gets keys
+            splits >>= 1;
+            kps = cdiv(ktiles, splits);
+        }
+        p.n_splits = splits;
+        p.keys_per_split = kps * attn_tc::BKV;
+        const double bytes = 4.0 * n_seq * h->nkv * (double)kv_len * h->hd + 4.0 * M * h->nq * h->hd;
+        const double flops = 4.0 * M * h->nq * (double)kv_len * h->hd;
+        if (splits > 1) {
+            // cluster along y: the `splits` consecutive y indices of one kv head
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(qtiles, h->nkv * splits, n_seq);
+            cfg.blockDim = dim3(192);
+            cfg.dynamicSmemBytes = attn_tc::SMEM;
+            cfg.stream = h->stream;
+            cudaLaunchAttribute attr[2];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 1;
+            attr[0].val.clusterDim.y = splits;
+            attr[0].val.clusterDim.z = 1;
+            attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[1].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = ALODLM_PDL ? 2 : 1;
+            LAUNCH(KC_ATTN, bytes, flops,
+                   cudaLaunchKernelEx(&cfg, attn_tc::attn_tc_kernel, h->tm_q, h->tm_kv_k, h->tm_kv_v, p));
+        } else {
+            LAUNCH(KC_ATTN, bytes, flops,
+                   klaunch(attn_tc::attn_tc_kernel, dim3(qtiles, h->nkv, n_seq), 192, attn_tc::SMEM, h->stream,
+                           h->tm_q, h->tm_kv_k, h->tm_kv_v, p));
+        }
+        return ALODLM_OK;
+    }
     attn::Params p{};
     p.q = h->qb;
     p.q_ld = h->nq * h->hd;
@@ -527,8 +607,8 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
     const int ktiles = cdiv(kv_len, 64);
     int splits = 1;
     if (!causal) {
-        // enough CTAs to cover the SMs, but at least 2 key tiles per split
-        splits = std::max(1, std::min(ktiles / 2, cdiv(h->num_sms, base)));
+        // enough CTAs to cover the SMs, but at least 4 key tiles per split
+        splits = std::max(1, std::min(ktiles / 4, cdiv(h->num_sms, base)));
         while (splits > 1 && ((size_t)splits * M * h->nq * (h->hd + 2) > ATTN_WS_FLOATS ||
                               (size_t)base > ATTN_COUNTERS))
             --splits;
@@ -777,6 +857,18 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
     cudaMemsetAsync(h->xn, 0, R * H * 2, h->stream);
     cudaMemsetAsync(h->attn_out, 0, R * qd * 2, h->stream);
     cudaMemsetAsync(h->act, 0, R * h->I * 2, h->stream);
+
+    // never-written arena positions are read (and masked) by 128-key tiles: keep them finite
+    cudaMemsetAsync(h->kv_k, 0, (size_t)h->slot_elems * h->n_slots * 2, h->stream);
+    cudaMemsetAsync(h->kv_v, 0, (size_t)h->slot_elems * h->n_slots * 2, h->stream);
+    {
+        const long long arena_rows = (long long)h->n_slots * cfg->max_batch * h->nkv * h->pos_stride;
+        h->tc_attn = h->hd == 128 && arena_rows + 256 < (1ll << 31) && (long long)R * h->nq < (1ll << 31);
+        if (h->tc_attn)
+            h->tc_attn = make_tmap(&h->tm_q, h->qb, h->hd, (int)(R * h->nq), attn_tc::BQ) &&
+                         make_tmap(&h->tm_kv_k, h->kv_k, h->hd, (int)arena_rows, attn_tc::BKV) &&
+                         make_tmap(&h->tm_kv_v, h->kv_v, h->hd, (int)arena_rows, attn_tc::BKV);
+    }
 
     h->R_cap = round_up(h->step_rows_cap, 128);
     h->n_vt = cdiv(h->V, 256);

@@ -13,7 +13,7 @@
 namespace attn {
 
 struct Params {
-    const bf16 *q;        // q[m * q_ld + h * HD + d]
+    const bf16 *q;        // packed: q[((j * nkv + kvh) * G * rows_per_seq + position * G + g) * HD + d]
     int q_ld;
     const bf16 *kc, *vc;  // this slot's K/V: + b * seq_stride + kvh * head_stride + pos * HD
     long long seq_stride, head_stride;
@@ -98,10 +98,9 @@ __global__ void __launch_bounds__(128) attn_kernel(Params p) {
     for (int c = tid; c < 64 * CPR; c += 128) {
         const int r = c / CPR, ch = c % CPR, rp = r0 + r;
         uint4 val = make_uint4(0, 0, 0, 0);
-        if (rp < rows_packed) {
-            const int t = rp / p.G, h = kvh * p.G + rp % p.G;
-            val = *reinterpret_cast<const uint4 *>(p.q + (long long)(j * Tq + t) * p.q_ld + h * HD + ch * 8);
-        }
+        if (rp < rows_packed)
+            val = *reinterpret_cast<const uint4 *>(p.q + (((long long)j * (p.nq / p.G) + kvh) * rows_packed + rp) * HD +
+                                                   ch * 8);
         *reinterpret_cast<uint4 *>(sQ + swz<HD>(r, ch)) = val;
     }
 

@@ -1,0 +1,379 @@
+// attention_tc.cuh — block attention of a denoising step on the fifth-generation tensor core.
+//
+// One CTA serves 128 packed query rows of one (sequence, KV head): packed row r is query head
+// kvh*G + r % G at block position r / G (q is stored in that packed order), so the G query
+// heads of a KV head share every K/V tile.  head_dim 128.  The block attends every prefix key
+// and every block key (no mask inside [0, kv_len)).
+//
+//   warp 0      TMA: Q once; K and V tiles of 128 keys (two 64-wide halves each, 128-byte
+//               swizzle) into a 2-stage ring, straight from the depth-aware KV arena
+//   warp 1      tcgen05.mma: S_i = Q K_i^T into a double-buffered TMEM tile (M=128, N=128),
+//               then O += P_i V_i into the TMEM accumulator (V read MN-major)
+//   warps 2-5   softmax, one thread per query row: tcgen05.ld its S row, exp2 with a running
+//               reference max that only moves when the row max passes it by more than 8
+//               (rescaling O in TMEM then), P_i as bf16 into shared memory in the MMA's
+//               128-byte-swizzled K-major layout; at the end O / l to global memory
+//
+// With n_splits > 1 the keys are split across the CTAs of a cluster; each parks (O, reference
+// max, l) in its shared memory and the cluster merges them in rank order through distributed
+// shared memory.
+#pragma once
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace attn_tc {
+
+namespace cg = cooperative_groups;
+
+constexpr int HD = 128;
+constexpr int BQ = 128;        // query rows per CTA
+constexpr int BKV = 128;       // keys per tile
+constexpr int KV_STAGES = 2;
+constexpr uint32_t HALF = BQ * 64 * 2;  // one [128 rows][64] bf16 region = 16 KB
+constexpr uint32_t Q_BYTES = 2 * HALF;
+constexpr uint32_t KV_BYTES = 2 * HALF;  // one K (or V) tile
+constexpr uint32_t P_BYTES = 2 * HALF;
+constexpr uint32_t TMEM_COLS = 512;      // S0 [0,128) S1 [128,256) O [256,384)
+constexpr uint32_t O_COL = 256;
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+constexpr size_t SMEM = 1024 + Q_BYTES + 2 * KV_STAGES * KV_BYTES + P_BYTES + 256;
+
+struct Params {
+    int RP;            // packed query rows per (sequence, kv head) = G * rows_per_seq
+    int G, nkv, nq, Tq;
+    int kv_len;        // keys [0, kv_len) of the slot
+    int slot, max_batch, pos_stride;
+    const int *seq_of;
+    int n_splits, keys_per_split;  // keys_per_split a multiple of BKV
+    bf16 *out;
+    int out_ld;
+    int m_rows;
+    float scale_log2;
+    int *err;
+};
+
+// K-major operand, 128-byte swizzle (8-row atoms of 128 B, 1024 B apart)
+__device__ __forceinline__ uint64_t sdesc_k(uint32_t saddr) { return umma_sdesc_sw128(saddr); }
+
+// MN-major operand, 128-byte swizzle: 64 MN elements per 128-byte row, one row per K index,
+// 8-row atoms 1024 B apart (stride byte offset), the next 64 MN elements `lbo` bytes on
+__device__ __forceinline__ uint64_t sdesc_mn(uint32_t saddr, uint32_t lbo) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+        "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+        "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+        "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+        "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    uint32_t u;
+    memcpy(&u, &v, 4);
+    return u;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(192, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem;
+    uint8_t *sK = sQ + Q_BYTES;                       // [stage] K tiles
+    uint8_t *sV = sK + KV_STAGES * KV_BYTES;          // [stage] V tiles
+    uint8_t *sP = sV + KV_STAGES * KV_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sP + P_BYTES);
+    uint64_t *q_full = bars;
+    uint64_t *k_full = bars + 1;                      // [2]
+    uint64_t *v_full = bars + 3;                      // [2]
+    uint64_t *kv_empty = bars + 5;                    // [2]
+    uint64_t *s_full = bars + 7;                      // [2]
+    uint64_t *p_full = bars + 9;
+    uint64_t *pv_done = bars + 10;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 11);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qtile = blockIdx.x;
+    const int kvh = blockIdx.y / p.n_splits, split = blockIdx.y % p.n_splits;
+    const int j = blockIdx.z;
+    const int kstart = split * p.keys_per_split;
+    const int kend = min(p.kv_len, kstart + p.keys_per_split);
+    const int n_tiles = kend > kstart ? (kend - kstart + BKV - 1) / BKV : 0;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(k_full + s, 1);
+            mbar_init(v_full + s, 1);
+            mbar_init(kv_empty + s, 1);
+            mbar_init(s_full + s, 1);
+        }
+        mbar_init(p_full, 128);
+        mbar_init(pv_done, 1);
+        fence_mbarrier_init();
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_wait();
+    pdl_trigger();
+    const int b = p.seq_of[j];
+
+    if (warp == 0) {
+        if (lane == 0 && n_tiles > 0) {
+            const int qrow = (j * p.nkv + kvh) * p.RP + qtile * BQ;
+            mbar_arrive_expect_tx(q_full, Q_BYTES);
+            tma_load_2d(sQ, &tmQ, q_full, 0, qrow);
+            tma_load_2d(sQ + HALF, &tmQ, q_full, 64, qrow);
+            const int kvrow0 = (int)((((long long)p.slot * p.max_batch + b) * p.nkv + kvh) * p.pos_stride);
+            int issued = 0;
+            for (int i = 0; i < n_tiles; ++i) {
+                const int s = i & 1;
+                if (!mbar_wait(kv_empty + s, ((uint32_t)(i >> 1) & 1u) ^ 1u, p.err)) break;
+                issued = i + 1;
+                const int row = kvrow0 + kstart + i * BKV;
+                mbar_arrive_expect_tx(k_full + s, KV_BYTES);
+                tma_load_2d(sK + s * KV_BYTES, &tmK, k_full + s, 0, row);
+                tma_load_2d(sK + s * KV_BYTES + HALF, &tmK, k_full + s, 64, row);
+                mbar_arrive_expect_tx(v_full + s, KV_BYTES);
+                tma_load_2d(sV + s * KV_BYTES, &tmV, v_full + s, 0, row);
+                tma_load_2d(sV + s * KV_BYTES + HALF, &tmV, v_full + s, 64, row);
+            }
+            // no copy into shared memory may still be in flight when the CTA exits
+            mbar_wait(q_full, 0, p.err);
+            for (int i = max(0, issued - KV_STAGES); i < issued; ++i) {
+                mbar_wait(k_full + (i & 1), ((uint32_t)(i >> 1)) & 1u, p.err);
+                mbar_wait(v_full + (i & 1), ((uint32_t)(i >> 1)) & 1u, p.err);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && n_tiles > 0) {
+            constexpr uint32_t idesc_s = umma_idesc_bf16(BQ, BKV);
+            constexpr uint32_t idesc_o = umma_idesc_bf16(BQ, HD) | (1u << 16);  // B (V) MN-major
+            const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
+            auto issue_s = [&](int i) {
+                const int s = i & 1;
+                const uint32_t k_addr = smem_u32(sK + s * KV_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
+                    umma_f16(tmem + s * BKV, sdesc_k(q_addr + off), sdesc_k(k_addr + off), idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(s_full + s);
+            };
+            bool ok = mbar_wait(q_full, 0, p.err) && mbar_wait(k_full, 0, p.err);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0);
+            }
+            for (int i = 0; i < n_tiles && ok; ++i) {
+                const int s = i & 1;
+                if (i + 1 < n_tiles) {
+                    if (!mbar_wait(k_full + ((i + 1) & 1), ((uint32_t)((i + 1) >> 1)) & 1u, p.err)) break;
+                    tc_fence_after();
+                    issue_s(i + 1);
+                }
+                if (!mbar_wait(p_full, (uint32_t)i & 1u, p.err)) break;
+                if (!mbar_wait(v_full + s, ((uint32_t)(i >> 1)) & 1u, p.err)) break;
+                tc_fence_after();
+                const uint32_t v_addr = smem_u32(sV + s * KV_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < BKV / 16; ++kk) {
+                    const uint32_t a_off = (kk >> 2) * HALF + (kk & 3) * 32;  // P: keys contiguous
+                    const uint32_t b_off = kk * 16 * 128;                      // V: 16 key rows of 128 B
+                    umma_f16(tmem + O_COL, sdesc_k(p_addr + a_off), sdesc_mn(v_addr + b_off, HALF), idesc_o,
+                             (i > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(pv_done);
+                umma_commit(kv_empty + s);
+            }
+        }
+    } else {
+        // ---------------- softmax warps: thread t owns query row t ----------------
+        const int q = warp & 3;
+        const int t = q * 32 + lane;  // TMEM lane = row of the tile
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = n_tiles > 0;
+        for (int i = 0; i < n_tiles && ok; ++i) {
+            const int s = i & 1;
+            if (!mbar_wait(s_full + s, ((uint32_t)(i >> 1)) & 1u, p.err)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float sv[BKV];
+#pragma unroll
+            for (int c0 = 0; c0 < BKV; c0 += 16) {
+                float v[16];
+                tmem_ld16(tmem + lane_base + s * BKV + c0, v);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) sv[c0 + e] = v[e];
+            }
+            const int key0 = kstart + i * BKV;
+            float mt = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < BKV; ++c) {
+                sv[c] = (key0 + c < kend) ? sv[c] * p.scale_log2 : -INFINITY;
+                mt = fmaxf(mt, sv[c]);
+            }
+            // O and the P buffer are free once the previous PV product has completed
+            if (i > 0 && !mbar_wait(pv_done, ((uint32_t)(i - 1)) & 1u, p.err)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (mt > m_ref + RESCALE_THRESHOLD) {
+                if (i > 0) {
+                    const float f = exp2f(m_ref - mt);
+                    l *= f;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < HD; c0 += 16) {
+                        float v[16];
+                        tmem_ld16(tmem + lane_base + O_COL + c0, v);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] *= f;
+                        tmem_st16(tmem + lane_base + O_COL + c0, v);
+                    }
+                }
+                m_ref = mt;
+            }
+            // P row in the K-major 128-byte-swizzled layout: keys 0-63 in the first region,
+            // 64-127 in the second; 16-byte chunk c of row t at (t/8)*1024 + (t%8)*128 + ((c ^ t%8)*16)
+#pragma unroll
+            for (int c = 0; c < BKV / 8; ++c) {
+                float pe[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    pe[e] = exp2f(sv[c * 8 + e] - m_ref);
+                    l += pe[e];
+                }
+                uint4 pk;
+                pk.x = pack2_bf16(pe[0], pe[1]);
+                pk.y = pack2_bf16(pe[2], pe[3]);
+                pk.z = pack2_bf16(pe[4], pe[5]);
+                pk.w = pack2_bf16(pe[6], pe[7]);
+                const int region = c >> 3, ch = c & 7;
+                uint8_t *dst = sP + region * HALF + (t >> 3) * 1024 + (t & 7) * 128 + ((ch ^ (t & 7)) << 4);
+                *reinterpret_cast<uint4 *>(dst) = pk;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(p_full);
+        }
+        // ---------------- output ----------------
+        if (ok && n_tiles > 0 && mbar_wait(pv_done, ((uint32_t)(n_tiles - 1)) & 1u, p.err)) {
+            tc_fence_after();
+            const int rp = qtile * BQ + t;
+            const bool valid = rp < p.RP;
+            const int tt = rp / p.G, h = kvh * p.G + rp % p.G;
+            const int m = j * p.Tq + tt;
+            if (p.n_splits == 1) {
+                const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+                for (int c0 = 0; c0 < HD; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tmem + lane_base + O_COL + c0, v);
+                    if (valid) {
+                        uint4 w0, w1;
+                        w0.x = pack2_bf16(v[0] * inv, v[1] * inv);
+                        w0.y = pack2_bf16(v[2] * inv, v[3] * inv);
+                        w0.z = pack2_bf16(v[4] * inv, v[5] * inv);
+                        w0.w = pack2_bf16(v[6] * inv, v[7] * inv);
+                        w1.x = pack2_bf16(v[8] * inv, v[9] * inv);
+                        w1.y = pack2_bf16(v[10] * inv, v[11] * inv);
+                        w1.z = pack2_bf16(v[12] * inv, v[13] * inv);
+                        w1.w = pack2_bf16(v[14] * inv, v[15] * inv);
+                        bf16 *dst = p.out + (long long)m * p.out_ld + h * HD + c0;
+                        *reinterpret_cast<uint4 *>(dst) = w0;
+                        *reinterpret_cast<uint4 *>(dst + 8) = w1;
+                    }
+                }
+            } else {
+                // split partial: O row (unnormalised) and (reference max, l) into our shared
+                // memory (the K/V ring is idle now) for the cluster merge below
+                float *po = reinterpret_cast<float *>(sK) + t * (HD + 1);
+#pragma unroll 1
+                for (int c0 = 0; c0 < HD; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tmem + lane_base + O_COL + c0, v);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) po[c0 + e] = v[e];
+                }
+                float *pml = reinterpret_cast<float *>(sP) + 2 * t;
+                pml[0] = m_ref;
+                pml[1] = l;
+            }
+        } else if (p.n_splits > 1) {
+            // no keys in this split (or a failed wait): an empty partial
+            float *po = reinterpret_cast<float *>(sK) + t * (HD + 1);
+            for (int d = 0; d < HD; ++d) po[d] = 0.f;
+            float *pml = reinterpret_cast<float *>(sP) + 2 * t;
+            pml[0] = -1e30f;
+            pml[1] = 0.f;
+        }
+        tc_fence_before();
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+    if (p.n_splits == 1) return;
+
+    // The splits of this (sequence, kv head, query tile) form one cluster (rank = split).  CTA r
+    // merges its share of the rows from every rank's partial, in rank order:
+    // O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const int S = p.n_splits;
+    const float *po[8], *pml[8];
+    for (int rr = 0; rr < S; ++rr) {
+        po[rr] = cluster.map_shared_rank(reinterpret_cast<float *>(sK), rr);
+        pml[rr] = cluster.map_shared_rank(reinterpret_cast<float *>(sP), rr);
+    }
+    const int rs = BQ / S;
+    for (int e = threadIdx.x; e < rs * (HD / 2); e += blockDim.x) {
+        const int tl = split * rs + e / (HD / 2), d = (e % (HD / 2)) * 2;
+        const int rp = qtile * BQ + tl;
+        if (rp >= p.RP) continue;
+        float M = -INFINITY;
+        for (int rr = 0; rr < S; ++rr) M = fmaxf(M, pml[rr][2 * tl]);
+        float L = 0.f, a0 = 0.f, a1 = 0.f;
+        for (int rr = 0; rr < S; ++rr) {
+            const float w = exp2f(pml[rr][2 * tl] - M);
+            L += w * pml[rr][2 * tl + 1];
+            a0 += w * po[rr][tl * (HD + 1) + d];
+            a1 += w * po[rr][tl * (HD + 1) + d + 1];
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const int tt = rp / p.G, h = kvh * p.G + rp % p.G;
+        bf16 *dst = p.out + (long long)(j * p.Tq + tt) * p.out_ld + h * HD + d;
+        *reinterpret_cast<__nv_bfloat162 *>(dst) = __floats2bfloat162_rn(a0 * inv, a1 * inv);
+    }
+    cluster.sync();  // no CTA leaves while its partial may still be read
+}
+
+}  // namespace attn_tc

@@ -2,7 +2,9 @@
 //
 // D[a, b] = sum_k A[a, k] * B[b, k], both operands K-major bf16 in global memory, f32
 // accumulation in tensor memory.  One CTA computes one 128 x BN tile (128 rows of A = the
-// MMA's M side, BN rows of B = its N side) over a range of K (split-K):
+// MMA's M side, BN rows of B = its N side) over a range of K.  With split-K the splits of a
+// tile form one thread-block cluster and add their partial tiles through distributed shared
+// memory in rank order (no global round trip, deterministic).  Roles:
 //   warp 0      one thread issues TMA loads of A and B k-tiles (64 wide, 128-byte swizzle)
 //               into a ring of STAGES shared-memory slots,
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, K=16) per
@@ -16,7 +18,11 @@
 // readout A is the readout rows and B the vocabulary, so each thread owns one row's logits
 // and reduces them without shuffles; the logits never leave the SM.
 #pragma once
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace gemm {
 
@@ -29,8 +35,8 @@ struct EpiParams {
     float *out;           // EPI_F32 / EPI_ADD: out[b_row * ldo + a_row]
     int ldo;
     long long split_stride;
-    float *ws;            // split-K (gridDim.z > 1): partials ws[split * split_stride + b_row * rowsA + a_row]
-    int *counters;        // split-K: per output tile, splits done (left at zero)
+    float *ws;            // (stream-K kernel only) split partials
+    int *counters;        // (stream-K kernel only) per output tile, segments done (left at zero)
     bf16 *act;            // EPI_SWIGLU: act[b_row * ld_act + feature]
     int ld_act;
     float4 *partials;     // EPI_READOUT: partials[a_row * n_btiles + b_tile] = (max, sum e, sum e*d, argmax)
@@ -45,6 +51,7 @@ struct Cfg {
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr uint32_t TMEM_COLS = BN;  // power of two >= 32
     static constexpr size_t SMEM = 1024 /*align slack*/ + (size_t)STAGES * STAGE_BYTES + 256;
+    static_assert((size_t)BM * (BN + 1) * 4 <= (size_t)STAGES * STAGE_BYTES, "split-K partial must fit the ring");
 };
 
 template <int BN, int EPI>
@@ -187,48 +194,15 @@ __global__ void __launch_bounds__(192, 1)
                         apply(c0, v);
                     }
                 } else {
-                    // split-K: store this split's partial tile; the CTA that completes the tile last
-                    // adds the partials in split order (deterministic) and applies the epilogue
-                    float *mine = ep.ws + (long long)split * ep.split_stride;
+                    // split-K inside a cluster: park this split's partial tile in our own shared
+                    // memory (the stage ring is idle once the accumulator is complete); the
+                    // cluster reduces the partials below
+                    float *red = reinterpret_cast<float *>(smem);
                     for (int c0 = 0; c0 < BN; c0 += 16) {
-                        if (b0 + c0 >= rowsB) break;
                         float v[16];
                         tmem_ld16(taddr + c0, v);
-                        if (a_row < rowsA) {
 #pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                if (b0 + c0 + j < rowsB) mine[(long long)(b0 + c0 + j) * rowsA + a_row] = v[j];
-                        }
-                    }
-                    __threadfence();
-                    asm volatile("bar.sync 1, 128;" ::: "memory");
-                    __shared__ int last_split;
-                    if (threadIdx.x == 64) {
-                        const int n_btiles = a_fastest ? gridDim.y : gridDim.x;
-                        int *cnt = ep.counters + a_tile * n_btiles + b_tile;
-                        const int prev = atomicAdd(cnt, 1);
-                        last_split = prev == (int)gridDim.z - 1;
-                        if (last_split) *cnt = 0;
-                    }
-                    asm volatile("bar.sync 1, 128;" ::: "memory");
-                    if (last_split) {
-                        __threadfence();
-                        for (int c0 = 0; c0 < BN; c0 += 16) {
-                            if (b0 + c0 >= rowsB) break;
-                            float v[16];
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) v[j] = 0.f;
-                            if (a_row < rowsA) {
-                                for (int sp = 0; sp < (int)gridDim.z; ++sp) {
-                                    const float *src = ep.ws + (long long)sp * ep.split_stride;
-#pragma unroll
-                                    for (int j = 0; j < 16; ++j)
-                                        if (b0 + c0 + j < rowsB)
-                                            v[j] += __ldcg(src + (long long)(b0 + c0 + j) * rowsA + a_row);
-                                }
-                            }
-                            apply(c0, v);
-                        }
+                        for (int jj = 0; jj < 16; ++jj) red[(q * 32 + lane) * (BN + 1) + c0 + jj] = v[jj];
                     }
                 }
             } else {  // EPI_READOUT: this thread's row of logits over BN vocabulary entries
@@ -267,6 +241,51 @@ __global__ void __launch_bounds__(192, 1)
                     ep.partials[(long long)a_row * ep.n_btiles + b_tile] =
                         make_float4(best, se, sed, __int_as_float(best_idx));
             }
+        }
+    }
+    if constexpr (EPI == EPI_F32 || EPI == EPI_ADD || EPI == EPI_SWIGLU) {
+        if (gridDim.z > 1) {
+            // Split-K partials of the cluster's CTAs (one per split, cluster rank = split) sit in
+            // their shared memory; CTA r adds, for its share of the tile, the partials of ranks
+            // 0..S-1 in rank order (deterministic) through distributed shared memory and applies
+            // the epilogue.
+            cg::cluster_group cluster = cg::this_cluster();
+            cluster.sync();
+            const int S = gridDim.z, r = split;
+            float *red = reinterpret_cast<float *>(smem);
+            const float *part[8];
+            for (int rr = 0; rr < S; ++rr) part[rr] = cluster.map_shared_rank(red, rr);
+            if constexpr (EPI == EPI_SWIGLU) {
+                const int fs = 64 / S;  // features of the tile handled here
+                for (int e = threadIdx.x; e < fs * BN; e += blockDim.x) {
+                    const int fl = r * fs + e % fs, col = e / fs;
+                    const int grow = (fl >> 4) * 32 + (fl & 15), urow = grow + 16;
+                    float g = 0.f, u = 0.f;
+                    for (int rr = 0; rr < S; ++rr) {
+                        g += part[rr][grow * (BN + 1) + col];
+                        u += part[rr][urow * (BN + 1) + col];
+                    }
+                    const int br = b_tile * BN + col;
+                    if (a_tile * BM + grow < rowsA && br < rowsB)
+                        ep.act[(long long)br * ep.ld_act + a_tile * 64 + fl] = __float2bfloat16_rn(silu_f(g) * u);
+                }
+            } else {
+                const int rs = BM / S;  // tile rows handled here
+                for (int e = threadIdx.x; e < rs * BN; e += blockDim.x) {
+                    const int row = r * rs + e % rs, col = e / rs;
+                    float acc = 0.f;
+                    for (int rr = 0; rr < S; ++rr) acc += part[rr][row * (BN + 1) + col];
+                    const int ar = a_tile * BM + row, br = b_tile * BN + col;
+                    if (ar < rowsA && br < rowsB) {
+                        float *pp = ep.out + (long long)br * ep.ldo + ar;
+                        if constexpr (EPI == EPI_ADD)
+                            *pp += acc;
+                        else
+                            *pp = acc;
+                    }
+                }
+            }
+            cluster.sync();  // no CTA leaves while its partial may still be read
         }
     }
     tc_fence_before();

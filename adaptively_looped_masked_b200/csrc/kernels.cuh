@@ -104,7 +104,8 @@ __global__ void rmsnorm_kernel(const float *x, const float *g, bf16 *y, int H, f
 }
 
 // Per row m and head: optional per-head RMSNorm of q and k, rotate-half RoPE at the row's
-// position, then q -> q_out (bf16) and k, v -> the KV arena slot (bf16).
+// position, then q -> q_out (bf16, packed: [slot j][kv head][position * G + head-in-group][hd],
+// so the G query heads of a KV head are consecutive rows) and k, v -> the KV arena slot (bf16).
 __global__ void qkv_post_kernel(const float *qkv, int nq, int nkv, int hd, const float *qn, const float *kn,
                                 int qk_norm, float eps, const float2 *rope, RowMap map, bf16 *q_out, bf16 *kc,
                                 bf16 *vc, long long seq_stride, long long head_stride) {
@@ -150,7 +151,10 @@ __global__ void qkv_post_kernel(const float *qkv, int nq, int nkv, int hd, const
         }
         bf16 *dst;
         if (hh < nq) {
-            dst = q_out + ((long long)m * nq + hh) * hd;
+            // packed query order: per (sequence slot, kv head), row = position * G + head-in-group
+            const int G = nq / nkv;
+            const int RP = G * map.rows_per_seq;
+            dst = q_out + (((long long)jj * nkv + hh / G) * RP + (long long)t * G + hh % G) * hd;
         } else if (hh < nq + nkv) {
             dst = kc + (long long)b * seq_stride + (long long)(hh - nq) * head_stride + (long long)pos * hd;
         } else {
