@@ -349,24 +349,22 @@ __global__ void __launch_bounds__(192, 1)
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
     const int S = p.n_splits;
-    const float *po[8], *pml[8];
-    for (int rr = 0; rr < S; ++rr) {
-        po[rr] = cluster.map_shared_rank(reinterpret_cast<float *>(sK), rr);
-        pml[rr] = cluster.map_shared_rank(reinterpret_cast<float *>(sP), rr);
-    }
+    auto po = [&](int rr) -> const float * { return cluster.map_shared_rank(reinterpret_cast<float *>(sK), rr); };
+    auto pml = [&](int rr) -> const float * { return cluster.map_shared_rank(reinterpret_cast<float *>(sP), rr); };
     const int rs = BQ / S;
     for (int e = threadIdx.x; e < rs * (HD / 2); e += blockDim.x) {
         const int tl = split * rs + e / (HD / 2), d = (e % (HD / 2)) * 2;
         const int rp = qtile * BQ + tl;
         if (rp >= p.RP) continue;
         float M = -INFINITY;
-        for (int rr = 0; rr < S; ++rr) M = fmaxf(M, pml[rr][2 * tl]);
+        for (int rr = 0; rr < S; ++rr) M = fmaxf(M, pml(rr)[2 * tl]);
         float L = 0.f, a0 = 0.f, a1 = 0.f;
         for (int rr = 0; rr < S; ++rr) {
-            const float w = exp2f(pml[rr][2 * tl] - M);
-            L += w * pml[rr][2 * tl + 1];
-            a0 += w * po[rr][tl * (HD + 1) + d];
-            a1 += w * po[rr][tl * (HD + 1) + d + 1];
+            const float *ml = pml(rr), *o = po(rr);
+            const float w = exp2f(ml[2 * tl] - M);
+            L += w * ml[2 * tl + 1];
+            a0 += w * o[tl * (HD + 1) + d];
+            a1 += w * o[tl * (HD + 1) + d + 1];
         }
         const float inv = L > 0.f ? 1.f / L : 0.f;
         const int tt = rp / p.G, h = kvh * p.G + rp % p.G;

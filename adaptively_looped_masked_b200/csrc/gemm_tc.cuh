@@ -253,8 +253,7 @@ __global__ void __launch_bounds__(192, 1)
             cluster.sync();
             const int S = gridDim.z, r = split;
             float *red = reinterpret_cast<float *>(smem);
-            const float *part[8];
-            for (int rr = 0; rr < S; ++rr) part[rr] = cluster.map_shared_rank(red, rr);
+            auto part = [&](int rr) -> const float * { return cluster.map_shared_rank(red, rr); };
             if constexpr (EPI == EPI_SWIGLU) {
                 const int fs = 64 / S;  // features of the tile handled here
                 for (int e = threadIdx.x; e < fs * BN; e += blockDim.x) {
@@ -262,8 +261,9 @@ __global__ void __launch_bounds__(192, 1)
                     const int grow = (fl >> 4) * 32 + (fl & 15), urow = grow + 16;
                     float g = 0.f, u = 0.f;
                     for (int rr = 0; rr < S; ++rr) {
-                        g += part[rr][grow * (BN + 1) + col];
-                        u += part[rr][urow * (BN + 1) + col];
+                        const float *pr = part(rr);
+                        g += pr[grow * (BN + 1) + col];
+                        u += pr[urow * (BN + 1) + col];
                     }
                     const int br = b_tile * BN + col;
                     if (a_tile * BM + grow < rowsA && br < rowsB)
@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(192, 1)
                 for (int e = threadIdx.x; e < rs * BN; e += blockDim.x) {
                     const int row = r * rs + e % rs, col = e / rs;
                     float acc = 0.f;
-                    for (int rr = 0; rr < S; ++rr) acc += part[rr][row * (BN + 1) + col];
+                    for (int rr = 0; rr < S; ++rr) acc += part(rr)[row * (BN + 1) + col];
                     const int ar = a_tile * BM + row, br = b_tile * BN + col;
                     if (ar < rowsA && br < rowsB) {
                         float *pp = ep.out + (long long)br * ep.ldo + ar;
