@@ -130,6 +130,11 @@ void set_gemm_attr() {
                          (int)gemm::Cfg<BN>::SMEM);
 }
 template <int BN, int EPI>
+void set_persist_attr() {
+    cudaFuncSetAttribute(gemm::gemm_persist_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)gemm::Cfg<BN>::SMEM);
+}
+template <int BN, int EPI>
 void set_sk_attr() {
     cudaFuncSetAttribute(gemm::gemm_sk_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)gemm::SkCfg<BN>::SMEM);
@@ -153,6 +158,13 @@ bool init_kernel_attrs() {
     set_gemm_attr<256, gemm::EPI_ADD>();
     set_gemm_attr<256, gemm::EPI_SWIGLU>();
     set_gemm_attr<256, gemm::EPI_READOUT>();
+    set_persist_attr<128, gemm::EPI_F32>();
+    set_persist_attr<128, gemm::EPI_ADD>();
+    set_persist_attr<128, gemm::EPI_SWIGLU>();
+    set_persist_attr<256, gemm::EPI_F32>();
+    set_persist_attr<256, gemm::EPI_ADD>();
+    set_persist_attr<256, gemm::EPI_SWIGLU>();
+    set_persist_attr<256, gemm::EPI_READOUT>();
     set_sk_attr<32, gemm::EPI_F32>();
     set_sk_attr<32, gemm::EPI_ADD>();
     set_sk_attr<32, gemm::EPI_SWIGLU>();
@@ -189,8 +201,10 @@ GemmShape plan_gemm(int M, int Nw, int K) {
     const int tiles = cdiv(Nw, gemm::BM) * cdiv(M, g.bn);
     const int per_sm = g.bn <= 64 ? 2 : 1;
     int splits = (NUM_SMS_HINT * per_sm) / tiles;
-    // splits form one cluster (portable size <= 8); at least 4 k-tiles each
+    // splits form one cluster (portable size <= 8, a power of two so that the ranks share the
+    // 128 tile rows evenly in the reduction); at least 4 k-tiles each
     splits = std::max(1, std::min(std::min(splits, 8), g.k_tiles / 4));
+    while (splits & (splits - 1)) --splits;
     g.kps = cdiv(g.k_tiles, splits);
     g.splits = cdiv(g.k_tiles, g.kps);
     return g;
@@ -209,6 +223,16 @@ void launch_gemm_bn(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int
     else
     klaunch(gemm::gemm_tc_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM, st, tA, tB, rowsA, rowsB, rowsA_dyn, k_tiles,
                                                                            kps, a_fastest, ep, err);
+}
+
+// persistent kernel: one CTA per SM at most, walking the tiles
+template <int BN, int EPI>
+void launch_persist(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int rowsB, const int *rowsA_dyn,
+                    int k_tiles, int a_fastest, const gemm::EpiParams &ep, int *err, cudaStream_t st, int num_sms) {
+    const int tiles = cdiv(rowsA, gemm::BM) * cdiv(rowsB, BN);
+    const int grid = std::max(1, std::min(num_sms, tiles));
+    klaunch(gemm::gemm_persist_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM, st, tA, tB, rowsA, rowsB, rowsA_dyn,
+            k_tiles, a_fastest, ep, err);
 }
 
 template <int EPI>
@@ -302,6 +326,26 @@ int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_b
     GemmShape g = plan_gemm(M, Nw, K);
     const CUtensorMap *tB = map_for_bn(g.bn);
     if (!tB) return -1;
+    if (g.splits == 1 && g.bn >= 128) {
+        if (g.bn == 128) {
+            if (epi == gemm::EPI_F32)
+                launch_persist<128, gemm::EPI_F32>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms);
+            else if (epi == gemm::EPI_ADD)
+                launch_persist<128, gemm::EPI_ADD>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms);
+            else
+                launch_persist<128, gemm::EPI_SWIGLU>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st,
+                                                      env.num_sms);
+        } else {
+            if (epi == gemm::EPI_F32)
+                launch_persist<256, gemm::EPI_F32>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms);
+            else if (epi == gemm::EPI_ADD)
+                launch_persist<256, gemm::EPI_ADD>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms);
+            else
+                launch_persist<256, gemm::EPI_SWIGLU>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st,
+                                                      env.num_sms);
+        }
+        return 1;
+    }
     if (epi == gemm::EPI_F32)
         launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, env.err, env.st);
     else if (epi == gemm::EPI_ADD)
@@ -1066,9 +1110,9 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
             const double R_est = Ml;  // upper bound on the readout rows (exact counts are on the device)
             const double bytes = 2.0 * h->V * H + 2.0 * R_est * H + 16.0 * R_est * h->n_vt;
             LAUNCH(KC_RGEMM, bytes, 2.0 * R_est * h->V * (double)H,
-                   launch_gemm_bn<256, gemm::EPI_READOUT>(h->tm_rb, h->tm_lm, Ml, h->V, cdiv(H, gemm::BK),
-                                                          cdiv(H, gemm::BK), 1, 1, ep, h->d_err, h->stream,
-                                                          h->counts + 1));
+                   (launch_persist<256, gemm::EPI_READOUT>(h->tm_rb, h->tm_lm, Ml, h->V, h->counts + 1,
+                                                           cdiv(H, gemm::BK), 1, ep, h->d_err, h->stream,
+                                                           h->num_sms)));
             LAUNCH(KC_RCOMB, 16.0 * R_est * h->n_vt, 0.0,
                    (klaunch(k::readout_combine_kernel, cdiv(Ml, 8), 256, 0, h->stream, 
                        h->part, h->n_vt, h->counts + 1, h->rr_b, h->rr_i, h->lam_rr, N, K, s, h->a, h->cur_H,

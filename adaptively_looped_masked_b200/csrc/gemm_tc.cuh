@@ -526,3 +526,234 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 }  // namespace gemm
+
+namespace gemm {
+
+// ---------------------------------------------------------------------------------
+// Persistent variant for many tiles: a grid of at most one CTA per SM walks the output tiles
+// (consecutive CTAs share the weight tile, so it is read from HBM once), with the TMEM
+// accumulator double-buffered so that the epilogue of one tile overlaps the MMAs of the next
+// and the TMA ring streams across tile boundaries without a pipeline refill.
+// ---------------------------------------------------------------------------------
+template <int EPI, int BN>
+__device__ __forceinline__ void linear_chunk(int c0, const float (&v)[16], int a_row, int lane, int b0, int rowsA,
+                                             int rowsB, const EpiParams &ep) {
+    if constexpr (EPI == EPI_SWIGLU) {
+        const int feat = (a_row >> 5) * 16 + (lane & 15);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const float up = __shfl_xor_sync(0xffffffffu, v[j], 16);
+            const int br = b0 + c0 + j;
+            if (lane < 16 && a_row < rowsA && br < rowsB)
+                ep.act[(long long)br * ep.ld_act + feat] = __float2bfloat16_rn(silu_f(v[j]) * up);
+        }
+    } else if (a_row < rowsA) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int br = b0 + c0 + j;
+            if (br < rowsB) {
+                float *p = ep.out + (long long)br * ep.ldo + a_row;
+                if constexpr (EPI == EPI_ADD)
+                    *p += v[j];
+                else
+                    *p = v[j];
+            }
+        }
+    }
+}
+
+template <int BN>
+__device__ __forceinline__ void readout_tile(uint32_t taddr, int a_row, int b0, int b_tile, int rowsA, int rowsB,
+                                             const EpiParams &ep) {
+    float best = -INFINITY;
+    int best_idx = b0;
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+        if (b0 + c0 >= rowsB) break;
+        float v[16];
+        tmem_ld16(taddr + c0, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int vid = b0 + c0 + j;
+            if (vid < rowsB && v[j] > best) {  // strict: lowest id wins ties
+                best = v[j];
+                best_idx = vid;
+            }
+        }
+    }
+    float se = 0.f, sed = 0.f;
+    const float LOG2E = 1.4426950408889634f;
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+        if (b0 + c0 >= rowsB) break;
+        float v[16];
+        tmem_ld16(taddr + c0, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            if (b0 + c0 + j < rowsB) {
+                const float d = v[j] - best;
+                const float e = exp2f(d * LOG2E);
+                se += e;
+                sed = fmaf(e, d, sed);
+            }
+        }
+    }
+    if (a_row < rowsA)
+        ep.partials[(long long)a_row * ep.n_btiles + b_tile] = make_float4(best, se, sed, __int_as_float(best_idx));
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_persist_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int rowsA,
+                        int rowsB, const int *rowsA_dyn, int k_tiles, int a_fastest, EpiParams ep, int *err) {
+    using C = Cfg<BN>;
+    constexpr int STAGES = C::STAGES;
+    constexpr uint32_t TCOLS = 2 * BN;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * C::STAGE_BYTES);
+    uint64_t *empty = full + STAGES;
+    uint64_t *tfull = empty + STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull + b, 1);
+            mbar_init(tempty + b, 4);
+        }
+        fence_mbarrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TCOLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_trigger();
+    if (rowsA_dyn) {  // row count known only on the device
+        pdl_wait();
+        rowsA = min(rowsA, *rowsA_dyn);
+    }
+    const int n_a = (rowsA + BM - 1) / BM, n_b = (rowsB + BN - 1) / BN;
+    const int total = n_a * n_b;
+    auto tile_of = [&](int t, int &a, int &b) {
+        if (a_fastest) {
+            a = t % n_a;
+            b = t / n_a;
+        } else {
+            b = t % n_b;
+            a = t / n_b;
+        }
+    };
+
+    if (warp == 0) {
+        if (lane == 0 && blockIdx.x < total) {
+            int a, b;
+            tile_of(blockIdx.x, a, b);
+            // weights (operand A of the linear layers) do not depend on earlier kernels: the
+            // first stages of the first tile are requested before waiting for them
+            const int pre = rowsA_dyn ? 0 : min(k_tiles, STAGES);
+            for (int it = 0; it < pre; ++it) {
+                mbar_arrive_expect_tx(full + it, C::STAGE_BYTES);
+                tma_load_2d(smem + it * C::STAGE_BYTES, &tmA, full + it, it * BK, a * BM);
+            }
+            pdl_wait();
+            for (int it = 0; it < pre; ++it)
+                tma_load_2d(smem + it * C::STAGE_BYTES + C::A_BYTES, &tmB, full + it, it * BK, b * BN);
+            int g = 0, issued = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                tile_of(t, a, b);
+                for (int kt = 0; kt < k_tiles; ++kt, ++g) {
+                    if (g < pre) continue;
+                    const int s = g % STAGES;
+                    if (!mbar_wait(empty + s, ((uint32_t)(g / STAGES) & 1u) ^ 1u, err)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(full + s, C::STAGE_BYTES);
+                    uint8_t *sa = smem + s * C::STAGE_BYTES;
+                    tma_load_2d(sa, &tmA, full + s, kt * BK, a * BM);
+                    tma_load_2d(sa + C::A_BYTES, &tmB, full + s, kt * BK, b * BN);
+                    issued = g + 1;
+                }
+            }
+            issued = max(issued, pre);
+            for (int it = max(0, issued - STAGES); it < issued; ++it)
+                mbar_wait(full + (it % STAGES), (uint32_t)(it / STAGES) & 1u, err);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16(BM, BN);
+            int g = 0, li = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++li) {
+                const int buf = li & 1;
+                if (!mbar_wait(tempty + buf, ((uint32_t)(li >> 1) & 1u) ^ 1u, err)) break;
+                tc_fence_after();
+                for (int kt = 0; kt < k_tiles; ++kt, ++g) {
+                    const int s = g % STAGES;
+                    if (!mbar_wait(full + s, (uint32_t)(g / STAGES) & 1u, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+                    const uint64_t da = umma_sdesc_sw128(sa);
+                    const uint64_t db = umma_sdesc_sw128(sa + C::A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        umma_f16(tmem_base + buf * BN, da + 2 * k, db + 2 * k, idesc, (kt > 0 || k > 0) ? 1u : 0u);
+                    umma_commit(empty + s);
+                }
+                umma_commit(tfull + buf);
+            }
+        }
+    } else {
+        const int q = warp & 3;
+        pdl_wait();
+        int li = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++li) {
+            int a, b;
+            tile_of(t, a, b);
+            const int buf = li & 1;
+            const bool ready = mbar_wait(tfull + buf, (uint32_t)(li >> 1) & 1u, err);
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
+            const int a_row = a * BM + q * 32 + lane;
+            const int b0 = b * BN;
+            if (ready) {
+                if constexpr (EPI == EPI_READOUT) {
+                    readout_tile<BN>(taddr, a_row, b0, b, rowsA, rowsB, ep);
+                } else {
+                    for (int c0 = 0; c0 < BN; c0 += 16) {
+                        if (b0 + c0 >= rowsB) break;  // warp-uniform
+                        float v[16];
+                        tmem_ld16(taddr + c0, v);
+                        linear_chunk<EPI, BN>(c0, v, a_row, lane, b0, rowsA, rowsB, ep);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty + buf);
+            if (!ready) break;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TCOLS);
+    }
+}
+
+}  // namespace gemm

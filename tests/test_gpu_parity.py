@@ -42,7 +42,8 @@ def _gemm_ref(A, W):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 128, 64), (16, 200, 256), (32, 384, 880), (33, 1376, 256), (100, 512, 320),
-                                   (128, 256, 4096), (300, 640, 768), (2048, 512, 1024), (20, 6144, 4096)])
+                                   (128, 256, 4096), (300, 640, 768), (2048, 512, 1024), (20, 6144, 4096),
+                                   (512, 4096, 1024), (2048, 6144, 4096), (1000, 3000, 880)])
 def test_gemm_tcgen05_against_fp64(M, N, K):
     import adaptively_looped_masked_b200 as alo
     g = torch.Generator(device="cuda").manual_seed(M * 7 + N)
