@@ -589,8 +589,8 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
         const int base = qtiles * h->nkv * n_seq;
         const int ktiles = cdiv(kv_len, attn_tc::BKV);
         // splits of a query tile form one cluster (<= 8 CTAs, a power of two so that they
-        // share the 128 rows evenly), at least 2 key tiles each
-        int splits = std::max(1, std::min(std::min(ktiles / 2, cdiv(h->num_sms, base)), 8));
+        // share the 128 rows evenly); enough CTAs to cover the SMs
+        int splits = std::max(1, std::min(std::min(ktiles, cdiv(h->num_sms, base)), 8));
         while (splits & (splits - 1)) --splits;
         int kps = cdiv(ktiles, splits);
         while (splits > 1 && cdiv(ktiles, kps) < splits) {  // every rank gets keys

@@ -356,15 +356,30 @@ __global__ void __launch_bounds__(192, 1)
         const int tl = split * rs + e / (HD / 2), d = (e % (HD / 2)) * 2;
         const int rp = qtile * BQ + tl;
         if (rp >= p.RP) continue;
+        // every rank's values first (independent remote loads), then the merge in rank order
+        float mr[8], lr[8], o0[8], o1[8];
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
+            const int src = rr < S ? rr : 0;
+            const float *ml = pml(src), *o = po(src);
+            mr[rr] = ml[2 * tl];
+            lr[rr] = ml[2 * tl + 1];
+            o0[rr] = o[tl * (HD + 1) + d];
+            o1[rr] = o[tl * (HD + 1) + d + 1];
+        }
         float M = -INFINITY;
-        for (int rr = 0; rr < S; ++rr) M = fmaxf(M, pml(rr)[2 * tl]);
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr)
+            if (rr < S) M = fmaxf(M, mr[rr]);
         float L = 0.f, a0 = 0.f, a1 = 0.f;
-        for (int rr = 0; rr < S; ++rr) {
-            const float *ml = pml(rr), *o = po(rr);
-            const float w = exp2f(ml[2 * tl] - M);
-            L += w * ml[2 * tl + 1];
-            a0 += w * o[tl * (HD + 1) + d];
-            a1 += w * o[tl * (HD + 1) + d + 1];
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
+            if (rr < S) {
+                const float w = exp2f(mr[rr] - M);
+                L += w * lr[rr];
+                a0 += w * o0[rr];
+                a1 += w * o1[rr];
+            }
         }
         const float inv = L > 0.f ? 1.f / L : 0.f;
         const int tt = rp / p.G, h = kvh * p.G + rp % p.G;

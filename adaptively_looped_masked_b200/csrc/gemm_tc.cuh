@@ -43,6 +43,25 @@ struct EpiParams {
     int n_btiles;
 };
 
+// Write (EPI_F32) or add to (EPI_ADD) 16 consecutive rows of one output column: p points at
+// row 0, rows `ld` floats apart, only the first `n_rows` exist.  For the residual add every
+// old value is loaded before any store, so the 16 loads are in flight together.
+template <int EPI>
+__device__ __forceinline__ void store_chunk(const float (&v)[16], float *__restrict__ p, int ld, int n_rows) {
+    if constexpr (EPI == EPI_ADD) {
+        float old[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) old[j] = (j < n_rows) ? p[(long long)j * ld] : 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < n_rows) p[(long long)j * ld] = old[j] + v[j];
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < n_rows) p[(long long)j * ld] = v[j];
+    }
+}
+
 template <int BN>
 struct Cfg {
     static constexpr int STAGES = (BN <= 64) ? 4 : (BN == 128 ? 5 : 4);
@@ -173,17 +192,7 @@ __global__ void __launch_bounds__(192, 1)
                                 ep.act[(long long)br * ep.ld_act + feat] = __float2bfloat16_rn(silu_f(v[j]) * up);
                         }
                     } else if (a_row < rowsA) {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int br = b0 + c0 + j;
-                            if (br < rowsB) {
-                                float *p = ep.out + (long long)br * ep.ldo + a_row;
-                                if constexpr (EPI == EPI_ADD)
-                                    *p += v[j];
-                                else
-                                    *p = v[j];
-                            }
-                        }
+                        store_chunk<EPI>(v, ep.out + (long long)(b0 + c0) * ep.ldo + a_row, ep.ldo, rowsB - (b0 + c0));
                     }
                 };
                 if (gridDim.z == 1) {
@@ -259,11 +268,20 @@ __global__ void __launch_bounds__(192, 1)
                 for (int e = threadIdx.x; e < fs * BN; e += blockDim.x) {
                     const int fl = r * fs + e % fs, col = e / fs;
                     const int grow = (fl >> 4) * 32 + (fl & 15), urow = grow + 16;
+                    float xg[8], xu[8];
+#pragma unroll
+                    for (int rr = 0; rr < 8; ++rr) {
+                        const float *pr = part(rr < S ? rr : 0);
+                        xg[rr] = rr < S ? pr[grow * (BN + 1) + col] : 0.f;
+                        xu[rr] = rr < S ? pr[urow * (BN + 1) + col] : 0.f;
+                    }
                     float g = 0.f, u = 0.f;
-                    for (int rr = 0; rr < S; ++rr) {
-                        const float *pr = part(rr);
-                        g += pr[grow * (BN + 1) + col];
-                        u += pr[urow * (BN + 1) + col];
+#pragma unroll
+                    for (int rr = 0; rr < 8; ++rr) {
+                        if (rr < S) {
+                            g += xg[rr];
+                            u += xu[rr];
+                        }
                     }
                     const int br = b_tile * BN + col;
                     if (a_tile * BM + grow < rowsA && br < rowsB)
@@ -273,8 +291,14 @@ __global__ void __launch_bounds__(192, 1)
                 const int rs = BM / S;  // tile rows handled here
                 for (int e = threadIdx.x; e < rs * BN; e += blockDim.x) {
                     const int row = r * rs + e % rs, col = e / rs;
+                    // every rank's value first (independent remote loads), then the sum in rank order
+                    float x[8];
+#pragma unroll
+                    for (int rr = 0; rr < 8; ++rr) x[rr] = rr < S ? part(rr)[row * (BN + 1) + col] : 0.f;
                     float acc = 0.f;
-                    for (int rr = 0; rr < S; ++rr) acc += part(rr)[row * (BN + 1) + col];
+#pragma unroll
+                    for (int rr = 0; rr < 8; ++rr)
+                        if (rr < S) acc += x[rr];
                     const int ar = a_tile * BM + row, br = b_tile * BN + col;
                     if (ar < rowsA && br < rowsB) {
                         float *pp = ep.out + (long long)br * ep.ldo + ar;
@@ -339,14 +363,11 @@ __device__ __forceinline__ void sk_epilogue(const float (&acc)[BN], int a_row, i
     } else {
         if (a_row < rowsA) {
 #pragma unroll
-            for (int j = 0; j < BN; ++j) {
-                if (j < rowsB) {
-                    float *p = ep.out + (long long)j * ep.ldo + a_row;
-                    if constexpr (EPI == EPI_ADD)
-                        *p += acc[j];
-                    else
-                        *p = acc[j];
-                }
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                float v[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = acc[c0 + j];
+                store_chunk<EPI>(v, ep.out + (long long)c0 * ep.ldo + a_row, ep.ldo, rowsB - c0);
             }
         }
     }
@@ -548,17 +569,7 @@ __device__ __forceinline__ void linear_chunk(int c0, const float (&v)[16], int a
                 ep.act[(long long)br * ep.ld_act + feat] = __float2bfloat16_rn(silu_f(v[j]) * up);
         }
     } else if (a_row < rowsA) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const int br = b0 + c0 + j;
-            if (br < rowsB) {
-                float *p = ep.out + (long long)br * ep.ldo + a_row;
-                if constexpr (EPI == EPI_ADD)
-                    *p += v[j];
-                else
-                    *p = v[j];
-            }
-        }
+        store_chunk<EPI>(v, ep.out + (long long)(b0 + c0) * ep.ldo + a_row, ep.ldo, rowsB - (b0 + c0));
     }
 }
 

@@ -122,10 +122,18 @@ __global__ void qkv_post_kernel(const float *qkv, int nq, int nkv, int hd, const
     const float *row = qkv + (long long)m * n_heads * hd;
     // blockIdx.y selects a group of nw heads: one warp per (row, head)
     for (int hh = blockIdx.y * nw + warp; hh < min(n_heads, (int)(blockIdx.y + 1) * nw); hh += nw) {
-        float x[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            if (e < E) x[e] = row[hh * hd + lane * E + e];
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (E == 4) {
+            const float4 t4 = *reinterpret_cast<const float4 *>(row + hh * hd + lane * 4);
+            x[0] = t4.x;
+            x[1] = t4.y;
+            x[2] = t4.z;
+            x[3] = t4.w;
+        } else {
+            const float2 t2 = *reinterpret_cast<const float2 *>(row + hh * hd + lane * 2);
+            x[0] = t2.x;
+            x[1] = t2.y;
+        }
         if (hh < nq + nkv) {
             const float *w = hh < nq ? qn : kn;
             if (qk_norm) {
@@ -160,9 +168,12 @@ __global__ void qkv_post_kernel(const float *qkv, int nq, int nkv, int hd, const
         } else {
             dst = vc + (long long)b * seq_stride + (long long)(hh - nq - nkv) * head_stride + (long long)pos * hd;
         }
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            if (e < E) dst[lane * E + e] = __float2bfloat16_rn(x[e]);
+        if (E == 4) {
+            __nv_bfloat162 b2[2] = {__floats2bfloat162_rn(x[0], x[1]), __floats2bfloat162_rn(x[2], x[3])};
+            *reinterpret_cast<uint2 *>(dst + lane * 4) = *reinterpret_cast<const uint2 *>(b2);
+        } else {
+            *reinterpret_cast<__nv_bfloat162 *>(dst + lane * 2) = __floats2bfloat162_rn(x[0], x[1]);
+        }
     }
 }
 
