@@ -592,11 +592,7 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
         // share the 128 rows evenly); enough CTAs to cover the SMs
         int splits = std::max(1, std::min(std::min(ktiles, cdiv(h->num_sms, base)), 8));
         while (splits & (splits - 1)) --splits;
-        int kps = cdiv(ktiles, splits);
-        while (splits > 1 && cdiv(ktiles, kps) < splits) {  // every rank gets keys
-            splits >>= 1;
-            kps = cdiv(ktiles, splits);
-        }
+        const int kps = cdiv(ktiles, splits);  // trailing ranks may get no keys (empty partials)
         p.n_splits = splits;
         p.keys_per_split = kps * attn_tc::BKV;
         const double bytes = 4.0 * n_seq * h->nkv * (double)kv_len * h->hd + 4.0 * M * h->nq * h->hd;

@@ -11,8 +11,9 @@
 //               then O += P_i V_i into the TMEM accumulator (V read MN-major)
 //   warps 2-5   softmax, one thread per query row: tcgen05.ld its S row, exp2 with a running
 //               reference max that only moves when the row max passes it by more than 8
-//               (rescaling O in TMEM then), P_i as bf16 into shared memory in the MMA's
-//               128-byte-swizzled K-major layout; at the end O / l to global memory
+//               (rescaling O in TMEM then), P_i as bf16 into a double-buffered shared-memory
+//               tile in the MMA's 128-byte-swizzled K-major layout (the exponentials of tile i
+//               overlap PV_{i-1}); at the end O / l to global memory
 //
 // With n_splits > 1 the keys are split across the CTAs of a cluster; each parks (O, reference
 // max, l) in its shared memory and the cluster merges them in rank order through distributed
@@ -37,7 +38,7 @@ constexpr uint32_t P_BYTES = 2 * HALF;
 constexpr uint32_t TMEM_COLS = 512;      // S0 [0,128) S1 [128,256) O [256,384)
 constexpr uint32_t O_COL = 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
-constexpr size_t SMEM = 1024 + Q_BYTES + 2 * KV_STAGES * KV_BYTES + P_BYTES + 256;
+constexpr size_t SMEM = 1024 + Q_BYTES + 2 * KV_STAGES * KV_BYTES + 2 * P_BYTES + 256;  // P double-buffered
 
 struct Params {
     int RP;            // packed query rows per (sequence, kv head) = G * rows_per_seq
@@ -96,15 +97,15 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t *sK = sQ + Q_BYTES;                       // [stage] K tiles
     uint8_t *sV = sK + KV_STAGES * KV_BYTES;          // [stage] V tiles
     uint8_t *sP = sV + KV_STAGES * KV_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sP + P_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sP + 2 * P_BYTES);
     uint64_t *q_full = bars;
     uint64_t *k_full = bars + 1;                      // [2]
     uint64_t *v_full = bars + 3;                      // [2]
     uint64_t *kv_empty = bars + 5;                    // [2]
     uint64_t *s_full = bars + 7;                      // [2]
     uint64_t *p_full = bars + 9;
-    uint64_t *pv_done = bars + 10;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 11);
+    uint64_t *pv_done = bars + 10;                    // [2], PV_i completes pv_done[i & 1]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 12);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qtile = blockIdx.x;
@@ -124,6 +125,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         mbar_init(p_full, 128);
         mbar_init(pv_done, 1);
+        mbar_init(pv_done + 1, 1);
         fence_mbarrier_init();
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
@@ -199,14 +201,15 @@ __global__ void __launch_bounds__(192, 1)
                 if (!mbar_wait(v_full + s, ((uint32_t)(i >> 1)) & 1u, p.err)) break;
                 tc_fence_after();
                 const uint32_t v_addr = smem_u32(sV + s * KV_BYTES);
+                const uint32_t pb_addr = p_addr + (i & 1) * P_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < BKV / 16; ++kk) {
                     const uint32_t a_off = (kk >> 2) * HALF + (kk & 3) * 32;  // P: keys contiguous
                     const uint32_t b_off = kk * 16 * 128;                      // V: 16 key rows of 128 B
-                    umma_f16(tmem + O_COL, sdesc_k(p_addr + a_off), sdesc_mn(v_addr + b_off, HALF), idesc_o,
+                    umma_f16(tmem + O_COL, sdesc_k(pb_addr + a_off), sdesc_mn(v_addr + b_off, HALF), idesc_o,
                              (i > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(pv_done);
+                umma_commit(pv_done + (i & 1));
                 umma_commit(kv_empty + s);
             }
         }
@@ -239,44 +242,49 @@ __global__ void __launch_bounds__(192, 1)
                 sv[c] = (key0 + c < kend) ? sv[c] * p.scale_log2 : -INFINITY;
                 mt = fmaxf(mt, sv[c]);
             }
-            // O and the P buffer are free once the previous PV product has completed
-            if (i > 0 && !mbar_wait(pv_done, ((uint32_t)(i - 1)) & 1u, p.err)) {
+            // the reference max moves only when this tile's max passes it by more than 2^8
+            const bool resc = mt > m_ref + RESCALE_THRESHOLD;
+            const float f = (resc && i > 0) ? exp2f(m_ref - mt) : 1.f;
+            if (resc) m_ref = mt;
+            float lt = 0.f;
+#pragma unroll
+            for (int c = 0; c < BKV; ++c) {
+                sv[c] = exp2f(sv[c] - m_ref);
+                lt += sv[c];
+            }
+            l = l * f + lt;
+            // P buffer i & 1 was last read by PV_{i-2}; a rescale of O needs PV_{i-1} complete
+            if (i >= 2 && !mbar_wait(pv_done + (i & 1), ((uint32_t)((i - 2) >> 1)) & 1u, p.err)) {
                 ok = false;
                 break;
             }
-            tc_fence_after();
-            if (mt > m_ref + RESCALE_THRESHOLD) {
-                if (i > 0) {
-                    const float f = exp2f(m_ref - mt);
-                    l *= f;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < HD; c0 += 16) {
-                        float v[16];
-                        tmem_ld16(tmem + lane_base + O_COL + c0, v);
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) v[e] *= f;
-                        tmem_st16(tmem + lane_base + O_COL + c0, v);
-                    }
+            if (resc && i > 0) {
+                if (!mbar_wait(pv_done + ((i - 1) & 1), ((uint32_t)((i - 1) >> 1)) & 1u, p.err)) {
+                    ok = false;
+                    break;
                 }
-                m_ref = mt;
+                tc_fence_after();
+#pragma unroll 1
+                for (int c0 = 0; c0 < HD; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tmem + lane_base + O_COL + c0, v);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] *= f;
+                    tmem_st16(tmem + lane_base + O_COL + c0, v);
+                }
             }
             // P row in the K-major 128-byte-swizzled layout: keys 0-63 in the first region,
             // 64-127 in the second; 16-byte chunk c of row t at (t/8)*1024 + (t%8)*128 + ((c ^ t%8)*16)
+            uint8_t *pbuf = sP + (i & 1) * P_BYTES;
 #pragma unroll
             for (int c = 0; c < BKV / 8; ++c) {
-                float pe[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    pe[e] = exp2f(sv[c * 8 + e] - m_ref);
-                    l += pe[e];
-                }
                 uint4 pk;
-                pk.x = pack2_bf16(pe[0], pe[1]);
-                pk.y = pack2_bf16(pe[2], pe[3]);
-                pk.z = pack2_bf16(pe[4], pe[5]);
-                pk.w = pack2_bf16(pe[6], pe[7]);
+                pk.x = pack2_bf16(sv[c * 8 + 0], sv[c * 8 + 1]);
+                pk.y = pack2_bf16(sv[c * 8 + 2], sv[c * 8 + 3]);
+                pk.z = pack2_bf16(sv[c * 8 + 4], sv[c * 8 + 5]);
+                pk.w = pack2_bf16(sv[c * 8 + 6], sv[c * 8 + 7]);
                 const int region = c >> 3, ch = c & 7;
-                uint8_t *dst = sP + region * HALF + (t >> 3) * 1024 + (t & 7) * 128 + ((ch ^ (t & 7)) << 4);
+                uint8_t *dst = pbuf + region * HALF + (t >> 3) * 1024 + (t & 7) * 128 + ((ch ^ (t & 7)) << 4);
                 *reinterpret_cast<uint4 *>(dst) = pk;
             }
             fence_proxy_async_smem();
@@ -284,7 +292,8 @@ __global__ void __launch_bounds__(192, 1)
             mbar_arrive(p_full);
         }
         // ---------------- output ----------------
-        if (ok && n_tiles > 0 && mbar_wait(pv_done, ((uint32_t)(n_tiles - 1)) & 1u, p.err)) {
+        if (ok && n_tiles > 0 &&
+            mbar_wait(pv_done + ((n_tiles - 1) & 1), ((uint32_t)((n_tiles - 1) >> 1)) & 1u, p.err)) {
             tc_fence_after();
             const int rp = qtile * BQ + t;
             const bool valid = rp < p.RP;

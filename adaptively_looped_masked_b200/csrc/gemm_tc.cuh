@@ -62,13 +62,31 @@ __device__ __forceinline__ void store_chunk(const float (&v)[16], float *__restr
     }
 }
 
+// 16 accumulator columns starting at column c0, summed over NACC accumulators BN columns
+// apart (in accumulator order)
+template <int NACC, int BN>
+__device__ __forceinline__ void acc_ld16(uint32_t taddr, int c0, float (&v)[16]) {
+    tmem_ld16(taddr + c0, v);
+#pragma unroll
+    for (int a = 1; a < NACC; ++a) {
+        float w[16];
+        tmem_ld16(taddr + a * BN + c0, w);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] += w[j];
+    }
+}
+
 template <int BN>
 struct Cfg {
     static constexpr int STAGES = (BN <= 64) ? 4 : (BN == 128 ? 5 : 4);
     static constexpr uint32_t A_BYTES = BM * BK * 2;
     static constexpr uint32_t B_BYTES = BN * BK * 2;
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr uint32_t TMEM_COLS = BN;  // power of two >= 32
+    // Few activation rows: the MMA per 16-wide k step is small and its latency, not the tensor
+    // pipe, would pace a single accumulation chain; the four k steps of a stage then go to four
+    // independent TMEM accumulators, summed in a fixed order by the epilogue.
+    static constexpr int NACC = (BN <= 64) ? 4 : 1;
+    static constexpr uint32_t TMEM_COLS = BN * NACC;  // power of two >= 32
     static constexpr size_t SMEM = 1024 /*align slack*/ + (size_t)STAGES * STAGE_BYTES + 256;
     static_assert((size_t)BM * (BN + 1) * 4 <= (size_t)STAGES * STAGE_BYTES, "split-K partial must fit the ring");
 };
@@ -162,7 +180,8 @@ __global__ void __launch_bounds__(192, 1)
                 const uint64_t db = umma_sdesc_sw128(sa + C::A_BYTES);
 #pragma unroll
                 for (int k = 0; k < BK / 16; ++k)  // 16 bf16 = 32 bytes = 2 descriptor units per k step
-                    umma_f16(tmem_base, da + 2 * k, db + 2 * k, idesc, (it > 0 || k > 0) ? 1u : 0u);
+                    umma_f16(tmem_base + (k % C::NACC) * BN, da + 2 * k, db + 2 * k, idesc,
+                             (it > 0 || k >= C::NACC) ? 1u : 0u);
                 umma_commit(empty + s);
             }
             umma_commit(accum);
@@ -199,7 +218,7 @@ __global__ void __launch_bounds__(192, 1)
                     for (int c0 = 0; c0 < BN; c0 += 16) {
                         if (b0 + c0 >= rowsB) break;  // warp-uniform
                         float v[16];
-                        tmem_ld16(taddr + c0, v);
+                        acc_ld16<C::NACC, BN>(taddr, c0, v);
                         apply(c0, v);
                     }
                 } else {
@@ -209,7 +228,7 @@ __global__ void __launch_bounds__(192, 1)
                     float *red = reinterpret_cast<float *>(smem);
                     for (int c0 = 0; c0 < BN; c0 += 16) {
                         float v[16];
-                        tmem_ld16(taddr + c0, v);
+                        acc_ld16<C::NACC, BN>(taddr, c0, v);
 #pragma unroll
                         for (int jj = 0; jj < 16; ++jj) red[(q * 32 + lane) * (BN + 1) + c0 + jj] = v[jj];
                     }
