@@ -6,6 +6,7 @@
 
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -212,37 +213,41 @@ GemmShape plan_gemm(int M, int Nw, int K) {
 
 template <int BN, int EPI>
 void launch_gemm_bn(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int rowsB, int k_tiles, int kps,
-                    int splits, int a_fastest, const gemm::EpiParams &ep, int *err, cudaStream_t st,
-                    const int *rowsA_dyn = nullptr) {
+                    int splits, int a_fastest, const gemm::EpiParams &ep, int *err, cudaStream_t st, int tiled) {
     dim3 grid;
     const int ta = cdiv(rowsA, gemm::BM), tb = cdiv(rowsB, BN);
     grid = a_fastest ? dim3(ta, tb, splits) : dim3(tb, ta, splits);
     if (splits > 1)
         klaunch_cluster(gemm::gemm_tc_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM, st, splits, tA, tB, rowsA,
-                        rowsB, rowsA_dyn, k_tiles, kps, a_fastest, ep, err);
+                        rowsB, (const int *)nullptr, k_tiles, kps, a_fastest, tiled, ep, err);
     else
-    klaunch(gemm::gemm_tc_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM, st, tA, tB, rowsA, rowsB, rowsA_dyn, k_tiles,
-                                                                           kps, a_fastest, ep, err);
+        klaunch(gemm::gemm_tc_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM, st, tA, tB, rowsA, rowsB,
+                (const int *)nullptr, k_tiles, kps, a_fastest, tiled, ep, err);
 }
 
 // persistent kernel: one CTA per SM at most, walking the tiles
 template <int BN, int EPI>
 void launch_persist(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int rowsB, const int *rowsA_dyn,
-                    int k_tiles, int a_fastest, const gemm::EpiParams &ep, int *err, cudaStream_t st, int num_sms) {
+                    int k_tiles, int a_fastest, const gemm::EpiParams &ep, int *err, cudaStream_t st, int num_sms,
+                    int tiled) {
     const int tiles = cdiv(rowsA, gemm::BM) * cdiv(rowsB, BN);
     const int grid = std::max(1, std::min(num_sms, tiles));
     klaunch(gemm::gemm_persist_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM, st, tA, tB, rowsA, rowsB, rowsA_dyn,
-            k_tiles, a_fastest, ep, err);
+            k_tiles, a_fastest, tiled, ep, err);
 }
 
 template <int EPI>
 void launch_gemm_epi(int bn, const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int rowsB, int k_tiles, int kps,
-                     int splits, int a_fastest, const gemm::EpiParams &ep, int *err, cudaStream_t st) {
+                     int splits, int a_fastest, const gemm::EpiParams &ep, int *err, cudaStream_t st, int tiled) {
     switch (bn) {
-        case 32: launch_gemm_bn<32, EPI>(tA, tB, rowsA, rowsB, k_tiles, kps, splits, a_fastest, ep, err, st); break;
-        case 64: launch_gemm_bn<64, EPI>(tA, tB, rowsA, rowsB, k_tiles, kps, splits, a_fastest, ep, err, st); break;
-        case 128: launch_gemm_bn<128, EPI>(tA, tB, rowsA, rowsB, k_tiles, kps, splits, a_fastest, ep, err, st); break;
-        default: launch_gemm_bn<256, EPI>(tA, tB, rowsA, rowsB, k_tiles, kps, splits, a_fastest, ep, err, st); break;
+        case 32: launch_gemm_bn<32, EPI>(tA, tB, rowsA, rowsB, k_tiles, kps, splits, a_fastest, ep, err, st, tiled); break;
+        case 64: launch_gemm_bn<64, EPI>(tA, tB, rowsA, rowsB, k_tiles, kps, splits, a_fastest, ep, err, st, tiled); break;
+        case 128:
+            launch_gemm_bn<128, EPI>(tA, tB, rowsA, rowsB, k_tiles, kps, splits, a_fastest, ep, err, st, tiled);
+            break;
+        default:
+            launch_gemm_bn<256, EPI>(tA, tB, rowsA, rowsB, k_tiles, kps, splits, a_fastest, ep, err, st, tiled);
+            break;
     }
 }
 
@@ -303,7 +308,7 @@ void launch_sk(const SkPlan &p, const CUtensorMap &tW, const CUtensorMap &tB, in
 // failure).
 template <typename MapFn>
 int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_bn, int M, int K, int epi, float *out,
-             int ldo, bf16 *act_out, int ld_act, bool stream_k) {
+             int ldo, bf16 *act_out, int ld_act, bool stream_k, int w_tiled) {
     gemm::EpiParams ep{};
     ep.out = out;
     ep.ldo = ldo;
@@ -329,29 +334,29 @@ int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_b
     if (g.splits == 1 && g.bn >= 128) {
         if (g.bn == 128) {
             if (epi == gemm::EPI_F32)
-                launch_persist<128, gemm::EPI_F32>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms);
+                launch_persist<128, gemm::EPI_F32>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled);
             else if (epi == gemm::EPI_ADD)
-                launch_persist<128, gemm::EPI_ADD>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms);
+                launch_persist<128, gemm::EPI_ADD>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled);
             else
                 launch_persist<128, gemm::EPI_SWIGLU>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st,
-                                                      env.num_sms);
+                                                      env.num_sms, w_tiled);
         } else {
             if (epi == gemm::EPI_F32)
-                launch_persist<256, gemm::EPI_F32>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms);
+                launch_persist<256, gemm::EPI_F32>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled);
             else if (epi == gemm::EPI_ADD)
-                launch_persist<256, gemm::EPI_ADD>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms);
+                launch_persist<256, gemm::EPI_ADD>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled);
             else
                 launch_persist<256, gemm::EPI_SWIGLU>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st,
-                                                      env.num_sms);
+                                                      env.num_sms, w_tiled);
         }
         return 1;
     }
     if (epi == gemm::EPI_F32)
-        launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, env.err, env.st);
+        launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, env.err, env.st, w_tiled);
     else if (epi == gemm::EPI_ADD)
-        launch_gemm_epi<gemm::EPI_ADD>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, env.err, env.st);
+        launch_gemm_epi<gemm::EPI_ADD>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, env.err, env.st, w_tiled);
     else
-        launch_gemm_epi<gemm::EPI_SWIGLU>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, env.err, env.st);
+        launch_gemm_epi<gemm::EPI_SWIGLU>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, env.err, env.st, w_tiled);
     return 1;
 }
 
@@ -560,7 +565,8 @@ int linear(alodlm *h, const CUtensorMap &tmW, int Nw, const bf16 *actp, int M, i
     auto map_for_bn = [&](int bn) { return act_map(h, actp, K, h->rows_cap, bn); };
     int n = 0;
     LAUNCH(KC_GEMM, bytes, flops,
-           n = run_gemm(env, tmW, Nw, map_for_bn, M, K, epi, out, ldo, act_out, ld_act, ALODLM_STEP_STREAM_K != 0));
+           n = run_gemm(env, tmW, Nw, map_for_bn, M, K, epi, out, ldo, act_out, ld_act, ALODLM_STEP_STREAM_K != 0,
+                        1));
     if (n < 0) return fail(h, ALODLM_ECUDA, "cuTensorMapEncodeTiled failed (activation)");
     h->launches += n - 1;
     return ALODLM_OK;
@@ -803,13 +809,35 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
         return code;
     };
 
-    // ---- weights: pack to bf16, rows padded to multiples of 128 with zeros ----
-    auto pack = [&](bf16 **dst, int rows_pad, int cols, const void *src, int src_rows) -> int {
-        int r;
-        if ((r = dalloc(h, dst, (size_t)rows_pad * cols))) return r;
-        cudaMemsetAsync(*dst, 0, (size_t)rows_pad * cols * 2, h->stream);
-        k::pack_rows_kernel<<<src_rows, 256, 0, h->stream>>>(src, f32, cols, nullptr, src_rows, cols, *dst, cols);
+    // ---- weights: pack to bf16 (rows padded with zeros), then store every matrix the GEMMs
+    // stream in the tiled layout (each [tile rows x 64] tile contiguous) ----
+    const size_t stage_elems =
+        std::max({(size_t)round_up(h->V, 256) * H, (size_t)round_up(h->n_qkv, 128) * H, (size_t)round_up(H, 128) * qd,
+                  (size_t)round_up(2 * h->I, 128) * H, (size_t)round_up(H, 128) * h->I});
+    bf16 *stage = nullptr;
+    if (cudaMalloc(&stage, stage_elems * 2) != cudaSuccess) {
+        cudaGetLastError();
+        h->err = "cudaMalloc failed (weight staging)";
+        return cleanup(ALODLM_ENOMEM);
+    }
+    struct StageGuard {
+        bf16 *p;
+        ~StageGuard() { cudaFree(p); }
+    } stage_guard{stage};
+    auto stage_rows = [&](int rows_pad, int cols, const void *src, int src_rows) -> int {
+        cudaMemsetAsync(stage, 0, (size_t)rows_pad * cols * 2, h->stream);
+        k::pack_rows_kernel<<<src_rows, 256, 0, h->stream>>>(src, f32, cols, nullptr, src_rows, cols, stage, cols);
         return check_launch(h, "pack_rows_kernel");
+    };
+    // stage (rows_pad x cols, row-major) -> tiled copy in handle memory + its tensor map
+    auto tile_from_stage = [&](bf16 **dst, CUtensorMap *map, int rows_pad, int cols, int RT) -> int {
+        const int KT = cdiv(cols, 64), n_rt = rows_pad / RT;
+        int r;
+        if ((r = dalloc(h, dst, (size_t)n_rt * KT * RT * 64))) return r;
+        k::tile_matrix_kernel<<<n_rt * KT, 256, 0, h->stream>>>(stage, rows_pad, cols, RT, KT, *dst);
+        if ((r = check_launch(h, "tile_matrix_kernel"))) return r;
+        if (!make_tmap(map, *dst, 64, n_rt * KT * RT, RT)) return fail(h, ALODLM_ECUDA, "cuTensorMapEncodeTiled failed");
+        return ALODLM_OK;
     };
     auto copy_vec = [&](float **dst, const void *src, int n) -> int {
         int r;
@@ -817,48 +845,49 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
         cudaMemcpyAsync(*dst, src, n * sizeof(float), cudaMemcpyDeviceToDevice, h->stream);
         return ALODLM_OK;
     };
-    if ((rc = pack(&h->embed, h->V, H, w->embed, h->V))) return cleanup(rc);
-    if ((rc = pack(&h->lm_head, round_up(h->V, 256), H, w->lm_head, h->V))) return cleanup(rc);
+    // the embedding is gathered by rows: plain layout
+    if ((rc = dalloc(h, &h->embed, (size_t)h->V * H))) return cleanup(rc);
+    k::pack_rows_kernel<<<h->V, 256, 0, h->stream>>>(w->embed, f32, H, nullptr, h->V, H, h->embed, H);
+    if ((rc = check_launch(h, "pack embed"))) return cleanup(rc);
+    if ((rc = stage_rows(round_up(h->V, 256), H, w->lm_head, h->V)) ||
+        (rc = tile_from_stage(&h->lm_head, &h->tm_lm, round_up(h->V, 256), H, 256)))
+        return cleanup(rc);
     if ((rc = copy_vec(&h->final_norm, w->final_norm, H))) return cleanup(rc);
     if ((rc = copy_vec(&h->exit_w, w->exit_w, H))) return cleanup(rc);
     h->exit_b = w->exit_b;
-    if (!make_tmap(&h->tm_lm, h->lm_head, H, round_up(h->V, 256), 256)) {
-        h->err = "cuTensorMapEncodeTiled failed (lm_head)";
-        return cleanup(ALODLM_ECUDA);
-    }
     h->layers.resize(L);
     for (int l = 0; l < L; ++l) {
         const alodlm_layer_w &lw = w->layers[l];
         LayerDev &d = h->layers[l];
         // fused QKV: rows [q; k; v]
-        if ((rc = dalloc(h, &d.wqkv, (size_t)round_up(h->n_qkv, 128) * H))) return cleanup(rc);
-        cudaMemsetAsync(d.wqkv, 0, (size_t)round_up(h->n_qkv, 128) * H * 2, h->stream);
-        k::pack_rows_kernel<<<qd, 256, 0, h->stream>>>(lw.q, f32, H, nullptr, qd, H, d.wqkv, H);
+        cudaMemsetAsync(stage, 0, (size_t)round_up(h->n_qkv, 128) * H * 2, h->stream);
+        k::pack_rows_kernel<<<qd, 256, 0, h->stream>>>(lw.q, f32, H, nullptr, qd, H, stage, H);
         k::pack_rows_kernel<<<h->nkv * h->hd, 256, 0, h->stream>>>(lw.k, f32, H, nullptr, h->nkv * h->hd, H,
-                                                                   d.wqkv + (size_t)qd * H, H);
+                                                                   stage + (size_t)qd * H, H);
         k::pack_rows_kernel<<<h->nkv * h->hd, 256, 0, h->stream>>>(
-            lw.v, f32, H, nullptr, h->nkv * h->hd, H, d.wqkv + (size_t)(qd + h->nkv * h->hd) * H, H);
+            lw.v, f32, H, nullptr, h->nkv * h->hd, H, stage + (size_t)(qd + h->nkv * h->hd) * H, H);
         if ((rc = check_launch(h, "pack qkv"))) return cleanup(rc);
-        if ((rc = pack(&d.wo, round_up(H, 128), qd, lw.o, H))) return cleanup(rc);
-        if ((rc = dalloc(h, &d.wgu, (size_t)round_up(2 * h->I, 128) * H))) return cleanup(rc);
-        cudaMemsetAsync(d.wgu, 0, (size_t)round_up(2 * h->I, 128) * H * 2, h->stream);
-        k::pack_gate_up_kernel<<<2 * h->I, 256, 0, h->stream>>>(lw.gate, lw.up, f32, h->I, H, d.wgu);
+        if ((rc = tile_from_stage(&d.wqkv, &d.tm_qkv, round_up(h->n_qkv, 128), H, 128))) return cleanup(rc);
+        if ((rc = stage_rows(round_up(H, 128), qd, lw.o, H)) ||
+            (rc = tile_from_stage(&d.wo, &d.tm_o, round_up(H, 128), qd, 128)))
+            return cleanup(rc);
+        cudaMemsetAsync(stage, 0, (size_t)round_up(2 * h->I, 128) * H * 2, h->stream);
+        k::pack_gate_up_kernel<<<2 * h->I, 256, 0, h->stream>>>(lw.gate, lw.up, f32, h->I, H, stage);
         if ((rc = check_launch(h, "pack gate/up"))) return cleanup(rc);
-        if ((rc = pack(&d.wd, round_up(H, 128), h->I, lw.down, H))) return cleanup(rc);
+        if ((rc = tile_from_stage(&d.wgu, &d.tm_gu, round_up(2 * h->I, 128), H, 128))) return cleanup(rc);
+        if ((rc = stage_rows(round_up(H, 128), h->I, lw.down, H)) ||
+            (rc = tile_from_stage(&d.wd, &d.tm_d, round_up(H, 128), h->I, 128)))
+            return cleanup(rc);
         if ((rc = copy_vec(&d.attn_norm, lw.attn_norm, H))) return cleanup(rc);
         if ((rc = copy_vec(&d.mlp_norm, lw.mlp_norm, H))) return cleanup(rc);
         if (cfg->qk_norm) {
             if ((rc = copy_vec(&d.q_norm, lw.q_norm, h->hd))) return cleanup(rc);
             if ((rc = copy_vec(&d.k_norm, lw.k_norm, h->hd))) return cleanup(rc);
         }
-        bool ok = make_tmap(&d.tm_qkv, d.wqkv, H, round_up(h->n_qkv, 128), 128) &&
-                  make_tmap(&d.tm_o, d.wo, qd, round_up(H, 128), 128) &&
-                  make_tmap(&d.tm_gu, d.wgu, H, round_up(2 * h->I, 128), 128) &&
-                  make_tmap(&d.tm_d, d.wd, h->I, round_up(H, 128), 128);
-        if (!ok) {
-            h->err = "cuTensorMapEncodeTiled failed (layer weights)";
-            return cleanup(ALODLM_ECUDA);
-        }
+    }
+    if (cudaStreamSynchronize(h->stream) != cudaSuccess) {
+        h->err = "weight packing failed";
+        return cleanup(ALODLM_ECUDA);
     }
 
     // ---- depth-aware KV arena ----
@@ -1108,7 +1137,7 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
             LAUNCH(KC_RGEMM, bytes, 2.0 * R_est * h->V * (double)H,
                    (launch_persist<256, gemm::EPI_READOUT>(h->tm_rb, h->tm_lm, Ml, h->V, h->counts + 1,
                                                            cdiv(H, gemm::BK), 1, ep, h->d_err, h->stream,
-                                                           h->num_sms)));
+                                                           h->num_sms, 2)));
             LAUNCH(KC_RCOMB, 16.0 * R_est * h->n_vt, 0.0,
                    (klaunch(k::readout_combine_kernel, cdiv(Ml, 8), 256, 0, h->stream, 
                        h->part, h->n_vt, h->counts + 1, h->rr_b, h->rr_i, h->lam_rr, N, K, s, h->a, h->cur_H,
@@ -1261,7 +1290,7 @@ int alodlm_gemm_bf16(const void *A, const void *W, float *C, int M, int N, int K
     CUtensorMap tW, tA;
     if (!make_tmap(&tW, W, K, N, gemm::BM)) return ALODLM_ECUDA;
     auto map_for_bn = [&](int bn) -> const CUtensorMap * { return make_tmap(&tA, A, K, M, bn) ? &tA : nullptr; };
-    if (run_gemm(env, tW, N, map_for_bn, M, K, gemm::EPI_F32, C, N, nullptr, 0, true) < 0) return ALODLM_ECUDA;
+    if (run_gemm(env, tW, N, map_for_bn, M, K, gemm::EPI_F32, C, N, nullptr, 0, true, 0) < 0) return ALODLM_ECUDA;
     return cudaGetLastError() == cudaSuccess ? ALODLM_OK : ALODLM_ECUDA;
 }
 

@@ -62,6 +62,19 @@ __device__ __forceinline__ void store_chunk(const float (&v)[16], float *__restr
     }
 }
 
+// Operand layouts in global memory.  Plain: row-major [rows, K] (TMA box at x = k, y = row).
+// Tiled (the library's own weights): every [tile_rows x 64] tile of the matrix stored
+// contiguously, tiles ordered (row tile, k tile), k padded with zeros to a multiple of 64 --
+// one TMA box then streams one contiguous run of HBM instead of tile_rows 128-byte pieces.
+// `tiled` bit 0: operand A tiled with 128-row tiles; bit 1: operand B tiled with BN-row tiles.
+__device__ __forceinline__ void tma_operand(void *dst, const CUtensorMap *map, uint64_t *bar, bool tiled, int tile,
+                                            int tile_rows, int kt, int k_tiles) {
+    if (tiled)
+        tma_load_2d(dst, map, bar, 0, (tile * k_tiles + kt) * tile_rows);
+    else
+        tma_load_2d(dst, map, bar, kt * BK, tile * tile_rows);
+}
+
 // 16 accumulator columns starting at column c0, summed over NACC accumulators BN columns
 // apart (in accumulator order)
 template <int NACC, int BN>
@@ -94,8 +107,8 @@ struct Cfg {
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int rowsA,
-                   int rowsB, const int *rowsA_dyn, int k_tiles, int kt_per_split, int a_fastest, EpiParams ep,
-                   int *err) {
+                   int rowsB, const int *rowsA_dyn, int k_tiles, int kt_per_split, int a_fastest, int tiled,
+                   EpiParams ep, int *err) {
     using C = Cfg<BN>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -147,11 +160,12 @@ __global__ void __launch_bounds__(192, 1)
             const int pre = rowsA_dyn ? 0 : min(nkt, STAGES);
             for (int it = 0; it < pre; ++it) {
                 mbar_arrive_expect_tx(full + it, C::STAGE_BYTES);
-                tma_load_2d(smem + it * C::STAGE_BYTES, &tmA, full + it, (kt0 + it) * BK, a_tile * BM);
+                tma_operand(smem + it * C::STAGE_BYTES, &tmA, full + it, tiled & 1, a_tile, BM, kt0 + it, k_tiles);
             }
             pdl_wait();
             for (int it = 0; it < pre; ++it)
-                tma_load_2d(smem + it * C::STAGE_BYTES + C::A_BYTES, &tmB, full + it, (kt0 + it) * BK, b_tile * BN);
+                tma_operand(smem + it * C::STAGE_BYTES + C::A_BYTES, &tmB, full + it, tiled & 2, b_tile, BN, kt0 + it,
+                            k_tiles);
             int issued = pre;
             for (int it = pre; it < nkt; ++it) {
                 const int s = it % STAGES;
@@ -160,8 +174,9 @@ __global__ void __launch_bounds__(192, 1)
                 mbar_arrive_expect_tx(full + s, C::STAGE_BYTES);
                 uint8_t *sa = smem + s * C::STAGE_BYTES;
                 const int kx = (kt0 + it) * BK;
-                tma_load_2d(sa, &tmA, full + s, kx, a_tile * BM);
-                tma_load_2d(sa + C::A_BYTES, &tmB, full + s, kx, b_tile * BN);
+                tma_operand(sa, &tmA, full + s, tiled & 1, a_tile, BM, kt0 + it, k_tiles);
+                tma_operand(sa + C::A_BYTES, &tmB, full + s, tiled & 2, b_tile, BN, kt0 + it, k_tiles);
+                (void)kx;
                 issued = it + 1;
             }
             // make sure no copy into shared memory is still in flight when the CTA exits
@@ -633,7 +648,8 @@ __device__ __forceinline__ void readout_tile(uint32_t taddr, int a_row, int b0, 
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     gemm_persist_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int rowsA,
-                        int rowsB, const int *rowsA_dyn, int k_tiles, int a_fastest, EpiParams ep, int *err) {
+                        int rowsB, const int *rowsA_dyn, int k_tiles, int a_fastest, int tiled, EpiParams ep,
+                        int *err) {
     using C = Cfg<BN>;
     constexpr int STAGES = C::STAGES;
     constexpr uint32_t TCOLS = 2 * BN;
@@ -693,11 +709,11 @@ __global__ void __launch_bounds__(192, 1)
             const int pre = rowsA_dyn ? 0 : min(k_tiles, STAGES);
             for (int it = 0; it < pre; ++it) {
                 mbar_arrive_expect_tx(full + it, C::STAGE_BYTES);
-                tma_load_2d(smem + it * C::STAGE_BYTES, &tmA, full + it, it * BK, a * BM);
+                tma_operand(smem + it * C::STAGE_BYTES, &tmA, full + it, tiled & 1, a, BM, it, k_tiles);
             }
             pdl_wait();
             for (int it = 0; it < pre; ++it)
-                tma_load_2d(smem + it * C::STAGE_BYTES + C::A_BYTES, &tmB, full + it, it * BK, b * BN);
+                tma_operand(smem + it * C::STAGE_BYTES + C::A_BYTES, &tmB, full + it, tiled & 2, b, BN, it, k_tiles);
             int g = 0, issued = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
@@ -711,8 +727,8 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     mbar_arrive_expect_tx(full + s, C::STAGE_BYTES);
                     uint8_t *sa = smem + s * C::STAGE_BYTES;
-                    tma_load_2d(sa, &tmA, full + s, kt * BK, a * BM);
-                    tma_load_2d(sa + C::A_BYTES, &tmB, full + s, kt * BK, b * BN);
+                    tma_operand(sa, &tmA, full + s, tiled & 1, a, BM, kt, k_tiles);
+                    tma_operand(sa + C::A_BYTES, &tmB, full + s, tiled & 2, b, BN, kt, k_tiles);
                     issued = g + 1;
                 }
             }

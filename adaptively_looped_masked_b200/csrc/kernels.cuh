@@ -44,6 +44,19 @@ __global__ void pack_gate_up_kernel(const void *gate, const void *up, int src_is
     }
 }
 
+// Tiled weight layout: tile (rt, kt) = rows [rt*RT, rt*RT+RT) x columns [kt*64, kt*64+64) of the
+// row-major source, stored contiguously (RT x 64, row-major) at tile index rt*KT + kt; columns
+// past `cols` are zero.  One block per tile.
+__global__ void tile_matrix_kernel(const bf16 *src, int rows, int cols, int RT, int KT, bf16 *dst) {
+    const int rt = blockIdx.x / KT, kt = blockIdx.x % KT;
+    bf16 *d = dst + (long long)blockIdx.x * RT * 64;
+    for (int idx = threadIdx.x; idx < RT * 64; idx += blockDim.x) {
+        const int r = idx >> 6, c = idx & 63;
+        const int row = rt * RT + r, col = kt * 64 + c;
+        d[idx] = (row < rows && col < cols) ? src[(long long)row * cols + col] : __float2bfloat16_rn(0.f);
+    }
+}
+
 // rope[pos][j] = (cos, sin)(pos * base^(-2j/hd)), evaluated in double precision
 __global__ void rope_table_kernel(float2 *rope, int n_pos, int half, double base) {
     const long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x;

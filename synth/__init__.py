@@ -62,6 +62,9 @@ MODELS: Dict[str, ModelShape] = {
     "mid": ModelShape("mid", 320, 6, 2, 128, 880, 3001, 2, 3, 2),
     # Prelude 0 / Coda 0 special case: the whole stack loops
     "tiny_fullcore": ModelShape("tiny_fullcore", 256, 4, 2, 64, 688, 2048, 0, 2, 0, weight_dtype="fp32"),
+    # narrow model with the Qwen3-8B attention geometry (32 q / 8 kv heads, head_dim 128):
+    # kernel-level profiling of the step's attention and small kernels on a few-MB footprint
+    "attn-probe": ModelShape("attn-probe", 256, 32, 8, 128, 256, 1024, 1, 1, 1),
     # Qwen3-1.7B shape, 28 layers split 8 / 12 / 8
     "qwen3-1.7b": ModelShape("qwen3-1.7b", 2048, 16, 8, 128, 6144, 151936, 8, 12, 8),
     # Qwen3-8B shape, 36 layers split 10 / 16 / 10
@@ -85,6 +88,8 @@ class Workload:
 WORKLOADS: Dict[str, Workload] = {
     "tiny": Workload("tiny", "tiny", 1, 48, 16, 4, (0.1, 0.6, 0.9), (0.1, 0.9)),
     "mid": Workload("mid", "mid", 3, 75, 20, 5, (0.1, 0.6, 0.9), (0.1, 0.9)),
+    "attn-probe-bs1": Workload("attn-probe-bs1", "attn-probe", 1, 1024, 32, 2, (0.6,), (0.5,)),
+    "attn-probe-bs32": Workload("attn-probe-bs32", "attn-probe", 32, 2048, 64, 2, (0.6,), (0.5,)),
     "qwen3-1.7b-bs1": Workload("qwen3-1.7b-bs1", "qwen3-1.7b", 1, 512, 32, 8, (0.6,), (0.5,)),
     "qwen3-8b-bs1": Workload("qwen3-8b-bs1", "qwen3-8b", 1, 1024, 32, 8, (0.6,), (0.5,)),
     "qwen3-8b-bs32": Workload("qwen3-8b-bs32", "qwen3-8b", 32, 2048, 64, 8, (0.1, 0.6, 0.9), (0.1, 0.9)),
