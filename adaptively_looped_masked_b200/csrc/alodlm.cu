@@ -28,6 +28,9 @@ namespace {
 // the weights faster than the stream-K kernel at 32-64 rows (0.77 vs 0.65 of the measured
 // HBM bandwidth on the 24576 x 4096 gate/up shape).  The GEMM entry points use stream-K for
 // up to 64 rows.
+#ifndef ALODLM_MAX_SPLITS
+#define ALODLM_MAX_SPLITS 8
+#endif
 #ifndef ALODLM_STEP_STREAM_K
 #define ALODLM_STEP_STREAM_K 0
 #endif
@@ -128,7 +131,7 @@ bool make_tmap(CUtensorMap *map, const void *ptr, int inner, int rows, int box_r
 template <int BN, int EPI>
 void set_gemm_attr() {
     cudaFuncSetAttribute(gemm::gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)gemm::Cfg<BN>::SMEM);
+                         (int)gemm::Cfg<BN>::SMEM_SPLIT);
 }
 template <int BN, int EPI>
 void set_persist_attr() {
@@ -204,7 +207,7 @@ GemmShape plan_gemm(int M, int Nw, int K) {
     int splits = (NUM_SMS_HINT * per_sm) / tiles;
     // splits form one cluster (portable size <= 8, a power of two so that the ranks share the
     // 128 tile rows evenly in the reduction); at least 4 k-tiles each
-    splits = std::max(1, std::min(std::min(splits, 8), g.k_tiles / 4));
+    splits = std::max(1, std::min(std::min(splits, ALODLM_MAX_SPLITS), g.k_tiles / 4));
     while (splits & (splits - 1)) --splits;
     g.kps = cdiv(g.k_tiles, splits);
     g.splits = cdiv(g.k_tiles, g.kps);
@@ -218,7 +221,7 @@ void launch_gemm_bn(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int
     const int ta = cdiv(rowsA, gemm::BM), tb = cdiv(rowsB, BN);
     grid = a_fastest ? dim3(ta, tb, splits) : dim3(tb, ta, splits);
     if (splits > 1)
-        klaunch_cluster(gemm::gemm_tc_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM, st, splits, tA, tB, rowsA,
+        klaunch_cluster(gemm::gemm_tc_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM_SPLIT, st, splits, tA, tB, rowsA,
                         rowsB, (const int *)nullptr, k_tiles, kps, a_fastest, tiled, ep, err);
     else
         klaunch(gemm::gemm_tc_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM, st, tA, tB, rowsA, rowsB,
@@ -1290,7 +1293,8 @@ int alodlm_gemm_bf16(const void *A, const void *W, float *C, int M, int N, int K
     CUtensorMap tW, tA;
     if (!make_tmap(&tW, W, K, N, gemm::BM)) return ALODLM_ECUDA;
     auto map_for_bn = [&](int bn) -> const CUtensorMap * { return make_tmap(&tA, A, K, M, bn) ? &tA : nullptr; };
-    if (run_gemm(env, tW, N, map_for_bn, M, K, gemm::EPI_F32, C, N, nullptr, 0, true, 0) < 0) return ALODLM_ECUDA;
+    if (run_gemm(env, tW, N, map_for_bn, M, K, gemm::EPI_F32, C, N, nullptr, 0, ALODLM_STEP_STREAM_K != 0, 0) < 0)
+        return ALODLM_ECUDA;
     return cudaGetLastError() == cudaSuccess ? ALODLM_OK : ALODLM_ECUDA;
 }
 

@@ -2,9 +2,11 @@
 //
 // D[a, b] = sum_k A[a, k] * B[b, k], both operands K-major bf16 in global memory, f32
 // accumulation in tensor memory.  One CTA computes one 128 x BN tile (128 rows of A = the
-// MMA's M side, BN rows of B = its N side) over a range of K.  With split-K the splits of a
-// tile form one thread-block cluster and add their partial tiles through distributed shared
-// memory in rank order (no global round trip, deterministic).  Roles:
+// MMA's M side, BN rows of B = its N side) over a range of K.  With split-K the S splits of a
+// tile form one thread-block cluster: each CTA owns 128/S rows of the tile, every CTA stores
+// its partial of those rows straight into the owner's shared memory (remote stores, no
+// round-trip latency), one cluster barrier, and each owner adds the S partials in rank order
+// (deterministic) and applies the epilogue.  Roles:
 //   warp 0      one thread issues TMA loads of A and B k-tiles (64 wide, 128-byte swizzle)
 //               into a ring of STAGES shared-memory slots,
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, K=16) per
@@ -75,33 +77,61 @@ __device__ __forceinline__ void tma_operand(void *dst, const CUtensorMap *map, u
         tma_load_2d(dst, map, bar, kt * BK, tile * tile_rows);
 }
 
-// 16 accumulator columns starting at column c0, summed over NACC accumulators BN columns
-// apart (in accumulator order)
+// NC accumulator columns starting at column c0, summed over NACC accumulators BN columns
+// apart (in accumulator order).  All loads are issued before one wait.
+template <int NACC, int BN, int NC>
+__device__ __forceinline__ void acc_ld(uint32_t taddr, int c0, float (&v)[NC]) {
+    uint32_t r[NACC][NC];
+#pragma unroll
+    for (int a = 0; a < NACC; ++a)
+#pragma unroll
+        for (int c = 0; c < NC; c += 16) tmem_ld16_async(taddr + a * BN + c0 + c, &r[a][c]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int a = 0; a < NACC; ++a)
+#pragma unroll
+        for (int j = 0; j < NC; ++j) reg_after_wait(r[a][j]);
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+        float x = __uint_as_float(r[0][j]);
+#pragma unroll
+        for (int a = 1; a < NACC; ++a) x += __uint_as_float(r[a][j]);
+        v[j] = x;
+    }
+}
 template <int NACC, int BN>
 __device__ __forceinline__ void acc_ld16(uint32_t taddr, int c0, float (&v)[16]) {
-    tmem_ld16(taddr + c0, v);
-#pragma unroll
-    for (int a = 1; a < NACC; ++a) {
-        float w[16];
-        tmem_ld16(taddr + a * BN + c0, w);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] += w[j];
-    }
+    acc_ld<NACC, BN, 16>(taddr, c0, v);
 }
 
 template <int BN>
 struct Cfg {
-    static constexpr int STAGES = (BN <= 64) ? 4 : (BN == 128 ? 5 : 4);
+#ifndef ALODLM_STAGES_SMALL
+#define ALODLM_STAGES_SMALL 4
+#endif
+    static constexpr int STAGES = (BN <= 64) ? ALODLM_STAGES_SMALL : (BN == 128 ? 5 : 4);
     static constexpr uint32_t A_BYTES = BM * BK * 2;
     static constexpr uint32_t B_BYTES = BN * BK * 2;
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
     // Few activation rows: the MMA per 16-wide k step is small and its latency, not the tensor
     // pipe, would pace a single accumulation chain; the four k steps of a stage then go to four
     // independent TMEM accumulators, summed in a fixed order by the epilogue.
-    static constexpr int NACC = (BN <= 64) ? 4 : 1;
+#ifndef ALODLM_NACC_SMALL
+#define ALODLM_NACC_SMALL 1
+#endif
+    static constexpr int NACC = (BN <= 64) ? ALODLM_NACC_SMALL : 1;
+    // epilogue columns per TMEM round trip: a narrow tile's whole row at once
+    static constexpr int EC = (BN <= 64) ? BN : 16;
     static constexpr uint32_t TMEM_COLS = BN * NACC;  // power of two >= 32
     static constexpr size_t SMEM = 1024 /*align slack*/ + (size_t)STAGES * STAGE_BYTES + 256;
-    static_assert((size_t)BM * (BN + 1) * 4 <= (size_t)STAGES * STAGE_BYTES, "split-K partial must fit the ring");
+    // split-K receive buffer: [split][owned row][BN + 4] f32.  Narrow tiles get a buffer of their own behind the barriers (a partial can then be
+    // pushed while the owner is still streaming); wide tiles reuse the stage ring once every CTA
+    // of the cluster is done with its own.
+    static constexpr bool RECV_SEPARATE = BN <= 64;
+    static constexpr int RECV_LD = BN + 4;  // floats per received row (16-byte aligned rows)
+    static constexpr size_t RECV_BYTES = (size_t)BM * RECV_LD * 4;
+    static constexpr size_t SMEM_SPLIT = SMEM + (RECV_SEPARATE ? RECV_BYTES : 0);
+    static_assert(RECV_SEPARATE || RECV_BYTES <= (size_t)STAGES * STAGE_BYTES, "split-K partials must fit the ring");
 };
 
 template <int BN, int EPI>
@@ -140,6 +170,18 @@ __global__ void __launch_bounds__(192, 1)
         fence_mbarrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        // The A operand of the linear layers is a weight, which no kernel writes: its first
+        // stages are requested right away (before the TMEM allocation and, under programmatic
+        // dependent launch, before the predecessor kernel has finished), so the pipeline fills
+        // while the rest starts up.  The readout's A operand is produced by the predecessor
+        // (rowsA_dyn set): then everything waits.
+        if (!rowsA_dyn) {
+            const int pre = min(nkt, STAGES);
+            for (int it = 0; it < pre; ++it) {
+                mbar_arrive_expect_tx(full + it, C::STAGE_BYTES);
+                tma_operand(smem + it * C::STAGE_BYTES, &tmA, full + it, tiled & 1, a_tile, BM, kt0 + it, k_tiles);
+            }
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -150,18 +192,17 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     pdl_trigger();
+    constexpr bool SPLIT_EPI = EPI == EPI_F32 || EPI == EPI_ADD || EPI == EPI_SWIGLU;
+    const bool split_k = SPLIT_EPI && gridDim.z > 1;
+    float *recv = reinterpret_cast<float *>(C::RECV_SEPARATE ? smem + STAGES * C::STAGE_BYTES + 256 : smem);
+    // phase 0 of the cluster barrier: "every CTA of the cluster has started" (separate receive
+    // buffer) or "every CTA is done with its stage ring" (receive buffer in the ring, arrived below)
+    if (split_k && C::RECV_SEPARATE) cluster_arrive_relaxed();
+    bool ep_ready = false;
 
     if (warp == 0) {
         if (lane == 0) {
-            // The A operand of the linear layers is a weight, which no kernel writes: its first
-            // stages are requested before waiting for the predecessor kernel, so the pipeline
-            // fills while the predecessor drains.  The readout's A operand is produced by the
-            // predecessor (rowsA_dyn set): then everything waits.
-            const int pre = rowsA_dyn ? 0 : min(nkt, STAGES);
-            for (int it = 0; it < pre; ++it) {
-                mbar_arrive_expect_tx(full + it, C::STAGE_BYTES);
-                tma_operand(smem + it * C::STAGE_BYTES, &tmA, full + it, tiled & 1, a_tile, BM, kt0 + it, k_tiles);
-            }
+            const int pre = rowsA_dyn ? 0 : min(nkt, STAGES);  // A stages already requested above
             pdl_wait();
             for (int it = 0; it < pre; ++it)
                 tma_operand(smem + it * C::STAGE_BYTES + C::A_BYTES, &tmB, full + it, tiled & 2, b_tile, BN, kt0 + it,
@@ -206,6 +247,7 @@ __global__ void __launch_bounds__(192, 1)
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         pdl_wait();
         const bool ready = mbar_wait(accum, 0, err);
+        ep_ready = ready;
         tc_fence_after();
         const int a_row = a_tile * BM + q * 32 + lane;
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
@@ -230,24 +272,17 @@ __global__ void __launch_bounds__(192, 1)
                     }
                 };
                 if (gridDim.z == 1) {
-                    for (int c0 = 0; c0 < BN; c0 += 16) {
+                    for (int c0 = 0; c0 < BN; c0 += C::EC) {
                         if (b0 + c0 >= rowsB) break;  // warp-uniform
-                        float v[16];
-                        acc_ld16<C::NACC, BN>(taddr, c0, v);
-                        apply(c0, v);
-                    }
-                } else {
-                    // split-K inside a cluster: park this split's partial tile in our own shared
-                    // memory (the stage ring is idle once the accumulator is complete); the
-                    // cluster reduces the partials below
-                    float *red = reinterpret_cast<float *>(smem);
-                    for (int c0 = 0; c0 < BN; c0 += 16) {
-                        float v[16];
-                        acc_ld16<C::NACC, BN>(taddr, c0, v);
+                        float v[C::EC];
+                        acc_ld<C::NACC, BN, C::EC>(taddr, c0, v);
 #pragma unroll
-                        for (int jj = 0; jj < 16; ++jj) red[(q * 32 + lane) * (BN + 1) + c0 + jj] = v[jj];
+                        for (int sc = 0; sc < C::EC; sc += 16) {
+                            if (b0 + c0 + sc >= rowsB) break;
+                            apply(c0 + sc, *reinterpret_cast<const float(*)[16]>(&v[sc]));
+                        }
                     }
-                }
+                }  // split-K: pushed to the owners below
             } else {  // EPI_READOUT: this thread's row of logits over BN vocabulary entries
                 float best = -INFINITY;
                 int best_idx = b0;
@@ -286,64 +321,90 @@ __global__ void __launch_bounds__(192, 1)
             }
         }
     }
-    if constexpr (EPI == EPI_F32 || EPI == EPI_ADD || EPI == EPI_SWIGLU) {
-        if (gridDim.z > 1) {
-            // Split-K partials of the cluster's CTAs (one per split, cluster rank = split) sit in
-            // their shared memory; CTA r adds, for its share of the tile, the partials of ranks
-            // 0..S-1 in rank order (deterministic) through distributed shared memory and applies
-            // the epilogue.
-            cg::cluster_group cluster = cg::this_cluster();
-            cluster.sync();
-            const int S = gridDim.z, r = split;
-            float *red = reinterpret_cast<float *>(smem);
-            auto part = [&](int rr) -> const float * { return cluster.map_shared_rank(red, rr); };
-            if constexpr (EPI == EPI_SWIGLU) {
-                const int fs = 64 / S;  // features of the tile handled here
-                for (int e = threadIdx.x; e < fs * BN; e += blockDim.x) {
-                    const int fl = r * fs + e % fs, col = e / fs;
-                    const int grow = (fl >> 4) * 32 + (fl & 15), urow = grow + 16;
-                    float xg[8], xu[8];
-#pragma unroll
-                    for (int rr = 0; rr < 8; ++rr) {
-                        const float *pr = part(rr < S ? rr : 0);
-                        xg[rr] = rr < S ? pr[grow * (BN + 1) + col] : 0.f;
-                        xu[rr] = rr < S ? pr[urow * (BN + 1) + col] : 0.f;
-                    }
-                    float g = 0.f, u = 0.f;
-#pragma unroll
-                    for (int rr = 0; rr < 8; ++rr) {
-                        if (rr < S) {
-                            g += xg[rr];
-                            u += xu[rr];
-                        }
-                    }
-                    const int br = b_tile * BN + col;
-                    if (a_tile * BM + grow < rowsA && br < rowsB)
-                        ep.act[(long long)br * ep.ld_act + a_tile * 64 + fl] = __float2bfloat16_rn(silu_f(g) * u);
+    if constexpr (SPLIT_EPI) {
+        if (split_k) {
+            const int S = gridDim.z, r = split;  // cluster rank = split (S a power of two)
+            const int rs = BM / S;                // tile rows owned by each rank
+            const int lg_rs = __ffs(rs) - 1;
+            constexpr int LD = C::RECV_LD;
+            // With the receive buffer in the ring: an epilogue thread gets here only once the
+            // accumulator is complete (every MMA has read its stage), so this arrival means
+            // "this CTA no longer uses its ring".
+            if (!C::RECV_SEPARATE) cluster_arrive_relaxed();
+            cluster_wait_acquire();
+            if (warp >= 2 && ep_ready) {
+                // push this split's partial rows to their owners: row -> (owner, owned-row index)
+                const int q = warp & 3, tr = q * 32 + lane;
+                int owner, lr;
+                if constexpr (EPI == EPI_SWIGLU) {
+                    // owners split by feature so that a feature's gate and up rows (16 apart in
+                    // each 32-row group) meet at one owner: features [o*fs, (o+1)*fs), gate rows
+                    // first, then the up rows
+                    const int fs = 64 / S, f = (tr >> 5) * 16 + (tr & 15);
+                    owner = f / fs;
+                    lr = (f - owner * fs) + ((tr & 16) ? fs : 0);
+                } else {
+                    owner = tr / rs;
+                    lr = tr - owner * rs;
                 }
-            } else {
-                const int rs = BM / S;  // tile rows handled here
-                for (int e = threadIdx.x; e < rs * BN; e += blockDim.x) {
-                    const int row = r * rs + e % rs, col = e / rs;
-                    // every rank's value first (independent remote loads), then the sum in rank order
-                    float x[8];
+                const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
+                const uint32_t dst = cluster_map(smem_u32(recv + (size_t)(r * rs + lr) * LD), (uint32_t)owner);
+                for (int c0 = 0; c0 < BN; c0 += C::EC) {
+                    float v[C::EC];
+                    acc_ld<C::NACC, BN, C::EC>(taddr, c0, v);
 #pragma unroll
-                    for (int rr = 0; rr < 8; ++rr) x[rr] = rr < S ? part(rr)[row * (BN + 1) + col] : 0.f;
-                    float acc = 0.f;
-#pragma unroll
-                    for (int rr = 0; rr < 8; ++rr)
-                        if (rr < S) acc += x[rr];
-                    const int ar = a_tile * BM + row, br = b_tile * BN + col;
-                    if (ar < rowsA && br < rowsB) {
-                        float *pp = ep.out + (long long)br * ep.ldo + ar;
-                        if constexpr (EPI == EPI_ADD)
-                            *pp += acc;
-                        else
-                            *pp = acc;
-                    }
+                    for (int j = 0; j < C::EC; j += 4)
+                        st_cluster_v4(dst + (uint32_t)(c0 + j) * 4u, v[j], v[j + 1], v[j + 2], v[j + 3]);
                 }
             }
-            cluster.sync();  // no CTA leaves while its partial may still be read
+            cluster_arrive_release();
+            cluster_wait_acquire();  // every partial of the rows owned here has landed
+            constexpr int NT = 192;
+            if constexpr (EPI == EPI_SWIGLU) {
+                const int fs = 64 / S, lg_fs = lg_rs - 1;
+                for (int e = threadIdx.x; e < fs * BN; e += NT) {
+                    const int fl = e & (fs - 1), col = e >> lg_fs;
+                    float g = 0.f, u = 0.f;
+                    for (int rr = 0; rr < S; ++rr) {
+                        g += recv[(rr * rs + fl) * LD + col];
+                        u += recv[(rr * rs + fs + fl) * LD + col];
+                    }
+                    const int ft = r * fs + fl, grow = (ft >> 4) * 32 + (ft & 15);
+                    const int br = b_tile * BN + col;
+                    if (a_tile * BM + grow < rowsA && br < rowsB)
+                        ep.act[(long long)br * ep.ld_act + a_tile * 64 + ft] = __float2bfloat16_rn(silu_f(g) * u);
+                }
+            } else {
+                // consecutive threads take consecutive rows of one output column (coalesced);
+                // eight elements per thread at a time so that the residual loads overlap
+                const int total = rs * BN;
+                for (int base = threadIdx.x; base < total; base += 8 * NT) {
+                    float acc[8], old[8];
+                    long long off[8];
+                    bool ok[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int e = base + i * NT;
+                        const int lrow = e & (rs - 1), col = e >> lg_rs;
+                        const int ar = a_tile * BM + r * rs + lrow, br = b_tile * BN + col;
+                        ok[i] = e < total && ar < rowsA && br < rowsB;
+                        off[i] = (long long)br * ep.ldo + ar;
+                        float a = 0.f;
+                        if (e < total)
+                            for (int rr = 0; rr < S; ++rr) a += recv[(rr * rs + lrow) * LD + col];
+                        acc[i] = a;
+                        old[i] = 0.f;
+                    }
+                    if constexpr (EPI == EPI_ADD) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            if (ok[i]) old[i] = ep.out[off[i]];
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        if (ok[i]) ep.out[off[i]] = old[i] + acc[i];
+                }
+            }
         }
     }
     tc_fence_before();

@@ -185,7 +185,8 @@ ALODLM_API int alodlm_set_graphs(alodlm_t *h, int on);
  * "readout_combine", "norm", "qkv_rope", "commit", "other". */
 ALODLM_API const char *alodlm_kernel_class_name(int k);
 
-/* Plain bf16 GEMM through the library's tcgen05 kernel: C[m, n] = sum_k A[m, k] * W[n, k],
+/* Plain bf16 GEMM through the library's tcgen05 kernels (the ones the step's linear layers use,
+ * with W in plain row-major layout): C[m, n] = sum_k A[m, k] * W[n, k],
  * A device bf16 [M, K], W device bf16 [N, K] (both row-major, K-major), C device float32
  * [M, N].  K a multiple of 8 (16-byte rows for TMA), M, N >= 1, all pointers 16-byte aligned.
  * workspace: caller-owned device scratch of workspace_bytes >= 256 bytes, zeroed by the caller
