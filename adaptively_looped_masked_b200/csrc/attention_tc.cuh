@@ -15,9 +15,10 @@
 //               tile in the MMA's 128-byte-swizzled K-major layout (the exponentials of tile i
 //               overlap PV_{i-1}); at the end O / l to global memory
 //
-// With n_splits > 1 the keys are split across the CTAs of a cluster; each parks (O, reference
-// max, l) in its shared memory and the cluster merges them in rank order through distributed
-// shared memory.
+// With n_splits > 1 the keys are split across the S CTAs of a cluster.  CTA r owns 128/S
+// query rows of the tile: once every CTA of the cluster is done with its K/V ring, each CTA
+// stores its partial (O row, reference max, l) of every row straight into the owner's ring
+// (remote stores), one cluster barrier, and each owner merges the S partials in rank order.
 #pragma once
 #include <cooperative_groups.h>
 
@@ -142,6 +143,8 @@ __global__ void __launch_bounds__(192, 1)
     pdl_wait();
     pdl_trigger();
     const int b = p.seq_of[j];
+    float m_ref = -INFINITY, l = 0.f;  // softmax thread: running reference max and sum
+    bool have_partial = false;         // split partial ready in TMEM
 
     if (warp == 0) {
         if (lane == 0 && n_tiles > 0) {
@@ -218,7 +221,6 @@ __global__ void __launch_bounds__(192, 1)
         const int q = warp & 3;
         const int t = q * 32 + lane;  // TMEM lane = row of the tile
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        float m_ref = -INFINITY, l = 0.f;
         bool ok = n_tiles > 0;
         for (int i = 0; i < n_tiles && ok; ++i) {
             const int s = i & 1;
@@ -228,12 +230,16 @@ __global__ void __launch_bounds__(192, 1)
             }
             tc_fence_after();
             float sv[BKV];
+            {
+                uint32_t r[BKV];
 #pragma unroll
-            for (int c0 = 0; c0 < BKV; c0 += 16) {
-                float v[16];
-                tmem_ld16(tmem + lane_base + s * BKV + c0, v);
+                for (int c0 = 0; c0 < BKV; c0 += 16) tmem_ld16_async(tmem + lane_base + s * BKV + c0, &r[c0]);
+                tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) sv[c0 + e] = v[e];
+                for (int c = 0; c < BKV; ++c) {
+                    reg_after_wait(r[c]);
+                    sv[c] = __uint_as_float(r[c]);
+                }
             }
             const int key0 = kstart + i * BKV;
             float mt = -INFINITY;
@@ -321,81 +327,96 @@ __global__ void __launch_bounds__(192, 1)
                     }
                 }
             } else {
-                // split partial: O row (unnormalised) and (reference max, l) into our shared
-                // memory (the K/V ring is idle now) for the cluster merge below
-                float *po = reinterpret_cast<float *>(sK) + t * (HD + 1);
-#pragma unroll 1
-                for (int c0 = 0; c0 < HD; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tmem + lane_base + O_COL + c0, v);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) po[c0 + e] = v[e];
-                }
-                float *pml = reinterpret_cast<float *>(sP) + 2 * t;
-                pml[0] = m_ref;
-                pml[1] = l;
+                have_partial = true;  // pushed to the row's owner below
             }
-        } else if (p.n_splits > 1) {
-            // no keys in this split (or a failed wait): an empty partial
-            float *po = reinterpret_cast<float *>(sK) + t * (HD + 1);
-            for (int d = 0; d < HD; ++d) po[d] = 0.f;
-            float *pml = reinterpret_cast<float *>(sP) + 2 * t;
-            pml[0] = -1e30f;
-            pml[1] = 0.f;
         }
         tc_fence_before();
     }
+    if (p.n_splits > 1) {
+        // The splits of this (sequence, kv head, query tile) form one cluster (rank = split).
+        // Phase 0: every CTA is done with its K/V ring and P tiles (a softmax thread gets here
+        // after the last PV product completed, or with no keys at all), which become receive
+        // buffers: [source rank][owned row][HD + 4] f32 partial O rows in the K/V ring (66 KB) and
+        // (reference max, l) pairs in the P tiles.
+        const int S = p.n_splits, rs = BQ / S;
+        float *recv_o = reinterpret_cast<float *>(sK);
+        float *recv_ml = reinterpret_cast<float *>(sP);
+        constexpr int LDO = HD + 4;
+        cluster_arrive_relaxed();
+        cluster_wait_acquire();
+        if (warp >= 2) {
+            const int t = (warp & 3) * 32 + lane;
+            const uint32_t owner = (uint32_t)(t / rs);
+            const int slot = split * rs + t % rs;
+            const uint32_t dst_ml = cluster_map(smem_u32(recv_ml + 2 * slot), owner);
+            st_cluster_v2(dst_ml, have_partial ? m_ref : -1e30f, have_partial ? l : 0.f);
+            if (have_partial) {
+                const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+                const uint32_t dst = cluster_map(smem_u32(recv_o + (size_t)slot * LDO), owner);
+#pragma unroll 1
+                for (int c0 = 0; c0 < HD; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld16_async(tmem + lane_base + O_COL + c0, &r[0]);
+                    tmem_ld16_async(tmem + lane_base + O_COL + c0 + 16, &r[16]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) reg_after_wait(r[e]);
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        st_cluster_v4(dst + (uint32_t)(c0 + e) * 4u, __uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                                      __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+                }
+            }
+        }
+        cluster_arrive_release();
+        cluster_wait_acquire();  // every partial of the rows owned here has landed
+        // merge, in rank order: O = sum_r 2^(m_r - M) O_r / sum_r 2^(m_r - M) l_r over the ranks
+        // that saw keys (l_r > 0); thread = (owned row, 8 columns)
+        constexpr int CH = HD / 8;
+        for (int e = threadIdx.x; e < rs * CH; e += blockDim.x) {
+            const int lr = e / CH, c8 = (e % CH) * 8;
+            const int rp = qtile * BQ + split * rs + lr;
+            if (rp >= p.RP) continue;
+            float M = -INFINITY;
+            for (int rr = 0; rr < S; ++rr) {
+                const float *ml = recv_ml + 2 * (rr * rs + lr);
+                if (ml[1] > 0.f) M = fmaxf(M, ml[0]);
+            }
+            float L = 0.f, acc[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+            for (int rr = 0; rr < S; ++rr) {
+                const float *ml = recv_ml + 2 * (rr * rs + lr);
+                if (!(ml[1] > 0.f)) continue;
+                const float w = exp2f(ml[0] - M);
+                L += w * ml[1];
+                const float4 *o = reinterpret_cast<const float4 *>(recv_o + (size_t)(rr * rs + lr) * LDO + c8);
+                const float4 a0 = o[0], a1 = o[1];
+                acc[0] += w * a0.x;
+                acc[1] += w * a0.y;
+                acc[2] += w * a0.z;
+                acc[3] += w * a0.w;
+                acc[4] += w * a1.x;
+                acc[5] += w * a1.y;
+                acc[6] += w * a1.z;
+                acc[7] += w * a1.w;
+            }
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            const int tt = rp / p.G, h = kvh * p.G + rp % p.G;
+            uint4 pk;
+            pk.x = pack2_bf16(acc[0] * inv, acc[1] * inv);
+            pk.y = pack2_bf16(acc[2] * inv, acc[3] * inv);
+            pk.z = pack2_bf16(acc[4] * inv, acc[5] * inv);
+            pk.w = pack2_bf16(acc[6] * inv, acc[7] * inv);
+            *reinterpret_cast<uint4 *>(p.out + (long long)(j * p.Tq + tt) * p.out_ld + h * HD + c8) = pk;
+        }
+    }
+    tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
-    if (p.n_splits == 1) return;
-
-    // The splits of this (sequence, kv head, query tile) form one cluster (rank = split).  CTA r
-    // merges its share of the rows from every rank's partial, in rank order:
-    // O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    const int S = p.n_splits;
-    auto po = [&](int rr) -> const float * { return cluster.map_shared_rank(reinterpret_cast<float *>(sK), rr); };
-    auto pml = [&](int rr) -> const float * { return cluster.map_shared_rank(reinterpret_cast<float *>(sP), rr); };
-    const int rs = BQ / S;
-    for (int e = threadIdx.x; e < rs * (HD / 2); e += blockDim.x) {
-        const int tl = split * rs + e / (HD / 2), d = (e % (HD / 2)) * 2;
-        const int rp = qtile * BQ + tl;
-        if (rp >= p.RP) continue;
-        // every rank's values first (independent remote loads), then the merge in rank order
-        float mr[8], lr[8], o0[8], o1[8];
-#pragma unroll
-        for (int rr = 0; rr < 8; ++rr) {
-            const int src = rr < S ? rr : 0;
-            const float *ml = pml(src), *o = po(src);
-            mr[rr] = ml[2 * tl];
-            lr[rr] = ml[2 * tl + 1];
-            o0[rr] = o[tl * (HD + 1) + d];
-            o1[rr] = o[tl * (HD + 1) + d + 1];
-        }
-        float M = -INFINITY;
-#pragma unroll
-        for (int rr = 0; rr < 8; ++rr)
-            if (rr < S) M = fmaxf(M, mr[rr]);
-        float L = 0.f, a0 = 0.f, a1 = 0.f;
-#pragma unroll
-        for (int rr = 0; rr < 8; ++rr) {
-            if (rr < S) {
-                const float w = exp2f(mr[rr] - M);
-                L += w * lr[rr];
-                a0 += w * o0[rr];
-                a1 += w * o1[rr];
-            }
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        const int tt = rp / p.G, h = kvh * p.G + rp % p.G;
-        bf16 *dst = p.out + (long long)(j * p.Tq + tt) * p.out_ld + h * HD + d;
-        *reinterpret_cast<__nv_bfloat162 *>(dst) = __floats2bfloat162_rn(a0 * inv, a1 * inv);
-    }
-    cluster.sync();  // no CTA leaves while its partial may still be read
 }
 
 }  // namespace attn_tc
