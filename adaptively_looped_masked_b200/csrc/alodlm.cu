@@ -28,6 +28,9 @@ namespace {
 // the weights faster than the stream-K kernel at 32-64 rows (0.77 vs 0.65 of the measured
 // HBM bandwidth on the 24576 x 4096 gate/up shape).  The GEMM entry points use stream-K for
 // up to 64 rows.
+#ifndef ALODLM_PERSIST_STREAM_K
+#define ALODLM_PERSIST_STREAM_K 1
+#endif
 #ifndef ALODLM_MAX_SPLITS
 #define ALODLM_MAX_SPLITS 8
 #endif
@@ -136,7 +139,7 @@ void set_gemm_attr() {
 template <int BN, int EPI>
 void set_persist_attr() {
     cudaFuncSetAttribute(gemm::gemm_persist_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)gemm::Cfg<BN>::SMEM);
+                         (int)gemm::Cfg<BN>::SMEM_PERSIST);
 }
 template <int BN, int EPI>
 void set_sk_attr() {
@@ -228,15 +231,31 @@ void launch_gemm_bn(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int
                 (const int *)nullptr, k_tiles, kps, a_fastest, tiled, ep, err);
 }
 
-// persistent kernel: one CTA per SM at most, walking the tiles
+// Stream-K (for the last wave and a half of tiles) pays when the tiles leave the last wave of a
+// one-CTA-per-SM grid well short of full: measured on B200 it wins at 1.3 waves (65% of the
+// last round busy) and loses its partial-tile traffic at 1.73 and 2.59 waves (87%).  It needs
+// at least one tile per CTA (a tile is then cut at most once), and the weight tiles of that
+// region plus the whole activation operand should stay in L2 while every CTA works on them.
+bool want_stream_k(int tiles, int grid, int n_b, int rowsB, int K) {
+    if (tiles < grid || tiles % grid == 0) return false;
+    const double waves = (double)tiles / grid;
+    if (waves / std::ceil(waves) >= 0.8) return false;
+    const int region = tiles - (tiles / grid - 1) * grid;
+    const double bytes = ((double)region / n_b + 1.0) * gemm::BM * K * 2.0 + (double)rowsB * K * 2.0;
+    return bytes <= 64.0e6;
+}
+
+// persistent kernel: one CTA per SM at most, walking the tiles (stream-K when `sk` and the
+// tile count fits the rule above; ep.ws / ep.counters then hold grid partial tiles / flags)
 template <int BN, int EPI>
 void launch_persist(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int rowsB, const int *rowsA_dyn,
                     int k_tiles, int a_fastest, const gemm::EpiParams &ep, int *err, cudaStream_t st, int num_sms,
-                    int tiled) {
+                    int tiled, bool sk = false) {
     const int tiles = cdiv(rowsA, gemm::BM) * cdiv(rowsB, BN);
     const int grid = std::max(1, std::min(num_sms, tiles));
-    klaunch(gemm::gemm_persist_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM, st, tA, tB, rowsA, rowsB, rowsA_dyn,
-            k_tiles, a_fastest, tiled, ep, err);
+    const int use_sk = sk && !rowsA_dyn && want_stream_k(tiles, grid, cdiv(rowsB, BN), rowsB, k_tiles * gemm::BK) ? 1 : 0;
+    klaunch(gemm::gemm_persist_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM_PERSIST, st, tA, tB, rowsA, rowsB, rowsA_dyn,
+            k_tiles, a_fastest, tiled, use_sk, ep, err);
 }
 
 template <int EPI>
@@ -335,22 +354,27 @@ int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_b
     const CUtensorMap *tB = map_for_bn(g.bn);
     if (!tB) return -1;
     if (g.splits == 1 && g.bn >= 128) {
+        // stream-K partials: one BM x BN tile and one flag per CTA
+        ep.ws = env.ws;
+        ep.counters = env.counters;
+        const bool sk = ALODLM_PERSIST_STREAM_K && env.ws && env.counters && env.n_counters >= env.num_sms &&
+                        env.ws_floats >= (size_t)env.num_sms * gemm::BM * g.bn;
         if (g.bn == 128) {
             if (epi == gemm::EPI_F32)
-                launch_persist<128, gemm::EPI_F32>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled);
+                launch_persist<128, gemm::EPI_F32>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled, sk);
             else if (epi == gemm::EPI_ADD)
-                launch_persist<128, gemm::EPI_ADD>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled);
+                launch_persist<128, gemm::EPI_ADD>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled, sk);
             else
                 launch_persist<128, gemm::EPI_SWIGLU>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st,
-                                                      env.num_sms, w_tiled);
+                                                      env.num_sms, w_tiled, sk);
         } else {
             if (epi == gemm::EPI_F32)
-                launch_persist<256, gemm::EPI_F32>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled);
+                launch_persist<256, gemm::EPI_F32>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled, sk);
             else if (epi == gemm::EPI_ADD)
-                launch_persist<256, gemm::EPI_ADD>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled);
+                launch_persist<256, gemm::EPI_ADD>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled, sk);
             else
                 launch_persist<256, gemm::EPI_SWIGLU>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st,
-                                                      env.num_sms, w_tiled);
+                                                      env.num_sms, w_tiled, sk);
         }
         return 1;
     }
@@ -1274,7 +1298,7 @@ int alodlm_gemm_bf16(const void *A, const void *W, float *C, int M, int N, int K
     // workspace: [status word | 63 spare floats | tile counters | partials]
     const size_t total_floats = workspace_bytes / sizeof(float);
     const int n_tiles = cdiv(N, gemm::BM);
-    const size_t counter_floats = (size_t)cdiv(n_tiles, 64) * 64;
+    const size_t counter_floats = (size_t)cdiv(std::max(n_tiles, sms), 64) * 64;
     GemmEnv env{};
     env.err = reinterpret_cast<int *>(workspace);
     env.st = static_cast<cudaStream_t>(stream);

@@ -242,22 +242,35 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             const int key0 = kstart + i * BKV;
-            float mt = -INFINITY;
+            if (key0 + BKV > kend) {  // ragged last tile (uniform across the CTA)
 #pragma unroll
-            for (int c = 0; c < BKV; ++c) {
-                sv[c] = (key0 + c < kend) ? sv[c] * p.scale_log2 : -INFINITY;
-                mt = fmaxf(mt, sv[c]);
+                for (int c = 0; c < BKV; ++c)
+                    if (key0 + c >= kend) sv[c] = -INFINITY;
             }
+            // row max of the raw scores (the scale is positive), as eight independent chains
+            float mx[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) mx[c] = sv[c];
+#pragma unroll
+            for (int c = 8; c < BKV; ++c) mx[c & 7] = fmaxf(mx[c & 7], sv[c]);
+            const float mt =
+                fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                p.scale_log2;
             // the reference max moves only when this tile's max passes it by more than 2^8
             const bool resc = mt > m_ref + RESCALE_THRESHOLD;
             const float f = (resc && i > 0) ? exp2f(m_ref - mt) : 1.f;
             if (resc) m_ref = mt;
-            float lt = 0.f;
+            // p = 2^(s * scale - m_ref), summed as eight independent chains
+            const float neg_m = -m_ref;
+            float sm[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) sm[c] = 0.f;
 #pragma unroll
             for (int c = 0; c < BKV; ++c) {
-                sv[c] = exp2f(sv[c] - m_ref);
-                lt += sv[c];
+                sv[c] = ex2_approx(fmaf(sv[c], p.scale_log2, neg_m));
+                sm[c & 7] += sv[c];
             }
+            const float lt = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
             l = l * f + lt;
             // P buffer i & 1 was last read by PV_{i-2}; a rescale of O needs PV_{i-1} complete
             if (i >= 2 && !mbar_wait(pv_done + (i & 1), ((uint32_t)((i - 2) >> 1)) & 1u, p.err)) {

@@ -51,6 +51,13 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, f
                  : "memory");
 }
 
+// 2^x by the PTX ex2.approx instruction (one special-function-unit op; 2^-inf = 0)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -113,12 +120,60 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
     }
 }
 
+// Flag handshake between CTAs of one kernel (global memory, GPU scope).
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(int *p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Wait until *flag == 1 (set by another resident CTA of the same kernel); false, with
+// DEVERR_TIMEOUT raised in *err, if that takes longer than WAIT_LIMIT_NS.
+__device__ __forceinline__ bool flag_wait(const int *flag, int *err) {
+    if (ld_acquire_gpu(flag) == 1) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (ld_acquire_gpu(flag) == 1) return true;
+        if ((it & 63u) == 0 && globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+            atomicOr(err, DEVERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+// named barrier of the 128 epilogue threads (warps 2-5) of a GEMM CTA
+__device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// the same barrier, returning whether `p` holds in every one of the 128 threads
+__device__ __forceinline__ bool epilogue_all(bool p) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
+        : "=r"(r)
+        : "r"((uint32_t)p)
+        : "memory");
+    return r != 0;
+}
+
 // ---------------------------------------------------------------------------------
 // TMA (tiled, 2D, no multicast)
 // ---------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
+
+// Untiled bulk copy global -> this CTA's shared memory, completing on `bar` (no multicast):
+// both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+// orders this thread's view of global memory (generic proxy) before its later async-proxy
+// (bulk copy) reads
+__device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
 
 // x = innermost (element) coordinate, y = row; x * sizeof(elem) must be a multiple of 16.
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {

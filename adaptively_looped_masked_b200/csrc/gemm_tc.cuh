@@ -64,6 +64,18 @@ __device__ __forceinline__ void store_chunk(const float (&v)[16], float *__restr
     }
 }
 
+// EPI_ADD over NC consecutive output columns (rows of p, `ld` floats apart; the first n_rows
+// exist): every old value is loaded before any store, so all NC loads are in flight together.
+template <int NC>
+__device__ __forceinline__ void add_cols(const float (&v)[NC], float *__restrict__ p, int ld, int n_rows) {
+    float old[NC];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) old[j] = (j < n_rows) ? p[(long long)j * ld] : 0.f;
+#pragma unroll
+    for (int j = 0; j < NC; ++j)
+        if (j < n_rows) p[(long long)j * ld] = old[j] + v[j];
+}
+
 // Operand layouts in global memory.  Plain: row-major [rows, K] (TMA box at x = k, y = row).
 // Tiled (the library's own weights): every [tile_rows x 64] tile of the matrix stored
 // contiguously, tiles ordered (row tile, k tile), k padded with zeros to a multiple of 64 --
@@ -131,6 +143,10 @@ struct Cfg {
     static constexpr int RECV_LD = BN + 4;  // floats per received row (16-byte aligned rows)
     static constexpr size_t RECV_BYTES = (size_t)BM * RECV_LD * 4;
     static constexpr size_t SMEM_SPLIT = SMEM + (RECV_SEPARATE ? RECV_BYTES : 0);
+    // persistent kernel: behind the barriers, a [64 columns][128 rows] f32 staging tile through
+    // which the epilogue turns its per-row registers into row-contiguous vector stores
+    static constexpr size_t STG_BYTES = 64 * BM * 4;
+    static constexpr size_t SMEM_PERSIST = SMEM + STG_BYTES;
     static_assert(RECV_SEPARATE || RECV_BYTES <= (size_t)STAGES * STAGE_BYTES, "split-K partials must fit the ring");
 };
 
@@ -706,10 +722,140 @@ __device__ __forceinline__ void readout_tile(uint32_t taddr, int a_row, int b0, 
         ep.partials[(long long)a_row * ep.n_btiles + b_tile] = make_float4(best, se, sed, __int_as_float(best_idx));
 }
 
+// Epilogue of 64 accumulator columns [c0, c0 + 64) of a 128-row tile, by the 128 epilogue
+// threads (thread = tile row `row`, v = its 64 values).  The values go through the staging tile
+// stg[col][row] so that each warp then writes whole output rows: for the f32 / residual-add
+// epilogues 128 consecutive features of one activation row as one 512-byte float4 store per
+// warp, for SwiGLU the tile's 64 features (gate rows (f/16)*32 + f%16, up rows 16 further) of
+// one activation row as bf16 pairs.  Falls back to per-element stores where a row is ragged or
+// not 16-byte aligned.  Every epilogue thread must call it (named barriers).
+template <int EPI>
+__device__ __forceinline__ void staged_cols(float *stg, const float (&v)[64], int row, int a, int b_first,
+                                            int rowsA, int rowsB, const EpiParams &ep) {
+    constexpr int LD = BM;  // floats per staged column
+#pragma unroll
+    for (int j = 0; j < 64; ++j) stg[j * LD + row] = v[j];
+    epilogue_bar();
+    const int w = (threadIdx.x >> 5) & 3, lane = threadIdx.x & 31;
+    if constexpr (EPI == EPI_SWIGLU) {
+        const int f = 2 * lane;                       // features f, f + 1 of the tile
+        const int g = (f >> 4) * 32 + (f & 15);       // their gate rows (adjacent)
+        const bool fits = a * BM + g + 17 < rowsA + 1 && (ep.ld_act % 2) == 0;
+#pragma unroll 4
+        for (int j = w; j < 64; j += 4) {
+            const int br = b_first + j;
+            if (br >= rowsB) break;
+            const float2 gt = *reinterpret_cast<const float2 *>(stg + j * LD + g);
+            const float2 up = *reinterpret_cast<const float2 *>(stg + j * LD + g + 16);
+            bf16 *dst = ep.act + (long long)br * ep.ld_act + a * 64 + f;
+            if (fits) {
+                *reinterpret_cast<__nv_bfloat162 *>(dst) = __floats2bfloat162_rn(silu_f(gt.x) * up.x, silu_f(gt.y) * up.y);
+            } else {
+                if (a * BM + g < rowsA) dst[0] = __float2bfloat16_rn(silu_f(gt.x) * up.x);
+                if (a * BM + g + 1 < rowsA) dst[1] = __float2bfloat16_rn(silu_f(gt.y) * up.y);
+            }
+        }
+    } else {
+        const int r0 = 4 * lane;                      // tile rows r0 .. r0 + 3
+        const bool vec = a * BM + BM <= rowsA && (ep.ldo % 4) == 0;
+        constexpr int PER = 16;                       // output rows per warp per call
+        float4 val[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) val[i] = *reinterpret_cast<const float4 *>(stg + (w + 4 * i) * LD + r0);
+        if (vec) {
+            float4 old[PER];
+            if constexpr (EPI == EPI_ADD) {
+#pragma unroll
+                for (int i = 0; i < PER; ++i) {
+                    const int br = b_first + w + 4 * i;
+                    old[i] = br < rowsB ? *reinterpret_cast<const float4 *>(ep.out + (long long)br * ep.ldo + a * BM + r0)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int br = b_first + w + 4 * i;
+                if (br >= rowsB) continue;
+                float4 x = val[i];
+                if constexpr (EPI == EPI_ADD) {
+                    x.x += old[i].x;
+                    x.y += old[i].y;
+                    x.z += old[i].z;
+                    x.w += old[i].w;
+                }
+                *reinterpret_cast<float4 *>(ep.out + (long long)br * ep.ldo + a * BM + r0) = x;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int br = b_first + w + 4 * i;
+                if (br >= rowsB) continue;
+                float *dst = ep.out + (long long)br * ep.ldo + a * BM + r0;
+                const float xs[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (a * BM + r0 + e < rowsA) {
+                        if constexpr (EPI == EPI_ADD)
+                            dst[e] += xs[e];
+                        else
+                            dst[e] = xs[e];
+                    }
+                }
+            }
+        }
+    }
+    epilogue_bar();  // the staging tile is free again
+}
+
+// One CTA's share of the work: segments (tile t, k-tiles [kb, ke)).  Plain persistent
+// schedule: whole tiles blockIdx.x, blockIdx.x + gridDim.x, ...  With stream-K (sk) only the
+// first W-1 of the W = total / gridDim.x full waves go that way; the remaining tiles (one full
+// wave plus the ragged rest, so at least one tile per CTA) have their k-iterations laid end to
+// end and cut into gridDim.x equal contiguous ranges.  Every CTA then streams the same number
+// of k-tiles, the tiles in flight at any time stay neighbours (their weight tiles are shared
+// through L2), and a tile is cut at most once: into a head [0, k) that ends one CTA's range
+// and a tail [k, K) that starts the next CTA's range.
+struct SegIter {
+    long long u = 0, u1 = 0;
+    int tnext, n_plain, k_tiles;
+    __device__ SegIter(bool sk, int total, int k_tiles_) : k_tiles(k_tiles_) {
+        tnext = blockIdx.x;
+        n_plain = total;
+        if (sk) {
+            n_plain = (total / (int)gridDim.x - 1) * (int)gridDim.x;
+            const long long U = (long long)(total - n_plain) * k_tiles_;
+            u = U * blockIdx.x / gridDim.x;
+            u1 = U * (blockIdx.x + 1) / gridDim.x;
+        }
+    }
+    __device__ bool next(int &t, int &kb, int &ke) {
+        if (tnext < n_plain) {
+            t = tnext;
+            kb = 0;
+            ke = k_tiles;
+            tnext += gridDim.x;
+            return true;
+        }
+        if (u >= u1) return false;
+        const int r = (int)(u / k_tiles);
+        t = n_plain + r;
+        kb = (int)(u - (long long)r * k_tiles);
+        ke = (int)min((long long)k_tiles, kb + (u1 - u));
+        u += ke - kb;
+        return true;
+    }
+};
+
+// Persistent kernel: at most one CTA per SM walks its segments with a double-buffered TMEM
+// accumulator, so the epilogue of one segment overlaps the MMAs of the next.  Under stream-K a
+// tail segment parks its partial tile in ep.ws (slot = this CTA, column-major) and raises
+// ep.counters[this CTA]; the CTA that ends with the head of the same tile (the previous CTA)
+// waits for the flag, adds head + tail in that order (deterministic), applies the epilogue and
+// lowers the flag again.  The grid never exceeds the SM count, so the CTAs are co-resident.
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     gemm_persist_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int rowsA,
-                        int rowsB, const int *rowsA_dyn, int k_tiles, int a_fastest, int tiled, EpiParams ep,
+                        int rowsB, const int *rowsA_dyn, int k_tiles, int a_fastest, int tiled, int sk, EpiParams ep,
                         int *err) {
     using C = Cfg<BN>;
     constexpr int STAGES = C::STAGES;
@@ -720,7 +866,9 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t *empty = full + STAGES;
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    uint64_t *staged_bar = tempty + 2;  // stream-K head: the next CTA's partial has landed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(staged_bar + 1);
+    float *stg = reinterpret_cast<float *>(smem + STAGES * C::STAGE_BYTES + 256);  // epilogue staging
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -732,6 +880,7 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(tfull + b, 1);
             mbar_init(tempty + b, 4);
         }
+        mbar_init(staged_bar, 1);
         fence_mbarrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
@@ -751,6 +900,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     const int n_a = (rowsA + BM - 1) / BM, n_b = (rowsB + BN - 1) / BN;
     const int total = n_a * n_b;
+    const bool use_sk = sk && !rowsA_dyn && EPI != EPI_READOUT && total >= (int)gridDim.x;
     auto tile_of = [&](int t, int &a, int &b) {
         if (a_fastest) {
             a = t % n_a;
@@ -762,24 +912,29 @@ __global__ void __launch_bounds__(192, 1)
     };
 
     if (warp == 0) {
-        if (lane == 0 && blockIdx.x < total) {
-            int a, b;
-            tile_of(blockIdx.x, a, b);
+        if (lane == 0) {
+            SegIter it(use_sk, total, k_tiles);
+            int t, kb, ke, a, b;
+            bool have = it.next(t, kb, ke);
             // weights (operand A of the linear layers) do not depend on earlier kernels: the
-            // first stages of the first tile are requested before waiting for them
-            const int pre = rowsA_dyn ? 0 : min(k_tiles, STAGES);
-            for (int it = 0; it < pre; ++it) {
-                mbar_arrive_expect_tx(full + it, C::STAGE_BYTES);
-                tma_operand(smem + it * C::STAGE_BYTES, &tmA, full + it, tiled & 1, a, BM, it, k_tiles);
+            // first stages of the first segment are requested before waiting for them
+            int pre = 0;
+            if (have) {
+                tile_of(t, a, b);
+                pre = rowsA_dyn ? 0 : min(ke - kb, STAGES);
+                for (int i = 0; i < pre; ++i) {
+                    mbar_arrive_expect_tx(full + i, C::STAGE_BYTES);
+                    tma_operand(smem + i * C::STAGE_BYTES, &tmA, full + i, tiled & 1, a, BM, kb + i, k_tiles);
+                }
             }
             pdl_wait();
-            for (int it = 0; it < pre; ++it)
-                tma_operand(smem + it * C::STAGE_BYTES + C::A_BYTES, &tmB, full + it, tiled & 2, b, BN, it, k_tiles);
-            int g = 0, issued = 0;
+            for (int i = 0; i < pre; ++i)
+                tma_operand(smem + i * C::STAGE_BYTES + C::A_BYTES, &tmB, full + i, tiled & 2, b, BN, kb + i, k_tiles);
+            int g = 0, issued = pre;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (; have && ok; have = it.next(t, kb, ke)) {
                 tile_of(t, a, b);
-                for (int kt = 0; kt < k_tiles; ++kt, ++g) {
+                for (int kt = kb; kt < ke; ++kt, ++g) {
                     if (g < pre) continue;
                     const int s = g % STAGES;
                     if (!mbar_wait(empty + s, ((uint32_t)(g / STAGES) & 1u) ^ 1u, err)) {
@@ -793,20 +948,20 @@ __global__ void __launch_bounds__(192, 1)
                     issued = g + 1;
                 }
             }
-            issued = max(issued, pre);
-            for (int it = max(0, issued - STAGES); it < issued; ++it)
-                mbar_wait(full + (it % STAGES), (uint32_t)(it / STAGES) & 1u, err);
+            for (int i = max(0, issued - STAGES); i < issued; ++i)
+                mbar_wait(full + (i % STAGES), (uint32_t)(i / STAGES) & 1u, err);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = umma_idesc_bf16(BM, BN);
-            int g = 0, li = 0;
+            SegIter it(use_sk, total, k_tiles);
+            int t, kb, ke, g = 0, li = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++li) {
+            while (ok && it.next(t, kb, ke)) {
                 const int buf = li & 1;
                 if (!mbar_wait(tempty + buf, ((uint32_t)(li >> 1) & 1u) ^ 1u, err)) break;
                 tc_fence_after();
-                for (int kt = 0; kt < k_tiles; ++kt, ++g) {
+                for (int kt = kb; kt < ke; ++kt, ++g) {
                     const int s = g % STAGES;
                     if (!mbar_wait(full + s, (uint32_t)(g / STAGES) & 1u, err)) {
                         ok = false;
@@ -818,41 +973,87 @@ __global__ void __launch_bounds__(192, 1)
                     const uint64_t db = umma_sdesc_sw128(sa + C::A_BYTES);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        umma_f16(tmem_base + buf * BN, da + 2 * k, db + 2 * k, idesc, (kt > 0 || k > 0) ? 1u : 0u);
+                        umma_f16(tmem_base + buf * BN, da + 2 * k, db + 2 * k, idesc, (kt > kb || k > 0) ? 1u : 0u);
                     umma_commit(empty + s);
                 }
                 umma_commit(tfull + buf);
+                ++li;
             }
         }
     } else {
         const int q = warp & 3;
+        const int row = q * 32 + lane;  // row of the tile = TMEM lane
         pdl_wait();
-        int li = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x, ++li) {
+        SegIter it(use_sk, total, k_tiles);
+        float *part = ep.ws + (size_t)blockIdx.x * BM * BN;  // this CTA's tail partial
+        int t, kb, ke, li = 0;
+        while (it.next(t, kb, ke)) {
             int a, b;
             tile_of(t, a, b);
             const int buf = li & 1;
-            const bool ready = mbar_wait(tfull + buf, (uint32_t)(li >> 1) & 1u, err);
+            // one verdict for all epilogue threads (they take named barriers below)
+            const bool ready = epilogue_all(mbar_wait(tfull + buf, (uint32_t)(li >> 1) & 1u, err));
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
-            const int a_row = a * BM + q * 32 + lane;
+            const int a_row = a * BM + row;
             const int b0 = b * BN;
-            if (ready) {
-                if constexpr (EPI == EPI_READOUT) {
-                    readout_tile<BN>(taddr, a_row, b0, b, rowsA, rowsB, ep);
-                } else {
-                    for (int c0 = 0; c0 < BN; c0 += 16) {
-                        if (b0 + c0 >= rowsB) break;  // warp-uniform
-                        float v[16];
-                        tmem_ld16(taddr + c0, v);
-                        linear_chunk<EPI, BN>(c0, v, a_row, lane, b0, rowsA, rowsB, ep);
+            const bool tail = kb > 0, head = kb == 0 && ke < k_tiles;
+            if (tail) {
+                // partial of k-tiles [kb, K): parked column-major (coalesced across lanes)
+                if (ready) {
+                    for (int c0 = 0; c0 < BN; c0 += 64) {
+                        float v[64];
+                        acc_ld<1, BN, 64>(taddr, c0, v);
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) part[(size_t)(c0 + j) * BM + row] = v[j];
+                    }
+                }
+                epilogue_bar();
+                if (threadIdx.x == 64) {
+                    __threadfence();
+                    st_release_gpu(ep.counters + blockIdx.x, 1);
+                }
+            } else {
+                // head: the rest of this tile is the first segment of the next CTA; its partial
+                // is bulk-copied into the stage ring (idle now: the head is this CTA's last
+                // segment and its MMAs are complete)
+                const float *staged = reinterpret_cast<const float *>(smem);
+                if (head) {
+                    if (threadIdx.x == 64) {
+                        flag_wait(ep.counters + blockIdx.x + 1, err);
+                        __threadfence();
+                        ep.counters[blockIdx.x + 1] = 0;
+                        fence_proxy_async_all();
+                        constexpr uint32_t BYTES = BM * BN * 4, PIECE = 32768;
+                        const uint8_t *src = reinterpret_cast<const uint8_t *>(ep.ws + (size_t)(blockIdx.x + 1) * BM * BN);
+                        mbar_arrive_expect_tx(staged_bar, BYTES);
+                        for (uint32_t o = 0; o < BYTES; o += PIECE) bulk_load(smem + o, src + o, PIECE, staged_bar);
+                    }
+                    mbar_wait(staged_bar, 0, err);  // at most one head per CTA: phase 0
+                }
+                if (ready) {
+                    if constexpr (EPI == EPI_READOUT) {
+                        readout_tile<BN>(taddr, a_row, b0, b, rowsA, rowsB, ep);
+                    } else {
+                        // rounds of 64 columns: one TMEM wait, then row-contiguous stores
+                        for (int c0 = 0; c0 < BN; c0 += 64) {
+                            if (b0 + c0 >= rowsB) break;  // uniform across the epilogue warps
+                            float v[64];
+                            acc_ld<1, BN, 64>(taddr, c0, v);
+                            if (head) {
+#pragma unroll
+                                for (int j = 0; j < 64; ++j) v[j] += staged[(size_t)(c0 + j) * BM + row];
+                            }
+                            staged_cols<EPI>(stg, v, row, a, b0 + c0, rowsA, rowsB, ep);
+                        }
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty + buf);
-            if (!ready) break;
+            ++li;
+            if (!ready) break;  // uniform: a stream-K partner waiting on us gives up after its bound
         }
     }
     tc_fence_before();

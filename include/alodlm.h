@@ -193,7 +193,8 @@ ALODLM_API const char *alodlm_kernel_class_name(int k);
  * before its first use (calls leave it ready for the next one).  Its first 4 bytes are the
  * device status word (non-zero after a call means a bounded wait inside the kernel timed out
  * and C is invalid; the caller clears it); then come per-tile counters and split partials.
- * With too little room for the split the heuristic picks, fewer splits are used.  Partial
+ * With too little room for the split the heuristic picks, fewer splits are used (and no
+ * stream-K balancing, which needs one 128 x BN f32 tile per SM).  Partial
  * sums are added in a fixed order, so results are deterministic.  Runs on `stream` of the
  * current device and allocates nothing.  For kernel-level tests and benchmarks.
  * Errors: EINVAL, ECUDA. */
