@@ -14,6 +14,7 @@
 #include <mutex>
 #include <string>
 #include <tuple>
+#include <type_traits>
 #include <vector>
 
 #include "attention.cuh"
@@ -323,11 +324,10 @@ void launch_sk(const SkPlan &p, const CUtensorMap &tW, const CUtensorMap &tB, in
         launch_sk_bn<64, EPI>(p, tW, tB, Nw, M, ep, env);
 }
 
-// out = act[M, K] x W[Nw, K]^T with epilogue `epi`.  Stream-K kernel (few rows, when asked) or
-// one CTA per 128 x BN tile with split-K when the tiles do not fill the SMs; split partials are
-// added in split order by the CTA that completes a tile last.  map_for_bn(bn) returns the activation's
-// tensor map with BN-row boxes.  Returns the number of kernels launched, or -1 (tensor map
-// failure).
+// out = act[M, K] x W[Nw, K]^T with epilogue `epi`.  Stream-K kernel (few rows, when asked);
+// one CTA per 128 x BN tile with split-K inside a cluster when the tiles do not fill the SMs;
+// otherwise the persistent kernel.  map_for_bn(bn) returns the activation's tensor map with
+// BN-row boxes.  Returns the number of kernels launched, or -1 (tensor map failure).
 template <typename MapFn>
 int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_bn, int M, int K, int epi, float *out,
              int ldo, bf16 *act_out, int ld_act, bool stream_k, int w_tiled) {
@@ -359,23 +359,27 @@ int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_b
         ep.counters = env.counters;
         const bool sk = ALODLM_PERSIST_STREAM_K && env.ws && env.counters && env.n_counters >= env.num_sms &&
                         env.ws_floats >= (size_t)env.num_sms * gemm::BM * g.bn;
-        if (g.bn == 128) {
-            if (epi == gemm::EPI_F32)
-                launch_persist<128, gemm::EPI_F32>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled, sk);
-            else if (epi == gemm::EPI_ADD)
-                launch_persist<128, gemm::EPI_ADD>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled, sk);
-            else
-                launch_persist<128, gemm::EPI_SWIGLU>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st,
+        auto go = [&](auto bn_tag) {
+            constexpr int BN = decltype(bn_tag)::value;
+            switch (epi) {
+                case gemm::EPI_F32:
+                    launch_persist<BN, gemm::EPI_F32>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st,
                                                       env.num_sms, w_tiled, sk);
-        } else {
-            if (epi == gemm::EPI_F32)
-                launch_persist<256, gemm::EPI_F32>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled, sk);
-            else if (epi == gemm::EPI_ADD)
-                launch_persist<256, gemm::EPI_ADD>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st, env.num_sms, w_tiled, sk);
-            else
-                launch_persist<256, gemm::EPI_SWIGLU>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st,
+                    break;
+                case gemm::EPI_ADD:
+                    launch_persist<BN, gemm::EPI_ADD>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st,
                                                       env.num_sms, w_tiled, sk);
-        }
+                    break;
+                default:
+                    launch_persist<BN, gemm::EPI_SWIGLU>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st,
+                                                         env.num_sms, w_tiled, sk);
+                    break;
+            }
+        };
+        if (g.bn == 128)
+            go(std::integral_constant<int, 128>{});
+        else
+            go(std::integral_constant<int, 256>{});
         return 1;
     }
     if (epi == gemm::EPI_F32)
@@ -709,20 +713,27 @@ struct Fallback {
     int P, b0, nb, depth, src_slot;
 };
 
+// xn = RMSNorm(x) * g (bf16) over M rows of the hidden size
+int rmsnorm(alodlm *h, const float *x, const float *g, bf16 *xn, int M) {
+    const int H = h->H;
+    LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
+           (klaunch(k::rmsnorm_kernel, M, h->norm_threads, 0, h->stream, x, g, xn, H, h->cfg.rms_eps)));
+    return ALODLM_OK;
+}
+
 // one pre-norm Qwen3 decoder layer over M rows, residual stream `x` updated in place
 int run_layer(alodlm *h, int li, int slot, int M, const RowMap &map, int n_seq, int kv_len, int causal, float *x,
               const Fallback *fb) {
     const LayerDev &Lw = h->layers[li];
     const int H = h->H, qd = h->nq * h->hd;
     int rc;
-    LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
-           (klaunch(k::rmsnorm_kernel, M, h->norm_threads, 0, h->stream, x, Lw.attn_norm, h->xn, H, h->cfg.rms_eps)));
-    if ((rc = linear(h, Lw.tm_qkv, h->n_qkv, h->xn, M, H, gemm::EPI_F32, h->qkv, h->n_qkv, nullptr, 0))) return rc;
+    if ((rc = rmsnorm(h, x, Lw.attn_norm, h->xn, M))) return rc;
     bf16 *kc = h->kv_k + (long long)slot * h->slot_elems, *vc = h->kv_v + (long long)slot * h->slot_elems;
+    if ((rc = linear(h, Lw.tm_qkv, h->n_qkv, h->xn, M, H, gemm::EPI_F32, h->qkv, h->n_qkv, nullptr, 0))) return rc;
     LAUNCH(KC_QKV, 6.0 * M * h->n_qkv, 0.0,
-           (klaunch(k::qkv_post_kernel, dim3(M, cdiv(h->nq + 2 * h->nkv, 8)), 256, 0, h->stream, h->qkv, h->nq, h->nkv, h->hd, Lw.q_norm, Lw.k_norm,
-                                                          h->cfg.qk_norm, h->cfg.rms_eps, h->rope, map, h->qb, kc, vc,
-                                                          h->seq_stride, h->head_stride)));
+           (klaunch(k::qkv_post_kernel, dim3(M, cdiv(h->nq + 2 * h->nkv, 8)), 256, 0, h->stream, h->qkv, h->nq,
+                    h->nkv, h->hd, Lw.q_norm, Lw.k_norm, h->cfg.qk_norm, h->cfg.rms_eps, h->rope, map, h->qb, kc, vc,
+                    h->seq_stride, h->head_stride)));
     if (fb) {
         const long long so = (long long)fb->src_slot * h->slot_elems;
         LAUNCH(KC_OTHER, 8.0 * fb->nb * h->nkv * fb->P * h->hd, 0.0,
@@ -732,8 +743,7 @@ int run_layer(alodlm *h, int li, int slot, int M, const RowMap &map, int n_seq, 
     }
     if ((rc = attention(h, slot, M, map, n_seq, kv_len, causal))) return rc;
     if ((rc = linear(h, Lw.tm_o, H, h->attn_out, M, qd, gemm::EPI_ADD, x, H, nullptr, 0))) return rc;
-    LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
-           (klaunch(k::rmsnorm_kernel, M, h->norm_threads, 0, h->stream, x, Lw.mlp_norm, h->xn, H, h->cfg.rms_eps)));
+    if ((rc = rmsnorm(h, x, Lw.mlp_norm, h->xn, M))) return rc;
     if ((rc = linear(h, Lw.tm_gu, 2 * h->I, h->xn, M, H, gemm::EPI_SWIGLU, nullptr, 0, h->act, h->I))) return rc;
     if ((rc = linear(h, Lw.tm_d, H, h->act, M, h->I, gemm::EPI_ADD, x, H, nullptr, 0))) return rc;
     return ALODLM_OK;
@@ -1151,10 +1161,10 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
             if ((r = run_layer(h, c.n_prelude + c.n_core + j, slot_coda(h, j), Ml, mp, n_act_, P + N, 0, h->hc,
                                nullptr)))
                 return r;
+        float *dbg_r = c.debug_dump ? h->dbg[2] + dbg_off : nullptr;
         LAUNCH(KC_NORM, 4.0 * Ml * H + 2.0 * Ml * H, 0.0,
                (klaunch(k::final_norm_kernel, Ml, 256, 0, h->stream, h->hc, h->final_norm, h->exit_w, h->exit_b, H,
-                                                                c.rms_eps, mp, h->ridx, h->rb, h->lam_rr,
-                                                                c.debug_dump ? h->dbg[2] + dbg_off : nullptr)));
+                        c.rms_eps, mp, h->ridx, h->rb, h->lam_rr, dbg_r)));
         {
             gemm::EpiParams ep{};
             ep.partials = h->part;
