@@ -730,10 +730,18 @@ int run_layer(alodlm *h, int li, int slot, int M, const RowMap &map, int n_seq, 
     if ((rc = rmsnorm(h, x, Lw.attn_norm, h->xn, M))) return rc;
     bf16 *kc = h->kv_k + (long long)slot * h->slot_elems, *vc = h->kv_v + (long long)slot * h->slot_elems;
     if ((rc = linear(h, Lw.tm_qkv, h->n_qkv, h->xn, M, H, gemm::EPI_F32, h->qkv, h->n_qkv, nullptr, 0))) return rc;
-    LAUNCH(KC_QKV, 6.0 * M * h->n_qkv, 0.0,
-           (klaunch(k::qkv_post_kernel, dim3(M, cdiv(h->nq + 2 * h->nkv, 8)), 256, 0, h->stream, h->qkv, h->nq,
-                    h->nkv, h->hd, Lw.q_norm, Lw.k_norm, h->cfg.qk_norm, h->cfg.rms_eps, h->rope, map, h->qb, kc, vc,
-                    h->seq_stride, h->head_stride)));
+    const int n_heads = h->nq + 2 * h->nkv;
+    if (h->hd == 128 && n_heads <= 64) {
+        LAUNCH(KC_QKV, 6.0 * M * h->n_qkv, 0.0,
+               (klaunch(k::qkv_post128_kernel, M, 256, 0, h->stream, h->qkv, h->nq, h->nkv, cdiv(n_heads, 8),
+                        Lw.q_norm, Lw.k_norm, h->cfg.qk_norm, h->cfg.rms_eps, h->rope, map, h->qb, kc, vc,
+                        h->seq_stride, h->head_stride)));
+    } else {
+        LAUNCH(KC_QKV, 6.0 * M * h->n_qkv, 0.0,
+               (klaunch(k::qkv_post_kernel, dim3(M, cdiv(n_heads, 8)), 256, 0, h->stream, h->qkv, h->nq, h->nkv,
+                        h->hd, Lw.q_norm, Lw.k_norm, h->cfg.qk_norm, h->cfg.rms_eps, h->rope, map, h->qb, kc, vc,
+                        h->seq_stride, h->head_stride)));
+    }
     if (fb) {
         const long long so = (long long)fb->src_slot * h->slot_elems;
         LAUNCH(KC_OTHER, 8.0 * fb->nb * h->nkv * fb->P * h->hd, 0.0,

@@ -190,6 +190,69 @@ __global__ void qkv_post_kernel(const float *qkv, int nq, int nkv, int hd, const
     }
 }
 
+// The same for head_dim 128 with one block per row and each warp taking `hpw` (<= 8) heads of
+// it: every head's load and the row's RoPE table entries are issued before any arithmetic, so
+// a warp waits for one memory round trip instead of one per head.
+__global__ void qkv_post128_kernel(const float *qkv, int nq, int nkv, int hpw, const float *qn, const float *kn,
+                                   int qk_norm, float eps, const float2 *rope, RowMap map, bf16 *q_out, bf16 *kc,
+                                   bf16 *vc, long long seq_stride, long long head_stride) {
+    pdl_wait();
+    pdl_trigger();
+    constexpr int HD = 128, MAXH = 8;
+    const int m = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int jj = m / map.rows_per_seq, t = m % map.rows_per_seq;
+    const int pos = map.pos0 + t;
+    const int n_heads = nq + 2 * nkv;
+    const int h0 = warp * hpw, h1 = min(n_heads, h0 + hpw);
+    if (h0 >= h1) return;
+    const float *row = qkv + (long long)m * n_heads * HD;
+    float4 x[MAXH];
+#pragma unroll
+    for (int i = 0; i < MAXH; ++i)
+        if (h0 + i < h1) x[i] = *reinterpret_cast<const float4 *>(row + (h0 + i) * HD + lane * 4);
+    // lane l holds d = 4l .. 4l + 3, RoPE angle index d % 64 (the same for every head)
+    float2 cs[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) cs[e] = rope[(long long)pos * 64 + ((lane * 4 + e) & 63)];
+    const float4 wq = qk_norm ? *reinterpret_cast<const float4 *>(qn + lane * 4) : make_float4(1.f, 1.f, 1.f, 1.f);
+    const float4 wk = qk_norm ? *reinterpret_cast<const float4 *>(kn + lane * 4) : make_float4(1.f, 1.f, 1.f, 1.f);
+    const int b = map.seq_of[jj];
+    const int G = nq / nkv, RP = G * map.rows_per_seq;
+#pragma unroll
+    for (int i = 0; i < MAXH; ++i) {
+        const int hh = h0 + i;
+        if (hh >= h1) break;  // uniform across the warp
+        float v[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+        if (hh < nq + nkv) {
+            if (qk_norm) {
+                const float4 w = hh < nq ? wq : wk;
+                float ss = v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3];
+                ss = warp_sum(ss);
+                const float r = rsqrtf(ss / HD + eps);
+                v[0] = v[0] * r * w.x;
+                v[1] = v[1] * r * w.y;
+                v[2] = v[2] * r * w.z;
+                v[3] = v[3] * r * w.w;
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float other = __shfl_xor_sync(0xffffffffu, v[e], 16);
+                v[e] = (lane < 16) ? (v[e] * cs[e].x - other * cs[e].y) : (v[e] * cs[e].x + other * cs[e].y);
+            }
+        }
+        bf16 *dst;
+        if (hh < nq)
+            dst = q_out + (((long long)jj * nkv + hh / G) * RP + (long long)t * G + hh % G) * HD;
+        else if (hh < nq + nkv)
+            dst = kc + (long long)b * seq_stride + (long long)(hh - nq) * head_stride + (long long)pos * HD;
+        else
+            dst = vc + (long long)b * seq_stride + (long long)(hh - nq - nkv) * head_stride + (long long)pos * HD;
+        __nv_bfloat162 b2[2] = {__floats2bfloat162_rn(v[0], v[1]), __floats2bfloat162_rn(v[2], v[3])};
+        *reinterpret_cast<uint2 *>(dst + lane * 4) = *reinterpret_cast<const uint2 *>(b2);
+    }
+}
+
 // Prefill depth fallback: for prefix positions whose exit depth is below the current depth,
 // the KV at this depth is the KV of the previous depth (which by induction is the KV of
 // their exit depth).  One block per (sequence in group, kv head), threads over positions.
