@@ -43,8 +43,13 @@ def _gemm_ref(A, W):
 
 @pytest.mark.parametrize("M,N,K", [(1, 128, 64), (16, 200, 256), (32, 384, 880), (33, 1376, 256), (100, 512, 320),
                                    (128, 256, 4096), (300, 640, 768), (2048, 512, 1024), (20, 6144, 4096),
-                                   (512, 4096, 1024), (2048, 6144, 4096), (1000, 3000, 880)])
+                                   (512, 4096, 1024), (2048, 6144, 4096), (1000, 3000, 880),
+                                   (832, 6144, 4096), (1536, 4096, 4096)])
 def test_gemm_tcgen05_against_fp64(M, N, K):
+    """The shapes cover every GEMM path: split-K clusters of 2-8 CTAs (few rows), the persistent
+    kernel with 128- and 256-wide tiles, and its stream-K schedule (1000 x 3000 x 880 with ragged
+    edges in M, N and K; 832 x 6144 and 1536 x 4096 at 1.3 waves) -- each with and without the
+    workspace room those need."""
     import adaptively_looped_masked_b200 as alo
     g = torch.Generator(device="cuda").manual_seed(M * 7 + N)
     A = torch.randn((M, K), device="cuda", generator=g).to(torch.bfloat16)
