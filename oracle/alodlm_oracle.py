@@ -553,3 +553,47 @@ class Oracle:
             out["h_in"].append(np.stack(h_ins))
             out["h_tilde"].append(np.stack(h_tildes))
         return out
+
+
+def decode_block(oracle: Oracle, block_ids: np.ndarray, tau: float, lam: float, k_max: int,
+                 rule: int = RULE_PAPER, max_steps: int = 0, follow_steps: Optional[List[dict]] = None,
+                 band: float = 1e-3) -> dict:
+    """Denoising steps over one block until no [MASK] is left, [digest] "Method steps",
+    Algorithm 1 (5): after each step the committed tokens are written into the sequence and
+    the next denoising step starts, until no [MASK] remains.
+
+    Every step sees the same prefix KV (the block is re-embedded from its ids each step); step
+    t + 1 takes the tokens of step t as its block ids.  The whole batch steps together; a
+    sequence without masks still runs a step (its U is empty, so nothing changes), and stops
+    counting steps once its block is complete.  ``max_steps`` (0 = N) bounds the steps.
+    ``follow_steps``: per step, another run's decisions (the ``follow`` argument of
+    ``Oracle.denoise_step``).
+
+    Returns tokens [B,N] (final), commit_step [B,N] (1-based step that committed the
+    position; 0 for given ids and positions never committed), commit_depth [B,N] (the loop s
+    of that step), steps_run [B] (steps that had masks at their start), loops [steps, B]
+    (loops run per step), steps (steps taken), and the per-step outputs ("per_step").
+    """
+    mask_id = oracle.cfg["mask_id"]
+    ids = np.asarray(block_ids).astype(np.int64).copy()
+    B, N = ids.shape
+    limit = max_steps if max_steps > 0 else N
+    commit_step = np.zeros((B, N), np.int64)
+    commit_depth = np.zeros((B, N), np.int64)
+    steps_run = np.zeros(B, np.int64)
+    loops, per_step = [], []
+    t = 0
+    while t < limit and (ids == mask_id).any():
+        t += 1
+        had_masks = (ids == mask_id).any(axis=1)
+        follow = follow_steps[t - 1] if follow_steps is not None and t - 1 < len(follow_steps) else None
+        out = oracle.denoise_step(ids, tau, lam, k_max, rule, follow=follow, band=band)
+        new = out["exit_depth"] > 0
+        commit_step[new] = t
+        commit_depth[new] = out["exit_depth"][new]
+        steps_run[had_masks] = t
+        loops.append(out["loops_run"].copy())
+        per_step.append(out)
+        ids = out["tokens"].astype(np.int64).copy()
+    return dict(tokens=ids, commit_step=commit_step, commit_depth=commit_depth, steps_run=steps_run,
+                loops=np.array(loops, dtype=np.int64).reshape(t, B), steps=t, per_step=per_step)

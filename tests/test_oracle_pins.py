@@ -577,3 +577,61 @@ def test_replay_of_own_traces_reproduces_decisions(rule):
         np.testing.assert_array_equal(rep["exit_depth"], out["exit_depth"])
         np.testing.assert_array_equal(rep["tokens"], out["tokens"])
         np.testing.assert_array_equal(rep["loops_run"], out["loops_run"])
+
+
+# ------------------------------------------------------------------------------------
+# decoding a block until no [MASK] is left (Algorithm 1 step (5))
+# ------------------------------------------------------------------------------------
+
+def _decoder(n_given=0, B=1, N=12, K=3):
+    shape = small_shape()
+    o, _ = build(shape, K)
+    o.prefill(make_prefix_ids(shape, B, 10))
+    return o, shape, make_block_ids(shape, B, N, n_given=n_given)
+
+
+def test_decode_per_token_finishes_in_one_step():
+    """PER_TOKEN commits all of U at s = K: one step decodes the whole block."""
+    o, shape, block = _decoder()
+    out = om.decode_block(o, block, tau=-1.0, lam=2.0, k_max=3, rule=RULE_PER_TOKEN)
+    assert out["steps"] == 1 and (out["tokens"] != shape.mask_id).all()
+    assert (out["commit_step"] == 1).all() and (out["commit_depth"] == 3).all()
+
+
+def test_decode_forced_commits_take_one_position_per_step():
+    """PAPER with nothing below tau and no halting: each step commits exactly the forced
+    position (lowest entropy of loop K), so a block of N masks takes N steps, each at depth K."""
+    o, shape, block = _decoder(N=6)
+    out = om.decode_block(o, block, tau=-1.0, lam=2.0, k_max=3, rule=RULE_PAPER)
+    assert out["steps"] == 6 and (out["tokens"] != shape.mask_id).all()
+    assert sorted(out["commit_step"][0].tolist()) == [1, 2, 3, 4, 5, 6]
+    assert (out["commit_depth"] == 3).all() and (out["loops"] == 3).all()
+    # the position committed at step t is the lowest-entropy one of that step's last loop
+    for t, st in enumerate(out["per_step"], start=1):
+        H = st["entropy"][0, 2]
+        assert out["commit_step"][0, np.nanargmin(H)] == t
+
+
+def test_decode_all_below_tau_is_one_loop():
+    o, shape, block = _decoder()
+    out = om.decode_block(o, block, tau=1e9, lam=0.5, k_max=3, rule=RULE_PAPER)
+    assert out["steps"] == 1 and (out["commit_depth"] == 1).all() and (out["loops"] == 1).all()
+
+
+def test_decode_keeps_given_ids_and_skips_finished_sequences():
+    """Given ids are never in U; a sequence without masks counts no step and is unchanged."""
+    o, shape, block = _decoder(n_given=4, B=2, N=8)
+    block[1] = np.arange(8) % (shape.vocab - 1)  # sequence 1: nothing to decode
+    out = om.decode_block(o, block, tau=-1.0, lam=2.0, k_max=3, rule=RULE_PAPER)
+    given = block != shape.mask_id
+    np.testing.assert_array_equal(out["tokens"][given], block[given])
+    assert (out["commit_step"][given] == 0).all()
+    assert out["steps_run"][1] == 0 and out["steps_run"][0] == 4 == out["steps"]
+    assert (out["tokens"] != shape.mask_id).all()
+
+
+def test_decode_step_bound():
+    o, shape, block = _decoder(N=6)
+    out = om.decode_block(o, block, tau=-1.0, lam=2.0, k_max=3, rule=RULE_PAPER, max_steps=2)
+    assert out["steps"] == 2 and (out["tokens"] == shape.mask_id).sum() == 4
+    assert ((out["commit_step"] > 0) == (out["tokens"] != shape.mask_id)).all()
