@@ -58,6 +58,10 @@ class StepOut(ctypes.Structure):
                                                "active_rows", "readout_rows")]
 
 
+class DecodeOut(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("tokens", "commit_step", "commit_depth", "steps_run", "loops", "rows")]
+
+
 _lib = None
 
 
@@ -72,6 +76,8 @@ def lib() -> ctypes.CDLL:
         L.alodlm_create.argtypes = [ctypes.POINTER(Cfg), ctypes.POINTER(Weights), vp, ctypes.POINTER(vp)]
         L.alodlm_prefill.argtypes = [vp, vp, ci, ci, vp]
         L.alodlm_denoise_step.argtypes = [vp, vp, ci, ci, cf, cf, ci, ci, ctypes.POINTER(StepOut)]
+        L.alodlm_decode_block.argtypes = [vp, vp, ci, ci, cf, cf, ci, ci, ci, ctypes.POINTER(DecodeOut),
+                                          ctypes.POINTER(ci)]
         L.alodlm_sync.argtypes = [vp]
         L.alodlm_destroy.argtypes = [vp]
         L.alodlm_destroy.restype = None
@@ -239,6 +245,27 @@ class Handle:
                                               rule, ctypes.byref(so)), "denoise_step")
         self._order_out()
         self.N = N
+        return out
+
+    def decode_block(self, block_ids: torch.Tensor, tau_H: float, lam: float, k_max: int, rule: int = RULE_PAPER,
+                     max_steps: int = 0) -> dict:
+        """Denoising steps until no [MASK] is left (alodlm_decode_block); max_steps 0 = N.
+        Returns the device outputs (tokens, commit_step, commit_depth, steps_run, loops
+        [S, B], rows [S, 2, K]) and "steps" (host int)."""
+        B, N = block_ids.shape
+        S = max_steps if max_steps > 0 else N
+        i32 = dict(dtype=torch.int32, device="cuda")
+        out = dict(tokens=torch.empty((B, N), **i32), commit_step=torch.empty((B, N), **i32),
+                   commit_depth=torch.empty((B, N), **i32), steps_run=torch.empty((B,), **i32),
+                   loops=torch.empty((S, B), **i32), rows=torch.empty((S, 2, k_max), **i32))
+        do = DecodeOut(**{k: _ptr(v) for k, v in out.items()})
+        steps = ctypes.c_int()
+        self._order_in()
+        self._check(lib().alodlm_decode_block(self._h, _ptr(block_ids), B, N, float(tau_H), float(lam), k_max, rule,
+                                              S, ctypes.byref(do), ctypes.byref(steps)), "decode_block")
+        self._order_out()
+        self.N = N
+        out["steps"] = steps.value
         return out
 
     def sync(self):

@@ -29,8 +29,11 @@ namespace {
 // the weights faster than the stream-K kernel at 32-64 rows (0.77 vs 0.65 of the measured
 // HBM bandwidth on the 24576 x 4096 gate/up shape).  The GEMM entry points use stream-K for
 // up to 64 rows.
+// Stream-K in the persistent GEMM: off by default.  It wins ~1% of the bs32 step (only O/down
+// at 1.3 waves qualify) and lost ~2.5% in block decoding; and it is the one place where a CTA
+// waits on another CTA of its grid, which relies on the whole grid being resident.
 #ifndef ALODLM_PERSIST_STREAM_K
-#define ALODLM_PERSIST_STREAM_K 1
+#define ALODLM_PERSIST_STREAM_K 0
 #endif
 #ifndef ALODLM_MAX_SPLITS
 #define ALODLM_MAX_SPLITS 8
@@ -478,6 +481,12 @@ struct alodlm {
     int *seq_of[2] = {nullptr, nullptr}, *old_slot = nullptr;
     int *counts = nullptr, *counts_host = nullptr, *d_err = nullptr;
 
+    // block decoding: two token buffers (a step's output is the next step's input), the
+    // per-step outputs at fixed addresses (so the loop graphs are reused), the "masks left" flag
+    int *dec_tok[2] = {nullptr, nullptr}, *dec_ex = nullptr, *dec_loops = nullptr, *dec_rows = nullptr;
+    int *dec_left = nullptr, *dec_left_host = nullptr;
+    float *dec_tr = nullptr;
+
     // debug copies [K][maxB][maxN][H]
     float *dbg[4] = {nullptr, nullptr, nullptr, nullptr};
 
@@ -809,6 +818,7 @@ void alodlm_destroy(alodlm_t *h) {
     for (void *p : h->allocs) cudaFree(p);
     for (auto e : h->ev_pool) cudaEventDestroy(e);
     if (h->counts_host) cudaFreeHost(h->counts_host);
+    if (h->dec_left_host) cudaFreeHost(h->dec_left_host);
     delete h;
 }
 
@@ -1001,7 +1011,11 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
         (rc = dalloc(h, &h->ncommit, cfg->max_batch)) || (rc = dalloc(h, &h->seq_of[0], cfg->max_batch)) ||
         (rc = dalloc(h, &h->seq_of[1], cfg->max_batch)) || (rc = dalloc(h, &h->old_slot, cfg->max_batch)) ||
         (rc = dalloc(h, &h->counts, 4)) || (rc = dalloc(h, &h->d_err, 1)) || (rc = dalloc(h, &h->iota, cfg->max_batch)) ||
-        (rc = dalloc(h, &h->exit_dev, (size_t)cfg->max_batch * cfg->max_prefix)))
+        (rc = dalloc(h, &h->exit_dev, (size_t)cfg->max_batch * cfg->max_prefix)) ||
+        (rc = dalloc(h, &h->dec_tok[0], BN_)) || (rc = dalloc(h, &h->dec_tok[1], BN_)) ||
+        (rc = dalloc(h, &h->dec_ex, BN_)) || (rc = dalloc(h, &h->dec_loops, cfg->max_batch)) ||
+        (rc = dalloc(h, &h->dec_rows, 2 * (size_t)cfg->k_max)) || (rc = dalloc(h, &h->dec_left, 1)) ||
+        (rc = dalloc(h, &h->dec_tr, 3 * (size_t)cfg->k_max * BN_)))
         return cleanup(rc);
     {
         std::vector<int> io(cfg->max_batch);
@@ -1013,7 +1027,8 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
         for (int i = 0; i < 4; ++i)
             if ((rc = dalloc(h, &h->dbg[i], (size_t)cfg->k_max * BN_ * H))) return cleanup(rc);
     }
-    if (cudaMallocHost(&h->counts_host, 4 * sizeof(int)) != cudaSuccess) {
+    if (cudaMallocHost(&h->counts_host, 4 * sizeof(int)) != cudaSuccess ||
+        cudaMallocHost(&h->dec_left_host, sizeof(int)) != cudaSuccess) {
         h->err = "cudaMallocHost failed";
         return cleanup(ALODLM_ENOMEM);
     }
@@ -1023,6 +1038,66 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
         return cleanup(ALODLM_ECUDA);
     }
     *out = h;
+    return ALODLM_OK;
+}
+
+int alodlm_decode_block(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda, int k_max,
+                        int rule, int max_steps, const alodlm_decode_out *out, int *steps_taken) {
+    if (steps_taken) *steps_taken = 0;
+    if (!h || !block_ids || !out || !out->tokens || !out->commit_step || !out->commit_depth || !out->steps_run ||
+        !out->loops || !out->rows)
+        return fail(h, ALODLM_EINVAL, "null argument");
+    if (max_steps < 1) return fail(h, ALODLM_EINVAL, "max_steps must be >= 1");
+    if (!h->prefilled) return fail(h, ALODLM_ESTATE, "decode_block before prefill");
+    if (B != h->B) return fail(h, ALODLM_ESTATE, "batch differs from the prefill's");
+    if (N < 1 || N > h->cfg.max_block) return fail(h, ALODLM_EINVAL, "N out of range");
+    if (k_max < 1 || k_max > h->cfg.k_max) return fail(h, ALODLM_EINVAL, "k_max out of range");
+    const long long BN = (long long)B * N;
+    const unsigned grid = (unsigned)std::min<long long>((BN + 255) / 256, 1024);
+    cudaMemsetAsync(out->commit_step, 0, BN * sizeof(int32_t), h->stream);
+    cudaMemsetAsync(out->commit_depth, 0, BN * sizeof(int32_t), h->stream);
+    cudaMemsetAsync(out->steps_run, 0, (size_t)B * sizeof(int32_t), h->stream);
+    cudaMemsetAsync(out->loops, 0, (size_t)max_steps * B * sizeof(int32_t), h->stream);
+    cudaMemsetAsync(out->rows, 0, (size_t)max_steps * 2 * k_max * sizeof(int32_t), h->stream);
+    cudaMemcpyAsync(out->tokens, block_ids, BN * sizeof(int32_t), cudaMemcpyDeviceToDevice, h->stream);
+    // a block without masks takes no step
+    cudaMemsetAsync(h->dec_left, 0, sizeof(int), h->stream);
+    klaunch(k::any_mask_kernel, grid, 256, 0, h->stream, (const int *)block_ids, BN, h->cfg.mask_id, h->dec_left);
+    const size_t KBN = (size_t)k_max * BN;
+    alodlm_step_out so{};
+    so.exit_depth = h->dec_ex;
+    so.entropy = h->dec_tr;
+    so.halt = h->dec_tr + KBN;
+    so.cum_halt = h->dec_tr + 2 * KBN;
+    so.loops_run = h->dec_loops;
+    so.active_rows = h->dec_rows;
+    so.readout_rows = h->dec_rows + k_max;
+    const int32_t *in = block_ids;
+    int t = 0;
+    for (;;) {
+        cudaError_t e = cudaMemcpyAsync(h->dec_left_host, h->dec_left, sizeof(int), cudaMemcpyDeviceToHost, h->stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(h->stream);
+        if (e != cudaSuccess) return cuda_fail(h, e, "decode_block: read the masks-left flag");
+        if (*h->dec_left_host == 0 || t == max_steps) break;
+        ++t;
+        so.tokens = h->dec_tok[t & 1];
+        int rc = alodlm_denoise_step(h, in, B, N, tau_H, lambda, k_max, rule, &so);
+        if (rc) return rc;
+        cudaMemsetAsync(h->dec_left, 0, sizeof(int), h->stream);
+        klaunch(k::decode_update_kernel, grid, 256, 0, h->stream, (const int *)in, (const int *)so.tokens,
+                (const int *)h->dec_ex, t, B, N, h->cfg.mask_id, out->commit_step, out->commit_depth, out->steps_run,
+                h->dec_left);
+        cudaMemcpyAsync(out->loops + (size_t)(t - 1) * B, h->dec_loops, (size_t)B * sizeof(int32_t),
+                        cudaMemcpyDeviceToDevice, h->stream);
+        cudaMemcpyAsync(out->rows + (size_t)(t - 1) * 2 * k_max, h->dec_rows, 2 * (size_t)k_max * sizeof(int32_t),
+                        cudaMemcpyDeviceToDevice, h->stream);
+        in = so.tokens;
+    }
+    if (t > 0)
+        cudaMemcpyAsync(out->tokens, in, BN * sizeof(int32_t), cudaMemcpyDeviceToDevice, h->stream);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(h, e, "decode_block");
+    if (steps_taken) *steps_taken = t;
     return ALODLM_OK;
 }
 

@@ -437,6 +437,36 @@ __global__ void step_init_kernel(const int *block_ids, int B, int N, int Kstep, 
     }
 }
 
+// *left = 1 if any of ids[0, total) is the mask id (*left cleared by the caller)
+__global__ void any_mask_kernel(const int *ids, long long total, int mask_id, int *left) {
+    pdl_wait();
+    pdl_trigger();
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x)
+        if (ids[idx] == mask_id) *left = 1;
+}
+
+// Block decoding, after denoising step t (1-based) of in_ids -> tokens / exit_depth: record the
+// step and depth of this step's commits, count the step for sequences that had masks at its
+// start, and raise *left if any [MASK] remains.
+__global__ void decode_update_kernel(const int *in_ids, const int *tokens, const int *exit_depth, int t, int B,
+                                     int N, int mask_id, int *commit_step, int *commit_depth, int *steps_run,
+                                     int *left) {
+    pdl_wait();
+    pdl_trigger();
+    const long long total = (long long)B * N;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const int d = exit_depth[idx];
+        if (d > 0) {
+            commit_step[idx] = t;
+            commit_depth[idx] = d;
+        }
+        if (in_ids[idx] == mask_id) steps_run[idx / N] = t;  // same value from every writer
+        if (tokens[idx] == mask_id) *left = 1;
+    }
+}
+
 // One block per looping sequence (slot j): commit per rule, halting decision, forced
 // commit, and the Eq. 3 merge of committed rows into the loop state h.
 __global__ void commit_kernel(RowMap map, int s, int Kstep, int rule, float tau, float lam, const bf16 *emb, int H,

@@ -379,6 +379,94 @@ def run_ours(args, world, rank, local):
     handle.close()
 
 
+def run_decode(args, world, rank, local):
+    """Block decoding (alodlm_decode_block): denoising steps over the workload's block until no
+    [MASK] is left.  value = masks decoded per second over whole decodes; the roofline sums
+    the step roofline of every step taken."""
+    import adaptively_looped_masked_b200 as alo
+    wl = WORKLOADS[args.workload]
+    m = MODELS[wl.model]
+    peaks, peaks_src = load_peaks()
+    stream = torch.cuda.Stream()
+    w = make_weights(m, seed=0, device="cuda")
+    handle = alo.Handle(m, w, k_max=wl.k_max, max_batch=wl.batch, max_prefix=wl.prefix, max_block=wl.block,
+                        stream=stream)
+    del w
+    torch.cuda.empty_cache()
+    prefix = torch.tensor(make_prefix_ids(m, wl.batch, wl.prefix, seed=1 + rank), device="cuda")
+    exit_depth = None
+    if wl.mixed_exit_depths:
+        exit_depth = torch.tensor(make_exit_depths(wl.batch, wl.prefix, wl.k_max, seed=2 + rank), device="cuda")
+    handle.prefill(prefix, exit_depth)
+    handle.sync()
+    block_np = make_block_ids(m, wl.batch, wl.block)
+    block = torch.tensor(block_np, device="cuda")
+    masks = int((block_np == m.mask_id).sum())
+    tau, lam, rule = args.tau, args.lam, args.rule
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            dec = handle.decode_block(block, tau, lam, wl.k_max, rule)
+        handle.sync()
+        steps = dec["steps"]
+        rows = dec["rows"].cpu().numpy()
+        left = int((dec["tokens"] == m.mask_id).sum().item())
+        clocks = ClockSampler(local)
+        clocks.start()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            dec = handle.decode_block(block, tau, lam, wl.k_max, rule)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        clk = clocks.stop()
+        handle.sync()
+        ms = e0.elapsed_time(e1)
+        assert dec["steps"] == steps, "decoding is deterministic"
+        # end to end: block ids from pinned host memory in, final tokens back out, every call
+        ids_host = torch.tensor(block_np).pin_memory()
+        tok_host = torch.empty(block_np.shape, dtype=torch.int32).pin_memory()
+        dev_ids = torch.empty_like(block)
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            dev_ids.copy_(ids_host, non_blocking=True)
+            dec = handle.decode_block(dev_ids, tau, lam, wl.k_max, rule)
+            tok_host.copy_(dec["tokens"], non_blocking=True)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = f0.elapsed_time(f1)
+    launches_last_step = handle.step_stats()["launches"]
+    max_ms = all_max(ms, world)
+    decoded = all_sum(float(masks - left) * args.steps, world)
+    value = decoded / (max_ms / 1e3)
+    t_roof = 0.0
+    for t in range(steps):
+        tr, _, _ = step_roofline(m, wl.batch, wl.prefix, wl.block, rows[t, 0].tolist(), rows[t, 1].tolist(), peaks)
+        t_roof += tr
+    ms_call = max_ms / args.steps
+    line = {
+        "metric": "decoded tokens/s (block denoised until no [MASK]; 8B-shape bf16)", "value": value,
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_call,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded random bf16 weights, random prefix ids, all-[MASK] block)",
+        "config": {"workload": args.workload, "model": wl.model, "batch_per_gpu": wl.batch, "prefix": wl.prefix,
+                   "block": wl.block, "k_max": wl.k_max, "tau_H": tau, "lambda": lam,
+                   "rule": ["paper", "per_token"][rule], "parallelism": f"replicas x{world}", "mode": "decode_block"},
+        "denoising_steps_per_block": steps, "masks_left": left,
+        "step_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_call, "peak_source": peaks_src},
+        "e2e": {"value": decoded / (all_max(e2e_ms, world) / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": block_np.size * 4, "d2h_bytes_per_step": block_np.size * 4},
+        "gpu_launches": launches_last_step * steps * args.steps, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    handle.close()
+
+
 # ------------------------------------------------------------------------------------
 # reference arm: the CPU oracle, as it stands, on bounded samples of the same workload
 # ------------------------------------------------------------------------------------
@@ -461,6 +549,8 @@ def main():
     ap.add_argument("--lam", type=float, default=0.5)
     ap.add_argument("--rule", type=int, default=0, choices=[0, 1])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", action="store_true",
+                    help="time block decoding (steps until no [MASK]) instead of one step")
     ap.add_argument("--kernel", default=None, choices=["gemm"],
                     help="micro-benchmark one kernel instead of the step")
     ap.add_argument("--shape", default="32,24576,4096", help="M,N,K for --kernel gemm")
@@ -473,6 +563,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.decode:
+            run_decode(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -141,6 +141,32 @@ ALODLM_API int alodlm_prefill(alodlm_t *h, const int32_t *prefix_ids, int B, int
 ALODLM_API int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda,
                         int k_max, int rule, const alodlm_step_out *out);
 
+/* Outputs of a block decode, all caller-owned DEVICE buffers (S = the call's max_steps,
+ * K = its k_max). */
+typedef struct {
+    int32_t *tokens;       /* [B,N] the block after the last step (mask_id where still masked) */
+    int32_t *commit_step;  /* [B,N] 1-based step that committed the position; 0 for given ids and
+                              positions never committed */
+    int32_t *commit_depth; /* [B,N] loop s (1..K) of that step, 0 if never committed */
+    int32_t *steps_run;    /* [B] steps that had masks of the sequence at their start */
+    int32_t *loops;        /* [S,B] loops run by each sequence in each step (0 for steps not taken) */
+    int32_t *rows;         /* [S,2,K] per step: active_rows[K] then readout_rows[K] (as in a step) */
+} alodlm_decode_out;
+
+/* Denoise one block until no [MASK] is left, or for max_steps steps.
+ * [digest "Method steps", Algorithm 1 (5)]: after each denoising step the committed tokens are
+ * written into the sequence and the next step starts, until no [MASK] remains.  Step t + 1
+ * takes the tokens of step t as its block ids (every step sees the same prefix KV; the block
+ * is re-embedded from its ids).  The whole batch steps together: a sequence without masks
+ * still takes part in a step (nothing of it changes) but stops counting steps.
+ * Arguments as for alodlm_denoise_step; max_steps >= 1 (N suffices under the paper's rule,
+ * which commits at least one position per step; 1 under ALODLM_RULE_PER_TOKEN).
+ * steps_taken (host, may be NULL) receives the number of steps run.  Synchronises with the
+ * host once per step (a 4-byte "masks left" flag) besides the steps' own reads.
+ * Errors: EINVAL, ESTATE, ECUDA, ETIMEOUT, EDEVICE. */
+ALODLM_API int alodlm_decode_block(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda,
+                                   int k_max, int rule, int max_steps, const alodlm_decode_out *out, int *steps_taken);
+
 /* Wait for the handle's stream; returns ETIMEOUT/EDEVICE if a kernel raised the device error
  * word since the last call (the word is then cleared), ECUDA on a CUDA error. */
 ALODLM_API int alodlm_sync(alodlm_t *h);

@@ -52,6 +52,7 @@ int main(void) {
          sizeof(alodlm_cfg), sizeof(alodlm_layer_w), sizeof(alodlm_weights), sizeof(alodlm_step_out));
   P(alodlm_cfg, rope_base); P(alodlm_cfg, mask_id); P(alodlm_cfg, mem_limit_bytes); P(alodlm_cfg, debug_dump);
   P(alodlm_weights, exit_b); P(alodlm_weights, layers); P(alodlm_step_out, readout_rows);
+  printf("alodlm_decode_out %zu\n", sizeof(alodlm_decode_out)); P(alodlm_decode_out, rows);
   return 0;
 }
 """
@@ -76,6 +77,8 @@ def test_struct_layout_matches_binding(L):
     assert got["alodlm_weights.exit_b"] == L.Weights.exit_b.offset
     assert got["alodlm_weights.layers"] == L.Weights.layers.offset
     assert got["alodlm_step_out.readout_rows"] == L.StepOut.readout_rows.offset
+    assert got["alodlm_decode_out"] == ctypes.sizeof(L.DecodeOut)
+    assert got["alodlm_decode_out.rows"] == L.DecodeOut.rows.offset
 
 
 def _cfg(L, **kw):
@@ -108,6 +111,7 @@ def test_null_arguments_are_rejected(L):
     assert lib.alodlm_create(None, None, None, ctypes.byref(h)) == -1
     assert lib.alodlm_prefill(None, None, 1, 1, None) == -1
     assert lib.alodlm_denoise_step(None, None, 1, 1, 0.5, 0.5, 1, 0, None) == -1
+    assert lib.alodlm_decode_block(None, None, 1, 1, 0.5, 0.5, 1, 0, 1, None, None) == -1
     assert lib.alodlm_sync(None) == -1
     lib.alodlm_destroy(None)
     assert lib.alodlm_kernel_class_name(0) == b"gemm"

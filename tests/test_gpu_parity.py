@@ -46,10 +46,10 @@ def _gemm_ref(A, W):
                                    (512, 4096, 1024), (2048, 6144, 4096), (1000, 3000, 880),
                                    (832, 6144, 4096), (1536, 4096, 4096)])
 def test_gemm_tcgen05_against_fp64(M, N, K):
-    """The shapes cover every GEMM path: split-K clusters of 2-8 CTAs (few rows), the persistent
-    kernel with 128- and 256-wide tiles, and its stream-K schedule (1000 x 3000 x 880 with ragged
-    edges in M, N and K; 832 x 6144 and 1536 x 4096 at 1.3 waves) -- each with and without the
-    workspace room those need."""
+    """The shapes cover every GEMM path: split-K clusters of 2-8 CTAs (few rows) and the persistent
+    kernel with 128- and 256-wide tiles (ragged edges in M, N and K; 1.3-wave tile counts, which
+    take the stream-K schedule when it is compiled in) -- each with and without the workspace
+    room those need."""
     import adaptively_looped_masked_b200 as alo
     g = torch.Generator(device="cuda").manual_seed(M * 7 + N)
     A = torch.randn((M, K), device="cuda", generator=g).to(torch.bfloat16)
