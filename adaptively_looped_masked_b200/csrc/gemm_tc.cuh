@@ -116,21 +116,25 @@ __device__ __forceinline__ void acc_ld16(uint32_t taddr, int c0, float (&v)[16])
     acc_ld<NACC, BN, 16>(taddr, c0, v);
 }
 
-template <int BN>
-struct Cfg {
+// Compile-time tuning of the few-row tiles (BN <= 64): ring depth (4 keeps two CTAs per SM,
+// which the 192-tile gate/up launch at 32 rows needs) and TMEM accumulators per tile (1: the
+// MMAs of a stage chain on one accumulator; more measured no faster).
 #ifndef ALODLM_STAGES_SMALL
 #define ALODLM_STAGES_SMALL 4
 #endif
+#ifndef ALODLM_NACC_SMALL
+#define ALODLM_NACC_SMALL 1
+#endif
+
+template <int BN>
+struct Cfg {
     static constexpr int STAGES = (BN <= 64) ? ALODLM_STAGES_SMALL : (BN == 128 ? 5 : 4);
     static constexpr uint32_t A_BYTES = BM * BK * 2;
     static constexpr uint32_t B_BYTES = BN * BK * 2;
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-    // Few activation rows: the MMA per 16-wide k step is small and its latency, not the tensor
-    // pipe, would pace a single accumulation chain; the four k steps of a stage then go to four
-    // independent TMEM accumulators, summed in a fixed order by the epilogue.
-#ifndef ALODLM_NACC_SMALL
-#define ALODLM_NACC_SMALL 1
-#endif
+    // With NACC > 1 the 16-wide k steps of a stage rotate over NACC independent TMEM
+    // accumulators (shorter dependency chains for the small few-row MMAs), summed in a fixed
+    // order by the epilogue; the default is one.
     static constexpr int NACC = (BN <= 64) ? ALODLM_NACC_SMALL : 1;
     // epilogue columns per TMEM round trip: a narrow tile's whole row at once
     static constexpr int EC = (BN <= 64) ? BN : 16;
