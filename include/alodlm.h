@@ -162,8 +162,10 @@ typedef struct {
  * Arguments as for alodlm_denoise_step; max_steps >= 1 (N suffices under the paper's rule,
  * which commits at least one position per step; 1 under ALODLM_RULE_PER_TOKEN).
  * steps_taken (host, may be NULL) receives the number of steps run.  Synchronises with the
- * host once per step (a 4-byte "masks left" flag) besides the steps' own reads.
- * Errors: EINVAL, ESTATE, ECUDA, ETIMEOUT, EDEVICE. */
+ * host once per step (a 4-byte "masks left" flag) besides the steps' own reads.  Uses
+ * handle-owned scratch for the steps' traces, so calls on one handle must not overlap.
+ * Errors: EINVAL, ESTATE, ECUDA, ETIMEOUT, EDEVICE; after an error the outputs are undefined
+ * (a failing step returns its own code). */
 ALODLM_API int alodlm_decode_block(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda,
                                    int k_max, int rule, int max_steps, const alodlm_decode_out *out, int *steps_taken);
 
