@@ -347,19 +347,34 @@ def test_fallback_special_cases():
             np.testing.assert_allclose(vv, ref[s][rkey][1], rtol=1e-12, atol=1e-14)
 
 
+def _golden(name):
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", name)
+    return json.load(open(path))
+
+
 def test_counts_printed_by_the_pages():
-    """8B at K = 4: L + (K-1) m = 36 + 3 x 16 = 84 KV buffers (Limitations section) and
-    10 + 4 x (16 + 10) = 114 layer executions without early exit (Technical novelty section)."""
+    """8B at K = 4 (tests/golden/page_counts.json): L + (K-1) m = 84 KV buffers (Limitations
+    section), 10 + 4 x (16 + 10) = 114 layer executions without early exit and 4 x 36 = 144 if
+    every layer looped (Technical novelty section)."""
+    g = _golden("page_counts.json")
     shape = small_shape(hidden=16, n_q_heads=2, n_kv_heads=1, head_dim=8, inter=16, vocab=20,
                         n_prelude=10, n_core=16, n_coda=10)
     o, _ = build(shape, 4)
-    assert o.n_kv_slots() == 36 + 3 * 16 == 84
+    assert o.n_kv_slots() == g["kv_buffers_8b_k4"]["value"]
     o.prefill(make_prefix_ids(shape, 1, 3)[None][0])
     kv = o.kv[0]
-    assert len(kv) == 84
+    assert len(kv) == g["kv_buffers_8b_k4"]["value"]
     out = o.denoise_step(make_block_ids(shape, 1, 2), tau=-1.0, lam=2.0, k_max=4)
-    assert o.layer_execs == 10 + 4 * (16 + 10) == 114
+    assert o.layer_execs == g["layer_executions_8b_k4"]["value"]
     assert out["loops_run"][0] == 4
+    full = small_shape(hidden=16, n_q_heads=2, n_kv_heads=1, head_dim=8, inter=16, vocab=20,
+                       n_prelude=0, n_core=36, n_coda=0)
+    of, _ = build(full, 4)
+    of.prefill(make_prefix_ids(full, 1, 3)[None][0])
+    of.denoise_step(make_block_ids(full, 1, 2), tau=-1.0, lam=2.0, k_max=4)
+    assert of.layer_execs == g["layer_executions_full_stack_k4"]["value"]
 
 
 def test_cumulative_halting_closed_form_and_invariants():
