@@ -1054,15 +1054,21 @@ int alodlm_decode_block(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
     if (k_max < 1 || k_max > h->cfg.k_max) return fail(h, ALODLM_EINVAL, "k_max out of range");
     const long long BN = (long long)B * N;
     const unsigned grid = (unsigned)std::min<long long>((BN + 255) / 256, 1024);
-    cudaMemsetAsync(out->commit_step, 0, BN * sizeof(int32_t), h->stream);
-    cudaMemsetAsync(out->commit_depth, 0, BN * sizeof(int32_t), h->stream);
-    cudaMemsetAsync(out->steps_run, 0, (size_t)B * sizeof(int32_t), h->stream);
-    cudaMemsetAsync(out->loops, 0, (size_t)max_steps * B * sizeof(int32_t), h->stream);
-    cudaMemsetAsync(out->rows, 0, (size_t)max_steps * 2 * k_max * sizeof(int32_t), h->stream);
-    cudaMemcpyAsync(out->tokens, block_ids, BN * sizeof(int32_t), cudaMemcpyDeviceToDevice, h->stream);
+    cudaError_t ce = cudaSuccess;  // first error of the asynchronous calls
+    auto ck = [&](cudaError_t e) {
+        if (ce == cudaSuccess) ce = e;
+    };
+    ck(cudaMemsetAsync(out->commit_step, 0, BN * sizeof(int32_t), h->stream));
+    ck(cudaMemsetAsync(out->commit_depth, 0, BN * sizeof(int32_t), h->stream));
+    ck(cudaMemsetAsync(out->steps_run, 0, (size_t)B * sizeof(int32_t), h->stream));
+    ck(cudaMemsetAsync(out->loops, 0, (size_t)max_steps * B * sizeof(int32_t), h->stream));
+    ck(cudaMemsetAsync(out->rows, 0, (size_t)max_steps * 2 * k_max * sizeof(int32_t), h->stream));
+    ck(cudaMemcpyAsync(out->tokens, block_ids, BN * sizeof(int32_t), cudaMemcpyDeviceToDevice, h->stream));
     // a block without masks takes no step
-    cudaMemsetAsync(h->dec_left, 0, sizeof(int), h->stream);
+    ck(cudaMemsetAsync(h->dec_left, 0, sizeof(int), h->stream));
     klaunch(k::any_mask_kernel, grid, 256, 0, h->stream, (const int *)block_ids, BN, h->cfg.mask_id, h->dec_left);
+    ck(cudaGetLastError());
+    if (ce != cudaSuccess) return cuda_fail(h, ce, "decode_block: set-up");
     const size_t KBN = (size_t)k_max * BN;
     alodlm_step_out so{};
     so.exit_depth = h->dec_ex;
@@ -1075,28 +1081,28 @@ int alodlm_decode_block(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
     const int32_t *in = block_ids;
     int t = 0;
     for (;;) {
-        cudaError_t e = cudaMemcpyAsync(h->dec_left_host, h->dec_left, sizeof(int), cudaMemcpyDeviceToHost, h->stream);
-        if (e == cudaSuccess) e = cudaStreamSynchronize(h->stream);
-        if (e != cudaSuccess) return cuda_fail(h, e, "decode_block: read the masks-left flag");
+        ck(cudaMemcpyAsync(h->dec_left_host, h->dec_left, sizeof(int), cudaMemcpyDeviceToHost, h->stream));
+        ck(cudaStreamSynchronize(h->stream));
+        if (ce != cudaSuccess) return cuda_fail(h, ce, "decode_block: read the masks-left flag");
         if (*h->dec_left_host == 0 || t == max_steps) break;
         ++t;
         so.tokens = h->dec_tok[t & 1];
-        int rc = alodlm_denoise_step(h, in, B, N, tau_H, lambda, k_max, rule, &so);
+        const int rc = alodlm_denoise_step(h, in, B, N, tau_H, lambda, k_max, rule, &so);
         if (rc) return rc;
-        cudaMemsetAsync(h->dec_left, 0, sizeof(int), h->stream);
+        ck(cudaMemsetAsync(h->dec_left, 0, sizeof(int), h->stream));
         klaunch(k::decode_update_kernel, grid, 256, 0, h->stream, (const int *)in, (const int *)so.tokens,
                 (const int *)h->dec_ex, t, B, N, h->cfg.mask_id, out->commit_step, out->commit_depth, out->steps_run,
                 h->dec_left);
-        cudaMemcpyAsync(out->loops + (size_t)(t - 1) * B, h->dec_loops, (size_t)B * sizeof(int32_t),
-                        cudaMemcpyDeviceToDevice, h->stream);
-        cudaMemcpyAsync(out->rows + (size_t)(t - 1) * 2 * k_max, h->dec_rows, 2 * (size_t)k_max * sizeof(int32_t),
-                        cudaMemcpyDeviceToDevice, h->stream);
+        ck(cudaGetLastError());
+        ck(cudaMemcpyAsync(out->loops + (size_t)(t - 1) * B, h->dec_loops, (size_t)B * sizeof(int32_t),
+                           cudaMemcpyDeviceToDevice, h->stream));
+        ck(cudaMemcpyAsync(out->rows + (size_t)(t - 1) * 2 * k_max, h->dec_rows, 2 * (size_t)k_max * sizeof(int32_t),
+                           cudaMemcpyDeviceToDevice, h->stream));
         in = so.tokens;
     }
-    if (t > 0)
-        cudaMemcpyAsync(out->tokens, in, BN * sizeof(int32_t), cudaMemcpyDeviceToDevice, h->stream);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(h, e, "decode_block");
+    if (t > 0) ck(cudaMemcpyAsync(out->tokens, in, BN * sizeof(int32_t), cudaMemcpyDeviceToDevice, h->stream));
+    ck(cudaGetLastError());
+    if (ce != cudaSuccess) return cuda_fail(h, ce, "decode_block");
     if (steps_taken) *steps_taken = t;
     return ALODLM_OK;
 }
