@@ -59,7 +59,7 @@ def dist_setup(n_gpus):
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local))
-    else:
+    elif torch.cuda.is_available():  # the reference arm (the CPU oracle) also runs without a GPU
         torch.cuda.set_device(0)
     return world, rank, local
 

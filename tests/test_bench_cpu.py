@@ -1,0 +1,53 @@
+"""bench.py's host side without a GPU: the reference arm (the CPU oracle on a bounded sample
+of the workload) prints one JSON line with the contract's keys, and the step-roofline
+arithmetic follows its stated formula."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def test_reference_arm_prints_one_contract_line():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                          "--steps", "1", "--warmup", "0"], capture_output=True, text=True, env=env, cwd=ROOT,
+                         timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "tokens/s"
+    for key in ("metric", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling", "vs_baseline",
+                "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert d["config"]["workload"] == "tiny"
+
+
+def test_step_roofline_formula():
+    """T_roof = T_prelude + sum over loops of max(F_s / P, B_s / BW), with F_s and B_s as the
+    docstring of bench.step_roofline and the measurement section state them."""
+    import bench
+    from synth import MODELS
+    m = MODELS["qwen3-8b"]
+    peaks = {"hbm_gbs": 1000.0, "bf16_tflops_sustained": 1000.0}
+    B, P, N = 2, 100, 10
+    p = m.hidden * m.n_q_heads * m.head_dim * 2 + 2 * m.hidden * m.n_kv_heads * m.head_dim + 3 * m.hidden * m.inter
+    assert p == 192_937_984  # 192.9 M parameters per 8B layer
+    CD = m.n_core + m.n_coda
+    kvl = 2 * 2 * m.n_kv_heads * (P + N) * m.head_dim
+    f_pre = 2.0 * B * N * m.n_prelude * p + 4.0 * B * N * (P + N) * m.n_q_heads * m.head_dim * m.n_prelude
+    b_pre = 2.0 * p * m.n_prelude + B * m.n_prelude * kvl
+    rows, R = 20, 7
+    f1 = 2.0 * rows * CD * p + 2.0 * R * m.vocab * m.hidden + 4.0 * rows * (P + N) * m.n_q_heads * m.head_dim * CD
+    b1 = 2.0 * p * CD + 2.0 * m.vocab * m.hidden + 2 * CD * kvl
+    want = max(f_pre / 1e15, b_pre / 1e12) + max(f1 / 1e15, b1 / 1e12)
+    t, F, Bt = bench.step_roofline(m, B, P, N, [rows, 0], [R, 0], peaks)
+    assert t == pytest.approx(want, rel=1e-12)
+    assert F == pytest.approx(f_pre + f1, rel=1e-12) and Bt == pytest.approx(b_pre + b1, rel=1e-12)
