@@ -50,18 +50,29 @@ def load_peaks():
 # ------------------------------------------------------------------------------------
 
 def dist_setup(n_gpus):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE).  The process group is
+    NCCL on GPUs; without a GPU (the CPU reference arm, the multi-process host tests) gloo.
+    A short timeout makes ranks that wait for a missing peer end with an error."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=float(os.environ.get("ALODLM_PG_TIMEOUT_S", "600")))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timeout)
     elif torch.cuda.is_available():  # the reference arm (the CPU oracle) also runs without a GPU
         torch.cuda.set_device(0)
     return world, rank, local
+
+
+def _coll_device():
+    import torch.distributed as dist
+    return "cuda" if dist.get_backend() == "nccl" else "cpu"
 
 
 def barrier(world):
@@ -71,19 +82,21 @@ def barrier(world):
 
 
 def all_max(x, world):
+    """Maximum over ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_coll_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
 def all_sum(x, world):
+    """Sum over ranks (the units every rank processed)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_coll_device())
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
 

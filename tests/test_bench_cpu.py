@@ -51,3 +51,58 @@ def test_step_roofline_formula():
     t, F, Bt = bench.step_roofline(m, B, P, N, [rows, 0], [R, 0], peaks)
     assert t == pytest.approx(want, rel=1e-12)
     assert F == pytest.approx(f_pre + f1, rel=1e-12) and Bt == pytest.approx(b_pre + b1, rel=1e-12)
+
+
+def _free_port():
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), LOCAL_RANK=str(rank),
+                      WORLD_SIZE=str(world), CUDA_VISIBLE_DEVICES="", ALODLM_PG_TIMEOUT_S="60")
+    sys.path.insert(0, ROOT)
+    import bench
+    import torch.distributed as dist
+    w, r, _ = bench.dist_setup(world)
+    bench.barrier(w)
+    # rank r "timed" 1 + r ms and processed 10 * (r + 1) units
+    mx = bench.all_max(1.0 + r, w)
+    sm = bench.all_sum(10.0 * (r + 1), w)
+    q.put((r, w, dist.get_backend(), mx, sm))
+    dist.destroy_process_group()
+
+
+def test_two_rank_collectives_on_gloo():
+    """The N > 1 host path of bench.py on CPU: gloo group, barrier, max-over-ranks time and
+    summed units (value = units of all ranks / slowest rank's time)."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=10) for _ in range(2))
+    for r, (rank, world, backend, mx, sm) in enumerate(got):
+        assert (rank, world, backend) == (r, 2, "gloo")
+        assert mx == 2.0 and sm == 30.0
+
+
+def test_reference_arm_under_two_ranks():
+    """torchrun with 2 ranks on CPU: rank 0 alone runs the oracle and prints the line, rank 1
+    exits 0 without work."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", ALODLM_PG_TIMEOUT_S="120")
+    out = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                          "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+                          os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference", "--workload",
+                          "tiny", "--steps", "1", "--warmup", "0"], capture_output=True, text=True, env=env,
+                         cwd=ROOT, timeout=600)
+    assert out.returncode == 0, out.stderr[-3000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1 and json.loads(lines[0])["impl"] == "reference"
