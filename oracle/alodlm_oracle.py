@@ -367,6 +367,74 @@ class Oracle:
         self.prefix_len = P
         return self.kv
 
+    def append(self, ids: np.ndarray, exit_depth: Optional[np.ndarray] = None) -> dict:
+        """Extend the cached prefix by N positions P..P+N-1 holding ``ids`` (a decoded block).
+
+        [digest] "Method steps", Algorithm 1 (5): the committed tokens are written into the
+        sequence, which later blocks attend to as context; "Technical novelty": every
+        position is served at its own loop depth, the deepest it reached standing in for
+        deeper ones.  The new positions go through exactly what ``prefill`` does for prefix
+        positions -- Prelude, the Core e_j times (Core KV at depth d > e_j = the depth-e_j KV),
+        the Coda once on the depth-e_j state -- attending to every cached position (at its
+        own slot, fallback already resolved) and causally to each other.  ``exit_depth``
+        [B, N] in 1..k_max (default k_max).  Extends self.kv in place; returns it.
+        """
+        c = self.cfg
+        K = c["k_max"]
+        assert self.kv is not None, "prefill first"
+        ids = np.asarray(ids)
+        B, N = ids.shape
+        P = self.prefix_len
+        if exit_depth is None:
+            exit_depth = np.full((B, N), K, dtype=np.int64)
+        exit_depth = np.asarray(exit_depth)
+        assert exit_depth.min() >= 1 and exit_depth.max() <= K
+        emb = self._global("embed")
+        pos = P + np.arange(N)
+        # new row i sees every cached position and the new positions up to itself
+        vis = np.concatenate([np.ones((N, P), dtype=bool), np.tril(np.ones((N, N), dtype=bool))], axis=1)
+
+        def extend(key, k_new, v_new):
+            kp, vp = kv[key]
+            kv[key] = (np.concatenate([kp, k_new], axis=0), np.concatenate([vp, v_new], axis=0))
+            return kv[key]
+
+        for b in range(B):
+            kv = self.kv[b]
+            h = emb[ids[b]].astype(self.dt)
+            for l in range(c["n_prelude"]):
+                lw = self.layer_weights(l)
+                q, k, v = self.qkv(lw, h, pos)
+                k_all, v_all = extend(("prelude", l), k, v)
+                h = self.finish_layer(lw, h, q, k_all, v_all, vis)
+            e = exit_depth[b]
+            h_exit = h.copy()
+            for d in range(1, K + 1):
+                act = np.nonzero(e >= d)[0]
+                for j in range(c["n_core"]):
+                    lw = self.layer_weights(self.core_layer_index(j))
+                    if d == 1:
+                        k_new = np.zeros((N, c["n_kv_heads"], c["head_dim"]), dtype=self.dt)
+                        v_new = np.zeros_like(k_new)
+                    else:
+                        # new positions that stopped before depth d keep their deepest KV
+                        k_new, v_new = (x[P:].copy() for x in kv[("core", j, d - 1)])
+                    if len(act):
+                        q, k, v = self.qkv(lw, h[act], pos[act])
+                        k_new[act], v_new[act] = k, v
+                    k_all, v_all = extend(("core", j, d), k_new, v_new)
+                    if len(act):
+                        h[act] = self.finish_layer(lw, h[act], q, k_all, v_all, vis[act])
+                h_exit[e == d] = h[e == d]
+            h = h_exit
+            for j in range(c["n_coda"]):
+                lw = self.layer_weights(self.coda_layer_index(j))
+                q, k, v = self.qkv(lw, h, pos)
+                k_all, v_all = extend(("coda", j), k, v)
+                h = self.finish_layer(lw, h, q, k_all, v_all, vis)
+        self.prefix_len = P + N
+        return self.kv
+
     # --- one layer over the block against the cached prefix ----------------------------
 
     def block_layer(self, b: int, key, lw: dict, h: np.ndarray) -> np.ndarray:

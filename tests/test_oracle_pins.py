@@ -650,3 +650,43 @@ def test_decode_step_bound():
     out = om.decode_block(o, block, tau=-1.0, lam=2.0, k_max=3, rule=RULE_PAPER, max_steps=2)
     assert out["steps"] == 2 and (out["tokens"] == shape.mask_id).sum() == 4
     assert ((out["commit_step"] > 0) == (out["tokens"] != shape.mask_id)).all()
+
+
+# ------------------------------------------------------------------------------------
+# appending a decoded block to the prefix
+# ------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("shape", [small_shape(), small_shape(n_prelude=0, n_coda=0, name="fullcore")])
+def test_append_equals_prefill_of_the_longer_prefix(shape):
+    """Prefix attention is causal, so extending a cached prefix by N positions must give the
+    KV (every slot, every depth, fallback included) of one prefill over the longer sequence."""
+    K = 3
+    ids = make_prefix_ids(shape, 2, 14)
+    e = make_exit_depths(2, 14, K, seed=5)
+    o1, _ = build(shape, K)
+    o1.prefill(ids[:, :9], e[:, :9])
+    o1.append(ids[:, 9:], e[:, 9:])
+    o2, _ = build(shape, K)
+    o2.prefill(ids, e)
+    assert o1.prefix_len == o2.prefix_len == 14
+    for b in range(2):
+        assert set(o1.kv[b]) == set(o2.kv[b])
+        for key in o2.kv[b]:
+            for a1, a2 in zip(o1.kv[b][key], o2.kv[b][key]):
+                np.testing.assert_allclose(a1, a2, rtol=1e-11, atol=1e-12)
+
+
+def test_step_after_append_equals_step_after_full_prefill():
+    shape = small_shape()
+    K = 3
+    ids = make_prefix_ids(shape, 1, 12)
+    block = make_block_ids(shape, 1, 6)
+    o1, _ = build(shape, K)
+    o1.prefill(ids[:, :7])
+    o1.append(ids[:, 7:])
+    o2, _ = build(shape, K)
+    o2.prefill(ids)
+    r1 = o1.denoise_step(block, tau=0.6, lam=0.5, k_max=K)
+    r2 = o2.denoise_step(block, tau=0.6, lam=0.5, k_max=K)
+    np.testing.assert_array_equal(r1["exit_depth"], r2["exit_depth"])
+    np.testing.assert_allclose(r1["entropy"], r2["entropy"], rtol=1e-10, equal_nan=True)
