@@ -216,8 +216,11 @@ GemmShape plan_gemm(int M, int Nw, int K) {
     // 128 tile rows evenly in the reduction); at least 4 k-tiles each
     splits = std::max(1, std::min(std::min(splits, ALODLM_MAX_SPLITS), g.k_tiles / 4));
     while (splits & (splits - 1)) --splits;
+    // equal k-ranges of cdiv(k_tiles, splits) must give exactly `splits` non-empty ranges (the
+    // cluster reduction needs a power of two; e.g. 33 k-tiles in 8 ranges of 5 leave only 7)
+    while (splits > 1 && cdiv(g.k_tiles, cdiv(g.k_tiles, splits)) != splits) splits >>= 1;
     g.kps = cdiv(g.k_tiles, splits);
-    g.splits = cdiv(g.k_tiles, g.kps);
+    g.splits = splits;
     return g;
 }
 

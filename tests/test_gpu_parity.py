@@ -44,12 +44,13 @@ def _gemm_ref(A, W):
 @pytest.mark.parametrize("M,N,K", [(1, 128, 64), (16, 200, 256), (32, 384, 880), (33, 1376, 256), (100, 512, 320),
                                    (128, 256, 4096), (300, 640, 768), (2048, 512, 1024), (20, 6144, 4096),
                                    (512, 4096, 1024), (2048, 6144, 4096), (1000, 3000, 880),
-                                   (832, 6144, 4096), (1536, 4096, 4096)])
+                                   (832, 6144, 4096), (1536, 4096, 4096), (32, 4096, 2112)])
 def test_gemm_tcgen05_against_fp64(M, N, K):
     """The shapes cover every GEMM path: split-K clusters of 2-8 CTAs (few rows) and the persistent
     kernel with 128- and 256-wide tiles (ragged edges in M, N and K; 1.3-wave tile counts, which
     take the stream-K schedule when it is compiled in) -- each with and without the workspace
-    room those need."""
+    room those need.  K = 2112 (33 k-tiles) cannot be cut into 8 equal non-empty ranges: the
+    plan must fall back to 4."""
     import adaptively_looped_masked_b200 as alo
     g = torch.Generator(device="cuda").manual_seed(M * 7 + N)
     A = torch.randn((M, K), device="cuda", generator=g).to(torch.bfloat16)
