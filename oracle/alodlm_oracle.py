@@ -155,6 +155,65 @@ def halts(n_left: int, mean_a_left: float, s: int, K: int, rule: int, lam: float
     return rule == RULE_PAPER and mean_a_left >= lam
 
 
+# ----------------------------------------------------------------------------------
+# sampling the committed token (digest "Method steps", Algorithm 1 (3): each committed
+# position samples y_i ~ p_i^(s)); counter-based random numbers so that any other
+# implementation can draw the same ones
+# ----------------------------------------------------------------------------------
+
+_M64 = np.uint64(0xFFFFFFFFFFFFFFFF)
+_LO32 = np.uint64(0xFFFFFFFF)
+_PHILOX_M = (np.uint64(0xD2E7470EE14C6C93), np.uint64(0xCA5A826395121157))
+_PHILOX_W = (np.uint64(0x9E3779B97F4A7C15), np.uint64(0xBB67AE8584CAA73B))
+
+
+def _mulhilo64(a: np.ndarray, b: np.uint64):
+    """(high, low) 64-bit halves of the 128-bit products a * b, through 32-bit limbs."""
+    s32 = np.uint64(32)
+    a0, a1 = a & _LO32, a >> s32
+    b0, b1 = b & _LO32, b >> s32
+    p00, p01, p10, p11 = a0 * b0, a0 * b1, a1 * b0, a1 * b1
+    mid = (p00 >> s32) + (p01 & _LO32) + (p10 & _LO32)
+    hi = p11 + (p01 >> s32) + (p10 >> s32) + (mid >> s32)
+    return hi, a * b
+
+
+def philox4x64(counter: np.ndarray, key) -> np.ndarray:
+    """Philox4x64-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as easy as 1,
+    2, 3", SC 2011): ten rounds of two 64 x 64 -> 128-bit multiplications and xors, the key
+    bumped by the Weyl constants between rounds.  counter [..., 4] uint64, key (2,) -> [..., 4]."""
+    with np.errstate(over="ignore"):
+        x = [np.asarray(counter, dtype=np.uint64)[..., i].copy() for i in range(4)]
+        k0, k1 = np.uint64(key[0]), np.uint64(key[1])
+        for r in range(10):
+            if r:
+                k0, k1 = k0 + _PHILOX_W[0], k1 + _PHILOX_W[1]
+            hi0, lo0 = _mulhilo64(x[0], _PHILOX_M[0])
+            hi1, lo1 = _mulhilo64(x[2], _PHILOX_M[1])
+            x = [hi1 ^ x[1] ^ k0, lo1, hi0 ^ x[3] ^ k1, lo0]
+    return np.stack(x, axis=-1)
+
+
+def gumbel_scores(z: np.ndarray, key, position: int, loop: int) -> np.ndarray:
+    """z_v + g_v with g_v = -log(-log(u_v)), u_v uniform in (0, 1) from the 53 high bits of
+    Philox4x64-10 output (v mod 4) at counter (v div 4, position, loop, 0) under ``key``."""
+    V = z.shape[0]
+    nb = (V + 3) // 4
+    ctr = np.zeros((nb, 4), dtype=np.uint64)
+    ctr[:, 0] = np.arange(nb, dtype=np.uint64)
+    ctr[:, 1] = np.uint64(position)
+    ctr[:, 2] = np.uint64(loop)
+    bits = philox4x64(ctr, key).reshape(-1)[:V]
+    u = ((bits >> np.uint64(11)).astype(np.float64) + 0.5) * 2.0 ** -53
+    g = -np.log(-np.log(u))
+    return z.astype(np.float64) + g
+
+
+def gumbel_argmax(z: np.ndarray, key, position: int, loop: int) -> int:
+    """A draw from softmax(z) by the Gumbel-max construction (lowest index on ties)."""
+    return int(np.argmax(gumbel_scores(z, key, position, loop)))
+
+
 def forced_pick(H_by_pos: Dict[int, float]) -> int:
     """Step (5): the lowest-entropy unresolved position (lowest index on ties)."""
     return min(H_by_pos.items(), key=lambda kv: (kv[1], kv[0]))[0]
@@ -476,7 +535,7 @@ class Oracle:
 
     def denoise_step(self, block_ids: np.ndarray, tau: float, lam: float, k_max: int,
                      rule: int = RULE_PAPER, follow: Optional[dict] = None, band: float = 1e-3,
-                     logit_rows: Optional[List[tuple]] = None) -> dict:
+                     logit_rows: Optional[List[tuple]] = None, sample_key=None) -> dict:
         """One denoising step, [digest] "Method steps" Algorithm 1 (1)-(5) and Eq. 3.
 
         block_ids [B, N]; positions holding mask_id form U.  ``lam`` is the halting
@@ -485,6 +544,8 @@ class Oracle:
         value lies within ``band`` of its threshold (or whose top-two gap is below ``band``),
         the oracle takes that run's decision and records it in "followed"; band=inf follows
         every decision.  ``logit_rows``: (b, s, i) triples whose logits are returned.
+        ``sample_key`` (two integers): committed tokens are drawn from p_i^(s) by Gumbel-max
+        (``gumbel_argmax`` at position b * N + i, loop s) instead of taken greedily.
 
         Returns tokens, exit_depth, entropy/halt/cum_halt [B,K,N] (NaN where not computed),
         loops_run [B], active_rows [K], readout_rows [K]; per sequence b, lists of
@@ -550,11 +611,16 @@ class Oracle:
                 out["halt"][b, s - 1, idx] = lmb
                 out["cum_halt"][b, s - 1, idx] = a[idx]
                 last_H = dict(zip(idx.tolist(), H.tolist()))
-                # greedy token choice, lowest id on ties
+                # greedy token choice (lowest id on ties), or a Gumbel-max draw
                 y = y.astype(np.int64).copy()
+                scores = z
+                if sample_key is not None:
+                    scores = np.stack([gumbel_scores(z[t], sample_key, b * N + int(idx[t]), s)
+                                       for t in range(len(idx))]) if len(idx) else z
+                    y = np.argmax(scores, axis=-1).astype(np.int64) if len(idx) else y
                 if follow is not None:
                     for t in range(len(idx)):
-                        top2 = np.partition(z[t], -2)[-2:]
+                        top2 = np.partition(scores[t], -2)[-2:]
                         if top2[1] - top2[0] < band:
                             i = int(idx[t])
                             if follow["exit_depth"][b, i] == s:
@@ -605,6 +671,8 @@ class Oracle:
                     if gpu_i:
                         i_star = gpu_i[0]
                 z_star = self.readout(rs[-1][[i_star]])[3][0]
+                if sample_key is not None:
+                    z_star = gumbel_scores(z_star, sample_key, b * N + int(i_star), s_last)
                 y_star = int(np.argmax(z_star))
                 if follow is not None and follow["exit_depth"][b, i_star] == s_last:
                     top2 = np.partition(z_star, -2)[-2:]
@@ -625,7 +693,7 @@ class Oracle:
 
 def decode_block(oracle: Oracle, block_ids: np.ndarray, tau: float, lam: float, k_max: int,
                  rule: int = RULE_PAPER, max_steps: int = 0, follow_steps: Optional[List[dict]] = None,
-                 band: float = 1e-3) -> dict:
+                 band: float = 1e-3, sample_seed: Optional[int] = None) -> dict:
     """Denoising steps over one block until no [MASK] is left, [digest] "Method steps",
     Algorithm 1 (5): after each step the committed tokens are written into the sequence and
     the next denoising step starts, until no [MASK] remains.
@@ -635,7 +703,7 @@ def decode_block(oracle: Oracle, block_ids: np.ndarray, tau: float, lam: float, 
     sequence without masks still runs a step (its U is empty, so nothing changes), and stops
     counting steps once its block is complete.  ``max_steps`` (0 = N) bounds the steps.
     ``follow_steps``: per step, another run's decisions (the ``follow`` argument of
-    ``Oracle.denoise_step``).
+    ``Oracle.denoise_step``).  ``sample_seed``: draw the committed tokens (key (seed, step)).
 
     Returns tokens [B,N] (final), commit_step [B,N] (1-based step that committed the
     position; 0 for given ids and positions never committed), commit_depth [B,N] (the loop s
@@ -655,7 +723,8 @@ def decode_block(oracle: Oracle, block_ids: np.ndarray, tau: float, lam: float, 
         t += 1
         had_masks = (ids == mask_id).any(axis=1)
         follow = follow_steps[t - 1] if follow_steps is not None and t - 1 < len(follow_steps) else None
-        out = oracle.denoise_step(ids, tau, lam, k_max, rule, follow=follow, band=band)
+        key = None if sample_seed is None else (int(sample_seed), t)
+        out = oracle.denoise_step(ids, tau, lam, k_max, rule, follow=follow, band=band, sample_key=key)
         new = out["exit_depth"] > 0
         commit_step[new] = t
         commit_depth[new] = out["exit_depth"][new]

@@ -11,6 +11,7 @@ import math
 import numpy as np
 import pytest
 import scipy.special
+import scipy.stats
 import torch
 
 import oracle.alodlm_oracle as om
@@ -690,3 +691,58 @@ def test_step_after_append_equals_step_after_full_prefill():
     r2 = o2.denoise_step(block, tau=0.6, lam=0.5, k_max=K)
     np.testing.assert_array_equal(r1["exit_depth"], r2["exit_depth"])
     np.testing.assert_allclose(r1["entropy"], r2["entropy"], rtol=1e-10, equal_nan=True)
+
+
+# ------------------------------------------------------------------------------------
+# sampled commits: Philox4x64-10 and the Gumbel-max draw
+# ------------------------------------------------------------------------------------
+
+def test_philox_matches_numpy_bit_generator():
+    """numpy's Philox bit generator is Philox4x64-10; it increments its counter before each
+    block, so its n-th block of four is the function at counter n + 1."""
+    for key in ((1, 2), (0, 0), (0xFFFFFFFFFFFFFFFF, 0x0123456789ABCDEF)):
+        bg = np.random.Philox(key=np.array(key, dtype=np.uint64), counter=np.zeros(4, dtype=np.uint64))
+        ref = bg.random_raw(4 * 6)
+        ctr = np.zeros((6, 4), dtype=np.uint64)
+        ctr[:, 0] = np.arange(1, 7, dtype=np.uint64)
+        np.testing.assert_array_equal(om.philox4x64(ctr, key).reshape(-1), ref)
+    # the higher counter words and a carry into them
+    bg = np.random.Philox(key=np.array((7, 9), dtype=np.uint64),
+                          counter=np.array((0xFFFFFFFFFFFFFFFF, 3, 5, 0), dtype=np.uint64))
+    got = om.philox4x64(np.array([[0, 4, 5, 0]], dtype=np.uint64), (7, 9)).reshape(-1)
+    np.testing.assert_array_equal(got, bg.random_raw(4))
+
+
+def test_gumbel_max_draws_follow_softmax():
+    """Gumbel-max: P(argmax_v z_v + g_v = w) = softmax(z)_w.  20000 draws (one per counter
+    position) of a 5-entry distribution pass a chi-square test at the 1e-6 level."""
+    z = np.array([1.0, 0.2, -0.5, 2.0, 0.0])
+    p = np.exp(z - z.max())
+    p /= p.sum()
+    n = 20000
+    counts = np.zeros(5)
+    for pos in range(n):
+        counts[om.gumbel_argmax(z, (11, 3), pos, 1)] += 1
+    chi2 = (((counts - n * p) ** 2) / (n * p)).sum()
+    assert chi2 < scipy.stats.chi2.isf(1e-6, df=4), chi2
+    # a logit far above the rest is always drawn
+    z2 = np.array([0.0, 60.0, 1.0, -3.0])
+    assert all(om.gumbel_argmax(z2, (5, 5), pos, 2) == 1 for pos in range(200))
+
+
+def test_sampled_step_commits_the_same_positions_at_loop_one():
+    """Sampling changes which token a committed position gets, not its entropy: at loop 1 the
+    entropies and the committed positions equal the greedy step's, and each committed token
+    is the Gumbel-max draw of its logits."""
+    shape = MODELS["tiny"]
+    o, _ = build(shape, 4)
+    o.prefill(make_prefix_ids(shape, 1, 48))
+    block = make_block_ids(shape, 1, 16)
+    g = o.denoise_step(block, tau=0.6, lam=0.9, k_max=4)
+    rows = [(0, 1, i) for i in range(16)]
+    sm = o.denoise_step(block, tau=0.6, lam=0.9, k_max=4, sample_key=(42, 1), logit_rows=rows)
+    np.testing.assert_allclose(sm["entropy"][0, 0], g["entropy"][0, 0], equal_nan=True)
+    first = g["exit_depth"][0] == 1
+    np.testing.assert_array_equal(sm["exit_depth"][0] == 1, first)
+    for i in np.nonzero(first)[0]:
+        assert sm["tokens"][0, i] == om.gumbel_argmax(sm["logits"][(0, 1, int(i))], (42, 1), int(i), 1)
