@@ -116,3 +116,34 @@ def test_null_arguments_are_rejected(L):
     lib.alodlm_destroy(None)
     assert lib.alodlm_kernel_class_name(0) == b"gemm"
     assert lib.alodlm_gemm_bf16(None, None, None, 1, 1, 8, None, 0, None) == -1
+
+
+LINK_C = r"""
+#include <stdio.h>
+#include "alodlm.h"
+int main(void) {
+  alodlm_t *h = (alodlm_t *)1;
+  alodlm_cfg cfg = {0};            /* hidden 0: rejected before any device work */
+  int rc = alodlm_create(&cfg, NULL, NULL, &h);
+  printf("%d %d %s\n", rc, h == NULL, alodlm_last_error(NULL) ? "msg" : "none");
+  printf("%d\n", alodlm_denoise_step(NULL, NULL, 1, 1, 0.5f, 0.5f, 1, ALODLM_RULE_PAPER, NULL));
+  printf("%s\n", alodlm_kernel_class_name(1));
+  alodlm_destroy(NULL);
+  return 0;
+}
+"""
+
+
+def test_plain_c_program_links_and_calls_the_library(L):
+    """The boundary is plain C: a C program compiled with gcc against include/alodlm.h links
+    libalodlm.so and gets clean errors (no GPU needed for argument validation)."""
+    lib_dir = os.path.dirname(L.LIB_PATH)
+    with tempfile.TemporaryDirectory() as d:
+        src, exe = os.path.join(d, "c.c"), os.path.join(d, "c")
+        open(src, "w").write(LINK_C)
+        subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), src, "-o", exe, "-L", lib_dir,
+                        "-l:libalodlm.so", f"-Wl,-rpath,{lib_dir}"], check=True)
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split("\n")
+    assert out[0] == "-1 1 msg"
+    assert out[1] == "-1"
+    assert out[2] == "attention"
