@@ -147,6 +147,14 @@ def commit_set(H: np.ndarray, a: np.ndarray, s: int, K: int, rule: int, tau: flo
     return (H <= tau) | (a >= lam) | (s == K)
 
 
+def halting_mean(a: np.ndarray, unresolved: np.ndarray) -> float:
+    """Step (4): the mean cumulative halt of the positions still unresolved after this loop's
+    commits.  The pages say "the unresolved positions" without fixing when; the reading taken
+    here is U once B^(s) has left it: positions committed in this or an earlier loop, and
+    given ids, do not count.  0 when U is empty."""
+    return float(np.mean(a[unresolved])) if unresolved.any() else 0.0
+
+
 def halts(n_left: int, mean_a_left: float, s: int, K: int, rule: int, lam: float) -> bool:
     """Step (4): the loop ends when nothing is unresolved, at s = K, or (PAPER) when the mean
     cumulative halt of the unresolved positions reaches the threshold."""
@@ -247,7 +255,7 @@ def replay_decisions(block_ids: np.ndarray, mask_id: int, entropy: np.ndarray, c
             U[idx[c]] = False
             n_commit += int(c.sum())
             left = np.nonzero(U)[0]
-            mean_a = float(np.mean(cum_halt[b, s - 1, left].astype(np.float64))) if len(left) else 0.0
+            mean_a = halting_mean(cum_halt[b, s - 1].astype(np.float64), U)
             if len(left) and rule == RULE_PAPER and abs(mean_a - float(lam32)) < mean_band:
                 ambiguous.append((b, s))
             if halts(len(left), np.float32(mean_a), s, K, rule, lam32):
@@ -651,7 +659,7 @@ class Oracle:
                 n_committed += len(ci)
                 h = self.merge(committed, tok, ht)
                 # (4) halting
-                mean_a = float(np.mean(a[U])) if U.any() else 0.0
+                mean_a = halting_mean(a, U)
                 stop = halts(int(U.sum()), mean_a, s, K, rule, lam)
                 if rule == RULE_PAPER and U.any() and s < K and near(mean_a, lam):
                     gpu = bool(follow["loops_run"][b] == s)

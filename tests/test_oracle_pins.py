@@ -746,3 +746,113 @@ def test_sampled_step_commits_the_same_positions_at_loop_one():
     np.testing.assert_array_equal(sm["exit_depth"][0] == 1, first)
     for i in np.nonzero(first)[0]:
         assert sm["tokens"][0, i] == om.gumbel_argmax(sm["logits"][(0, 1, int(i))], (42, 1), int(i), 1)
+
+
+# ------------------------------------------------------------------------------------
+# the halting criterion on hand-built traces ([digest] "Method steps", Algorithm 1 (3)-(4))
+# ------------------------------------------------------------------------------------
+
+def _scripted_step(H, lam_loop, tau, q, K, rule, monkeypatch):
+    """Run the oracle's denoise_step with every layer replaced by "row i -> basis vector e_i"
+    and the readout by a script: at loop s, position i has entropy H[s-1][i], gate output
+    lam_loop[s-1][i] and argmax token 10 + i.  Only the decision logic of the step is left."""
+    shape = small_shape()
+    o, _ = build(shape, K)
+    N = len(H[0])
+    o.kv = [{}]
+    o.prefix_len = 0
+    state = {"s": 0}
+
+    def layer(self, b, key, lw, h):
+        if key[0] == "core":
+            state["s"] = key[2]
+        out = np.zeros_like(h)
+        out[np.arange(N), np.arange(N)] = 1.0
+        return out
+
+    def readout(self, r):
+        pos = np.argmax(r, axis=1)
+        s = state["s"]
+        z = np.zeros((len(pos), shape.vocab))
+        z[np.arange(len(pos)), 10 + pos] = 5.0
+        return (np.array([H[s - 1][i] for i in pos], float), 10 + pos,
+                np.array([lam_loop[s - 1][i] for i in pos], float), z)
+
+    monkeypatch.setattr(om.Oracle, "block_layer", layer)
+    monkeypatch.setattr(om.Oracle, "readout", readout)
+    block = np.full((1, N), shape.mask_id, dtype=np.int32)
+    return o.denoise_step(block, tau, q, K, rule)
+
+
+# PAPER, K 4, tau 0.5, q 0.5.  Loop 1 commits position 0 (H 0.1); its a (0.95) must leave the
+# mean.  Mean over U after the commits: 0.4, 0.46, 0.568 -> the loop stops at s = 3.  Taken before
+# the commits are removed, loop 1's mean is (0.95 + 3 x 0.4) / 4 = 0.5375 -> stop at 1; over all
+# masked positions (committed ones kept at their last a), loop 2's is (0.95 + 3 x 0.46) / 4 =
+# 0.5825 -> stop at 2.
+HALT_H = [[0.1, 5, 5, 5], [9, 5, 5, 5], [9, 5, 5, 5], [9, 5, 5, 5]]
+HALT_LAM = [[0.95, 0.4, 0.4, 0.4], [0, 0.1, 0.1, 0.1], [0, 0.2, 0.2, 0.2], [0, 0.5, 0.5, 0.5]]
+
+
+def check_halting_mean(monkeypatch):
+    out = _scripted_step(HALT_H, HALT_LAM, 0.5, 0.5, 4, RULE_PAPER, monkeypatch)
+    assert out["loops_run"][0] == 3, out["loops_run"]
+    np.testing.assert_array_equal(out["exit_depth"][0], [1, 0, 0, 0])
+    np.testing.assert_array_equal(out["tokens"][0][:1], [10])
+    np.testing.assert_allclose(out["cum_halt"][0, 2, 1:], 1 - 0.6 * 0.9 * 0.8, rtol=1e-12)
+    # the same decisions re-taken from the traces
+    rep = om.replay_decisions(np.full((1, 4), small_shape().mask_id), small_shape().mask_id, out["entropy"],
+                              out["cum_halt"], lambda b, s, i: 10 + i, 0.5, 0.5, 4, RULE_PAPER)
+    assert rep["loops_run"][0] == 3
+    np.testing.assert_array_equal(rep["exit_depth"][0], [1, 0, 0, 0])
+
+
+def test_halting_mean_is_over_u_after_this_loops_commits(monkeypatch):
+    check_halting_mean(monkeypatch)
+
+
+def test_planted_halting_mean_before_commits_are_removed(monkeypatch):
+    monkeypatch.setattr(om, "halting_mean", _plant_population("before"))
+    with pytest.raises(AssertionError):
+        check_halting_mean(monkeypatch)
+
+
+def test_planted_halting_mean_over_all_masked_positions(monkeypatch):
+    monkeypatch.setattr(om, "halting_mean", _plant_population("all"))
+    with pytest.raises(AssertionError):
+        check_halting_mean(monkeypatch)
+
+
+def _plant_population(kind):
+    """A halting mean over the wrong population, recovered from the oracle's own state: the
+    loop's a holds a value for every position the loop read out (U before the commits) and
+    keeps the last value of positions committed earlier (all masked positions)."""
+    import inspect
+
+    def bad(a, unresolved):
+        frame = inspect.currentframe().f_back
+        loc = frame.f_locals
+        if kind == "before":
+            pop = unresolved.copy()
+            pop[loc["idx"]] = True          # this loop's readout rows, commits included
+        else:
+            pop = loc["block_ids"][loc["b"]] == loc["mask_id"]  # every masked position
+        return float(np.mean(a[pop])) if pop.any() else 0.0
+    return bad
+
+
+# PER_TOKEN, K 3, tau 0.5, lambda 0.5, no entropy passes tau.  a after loop 1: 0.6 (commits),
+# 0.3, 0.1, 0.1; after loop 2: 0.51 (commits), 0.19, 0.55 (commits); loop 3 = K commits the rest.
+# A test on the loop's own lambda instead of the cumulative a would commit position 1 at loop 3.
+TOK_H = [[5, 5, 5, 5]] * 3
+TOK_LAM = [[0.6, 0.3, 0.1, 0.1], [0, 0.3, 0.1, 0.5], [0, 0, 0.1, 0]]
+
+
+def test_per_token_rule_on_cumulative_halt_at_k3(monkeypatch):
+    out = _scripted_step(TOK_H, TOK_LAM, 0.5, 0.5, 3, RULE_PER_TOKEN, monkeypatch)
+    np.testing.assert_array_equal(out["exit_depth"][0], [1, 2, 3, 2])
+    np.testing.assert_array_equal(out["tokens"][0], [10, 11, 12, 13])
+    assert out["loops_run"][0] == 3
+    np.testing.assert_allclose(out["cum_halt"][0, 1, [1, 2, 3]], [0.51, 0.19, 0.55], rtol=1e-12)
+    rep = om.replay_decisions(np.full((1, 4), small_shape().mask_id), small_shape().mask_id, out["entropy"],
+                              out["cum_halt"], lambda b, s, i: 10 + i, 0.5, 0.5, 3, RULE_PER_TOKEN)
+    np.testing.assert_array_equal(rep["exit_depth"][0], [1, 2, 3, 2])
