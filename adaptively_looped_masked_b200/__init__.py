@@ -93,7 +93,7 @@ def lib() -> ctypes.CDLL:
         L.alodlm_kernel_class_name.argtypes = [ci]
         L.alodlm_kernel_class_name.restype = ctypes.c_char_p
         L.alodlm_gemm_bf16.argtypes = [vp, vp, vp, ci, ci, ci, vp, csz, vp]
-        L.alodlm_gemm_bf16_noalloc.argtypes = [vp, vp, vp, ci, ci, ci, vp]
+        L.alodlm_gemm_bf16_noalloc.argtypes = [vp, vp, vp, ci, ci, ci, vp, vp]
         for f in ("alodlm_create", "alodlm_prefill", "alodlm_denoise_step", "alodlm_sync", "alodlm_debug_state",
                   "alodlm_kv_slot", "alodlm_step_stats", "alodlm_set_timing", "alodlm_set_graphs",
                   "alodlm_gemm_bf16", "alodlm_gemm_bf16_noalloc"):
@@ -134,12 +134,16 @@ def gemm_bf16(A: torch.Tensor, W: torch.Tensor, out: Optional[torch.Tensor] = No
     return out
 
 
-def gemm_bf16_noalloc(A: torch.Tensor, W: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+def gemm_bf16_noalloc(A: torch.Tensor, W: torch.Tensor, out: torch.Tensor, status: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
     """C = A @ W^T through the allocation-free entry point (scratch compiled into the library).
-    ``out`` must be given: this call allocates nothing."""
+    ``out`` must be given: this call allocates nothing.  ``status`` (optional, device int32
+    [1]) receives the call's status word (non-zero: a bounded wait timed out, C invalid)."""
     M, K = A.shape
     N = W.shape[0]
-    rc = lib().alodlm_gemm_bf16_noalloc(_ptr(A), _ptr(W), _ptr(out), M, N, K, _stream_ptr(stream))
+    if status is not None and (status.dtype != torch.int32 or status.numel() < 1):
+        raise ValueError("status must be a device int32 tensor")
+    rc = lib().alodlm_gemm_bf16_noalloc(_ptr(A), _ptr(W), _ptr(out), M, N, K, _ptr(status), _stream_ptr(stream))
     if rc:
         raise AlodlmError(rc, lib().alodlm_last_error(None).decode())
     return out

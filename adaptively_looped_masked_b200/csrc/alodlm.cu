@@ -29,12 +29,6 @@ namespace {
 // the weights faster than the stream-K kernel at 32-64 rows (0.77 vs 0.65 of the measured
 // HBM bandwidth on the 24576 x 4096 gate/up shape).  The GEMM entry points use stream-K for
 // up to 64 rows.
-// Stream-K in the persistent GEMM: off by default.  It wins ~1% of the bs32 step (only O/down
-// at 1.3 waves qualify) and lost ~2.5% in block decoding; and it is the one place where a CTA
-// waits on another CTA of its grid, which relies on the whole grid being resident.
-#ifndef ALODLM_PERSIST_STREAM_K
-#define ALODLM_PERSIST_STREAM_K 0
-#endif
 #ifndef ALODLM_MAX_SPLITS
 #define ALODLM_MAX_SPLITS 8
 #endif
@@ -238,31 +232,15 @@ void launch_gemm_bn(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int
                 (const int *)nullptr, k_tiles, kps, a_fastest, tiled, ep, err);
 }
 
-// Stream-K (for the last wave and a half of tiles) pays when the tiles leave the last wave of a
-// one-CTA-per-SM grid well short of full: measured on B200 it wins at 1.3 waves (65% of the
-// last round busy) and loses its partial-tile traffic at 1.73 and 2.59 waves (87%).  It needs
-// at least one tile per CTA (a tile is then cut at most once), and the weight tiles of that
-// region plus the whole activation operand should stay in L2 while every CTA works on them.
-bool want_stream_k(int tiles, int grid, int n_b, int rowsB, int K) {
-    if (tiles < grid || tiles % grid == 0) return false;
-    const double waves = (double)tiles / grid;
-    if (waves / std::ceil(waves) >= 0.8) return false;
-    const int region = tiles - (tiles / grid - 1) * grid;
-    const double bytes = ((double)region / n_b + 1.0) * gemm::BM * K * 2.0 + (double)rowsB * K * 2.0;
-    return bytes <= 64.0e6;
-}
-
-// persistent kernel: one CTA per SM at most, walking the tiles (stream-K when `sk` and the
-// tile count fits the rule above; ep.ws / ep.counters then hold grid partial tiles / flags)
+// persistent kernel: one CTA per SM at most, walking whole tiles
 template <int BN, int EPI>
 void launch_persist(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int rowsB, const int *rowsA_dyn,
                     int k_tiles, int a_fastest, const gemm::EpiParams &ep, int *err, cudaStream_t st, int num_sms,
-                    int tiled, bool sk = false) {
+                    int tiled) {
     const int tiles = cdiv(rowsA, gemm::BM) * cdiv(rowsB, BN);
     const int grid = std::max(1, std::min(num_sms, tiles));
-    const int use_sk = sk && !rowsA_dyn && want_stream_k(tiles, grid, cdiv(rowsB, BN), rowsB, k_tiles * gemm::BK) ? 1 : 0;
     klaunch(gemm::gemm_persist_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM_PERSIST, st, tA, tB, rowsA, rowsB, rowsA_dyn,
-            k_tiles, a_fastest, tiled, use_sk, ep, err);
+            k_tiles, a_fastest, tiled, ep, err);
 }
 
 template <int EPI>
@@ -360,25 +338,20 @@ int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_b
     const CUtensorMap *tB = map_for_bn(g.bn);
     if (!tB) return -1;
     if (g.splits == 1 && g.bn >= 128) {
-        // stream-K partials: one BM x BN tile and one flag per CTA
-        ep.ws = env.ws;
-        ep.counters = env.counters;
-        const bool sk = ALODLM_PERSIST_STREAM_K && env.ws && env.counters && env.n_counters >= env.num_sms &&
-                        env.ws_floats >= (size_t)env.num_sms * gemm::BM * g.bn;
         auto go = [&](auto bn_tag) {
             constexpr int BN = decltype(bn_tag)::value;
             switch (epi) {
                 case gemm::EPI_F32:
                     launch_persist<BN, gemm::EPI_F32>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st,
-                                                      env.num_sms, w_tiled, sk);
+                                                      env.num_sms, w_tiled);
                     break;
                 case gemm::EPI_ADD:
                     launch_persist<BN, gemm::EPI_ADD>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st,
-                                                      env.num_sms, w_tiled, sk);
+                                                      env.num_sms, w_tiled);
                     break;
                 default:
                     launch_persist<BN, gemm::EPI_SWIGLU>(tmW, *tB, Nw, M, nullptr, g.k_tiles, 0, ep, env.err, env.st,
-                                                         env.num_sms, w_tiled, sk);
+                                                         env.num_sms, w_tiled);
                     break;
             }
         };
@@ -1124,7 +1097,14 @@ int alodlm_sync(alodlm_t *h) {
     e = cudaMemcpy(&dev_err, h->d_err, sizeof(int), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(h, e, "sync: read error word");
     if (dev_err) {
-        cudaMemset(h->d_err, 0, sizeof(int));
+        // A kernel that gave up may have left a split tile's arrival counter part-way (its
+        // epilogue skipped the increment): re-arm every counter, so that the next launch does
+        // not take a CTA for the last arriver too early.
+        cudaMemsetAsync(h->sk_counters, 0, SK_COUNTERS * sizeof(int), h->stream);
+        cudaMemsetAsync(h->attn_counters, 0, ATTN_COUNTERS * sizeof(int), h->stream);
+        cudaMemsetAsync(h->d_err, 0, sizeof(int), h->stream);
+        e = cudaStreamSynchronize(h->stream);
+        if (e != cudaSuccess) return cuda_fail(h, e, "sync: re-arm counters");
         if (dev_err & DEVERR_TIMEOUT) return fail(h, ALODLM_ETIMEOUT, "a bounded device wait timed out");
         return fail(h, ALODLM_EDEVICE, "a kernel flagged an out-of-range value (token id or exit depth)");
     }
@@ -1439,29 +1419,50 @@ constexpr size_t NOALLOC_FLOATS = NOALLOC_HEAD_FLOATS + NOALLOC_COUNTER_FLOATS +
 constexpr int NOALLOC_MAX_M = 64, NOALLOC_MAX_N = 32768, NOALLOC_MAX_K = 32768;
 
 std::mutex g_noalloc_mu;
+// per device: the context the address was looked up in, and the address
+CUcontext g_noalloc_ctx[64] = {nullptr};
 float *g_noalloc_addr[64] = {nullptr};
+
+// the driver's cuCtxGetCurrent, fetched through the runtime like the tensor-map encoder
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+CtxGetCurrentFn get_ctx_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    }
+    return fn;
+}
 }  // namespace
 
 static __device__ __align__(256) float g_noalloc_scratch[NOALLOC_FLOATS];
 
 extern "C" {
 
-int alodlm_gemm_bf16_noalloc(const void *A, const void *W, float *C, int M, int N, int K, void *stream) {
+int alodlm_gemm_bf16_noalloc(const void *A, const void *W, float *C, int M, int N, int K, int32_t *status,
+                             void *stream) {
     if (!A || !W || !C) return fail(nullptr, ALODLM_EINVAL, "gemm_bf16_noalloc: null pointer");
     if (M < 1 || M > NOALLOC_MAX_M || N < 1 || N > NOALLOC_MAX_N || K < 8 || K > NOALLOC_MAX_K || K % 8)
         return fail(nullptr, ALODLM_EINVAL,
                     "gemm_bf16_noalloc: needs 1 <= M <= 64, 1 <= N <= 32768, 8 <= K <= 32768, K % 8 == 0");
-    if (!get_encode_fn() || !init_kernel_attrs())
-        return fail(nullptr, ALODLM_ECUDA, "gemm_bf16_noalloc: tensor-map encoder or kernel attributes");
+    if (!get_encode_fn() || !init_kernel_attrs() || !get_ctx_fn())
+        return fail(nullptr, ALODLM_ECUDA, "gemm_bf16_noalloc: driver entry points or kernel attributes");
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return fail(nullptr, ALODLM_ECUDA, "gemm_bf16_noalloc: device index");
+    CUcontext ctx = nullptr;
+    if (get_ctx_fn()(&ctx) != CUDA_SUCCESS || !ctx)
+        return fail(nullptr, ALODLM_ECUDA, "gemm_bf16_noalloc: no current context");
     float *scratch = nullptr;
     {
-        // first call on this device: look up the device address of the scratch array (the
-        // array's name in host code is only a stand-in for it)
+        // first call on this device (or in a new context of it, e.g. after cudaDeviceReset):
+        // look up the device address of the scratch array -- its name in host code is only a
+        // stand-in for it
         std::lock_guard<std::mutex> lk(g_noalloc_mu);
-        if (!g_noalloc_addr[dev]) {
+        if (!g_noalloc_addr[dev] || g_noalloc_ctx[dev] != ctx) {
             void *p = nullptr;
             cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
             if (e != cudaSuccess) {
@@ -1470,6 +1471,7 @@ int alodlm_gemm_bf16_noalloc(const void *A, const void *W, float *C, int M, int 
                                                        cudaGetErrorString(e));
             }
             g_noalloc_addr[dev] = static_cast<float *>(p);
+            g_noalloc_ctx[dev] = ctx;
         }
         scratch = g_noalloc_addr[dev];
     }
@@ -1499,6 +1501,12 @@ int alodlm_gemm_bf16_noalloc(const void *A, const void *W, float *C, int M, int 
     launch_sk<gemm::EPI_F32>(plan, tW, tA, N, M, ep, env);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail(nullptr, ALODLM_ECUDA, std::string("gemm_bf16_noalloc: ") + cudaGetErrorString(e));
+    // hand the call's status word to the caller before the next call clears it
+    if (status) {
+        e = cudaMemcpyAsync(status, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess)
+            return fail(nullptr, ALODLM_ECUDA, std::string("gemm_bf16_noalloc: status copy: ") + cudaGetErrorString(e));
+    }
     return ALODLM_OK;
 }
 

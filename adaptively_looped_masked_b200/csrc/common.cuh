@@ -120,28 +120,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
     }
 }
 
-// Flag handshake between CTAs of one kernel (global memory, GPU scope).
-__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release_gpu(int *p, int v) {
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-// Wait until *flag == 1 (set by another resident CTA of the same kernel); false, with
-// DEVERR_TIMEOUT raised in *err, if that takes longer than WAIT_LIMIT_NS.
-__device__ __forceinline__ bool flag_wait(const int *flag, int *err) {
-    if (ld_acquire_gpu(flag) == 1) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (ld_acquire_gpu(flag) == 1) return true;
-        if ((it & 63u) == 0 && globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
-            atomicOr(err, DEVERR_TIMEOUT);
-            return false;
-        }
-    }
-}
 // named barrier of the 128 epilogue threads (warps 2-5) of a GEMM CTA
 __device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 // the same barrier, returning whether `p` holds in every one of the 128 threads

@@ -36,9 +36,6 @@ enum Epi { EPI_F32 = 0, EPI_ADD = 1, EPI_SWIGLU = 2, EPI_READOUT = 3 };
 struct EpiParams {
     float *out;           // EPI_F32 / EPI_ADD: out[b_row * ldo + a_row]
     int ldo;
-    long long split_stride;
-    float *ws;            // (stream-K kernel only) split partials
-    int *counters;        // (stream-K kernel only) per output tile, segments done (left at zero)
     bf16 *act;            // EPI_SWIGLU: act[b_row * ld_act + feature]
     int ld_act;
     float4 *partials;     // EPI_READOUT: partials[a_row * n_btiles + b_tile] = (max, sum e, sum e*d, argmax)
@@ -811,55 +808,14 @@ __device__ __forceinline__ void staged_cols(float *stg, const float (&v)[64], in
     epilogue_bar();  // the staging tile is free again
 }
 
-// One CTA's share of the work: segments (tile t, k-tiles [kb, ke)).  Plain persistent
-// schedule: whole tiles blockIdx.x, blockIdx.x + gridDim.x, ...  With stream-K (sk) only the
-// first W-1 of the W = total / gridDim.x full waves go that way; the remaining tiles (one full
-// wave plus the ragged rest, so at least one tile per CTA) have their k-iterations laid end to
-// end and cut into gridDim.x equal contiguous ranges.  Every CTA then streams the same number
-// of k-tiles, the tiles in flight at any time stay neighbours (their weight tiles are shared
-// through L2), and a tile is cut at most once: into a head [0, k) that ends one CTA's range
-// and a tail [k, K) that starts the next CTA's range.
-struct SegIter {
-    long long u = 0, u1 = 0;
-    int tnext, n_plain, k_tiles;
-    __device__ SegIter(bool sk, int total, int k_tiles_) : k_tiles(k_tiles_) {
-        tnext = blockIdx.x;
-        n_plain = total;
-        if (sk) {
-            n_plain = (total / (int)gridDim.x - 1) * (int)gridDim.x;
-            const long long U = (long long)(total - n_plain) * k_tiles_;
-            u = U * blockIdx.x / gridDim.x;
-            u1 = U * (blockIdx.x + 1) / gridDim.x;
-        }
-    }
-    __device__ bool next(int &t, int &kb, int &ke) {
-        if (tnext < n_plain) {
-            t = tnext;
-            kb = 0;
-            ke = k_tiles;
-            tnext += gridDim.x;
-            return true;
-        }
-        if (u >= u1) return false;
-        const int r = (int)(u / k_tiles);
-        t = n_plain + r;
-        kb = (int)(u - (long long)r * k_tiles);
-        ke = (int)min((long long)k_tiles, kb + (u1 - u));
-        u += ke - kb;
-        return true;
-    }
-};
-
-// Persistent kernel: at most one CTA per SM walks its segments with a double-buffered TMEM
-// accumulator, so the epilogue of one segment overlaps the MMAs of the next.  Under stream-K a
-// tail segment parks its partial tile in ep.ws (slot = this CTA, column-major) and raises
-// ep.counters[this CTA]; the CTA that ends with the head of the same tile (the previous CTA)
-// waits for the flag, adds head + tail in that order (deterministic), applies the epilogue and
-// lowers the flag again.  The grid never exceeds the SM count, so the CTAs are co-resident.
+// Persistent kernel: at most one CTA per SM walks whole output tiles blockIdx.x,
+// blockIdx.x + gridDim.x, ... with a double-buffered TMEM accumulator, so the epilogue of one
+// tile overlaps the MMAs of the next and the TMA ring streams across tile boundaries.  No CTA
+// waits on another CTA: every wait is on this CTA's own mbarriers.
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     gemm_persist_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int rowsA,
-                        int rowsB, const int *rowsA_dyn, int k_tiles, int a_fastest, int tiled, int sk, EpiParams ep,
+                        int rowsB, const int *rowsA_dyn, int k_tiles, int a_fastest, int tiled, EpiParams ep,
                         int *err) {
     using C = Cfg<BN>;
     constexpr int STAGES = C::STAGES;
@@ -870,8 +826,7 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t *empty = full + STAGES;
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + 2;
-    uint64_t *staged_bar = tempty + 2;  // stream-K head: the next CTA's partial has landed
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(staged_bar + 1);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
     float *stg = reinterpret_cast<float *>(smem + STAGES * C::STAGE_BYTES + 256);  // epilogue staging
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -884,7 +839,6 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(tfull + b, 1);
             mbar_init(tempty + b, 4);
         }
-        mbar_init(staged_bar, 1);
         fence_mbarrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
@@ -904,7 +858,6 @@ __global__ void __launch_bounds__(192, 1)
     }
     const int n_a = (rowsA + BM - 1) / BM, n_b = (rowsB + BN - 1) / BN;
     const int total = n_a * n_b;
-    const bool use_sk = sk && !rowsA_dyn && EPI != EPI_READOUT && total >= (int)gridDim.x;
     auto tile_of = [&](int t, int &a, int &b) {
         if (a_fastest) {
             a = t % n_a;
@@ -917,28 +870,26 @@ __global__ void __launch_bounds__(192, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            SegIter it(use_sk, total, k_tiles);
-            int t, kb, ke, a, b;
-            bool have = it.next(t, kb, ke);
+            int t = blockIdx.x, a = 0, b = 0;
             // weights (operand A of the linear layers) do not depend on earlier kernels: the
-            // first stages of the first segment are requested before waiting for them
+            // first stages of the first tile are requested before waiting for them
             int pre = 0;
-            if (have) {
+            if (t < total) {
                 tile_of(t, a, b);
-                pre = rowsA_dyn ? 0 : min(ke - kb, STAGES);
+                pre = rowsA_dyn ? 0 : min(k_tiles, STAGES);
                 for (int i = 0; i < pre; ++i) {
                     mbar_arrive_expect_tx(full + i, C::STAGE_BYTES);
-                    tma_operand(smem + i * C::STAGE_BYTES, &tmA, full + i, tiled & 1, a, BM, kb + i, k_tiles);
+                    tma_operand(smem + i * C::STAGE_BYTES, &tmA, full + i, tiled & 1, a, BM, i, k_tiles);
                 }
             }
             pdl_wait();
             for (int i = 0; i < pre; ++i)
-                tma_operand(smem + i * C::STAGE_BYTES + C::A_BYTES, &tmB, full + i, tiled & 2, b, BN, kb + i, k_tiles);
+                tma_operand(smem + i * C::STAGE_BYTES + C::A_BYTES, &tmB, full + i, tiled & 2, b, BN, i, k_tiles);
             int g = 0, issued = pre;
             bool ok = true;
-            for (; have && ok; have = it.next(t, kb, ke)) {
+            for (; t < total && ok; t += gridDim.x) {
                 tile_of(t, a, b);
-                for (int kt = kb; kt < ke; ++kt, ++g) {
+                for (int kt = 0; kt < k_tiles; ++kt, ++g) {
                     if (g < pre) continue;
                     const int s = g % STAGES;
                     if (!mbar_wait(empty + s, ((uint32_t)(g / STAGES) & 1u) ^ 1u, err)) {
@@ -958,14 +909,13 @@ __global__ void __launch_bounds__(192, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = umma_idesc_bf16(BM, BN);
-            SegIter it(use_sk, total, k_tiles);
-            int t, kb, ke, g = 0, li = 0;
+            int g = 0, li = 0;
             bool ok = true;
-            while (ok && it.next(t, kb, ke)) {
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++li) {
                 const int buf = li & 1;
                 if (!mbar_wait(tempty + buf, ((uint32_t)(li >> 1) & 1u) ^ 1u, err)) break;
                 tc_fence_after();
-                for (int kt = kb; kt < ke; ++kt, ++g) {
+                for (int kt = 0; kt < k_tiles; ++kt, ++g) {
                     const int s = g % STAGES;
                     if (!mbar_wait(full + s, (uint32_t)(g / STAGES) & 1u, err)) {
                         ok = false;
@@ -977,21 +927,18 @@ __global__ void __launch_bounds__(192, 1)
                     const uint64_t db = umma_sdesc_sw128(sa + C::A_BYTES);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        umma_f16(tmem_base + buf * BN, da + 2 * k, db + 2 * k, idesc, (kt > kb || k > 0) ? 1u : 0u);
+                        umma_f16(tmem_base + buf * BN, da + 2 * k, db + 2 * k, idesc, (kt > 0 || k > 0) ? 1u : 0u);
                     umma_commit(empty + s);
                 }
                 umma_commit(tfull + buf);
-                ++li;
             }
         }
     } else {
         const int q = warp & 3;
         const int row = q * 32 + lane;  // row of the tile = TMEM lane
         pdl_wait();
-        SegIter it(use_sk, total, k_tiles);
-        float *part = ep.ws + (size_t)blockIdx.x * BM * BN;  // this CTA's tail partial
-        int t, kb, ke, li = 0;
-        while (it.next(t, kb, ke)) {
+        int li = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++li) {
             int a, b;
             tile_of(t, a, b);
             const int buf = li & 1;
@@ -1001,63 +948,23 @@ __global__ void __launch_bounds__(192, 1)
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
             const int a_row = a * BM + row;
             const int b0 = b * BN;
-            const bool tail = kb > 0, head = kb == 0 && ke < k_tiles;
-            if (tail) {
-                // partial of k-tiles [kb, K): parked column-major (coalesced across lanes)
-                if (ready) {
+            if (ready) {
+                if constexpr (EPI == EPI_READOUT) {
+                    readout_tile<BN>(taddr, a_row, b0, b, rowsA, rowsB, ep);
+                } else {
+                    // rounds of 64 columns: one TMEM wait, then row-contiguous stores
                     for (int c0 = 0; c0 < BN; c0 += 64) {
+                        if (b0 + c0 >= rowsB) break;  // uniform across the epilogue warps
                         float v[64];
                         acc_ld<1, BN, 64>(taddr, c0, v);
-#pragma unroll
-                        for (int j = 0; j < 64; ++j) part[(size_t)(c0 + j) * BM + row] = v[j];
-                    }
-                }
-                epilogue_bar();
-                if (threadIdx.x == 64) {
-                    __threadfence();
-                    st_release_gpu(ep.counters + blockIdx.x, 1);
-                }
-            } else {
-                // head: the rest of this tile is the first segment of the next CTA; its partial
-                // is bulk-copied into the stage ring (idle now: the head is this CTA's last
-                // segment and its MMAs are complete)
-                const float *staged = reinterpret_cast<const float *>(smem);
-                if (head) {
-                    if (threadIdx.x == 64) {
-                        flag_wait(ep.counters + blockIdx.x + 1, err);
-                        __threadfence();
-                        ep.counters[blockIdx.x + 1] = 0;
-                        fence_proxy_async_all();
-                        constexpr uint32_t BYTES = BM * BN * 4, PIECE = 32768;
-                        const uint8_t *src = reinterpret_cast<const uint8_t *>(ep.ws + (size_t)(blockIdx.x + 1) * BM * BN);
-                        mbar_arrive_expect_tx(staged_bar, BYTES);
-                        for (uint32_t o = 0; o < BYTES; o += PIECE) bulk_load(smem + o, src + o, PIECE, staged_bar);
-                    }
-                    mbar_wait(staged_bar, 0, err);  // at most one head per CTA: phase 0
-                }
-                if (ready) {
-                    if constexpr (EPI == EPI_READOUT) {
-                        readout_tile<BN>(taddr, a_row, b0, b, rowsA, rowsB, ep);
-                    } else {
-                        // rounds of 64 columns: one TMEM wait, then row-contiguous stores
-                        for (int c0 = 0; c0 < BN; c0 += 64) {
-                            if (b0 + c0 >= rowsB) break;  // uniform across the epilogue warps
-                            float v[64];
-                            acc_ld<1, BN, 64>(taddr, c0, v);
-                            if (head) {
-#pragma unroll
-                                for (int j = 0; j < 64; ++j) v[j] += staged[(size_t)(c0 + j) * BM + row];
-                            }
-                            staged_cols<EPI>(stg, v, row, a, b0 + c0, rowsA, rowsB, ep);
-                        }
+                        staged_cols<EPI>(stg, v, row, a, b0 + c0, rowsA, rowsB, ep);
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty + buf);
-            ++li;
-            if (!ready) break;  // uniform: a stream-K partner waiting on us gives up after its bound
+            if (!ready) break;
         }
     }
     tc_fence_before();

@@ -222,8 +222,10 @@ ALODLM_API const char *alodlm_kernel_class_name(int k);
  * device status word (non-zero after a call means a bounded wait inside the kernel timed out
  * and C is invalid; the caller clears it); then come per-tile counters and split partials.
  * With too little room for the split the heuristic picks, fewer splits are used (and no
- * stream-K balancing, which needs one 128 x BN f32 tile per SM).  Partial
- * sums are added in a fixed order, so results are deterministic.  Runs on `stream` of the
+ * stream-K balancing, which needs one 128 x BN f32 tile per SM).  After a call that left the
+ * status word non-zero, zero the whole workspace again (a timed-out split may have left its
+ * tile counter part-way).  Partial sums are added in a fixed order, so results are
+ * deterministic.  Runs on `stream` of the
  * current device and allocates nothing.  For kernel-level tests and benchmarks.
  * Errors: EINVAL, ECUDA. */
 ALODLM_API int alodlm_gemm_bf16(const void *A, const void *W, float *C, int M, int N, int K, float *workspace,
@@ -242,13 +244,17 @@ ALODLM_API int alodlm_gemm_bf16(const void *A, const void *W, float *C, int M, i
  * Limits: 1 <= M <= 64, 1 <= N <= 32768, 8 <= K <= 32768, K % 8 == 0; outside them (or if
  * the split of a shape would not fit the array) it returns EINVAL, reason in
  * alodlm_last_error(NULL).
- * The first call on a device looks up the array's device address with that device
- * current; make that first call before any stream capture.  Every call shares the one
- * array: each call clears its status word and counters on `stream` before the kernel, and
- * calls that overlap on the GPU (other streams, other host threads) race and corrupt each
- * other's results — serialise them.  A bounded wait that times out inside the kernel leaves C
- * invalid and is not reported.  Errors: EINVAL, ECUDA. */
-ALODLM_API int alodlm_gemm_bf16_noalloc(const void *A, const void *W, float *C, int M, int N, int K, void *stream);
+ * status: NULL, or a caller-owned device int32 that receives this call's status word after
+ * the kernel (on `stream`): 0, or non-zero if a bounded wait inside the kernel timed out, in
+ * which case C is invalid.
+ * The first call on a device (and the first call after the device's context changed, e.g.
+ * after cudaDeviceReset) looks up the array's device address with that device current; make
+ * that first call before any stream capture.  Every call shares the one array: each call
+ * clears its status word and counters on `stream` before the kernel, and calls that overlap
+ * on the GPU (other streams, other host threads) race and corrupt each other's results --
+ * serialise them.  Errors: EINVAL, ECUDA. */
+ALODLM_API int alodlm_gemm_bf16_noalloc(const void *A, const void *W, float *C, int M, int N, int K, int32_t *status,
+                                        void *stream);
 
 #ifdef __cplusplus
 }
