@@ -191,14 +191,56 @@ def step_roofline(m, B, P, N, active_rows, readout_rows, peaks):
     return t, total_f, total_b
 
 
+# DRAM traffic of the GEMM class per launch, from an ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum over every GEMM launch of one step), keyed by workload and by a hash of
+# the GEMM kernel source it was taken on: a changed kernel reports null until captured again.
+GEMM_TRAFFIC = {}
+
+
+def gemm_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm_tc.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "adaptively_looped_masked_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def gemm_traffic_per_launch(workload, launches):
+    rec = GEMM_TRAFFIC.get(workload)
+    if rec is None or rec["source"] != gemm_source_hash():
+        return None
+    return rec["bytes_per_launch"]
+
+
 # ------------------------------------------------------------------------------------
 # CPU baseline: the oracle on a bounded sample
 # ------------------------------------------------------------------------------------
 
+# Loop profile of each workload's step (tau 0.6, lambda 0.5, the paper's rule) as the GPU arm
+# measured it: loops run per sequence and tokens committed per step.  The reference arm runs
+# without the GPU arm's results and scales its per-layer timing by this profile.
+GPU_LOOP_PROFILE = {
+    "qwen3-8b-bs32": dict(loops=[3, 3, 2, 3, 2, 6, 5, 3, 3, 4, 3, 6, 3, 3, 3, 2, 2, 2, 2, 5, 4, 4, 2, 5, 5, 3, 2,
+                                 3, 3, 5, 4, 4], commits=1654),
+}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        nt = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if nt:
+            return int(nt[0])
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
 def cpu_sample(m, wl, loops_per_seq, commits_per_step, w_dev, budget_s=20.0):
     """Time the oracle (as it stands) on one sequence: one Core layer over the block against a
     prefix-sized KV context and one readout of the block; scale to a whole step of the
-    workload using the loops the GPU ran."""
+    workload using the given loop profile (an extrapolation: no whole step is run)."""
     from oracle import Oracle
     from synth import weights_to_numpy
     from tests.helpers import oracle_cfg
@@ -227,15 +269,8 @@ def cpu_sample(m, wl, loops_per_seq, commits_per_step, w_dev, budget_s=20.0):
     CD = m.n_core + m.n_coda
     per_seq = [m.n_prelude * t_layer + L * (CD * t_layer + t_read) for L in loops_per_seq]
     t_step = float(sum(per_seq))
-    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    try:
-        from threadpoolctl import threadpool_info
-        nt = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
-        if nt:
-            cores = int(nt[0])
-    except Exception:
-        pass
-    return dict(value=commits_per_step / t_step, unit="tokens/s", cores=cores, kind="oracle",
+    return dict(value=commits_per_step / t_step, unit="tokens/s", cores=blas_threads(), kind="oracle",
+                extrapolated=True,
                 sample=(f"oracle float64, one sequence: one Core layer over the {N}-row block against a "
                         f"{P}-position KV context ({t_layer:.2f} s) and one {m.vocab}-vocab readout of the block "
                         f"({t_read:.2f} s), scaled to the step's {sum(loops_per_seq)} sequence-loops "
@@ -243,9 +278,180 @@ def cpu_sample(m, wl, loops_per_seq, commits_per_step, w_dev, budget_s=20.0):
                 seconds_per_step=t_step)
 
 
+def time_oracle_step(o, block, tau, lam, k_max, rule, threads=None):
+    """Wall time of one whole oracle denoise_step (prefix KV already in the oracle), with the BLAS
+    pool limited to `threads` (None: as configured).  Returns (seconds, committed, threads used)."""
+    from threadpoolctl import threadpool_limits
+    if threads is None:
+        t0 = time.perf_counter()
+        out = o.denoise_step(block, tau, lam, k_max, rule)
+        dt = time.perf_counter() - t0
+        used = blas_threads()
+    else:
+        with threadpool_limits(limits=threads, user_api="blas"):
+            t0 = time.perf_counter()
+            out = o.denoise_step(block, tau, lam, k_max, rule)
+            dt = time.perf_counter() - t0
+            used = threads
+    return dt, int((out["exit_depth"] > 0).sum()), used
+
+
+def kv_from_handle(handle, m, k_max, b, P):
+    """Sequence b's prefix KV cache read from a library handle, in the oracle's layout."""
+    keys = [(("prelude", l), l) for l in range(m.n_prelude)]
+    keys += [(("core", c, d), m.n_prelude + (d - 1) * m.n_core + c) for d in range(1, k_max + 1)
+             for c in range(m.n_core)]
+    keys += [(("coda", j), m.n_prelude + k_max * m.n_core + j) for j in range(m.n_coda)]
+    out = {}
+    for key, slot in keys:
+        kk = handle.kv_slot(0, slot, b, P).double().cpu().numpy().transpose(1, 0, 2)
+        vv = handle.kv_slot(1, slot, b, P).double().cpu().numpy().transpose(1, 0, 2)
+        out[key] = (kk, vv)
+    return out
+
+
+def cpu_measured_steps(tau, lam, rule, handle_17=None, w_17=None, one_core_budget_s=40.0):
+    """Whole oracle denoise_steps (float64, as it stands) timed on the host cores, all cores
+    and one core: the tiny config (the oracle's own prefill, untimed) and, when a 1.7B handle
+    is given, one 1.7B bs 1 sequence whose prefix KV is read from that handle (the oracle's
+    prefill at this size alone would take minutes)."""
+    from oracle import Oracle
+    from synth import weights_to_numpy
+    from tests.helpers import oracle_cfg
+    res = []
+    wl = WORKLOADS["tiny"]
+    m = MODELS["tiny"]
+    o = Oracle(oracle_cfg(m, wl.k_max), weights_to_numpy(make_weights(m, seed=0)), precision="fp64")
+    o.prefill(make_prefix_ids(m, wl.batch, wl.prefix))
+    blk = make_block_ids(m, wl.batch, wl.block)
+    time_oracle_step(o, blk, tau, lam, wl.k_max, rule, None)  # untimed: the oracle's per-layer weight cache fills
+    for threads in (None, 1):
+        dt, c, used = time_oracle_step(o, blk, tau, lam, wl.k_max, rule, threads)
+        res.append(dict(workload="tiny", cores=used, seconds=dt, committed=c, value=c / dt, unit="tokens/s"))
+    if handle_17 is not None:
+        wl = WORKLOADS["qwen3-1.7b-bs1"]
+        m = MODELS[wl.model]
+        o = Oracle(oracle_cfg(m, wl.k_max), weights_to_numpy(w_17), precision="fp64")
+        o.kv = [kv_from_handle(handle_17, m, wl.k_max, 0, wl.prefix)]
+        o.prefix_len = wl.prefix
+        blk = make_block_ids(m, 1, wl.block)
+        dt, c, used = time_oracle_step(o, blk, tau, lam, wl.k_max, rule, None)
+        res.append(dict(workload=wl.name, cores=used, seconds=dt, committed=c, value=c / dt, unit="tokens/s",
+                        prefix_kv="read from the library's arena"))
+        if dt * used <= one_core_budget_s * 4:
+            dt, c, used = time_oracle_step(o, blk, tau, lam, wl.k_max, rule, 1)
+            res.append(dict(workload=wl.name, cores=used, seconds=dt, committed=c, value=c / dt, unit="tokens/s",
+                            prefix_kv="read from the library's arena"))
+    return res
+
+
 # ------------------------------------------------------------------------------------
 # our arm
 # ------------------------------------------------------------------------------------
+
+def measure_step(handle, m, wl, block_np, tau, lam, rule, steps, warmup, world, local, peaks, stream,
+                 classes=True, e2e=True, clocks=True):
+    """Time `steps` denoising steps of the handle (inputs resident, CUDA events on the handle's
+    stream, barrier + synchronize on both sides), then optionally the per-kernel-class device
+    times and the end-to-end figure through the public API with host buffers."""
+    block = torch.tensor(block_np, device="cuda")
+    out = handle.alloc_outputs(wl.batch, wl.block, wl.k_max)
+    res = {}
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            handle.denoise_step(block, tau, lam, wl.k_max, rule, out=out)
+        handle.sync()
+        commits = int((out["exit_depth"] > 0).sum().item())
+        res.update(commits=commits, loops=out["loops_run"].cpu().tolist(),
+                   active_rows=out["active_rows"].cpu().tolist(), readout_rows=out["readout_rows"].cpu().tolist())
+        clk = ClockSampler(local) if clocks else None
+        if clk:
+            clk.start()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            handle.denoise_step(block, tau, lam, wl.k_max, rule, out=out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        res["clocks"] = clk.stop() if clk else None
+        handle.sync()
+        res["ms"] = e0.elapsed_time(e1)
+        res["launches_per_step"] = handle.step_stats()["launches"]
+        assert int((out["exit_depth"] > 0).sum().item()) == commits, "every timed step commits the same tokens"
+
+        if classes:
+            handle.set_timing(True)
+            prof_steps = max(1, min(steps, 5))
+            cls = {}
+            for _ in range(prof_steps):
+                handle.denoise_step(block, tau, lam, wl.k_max, rule, out=out)
+                for k_, v in handle.step_stats()["classes"].items():
+                    c = cls.setdefault(k_, dict(ms=0.0, launches=0, bytes=0.0, flops=0.0))
+                    for f in c:
+                        c[f] += v[f]
+            handle.set_timing(False)
+            res["classes"] = {k_: {f: v / prof_steps for f, v in c.items()} for k_, c in cls.items()}
+
+        if e2e:
+            ids_host = torch.tensor(block_np).pin_memory()
+            host_out = {k_: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k_, v in out.items()}
+            dev_ids = torch.empty_like(block)
+            res["h2d"] = ids_host.numel() * 4
+            res["d2h"] = sum(v.numel() * v.element_size() for v in host_out.values())
+            barrier(world)
+            torch.cuda.synchronize()
+            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            for _ in range(steps):
+                dev_ids.copy_(ids_host, non_blocking=True)
+                handle.denoise_step(dev_ids, tau, lam, wl.k_max, rule, out=out)
+                for k_, v in out.items():
+                    host_out[k_].copy_(v, non_blocking=True)
+            f1.record(stream)
+            torch.cuda.synchronize()
+            barrier(world)
+            res["e2e_ms"] = f0.elapsed_time(f1)
+    t_roof, F, Bt = step_roofline(m, wl.batch, wl.prefix, wl.block, res["active_rows"], res["readout_rows"], peaks)
+    res["t_roof"], res["F"], res["B"] = t_roof, F, Bt
+    res["tensor_bound"] = (F / (peaks["bf16_tflops_sustained"] * 1e12)) > (Bt / (peaks["hbm_gbs"] * 1e9))
+    return res
+
+
+def step_summary(name, wl, r, steps, world):
+    """The secondary-workload record: the same figures as the headline, one workload."""
+    ms_step = r["ms"] / steps
+    d = {"workload": name, "value": r["commits"] / (ms_step / 1e3), "unit": "tokens/s", "ms_per_step": ms_step,
+         "committed_per_step": r["commits"], "loops_run": r["loops"], "active_rows": r["active_rows"],
+         "readout_rows": r["readout_rows"],
+         "step_roofline": {"t_roof_ms": r["t_roof"] * 1e3, "frac": r["t_roof"] * 1e3 / ms_step,
+                           "bound": "tensor" if r["tensor_bound"] else "hbm"},
+         "config": {"model": wl.model, "batch": wl.batch, "prefix": wl.prefix, "block": wl.block, "k_max": wl.k_max,
+                    "mixed_exit_depths": wl.mixed_exit_depths},
+         "clocks": r.get("clocks"), "gpu_launches_per_step": r["launches_per_step"]}
+    if "e2e_ms" in r:
+        d["e2e"] = {"value": r["commits"] * steps / (r["e2e_ms"] / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]}
+    if "classes" in r:
+        tot = max(sum(v["ms"] for v in r["classes"].values()), 1e-9)
+        d["kernel_time_share"] = {k_: round(v["ms"] / tot, 4) for k_, v in r["classes"].items()}
+    return d
+
+
+def make_handle(alo, m, wl, w, stream, rank):
+    handle = alo.Handle(m, w, k_max=wl.k_max, max_batch=wl.batch, max_prefix=wl.prefix, max_block=wl.block,
+                        stream=stream)
+    prefix = torch.tensor(make_prefix_ids(m, wl.batch, wl.prefix, seed=1 + rank), device="cuda")
+    exit_depth = None
+    if wl.mixed_exit_depths:
+        exit_depth = torch.tensor(make_exit_depths(wl.batch, wl.prefix, wl.k_max, seed=2 + rank), device="cuda")
+    t0 = time.time()
+    handle.prefill(prefix, exit_depth)
+    handle.sync()
+    return handle, time.time() - t0
+
 
 def run_ours(args, world, rank, local):
     import adaptively_looped_masked_b200 as alo
@@ -254,114 +460,39 @@ def run_ours(args, world, rank, local):
     peaks, peaks_src = load_peaks()
     stream = torch.cuda.Stream()
     w = make_weights(m, seed=0, device="cuda")
-    handle = alo.Handle(m, w, k_max=wl.k_max, max_batch=wl.batch, max_prefix=wl.prefix, max_block=wl.block,
-                        stream=stream)
-    keep_w = w if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
-    del w
+    handle, prefill_s = make_handle(alo, m, wl, w, stream, rank)
     torch.cuda.empty_cache()
-    prefix = torch.tensor(make_prefix_ids(m, wl.batch, wl.prefix, seed=1 + rank), device="cuda")
-    exit_depth = None
-    if wl.mixed_exit_depths:
-        exit_depth = torch.tensor(make_exit_depths(wl.batch, wl.prefix, wl.k_max, seed=2 + rank), device="cuda")
-    t0 = time.time()
-    handle.prefill(prefix, exit_depth)
-    handle.sync()
-    prefill_s = time.time() - t0
     block_np = make_block_ids(m, wl.batch, wl.block)
-    block = torch.tensor(block_np, device="cuda")
-    out = handle.alloc_outputs(wl.batch, wl.block, wl.k_max)
     tau, lam, rule = args.tau, args.lam, args.rule
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            handle.denoise_step(block, tau, lam, wl.k_max, rule, out=out)
-        handle.sync()
-        commits = int((out["exit_depth"] > 0).sum().item())
-        loops = out["loops_run"].cpu().tolist()
-        active_rows = out["active_rows"].cpu().tolist()
-        readout_rows = out["readout_rows"].cpu().tolist()
+    r = measure_step(handle, m, wl, block_np, tau, lam, rule, args.steps, args.warmup, world, local, peaks, stream)
 
-        # ---- timed region (device events on the handle's stream) ----
-        clocks = ClockSampler(local)
-        clocks.start()
-        barrier(world)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            handle.denoise_step(block, tau, lam, wl.k_max, rule, out=out)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier(world)
-        clk = clocks.stop()
-        handle.sync()
-        ms = e0.elapsed_time(e1)
-        launches_per_step = handle.step_stats()["launches"]
-        commits_last = int((out["exit_depth"] > 0).sum().item())
-        assert commits_last == commits, "the step is deterministic: every timed step commits the same tokens"
-
-        # ---- per-kernel-class device time (separate pass with event records between launches) ----
-        handle.set_timing(True)
-        prof_steps = max(1, min(args.steps, 5))
-        cls_ms, cls_n, cls_b, cls_f = {}, {}, {}, {}
-        for _ in range(prof_steps):
-            handle.denoise_step(block, tau, lam, wl.k_max, rule, out=out)
-            st = handle.step_stats()
-            for k_, v in st["classes"].items():
-                cls_ms[k_] = cls_ms.get(k_, 0.0) + v["ms"]
-                cls_n[k_] = cls_n.get(k_, 0) + v["launches"]
-                cls_b[k_] = cls_b.get(k_, 0.0) + v["bytes"]
-                cls_f[k_] = cls_f.get(k_, 0.0) + v["flops"]
-        handle.set_timing(False)
-
-        # ---- end to end through the public API with host buffers ----
-        ids_host = torch.tensor(block_np).pin_memory()
-        host_out = {k_: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k_, v in out.items()}
-        dev_ids = torch.empty_like(block)
-        h2d = ids_host.numel() * 4
-        d2h = sum(v.numel() * v.element_size() for v in host_out.values())
-        barrier(world)
-        torch.cuda.synchronize()
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for _ in range(args.steps):
-            dev_ids.copy_(ids_host, non_blocking=True)
-            handle.denoise_step(dev_ids, tau, lam, wl.k_max, rule, out=out)
-            for k_, v in out.items():
-                host_out[k_].copy_(v, non_blocking=True)
-        f1.record(stream)
-        torch.cuda.synchronize()
-        barrier(world)
-        e2e_ms = f0.elapsed_time(f1)
-
-    max_ms = all_max(ms, world)
-    max_e2e = all_max(e2e_ms, world)
-    total_commits = all_sum(float(commits) * args.steps, world)
+    max_ms = all_max(r["ms"], world)
+    max_e2e = all_max(r["e2e_ms"], world)
+    total_commits = all_sum(float(r["commits"]) * args.steps, world)
     value = total_commits / (max_ms / 1e3)
     e2e_value = total_commits / (max_e2e / 1e3)
     ms_step = max_ms / args.steps
 
-    # roofline of the dominant kernel class
-    dom = max(cls_ms, key=lambda k_: cls_ms[k_])
-    g_ms = cls_ms["gemm"] / prof_steps
-    g_launch = cls_n["gemm"] / prof_steps
-    g_b = cls_b["gemm"] / prof_steps
-    g_f = cls_f["gemm"] / prof_steps
-    t_roof, F_step, B_step = step_roofline(m, wl.batch, wl.prefix, wl.block, active_rows, readout_rows, peaks)
-    tensor_bound = (F_step / (peaks["bf16_tflops_sustained"] * 1e12)) > (B_step / (peaks["hbm_gbs"] * 1e9))
+    # roofline of the dominant kernel class (the tcgen05 linear layers)
+    cls = r["classes"]
+    dom = max(cls, key=lambda k_: cls[k_]["ms"])
+    g = cls["gemm"]
+    tensor_bound = r["tensor_bound"]
     if tensor_bound:
-        achieved = g_f / (g_ms / 1e3) / 1e12
+        achieved = g["flops"] / (g["ms"] / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
-        roof = dict(bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s", frac=achieved / peak,
-                    traffic=None)
+        roof = dict(bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s", frac=achieved / peak)
     else:
-        achieved = g_b / (g_ms / 1e3) / 1e9
+        achieved = g["bytes"] / (g["ms"] / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
-        roof = dict(bound="hbm", achieved=achieved, peak=peak, unit="GB/s", frac=achieved / peak, traffic=None)
+        roof = dict(bound="hbm", achieved=achieved, peak=peak, unit="GB/s", frac=achieved / peak)
+    roof["traffic"] = gemm_traffic_per_launch(args.workload, g["launches"])
     roof.update(kernel="gemm (tcgen05 linear layers, incl. split-K reduce)", peak_source=peaks_src,
-                launches_per_step=g_launch, ms_per_step=g_ms,
-                algorithmic_per_launch=(g_f / g_launch if tensor_bound else g_b / g_launch),
-                algorithmic_unit=("flop" if tensor_bound else "byte"))
-    kernel_share = {k_: round(v / max(sum(cls_ms.values()), 1e-9), 4) for k_, v in cls_ms.items()}
+                launches_per_step=g["launches"], ms_per_step=g["ms"],
+                algorithmic_per_launch=(g["flops"] / g["launches"] if tensor_bound else g["bytes"] / g["launches"]),
+                algorithmic_unit=("flop" if tensor_bound else "byte"),
+                algorithmic_bytes_per_launch=g["bytes"] / g["launches"])
+    kernel_share = {k_: round(v["ms"] / max(sum(c["ms"] for c in cls.values()), 1e-9), 4) for k_, v in cls.items()}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -373,23 +504,65 @@ def run_ours(args, world, rank, local):
                    "rule": ["paper", "per_token"][rule], "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (weights 16 GB + KV arena)"},
         "roofline": roof,
-        "step_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_step,
-                          "bound": "tensor" if tensor_bound else "hbm", "flops": F_step, "bytes": B_step},
-        "committed_per_step": commits, "loops_run": loops, "active_rows": active_rows,
-        "readout_rows": readout_rows, "per_sequence_tokens_per_s": value / (wl.batch * world),
-        "gpu_launches": launches_per_step * args.steps, "kernel_time_share": kernel_share,
+        "step_roofline": {"t_roof_ms": r["t_roof"] * 1e3, "frac": r["t_roof"] * 1e3 / ms_step,
+                          "bound": "tensor" if tensor_bound else "hbm", "flops": r["F"], "bytes": r["B"],
+                          "peak_source": peaks_src},
+        "committed_per_step": r["commits"], "loops_run": r["loops"], "active_rows": r["active_rows"],
+        "readout_rows": r["readout_rows"], "per_sequence_tokens_per_s": value / (wl.batch * world),
+        "gpu_launches": r["launches_per_step"] * args.steps, "kernel_time_share": kernel_share,
         "dominant_kernel_class": dom, "prefill_s": prefill_s,
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "clocks": clk,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "clocks": r["clocks"],
     }
+
+    if world == 1 and not args.no_extras:
+        # the pages' sweep: tau x lambda on the same workload, active-row fraction per loop
+        sweep = []
+        for t_ in wl.taus:
+            for l_ in wl.lambdas:
+                rs = measure_step(handle, m, wl, block_np, t_, l_, rule, 5, 3, world, local, peaks, stream,
+                                  classes=False, e2e=False, clocks=False)
+                ms_s = rs["ms"] / 5
+                BN = wl.batch * wl.block
+                sweep.append({"tau_H": t_, "lambda": l_, "value": rs["commits"] / (ms_s / 1e3), "ms_per_step": ms_s,
+                              "committed_per_step": rs["commits"], "mean_loops": float(np.mean(rs["loops"])),
+                              "active_row_fraction": [round(x / BN, 4) for x in rs["active_rows"]],
+                              "readout_row_fraction": [round(x / BN, 4) for x in rs["readout_rows"]],
+                              "step_roofline_frac": rs["t_roof"] * 1e3 / ms_s})
+        line["sweep"] = sweep
+    handle.close()
+    del handle
+    torch.cuda.empty_cache()
+
+    handle_17 = w_17 = None
+    if world == 1 and not args.no_extras:
+        # the other single-GPU configurations, each measured the same way
+        secondary = {}
+        for name in [n for n in ("qwen3-8b-bs1", "qwen3-1.7b-bs1", "qwen3-8b-long") if n != args.workload]:
+            wl2 = WORKLOADS[name]
+            m2 = MODELS[wl2.model]
+            w2 = w if wl2.model == wl.model else make_weights(m2, seed=0, device="cuda")
+            h2, p2 = make_handle(alo, m2, wl2, w2, stream, rank)
+            r2 = measure_step(h2, m2, wl2, make_block_ids(m2, wl2.batch, wl2.block), tau,
+                              wl2.lambdas[-1] if wl2.mixed_exit_depths else lam, rule, args.steps, args.warmup,
+                              world, local, peaks, stream)
+            secondary[name] = step_summary(name, wl2, r2, args.steps, world)
+            secondary[name]["prefill_s"] = p2
+            if name == "qwen3-1.7b-bs1" and rank == 0 and not args.no_cpu_baseline:
+                handle_17, w_17 = h2, w2
+            else:
+                h2.close()
+            torch.cuda.empty_cache()
+        line["secondary"] = secondary
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_sample(m, wl, loops, commits, keep_w)
-        line["cpu_baseline"] = {k_: cb[k_] for k_ in ("value", "unit", "cores", "kind", "sample")}
-    if args.secondary and world == 1:
-        line["secondary"] = args.secondary_result
+        cb = cpu_sample(m, wl, r["loops"], r["commits"], w)
+        line["cpu_baseline"] = {k_: cb[k_] for k_ in ("value", "unit", "cores", "kind", "sample", "extrapolated")}
+        line["cpu_baseline"]["measured_steps"] = cpu_measured_steps(tau, lam, rule, handle_17, w_17)
+    if handle_17 is not None:
+        handle_17.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
-    handle.close()
 
 
 def run_decode(args, world, rank, local):
@@ -485,16 +658,22 @@ def run_decode(args, world, rank, local):
 # ------------------------------------------------------------------------------------
 
 def run_reference(args, world, rank):
+    """The oracle, as it stands, on the host cores: each step times one Core layer and one
+    readout of one sequence and scales them to the workload's step by the loop profile the GPU
+    arm measured for it (GPU_LOOP_PROFILE), so the line is an extrapolation and says so."""
     if rank != 0:
         return
     wl = WORKLOADS[args.workload]
     m = MODELS[wl.model]
-    # one Core layer of weights on the host is all the sample needs
-    w = make_weights(m, seed=0, device="cuda" if torch.cuda.is_available() else "cpu")
-    # the GPU arm's loop count is not known here: take every sequence to loop 2 times and
-    # commit the whole block (an optimistic bound for the CPU side)
-    loops = [2] * wl.batch
-    commits = wl.batch * wl.block
+    # only the timed Core layer and the heads are generated
+    w = make_weights(m, seed=0, device="cuda" if torch.cuda.is_available() else "cpu", only_layers=[m.n_prelude])
+    prof = GPU_LOOP_PROFILE.get(args.workload)
+    if prof is not None:
+        loops, commits = prof["loops"], prof["commits"]
+        how = "loop profile of the GPU arm's measured step (loops per sequence, tokens committed)"
+    else:
+        loops, commits = [2] * wl.batch, wl.batch * wl.block
+        how = "no GPU loop profile recorded for this workload: 2 loops per sequence, whole block committed"
     vals = []
     t_all = time.perf_counter()
     for i in range(args.warmup + args.steps):
@@ -507,10 +686,12 @@ def run_reference(args, world, rank):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": statistics.median(v["seconds_per_step"] for v in vals) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": args.workload, "model": wl.model, "batch": wl.batch,
-                                            "prefix": wl.prefix, "block": wl.block, "k_max": wl.k_max},
+            "data": "synthetic", "extrapolated": True,
+            "config": {"workload": args.workload, "model": wl.model, "batch_per_gpu": wl.batch, "prefix": wl.prefix,
+                       "block": wl.block, "k_max": wl.k_max, "tau_H": args.tau, "lambda": args.lam,
+                       "rule": ["paper", "per_token"][args.rule]},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": vals[0]["cores"], "kind": "oracle",
-                             "sample": vals[0]["sample"] + "; loops per sequence assumed 2, whole block committed"},
+                             "extrapolated": True, "sample": vals[0]["sample"] + "; scaled with the " + how},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "wall_s": elapsed}
     print(json.dumps(line), flush=True)
@@ -562,6 +743,8 @@ def main():
     ap.add_argument("--lam", type=float, default=0.5)
     ap.add_argument("--rule", type=int, default=0, choices=[0, 1])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="headline workload only: no tau x lambda sweep and no secondary workloads")
     ap.add_argument("--decode", action="store_true",
                     help="time block decoding (steps until no [MASK]) instead of one step")
     ap.add_argument("--kernel", default=None, choices=["gemm"],
@@ -571,7 +754,6 @@ def main():
     if args.kernel == "gemm":
         run_kernel_gemm(args)
         return
-    args.secondary = None
     world, rank, local = dist_setup(args.gpus)
     try:
         if args.impl == "reference":

@@ -542,16 +542,20 @@ class Oracle:
     # --- the denoising step --------------------------------------------------------------
 
     def denoise_step(self, block_ids: np.ndarray, tau: float, lam: float, k_max: int,
-                     rule: int = RULE_PAPER, follow: Optional[dict] = None, band: float = 1e-3,
+                     rule: int = RULE_PAPER, follow: Optional[dict] = None, band=1e-3,
                      logit_rows: Optional[List[tuple]] = None, sample_key=None) -> dict:
         """One denoising step, [digest] "Method steps" Algorithm 1 (1)-(5) and Eq. 3.
 
         block_ids [B, N]; positions holding mask_id form U.  ``lam`` is the halting
         threshold (q in the pages).  ``follow`` (optional) holds another run's decisions
         {"tokens" [B,N], "exit_depth" [B,N], "loops_run" [B]}: at a decision whose deciding
-        value lies within ``band`` of its threshold (or whose top-two gap is below ``band``),
-        the oracle takes that run's decision and records it in "followed"; band=inf follows
-        every decision.  ``logit_rows``: (b, s, i) triples whose logits are returned.
+        value lies within the band of its threshold, the oracle takes that run's decision and
+        records it in "followed" (with its own decision and the margin).  ``band`` is one
+        number for every kind of decision, or a dict with keys "entropy" (a commit on H <= tau,
+        and the forced pick when the two lowest entropies are that close), "halt" (a decision
+        on a cumulative halt or its mean) and "argmax" (the top-two score gap; the other run's
+        token is taken only if its score lies within the band of the maximum).  band=inf
+        follows every decision.  ``logit_rows``: (b, s, i) triples whose logits are returned.
         ``sample_key`` (two integers): committed tokens are drawn from p_i^(s) by Gumbel-max
         (``gumbel_argmax`` at position b * N + i, loop s) instead of taken greedily.
 
@@ -577,8 +581,11 @@ class Oracle:
         want_logits = set(logit_rows or [])
         self.layer_execs = 0
 
-        def near(x, thr):
-            return follow is not None and abs(float(x) - float(thr)) < band
+        bands = band if isinstance(band, dict) else dict(entropy=band, halt=band, argmax=band)
+        band_h, band_a, band_z = float(bands["entropy"]), float(bands["halt"]), float(bands["argmax"])
+
+        def near(x, thr, width):
+            return follow is not None and abs(float(x) - float(thr)) < width
 
         for b in range(B):
             # (1) U = masked positions; h^(0) = Prelude(x); a = 0; C = empty
@@ -629,21 +636,23 @@ class Oracle:
                 if follow is not None:
                     for t in range(len(idx)):
                         top2 = np.partition(scores[t], -2)[-2:]
-                        if top2[1] - top2[0] < band:
-                            i = int(idx[t])
-                            if follow["exit_depth"][b, i] == s:
-                                out["followed"].append(dict(b=b, s=s, i=i, kind="argmax",
-                                                            margin=float(top2[1] - top2[0])))
-                                y[t] = int(follow["tokens"][b, i])
+                        i = int(idx[t])
+                        other = int(follow["tokens"][b, i])
+                        if (top2[1] - top2[0] < band_z and follow["exit_depth"][b, i] == s
+                                and 0 <= other < scores.shape[1] and scores[t][other] >= top2[1] - band_z):
+                            out["followed"].append(dict(b=b, s=s, i=i, kind="argmax",
+                                                        margin=float(top2[1] - top2[0]), own=int(y[t]),
+                                                        taken=other))
+                            y[t] = other
                 # (3) commit set B^(s)
                 commit = commit_set(H, a[idx], s, K, rule, tau, lam)
                 for t, i in enumerate(idx):
                     dec = bool(commit[t])
                     if rule == RULE_PAPER:
-                        is_near = near(H[t], tau)
+                        is_near = near(H[t], tau, band_h)
                         margin = H[t] - tau
                     else:
-                        is_near = s < K and (near(H[t], tau) or near(a[i], lam))
+                        is_near = s < K and (near(H[t], tau, band_h) or near(a[i], lam, band_a))
                         margin = min(abs(H[t] - tau), abs(a[i] - lam))
                     if is_near:
                         gpu = bool(follow["exit_depth"][b, i] == s)
@@ -661,7 +670,7 @@ class Oracle:
                 # (4) halting
                 mean_a = halting_mean(a, U)
                 stop = halts(int(U.sum()), mean_a, s, K, rule, lam)
-                if rule == RULE_PAPER and U.any() and s < K and near(mean_a, lam):
+                if rule == RULE_PAPER and U.any() and s < K and near(mean_a, lam, band_a):
                     gpu = bool(follow["loops_run"][b] == s)
                     out["followed"].append(dict(b=b, s=s, i=-1, kind="halt",
                                                 margin=float(mean_a - lam), own=stop, taken=gpu))
@@ -672,11 +681,13 @@ class Oracle:
             if rule == RULE_PAPER and n_committed == 0 and U.any():
                 cand = sorted(last_H.items(), key=lambda kv: (kv[1], kv[0]))
                 i_star = forced_pick(last_H)
-                if follow is not None and len(cand) > 1 and cand[1][1] - cand[0][1] < band:
-                    gpu_i = [i for i in last_H if follow["exit_depth"][b, i] == s_last]
-                    out["followed"].append(dict(b=b, s=s_last, i=int(i_star), kind="forced",
-                                                margin=float(cand[1][1] - cand[0][1])))
+                if follow is not None and len(cand) > 1 and cand[1][1] - cand[0][1] < band_h:
+                    gpu_i = [i for i in last_H if follow["exit_depth"][b, i] == s_last
+                             and last_H[i] <= cand[0][1] + band_h]
                     if gpu_i:
+                        out["followed"].append(dict(b=b, s=s_last, i=int(i_star), kind="forced",
+                                                    margin=float(cand[1][1] - cand[0][1]), own=int(i_star),
+                                                    taken=int(gpu_i[0])))
                         i_star = gpu_i[0]
                 z_star = self.readout(rs[-1][[i_star]])[3][0]
                 if sample_key is not None:
@@ -684,8 +695,12 @@ class Oracle:
                 y_star = int(np.argmax(z_star))
                 if follow is not None and follow["exit_depth"][b, i_star] == s_last:
                     top2 = np.partition(z_star, -2)[-2:]
-                    if top2[1] - top2[0] < band:
-                        y_star = int(follow["tokens"][b, i_star])
+                    other = int(follow["tokens"][b, i_star])
+                    if top2[1] - top2[0] < band_z and 0 <= other < z_star.shape[0] and \
+                            z_star[other] >= top2[1] - band_z:
+                        out["followed"].append(dict(b=b, s=s_last, i=int(i_star), kind="argmax",
+                                                    margin=float(top2[1] - top2[0]), own=y_star, taken=other))
+                        y_star = other
                 tok[i_star] = y_star
                 out["exit_depth"][b, i_star] = s_last
                 U[i_star] = False
@@ -701,7 +716,7 @@ class Oracle:
 
 def decode_block(oracle: Oracle, block_ids: np.ndarray, tau: float, lam: float, k_max: int,
                  rule: int = RULE_PAPER, max_steps: int = 0, follow_steps: Optional[List[dict]] = None,
-                 band: float = 1e-3, sample_seed: Optional[int] = None) -> dict:
+                 band=1e-3, sample_seed: Optional[int] = None) -> dict:
     """Denoising steps over one block until no [MASK] is left, [digest] "Method steps",
     Algorithm 1 (5): after each step the committed tokens are written into the sequence and
     the next denoising step starts, until no [MASK] remains.

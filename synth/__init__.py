@@ -133,7 +133,7 @@ def _normal(shape, std: float, seed: int, index: int, device) -> torch.Tensor:
     return torch.randn(shape, generator=g, device=device, dtype=torch.float32).mul_(std)
 
 
-def make_weights(m: ModelShape, seed: int = 0, device: str = "cpu") -> dict:
+def make_weights(m: ModelShape, seed: int = 0, device: str = "cpu", only_layers: Optional[List[int]] = None) -> dict:
     """Seeded random weights.
 
     Returns {"embed", "lm_head", "final_norm", "exit_w", "exit_b", "layers": [dict, ...]}.
@@ -142,23 +142,24 @@ def make_weights(m: ModelShape, seed: int = 0, device: str = "cpu") -> dict:
     drawn from its own generator seeded with (seed << 20) + t, so one tensor can be
     regenerated alone.  On "cpu" the stream is identical on every machine; on "cuda" it is
     the CUDA generator's stream (used for the 1.7B/8B shapes, whose host copy is taken
-    from the device tensors when needed).
+    from the device tensors when needed).  ``only_layers``: generate just these layers (the
+    others are None); each generated tensor is the same as in the full draw.
     """
     H = m.hidden
     mat_dtype = torch.bfloat16 if m.weight_dtype == "bf16" else torch.float32
     out: dict = {}
     idx = 0
 
-    def mat(shape, std):
+    def mat(shape, std, make=True):
         nonlocal idx
-        t = _normal(shape, std, seed, idx, device).to(mat_dtype)
+        t = _normal(shape, std, seed, idx, device).to(mat_dtype) if make else None
         idx += 1
         return t
 
-    def vec(shape, value):
+    def vec(shape, value, make=True):
         nonlocal idx
         idx += 1
-        return torch.full(shape, float(value), dtype=torch.float32, device=device)
+        return torch.full(shape, float(value), dtype=torch.float32, device=device) if make else None
 
     out["embed"] = mat((m.vocab, H), 0.02)
     out["lm_head"] = mat((m.vocab, H), 3.2 / math.sqrt(H))
@@ -167,17 +168,18 @@ def make_weights(m: ModelShape, seed: int = 0, device: str = "cpu") -> dict:
     out["exit_w"] = _normal((H,), 0.02 * math.sqrt(256.0 / H), seed, idx_exit, device)
     idx += 1
     out["exit_b"] = -1.0
-    layers: List[dict] = []
+    layers: List[Optional[dict]] = []
     shapes = layer_shapes(m)
-    for _ in range(m.n_layers):
+    for li in range(m.n_layers):
+        make = only_layers is None or li in only_layers
         lw = {}
         for key in LAYER_KEYS:
             shp = shapes[key]
             if len(shp) == 1:
-                lw[key] = vec(shp, 1.0)
+                lw[key] = vec(shp, 1.0, make)
             else:
-                lw[key] = mat(shp, 0.02)
-        layers.append(lw)
+                lw[key] = mat(shp, 0.02, make)
+        layers.append(lw if make else None)
     out["layers"] = layers
     return out
 

@@ -1,5 +1,28 @@
 """Helpers of the GPU tests: build a library handle and an oracle from the same seeded
-inputs, and compare a step's outputs with the oracle's."""
+inputs, and compare a step's outputs with the oracle's.
+
+Every tolerance and band below is a fixed number.
+
+Readout stage, on the GPU's own readout states r^(s), i.e. the same inputs on both sides:
+  ENTROPY_TOL  |dH| <= 1e-2 nats
+  GATE_TOL     |d lambda| <= 1e-3
+  BAND         the argmax must match unless the top-two logit gap is below 1e-3
+
+End to end, the float64 oracle running the whole step from the same ids and weights:
+  STATE_REL_TOL    per-row ||d|| / ||ref|| <= 2e-2 for h^(s-1), h~^(s), r^(s) and the logits
+  E2E_ENTROPY_TOL  |dH| <= 0.1 nats; also the band within which a commit on H <= tau may go
+                   either way
+  E2E_HALT_TOL     |d lambda|, |d a| <= 1e-2; also the band of decisions on a or on its mean
+  E2E_ARGMAX_BAND  top-two logit gap below which either token is a correct argmax (the GPU's
+                   token must then score within the band of the oracle's maximum)
+
+Outside those bands every decision (commit, exit depth, token, halt, forced pick) must be
+the oracle's own.  Why the end-to-end numbers are what they are: with bf16 activations,
+two correct implementations that round at the same points but add in a different order
+(the oracle itself in float32 and in float64) already drift apart end to end by up to
+0.05 nats at the synthetic configs' logit scale (logit std 12.8); the end-to-end bands
+are twice that spread.
+"""
 import numpy as np
 import torch
 
@@ -7,24 +30,31 @@ from oracle import Oracle
 from synth import MODELS, WORKLOADS, make_weights, weights_to_numpy, make_prefix_ids, make_block_ids
 from tests.helpers import oracle_cfg
 
-ENTROPY_TOL = 1e-2      # nats
-STATE_REL_TOL = 2e-2    # per-row ||d||/||ref|| of hidden / readout states
-GATE_TOL = 1e-2         # lambda and cumulative halt (absolute)
-BAND = 1e-3             # near-threshold band within which a decision is followed
+ENTROPY_TOL = 1e-2
+GATE_TOL = 1e-3
+BAND = 1e-3
+STATE_REL_TOL = 2e-2
+E2E_ENTROPY_TOL = 0.1
+E2E_HALT_TOL = 1e-2
+E2E_ARGMAX_BAND = 0.5
+E2E_BANDS = dict(entropy=E2E_ENTROPY_TOL, halt=E2E_HALT_TOL, argmax=E2E_ARGMAX_BAND)
 
 
 class Case:
     """One model + workload: device weights, a library handle, and host copies for the oracle."""
 
     def __init__(self, model: str, batch: int, prefix: int, block: int, k_max: int, debug=True, seed=0,
-                 stream=None):
+                 stream=None, weights=None):
         import adaptively_looped_masked_b200 as alo
         self.m = MODELS[model]
         self.batch, self.prefix, self.block, self.k_max = batch, prefix, block, k_max
         big = self.m.hidden >= 1024
-        self.w_dev = make_weights(self.m, seed=seed, device="cuda" if big else "cpu")
-        if not big:
-            self.w_dev = _to_cuda(self.w_dev)
+        if weights is not None:
+            self.w_dev = weights
+        else:
+            self.w_dev = make_weights(self.m, seed=seed, device="cuda" if big else "cpu")
+            if not big:
+                self.w_dev = _to_cuda(self.w_dev)
         self.stream = stream if stream is not None else torch.cuda.Stream()
         self.handle = alo.Handle(self.m, self.w_dev, k_max=k_max, max_batch=batch, max_prefix=prefix,
                                  max_block=block, debug_dump=debug, stream=self.stream)
@@ -54,6 +84,21 @@ class Case:
         self.handle.sync()
         return {kk: v.cpu().numpy() for kk, v in out.items()}
 
+    def kv_from_gpu(self, b: int, dtype=np.float32) -> dict:
+        """Sequence b's depth-aware KV cache as the oracle stores it, read from the library's
+        arena: {("prelude", l) | ("core", c, d) | ("coda", j): (K, V)}, each [P, nkv, hd]."""
+        m, K, P = self.m, self.k_max, self.prefix
+        keys = [(("prelude", l), l) for l in range(m.n_prelude)]
+        keys += [(("core", c, d), m.n_prelude + (d - 1) * m.n_core + c)
+                 for d in range(1, K + 1) for c in range(m.n_core)]
+        keys += [(("coda", j), m.n_prelude + K * m.n_core + j) for j in range(m.n_coda)]
+        out = {}
+        for key, slot in keys:
+            kk = self.handle.kv_slot(0, slot, b, P).float().cpu().numpy().transpose(1, 0, 2)
+            vv = self.handle.kv_slot(1, slot, b, P).float().cpu().numpy().transpose(1, 0, 2)
+            out[key] = (kk.astype(dtype), vv.astype(dtype))
+        return out
+
 
 def _to_cuda(w):
     out = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in w.items() if k != "layers"}
@@ -61,108 +106,125 @@ def _to_cuda(w):
     return out
 
 
-def follow_of(gpu: dict) -> dict:
-    return dict(tokens=gpu["tokens"], exit_depth=gpu["exit_depth"], loops_run=gpu["loops_run"])
+def follow_of(gpu: dict, seqs=None) -> dict:
+    sel = slice(None) if seqs is None else np.asarray(seqs)
+    return dict(tokens=gpu["tokens"][sel], exit_depth=gpu["exit_depth"][sel], loops_run=gpu["loops_run"][sel])
 
 
-
-
-def compare_decisions(gpu: dict, ref: dict):
-    """Tokens, exit depths, loops, row counters and the NaN pattern of the traces match exactly."""
+def compare_decisions(gpu: dict, ref: dict, rows=True):
+    """Tokens, exit depths, loops and the NaN pattern of the traces match exactly (and the
+    per-loop row counters, for a whole batch)."""
     np.testing.assert_array_equal(gpu["loops_run"], ref["loops_run"])
     np.testing.assert_array_equal(gpu["exit_depth"], ref["exit_depth"])
     np.testing.assert_array_equal(gpu["tokens"], ref["tokens"])
     np.testing.assert_array_equal(np.isnan(gpu["entropy"]), np.isnan(ref["entropy"]))
-    np.testing.assert_array_equal(gpu["active_rows"], ref["active_rows"])
-    np.testing.assert_array_equal(gpu["readout_rows"], ref["readout_rows"])
+    if rows:
+        np.testing.assert_array_equal(gpu["active_rows"], ref["active_rows"])
+        np.testing.assert_array_equal(gpu["readout_rows"], ref["readout_rows"])
 
 
 def row_rel_err(a: np.ndarray, ref: np.ndarray) -> np.ndarray:
     return np.linalg.norm(a - ref, axis=-1) / np.maximum(np.linalg.norm(ref, axis=-1), 1e-30)
 
 
-def readout_stage_check(case, gpu: dict, r_by_loop: dict):
+def readout_stage_check(case, gpu: dict, r_by_loop: dict, seqs=None, rows_per_loop=None, rng=None, ob=None):
     """Readout parity on the GPU's own readout states r^(s): the oracle's LM head + entropy +
     argmax + ExitGate in the kernels' precision.  Returns token_at(b, s, i) for the replay and
-    the max deviations."""
-    ob = case.oracle("bf16")
+    the max deviations.  rows_per_loop (optional) samples that many rows per (b, s)."""
+    ob = ob if ob is not None else case.oracle("bf16")
     toks, max_dH, max_dl, n_ties = {}, 0.0, 0.0, 0
     B, K, N = gpu["entropy"].shape
-    for b in range(B):
+    for b in (range(B) if seqs is None else seqs):
         for s in range(1, int(gpu["loops_run"][b]) + 1):
             idx = np.nonzero(~np.isnan(gpu["entropy"][b, s - 1]))[0]
             if len(idx) == 0:
                 continue
-            H, y, lam, z = ob.readout(r_by_loop[s][b][idx])
+            if rows_per_loop is not None and len(idx) > rows_per_loop:
+                idx = np.sort(rng.choice(idx, size=rows_per_loop, replace=False))
+            H, y, lam, z = ob.readout(r_by_loop[s][b][idx].astype(ob.dt))
             dH = np.abs(H - gpu["entropy"][b, s - 1, idx])
             dl = np.abs(lam - gpu["halt"][b, s - 1, idx])
             max_dH, max_dl = max(max_dH, float(dH.max())), max(max_dl, float(dl.max()))
             top2 = np.sort(z, axis=-1)[:, -2:]
             for t, i in enumerate(idx):
                 tok = int(y[t])
+                committed_here = gpu["exit_depth"][b, i] == s
                 if top2[t, 1] - top2[t, 0] < BAND:  # near tie: either id is a correct argmax
                     n_ties += 1
-                    if gpu["exit_depth"][b, i] == s and z[t, gpu["tokens"][b, i]] >= top2[t, 1] - BAND:
+                    if committed_here and z[t, gpu["tokens"][b, i]] >= top2[t, 1] - BAND:
                         tok = int(gpu["tokens"][b, i])
+                elif committed_here:
+                    assert gpu["tokens"][b, i] == tok, ("argmax", b, s, int(i))
                 toks[(b, s, int(i))] = tok
     assert max_dH <= ENTROPY_TOL, f"readout entropy |d| {max_dH}"
     assert max_dl <= GATE_TOL, f"exit gate |d| {max_dl}"
-    return (lambda b, s, i: toks[(b, s, i)]), dict(readout_dH=max_dH, readout_dlam=max_dl, argmax_ties=n_ties)
+
+    def token_at(b, s, i):
+        return toks.get((b, s, i), int(gpu["tokens"][b, i]))
+    return token_at, dict(readout_dH=max_dH, readout_dlam=max_dl, argmax_ties=n_ties)
 
 
 def step_parity(case, gpu: dict, tau: float, lam: float, K: int, rule: int, block_ids: np.ndarray,
-                states=True) -> dict:
-    """The three parity checks of one step (see tests/test_gpu_parity.py)."""
+                states=True, oracle=None, seqs=None, rows_per_loop=None, ob=None) -> dict:
+    """The three parity checks of one step (see tests/test_gpu_parity.py).
+
+    oracle: a float64 (or float32) oracle whose prefix KV is ready -- prefilled by the oracle
+    itself, or read from the library's arena; default: a float64 oracle prefilled here.
+    seqs: the sequences to check end to end (default all; the oracle then holds only these)."""
     from oracle.alodlm_oracle import replay_decisions
     B = block_ids.shape[0]
+    seq_list = list(range(B)) if seqs is None else [int(b) for b in seqs]
+    rng = np.random.default_rng(0)
     r_by_loop = {s: case.handle.debug_state(2, s).cpu().numpy() for s in range(1, int(gpu["loops_run"].max()) + 1)}
     # (1) readout stage on the GPU's own r
-    token_at, stats = readout_stage_check(case, gpu, r_by_loop)
+    token_at, stats = readout_stage_check(case, gpu, r_by_loop, seqs=seq_list, rows_per_loop=rows_per_loop,
+                                          rng=rng, ob=ob)
     # (2) every decision re-taken from the GPU's traces by the oracle's rules: exact
     rep = replay_decisions(block_ids, case.m.mask_id, gpu["entropy"], gpu["cum_halt"], token_at, tau, lam, K, rule)
     assert not rep["ambiguous"], rep["ambiguous"]
     np.testing.assert_array_equal(gpu["exit_depth"], rep["exit_depth"])
     np.testing.assert_array_equal(gpu["tokens"], rep["tokens"])
     np.testing.assert_array_equal(gpu["loops_run"], rep["loops_run"])
-    # (3) end to end against the float64 oracle taking the GPU's decisions
-    of = case.oracle("fp64")
-    of.prefill(case.prefix_ids)
-    ref = of.denoise_step(block_ids, tau, lam, K, rule, follow=follow_of(gpu), band=np.inf)
-    compare_decisions(gpu, ref)
+    # (3) end to end: the oracle takes its own decisions except inside the fixed bands
+    of = oracle
+    if of is None:
+        of = case.oracle("fp64")
+        of.prefill(case.prefix_ids)
+    sel = np.asarray(seq_list)
+    ref = of.denoise_step(block_ids[sel], tau, lam, K, rule, follow=follow_of(gpu, sel), band=E2E_BANDS)
+    sub = {k: gpu[k][sel] for k in ("tokens", "exit_depth", "loops_run", "entropy", "halt", "cum_halt")}
+    sub["active_rows"], sub["readout_rows"] = gpu["active_rows"], gpu["readout_rows"]
+    compare_decisions(sub, ref, rows=seqs is None)
     W = of._global("lm_head")
-    worst = dict(state=0.0, logits=0.0, entropy=0.0, entropy_excess=0.0)
-    for b in range(B):
+    worst = dict(state=0.0, logits=0.0, entropy=0.0, halt=0.0)
+    keys = ((2, "r"),) if not states else ((0, "h_in"), (1, "h_tilde"), (2, "r"))
+    dbg = {(which, s): (r_by_loop[s] if which == 2 else case.handle.debug_state(which, s).cpu().numpy())
+           for which, _ in keys for s in range(1, int(gpu["loops_run"][sel].max()) + 1)}
+    for j, b in enumerate(seq_list):
         for s in range(1, int(gpu["loops_run"][b]) + 1):
-            r_gpu, r_ref = r_by_loop[s][b], ref["r"][b][s - 1]
-            keys = ((2, "r"),) if not states else ((0, "h_in"), (1, "h_tilde"), (2, "r"))
             for which, key in keys:
-                st = r_gpu if which == 2 else case.handle.debug_state(which, s)[b].cpu().numpy()
-                rel = row_rel_err(st, ref[key][b][s - 1])
+                rel = row_rel_err(dbg[(which, s)][b], ref[key][j][s - 1])
                 worst["state"] = max(worst["state"], float(rel.max()))
                 assert rel.max() <= STATE_REL_TOL, (key, b, s, rel.max())
             idx = np.nonzero(~np.isnan(gpu["entropy"][b, s - 1]))[0]
             if len(idx) == 0:
                 continue
-            z_ref = r_ref[idx] @ W.T
-            dz = (r_gpu[idx].astype(np.float64) - r_ref[idx]) @ W.T
+            r_ref = ref["r"][j][s - 1][idx]
+            z_ref = r_ref @ W.T
+            dz = (dbg[(2, s)][b][idx].astype(z_ref.dtype) - r_ref) @ W.T
             lrel = np.linalg.norm(dz, axis=-1) / np.linalg.norm(z_ref, axis=-1)
             worst["logits"] = max(worst["logits"], float(lrel.max()))
             assert lrel.max() <= STATE_REL_TOL, ("logits", b, s, lrel.max())
-            # entropy: |dH| <= 1e-2 + 1.5 * sum_v |dH/dz_v| * max_v |dz_v| (first-order bound
-            # from the logit deviation; dH/dz_v = -p_v (log p_v + H))
-            logp = z_ref - z_ref.max(-1, keepdims=True)
-            logp = logp - np.log(np.exp(logp).sum(-1, keepdims=True))
-            p = np.exp(logp)
-            Hr = -(p * logp).sum(-1)
-            L1 = (p * np.abs(logp + Hr[:, None])).sum(-1)
-            dzc = dz - dz.mean(-1, keepdims=True)
-            bound = ENTROPY_TOL + 1.5 * L1 * np.abs(dzc).max(-1)
-            dH = np.abs(gpu["entropy"][b, s - 1, idx] - ref["entropy"][b, s - 1, idx])
+            dH = np.abs(gpu["entropy"][b, s - 1, idx] - ref["entropy"][j, s - 1, idx])
             worst["entropy"] = max(worst["entropy"], float(dH.max()))
-            worst["entropy_excess"] = max(worst["entropy_excess"], float((dH - bound).max()))
-            assert (dH <= bound).all(), ("entropy", b, s, dH.max(), bound.min())
-    disagree = [f for f in ref["followed"] if f["kind"] in ("commit", "halt") and f.get("own") != f.get("taken")]
-    stats.update(worst)
-    stats["e2e_decisions_differing"] = len(disagree)
-    stats["e2e_margins"] = sorted(abs(f["margin"]) for f in disagree)[:5]
+            assert dH.max() <= E2E_ENTROPY_TOL, ("entropy", b, s, float(dH.max()))
+            for key in ("halt", "cum_halt"):
+                da = np.abs(gpu[key][b, s - 1, idx] - ref[key][j, s - 1, idx])
+                worst["halt"] = max(worst["halt"], float(da.max()))
+                assert da.max() <= E2E_HALT_TOL, (key, b, s, float(da.max()))
+    differing = [f for f in ref["followed"] if f.get("own") != f.get("taken")]
+    stats.update({f"e2e_{k}": v for k, v in worst.items()})
+    stats["e2e_followed"] = len(ref["followed"])
+    stats["e2e_followed_differing"] = len(differing)
+    stats["e2e_differing_margins"] = sorted((f["kind"], round(abs(f["margin"]), 4)) for f in differing)[:8]
     return stats
