@@ -75,9 +75,14 @@ def lib() -> ctypes.CDLL:
         vp, ci, cf, csz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         L.alodlm_create.argtypes = [ctypes.POINTER(Cfg), ctypes.POINTER(Weights), vp, ctypes.POINTER(vp)]
         L.alodlm_prefill.argtypes = [vp, vp, ci, ci, vp]
+        L.alodlm_append.argtypes = [vp, vp, ci, ci, vp]
         L.alodlm_denoise_step.argtypes = [vp, vp, ci, ci, cf, cf, ci, ci, ctypes.POINTER(StepOut)]
         L.alodlm_decode_block.argtypes = [vp, vp, ci, ci, cf, cf, ci, ci, ci, ctypes.POINTER(DecodeOut),
                                           ctypes.POINTER(ci)]
+        u64 = ctypes.c_uint64
+        L.alodlm_denoise_step_sampled.argtypes = [vp, vp, ci, ci, cf, cf, ci, ci, u64, u64, ctypes.POINTER(StepOut)]
+        L.alodlm_decode_block_sampled.argtypes = [vp, vp, ci, ci, cf, cf, ci, ci, ci, u64, ctypes.POINTER(DecodeOut),
+                                                  ctypes.POINTER(ci)]
         L.alodlm_sync.argtypes = [vp]
         L.alodlm_destroy.argtypes = [vp]
         L.alodlm_destroy.restype = None
@@ -94,7 +99,8 @@ def lib() -> ctypes.CDLL:
         L.alodlm_kernel_class_name.restype = ctypes.c_char_p
         L.alodlm_gemm_bf16.argtypes = [vp, vp, vp, ci, ci, ci, vp, csz, vp]
         L.alodlm_gemm_bf16_noalloc.argtypes = [vp, vp, vp, ci, ci, ci, vp, vp]
-        for f in ("alodlm_create", "alodlm_prefill", "alodlm_denoise_step", "alodlm_sync", "alodlm_debug_state",
+        for f in ("alodlm_create", "alodlm_prefill", "alodlm_append", "alodlm_denoise_step",
+                  "alodlm_denoise_step_sampled", "alodlm_decode_block_sampled", "alodlm_decode_block", "alodlm_sync", "alodlm_debug_state",
                   "alodlm_kv_slot", "alodlm_step_stats", "alodlm_set_timing", "alodlm_set_graphs",
                   "alodlm_gemm_bf16", "alodlm_gemm_bf16_noalloc"):
             getattr(L, f).restype = ci
@@ -226,6 +232,18 @@ class Handle:
         self._order_out()
         self.B, self.P = B, P
 
+    def append(self, ids: torch.Tensor, exit_depth: Optional[torch.Tensor] = None):
+        """Append positions P..P+N-1 holding ids [B, N] to the cached prefix (alodlm_append);
+        exit_depth [B, N] in 1..k_max or None (k_max)."""
+        B, N = ids.shape
+        ids = ids.to(torch.int32).contiguous()
+        e = None if exit_depth is None else exit_depth.to(torch.int32).contiguous()
+        self._keep_append = (ids, e)
+        self._order_in()
+        self._check(lib().alodlm_append(self._h, _ptr(ids), B, N, _ptr(e)), "append")
+        self._order_out()
+        self.P += N
+
     def alloc_outputs(self, B: int, N: int, k_max: int, device=None) -> dict:
         dev = device or torch.device("cuda", torch.cuda.current_device())
         i32, f32 = torch.int32, torch.float32
@@ -239,20 +257,27 @@ class Handle:
                     readout_rows=torch.empty((k_max,), dtype=i32, device=dev))
 
     def denoise_step(self, block_ids: torch.Tensor, tau_H: float, lam: float, k_max: int,
-                     rule: int = RULE_PAPER, out: Optional[dict] = None) -> dict:
+                     rule: int = RULE_PAPER, out: Optional[dict] = None, sample: Optional[tuple] = None) -> dict:
+        """One step (alodlm_denoise_step); sample=(seed, step) draws the committed tokens
+        (alodlm_denoise_step_sampled)."""
         B, N = block_ids.shape
         if out is None:
             out = self.alloc_outputs(B, N, k_max)
         so = StepOut(**{k: _ptr(v) for k, v in out.items()})
         self._order_in()
-        self._check(lib().alodlm_denoise_step(self._h, _ptr(block_ids), B, N, float(tau_H), float(lam), k_max,
-                                              rule, ctypes.byref(so)), "denoise_step")
+        if sample is None:
+            rc = lib().alodlm_denoise_step(self._h, _ptr(block_ids), B, N, float(tau_H), float(lam), k_max, rule,
+                                           ctypes.byref(so))
+        else:
+            rc = lib().alodlm_denoise_step_sampled(self._h, _ptr(block_ids), B, N, float(tau_H), float(lam), k_max,
+                                                   rule, int(sample[0]), int(sample[1]), ctypes.byref(so))
+        self._check(rc, "denoise_step")
         self._order_out()
         self.N = N
         return out
 
     def decode_block(self, block_ids: torch.Tensor, tau_H: float, lam: float, k_max: int, rule: int = RULE_PAPER,
-                     max_steps: int = 0) -> dict:
+                     max_steps: int = 0, sample_seed: Optional[int] = None) -> dict:
         """Denoising steps until no [MASK] is left (alodlm_decode_block); max_steps 0 = N.
         Returns the device outputs (tokens, commit_step, commit_depth, steps_run, loops
         [S, B], rows [S, 2, K]) and "steps" (host int)."""
@@ -265,8 +290,13 @@ class Handle:
         do = DecodeOut(**{k: _ptr(v) for k, v in out.items()})
         steps = ctypes.c_int()
         self._order_in()
-        self._check(lib().alodlm_decode_block(self._h, _ptr(block_ids), B, N, float(tau_H), float(lam), k_max, rule,
-                                              S, ctypes.byref(do), ctypes.byref(steps)), "decode_block")
+        if sample_seed is None:
+            rc = lib().alodlm_decode_block(self._h, _ptr(block_ids), B, N, float(tau_H), float(lam), k_max, rule, S,
+                                           ctypes.byref(do), ctypes.byref(steps))
+        else:
+            rc = lib().alodlm_decode_block_sampled(self._h, _ptr(block_ids), B, N, float(tau_H), float(lam), k_max,
+                                                   rule, S, int(sample_seed), ctypes.byref(do), ctypes.byref(steps))
+        self._check(rc, "decode_block")
         self._order_out()
         self.N = N
         out["steps"] = steps.value

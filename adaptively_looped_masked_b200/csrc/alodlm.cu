@@ -162,7 +162,6 @@ bool init_kernel_attrs() {
     set_gemm_attr<256, gemm::EPI_F32>();
     set_gemm_attr<256, gemm::EPI_ADD>();
     set_gemm_attr<256, gemm::EPI_SWIGLU>();
-    set_gemm_attr<256, gemm::EPI_READOUT>();
     set_persist_attr<128, gemm::EPI_F32>();
     set_persist_attr<128, gemm::EPI_ADD>();
     set_persist_attr<128, gemm::EPI_SWIGLU>();
@@ -431,6 +430,7 @@ struct alodlm {
     int B = 0, P = 0, last_N = 0;
     bool prefilled = false;
     int *exit_dev = nullptr;
+    int *app_exit = nullptr;  // exit depths of the positions being appended [max_batch * max_block]
     int *iota = nullptr;
 
     // activation scratch (rows_cap rows)
@@ -447,6 +447,8 @@ struct alodlm {
     bf16 *rb = nullptr;
     float *lam_rr = nullptr;
     float4 *part = nullptr;
+    double2 *spart = nullptr;        // sampled commits: per (row, vocab tile) max of z + g and its id
+    SampleParams *samp = nullptr;    // sampling state of the current step (device)
     int *ridx = nullptr, *rr_b = nullptr, *rr_i = nullptr;
     CUtensorMap tm_rb;
 
@@ -694,8 +696,11 @@ int slot_prelude(const alodlm *h, int l) { return l; }
 int slot_core(const alodlm *h, int c, int d) { return h->cfg.n_prelude + (d - 1) * h->cfg.n_core + c; }
 int slot_coda(const alodlm *h, int j) { return h->cfg.n_prelude + h->cfg.k_max * h->cfg.n_core + j; }
 
+// Depth fallback of one Core layer at depth `depth` during a prefill or an append: rows of
+// sequences b0 .. b0+nb-1, positions pos0 .. pos0+n-1 with exit depths exit[b * n + t]
 struct Fallback {
-    int P, b0, nb, depth, src_slot;
+    const int *exit;
+    int n, pos0, b0, nb, depth, src_slot;
 };
 
 // xn = RMSNorm(x) * g (bf16) over M rows of the hidden size
@@ -729,10 +734,10 @@ int run_layer(alodlm *h, int li, int slot, int M, const RowMap &map, int n_seq, 
     }
     if (fb) {
         const long long so = (long long)fb->src_slot * h->slot_elems;
-        LAUNCH(KC_OTHER, 8.0 * fb->nb * h->nkv * fb->P * h->hd, 0.0,
-               (klaunch(k::kv_fallback_kernel, dim3(fb->nb, h->nkv), 256, 0, h->stream, 
-                   h->exit_dev, fb->P, fb->b0, fb->depth, h->kv_k + so, h->kv_v + so, kc, vc, h->seq_stride,
-                   h->head_stride, h->hd)));
+        LAUNCH(KC_OTHER, 8.0 * fb->nb * h->nkv * fb->n * h->hd, 0.0,
+               (klaunch(k::kv_fallback_kernel, dim3(fb->nb, h->nkv), 256, 0, h->stream, fb->exit, fb->n, fb->pos0,
+                        fb->b0, fb->depth, h->kv_k + so, h->kv_v + so, kc, vc, h->seq_stride, h->head_stride,
+                        h->hd)));
     }
     if ((rc = attention(h, slot, M, map, n_seq, kv_len, causal))) return rc;
     if ((rc = linear(h, Lw.tm_o, H, h->attn_out, M, qd, gemm::EPI_ADD, x, H, nullptr, 0))) return rc;
@@ -974,6 +979,7 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
     h->n_vt = cdiv(h->V, 256);
     if ((rc = dalloc(h, &h->rb, (size_t)h->R_cap * H)) || (rc = dalloc(h, &h->lam_rr, h->R_cap)) ||
         (rc = dalloc(h, &h->part, (size_t)h->R_cap * h->n_vt)) || (rc = dalloc(h, &h->ridx, h->step_rows_cap)) ||
+        (rc = dalloc(h, &h->spart, (size_t)h->R_cap * h->n_vt)) || (rc = dalloc(h, &h->samp, 1)) ||
         (rc = dalloc(h, &h->rr_b, h->R_cap)) || (rc = dalloc(h, &h->rr_i, h->R_cap)))
         return cleanup(rc);
     cudaMemsetAsync(h->rb, 0, (size_t)h->R_cap * H * 2, h->stream);
@@ -988,6 +994,7 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
         (rc = dalloc(h, &h->seq_of[1], cfg->max_batch)) || (rc = dalloc(h, &h->old_slot, cfg->max_batch)) ||
         (rc = dalloc(h, &h->counts, 4)) || (rc = dalloc(h, &h->d_err, 1)) || (rc = dalloc(h, &h->iota, cfg->max_batch)) ||
         (rc = dalloc(h, &h->exit_dev, (size_t)cfg->max_batch * cfg->max_prefix)) ||
+        (rc = dalloc(h, &h->app_exit, BN_)) ||
         (rc = dalloc(h, &h->dec_tok[0], BN_)) || (rc = dalloc(h, &h->dec_tok[1], BN_)) ||
         (rc = dalloc(h, &h->dec_ex, BN_)) || (rc = dalloc(h, &h->dec_loops, cfg->max_batch)) ||
         (rc = dalloc(h, &h->dec_rows, 2 * (size_t)cfg->k_max)) || (rc = dalloc(h, &h->dec_left, 1)) ||
@@ -1017,8 +1024,16 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
     return ALODLM_OK;
 }
 
-int alodlm_decode_block(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda, int k_max,
-                        int rule, int max_steps, const alodlm_decode_out *out, int *steps_taken) {
+}  // extern "C"
+
+namespace {
+
+int denoise_step_impl(alodlm *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda, int k_max,
+                      int rule, const SampleParams &sp, const alodlm_step_out *out);
+
+int decode_block_impl(alodlm *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda, int k_max,
+                      int rule, int max_steps, bool sampled, uint64_t seed, const alodlm_decode_out *out,
+                      int *steps_taken) {
     if (steps_taken) *steps_taken = 0;
     if (!h || !block_ids || !out || !out->tokens || !out->commit_step || !out->commit_depth || !out->steps_run ||
         !out->loops || !out->rows)
@@ -1063,7 +1078,8 @@ int alodlm_decode_block(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
         if (*h->dec_left_host == 0 || t == max_steps) break;
         ++t;
         so.tokens = h->dec_tok[t & 1];
-        const int rc = alodlm_denoise_step(h, in, B, N, tau_H, lambda, k_max, rule, &so);
+        const SampleParams sp{(unsigned long long)seed, (unsigned long long)t, sampled ? 1 : 0, 0};
+        const int rc = denoise_step_impl(h, in, B, N, tau_H, lambda, k_max, rule, sp, &so);
         if (rc) return rc;
         ck(cudaMemsetAsync(h->dec_left, 0, sizeof(int), h->stream));
         klaunch(k::decode_update_kernel, grid, 256, 0, h->stream, (const int *)in, (const int *)so.tokens,
@@ -1081,6 +1097,21 @@ int alodlm_decode_block(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
     if (ce != cudaSuccess) return cuda_fail(h, ce, "decode_block");
     if (steps_taken) *steps_taken = t;
     return ALODLM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int alodlm_decode_block(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda, int k_max,
+                        int rule, int max_steps, const alodlm_decode_out *out, int *steps_taken) {
+    return decode_block_impl(h, block_ids, B, N, tau_H, lambda, k_max, rule, max_steps, false, 0, out, steps_taken);
+}
+
+int alodlm_decode_block_sampled(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda,
+                                int k_max, int rule, int max_steps, uint64_t seed, const alodlm_decode_out *out,
+                                int *steps_taken) {
+    return decode_block_impl(h, block_ids, B, N, tau_H, lambda, k_max, rule, max_steps, true, seed, out, steps_taken);
 }
 
 int alodlm_set_timing(alodlm_t *h, int on) {
@@ -1111,6 +1142,56 @@ int alodlm_sync(alodlm_t *h) {
     return ALODLM_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Prefix rows through the whole stack, writing their K/V into every slot of the arena:
+// sequences b0 .. b0+nb-1, positions pos0 .. pos0+n-1 holding ids[b * n + t], attending
+// causally to keys [0, pos0 + n) (the positions before pos0 are already in the arena, every
+// slot resolved to its depth).  A position with exit depth e runs the Core e times: at depth
+// d > e its Core K/V is the depth-e K/V (copied from slot d-1), and the Coda runs once on its
+// depth-e state.  exit: device [B, n] exit depths in 1..k_max, or nullptr for k_max everywhere.
+int build_prefix_rows(alodlm *h, const int32_t *ids, int b0, int nb, int n, int pos0, const int *exit) {
+    const alodlm_cfg &c = h->cfg;
+    const int M = nb * n, kv_len = pos0 + n;
+    RowMap map{h->iota + b0, n, pos0};
+    float *x = h->hbuf[0];
+    int rc;
+    LAUNCH(KC_OTHER, 6.0 * M * h->H, 0.0,
+           (klaunch(k::embed_kernel, M, 256, 0, h->stream, ids, n, map, h->embed, h->V, h->H, x, h->d_err)));
+    for (int l = 0; l < c.n_prelude; ++l)
+        if ((rc = run_layer(h, l, slot_prelude(h, l), M, map, nb, kv_len, 1, x, nullptr))) return rc;
+    for (int d = 1; d <= c.k_max; ++d) {
+        for (int cc = 0; cc < c.n_core; ++cc) {
+            Fallback fb{exit, n, pos0, b0, nb, d, d > 1 ? slot_core(h, cc, d - 1) : 0};
+            const bool use_fb = exit && d > 1;
+            if ((rc = run_layer(h, c.n_prelude + cc, slot_core(h, cc, d), M, map, nb, kv_len, 1, x,
+                                use_fb ? &fb : nullptr)))
+                return rc;
+        }
+        if (exit)
+            LAUNCH(KC_OTHER, 8.0 * M * h->H / c.k_max, 0.0,
+                   (klaunch(k::capture_exit_kernel, M, 256, 0, h->stream, exit, n, b0, d, x, h->hexit, h->H)));
+    }
+    if (exit) x = h->hexit;
+    for (int j = 0; j < c.n_coda; ++j)
+        if ((rc = run_layer(h, c.n_prelude + c.n_core + j, slot_coda(h, j), M, map, nb, kv_len, 1, x, nullptr)))
+            return rc;
+    return check_launch(h, "prefix rows");
+}
+
+// EDEVICE on the next sync if an exit depth lies outside 1..k_max
+void check_exit_depths(alodlm *h, const int *exit, long long n) {
+    const unsigned grid = (unsigned)std::min<long long>((n + 255) / 256, 1024);
+    LAUNCH(KC_OTHER, 4.0 * n, 0.0,
+           (klaunch(k::check_range_kernel, grid, 256, 0, h->stream, exit, n, 1, h->cfg.k_max, h->d_err)));
+}
+
+}  // namespace
+
+extern "C" {
+
 int alodlm_prefill(alodlm_t *h, const int32_t *prefix_ids, int B, int P, const int32_t *exit_depth) {
     if (!h || !prefix_ids) return fail(h, ALODLM_EINVAL, "null argument");
     const alodlm_cfg &c = h->cfg;
@@ -1118,44 +1199,48 @@ int alodlm_prefill(alodlm_t *h, const int32_t *prefix_ids, int B, int P, const i
         return fail(h, ALODLM_EINVAL, "prefill: B or P out of range");
     reset_stats(h);
     h->prefilled = false;
-    if (exit_depth)
+    if (exit_depth) {
         cudaMemcpyAsync(h->exit_dev, exit_depth, (size_t)B * P * sizeof(int), cudaMemcpyDeviceToDevice, h->stream);
+        check_exit_depths(h, h->exit_dev, (long long)B * P);
+    }
     const int g = std::max(1, std::min(B, h->rows_cap / P));
     int rc;
-    for (int b0 = 0; b0 < B; b0 += g) {
-        const int nb = std::min(g, B - b0), M = nb * P;
-        RowMap map{h->iota + b0, P, 0};
-        float *x = h->hbuf[0];
-        LAUNCH(KC_OTHER, 6.0 * M * h->H, 0.0,
-               (klaunch(k::embed_kernel, M, 256, 0, h->stream, prefix_ids, P, map, h->embed, h->V, h->H, x, h->d_err)));
-        for (int l = 0; l < c.n_prelude; ++l)
-            if ((rc = run_layer(h, l, slot_prelude(h, l), M, map, nb, P, 1, x, nullptr))) return rc;
-        for (int d = 1; d <= c.k_max; ++d) {
-            for (int cc = 0; cc < c.n_core; ++cc) {
-                Fallback fb{P, b0, nb, d, d > 1 ? slot_core(h, cc, d - 1) : 0};
-                const bool use_fb = exit_depth && d > 1;
-                if ((rc = run_layer(h, c.n_prelude + cc, slot_core(h, cc, d), M, map, nb, P, 1, x,
-                                    use_fb ? &fb : nullptr)))
-                    return rc;
-            }
-            if (exit_depth)
-                LAUNCH(KC_OTHER, 8.0 * M * h->H / c.k_max, 0.0,
-                       (klaunch(k::capture_exit_kernel, M, 256, 0, h->stream, h->exit_dev, P, b0, d, x, h->hexit, h->H)));
-        }
-        if (exit_depth) x = h->hexit;
-        for (int j = 0; j < c.n_coda; ++j)
-            if ((rc = run_layer(h, c.n_prelude + c.n_core + j, slot_coda(h, j), M, map, nb, P, 1, x, nullptr)))
-                return rc;
-        if ((rc = check_launch(h, "prefill"))) return rc;
-    }
+    for (int b0 = 0; b0 < B; b0 += g)
+        if ((rc = build_prefix_rows(h, prefix_ids, b0, std::min(g, B - b0), P, 0, exit_depth ? h->exit_dev : nullptr)))
+            return rc;
     h->B = B;
     h->P = P;
     h->prefilled = true;
     return ALODLM_OK;
 }
 
-int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda, int k_max,
-                        int rule, const alodlm_step_out *out) {
+int alodlm_append(alodlm_t *h, const int32_t *ids, int B, int N, const int32_t *exit_depth) {
+    if (!h || !ids) return fail(h, ALODLM_EINVAL, "null argument");
+    const alodlm_cfg &c = h->cfg;
+    if (!h->prefilled) return fail(h, ALODLM_ESTATE, "append before prefill");
+    if (B != h->B) return fail(h, ALODLM_ESTATE, "batch differs from the prefill's");
+    if (N < 1 || N > c.max_block) return fail(h, ALODLM_EINVAL, "append: N out of range (1..max_block)");
+    if (h->P + N > c.max_prefix) return fail(h, ALODLM_EINVAL, "append: the prefix would pass max_prefix");
+    reset_stats(h);
+    if (exit_depth) {
+        cudaMemcpyAsync(h->app_exit, exit_depth, (size_t)B * N * sizeof(int), cudaMemcpyDeviceToDevice, h->stream);
+        check_exit_depths(h, h->app_exit, (long long)B * N);
+    }
+    int rc;
+    if ((rc = build_prefix_rows(h, ids, 0, B, N, h->P, exit_depth ? h->app_exit : nullptr))) {
+        h->prefilled = false;  // the arena may hold part of the new positions
+        return rc;
+    }
+    h->P += N;
+    return ALODLM_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+int denoise_step_impl(alodlm *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda, int k_max,
+                      int rule, const SampleParams &sp, const alodlm_step_out *out) {
     if (!h || !block_ids || !out || !out->tokens || !out->exit_depth || !out->entropy || !out->halt ||
         !out->cum_halt || !out->loops_run || !out->active_rows || !out->readout_rows)
         return fail(h, ALODLM_EINVAL, "null argument");
@@ -1190,7 +1275,7 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
     const long long BNt = (long long)B * N;
     LAUNCH(KC_COMMIT, 16.0 * BNt, 0.0,
            (klaunch(k::step_init_kernel, (unsigned)std::min<long long>((BNt + 255) / 256, 1024), 256, 0, h->stream, 
-               block_ids, B, N, K, c.mask_id, st)));
+               block_ids, B, N, K, c.mask_id, st, sp, h->samp)));
     LAUNCH(KC_COMMIT, 8.0 * BNt, 0.0,
            (klaunch(k::plan_kernel, 1, 1024, 0, h->stream, B, h->iota, N, h->cont, h->U, h->seq_of[0], h->old_slot,
                                                       h->ridx, h->rr_b, h->rr_i, h->counts, 1, K, out->active_rows,
@@ -1241,6 +1326,12 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
             gemm::EpiParams ep{};
             ep.partials = h->part;
             ep.n_btiles = h->n_vt;
+            ep.spartials = h->spart;
+            ep.samp = h->samp;
+            ep.rr_b = h->rr_b;
+            ep.rr_i = h->rr_i;
+            ep.N = N;
+            ep.loop = s;
             const double R_est = Ml;  // upper bound on the readout rows (exact counts are on the device)
             const double bytes = 2.0 * h->V * H + 2.0 * R_est * H + 16.0 * R_est * h->n_vt;
             LAUNCH(KC_RGEMM, bytes, 2.0 * R_est * h->V * (double)H,
@@ -1248,8 +1339,8 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
                                                            cdiv(H, gemm::BK), 1, ep, h->d_err, h->stream,
                                                            h->num_sms, 2)));
             LAUNCH(KC_RCOMB, 16.0 * R_est * h->n_vt, 0.0,
-                   (klaunch(k::readout_combine_kernel, cdiv(Ml, 8), 256, 0, h->stream, 
-                       h->part, h->n_vt, h->counts + 1, h->rr_b, h->rr_i, h->lam_rr, N, K, s, h->a, h->cur_H,
+                   (klaunch(k::readout_combine_kernel, cdiv(Ml, 8), 256, 0, h->stream, h->part,
+                            (const double2 *)h->spart, (const SampleParams *)h->samp, h->n_vt, h->counts + 1, h->rr_b, h->rr_i, h->lam_rr, N, K, s, h->a, h->cur_H,
                        h->cur_y, out->entropy, out->halt, out->cum_halt)));
         }
         LAUNCH(KC_COMMIT, 16.0 * Ml, 0.0,
@@ -1316,6 +1407,22 @@ int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, flo
         n_act = n_next;
     }
     return check_launch(h, "step end");
+}
+
+}  // namespace
+
+extern "C" {
+
+int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda, int k_max,
+                        int rule, const alodlm_step_out *out) {
+    const SampleParams greedy{0ull, 0ull, 0, 0};
+    return denoise_step_impl(h, block_ids, B, N, tau_H, lambda, k_max, rule, greedy, out);
+}
+
+int alodlm_denoise_step_sampled(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda,
+                                int k_max, int rule, uint64_t seed, uint64_t step, const alodlm_step_out *out) {
+    const SampleParams sp{(unsigned long long)seed, (unsigned long long)step, 1, 0};
+    return denoise_step_impl(h, block_ids, B, N, tau_H, lambda, k_max, rule, sp, out);
 }
 
 int alodlm_set_graphs(alodlm_t *h, int on) {

@@ -299,6 +299,48 @@ __device__ __forceinline__ float block_sum(float v, float *red) {
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.f + __expf(-x)); }
 
+// ---------------------------------------------------------------------------------
+// sampled commits: counter-based random numbers
+// ---------------------------------------------------------------------------------
+
+// Sampling state of a step (device memory, written by the step's first kernel): Gumbel noise
+// is drawn under key (seed, step) when enabled.
+struct SampleParams {
+    unsigned long long seed, step;
+    int enabled, pad;
+};
+
+// Philox4x64-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as easy as 1, 2, 3",
+// SC 2011): ten rounds, each two 64 x 64 -> 128-bit products of counter words with the
+// round multipliers, the high halves xor-ed with the other counter words and the key; the key
+// advances by the Weyl constants before every round but the first.  x: counter in, four
+// random 64-bit words out.
+__device__ __forceinline__ void philox4x64_10(uint64_t (&x)[4], uint64_t k0, uint64_t k1) {
+    constexpr uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+    constexpr uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        if (r) {
+            k0 += W0;
+            k1 += W1;
+        }
+        const uint64_t hi0 = __umul64hi(M0, x[0]), lo0 = M0 * x[0];
+        const uint64_t hi1 = __umul64hi(M1, x[2]), lo1 = M1 * x[2];
+        const uint64_t y0 = hi1 ^ x[1] ^ k0, y2 = hi0 ^ x[3] ^ k1;
+        x[0] = y0;
+        x[1] = lo1;
+        x[2] = y2;
+        x[3] = lo0;
+    }
+}
+
+// Standard Gumbel variate from 64 random bits: u = (53 high bits + 1/2) * 2^-53 in (0, 1),
+// g = -log(-log(u)), in double precision
+__device__ __forceinline__ double gumbel_from_bits(uint64_t bits) {
+    const double u = ((double)(bits >> 11) + 0.5) * 0x1.0p-53;
+    return -log(-log(u));
+}
+
 // row -> (sequence, position) of a batch of blocks laid out contiguously per sequence
 struct RowMap {
     const int *seq_of;  // slot j -> sequence index b

@@ -40,6 +40,13 @@ struct EpiParams {
     int ld_act;
     float4 *partials;     // EPI_READOUT: partials[a_row * n_btiles + b_tile] = (max, sum e, sum e*d, argmax)
     int n_btiles;
+    // EPI_READOUT with sampling (samp->enabled): spartials[a_row * n_btiles + b_tile] = (max of
+    // z_v + g_v, its id v) with g_v the Gumbel noise of readout row a_row = position
+    // rr_b[a_row] * N + rr_i[a_row] at loop `loop`
+    double2 *spartials;
+    const SampleParams *samp;
+    const int *rr_b, *rr_i;
+    int N, loop;
 };
 
 // Write (EPI_F32) or add to (EPI_ADD) 16 consecutive rows of one output column: p points at
@@ -156,6 +163,7 @@ __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int rowsA,
                    int rowsB, const int *rowsA_dyn, int k_tiles, int kt_per_split, int a_fastest, int tiled,
                    EpiParams ep, int *err) {
+    static_assert(EPI != EPI_READOUT, "the LM-head readout runs in the persistent kernel");
     using C = Cfg<BN>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -300,41 +308,6 @@ __global__ void __launch_bounds__(192, 1)
                         }
                     }
                 }  // split-K: pushed to the owners below
-            } else {  // EPI_READOUT: this thread's row of logits over BN vocabulary entries
-                float best = -INFINITY;
-                int best_idx = b0;
-                for (int c0 = 0; c0 < BN; c0 += 16) {
-                    if (b0 + c0 >= rowsB) break;
-                    float v[16];
-                    tmem_ld16(taddr + c0, v);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int vid = b0 + c0 + j;
-                        if (vid < rowsB && v[j] > best) {  // strict: lowest id wins ties
-                            best = v[j];
-                            best_idx = vid;
-                        }
-                    }
-                }
-                float se = 0.f, sed = 0.f;
-                const float LOG2E = 1.4426950408889634f;
-                for (int c0 = 0; c0 < BN; c0 += 16) {
-                    if (b0 + c0 >= rowsB) break;
-                    float v[16];
-                    tmem_ld16(taddr + c0, v);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        if (b0 + c0 + j < rowsB) {
-                            const float d = v[j] - best;
-                            const float e = exp2f(d * LOG2E);
-                            se += e;
-                            sed = fmaf(e, d, sed);
-                        }
-                    }
-                }
-                if (a_row < rowsA)
-                    ep.partials[(long long)a_row * ep.n_btiles + b_tile] =
-                        make_float4(best, se, sed, __int_as_float(best_idx));
             }
         }
     }
@@ -721,6 +694,35 @@ __device__ __forceinline__ void readout_tile(uint32_t taddr, int a_row, int b0, 
     }
     if (a_row < rowsA)
         ep.partials[(long long)a_row * ep.n_btiles + b_tile] = make_float4(best, se, sed, __int_as_float(best_idx));
+    if (ep.samp != nullptr && ep.samp->enabled) {  // uniform: every lane takes part in the TMEM loads
+        // Gumbel-max: the largest z_v + g_v of the tile and its id, in double precision
+        const long long pos = a_row < rowsA ? (long long)ep.rr_b[a_row] * ep.N + ep.rr_i[a_row] : 0;
+        const uint64_t k0 = ep.samp->seed, k1 = ep.samp->step;
+        double sbest = -INFINITY;
+        int sidx = b0;
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+            if (b0 + c0 >= rowsB) break;
+            float v[16];
+            tmem_ld16(taddr + c0, v);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint64_t x[4] = {(uint64_t)((b0 + c0) / 4 + q), (uint64_t)pos, (uint64_t)ep.loop, 0ull};
+                philox4x64_10(x, k0, k1);
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const int vid = b0 + c0 + 4 * q + w;
+                    if (vid < rowsB) {
+                        const double sc = (double)v[4 * q + w] + gumbel_from_bits(x[w]);
+                        if (sc > sbest) {  // strict: lowest id wins ties
+                            sbest = sc;
+                            sidx = vid;
+                        }
+                    }
+                }
+            }
+        }
+        if (a_row < rowsA) ep.spartials[(long long)a_row * ep.n_btiles + b_tile] = make_double2(sbest, (double)sidx);
+    }
 }
 
 // Epilogue of 64 accumulator columns [c0, c0 + 64) of a 128-row tile, by the 128 epilogue

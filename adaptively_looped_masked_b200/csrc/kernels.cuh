@@ -255,8 +255,10 @@ __global__ void qkv_post128_kernel(const float *qkv, int nq, int nkv, int hpw, c
 
 // Prefill depth fallback: for prefix positions whose exit depth is below the current depth,
 // the KV at this depth is the KV of the previous depth (which by induction is the KV of
-// their exit depth).  One block per (sequence in group, kv head), threads over positions.
-__global__ void kv_fallback_kernel(const int *exit_depth, int P, int b0, int depth, const bf16 *src_k,
+// their exit depth).  Positions pos0 .. pos0+n-1 of sequence b0 + blockIdx.x, whose exit
+// depths are exit_depth[(b0 + blockIdx.x) * n + t]; one block per (sequence, kv head),
+// threads over positions.
+__global__ void kv_fallback_kernel(const int *exit_depth, int n, int pos0, int b0, int depth, const bf16 *src_k,
                                    const bf16 *src_v, bf16 *dst_k, bf16 *dst_v, long long seq_stride,
                                    long long head_stride, int hd) {
     pdl_wait();
@@ -264,13 +266,21 @@ __global__ void kv_fallback_kernel(const int *exit_depth, int P, int b0, int dep
     const int b = b0 + blockIdx.x, kvh = blockIdx.y;
     const long long base = (long long)b * seq_stride + (long long)kvh * head_stride;
     const int chunks = hd / 8;
-    for (long long idx = threadIdx.x; idx < (long long)P * chunks; idx += blockDim.x) {
-        const int pos = (int)(idx / chunks), ch = (int)(idx % chunks);
-        if (exit_depth[(long long)b * P + pos] >= depth) continue;
-        const long long off = base + (long long)pos * hd + ch * 8;
+    for (long long idx = threadIdx.x; idx < (long long)n * chunks; idx += blockDim.x) {
+        const int t = (int)(idx / chunks), ch = (int)(idx % chunks);
+        if (exit_depth[(long long)b * n + t] >= depth) continue;
+        const long long off = base + (long long)(pos0 + t) * hd + ch * 8;
         *reinterpret_cast<uint4 *>(dst_k + off) = *reinterpret_cast<const uint4 *>(src_k + off);
         *reinterpret_cast<uint4 *>(dst_v + off) = *reinterpret_cast<const uint4 *>(src_v + off);
     }
+}
+
+// Raise DEVERR_BOUNDS if any of v[0, n) lies outside [lo, hi]
+__global__ void check_range_kernel(const int *v, long long n, int lo, int hi, int *err) {
+    pdl_wait();
+    pdl_trigger();
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+        if (v[i] < lo || v[i] > hi) atomicOr(err, DEVERR_BOUNDS);
 }
 
 // h_exit[m] = h[m] for prefix rows whose exit depth equals `depth`
@@ -339,9 +349,12 @@ __device__ __forceinline__ Stat merge_stat(Stat a, Stat b) {
 // One warp per readout row: merge the per-vocab-tile (max, sum e^(z-max), sum e^(z-max)(z-max),
 // argmax) in a fixed order -> entropy H = log S - T/S (nats) and argmax; then the cumulative
 // halt a <- a + (1 - a) lambda and the traces.
-__global__ void readout_combine_kernel(const float4 *part, int n_vt, const int *R_dev, const int *rr_b,
-                                       const int *rr_i, const float *lam_rr, int N, int Kstep, int s, float *a_state,
-                                       float *cur_H, int *cur_y, float *tr_H, float *tr_lam, float *tr_a) {
+// With sampling on, the committed token is instead the id of the largest z_v + g_v over the
+// per-tile (score, id) partials (larger score first, the lower id on equal scores).
+__global__ void readout_combine_kernel(const float4 *part, const double2 *spart, const SampleParams *samp, int n_vt,
+                                       const int *R_dev, const int *rr_b, const int *rr_i, const float *lam_rr, int N,
+                                       int Kstep, int s, float *a_state, float *cur_H, int *cur_y, float *tr_H,
+                                       float *tr_lam, float *tr_a) {
     pdl_wait();
     pdl_trigger();
     const int rr = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -373,6 +386,30 @@ __global__ void readout_combine_kernel(const float4 *part, int n_vt, const int *
         }
         have = have || other_have;
     }
+    int token = acc.idx;
+    if (samp->enabled) {
+        const double2 *sp = spart + (long long)rr * n_vt;
+        double best = -INFINITY;
+        int bid = 0x7fffffff;
+        for (int v = lane; v < n_vt; v += 32) {
+            const double2 x = sp[v];
+            const int id = (int)x.y;
+            if (x.x > best || (x.x == best && id < bid)) {
+                best = x.x;
+                bid = id;
+            }
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bid, o);
+            if (ob > best || (ob == best && oi < bid)) {
+                best = ob;
+                bid = oi;
+            }
+        }
+        token = bid;
+    }
     if (lane == 0) {
         const int b = rr_b[rr], i = rr_i[rr];
         const float H = logf(acc.s) - acc.t / acc.s;
@@ -381,7 +418,7 @@ __global__ void readout_combine_kernel(const float4 *part, int n_vt, const int *
         const float a = a_state[bi] + (1.f - a_state[bi]) * lam;
         a_state[bi] = a;
         cur_H[bi] = H;
-        cur_y[bi] = acc.idx;
+        cur_y[bi] = token;
         const long long tr = ((long long)b * Kstep + (s - 1)) * N + i;
         tr_H[tr] = H;
         tr_lam[tr] = lam;
@@ -405,9 +442,11 @@ struct StepState {
     int *n_commit;             // [B] commits in this step
 };
 
-__global__ void step_init_kernel(const int *block_ids, int B, int N, int Kstep, int mask_id, StepState st) {
+__global__ void step_init_kernel(const int *block_ids, int B, int N, int Kstep, int mask_id, StepState st,
+                                 SampleParams sp, SampleParams *samp) {
     pdl_wait();
     pdl_trigger();
+    if (blockIdx.x == 0 && threadIdx.x == 0) *samp = sp;
     const long long total = (long long)B * N;
     const float qnan = __int_as_float(0x7fc00000);
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;

@@ -122,8 +122,27 @@ ALODLM_API int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *weight
  * Prefix attention is causal; positions are 0..P-1.
  * prefix_ids: device int32 [B,P], ids in [0, vocab).  exit_depth: device int32 [B,P] in
  * 1..k_max, or NULL for k_max everywhere.  1 <= B <= max_batch, 1 <= P <= max_prefix.
- * Replaces any previous prefill.  Errors: EINVAL, ECUDA, EDEVICE (id out of range). */
+ * Replaces any previous prefill.  Errors: EINVAL, ECUDA, EDEVICE (id or exit depth out of range, on
+ * the next sync). */
 ALODLM_API int alodlm_prefill(alodlm_t *h, const int32_t *prefix_ids, int B, int P, const int32_t *exit_depth);
+
+/* Append N positions to every sequence's cached prefix: positions P..P+N-1 holding ids (a
+ * decoded block), so that the next step's block sits at P+N.
+ * [digest "Method steps", Algorithm 1 (5); "Technical novelty"]: committed tokens are written
+ * into the sequence and later blocks attend to them; every position is served at its own loop
+ * depth, the deepest it reached standing in for deeper ones.  The new positions go through
+ * what alodlm_prefill does for prefix positions -- Prelude, the Core e_j times (Core KV at depth
+ * d > e_j = the depth-e_j KV), the Coda once on the depth-e_j state -- attending to every
+ * cached position (at its own slot) and causally to each other.  The result equals one
+ * prefill of the longer prefix (prefix attention is causal).
+ * ids: device int32 [B,N] in [0, vocab); B must equal the prefill's; 1 <= N <= max_block and
+ * P + N <= max_prefix.  exit_depth: device int32 [B,N] in 1..k_max (e.g. a decoded block's
+ * commit depths, with positions that held a given id or never committed set to k_max), or
+ * NULL for k_max everywhere.
+ * Errors: EINVAL, ESTATE (before prefill, batch differs), ECUDA, EDEVICE (id or exit depth out
+ * of range, on the next sync).  After an error the cached prefix is invalid until the next
+ * prefill. */
+ALODLM_API int alodlm_append(alodlm_t *h, const int32_t *ids, int B, int N, const int32_t *exit_depth);
 
 /* One denoising step over a block of N positions per sequence (positions P..P+N-1).
  * [digest "Method steps", Algorithm 1 (1)-(5); Eq. 3]:
@@ -140,6 +159,22 @@ ALODLM_API int alodlm_prefill(alodlm_t *h, const int32_t *prefix_ids, int B, int
  * Errors: EINVAL, ESTATE, ECUDA, ETIMEOUT, EDEVICE. */
 ALODLM_API int alodlm_denoise_step(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda,
                         int k_max, int rule, const alodlm_step_out *out);
+
+/* alodlm_denoise_step with sampled commits: a position that commits takes a token drawn from
+ * its distribution p_i^(s) instead of the argmax.
+ * [digest "Method steps", Algorithm 1 (3)]: each committed position samples y_i ~ p_i^(s).
+ * The draw is Gumbel-max with counter-based random numbers, so any other implementation can
+ * draw the same tokens: for vocabulary id v of position i of sequence b at loop s, the 64-bit
+ * word v mod 4 of Philox4x64-10 (Salmon et al., SC 2011) at counter (v div 4, b*N + i, s, 0)
+ * under key (seed, step) gives u = (its 53 high bits + 1/2) * 2^-53 and g_v = -log(-log u);
+ * the token is the id of the largest z_v + g_v (in double precision, the lowest id on ties).
+ * It is fused into the LM-head readout: the logits still never reach global memory.  The
+ * entropy, the halting and the forced commit are as in alodlm_denoise_step (a forced commit
+ * takes its position's sampled token).  Arguments and errors as for alodlm_denoise_step;
+ * `step` is the caller's denoising-step index (part of the key). */
+ALODLM_API int alodlm_denoise_step_sampled(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H,
+                                           float lambda, int k_max, int rule, uint64_t seed, uint64_t step,
+                                           const alodlm_step_out *out);
 
 /* Outputs of a block decode, all caller-owned DEVICE buffers (S = the call's max_steps,
  * K = its k_max). */
@@ -168,6 +203,12 @@ typedef struct {
  * (a failing step returns its own code). */
 ALODLM_API int alodlm_decode_block(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda,
                                    int k_max, int rule, int max_steps, const alodlm_decode_out *out, int *steps_taken);
+
+/* alodlm_decode_block with sampled commits (alodlm_denoise_step_sampled): step t (1-based) of
+ * the decode draws under key (seed, t). */
+ALODLM_API int alodlm_decode_block_sampled(alodlm_t *h, const int32_t *block_ids, int B, int N, float tau_H,
+                                           float lambda, int k_max, int rule, int max_steps, uint64_t seed,
+                                           const alodlm_decode_out *out, int *steps_taken);
 
 /* Wait for the handle's stream; returns ETIMEOUT/EDEVICE if a kernel raised the device error
  * word since the last call (the word is then cleared), ECUDA on a CUDA error. */

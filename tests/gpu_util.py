@@ -127,10 +127,13 @@ def row_rel_err(a: np.ndarray, ref: np.ndarray) -> np.ndarray:
     return np.linalg.norm(a - ref, axis=-1) / np.maximum(np.linalg.norm(ref, axis=-1), 1e-30)
 
 
-def readout_stage_check(case, gpu: dict, r_by_loop: dict, seqs=None, rows_per_loop=None, rng=None, ob=None):
+def readout_stage_check(case, gpu: dict, r_by_loop: dict, seqs=None, rows_per_loop=None, rng=None, ob=None,
+                        sample_key=None):
     """Readout parity on the GPU's own readout states r^(s): the oracle's LM head + entropy +
     argmax + ExitGate in the kernels' precision.  Returns token_at(b, s, i) for the replay and
-    the max deviations.  rows_per_loop (optional) samples that many rows per (b, s)."""
+    the max deviations.  rows_per_loop (optional) samples that many rows per (b, s).  With
+    sample_key the token is the oracle's Gumbel-max draw on the same logits."""
+    from oracle.alodlm_oracle import gumbel_scores
     ob = ob if ob is not None else case.oracle("bf16")
     toks, max_dH, max_dl, n_ties = {}, 0.0, 0.0, 0
     B, K, N = gpu["entropy"].shape
@@ -142,6 +145,9 @@ def readout_stage_check(case, gpu: dict, r_by_loop: dict, seqs=None, rows_per_lo
             if rows_per_loop is not None and len(idx) > rows_per_loop:
                 idx = np.sort(rng.choice(idx, size=rows_per_loop, replace=False))
             H, y, lam, z = ob.readout(r_by_loop[s][b][idx].astype(ob.dt))
+            if sample_key is not None:  # the token is the draw: argmax of z + g
+                z = np.stack([gumbel_scores(z[t], sample_key, b * N + int(i), s) for t, i in enumerate(idx)])
+                y = np.argmax(z, axis=-1)
             dH = np.abs(H - gpu["entropy"][b, s - 1, idx])
             dl = np.abs(lam - gpu["halt"][b, s - 1, idx])
             max_dH, max_dl = max(max_dH, float(dH.max())), max(max_dl, float(dl.max()))
@@ -165,12 +171,13 @@ def readout_stage_check(case, gpu: dict, r_by_loop: dict, seqs=None, rows_per_lo
 
 
 def step_parity(case, gpu: dict, tau: float, lam: float, K: int, rule: int, block_ids: np.ndarray,
-                states=True, oracle=None, seqs=None, rows_per_loop=None, ob=None) -> dict:
+                states=True, oracle=None, seqs=None, rows_per_loop=None, ob=None, sample_key=None) -> dict:
     """The three parity checks of one step (see tests/test_gpu_parity.py).
 
     oracle: a float64 (or float32) oracle whose prefix KV is ready -- prefilled by the oracle
     itself, or read from the library's arena; default: a float64 oracle prefilled here.
-    seqs: the sequences to check end to end (default all; the oracle then holds only these)."""
+    seqs: the sequences to check end to end (default all; the oracle then holds only these).
+    sample_key: (seed, step) of a sampled step (tokens drawn by Gumbel-max)."""
     from oracle.alodlm_oracle import replay_decisions
     B = block_ids.shape[0]
     seq_list = list(range(B)) if seqs is None else [int(b) for b in seqs]
@@ -178,7 +185,7 @@ def step_parity(case, gpu: dict, tau: float, lam: float, K: int, rule: int, bloc
     r_by_loop = {s: case.handle.debug_state(2, s).cpu().numpy() for s in range(1, int(gpu["loops_run"].max()) + 1)}
     # (1) readout stage on the GPU's own r
     token_at, stats = readout_stage_check(case, gpu, r_by_loop, seqs=seq_list, rows_per_loop=rows_per_loop,
-                                          rng=rng, ob=ob)
+                                          rng=rng, ob=ob, sample_key=sample_key)
     # (2) every decision re-taken from the GPU's traces by the oracle's rules: exact
     rep = replay_decisions(block_ids, case.m.mask_id, gpu["entropy"], gpu["cum_halt"], token_at, tau, lam, K, rule)
     assert not rep["ambiguous"], rep["ambiguous"]
@@ -191,7 +198,9 @@ def step_parity(case, gpu: dict, tau: float, lam: float, K: int, rule: int, bloc
         of = case.oracle("fp64")
         of.prefill(case.prefix_ids)
     sel = np.asarray(seq_list)
-    ref = of.denoise_step(block_ids[sel], tau, lam, K, rule, follow=follow_of(gpu, sel), band=E2E_BANDS)
+    assert seqs is None or sample_key is None, "a sampled draw depends on the sequence's index in the batch"
+    ref = of.denoise_step(block_ids[sel], tau, lam, K, rule, follow=follow_of(gpu, sel), band=E2E_BANDS,
+                          sample_key=sample_key)
     sub = {k: gpu[k][sel] for k in ("tokens", "exit_depth", "loops_run", "entropy", "halt", "cum_halt")}
     sub["active_rows"], sub["readout_rows"] = gpu["active_rows"], gpu["readout_rows"]
     compare_decisions(sub, ref, rows=seqs is None)

@@ -110,6 +110,9 @@ def test_null_arguments_are_rejected(L):
     h = ctypes.c_void_p()
     assert lib.alodlm_create(None, None, None, ctypes.byref(h)) == -1
     assert lib.alodlm_prefill(None, None, 1, 1, None) == -1
+    assert lib.alodlm_append(None, None, 1, 1, None) == -1
+    assert lib.alodlm_denoise_step_sampled(None, None, 1, 1, 0.5, 0.5, 1, 0, 1, 1, None) == -1
+    assert lib.alodlm_decode_block_sampled(None, None, 1, 1, 0.5, 0.5, 1, 0, 1, 1, None, None) == -1
     assert lib.alodlm_denoise_step(None, None, 1, 1, 0.5, 0.5, 1, 0, None) == -1
     assert lib.alodlm_decode_block(None, None, 1, 1, 0.5, 0.5, 1, 0, 1, None, None) == -1
     assert lib.alodlm_sync(None) == -1
