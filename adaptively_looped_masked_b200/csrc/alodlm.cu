@@ -83,6 +83,26 @@ void klaunch_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
     cfg.numAttrs = (ALODLM_PDL && st != nullptr && st != cudaStreamLegacy && st != cudaStreamPerThread) ? 2 : 1;
     cudaLaunchKernelEx(&cfg, kern, args...);
 }
+// The same with a thread-block cluster of (cluster_x, 1, 1) CTAs.
+template <typename... KArgs, typename... Args>
+void klaunch_cluster_x(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_x,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster_x;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (ALODLM_PDL && st != nullptr && st != cudaStreamLegacy && st != cudaStreamPerThread) ? 2 : 1;
+    cudaLaunchKernelEx(&cfg, kern, args...);
+}
 constexpr int PREFILL_ROWS = 16384;         // rows of one prefill group (sequences x P)
 constexpr size_t SPLITK_WS_FLOATS = 32u << 20;  // split-K partials (128 MB)
 constexpr size_t ATTN_WS_FLOATS = 16u << 20;    // split-KV partials (64 MB)
@@ -139,11 +159,49 @@ void set_persist_attr() {
     cudaFuncSetAttribute(gemm::gemm_persist_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)gemm::Cfg<BN>::SMEM_PERSIST);
 }
+template <int EPI>
+void set_pair_attr() {
+    cudaFuncSetAttribute(gemm::gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)gemm::PairCfg::SMEM);
+}
 template <int BN, int EPI>
 void set_sk_attr() {
     cudaFuncSetAttribute(gemm::gemm_sk_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)gemm::SkCfg<BN>::SMEM);
 }
+// CTA-pair kernel: clusters of two CTAs, as many pairs as the device holds at once (at most one
+// per two SMs), each walking 256 x 256 tiles
+#ifndef ALODLM_PAIR_GEMM
+#define ALODLM_PAIR_GEMM 1
+#endif
+template <int EPI>
+int pair_slots() {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 0;
+    if (!cached[dev]) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (NUM_SMS_HINT / 2));
+        cfg.blockDim = dim3(192);
+        cfg.dynamicSmemBytes = gemm::PairCfg::SMEM;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, gemm::gemm_pair_kernel<EPI>, &cfg) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = -1;  // the pair kernel cannot run here: the single-CTA kernels take its shapes
+        }
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 bool init_kernel_attrs() {
     static bool done[64] = {false};
     int dev = 0;
@@ -169,6 +227,9 @@ bool init_kernel_attrs() {
     set_persist_attr<256, gemm::EPI_ADD>();
     set_persist_attr<256, gemm::EPI_SWIGLU>();
     set_persist_attr<256, gemm::EPI_READOUT>();
+    set_pair_attr<gemm::EPI_F32>();
+    set_pair_attr<gemm::EPI_ADD>();
+    set_pair_attr<gemm::EPI_SWIGLU>();
     set_sk_attr<32, gemm::EPI_F32>();
     set_sk_attr<32, gemm::EPI_ADD>();
     set_sk_attr<32, gemm::EPI_SWIGLU>();
@@ -179,6 +240,11 @@ bool init_kernel_attrs() {
     cudaFuncSetAttribute(attn_tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_tc::SMEM);
     cudaFuncSetAttribute(attn::attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 5 * 64 * 128 * 2);
     done[dev] = cudaGetLastError() == cudaSuccess;
+    if (done[dev]) {  // the pair kernel's occupancy, looked up here (never during a graph capture)
+        pair_slots<gemm::EPI_F32>();
+        pair_slots<gemm::EPI_ADD>();
+        pair_slots<gemm::EPI_SWIGLU>();
+    }
     return done[dev];
 }
 
@@ -240,6 +306,13 @@ void launch_persist(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int
     const int grid = std::max(1, std::min(num_sms, tiles));
     klaunch(gemm::gemm_persist_kernel<BN, EPI>, grid, 192, gemm::Cfg<BN>::SMEM_PERSIST, st, tA, tB, rowsA, rowsB, rowsA_dyn,
             k_tiles, a_fastest, tiled, ep, err);
+}
+
+template <int EPI>
+void launch_pair(const CUtensorMap &tA, const CUtensorMap &tB, int rowsA, int rowsB, int k_tiles, int tiled_a,
+                 const gemm::EpiParams &ep, int *err, cudaStream_t st, int n_pairs) {
+    klaunch_cluster_x(gemm::gemm_pair_kernel<EPI>, dim3(2 * n_pairs), dim3(192), gemm::PairCfg::SMEM, st, 2, tA, tB,
+                      rowsA, rowsB, k_tiles, tiled_a, ep, err);
 }
 
 template <int EPI>
@@ -334,6 +407,23 @@ int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_b
         }
     }
     GemmShape g = plan_gemm(M, Nw, K);
+    if (ALODLM_PAIR_GEMM && g.splits == 1 && g.bn >= 128 && M > 128) {
+        // 256 x 256 tiles on CTA pairs once they fill every pair at least once
+        const int slots = epi == gemm::EPI_F32 ? pair_slots<gemm::EPI_F32>()
+                          : epi == gemm::EPI_ADD ? pair_slots<gemm::EPI_ADD>() : pair_slots<gemm::EPI_SWIGLU>();
+        const int tiles = cdiv(Nw, 256) * cdiv(M, 256);
+        if (slots > 0 && tiles >= slots) {
+            const CUtensorMap *tB = map_for_bn(128);
+            if (!tB) return -1;
+            if (epi == gemm::EPI_F32)
+                launch_pair<gemm::EPI_F32>(tmW, *tB, Nw, M, g.k_tiles, w_tiled, ep, env.err, env.st, slots);
+            else if (epi == gemm::EPI_ADD)
+                launch_pair<gemm::EPI_ADD>(tmW, *tB, Nw, M, g.k_tiles, w_tiled, ep, env.err, env.st, slots);
+            else
+                launch_pair<gemm::EPI_SWIGLU>(tmW, *tB, Nw, M, g.k_tiles, w_tiled, ep, env.err, env.st, slots);
+            return 1;
+        }
+    }
     const CUtensorMap *tB = map_for_bn(g.bn);
     if (!tB) return -1;
     if (g.splits == 1 && g.bn >= 128) {

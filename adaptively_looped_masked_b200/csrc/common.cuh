@@ -267,6 +267,60 @@ __device__ __forceinline__ uint64_t umma_sdesc_sw128(uint32_t saddr) {
 }
 
 // ---------------------------------------------------------------------------------
+// CTA pairs: tcgen05 with cta_group::2 (two CTAs of a cluster, ranks 2k and 2k+1, run one
+// MMA of M = 256: each holds 128 rows of A and half of B in its own shared memory and gets its
+// 128 accumulator rows in its own tensor memory).  No multicast anywhere: every load lands in
+// the CTA that issues it.
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// allocate / release the same tensor-memory columns in both CTAs of the pair (one warp of each)
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *smem_slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D[tmem, both CTAs] (+)= A * B^T over the pair, kind::f16 (bf16 in, f32 accumulate); issued by
+// one thread of the even CTA
+__device__ __forceinline__ void umma_f16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// arrive on the mbarrier at shared::cluster address `bar` (this CTA's or its peer's) once every
+// pair MMA issued so far by this thread has completed
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+// TMA 2D load into this CTA's shared memory whose completed bytes count on the mbarrier at
+// shared::cluster address `bar`, which may be the peer's (the pair's MMA waits there)
+__device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+        "%4}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(map), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+// arrive (release, cluster scope) on the mbarrier at shared::cluster address `bar`
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// ---------------------------------------------------------------------------------
 // misc math
 // ---------------------------------------------------------------------------------
 __device__ __forceinline__ float warp_sum(float v) {

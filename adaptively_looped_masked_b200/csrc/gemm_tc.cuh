@@ -978,3 +978,203 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 }  // namespace gemm
+
+namespace gemm {
+
+// ---------------------------------------------------------------------------------
+// Persistent GEMM on CTA pairs (cta_group::2) for linear layers over many activation rows.
+// A cluster of two CTAs computes 256 x 256 output tiles: 256 weight rows (each CTA loads its
+// own 128, in the tiled weight layout) x 256 activation rows (each CTA loads its own 128), so
+// per k-tile an SM streams 32 KB for 128 x 256 x 64 multiply-adds, two thirds of what a
+// 128 x 256 tile on one SM needs.  The even CTA's MMA thread issues M = 256, N = 256 MMAs over
+// both CTAs' shared memory; each CTA receives its 128 accumulator rows in its own tensor memory
+// (double-buffered) and runs the usual staged epilogue on them.  Both CTAs' loads complete on
+// the even CTA's stage barrier (which expects the bytes of both); the MMA releases each stage,
+// and announces each finished accumulator, to both CTAs with one commit per CTA; both CTAs'
+// epilogues report a drained accumulator to the even CTA.  No load is multicast.
+// ---------------------------------------------------------------------------------
+struct PairCfg {
+    static constexpr int TN = 256;                        // activation rows per pair tile
+    static constexpr int HALF = 128;                      // ... loaded by each CTA
+    static constexpr int STAGES = 6;
+    static constexpr uint32_t A_BYTES = BM * BK * 2;      // this CTA's 128 weight rows x 64
+    static constexpr uint32_t B_BYTES = HALF * BK * 2;    // this CTA's 128 activation rows x 64
+    static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr uint32_t TMEM_COLS = 2 * TN;         // two 128 x 256 f32 accumulators
+    static constexpr size_t STG_BYTES = 64 * BM * 4;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + STG_BYTES;
+};
+
+__device__ __forceinline__ void tma_operand_pair(void *dst, const CUtensorMap *map, uint32_t bar, bool tiled, int tile,
+                                                 int tile_rows, int kt, int k_tiles) {
+    if (tiled)
+        tma_load_2d_pair(dst, map, bar, 0, (tile * k_tiles + kt) * tile_rows);
+    else
+        tma_load_2d_pair(dst, map, bar, kt * BK, tile * tile_rows);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int rowsA,
+                     int rowsB, int k_tiles, int tiled_a, EpiParams ep, int *err) {
+    static_assert(EPI == EPI_F32 || EPI == EPI_ADD || EPI == EPI_SWIGLU, "linear-layer epilogues only");
+    using C = PairCfg;
+    constexpr int STAGES = C::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * C::STAGE_BYTES);  // used in the even CTA
+    uint64_t *empty = full + STAGES;
+    uint64_t *tfull = empty + STAGES;
+    uint64_t *tempty = tfull + 2;    // used in the even CTA: 4 epilogue warps of each CTA arrive
+    uint64_t *mma_done = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    float *stg = reinterpret_cast<float *>(smem + STAGES * C::STAGE_BYTES + 256);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank() & 1u;  // 0: the CTA whose thread issues the pair's MMAs
+    const int pair = (int)(blockIdx.x >> 1), n_pairs = (int)(gridDim.x >> 1);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull + b, 1);
+            mbar_init(tempty + b, 8);
+        }
+        mbar_init(mma_done, 1);
+        fence_mbarrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_arrive_release();
+    cluster_wait_acquire();  // both CTAs' barriers are initialised before any cross-CTA signal
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_trigger();
+    const int n_a = (rowsA + 2 * BM - 1) / (2 * BM), n_b = (rowsB + C::TN - 1) / C::TN;
+    const int total = n_a * n_b;
+    // shared::cluster addresses: the even CTA's stage and drain barriers, and each CTA's own
+    const uint32_t full_lead = cluster_map(smem_u32(full), 0u);
+    const uint32_t tempty_lead = cluster_map(smem_u32(tempty), 0u);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int t = pair, issued = 0, g = 0, pre = 0;
+            bool ok = true;
+            // the weights do not depend on earlier kernels: the first stages of the first tile are
+            // requested before waiting for them
+            if (t < total) {
+                const int a = t / n_b;
+                pre = min(k_tiles, STAGES);
+                for (int i = 0; i < pre; ++i) {
+                    if (rank == 0) mbar_arrive_expect_tx(full + i, 2 * C::STAGE_BYTES);
+                    tma_operand_pair(smem + i * C::STAGE_BYTES, &tmA, full_lead + 8u * i, tiled_a & 1, 2 * a + rank, BM,
+                                     i, k_tiles);
+                }
+            }
+            pdl_wait();
+            if (t < total) {
+                const int b = t % n_b;
+                for (int i = 0; i < pre; ++i)
+                    tma_load_2d_pair(smem + i * C::STAGE_BYTES + C::A_BYTES, &tmB, full_lead + 8u * i, i * BK,
+                                     b * C::TN + (int)rank * C::HALF);
+            }
+            issued = pre;
+            for (; t < total && ok; t += n_pairs) {
+                const int a = t / n_b, b = t % n_b;
+                for (int kt = 0; kt < k_tiles; ++kt, ++g) {
+                    if (g < pre) continue;
+                    const int s = g % STAGES;
+                    if (!mbar_wait(empty + s, ((uint32_t)(g / STAGES) & 1u) ^ 1u, err)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0) mbar_arrive_expect_tx(full + s, 2 * C::STAGE_BYTES);
+                    uint8_t *sa = smem + s * C::STAGE_BYTES;
+                    tma_operand_pair(sa, &tmA, full_lead + 8u * s, tiled_a & 1, 2 * a + rank, BM, kt, k_tiles);
+                    tma_load_2d_pair(sa + C::A_BYTES, &tmB, full_lead + 8u * s, kt * BK, b * C::TN + (int)rank * C::HALF);
+                    issued = g + 1;
+                }
+            }
+            // no copy into this CTA's shared memory may still be in flight when it exits: a stage
+            // is released (to both CTAs) only after the MMAs that read it, i.e. after it landed
+            for (int i = max(0, issued - STAGES); i < issued; ++i)
+                mbar_wait(empty + (i % STAGES), (uint32_t)(i / STAGES) & 1u, err);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16(2 * BM, C::TN);
+            const uint32_t empty_self = cluster_map(smem_u32(empty), 0u), empty_peer = cluster_map(smem_u32(empty), 1u);
+            const uint32_t tfull_self = cluster_map(smem_u32(tfull), 0u), tfull_peer = cluster_map(smem_u32(tfull), 1u);
+            int g = 0, li = 0;
+            bool ok = true;
+            for (int t = pair; t < total && ok; t += n_pairs, ++li) {
+                const int buf = li & 1;
+                if (!mbar_wait(tempty + buf, ((uint32_t)(li >> 1) & 1u) ^ 1u, err)) break;
+                tc_fence_after();
+                for (int kt = 0; kt < k_tiles; ++kt, ++g) {
+                    const int s = g % STAGES;
+                    if (!mbar_wait(full + s, (uint32_t)(g / STAGES) & 1u, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+                    const uint64_t da = umma_sdesc_sw128(sa);
+                    const uint64_t db = umma_sdesc_sw128(sa + C::A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        umma_f16_pair(tmem_base + buf * C::TN, da + 2 * k, db + 2 * k, idesc, (kt > 0 || k > 0) ? 1u : 0u);
+                    umma_commit_pair(empty_self + 8u * s);
+                    umma_commit_pair(empty_peer + 8u * s);
+                }
+                if (!ok) break;
+                umma_commit_pair(tfull_self + 8u * buf);
+                umma_commit_pair(tfull_peer + 8u * buf);
+            }
+            // every MMA issued above has completed before tensor memory is released
+            umma_commit_pair(smem_u32(mma_done));
+            mbar_wait(mma_done, 0, err);
+        }
+    } else {
+        const int q = warp & 3;
+        const int row = q * 32 + lane;  // row of this CTA's 128-row half = TMEM lane
+        pdl_wait();
+        int li = 0;
+        for (int t = pair; t < total; t += n_pairs, ++li) {
+            const int a = t / n_b, b = t % n_b;
+            const int buf = li & 1;
+            const bool ready = epilogue_all(mbar_wait(tfull + buf, (uint32_t)(li >> 1) & 1u, err));
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * C::TN;
+            const int a128 = 2 * a + (int)rank;  // this CTA's 128 weight rows
+            if (ready) {
+                for (int c0 = 0; c0 < C::TN; c0 += 64) {
+                    if (b * C::TN + c0 >= rowsB) break;  // uniform across the epilogue warps
+                    float v[64];
+                    acc_ld<1, C::TN, 64>(taddr, c0, v);
+                    staged_cols<EPI>(stg, v, row, a128, b * C::TN + c0, rowsA, rowsB, ep);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty_lead + 8u * buf);
+            if (!ready) break;
+        }
+    }
+    tc_fence_before();
+    cluster_arrive_release();
+    cluster_wait_acquire();  // the pair is done with each other's barriers and tensor memory
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace gemm

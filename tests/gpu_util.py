@@ -1,28 +1,31 @@
 """Helpers of the GPU tests: build a library handle and an oracle from the same seeded
 inputs, and compare a step's outputs with the oracle's.
 
-Every tolerance and band below is a fixed number.
+Every tolerance and band below is fixed before the GPU runs.
 
 Readout stage, on the GPU's own readout states r^(s), i.e. the same inputs on both sides:
   ENTROPY_TOL  |dH| <= 1e-2 nats
   GATE_TOL     |d lambda| <= 1e-3
   BAND         the argmax must match unless the top-two logit gap is below 1e-3
 
-End to end, the float64 oracle running the whole step from the same ids and weights:
-  STATE_REL_TOL    per-row ||d|| / ||ref|| <= 2e-2 for h^(s-1), h~^(s), r^(s) and the logits
-  E2E_ENTROPY_TOL  |dH| <= 0.1 nats; also the band within which a commit on H <= tau may go
-                   either way
-  E2E_HALT_TOL     |d lambda|, |d a| <= 1e-2; also the band of decisions on a or on its mean
-  E2E_ARGMAX_BAND  top-two logit gap below which either token is a correct argmax (the GPU's
-                   token must then score within the band of the oracle's maximum)
+End to end, the float64 oracle running the whole step from the same ids and weights, at loop
+s (e2e_tolerances): per-row relative deviation of the states h^(s-1), h~^(s), r^(s) and of
+the logits, |dH|, |d lambda| and |d a|, and the top-two logit gap below which either token
+is a correct argmax.  Each is twice the spread between the oracle in its bf16 precision and
+the oracle in float64 at that loop (tests/golden/oracle_spread.json, written by
+make_oracle_spread.py from the oracle alone), and never below the fixed values 2e-2 (states,
+logits), 1e-2 nats, 1e-3 (halts, argmax gap).  The entropy, halt and argmax values are also
+the bands within which a decision may go either way: outside them every decision (commit,
+exit depth, token, halt, forced pick) must be the oracle's own.
 
-Outside those bands every decision (commit, exit depth, token, halt, forced pick) must be
-the oracle's own.  Why the end-to-end numbers are what they are: with bf16 activations,
-two correct implementations that round at the same points but add in a different order
-(the oracle itself in float32 and in float64) already drift apart end to end by up to
-0.05 nats at the synthetic configs' logit scale (logit std 12.8); the end-to-end bands
-are twice that spread.
+Why a per-loop table: with bf16 activations the rounding of every matrix operand adds an
+independent error at every layer application, so two correct implementations drift apart as
+the loop deepens -- at the Qwen3-1.7B shape the bf16 oracle lies 3.6e-2 (state) and 0.56
+nats from the float64 oracle after 8 loops of 20 layers; at the tiny config 7e-3 and 0.05.
 """
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -34,10 +37,31 @@ ENTROPY_TOL = 1e-2
 GATE_TOL = 1e-3
 BAND = 1e-3
 STATE_REL_TOL = 2e-2
-E2E_ENTROPY_TOL = 0.1
-E2E_HALT_TOL = 1e-2
-E2E_ARGMAX_BAND = 0.5
-E2E_BANDS = dict(entropy=E2E_ENTROPY_TOL, halt=E2E_HALT_TOL, argmax=E2E_ARGMAX_BAND)
+SPREAD_FACTOR = 2.0
+SPREAD_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "oracle_spread.json")
+_SPREAD_MODEL = {"tiny_fullcore": "tiny"}
+
+
+def e2e_tolerances(model: str, K: int) -> dict:
+    """Per-loop end-to-end tolerances, lists indexed by s - 1 (s = 1..K): state, logits,
+    entropy, halt, argmax.  A deeper loop is never held tighter than a shallower one."""
+    with open(SPREAD_FILE) as f:
+        rows = json.load(f)[_SPREAD_MODEL.get(model, model)]["per_loop"]
+    floor = dict(state=STATE_REL_TOL, logits=STATE_REL_TOL, entropy=ENTROPY_TOL, halt=GATE_TOL, gap=BAND)
+    run = {k: 0.0 for k in floor}
+    out = {k: [] for k in floor}
+    for s in range(1, K + 1):
+        r = rows[min(s, len(rows)) - 1]
+        for k in floor:
+            run[k] = max(run[k], r[k])
+            out[k].append(max(floor[k], SPREAD_FACTOR * run[k]))
+    out["argmax"] = out.pop("gap")
+    return out
+
+
+def e2e_bands(model: str, K: int) -> dict:
+    t = e2e_tolerances(model, K)
+    return dict(entropy=t["entropy"], halt=t["halt"], argmax=t["argmax"])
 
 
 class Case:
@@ -199,7 +223,9 @@ def step_parity(case, gpu: dict, tau: float, lam: float, K: int, rule: int, bloc
         of.prefill(case.prefix_ids)
     sel = np.asarray(seq_list)
     assert seqs is None or sample_key is None, "a sampled draw depends on the sequence's index in the batch"
-    ref = of.denoise_step(block_ids[sel], tau, lam, K, rule, follow=follow_of(gpu, sel), band=E2E_BANDS,
+    tol = e2e_tolerances(case.m.name, K)
+    ref = of.denoise_step(block_ids[sel], tau, lam, K, rule, follow=follow_of(gpu, sel),
+                          band=dict(entropy=tol["entropy"], halt=tol["halt"], argmax=tol["argmax"]),
                           sample_key=sample_key)
     sub = {k: gpu[k][sel] for k in ("tokens", "exit_depth", "loops_run", "entropy", "halt", "cum_halt")}
     sub["active_rows"], sub["readout_rows"] = gpu["active_rows"], gpu["readout_rows"]
@@ -214,7 +240,7 @@ def step_parity(case, gpu: dict, tau: float, lam: float, K: int, rule: int, bloc
             for which, key in keys:
                 rel = row_rel_err(dbg[(which, s)][b], ref[key][j][s - 1])
                 worst["state"] = max(worst["state"], float(rel.max()))
-                assert rel.max() <= STATE_REL_TOL, (key, b, s, rel.max())
+                assert rel.max() <= tol["state"][s - 1], (key, b, s, rel.max(), tol["state"][s - 1])
             idx = np.nonzero(~np.isnan(gpu["entropy"][b, s - 1]))[0]
             if len(idx) == 0:
                 continue
@@ -223,14 +249,14 @@ def step_parity(case, gpu: dict, tau: float, lam: float, K: int, rule: int, bloc
             dz = (dbg[(2, s)][b][idx].astype(z_ref.dtype) - r_ref) @ W.T
             lrel = np.linalg.norm(dz, axis=-1) / np.linalg.norm(z_ref, axis=-1)
             worst["logits"] = max(worst["logits"], float(lrel.max()))
-            assert lrel.max() <= STATE_REL_TOL, ("logits", b, s, lrel.max())
+            assert lrel.max() <= tol["logits"][s - 1], ("logits", b, s, lrel.max(), tol["logits"][s - 1])
             dH = np.abs(gpu["entropy"][b, s - 1, idx] - ref["entropy"][j, s - 1, idx])
             worst["entropy"] = max(worst["entropy"], float(dH.max()))
-            assert dH.max() <= E2E_ENTROPY_TOL, ("entropy", b, s, float(dH.max()))
+            assert dH.max() <= tol["entropy"][s - 1], ("entropy", b, s, float(dH.max()), tol["entropy"][s - 1])
             for key in ("halt", "cum_halt"):
                 da = np.abs(gpu[key][b, s - 1, idx] - ref[key][j, s - 1, idx])
                 worst["halt"] = max(worst["halt"], float(da.max()))
-                assert da.max() <= E2E_HALT_TOL, (key, b, s, float(da.max()))
+                assert da.max() <= tol["halt"][s - 1], (key, b, s, float(da.max()), tol["halt"][s - 1])
     differing = [f for f in ref["followed"] if f.get("own") != f.get("taken")]
     stats.update({f"e2e_{k}": v for k, v in worst.items()})
     stats["e2e_followed"] = len(ref["followed"])

@@ -19,7 +19,7 @@ import torch
 
 from oracle.alodlm_oracle import decode_block
 from synth import MODELS, WORKLOADS, make_block_ids, make_exit_depths
-from tests.gpu_util import E2E_BANDS, STATE_REL_TOL, Case, follow_of, row_rel_err, step_parity
+from tests.gpu_util import e2e_bands, STATE_REL_TOL, Case, follow_of, row_rel_err, step_parity
 
 pytestmark = pytest.mark.gpu
 
@@ -124,7 +124,7 @@ def test_two_blocks_decoded_in_a_stream():
             step_ex = np.where(got["commit_step"] == t + 1, got["commit_depth"], 0)
             follow.append(dict(tokens=step_tok, exit_depth=step_ex, loops_run=got["loops"][t]))
             ids = step_tok
-        ref = decode_block(of, block, tau, lam, K, rule, follow_steps=follow, band=E2E_BANDS)
+        ref = decode_block(of, block, tau, lam, K, rule, follow_steps=follow, band=e2e_bands(m.name, K))
         assert ref["steps"] == T
         for key in ("tokens", "commit_step", "commit_depth", "steps_run"):
             np.testing.assert_array_equal(ref[key], got[key], err_msg=f"block {blk_i} {key}")

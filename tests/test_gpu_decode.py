@@ -16,7 +16,7 @@ import torch
 
 from oracle.alodlm_oracle import decode_block
 from synth import MODELS, WORKLOADS
-from tests.gpu_util import E2E_BANDS, Case, follow_of, step_parity
+from tests.gpu_util import e2e_bands, Case, follow_of, step_parity
 
 pytestmark = pytest.mark.gpu
 
@@ -25,7 +25,10 @@ def _np(d):
     return {k: (v.cpu().numpy() if torch.is_tensor(v) else v) for k, v in d.items()}
 
 
-@pytest.mark.parametrize("name,tau,lam", [("tiny", 0.6, 0.5), ("tiny", 0.1, 0.9), ("mid", 0.6, 0.5)])
+# (mid, -1, 0.5) is the pages' conservative quality mode (digest "Results", Table 1): no entropy
+# passes tau, so under the paper's rule every step commits exactly its lowest-entropy position
+@pytest.mark.parametrize("name,tau,lam", [("tiny", 0.6, 0.5), ("tiny", 0.1, 0.9), ("mid", 0.6, 0.5),
+                                          ("mid", -1.0, 0.5)])
 @pytest.mark.parametrize("rule", [0, 1])
 def test_decode_block_stepwise_and_oracle(name, tau, lam, rule):
     wl = WORKLOADS[name]
@@ -48,6 +51,9 @@ def test_decode_block_stepwise_and_oracle(name, tau, lam, rule):
         ids = gpu["tokens"]
     T = len(steps)
     assert dec["steps"] == T and not (ids == m.mask_id).any()
+    if tau < 0 and rule == 0:  # quality mode: one commit per sequence per step while it has masks
+        for _, g in steps:
+            assert ((g["exit_depth"] > 0).sum(axis=1) <= 1).all()
     np.testing.assert_array_equal(dec["tokens"], ids)
     cs = np.zeros_like(block)
     cd = np.zeros_like(block)
@@ -68,7 +74,7 @@ def test_decode_block_stepwise_and_oracle(name, tau, lam, rule):
     # the oracle composes the same steps, taking the GPU's decisions only inside the fixed bands
     of = case.oracle("fp64")
     of.prefill(case.prefix_ids)
-    ref = decode_block(of, block, tau, lam, K, rule, follow_steps=[follow_of(g) for _, g in steps], band=E2E_BANDS)
+    ref = decode_block(of, block, tau, lam, K, rule, follow_steps=[follow_of(g) for _, g in steps], band=e2e_bands(m.name, K))
     assert ref["steps"] == T
     for key in ("tokens", "commit_step", "commit_depth", "steps_run"):
         np.testing.assert_array_equal(ref[key], dec[key])

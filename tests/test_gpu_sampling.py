@@ -18,7 +18,7 @@ import torch
 
 from oracle.alodlm_oracle import decode_block
 from synth import MODELS, WORKLOADS
-from tests.gpu_util import E2E_BANDS, Case, follow_of, step_parity
+from tests.gpu_util import e2e_bands, Case, follow_of, step_parity
 
 pytestmark = pytest.mark.gpu
 
@@ -87,7 +87,8 @@ def test_sampled_decode_matches_oracle(mid, rule):
         ids = step_tok
     of = mid.oracle("fp64")
     of.prefill(mid.prefix_ids)
-    ref = decode_block(of, mid.block_ids, tau, lam, K, rule, follow_steps=follow, band=E2E_BANDS, sample_seed=seed)
+    ref = decode_block(of, mid.block_ids, tau, lam, K, rule, follow_steps=follow, band=e2e_bands("mid", K),
+                       sample_seed=seed)
     assert ref["steps"] == T
     for key in ("tokens", "commit_step", "commit_depth", "steps_run"):
         np.testing.assert_array_equal(ref[key], got[key], err_msg=key)
