@@ -470,14 +470,16 @@ struct TimedLaunch {
     cudaEvent_t e0, e1;
 };
 
+// A loop's recorded graph bakes in everything below: the prefix length and the deepest built
+// Core depth fix the attended positions and slots.
 struct GraphKey {
-    int s, n_act, cur, hi, N, K, rule;
+    int s, n_act, cur, hi, N, K, rule, P, depth;
     float tau, lam;
     const void *p0, *p1, *p2, *p3, *p4, *p5, *p6, *p7;
     bool operator==(const GraphKey &o) const {
         return s == o.s && n_act == o.n_act && cur == o.cur && hi == o.hi && N == o.N && K == o.K &&
-               rule == o.rule && tau == o.tau && lam == o.lam && p0 == o.p0 && p1 == o.p1 && p2 == o.p2 &&
-               p3 == o.p3 && p4 == o.p4 && p5 == o.p5 && p6 == o.p6 && p7 == o.p7;
+               rule == o.rule && P == o.P && depth == o.depth && tau == o.tau && lam == o.lam && p0 == o.p0 &&
+               p1 == o.p1 && p2 == o.p2 && p3 == o.p3 && p4 == o.p4 && p5 == o.p5 && p6 == o.p6 && p7 == o.p7;
     }
 };
 
@@ -519,8 +521,12 @@ struct alodlm {
     // prefill state
     int B = 0, P = 0, last_N = 0;
     bool prefilled = false;
+    int depth_built = 0;  // Core depths 1..depth_built are materialised for every cached position
     int *exit_dev = nullptr;
     int *app_exit = nullptr;  // exit depths of the positions being appended [max_batch * max_block]
+    // depth-on-demand prefill: the compacted rows of one depth (row tables rows_cap, slot tables max_batch)
+    int *pf_row_seq = nullptr, *pf_row_u = nullptr, *pf_row_t = nullptr, *pf_gather = nullptr;
+    int *pf_seq_off = nullptr, *pf_seq_cnt = nullptr;
     int *iota = nullptr;
 
     // activation scratch (rows_cap rows)
@@ -837,6 +843,16 @@ int run_layer(alodlm *h, int li, int slot, int M, const RowMap &map, int n_seq, 
     return ALODLM_OK;
 }
 
+// the depth fallback of one Core slot on its own (a depth that no position runs)
+void launch_fallback(alodlm *h, int slot, const Fallback &fb) {
+    const long long so = (long long)fb.src_slot * h->slot_elems;
+    bf16 *kc = h->kv_k + (long long)slot * h->slot_elems, *vc = h->kv_v + (long long)slot * h->slot_elems;
+    LAUNCH(KC_OTHER, 8.0 * fb.nb * h->nkv * fb.n * h->hd, 0.0,
+           (klaunch(k::kv_fallback_kernel, dim3(fb.nb, h->nkv), 256, 0, h->stream, fb.exit, fb.n, fb.pos0, fb.b0,
+                    fb.depth, (const bf16 *)(h->kv_k + so), (const bf16 *)(h->kv_v + so), kc, vc, h->seq_stride,
+                    h->head_stride, h->hd)));
+}
+
 int check_launch(alodlm *h, const char *what) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(h, e, what);
@@ -1084,7 +1100,10 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
         (rc = dalloc(h, &h->seq_of[1], cfg->max_batch)) || (rc = dalloc(h, &h->old_slot, cfg->max_batch)) ||
         (rc = dalloc(h, &h->counts, 4)) || (rc = dalloc(h, &h->d_err, 1)) || (rc = dalloc(h, &h->iota, cfg->max_batch)) ||
         (rc = dalloc(h, &h->exit_dev, (size_t)cfg->max_batch * cfg->max_prefix)) ||
-        (rc = dalloc(h, &h->app_exit, BN_)) ||
+        (rc = dalloc(h, &h->app_exit, BN_)) || (rc = dalloc(h, &h->pf_row_seq, h->rows_cap)) ||
+        (rc = dalloc(h, &h->pf_row_u, h->rows_cap)) || (rc = dalloc(h, &h->pf_row_t, h->rows_cap)) ||
+        (rc = dalloc(h, &h->pf_gather, h->rows_cap)) || (rc = dalloc(h, &h->pf_seq_off, cfg->max_batch)) ||
+        (rc = dalloc(h, &h->pf_seq_cnt, cfg->max_batch)) ||
         (rc = dalloc(h, &h->dec_tok[0], BN_)) || (rc = dalloc(h, &h->dec_tok[1], BN_)) ||
         (rc = dalloc(h, &h->dec_ex, BN_)) || (rc = dalloc(h, &h->dec_loops, cfg->max_batch)) ||
         (rc = dalloc(h, &h->dec_rows, 2 * (size_t)cfg->k_max)) || (rc = dalloc(h, &h->dec_left, 1)) ||
@@ -1236,46 +1255,132 @@ int alodlm_sync(alodlm_t *h) {
 
 namespace {
 
-// Prefix rows through the whole stack, writing their K/V into every slot of the arena:
-// sequences b0 .. b0+nb-1, positions pos0 .. pos0+n-1 holding ids[b * n + t], attending
+// Prefix rows through the whole stack, writing their K/V into Core depths 1..n_depths of the
+// arena: sequences b0 .. b0+nb-1, positions pos0 .. pos0+n-1 holding ids[b * n + t], attending
 // causally to keys [0, pos0 + n) (the positions before pos0 are already in the arena, every
 // slot resolved to its depth).  A position with exit depth e runs the Core e times: at depth
 // d > e its Core K/V is the depth-e K/V (copied from slot d-1), and the Coda runs once on its
-// depth-e state.  exit: device [B, n] exit depths in 1..k_max, or nullptr for k_max everywhere.
-int build_prefix_rows(alodlm *h, const int32_t *ids, int b0, int nb, int n, int pos0, const int *exit) {
+// depth-e state.  Depth on demand: at depth d only the positions with e >= d run the Core (the
+// rows are compacted to them), and no depth beyond n_depths is built.  exit: device [B, n]
+// exit depths in 1..k_max with e_host its host copy (rows b * n + t), or nullptr / empty for
+// k_max everywhere (then n_depths = k_max and every row runs every depth).
+int build_prefix_rows(alodlm *h, const int32_t *ids, int b0, int nb, int n, int pos0, const int *exit,
+                      const std::vector<int> &e_host, int n_depths) {
     const alodlm_cfg &c = h->cfg;
     const int M = nb * n, kv_len = pos0 + n;
-    RowMap map{h->iota + b0, n, pos0};
+    RowMap full_map{h->iota + b0, n, pos0};
     float *x = h->hbuf[0];
     int rc;
     LAUNCH(KC_OTHER, 6.0 * M * h->H, 0.0,
-           (klaunch(k::embed_kernel, M, 256, 0, h->stream, ids, n, map, h->embed, h->V, h->H, x, h->d_err)));
+           (klaunch(k::embed_kernel, M, 256, 0, h->stream, ids, n, full_map, h->embed, h->V, h->H, x, h->d_err)));
     for (int l = 0; l < c.n_prelude; ++l)
-        if ((rc = run_layer(h, l, slot_prelude(h, l), M, map, nb, kv_len, 1, x, nullptr))) return rc;
-    for (int d = 1; d <= c.k_max; ++d) {
+        if ((rc = run_layer(h, l, slot_prelude(h, l), M, full_map, nb, kv_len, 1, x, nullptr))) return rc;
+    // rows of the current depth as (slot, position) pairs, in slot then position order
+    std::vector<int> cur_seq, cur_t;
+    for (int jj = 0; jj < nb; ++jj)
+        for (int t = 0; t < n; ++t) {
+            cur_seq.push_back(jj);
+            cur_t.push_back(t);
+        }
+    int par = 0;  // x = hbuf[par]
+    for (int d = 1; d <= n_depths; ++d) {
+        RowMap map = full_map;
+        int Md = (int)cur_seq.size();
+        if (exit) {
+            // the rows that still run at depth d
+            std::vector<int> nseq, nt, gather, off(nb, 0), cnt(nb, 0), u;
+            for (int m = 0; m < Md; ++m)
+                if (e_host[(size_t)(b0 + cur_seq[m]) * n + cur_t[m]] >= d) {
+                    gather.push_back(m);
+                    nseq.push_back(cur_seq[m]);
+                    nt.push_back(cur_t[m]);
+                    u.push_back(cnt[cur_seq[m]]++);
+                }
+            const int Mn = (int)nseq.size();
+            if (Mn != Md && Mn > 0) {
+                cudaMemcpyAsync(h->pf_gather, gather.data(), Mn * sizeof(int), cudaMemcpyHostToDevice, h->stream);
+                LAUNCH(KC_OTHER, 8.0 * Mn * h->H, 0.0,
+                       (klaunch(k::gather_idx_rows_kernel, Mn, 256, 0, h->stream, (const float *)h->hbuf[par],
+                                h->hbuf[par ^ 1], (const int *)h->pf_gather, h->H)));
+                par ^= 1;
+                x = h->hbuf[par];
+            }
+            cur_seq.swap(nseq);
+            cur_t.swap(nt);
+            Md = Mn;
+            if (Md < M) {  // compacted: this depth's row tables
+                for (int jj = 1; jj < nb; ++jj) off[jj] = off[jj - 1] + cnt[jj - 1];
+                if (Md > 0) {
+                    cudaMemcpyAsync(h->pf_row_seq, cur_seq.data(), Md * sizeof(int), cudaMemcpyHostToDevice, h->stream);
+                    cudaMemcpyAsync(h->pf_row_t, cur_t.data(), Md * sizeof(int), cudaMemcpyHostToDevice, h->stream);
+                    cudaMemcpyAsync(h->pf_row_u, u.data(), Md * sizeof(int), cudaMemcpyHostToDevice, h->stream);
+                }
+                cudaMemcpyAsync(h->pf_seq_off, off.data(), nb * sizeof(int), cudaMemcpyHostToDevice, h->stream);
+                cudaMemcpyAsync(h->pf_seq_cnt, cnt.data(), nb * sizeof(int), cudaMemcpyHostToDevice, h->stream);
+                map.row_seq = h->pf_row_seq;
+                map.row_u = h->pf_row_u;
+                map.row_t = h->pf_row_t;
+                map.seq_off = h->pf_seq_off;
+                map.seq_cnt = h->pf_seq_cnt;
+            }
+        }
         for (int cc = 0; cc < c.n_core; ++cc) {
             Fallback fb{exit, n, pos0, b0, nb, d, d > 1 ? slot_core(h, cc, d - 1) : 0};
             const bool use_fb = exit && d > 1;
-            if ((rc = run_layer(h, c.n_prelude + cc, slot_core(h, cc, d), M, map, nb, kv_len, 1, x,
+            if (Md == 0) {  // nothing runs this deep: every position's K/V is its shallower one
+                if (use_fb) launch_fallback(h, slot_core(h, cc, d), fb);
+                continue;
+            }
+            if ((rc = run_layer(h, c.n_prelude + cc, slot_core(h, cc, d), Md, map, nb, kv_len, 1, x,
                                 use_fb ? &fb : nullptr)))
                 return rc;
         }
-        if (exit)
-            LAUNCH(KC_OTHER, 8.0 * M * h->H / c.k_max, 0.0,
-                   (klaunch(k::capture_exit_kernel, M, 256, 0, h->stream, exit, n, b0, d, x, h->hexit, h->H)));
+        if (exit && Md > 0) {
+            if (Md == M)
+                LAUNCH(KC_OTHER, 8.0 * M * h->H / c.k_max, 0.0,
+                       (klaunch(k::capture_exit_kernel, M, 256, 0, h->stream, exit, n, b0, d, x, h->hexit, h->H)));
+            else
+                LAUNCH(KC_OTHER, 8.0 * Md * h->H / c.k_max, 0.0,
+                       (klaunch(k::scatter_exit_kernel, Md, 256, 0, h->stream, exit, n, b0, d, (const int *)h->pf_row_seq,
+                                (const int *)h->pf_row_t, (const float *)x, h->hexit, h->H)));
+        }
     }
     if (exit) x = h->hexit;
     for (int j = 0; j < c.n_coda; ++j)
-        if ((rc = run_layer(h, c.n_prelude + c.n_core + j, slot_coda(h, j), M, map, nb, kv_len, 1, x, nullptr)))
+        if ((rc = run_layer(h, c.n_prelude + c.n_core + j, slot_coda(h, j), M, full_map, nb, kv_len, 1, x, nullptr)))
             return rc;
     return check_launch(h, "prefix rows");
 }
 
-// EDEVICE on the next sync if an exit depth lies outside 1..k_max
-void check_exit_depths(alodlm *h, const int *exit, long long n) {
-    const unsigned grid = (unsigned)std::min<long long>((n + 255) / 256, 1024);
-    LAUNCH(KC_OTHER, 4.0 * n, 0.0,
-           (klaunch(k::check_range_kernel, grid, 256, 0, h->stream, exit, n, 1, h->cfg.k_max, h->d_err)));
+// Core depths (from, to] of every cached position [0, n_pos) of every sequence become copies of
+// depth `from`: a depth that no position had reached, filled when a longer-looping position
+// joins the prefix.
+void fill_depths(alodlm *h, int from, int to, int n_pos) {
+    for (int d = from + 1; d <= to; ++d)
+        for (int cc = 0; cc < h->cfg.n_core; ++cc) {
+            const long long so = (long long)slot_core(h, cc, from) * h->slot_elems;
+            const long long dst = (long long)slot_core(h, cc, d) * h->slot_elems;
+            LAUNCH(KC_OTHER, 8.0 * h->B * h->nkv * n_pos * h->hd, 0.0,
+                   (klaunch(k::copy_positions_kernel, dim3(h->B, h->nkv), 256, 0, h->stream,
+                            (const bf16 *)(h->kv_k + so), (const bf16 *)(h->kv_v + so), h->kv_k + dst, h->kv_v + dst,
+                            n_pos, h->seq_stride, h->head_stride, h->hd)));
+        }
+}
+
+// host copy of device exit depths and their maximum (0 when exit is null)
+int exit_depths_to_host(alodlm *h, const int *exit, long long n, std::vector<int> &e_host, int &max_e) {
+    max_e = 0;
+    e_host.clear();
+    if (!exit) return ALODLM_OK;
+    e_host.resize(n);
+    cudaError_t e = cudaMemcpyAsync(e_host.data(), exit, n * sizeof(int), cudaMemcpyDeviceToHost, h->stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(h->stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "exit depths");
+    for (int v : e_host) {
+        if (v < 1 || v > h->cfg.k_max) return fail(h, ALODLM_EDEVICE, "exit depth outside 1..k_max");
+        max_e = std::max(max_e, v);
+    }
+    return ALODLM_OK;
 }
 
 }  // namespace
@@ -1289,17 +1394,22 @@ int alodlm_prefill(alodlm_t *h, const int32_t *prefix_ids, int B, int P, const i
         return fail(h, ALODLM_EINVAL, "prefill: B or P out of range");
     reset_stats(h);
     h->prefilled = false;
+    std::vector<int> e_host;
+    int max_e = 0, rc;
     if (exit_depth) {
         cudaMemcpyAsync(h->exit_dev, exit_depth, (size_t)B * P * sizeof(int), cudaMemcpyDeviceToDevice, h->stream);
-        check_exit_depths(h, h->exit_dev, (long long)B * P);
+        if ((rc = exit_depths_to_host(h, h->exit_dev, (long long)B * P, e_host, max_e))) return rc;
     }
+    // depth on demand: no Core depth beyond the deepest exit depth is built
+    const int depths = exit_depth ? max_e : c.k_max;
     const int g = std::max(1, std::min(B, h->rows_cap / P));
-    int rc;
     for (int b0 = 0; b0 < B; b0 += g)
-        if ((rc = build_prefix_rows(h, prefix_ids, b0, std::min(g, B - b0), P, 0, exit_depth ? h->exit_dev : nullptr)))
+        if ((rc = build_prefix_rows(h, prefix_ids, b0, std::min(g, B - b0), P, 0, exit_depth ? h->exit_dev : nullptr,
+                                    e_host, depths)))
             return rc;
     h->B = B;
     h->P = P;
+    h->depth_built = depths;
     h->prefilled = true;
     return ALODLM_OK;
 }
@@ -1312,12 +1422,19 @@ int alodlm_append(alodlm_t *h, const int32_t *ids, int B, int N, const int32_t *
     if (N < 1 || N > c.max_block) return fail(h, ALODLM_EINVAL, "append: N out of range (1..max_block)");
     if (h->P + N > c.max_prefix) return fail(h, ALODLM_EINVAL, "append: the prefix would pass max_prefix");
     reset_stats(h);
+    std::vector<int> e_host;
+    int max_e = 0, rc;
     if (exit_depth) {
         cudaMemcpyAsync(h->app_exit, exit_depth, (size_t)B * N * sizeof(int), cudaMemcpyDeviceToDevice, h->stream);
-        check_exit_depths(h, h->app_exit, (long long)B * N);
+        if ((rc = exit_depths_to_host(h, h->app_exit, (long long)B * N, e_host, max_e))) return rc;
     }
-    int rc;
-    if ((rc = build_prefix_rows(h, ids, 0, B, N, h->P, exit_depth ? h->app_exit : nullptr))) {
+    const int need = exit_depth ? max_e : c.k_max;
+    if (need > h->depth_built) {  // the cached positions get the depths the new ones reach first
+        fill_depths(h, h->depth_built, need, h->P);
+        h->depth_built = need;
+    }
+    if ((rc = build_prefix_rows(h, ids, 0, B, N, h->P, exit_depth ? h->app_exit : nullptr, e_host,
+                                h->depth_built))) {
         h->prefilled = false;  // the arena may hold part of the new positions
         return rc;
     }
@@ -1394,7 +1511,8 @@ int denoise_step_impl(alodlm *h, const int32_t *block_ids, int B, int N, float t
             LAUNCH(KC_OTHER, 0.0, 0.0,
                    (klaunch(k::dump_rows_kernel, Ml, 256, 0, h->stream, xl, mp, H, h->dbg[0] + dbg_off)));
         for (int cc = 0; cc < c.n_core; ++cc) {
-            if ((r = run_layer(h, c.n_prelude + cc, slot_core(h, cc, s), Ml, mp, n_act_, P + N, 0, xl, nullptr)))
+            if ((r = run_layer(h, c.n_prelude + cc, slot_core(h, cc, std::min(s, h->depth_built)), Ml, mp, n_act_,
+                               P + N, 0, xl, nullptr)))
                 return r;
             if (cc == 0 && c.debug_dump)
                 LAUNCH(KC_OTHER, 0.0, 0.0,
@@ -1449,7 +1567,7 @@ int denoise_step_impl(alodlm *h, const int32_t *block_ids, int B, int N, float t
                         h->stream != cudaStreamPerThread;
     for (int s = 1; s <= K; ++s) {
         if (graphs) {
-            const GraphKey key{s, n_act, cur, hi, N, K, rule, tau_H, lambda, out->tokens, out->exit_depth,
+            const GraphKey key{s, n_act, cur, hi, N, K, rule, P, h->depth_built, tau_H, lambda, out->tokens, out->exit_depth,
                                out->entropy, out->halt, out->cum_halt, out->loops_run, out->active_rows,
                                out->readout_rows};
             cudaGraphExec_t exec = nullptr;
@@ -1537,6 +1655,12 @@ int alodlm_kv_slot(alodlm_t *h, int which, int slot, int b, int n_pos, void *dst
     if (!h || !dst || which < 0 || which > 1 || slot < 0 || slot >= h->n_slots || b < 0 ||
         b >= h->cfg.max_batch || n_pos < 1 || n_pos > h->pos_stride)
         return h ? fail(h, ALODLM_EINVAL, "kv_slot: out of range") : ALODLM_EINVAL;
+    // a Core depth beyond the deepest built one is served by the deepest built one
+    const int core0 = h->cfg.n_prelude, core_end = core0 + h->cfg.k_max * h->cfg.n_core;
+    if (slot >= core0 && slot < core_end && h->depth_built > 0) {
+        const int d = (slot - core0) / h->cfg.n_core + 1, cc = (slot - core0) % h->cfg.n_core;
+        if (d > h->depth_built) slot = slot_core(h, cc, h->depth_built);
+    }
     const bf16 *base = (which ? h->kv_v : h->kv_k) + (long long)slot * h->slot_elems + (long long)b * h->seq_stride;
     cudaError_t e = cudaMemcpy2DAsync(dst, (size_t)n_pos * h->hd * 2, base, (size_t)h->head_stride * 2,
                                       (size_t)n_pos * h->hd * 2, h->nkv, cudaMemcpyDeviceToDevice, h->stream);

@@ -83,15 +83,21 @@ __global__ void __launch_bounds__(128) attn_kernel(Params p) {
     const int kvh = blockIdx.y / p.n_splits, split = blockIdx.y % p.n_splits;
     const int b = p.map.seq_of[j];
     const int Tq = p.map.rows_per_seq;
-    const int rows_packed = p.G * Tq;
+    const int stride_packed = p.G * Tq;  // packed q rows per (sequence slot, kv head)
+    // rows of this sequence slot (fewer than Tq when the rows are compacted) and their positions
+    const int seq_rows = p.map.seq_cnt ? p.map.seq_cnt[j] : Tq;
+    const int off = p.map.seq_off ? p.map.seq_off[j] : j * Tq;
+    const int rows_packed = p.G * seq_rows;
     const int r0 = blockIdx.x * 64;
+    if (r0 >= rows_packed) return;  // uniform: no query rows in this tile
+    auto pos_of = [&](int u) { return p.map.pos0 + (p.map.row_t ? p.map.row_t[off + u] : u); };
 
     // key range of this CTA
     int kstart = split * p.keys_per_split;
     int kend = min(p.kv_len, kstart + p.keys_per_split);
     if (p.causal) {
         const int last = min(r0 + 63, rows_packed - 1);
-        kend = min(kend, p.map.pos0 + last / p.G + 1);
+        kend = min(kend, pos_of(last / p.G) + 1);
     }
 
     // Q tile
@@ -99,7 +105,7 @@ __global__ void __launch_bounds__(128) attn_kernel(Params p) {
         const int r = c / CPR, ch = c % CPR, rp = r0 + r;
         uint4 val = make_uint4(0, 0, 0, 0);
         if (rp < rows_packed)
-            val = *reinterpret_cast<const uint4 *>(p.q + (((long long)j * (p.nq / p.G) + kvh) * rows_packed + rp) * HD +
+            val = *reinterpret_cast<const uint4 *>(p.q + (((long long)j * (p.nq / p.G) + kvh) * stride_packed + rp) * HD +
                                                    ch * 8);
         *reinterpret_cast<uint4 *>(sQ + swz<HD>(r, ch)) = val;
     }
@@ -128,7 +134,7 @@ __global__ void __launch_bounds__(128) attn_kernel(Params p) {
     for (int i = 0; i < 2; ++i) {
         const int rp = r0 + warp * 16 + g8 + i * 8;
         rvalid[i] = rp < rows_packed;
-        qpos[i] = p.map.pos0 + (rvalid[i] ? rp / p.G : 0);
+        qpos[i] = rvalid[i] ? pos_of(rp / p.G) : p.map.pos0;
     }
 
     uint32_t qf[HD / 16][4];
@@ -246,7 +252,7 @@ __global__ void __launch_bounds__(128) attn_kernel(Params p) {
         if (!rvalid[ri]) continue;
         const int rp = r0 + warp * 16 + g8 + ri * 8;
         const int t = rp / p.G, h = kvh * p.G + rp % p.G;
-        const int m = j * Tq + t;
+        const int m = off + t;
         if (p.n_splits == 1) {
             const float inv = l_run[ri] > 0.f ? 1.f / l_run[ri] : 0.f;
             bf16 *dst = p.out + (long long)m * p.out_ld + h * HD;
@@ -291,7 +297,7 @@ __global__ void __launch_bounds__(128) attn_kernel(Params p) {
         const int rl = idx / (HD / 4), d = (idx % (HD / 4)) * 4;
         const int rp = r0 + rl;
         const int t = rp / p.G, h = kvh * p.G + rp % p.G;
-        const int m = j * Tq + t;
+        const int m = off + t;
         float M = -INFINITY;
         for (int s = 0; s < p.n_splits; ++s)
             M = fmaxf(M, __ldcg(p.ws_ml + (((long long)s * p.m_rows + m) * p.nq + h) * 2));

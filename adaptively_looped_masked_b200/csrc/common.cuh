@@ -398,6 +398,22 @@ __device__ __forceinline__ double gumbel_from_bits(uint64_t bits) {
 // row -> (sequence, position) of a batch of blocks laid out contiguously per sequence
 struct RowMap {
     const int *seq_of;  // slot j -> sequence index b
-    int rows_per_seq;   // N for a step, P for a prefill group
+    int rows_per_seq;   // N for a step, P for a prefill group (also the per-sequence packing stride of q)
     int pos0;           // position of row 0 of a sequence (P for a step, 0 for prefill)
+    // Compacted rows (a prefill depth that runs only the positions whose exit depth reaches it),
+    // all null otherwise: row m is the row_u[m]-th row of sequence slot row_seq[m], at position
+    // pos0 + row_t[m]; slot j owns rows [seq_off[j], seq_off[j] + seq_cnt[j]).
+    const int *row_seq = nullptr, *row_u = nullptr, *row_t = nullptr, *seq_off = nullptr, *seq_cnt = nullptr;
 };
+
+// sequence slot jj, index u among the slot's rows and position offset t of row m
+__device__ __forceinline__ void row_of(const RowMap &mp, int m, int &jj, int &u, int &t) {
+    if (mp.row_seq) {
+        jj = mp.row_seq[m];
+        u = mp.row_u[m];
+        t = mp.row_t[m];
+    } else {
+        jj = m / mp.rows_per_seq;
+        u = t = m % mp.rows_per_seq;
+    }
+}

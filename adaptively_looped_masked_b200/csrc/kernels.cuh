@@ -126,7 +126,8 @@ __global__ void qkv_post_kernel(const float *qkv, int nq, int nkv, int hd, const
     pdl_trigger();
     const int m = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    const int jj = m / map.rows_per_seq, t = m % map.rows_per_seq;
+    int jj, u, t;
+    row_of(map, m, jj, u, t);
     const int b = map.seq_of[jj];
     const int pos = map.pos0 + t;
     const int E = hd >> 5;  // 2 or 4 elements per lane, lane l holds d = l*E .. l*E+E-1
@@ -175,7 +176,7 @@ __global__ void qkv_post_kernel(const float *qkv, int nq, int nkv, int hd, const
             // packed query order: per (sequence slot, kv head), row = position * G + head-in-group
             const int G = nq / nkv;
             const int RP = G * map.rows_per_seq;
-            dst = q_out + (((long long)jj * nkv + hh / G) * RP + (long long)t * G + hh % G) * hd;
+            dst = q_out + (((long long)jj * nkv + hh / G) * RP + (long long)u * G + hh % G) * hd;
         } else if (hh < nq + nkv) {
             dst = kc + (long long)b * seq_stride + (long long)(hh - nq) * head_stride + (long long)pos * hd;
         } else {
@@ -201,7 +202,8 @@ __global__ void qkv_post128_kernel(const float *qkv, int nq, int nkv, int hpw, c
     constexpr int HD = 128, MAXH = 8;
     const int m = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int jj = m / map.rows_per_seq, t = m % map.rows_per_seq;
+    int jj, u, t;
+    row_of(map, m, jj, u, t);
     const int pos = map.pos0 + t;
     const int n_heads = nq + 2 * nkv;
     const int h0 = warp * hpw, h1 = min(n_heads, h0 + hpw);
@@ -243,7 +245,7 @@ __global__ void qkv_post128_kernel(const float *qkv, int nq, int nkv, int hpw, c
         }
         bf16 *dst;
         if (hh < nq)
-            dst = q_out + (((long long)jj * nkv + hh / G) * RP + (long long)t * G + hh % G) * HD;
+            dst = q_out + (((long long)jj * nkv + hh / G) * RP + (long long)u * G + hh % G) * HD;
         else if (hh < nq + nkv)
             dst = kc + (long long)b * seq_stride + (long long)(hh - nq) * head_stride + (long long)pos * HD;
         else
@@ -294,6 +296,46 @@ __global__ void capture_exit_kernel(const int *exit_depth, int P, int b0, int de
     const float4 *src = reinterpret_cast<const float4 *>(h + (long long)m * H);
     float4 *dst = reinterpret_cast<float4 *>(h_exit + (long long)m * H);
     for (int c = threadIdx.x; c < H / 4; c += blockDim.x) dst[c] = src[c];
+}
+
+// Depth-on-demand prefill.  Rows of depth d are compacted to the positions whose exit depth
+// reaches d: row m of depth d is original row orig[m] = row_seq[m] * n + row_t[m] of the group.
+// h_exit[orig] = h[m] for the rows whose exit depth equals d
+__global__ void scatter_exit_kernel(const int *exit_depth, int n, int b0, int depth, const int *row_seq,
+                                    const int *row_t, const float *h, float *h_exit, int H) {
+    pdl_wait();
+    pdl_trigger();
+    const int m = blockIdx.x;
+    const int jj = row_seq[m], t = row_t[m];
+    if (exit_depth[(long long)(b0 + jj) * n + t] != depth) return;
+    const float4 *src = reinterpret_cast<const float4 *>(h + (long long)m * H);
+    float4 *dst = reinterpret_cast<float4 *>(h_exit + ((long long)jj * n + t) * H);
+    for (int c = threadIdx.x; c < H / 4; c += blockDim.x) dst[c] = src[c];
+}
+
+// dst[m] = src[idx[m]] (rows of H floats)
+__global__ void gather_idx_rows_kernel(const float *src, float *dst, const int *idx, int H) {
+    pdl_wait();
+    pdl_trigger();
+    const int m = blockIdx.x;
+    const float4 *s = reinterpret_cast<const float4 *>(src + (long long)idx[m] * H);
+    float4 *d = reinterpret_cast<float4 *>(dst + (long long)m * H);
+    for (int c = threadIdx.x; c < H / 4; c += blockDim.x) d[c] = s[c];
+}
+
+// Positions [0, n_pos) of sequences 0..nb-1, every KV head: slot dst = slot src (K and V).
+// Fills a Core depth that no position had reached yet from the deepest one built.
+__global__ void copy_positions_kernel(const bf16 *src_k, const bf16 *src_v, bf16 *dst_k, bf16 *dst_v, int n_pos,
+                                      long long seq_stride, long long head_stride, int hd) {
+    pdl_wait();
+    pdl_trigger();
+    const int b = blockIdx.x, kvh = blockIdx.y;
+    const long long base = (long long)b * seq_stride + (long long)kvh * head_stride;
+    const long long n = (long long)n_pos * hd / 8;
+    for (long long i = threadIdx.x; i < n; i += blockDim.x) {
+        *reinterpret_cast<uint4 *>(dst_k + base + i * 8) = *reinterpret_cast<const uint4 *>(src_k + base + i * 8);
+        *reinterpret_cast<uint4 *>(dst_v + base + i * 8) = *reinterpret_cast<const uint4 *>(src_v + base + i * 8);
+    }
 }
 
 // ---------------------------------------------------------------------------------

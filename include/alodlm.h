@@ -120,10 +120,14 @@ ALODLM_API int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *weight
  * the Core e_j times; its Core KV at depth d > e_j is its depth-e_j KV (written at prefill
  * time, so a step reads one dense slot per depth); the Coda runs once on the depth-e_j state.
  * Prefix attention is causal; positions are 0..P-1.
+ * Depth on demand (digest "Limitations": build the cache only as deep as needed and fill deeper
+ * depths incrementally): at depth d only the positions with e_j >= d run the Core (rows
+ * compacted), and no Core depth beyond max_j e_j is built -- a step at a deeper loop reads the
+ * deepest built one, which holds every position's KV at that depth under the fallback rule.
  * prefix_ids: device int32 [B,P], ids in [0, vocab).  exit_depth: device int32 [B,P] in
- * 1..k_max, or NULL for k_max everywhere.  1 <= B <= max_batch, 1 <= P <= max_prefix.
- * Replaces any previous prefill.  Errors: EINVAL, ECUDA, EDEVICE (id or exit depth out of range, on
- * the next sync). */
+ * 1..k_max, or NULL for k_max everywhere (read back to the host once).  1 <= B <= max_batch,
+ * 1 <= P <= max_prefix.  Replaces any previous prefill.  Errors: EINVAL, ECUDA, EDEVICE (exit
+ * depth out of range at once; id out of range on the next sync). */
 ALODLM_API int alodlm_prefill(alodlm_t *h, const int32_t *prefix_ids, int B, int P, const int32_t *exit_depth);
 
 /* Append N positions to every sequence's cached prefix: positions P..P+N-1 holding ids (a
@@ -138,10 +142,11 @@ ALODLM_API int alodlm_prefill(alodlm_t *h, const int32_t *prefix_ids, int B, int
  * ids: device int32 [B,N] in [0, vocab); B must equal the prefill's; 1 <= N <= max_block and
  * P + N <= max_prefix.  exit_depth: device int32 [B,N] in 1..k_max (e.g. a decoded block's
  * commit depths, with positions that held a given id or never committed set to k_max), or
- * NULL for k_max everywhere.
- * Errors: EINVAL, ESTATE (before prefill, batch differs), ECUDA, EDEVICE (id or exit depth out
- * of range, on the next sync).  After an error the cached prefix is invalid until the next
- * prefill. */
+ * NULL for k_max everywhere.  If a new position loops deeper than any cached one, the cached
+ * positions' Core KV is first extended to that depth (copies of their deepest built depth).
+ * Errors: EINVAL, ESTATE (before prefill, batch differs), ECUDA, EDEVICE (exit depth out of
+ * range at once, id out of range on the next sync).  After an error the cached prefix is
+ * invalid until the next prefill. */
 ALODLM_API int alodlm_append(alodlm_t *h, const int32_t *ids, int B, int N, const int32_t *exit_depth);
 
 /* One denoising step over a block of N positions per sequence (positions P..P+N-1).
@@ -232,7 +237,8 @@ ALODLM_API int alodlm_debug_state(alodlm_t *h, int which, int loop, float *dst);
  * caller's device buffer dst laid out bf16 [n_kv_heads, n_pos, head_dim] (handle's stream).
  * Slots: Prelude layer l -> l; Core layer c at depth d (1-based) -> n_prelude + (d-1)*n_core + c;
  * Coda layer j -> n_prelude + k_max*n_core + j.  Positions P..P+N-1 hold the last step's block
- * K/V of the last loop that wrote the slot.  For parity checks.  EINVAL out of range. */
+ * K/V of the last loop that wrote the slot.  A Core depth beyond the deepest one built reads that
+ * one (the same values under the fallback rule).  For parity checks.  EINVAL out of range. */
 ALODLM_API int alodlm_kv_slot(alodlm_t *h, int which, int slot, int b, int n_pos, void *dst);
 
 /* Counters of the last denoise step: kernels launched, loops run (max over the batch) and,
