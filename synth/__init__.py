@@ -133,7 +133,8 @@ def _normal(shape, std: float, seed: int, index: int, device) -> torch.Tensor:
     return torch.randn(shape, generator=g, device=device, dtype=torch.float32).mul_(std)
 
 
-def make_weights(m: ModelShape, seed: int = 0, device: str = "cpu", only_layers: Optional[List[int]] = None) -> dict:
+def make_weights(m: ModelShape, seed: int = 0, device: str = "cpu", only_layers: Optional[List[int]] = None,
+                 with_globals: bool = True) -> dict:
     """Seeded random weights.
 
     Returns {"embed", "lm_head", "final_norm", "exit_w", "exit_b", "layers": [dict, ...]}.
@@ -143,7 +144,8 @@ def make_weights(m: ModelShape, seed: int = 0, device: str = "cpu", only_layers:
     regenerated alone.  On "cpu" the stream is identical on every machine; on "cuda" it is
     the CUDA generator's stream (used for the 1.7B/8B shapes, whose host copy is taken
     from the device tensors when needed).  ``only_layers``: generate just these layers (the
-    others are None); each generated tensor is the same as in the full draw.
+    others are None); ``with_globals=False`` leaves the embedding, LM head, final norm and
+    ExitGate weight None; each generated tensor is the same as in the full draw.
     """
     H = m.hidden
     mat_dtype = torch.bfloat16 if m.weight_dtype == "bf16" else torch.float32
@@ -161,11 +163,11 @@ def make_weights(m: ModelShape, seed: int = 0, device: str = "cpu", only_layers:
         idx += 1
         return torch.full(shape, float(value), dtype=torch.float32, device=device) if make else None
 
-    out["embed"] = mat((m.vocab, H), 0.02)
-    out["lm_head"] = mat((m.vocab, H), 3.2 / math.sqrt(H))
-    out["final_norm"] = vec((H,), 4.0)
+    out["embed"] = mat((m.vocab, H), 0.02, with_globals)
+    out["lm_head"] = mat((m.vocab, H), 3.2 / math.sqrt(H), with_globals)
+    out["final_norm"] = vec((H,), 4.0, with_globals)
     idx_exit = idx
-    out["exit_w"] = _normal((H,), 0.02 * math.sqrt(256.0 / H), seed, idx_exit, device)
+    out["exit_w"] = _normal((H,), 0.02 * math.sqrt(256.0 / H), seed, idx_exit, device) if with_globals else None
     idx += 1
     out["exit_b"] = -1.0
     layers: List[Optional[dict]] = []

@@ -11,10 +11,13 @@ Readout stage, on the GPU's own readout states r^(s), i.e. the same inputs on bo
 End to end, the float64 oracle running the whole step from the same ids and weights, at loop
 s (e2e_tolerances): per-row relative deviation of the states h^(s-1), h~^(s), r^(s) and of
 the logits, |dH|, |d lambda| and |d a|, and the top-two logit gap below which either token
-is a correct argmax.  Each is twice the spread between the oracle in its bf16 precision and
-the oracle in float64 at that loop (tests/golden/oracle_spread.json, written by
-make_oracle_spread.py from the oracle alone), and never below the fixed values 2e-2 (states,
-logits), 1e-2 nats, 1e-3 (halts, argmax gap).  The entropy, halt and argmax values are also
+is a correct argmax.  Each is three times the spread between the oracle in its bf16
+precision (float64 or float32 accumulation, whichever lies further) and the oracle in
+float64 at that loop (tests/golden/oracle_spread.json, written by make_oracle_spread.py from
+the oracle alone), and never below the fixed values 2e-2 (states, logits), 1e-2 nats, 1e-3
+(halts, argmax gap).  The factor covers the kernels' own rounding that no oracle variant
+models (approximate exp2, softmax probabilities rounded against a running maximum, the
+order of additions).  The entropy, halt and argmax values are also
 the bands within which a decision may go either way: outside them every decision (commit,
 exit depth, token, halt, forced pick) must be the oracle's own.
 
@@ -37,7 +40,7 @@ ENTROPY_TOL = 1e-2
 GATE_TOL = 1e-3
 BAND = 1e-3
 STATE_REL_TOL = 2e-2
-SPREAD_FACTOR = 2.0
+SPREAD_FACTOR = 3.0
 SPREAD_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "oracle_spread.json")
 _SPREAD_MODEL = {"tiny_fullcore": "tiny"}
 
