@@ -18,6 +18,7 @@
 #include <vector>
 
 #include "attention.cuh"
+#include "attention_pq.cuh"
 #include "attention_tc.cuh"
 #include "common.cuh"
 #include "gemm_tc.cuh"
@@ -41,6 +42,9 @@ namespace {
 
 #ifndef ALODLM_PDL
 #define ALODLM_PDL 1
+#endif
+#ifndef ALODLM_ATTN_PQ
+#define ALODLM_ATTN_PQ 1
 #endif
 
 constexpr int NUM_SMS_HINT = 148;
@@ -238,6 +242,7 @@ bool init_kernel_attrs() {
     set_sk_attr<64, gemm::EPI_SWIGLU>();
     cudaFuncSetAttribute(attn::attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 5 * 64 * 64 * 2);
     cudaFuncSetAttribute(attn_tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_tc::SMEM);
+    cudaFuncSetAttribute(attn_pq::attn_pq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_pq::SMEM);
     cudaFuncSetAttribute(attn::attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 5 * 64 * 128 * 2);
     done[dev] = cudaGetLastError() == cudaSuccess;
     if (done[dev]) {  // the pair kernel's occupancy, looked up here (never during a graph capture)
@@ -708,6 +713,19 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
         const int qtiles = cdiv(p.RP, attn_tc::BQ);
         const int base = qtiles * h->nkv * n_seq;
         const int ktiles = cdiv(kv_len, attn_tc::BKV);
+        const double bytes = 4.0 * n_seq * h->nkv * (double)kv_len * h->hd + 4.0 * M * h->nq * h->hd;
+        const double flops = 4.0 * M * h->nq * (double)kv_len * h->hd;
+        // two query tiles per CTA (K/V loaded once for both, softmax warpgroups in turn) where a
+        // (sequence, KV head) has two and the pairs still cover half the SMs without a key split
+        const int qpairs = cdiv(qtiles, 2);
+        if (ALODLM_ATTN_PQ && qtiles >= 2 && 2 * qpairs * h->nkv * n_seq >= h->num_sms) {
+            p.n_splits = 1;
+            p.keys_per_split = ktiles * attn_tc::BKV;
+            LAUNCH(KC_ATTN, bytes, flops,
+                   klaunch(attn_pq::attn_pq_kernel, dim3(qpairs, h->nkv, n_seq), attn_pq::THREADS, attn_pq::SMEM,
+                           h->stream, h->tm_q, h->tm_kv_k, h->tm_kv_v, p));
+            return ALODLM_OK;
+        }
         // splits of a query tile form one cluster (<= 8 CTAs, a power of two so that they
         // share the 128 rows evenly); enough CTAs to cover the SMs
         int splits = std::max(1, std::min(std::min(ktiles, cdiv(h->num_sms, base)), 8));
@@ -715,8 +733,6 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
         const int kps = cdiv(ktiles, splits);  // trailing ranks may get no keys (empty partials)
         p.n_splits = splits;
         p.keys_per_split = kps * attn_tc::BKV;
-        const double bytes = 4.0 * n_seq * h->nkv * (double)kv_len * h->hd + 4.0 * M * h->nq * h->hd;
-        const double flops = 4.0 * M * h->nq * (double)kv_len * h->hd;
         if (splits > 1) {
             // cluster along y: the `splits` consecutive y indices of one kv head
             cudaLaunchConfig_t cfg = {};

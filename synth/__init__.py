@@ -90,6 +90,8 @@ WORKLOADS: Dict[str, Workload] = {
     "mid": Workload("mid", "mid", 3, 75, 20, 5, (0.1, 0.6, 0.9), (0.1, 0.9)),
     "attn-probe-bs1": Workload("attn-probe-bs1", "attn-probe", 1, 1024, 32, 2, (0.6,), (0.5,)),
     "attn-probe-bs32": Workload("attn-probe-bs32", "attn-probe", 32, 2048, 64, 2, (0.6,), (0.5,)),
+    # two and three 128-row query tiles per (sequence, KV head): the step attention's two-tile kernel
+    "attn-probe-pq": Workload("attn-probe-pq", "attn-probe", 12, 160, 72, 3, (0.6,), (0.5,)),
     "qwen3-1.7b-bs1": Workload("qwen3-1.7b-bs1", "qwen3-1.7b", 1, 512, 32, 8, (0.6,), (0.5,)),
     "qwen3-8b-bs1": Workload("qwen3-8b-bs1", "qwen3-8b", 1, 1024, 32, 8, (0.6,), (0.5,)),
     "qwen3-8b-bs32": Workload("qwen3-8b-bs32", "qwen3-8b", 32, 2048, 64, 8, (0.1, 0.6, 0.9), (0.1, 0.9)),

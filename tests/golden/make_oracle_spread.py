@@ -19,7 +19,7 @@ positions); the Qwen3 shapes use a shorter prefix than their workloads (the spre
 with the number of layer applications, not with the prefix length) and host-generated
 weights of the same scales.
 
-    python tests/golden/make_oracle_spread.py [tiny mid qwen3-1.7b qwen3-8b]
+    python tests/golden/make_oracle_spread.py [tiny mid attn-probe qwen3-1.7b qwen3-8b]
 """
 import json
 import os
@@ -39,8 +39,8 @@ from tests.helpers import oracle_cfg  # noqa: E402
 OUT = os.path.join(os.path.dirname(os.path.abspath(__file__)), "oracle_spread.json")
 
 # model -> (batch, prefix, block, K): K covers the deepest loop any workload of the model runs
-CALIB = {"tiny": (1, 48, 16, 4), "mid": (3, 75, 20, 5), "qwen3-1.7b": (1, 256, 32, 8),
-         "qwen3-8b": (2, 128, 64, 12)}
+CALIB = {"tiny": (1, 48, 16, 4), "mid": (3, 75, 20, 5), "attn-probe": (12, 160, 72, 3),
+         "qwen3-1.7b": (1, 256, 32, 8), "qwen3-8b": (2, 128, 64, 12)}
 
 
 def host_weights(m):
@@ -101,8 +101,9 @@ def spread(name):
 
 if __name__ == "__main__":
     names = sys.argv[1:] or list(CALIB)
-    table = json.load(open(OUT)) if os.path.exists(OUT) else {}
     for n in names:
-        table[n] = spread(n)
+        row = spread(n)
+        table = json.load(open(OUT)) if os.path.exists(OUT) else {}  # merge with rows written meanwhile
+        table[n] = row
         with open(OUT, "w") as f:
             json.dump(table, f, indent=1)

@@ -222,3 +222,16 @@ def test_memory_limit_gives_enomem():
     with pytest.raises(alo.AlodlmError) as e:
         alo.Handle(m, w, k_max=4, max_batch=1, max_prefix=48, max_block=16, mem_limit_bytes=1 << 20)
     assert e.value.code == -2
+
+
+@pytest.mark.parametrize("rule", [0, 1])
+def test_step_parity_two_query_tiles_per_cta(rule):
+    """The Qwen3-8B attention geometry (32 q / 8 kv heads, head_dim 128) with 12 sequences and a
+    72-position block: 288 packed query rows per (sequence, KV head), so the step attention runs
+    two 128-row query tiles per CTA and, for the third tile, one (attention_pq.cuh); loops whose
+    looping sequences no longer fill the SMs fall back to one tile per CTA."""
+    wl = WORKLOADS["attn-probe-pq"]
+    case = Case(wl.model, wl.batch, wl.prefix, wl.block, wl.k_max)
+    case.prefill()
+    print("two query tiles per CTA", rule, _step_parity(case, 0.6, 0.5, rule))
+    case.handle.close()
