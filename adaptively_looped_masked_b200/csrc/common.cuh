@@ -395,6 +395,46 @@ __device__ __forceinline__ double gumbel_from_bits(uint64_t bits) {
     return -log(-log(u));
 }
 
+// ---------------------------------------------------------------------------------
+// q / k / v post-processing of one head (head_dim 128)
+// ---------------------------------------------------------------------------------
+// One head vector of head_dim 128 held by a warp, lane l owning d = 4l .. 4l+3: the per-head
+// RMSNorm (weights w, when qk_norm) and rotate-half RoPE at the angles cs[e] of d % 64, for q
+// and k heads (rope = true); v heads pass through.  Every path that prepares q, k or v calls
+// this, so they all give the same bits.
+__device__ __forceinline__ float4 head_post128(float4 x, bool rope, int qk_norm, float4 w, float eps,
+                                               const float2 (&cs)[4], int lane) {
+    float v[4] = {x.x, x.y, x.z, x.w};
+    if (rope) {
+        if (qk_norm) {
+            float ss = v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3];
+            ss = warp_sum(ss);
+            const float r = rsqrtf(ss / 128.f + eps);
+            v[0] = v[0] * r * w.x;
+            v[1] = v[1] * r * w.y;
+            v[2] = v[2] * r * w.z;
+            v[3] = v[3] * r * w.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float other = __shfl_xor_sync(0xffffffffu, v[e], 16);
+            v[e] = (lane < 16) ? (v[e] * cs[e].x - other * cs[e].y) : (v[e] * cs[e].x + other * cs[e].y);
+        }
+    }
+    return make_float4(v[0], v[1], v[2], v[3]);
+}
+
+// the RoPE angles (cos, sin) a lane needs for position pos (d = 4l + e, angle index d % 64)
+__device__ __forceinline__ void rope_lane128(const float2 *rope, int pos, int lane, float2 (&cs)[4]) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) cs[e] = rope[(long long)pos * 64 + ((lane * 4 + e) & 63)];
+}
+
+__device__ __forceinline__ void store_bf16x4(bf16 *dst, float4 v) {
+    __nv_bfloat162 b2[2] = {__floats2bfloat162_rn(v.x, v.y), __floats2bfloat162_rn(v.z, v.w)};
+    *reinterpret_cast<uint2 *>(dst) = *reinterpret_cast<const uint2 *>(b2);
+}
+
 // row -> (sequence, position) of a batch of blocks laid out contiguously per sequence
 struct RowMap {
     const int *seq_of;  // slot j -> sequence index b

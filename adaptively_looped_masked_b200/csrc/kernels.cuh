@@ -213,10 +213,8 @@ __global__ void qkv_post128_kernel(const float *qkv, int nq, int nkv, int hpw, c
 #pragma unroll
     for (int i = 0; i < MAXH; ++i)
         if (h0 + i < h1) x[i] = *reinterpret_cast<const float4 *>(row + (h0 + i) * HD + lane * 4);
-    // lane l holds d = 4l .. 4l + 3, RoPE angle index d % 64 (the same for every head)
     float2 cs[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) cs[e] = rope[(long long)pos * 64 + ((lane * 4 + e) & 63)];
+    rope_lane128(rope, pos, lane, cs);
     const float4 wq = qk_norm ? *reinterpret_cast<const float4 *>(qn + lane * 4) : make_float4(1.f, 1.f, 1.f, 1.f);
     const float4 wk = qk_norm ? *reinterpret_cast<const float4 *>(kn + lane * 4) : make_float4(1.f, 1.f, 1.f, 1.f);
     const int b = map.seq_of[jj];
@@ -225,24 +223,7 @@ __global__ void qkv_post128_kernel(const float *qkv, int nq, int nkv, int hpw, c
     for (int i = 0; i < MAXH; ++i) {
         const int hh = h0 + i;
         if (hh >= h1) break;  // uniform across the warp
-        float v[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
-        if (hh < nq + nkv) {
-            if (qk_norm) {
-                const float4 w = hh < nq ? wq : wk;
-                float ss = v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3];
-                ss = warp_sum(ss);
-                const float r = rsqrtf(ss / HD + eps);
-                v[0] = v[0] * r * w.x;
-                v[1] = v[1] * r * w.y;
-                v[2] = v[2] * r * w.z;
-                v[3] = v[3] * r * w.w;
-            }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float other = __shfl_xor_sync(0xffffffffu, v[e], 16);
-                v[e] = (lane < 16) ? (v[e] * cs[e].x - other * cs[e].y) : (v[e] * cs[e].x + other * cs[e].y);
-            }
-        }
+        const float4 v = head_post128(x[i], hh < nq + nkv, qk_norm, hh < nq ? wq : wk, eps, cs, lane);
         bf16 *dst;
         if (hh < nq)
             dst = q_out + (((long long)jj * nkv + hh / G) * RP + (long long)u * G + hh % G) * HD;
@@ -250,8 +231,7 @@ __global__ void qkv_post128_kernel(const float *qkv, int nq, int nkv, int hpw, c
             dst = kc + (long long)b * seq_stride + (long long)(hh - nq) * head_stride + (long long)pos * HD;
         else
             dst = vc + (long long)b * seq_stride + (long long)(hh - nq - nkv) * head_stride + (long long)pos * HD;
-        __nv_bfloat162 b2[2] = {__floats2bfloat162_rn(v[0], v[1]), __floats2bfloat162_rn(v[2], v[3])};
-        *reinterpret_cast<uint2 *>(dst + lane * 4) = *reinterpret_cast<const uint2 *>(b2);
+        store_bf16x4(dst + lane * 4, v);
     }
 }
 
