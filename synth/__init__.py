@@ -65,6 +65,9 @@ MODELS: Dict[str, ModelShape] = {
     # narrow model with the Qwen3-8B attention geometry (32 q / 8 kv heads, head_dim 128):
     # kernel-level profiling of the step's attention and small kernels on a few-MB footprint
     "attn-probe": ModelShape("attn-probe", 256, 32, 8, 128, 256, 1024, 1, 1, 1),
+    # the Qwen3-8B LM head and width with one layer per stage: profiling the fused readout on a
+    # few GB of device memory
+    "readout-probe": ModelShape("readout-probe", 4096, 32, 8, 128, 12288, 151936, 1, 1, 1),
     # Qwen3-1.7B shape, 28 layers split 8 / 12 / 8
     "qwen3-1.7b": ModelShape("qwen3-1.7b", 2048, 16, 8, 128, 6144, 151936, 8, 12, 8),
     # Qwen3-8B shape, 36 layers split 10 / 16 / 10
@@ -92,6 +95,7 @@ WORKLOADS: Dict[str, Workload] = {
     "attn-probe-bs32": Workload("attn-probe-bs32", "attn-probe", 32, 2048, 64, 2, (0.6,), (0.5,)),
     # two and three 128-row query tiles per (sequence, KV head): the step attention's two-tile kernel
     "attn-probe-pq": Workload("attn-probe-pq", "attn-probe", 12, 160, 72, 3, (0.6,), (0.5,)),
+    "readout-probe-bs1": Workload("readout-probe-bs1", "readout-probe", 1, 1024, 32, 2, (0.6,), (0.5,)),
     "qwen3-1.7b-bs1": Workload("qwen3-1.7b-bs1", "qwen3-1.7b", 1, 512, 32, 8, (0.6,), (0.5,)),
     "qwen3-8b-bs1": Workload("qwen3-8b-bs1", "qwen3-8b", 1, 1024, 32, 8, (0.6,), (0.5,)),
     "qwen3-8b-bs32": Workload("qwen3-8b-bs32", "qwen3-8b", 32, 2048, 64, 8, (0.1, 0.6, 0.9), (0.1, 0.9)),
