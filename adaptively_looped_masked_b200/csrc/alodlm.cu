@@ -691,24 +691,10 @@ int linear(alodlm *h, const CUtensorMap &tmW, int Nw, const bf16 *actp, int M, i
     return ALODLM_OK;
 }
 
-// attention of M rows (n_seq sequences x rows_per_seq) against slot `slot`, keys [0, kv_len).
-// With ln (the step's tcgen05 attention) the q / k / v post-processing of the QKV projection
-// in h->qkv is done by the attention kernel itself.
-int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_len, int causal,
-              const LayerDev *ln = nullptr) {
+// attention of M rows (n_seq sequences x rows_per_seq) against slot `slot`, keys [0, kv_len)
+int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_len, int causal) {
     if (!causal && h->tc_attn) {
         attn_tc::Params p{};
-        if (ln) {
-            p.qkv = h->qkv;
-            p.q_norm = ln->q_norm;
-            p.k_norm = ln->k_norm;
-            p.qk_norm = h->cfg.qk_norm;
-            p.eps = h->cfg.rms_eps;
-            p.rope = h->rope;
-            p.pos0 = map.pos0;
-            p.kv_k = h->kv_k;
-            p.kv_v = h->kv_v;
-        }
         p.G = h->nq / h->nkv;
         p.RP = p.G * map.rows_per_seq;
         p.nkv = h->nkv;
@@ -829,11 +815,16 @@ struct Fallback {
     int n, pos0, b0, nb, depth, src_slot;
 };
 
-// xn = RMSNorm(x) * g (bf16) over M rows of the hidden size
+// xn = RMSNorm(x) * g (bf16) over M rows of the hidden size: one block per row for few rows
+// (the whole GPU works on each), one warp per row once the rows alone fill it
 int rmsnorm(alodlm *h, const float *x, const float *g, bf16 *xn, int M) {
     const int H = h->H;
-    LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
-           (klaunch(k::rmsnorm_kernel, M, h->norm_threads, 0, h->stream, x, g, xn, H, h->cfg.rms_eps)));
+    if (M >= 256 && H % 128 == 0)
+        LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
+               (klaunch(k::rmsnorm_warp_kernel, cdiv(M, 8), 256, 0, h->stream, x, g, xn, M, H, h->cfg.rms_eps)));
+    else
+        LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
+               (klaunch(k::rmsnorm_kernel, M, h->norm_threads, 0, h->stream, x, g, xn, H, h->cfg.rms_eps)));
     return ALODLM_OK;
 }
 
@@ -847,10 +838,7 @@ int run_layer(alodlm *h, int li, int slot, int M, const RowMap &map, int n_seq, 
     bf16 *kc = h->kv_k + (long long)slot * h->slot_elems, *vc = h->kv_v + (long long)slot * h->slot_elems;
     if ((rc = linear(h, Lw.tm_qkv, h->n_qkv, h->xn, M, H, gemm::EPI_F32, h->qkv, h->n_qkv, nullptr, 0))) return rc;
     const int n_heads = h->nq + 2 * h->nkv;
-    const bool fused_post = !causal && h->tc_attn;  // the step's attention post-processes q / k / v itself
-    if (fused_post) {
-        // nothing here: the step's attention kernel norms and rotates q and k itself
-    } else if (h->hd == 128 && n_heads <= 64) {
+    if (h->hd == 128 && n_heads <= 64) {
         LAUNCH(KC_QKV, 6.0 * M * h->n_qkv, 0.0,
                (klaunch(k::qkv_post128_kernel, M, 256, 0, h->stream, h->qkv, h->nq, h->nkv, cdiv(n_heads, 8),
                         Lw.q_norm, Lw.k_norm, h->cfg.qk_norm, h->cfg.rms_eps, h->rope, map, h->qb, kc, vc,
@@ -868,7 +856,7 @@ int run_layer(alodlm *h, int li, int slot, int M, const RowMap &map, int n_seq, 
                         fb->b0, fb->depth, h->kv_k + so, h->kv_v + so, kc, vc, h->seq_stride, h->head_stride,
                         h->hd)));
     }
-    if ((rc = attention(h, slot, M, map, n_seq, kv_len, causal, fused_post ? &Lw : nullptr))) return rc;
+    if ((rc = attention(h, slot, M, map, n_seq, kv_len, causal))) return rc;
     if ((rc = linear(h, Lw.tm_o, H, h->attn_out, M, qd, gemm::EPI_ADD, x, H, nullptr, 0))) return rc;
     if ((rc = rmsnorm(h, x, Lw.mlp_norm, h->xn, M))) return rc;
     if ((rc = linear(h, Lw.tm_gu, 2 * h->I, h->xn, M, H, gemm::EPI_SWIGLU, nullptr, 0, h->act, h->I))) return rc;

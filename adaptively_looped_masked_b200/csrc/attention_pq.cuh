@@ -91,26 +91,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     pdl_wait();
     pdl_trigger();
     const int b = p.seq_of[j];
-    if (p.qkv && n_tiles > 0) {
-        // q / k / v post-processing fused here: both Q tiles, and the block's K/V rows once (every
-        // key of the slot is this CTA's; the second call gets an empty key range)
-        for (int w = 0; w < n_str; ++w)
-            attn_tc::post_qkv_into_tile(p, j, kvh, b, (qt0 + w) * BQ, BQ, sQ + w * Q_BYTES, 0, w == 0 ? p.kv_len : 0, 0,
-                                        THREADS / 32);
-        fence_proxy_async_all();
-        __syncthreads();
-        if (threadIdx.x == 0) mbar_arrive(q_full);
-    }
-
     if (warp == 0) {
         if (lane == 0 && n_tiles > 0) {
             const int qrow = (j * p.nkv + kvh) * p.RP + qt0 * BQ;
-            if (!p.qkv) {
-                mbar_arrive_expect_tx(q_full, n_str * Q_BYTES);
-                for (int w = 0; w < n_str; ++w) {
-                    tma_load_2d(sQ + w * Q_BYTES, &tmQ, q_full, 0, qrow + w * BQ);
-                    tma_load_2d(sQ + w * Q_BYTES + HALF, &tmQ, q_full, 64, qrow + w * BQ);
-                }
+            mbar_arrive_expect_tx(q_full, n_str * Q_BYTES);
+            for (int w = 0; w < n_str; ++w) {
+                tma_load_2d(sQ + w * Q_BYTES, &tmQ, q_full, 0, qrow + w * BQ);
+                tma_load_2d(sQ + w * Q_BYTES + HALF, &tmQ, q_full, 64, qrow + w * BQ);
             }
             const int kvrow0 = (int)((((long long)p.slot * p.max_batch + b) * p.nkv + kvh) * p.pos_stride);
             int k_issued = 0, v_issued = 0;

@@ -53,91 +53,7 @@ struct Params {
     int m_rows;
     float scale_log2;
     int *err;
-    // Fused q / k / v post-processing (null qkv: q arrives packed in the q buffer and the block's
-    // K/V are already in the arena).  qkv: the QKV projection [rows][(nq + 2 nkv) * 128] f32 of
-    // the block rows; the CTA norms and rotates its query rows into its Q tile and the block's
-    // k / v rows of its KV head (positions pos0 .. pos0 + Tq - 1) into the arena.
-    const float *qkv;
-    const float *q_norm, *k_norm;
-    int qk_norm;
-    float eps;
-    const float2 *rope;
-    int pos0;
-    bf16 *kv_k, *kv_v;  // arena bases
 };
-
-// The fused post-processing: query rows [r0, r0 + n_rows) of the packed order of (slot j, KV
-// head kvh) into the Q tile at sq (128-byte-swizzled K-major, rows past RP zero), and the
-// block's k / v rows of kvh whose positions lie in [key_lo, key_hi) into the arena.  Warps
-// w0 .. w0+nw-1 of the CTA take part; each loads eight row vectors before it works on them, so
-// it waits for one memory round trip per eight rows.
-__device__ __forceinline__ void post_qkv_into_tile(const Params &p, int j, int kvh, int b, int r0, int n_rows,
-                                                   uint8_t *sq, int key_lo, int key_hi, int w0, int nw) {
-    constexpr int R = 8;
-    const int warp = (threadIdx.x >> 5) - w0, lane = threadIdx.x & 31;
-    if (warp < 0 || warp >= nw) return;
-    const int n_heads = p.nq + 2 * p.nkv;
-    const float4 wq = p.qk_norm ? *reinterpret_cast<const float4 *>(p.q_norm + lane * 4) : make_float4(1.f, 1.f, 1.f, 1.f);
-    const float4 wk = p.qk_norm ? *reinterpret_cast<const float4 *>(p.k_norm + lane * 4) : make_float4(1.f, 1.f, 1.f, 1.f);
-    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
-    // query rows
-    for (int r_base = warp; r_base < n_rows; r_base += nw * R) {
-        float4 x[R];
-#pragma unroll
-        for (int i = 0; i < R; ++i) {
-            const int r = r_base + i * nw, rp = r0 + r;
-            x[i] = zero;
-            if (r < n_rows && rp < p.RP) {
-                const int t = rp / p.G, h = kvh * p.G + rp % p.G;
-                x[i] = *reinterpret_cast<const float4 *>(p.qkv + ((long long)(j * p.Tq + t) * n_heads + h) * HD +
-                                                         lane * 4);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < R; ++i) {
-            const int r = r_base + i * nw, rp = r0 + r;
-            if (r >= n_rows) break;  // uniform across the warp
-            float4 v = zero;
-            if (rp < p.RP) {
-                float2 cs[4];
-                rope_lane128(p.rope, p.pos0 + rp / p.G, lane, cs);
-                v = head_post128(x[i], true, p.qk_norm, wq, p.eps, cs, lane);
-            }
-            // dims 4 lane .. 4 lane + 3: 64-column half lane / 16, 16-byte chunk (lane % 16) / 2
-            const int half = lane >> 4, ch = (lane & 15) >> 1;
-            store_bf16x4(reinterpret_cast<bf16 *>(sq + half * HALF + (r >> 3) * 1024 + (r & 7) * 128 +
-                                                  ((ch ^ (r & 7)) << 4) + (lane & 1) * 8),
-                         v);
-        }
-    }
-    // the block's k and v rows of this KV head in [key_lo, key_hi)
-    const long long base = (((long long)p.slot * p.max_batch + b) * p.nkv + kvh) * p.pos_stride;
-    const int lo = max(0, key_lo - p.pos0), hi = min(p.Tq, key_hi - p.pos0);
-    const int n_kv = hi > lo ? 2 * (hi - lo) : 0;  // rows (which, t), t in [lo, hi)
-    for (int r_base = warp; r_base < n_kv; r_base += nw * R) {
-        float4 x[R];
-#pragma unroll
-        for (int i = 0; i < R; ++i) {
-            const int rr = r_base + i * nw;
-            x[i] = zero;
-            if (rr < n_kv) {
-                const int which = rr & 1, t = lo + (rr >> 1);
-                x[i] = *reinterpret_cast<const float4 *>(
-                    p.qkv + ((long long)(j * p.Tq + t) * n_heads + p.nq + which * p.nkv + kvh) * HD + lane * 4);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < R; ++i) {
-            const int rr = r_base + i * nw;
-            if (rr >= n_kv) break;  // uniform across the warp
-            const int which = rr & 1, t = lo + (rr >> 1), pos = p.pos0 + t;
-            float2 cs[4];
-            rope_lane128(p.rope, pos, lane, cs);
-            const float4 v = head_post128(x[i], which == 0, p.qk_norm, wk, p.eps, cs, lane);
-            store_bf16x4((which ? p.kv_v : p.kv_k) + (base + pos) * HD + lane * 4, v);
-        }
-    }
-}
 
 // K-major operand, 128-byte swizzle (8-row atoms of 128 B, 1024 B apart)
 __device__ __forceinline__ uint64_t sdesc_k(uint32_t saddr) { return umma_sdesc_sw128(saddr); }
@@ -229,23 +145,13 @@ __global__ void __launch_bounds__(192, 1)
     const int b = p.seq_of[j];
     float m_ref = -INFINITY, l = 0.f;  // softmax thread: running reference max and sum
     bool have_partial = false;         // split partial ready in TMEM
-    if (p.qkv && n_tiles > 0) {
-        // q / k / v post-processing fused here: the Q tile by all warps, the block's K/V rows of
-        // this CTA's key range into the arena, visible to the tensor core and TMA below
-        post_qkv_into_tile(p, j, kvh, b, qtile * BQ, BQ, sQ, kstart, kend, 0, 6);
-        fence_proxy_async_all();
-        __syncthreads();
-        if (threadIdx.x == 0) mbar_arrive(q_full);
-    }
 
     if (warp == 0) {
         if (lane == 0 && n_tiles > 0) {
             const int qrow = (j * p.nkv + kvh) * p.RP + qtile * BQ;
-            if (!p.qkv) {
-                mbar_arrive_expect_tx(q_full, Q_BYTES);
-                tma_load_2d(sQ, &tmQ, q_full, 0, qrow);
-                tma_load_2d(sQ + HALF, &tmQ, q_full, 64, qrow);
-            }
+            mbar_arrive_expect_tx(q_full, Q_BYTES);
+            tma_load_2d(sQ, &tmQ, q_full, 0, qrow);
+            tma_load_2d(sQ + HALF, &tmQ, q_full, 64, qrow);
             const int kvrow0 = (int)((((long long)p.slot * p.max_batch + b) * p.nkv + kvh) * p.pos_stride);
             int issued = 0;
             for (int i = 0; i < n_tiles; ++i) {

@@ -116,6 +116,39 @@ __global__ void rmsnorm_kernel(const float *x, const float *g, bf16 *y, int H, f
     }
 }
 
+// The same with one warp per row (rows per block = blockDim / 32), for many rows: every lane
+// keeps eight float4 loads in flight, the sum of squares is a fixed per-lane order and a fixed
+// butterfly, and the second pass re-reads the row (from L1).  H a multiple of 128.
+__global__ void rmsnorm_warp_kernel(const float *x, const float *g, bf16 *y, int M, int H, float eps) {
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const long long m = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (m >= M) return;
+    const float4 *xr = reinterpret_cast<const float4 *>(x + m * H);
+    const int n4 = H / 4;
+    float ss[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int c0 = 0; c0 < n4; c0 += 32 * 8) {
+        float4 v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int c = c0 + i * 32 + lane;
+            v[i] = c < n4 ? xr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss[i] += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+    }
+    const float tot = warp_sum(((ss[0] + ss[1]) + (ss[2] + ss[3])) + ((ss[4] + ss[5]) + (ss[6] + ss[7])));
+    const float r = rsqrtf(tot / H + eps);
+    const float4 *gr = reinterpret_cast<const float4 *>(g);
+    __nv_bfloat162 *yr = reinterpret_cast<__nv_bfloat162 *>(y + m * H);
+    for (int c = lane; c < n4; c += 32) {
+        const float4 v = xr[c], w = gr[c];
+        yr[2 * c] = __floats2bfloat162_rn(v.x * r * w.x, v.y * r * w.y);
+        yr[2 * c + 1] = __floats2bfloat162_rn(v.z * r * w.z, v.w * r * w.w);
+    }
+}
+
 // Per row m and head: optional per-head RMSNorm of q and k, rotate-half RoPE at the row's
 // position, then q -> q_out (bf16, packed: [slot j][kv head][position * G + head-in-group][hd],
 // so the G query heads of a KV head are consecutive rows) and k, v -> the KV arena slot (bf16).
