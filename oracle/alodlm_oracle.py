@@ -71,12 +71,14 @@ RULE_PER_TOKEN = 1
 # ----------------------------------------------------------------------------------
 
 def round_bf16(x: np.ndarray) -> np.ndarray:
-    """Nearest bfloat16 value of x (via float32, ties to even), in x's float type."""
+    """Nearest bfloat16 value of x (via float32, ties to even), in x's float type.
+
+    On the float32 bit pattern: add 0x7FFF plus the lowest kept bit, clear the 16 low bits
+    (no finite pattern, nor infinity, overflows 32 bits doing so)."""
     x = np.asarray(x)
-    f = np.ascontiguousarray(x, dtype=np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
-    return u.astype(np.uint32).view(np.float32).astype(x.dtype)
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
+    return r.view(np.float32).astype(x.dtype)
 
 
 def rmsnorm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
@@ -302,8 +304,9 @@ class Oracle:
         return L if isinstance(L, list) else [L[i] for i in sorted(L)]
 
     def _mat(self, a):
-        a = np.asarray(a, dtype=self.dt)
-        return round_bf16(a) if self.bf16 else a
+        if self.bf16:  # the rounding is done on float32 either way
+            return round_bf16(np.asarray(a, dtype=np.float32)).astype(self.dt, copy=False)
+        return np.asarray(a, dtype=self.dt)
 
     def _vec(self, a):
         # norm gains and the ExitGate weight are float32 in the kernels: no bf16 rounding
@@ -554,8 +557,9 @@ class Oracle:
         number for every kind of decision, or a dict with keys "entropy" (a commit on H <= tau,
         and the forced pick when the two lowest entropies are that close), "halt" (a decision
         on a cumulative halt or its mean) and "argmax" (the top-two score gap; the other run's
-        token is taken only if its score lies within the band of the maximum).  band=inf
-        follows every decision.  ``logit_rows``: (b, s, i) triples whose logits are returned.
+        token is taken only if its score lies within the band of the maximum); each value is
+        a number or a sequence indexed by loop s - 1 (its last entry for deeper loops).
+        band=inf follows every decision.  ``logit_rows``: (b, s, i) triples whose logits are returned.
         ``sample_key`` (two integers): committed tokens are drawn from p_i^(s) by Gumbel-max
         (``gumbel_argmax`` at position b * N + i, loop s) instead of taken greedily.
 
@@ -582,7 +586,10 @@ class Oracle:
         self.layer_execs = 0
 
         bands = band if isinstance(band, dict) else dict(entropy=band, halt=band, argmax=band)
-        band_h, band_a, band_z = float(bands["entropy"]), float(bands["halt"]), float(bands["argmax"])
+
+        def band_at(kind, s):
+            v = bands[kind]
+            return float(v) if np.ndim(v) == 0 else float(v[min(s, len(v)) - 1])
 
         def near(x, thr, width):
             return follow is not None and abs(float(x) - float(thr)) < width
@@ -633,6 +640,7 @@ class Oracle:
                     scores = np.stack([gumbel_scores(z[t], sample_key, b * N + int(idx[t]), s)
                                        for t in range(len(idx))]) if len(idx) else z
                     y = np.argmax(scores, axis=-1).astype(np.int64) if len(idx) else y
+                band_h, band_a, band_z = band_at("entropy", s), band_at("halt", s), band_at("argmax", s)
                 if follow is not None:
                     for t in range(len(idx)):
                         top2 = np.partition(scores[t], -2)[-2:]
@@ -679,6 +687,7 @@ class Oracle:
                     break
             # (5) forced progress: nothing committed in this step -> lowest entropy of the last loop
             if rule == RULE_PAPER and n_committed == 0 and U.any():
+                band_h, band_z = band_at("entropy", s_last), band_at("argmax", s_last)
                 cand = sorted(last_H.items(), key=lambda kv: (kv[1], kv[0]))
                 i_star = forced_pick(last_H)
                 if follow is not None and len(cand) > 1 and cand[1][1] - cand[0][1] < band_h:
