@@ -194,7 +194,11 @@ def step_roofline(m, B, P, N, active_rows, readout_rows, peaks):
 # DRAM traffic of the GEMM class per launch, from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum over every GEMM launch of one step), keyed by workload and by a hash of
 # the GEMM kernel source it was taken on: a changed kernel reports null until captured again.
-GEMM_TRAFFIC = {}
+GEMM_TRAFFIC = {
+    # one bs32 step: 768 linear-layer launches, 102.56 GB read + written
+    # (profiles/gemm_traffic_qwen3-8b-bs32.md)
+    "qwen3-8b-bs32": dict(source="bb9ab5e82b70b75e", bytes_per_launch=102.56e9 / 768),
+}
 
 
 def gemm_source_hash():
