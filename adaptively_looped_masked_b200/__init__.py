@@ -132,7 +132,7 @@ def gemm_bf16(A: torch.Tensor, W: torch.Tensor, out: Optional[torch.Tensor] = No
     if out is None:
         out = torch.empty((M, N), dtype=torch.float32, device=A.device)
     if workspace is None:
-        workspace = torch.zeros(64 + 8 * M * N, dtype=torch.float32, device=A.device)
+        workspace = torch.zeros(64, dtype=torch.float32, device=A.device)  # the status word
     rc = lib().alodlm_gemm_bf16(_ptr(A), _ptr(W), _ptr(out), M, N, K, _ptr(workspace),
                                 workspace.numel() * 4, _stream_ptr(stream))
     if rc:

@@ -26,18 +26,19 @@
 
 namespace {
 
-// The step's linear layers use the per-tile kernel at every row count: on B200 it streams
-// the weights faster than the stream-K kernel at 32-64 rows (0.77 vs 0.65 of the measured
-// HBM bandwidth on the 24576 x 4096 gate/up shape).  The GEMM entry points use stream-K for
-// up to 64 rows.
+// The step's linear layers and alodlm_gemm_bf16 use the per-tile kernel for few rows: on
+// B200 it streams the weights faster than the stream-K kernel at 32-64 rows (0.77 vs 0.65 of
+// the measured HBM bandwidth on the 24576 x 4096 gate/up shape).  Only the allocation-free
+// entry point runs stream-K (its partials fit a fixed array there).
 #ifndef ALODLM_MAX_SPLITS
 #define ALODLM_MAX_SPLITS 8
 #endif
-#ifndef ALODLM_STEP_STREAM_K
-#define ALODLM_STEP_STREAM_K 0
-#endif
-#ifndef ALODLM_SK_CTAS_PER_SM
-#define ALODLM_SK_CTAS_PER_SM 1
+// RMSNorm folded into the residual-add and projection epilogues (1) or a norm kernel before
+// every projection (0, the default: on a B200 the folded epilogues cost more than the norm
+// launches they replace -- Qwen3-8B shape bs 1 10.24 vs 9.86 ms per step, bs 32 114.5 vs
+// 110.6 ms -- although they pass the same parity tests)
+#ifndef ALODLM_FOLD_NORM
+#define ALODLM_FOLD_NORM 0
 #endif
 
 #ifndef ALODLM_PDL
@@ -108,9 +109,7 @@ void klaunch_cluster_x(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     cudaLaunchKernelEx(&cfg, kern, args...);
 }
 constexpr int PREFILL_ROWS = 16384;         // rows of one prefill group (sequences x P)
-constexpr size_t SPLITK_WS_FLOATS = 32u << 20;  // split-K partials (128 MB)
 constexpr size_t ATTN_WS_FLOATS = 16u << 20;    // split-KV partials (64 MB)
-constexpr int SK_COUNTERS = 4096;               // stream-K tile counters
 constexpr int ATTN_COUNTERS = 16384;            // split-KV merge counters
 
 enum KClass { KC_GEMM = 0, KC_ATTN, KC_RGEMM, KC_RCOMB, KC_NORM, KC_QKV, KC_COMMIT, KC_OTHER };
@@ -385,32 +384,41 @@ void launch_sk(const SkPlan &p, const CUtensorMap &tW, const CUtensorMap &tB, in
         launch_sk_bn<64, EPI>(p, tW, tB, Nw, M, ep, env);
 }
 
-// out = act[M, K] x W[Nw, K]^T with epilogue `epi`.  Stream-K kernel (few rows, when asked);
-// one CTA per 128 x BN tile with split-K inside a cluster when the tiles do not fill the SMs;
-// otherwise the persistent kernel.  map_for_bn(bn) returns the activation's tensor map with
-// BN-row boxes.  Returns the number of kernels launched, or -1 (tensor map failure).
+// The RMSNorm folded into the linear layers around it (see EpiParams): what a residual-add
+// GEMM also writes for the next projection, and what a projection reads in its place.
+struct Fold {
+    bf16 *xg = nullptr;            // producer: bf16(x * g_next)
+    const float *g_next = nullptr;
+    float *ss = nullptr;           // producer: partial sums of x^2, [row][ss_ld]
+    const float *ss_in = nullptr;  // consumer: the partials to scale by
+    int ss_ld = 0, ss_n = 0;
+    float norm_h = 0.f, eps = 0.f;
+};
+
+// out = act[M, K] x W[Nw, K]^T with epilogue `epi`: one CTA per 128 x BN tile with split-K
+// inside a cluster when the tiles do not fill the SMs; otherwise the pair or the persistent
+// kernel.  map_for_bn(bn) returns the activation's tensor map with BN-row boxes.  `ss_group`
+// (if set) receives the number of features per partial sum a folding residual add writes on
+// the path taken.  Returns the number of kernels launched, or -1 (tensor map failure).
 template <typename MapFn>
 int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_bn, int M, int K, int epi, float *out,
-             int ldo, bf16 *act_out, int ld_act, bool stream_k, int w_tiled) {
+             int ldo, bf16 *act_out, int ld_act, int w_tiled, const Fold &fold = Fold{}, int *ss_group = nullptr) {
     gemm::EpiParams ep{};
     ep.out = out;
     ep.ldo = ldo;
     ep.act = act_out;
     ep.ld_act = ld_act;
-    if (M <= 64 && stream_k) {
-        const SkPlan p = plan_sk(M, Nw, K, env.num_sms * ALODLM_SK_CTAS_PER_SM);
-        if (p.n_tiles <= env.n_counters && (size_t)p.n_tiles * p.max_seg * gemm::BM * p.bn <= env.ws_floats) {
-            const CUtensorMap *tB = map_for_bn(p.bn);
-            if (!tB) return -1;
-            if (epi == gemm::EPI_F32)
-                launch_sk<gemm::EPI_F32>(p, tmW, *tB, Nw, M, ep, env);
-            else if (epi == gemm::EPI_ADD)
-                launch_sk<gemm::EPI_ADD>(p, tmW, *tB, Nw, M, ep, env);
-            else
-                launch_sk<gemm::EPI_SWIGLU>(p, tmW, *tB, Nw, M, ep, env);
-            return 1;
-        }
-    }
+    ep.xg = fold.xg;
+    ep.g_next = fold.g_next;
+    ep.ss = fold.ss;
+    ep.ss_in = fold.ss_in;
+    ep.ss_ld = fold.ss_ld;
+    ep.ss_n = fold.ss_n;
+    ep.norm_h = fold.norm_h;
+    ep.norm_eps = fold.eps;
+    int group_dummy;
+    int &group = ss_group ? *ss_group : group_dummy;
+    group = 128;  // the staged epilogue of the pair and persistent kernels
     GemmShape g = plan_gemm(M, Nw, K);
     if (ALODLM_PAIR_GEMM && g.splits == 1 && g.bn >= 128 && M > 128) {
         // 256 x 256 tiles on CTA pairs once they fill every pair at least once
@@ -455,6 +463,7 @@ int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_b
             go(std::integral_constant<int, 256>{});
         return 1;
     }
+    group = g.splits > 1 ? 16 : 32;  // split-K owners: half-warps; one CTA per tile: warps
     if (epi == gemm::EPI_F32)
         launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, env.err, env.st, w_tiled);
     else if (epi == gemm::EPI_ADD)
@@ -538,8 +547,14 @@ struct alodlm {
     int rows_cap = 0, step_rows_cap = 0;
     float *hbuf[2] = {nullptr, nullptr}, *hc = nullptr, *hexit = nullptr, *qkv = nullptr;
     bf16 *xn = nullptr, *qb = nullptr, *attn_out = nullptr, *act = nullptr;
-    float *ws = nullptr, *aws_o = nullptr, *aws_ml = nullptr;
-    int *sk_counters = nullptr, *attn_counters = nullptr;
+    float *aws_o = nullptr, *aws_ml = nullptr;  // split-KV partials of the mma.sync attention
+    // folded RMSNorm: per-row partial sums of squares [rows_cap][ss_cap] (ss_cap = H / 16 rounded
+    // up), and which layer's first norm the last residual add already prepared: layer fold_layer
+    // over the M = fold_M rows of residual stream fold_x, with fold_n partials per row (-1: none)
+    float *ss = nullptr;
+    int ss_cap = 0, fold_layer = -1, fold_M = 0, fold_n = 0;
+    const float *fold_x = nullptr;
+    int *attn_counters = nullptr;
     int norm_threads = 256;  // one float4 per thread per row where possible
     int num_sms = 148;
 
@@ -571,6 +586,7 @@ struct alodlm {
 
     // activation tensor maps by (pointer, inner, rows, box rows)
     std::map<std::tuple<const void *, int, int, int>, CUtensorMap> tmcache;
+
 
     // CUDA graphs of the loop body
     bool use_graphs = true;
@@ -674,18 +690,17 @@ const CUtensorMap *act_map(alodlm *h, const void *ptr, int inner, int rows, int 
     return &(h->tmcache[key] = m);
 }
 
-// C = act[M, K] x W[Nw, K]^T with a fused epilogue (weights on the MMA's M side)
+// C = act[M, K] x W[Nw, K]^T with a fused epilogue (tiled weights on the MMA's M side)
 int linear(alodlm *h, const CUtensorMap &tmW, int Nw, const bf16 *actp, int M, int K, int epi, float *out, int ldo,
-           bf16 *act_out, int ld_act) {
+           bf16 *act_out, int ld_act, const Fold &fold = Fold{}, int *ss_group = nullptr) {
     const double bytes = 2.0 * Nw * K + 2.0 * M * K +
                          (epi == gemm::EPI_ADD ? 8.0 : (epi == gemm::EPI_SWIGLU ? 1.0 : 4.0)) * M * Nw;
     const double flops = 2.0 * M * Nw * K;
-    const GemmEnv env{h->ws, SPLITK_WS_FLOATS, h->sk_counters, SK_COUNTERS, h->d_err, h->stream, h->num_sms};
+    const GemmEnv env{nullptr, 0, nullptr, 0, h->d_err, h->stream, h->num_sms};
     auto map_for_bn = [&](int bn) { return act_map(h, actp, K, h->rows_cap, bn); };
     int n = 0;
     LAUNCH(KC_GEMM, bytes, flops,
-           n = run_gemm(env, tmW, Nw, map_for_bn, M, K, epi, out, ldo, act_out, ld_act, ALODLM_STEP_STREAM_K != 0,
-                        1));
+           n = run_gemm(env, tmW, Nw, map_for_bn, M, K, epi, out, ldo, act_out, ld_act, 1, fold, ss_group));
     if (n < 0) return fail(h, ALODLM_ECUDA, "cuTensorMapEncodeTiled failed (activation)");
     h->launches += n - 1;
     return ALODLM_OK;
@@ -695,6 +710,7 @@ int linear(alodlm *h, const CUtensorMap &tmW, int Nw, const bf16 *actp, int M, i
 int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_len, int causal) {
     if (!causal && h->tc_attn) {
         attn_tc::Params p{};
+        p.static_keys = std::max(0, kv_len - map.rows_per_seq);  // the step's cached prefix
         p.G = h->nq / h->nkv;
         p.RP = p.G * map.rows_per_seq;
         p.nkv = h->nkv;
@@ -828,15 +844,43 @@ int rmsnorm(alodlm *h, const float *x, const float *g, bf16 *xn, int M) {
     return ALODLM_OK;
 }
 
-// one pre-norm Qwen3 decoder layer over M rows, residual stream `x` updated in place
+// one pre-norm Qwen3 decoder layer over M rows, residual stream `x` updated in place.  With the
+// RMSNorm folded (ALODLM_FOLD_NORM), the two residual adds write the next projection's operand
+// bf16(x * g) and per-row partial sums of x^2, and the Q/K/V and gate/up projections scale their
+// rows by 1 / rms: no separate norm kernel runs except where the layer's input did not come from
+// the previous layer's residual add on the same rows (the first layer of a chain).
 int run_layer(alodlm *h, int li, int slot, int M, const RowMap &map, int n_seq, int kv_len, int causal, float *x,
               const Fallback *fb) {
     const LayerDev &Lw = h->layers[li];
     const int H = h->H, qd = h->nq * h->hd;
+    const bool fold = ALODLM_FOLD_NORM != 0;
     int rc;
-    if ((rc = rmsnorm(h, x, Lw.attn_norm, h->xn, M))) return rc;
+    auto consumer = [&](int n_parts) {
+        Fold f;
+        f.ss_in = h->ss;
+        f.ss_ld = h->ss_cap;
+        f.ss_n = n_parts;
+        f.norm_h = (float)H;
+        f.eps = h->cfg.rms_eps;
+        return f;
+    };
+    auto producer = [&](const float *g_next) {
+        Fold f;
+        f.xg = h->xn;
+        f.g_next = g_next;
+        f.ss = h->ss;
+        f.ss_ld = h->ss_cap;
+        return f;
+    };
+    Fold f_qkv;
+    if (fold && h->fold_layer == li && h->fold_x == x && h->fold_M == M)
+        f_qkv = consumer(h->fold_n);
+    else if ((rc = rmsnorm(h, x, Lw.attn_norm, h->xn, M)))
+        return rc;
+    h->fold_layer = -1;
     bf16 *kc = h->kv_k + (long long)slot * h->slot_elems, *vc = h->kv_v + (long long)slot * h->slot_elems;
-    if ((rc = linear(h, Lw.tm_qkv, h->n_qkv, h->xn, M, H, gemm::EPI_F32, h->qkv, h->n_qkv, nullptr, 0))) return rc;
+    if ((rc = linear(h, Lw.tm_qkv, h->n_qkv, h->xn, M, H, gemm::EPI_F32, h->qkv, h->n_qkv, nullptr, 0, f_qkv)))
+        return rc;
     const int n_heads = h->nq + 2 * h->nkv;
     if (h->hd == 128 && n_heads <= 64) {
         LAUNCH(KC_QKV, 6.0 * M * h->n_qkv, 0.0,
@@ -857,10 +901,29 @@ int run_layer(alodlm *h, int li, int slot, int M, const RowMap &map, int n_seq, 
                         h->hd)));
     }
     if ((rc = attention(h, slot, M, map, n_seq, kv_len, causal))) return rc;
-    if ((rc = linear(h, Lw.tm_o, H, h->attn_out, M, qd, gemm::EPI_ADD, x, H, nullptr, 0))) return rc;
-    if ((rc = rmsnorm(h, x, Lw.mlp_norm, h->xn, M))) return rc;
-    if ((rc = linear(h, Lw.tm_gu, 2 * h->I, h->xn, M, H, gemm::EPI_SWIGLU, nullptr, 0, h->act, h->I))) return rc;
-    if ((rc = linear(h, Lw.tm_d, H, h->act, M, h->I, gemm::EPI_ADD, x, H, nullptr, 0))) return rc;
+    int group = 0;
+    if ((rc = linear(h, Lw.tm_o, H, h->attn_out, M, qd, gemm::EPI_ADD, x, H, nullptr, 0,
+                     fold ? producer(Lw.mlp_norm) : Fold{}, &group)))
+        return rc;
+    Fold f_gu;
+    if (fold)
+        f_gu = consumer(cdiv(H, group));
+    else if ((rc = rmsnorm(h, x, Lw.mlp_norm, h->xn, M)))
+        return rc;
+    if ((rc = linear(h, Lw.tm_gu, 2 * h->I, h->xn, M, H, gemm::EPI_SWIGLU, nullptr, 0, h->act, h->I, f_gu)))
+        return rc;
+    // the next layer in the stack takes its first norm from this residual add (the callers
+    // invalidate it wherever something else runs in between)
+    const bool chain = fold && li + 1 < h->L;
+    if ((rc = linear(h, Lw.tm_d, H, h->act, M, h->I, gemm::EPI_ADD, x, H, nullptr, 0,
+                     chain ? producer(h->layers[li + 1].attn_norm) : Fold{}, &group)))
+        return rc;
+    if (chain) {
+        h->fold_layer = li + 1;
+        h->fold_x = x;
+        h->fold_M = M;
+        h->fold_n = cdiv(H, group);
+    }
     return ALODLM_OK;
 }
 
@@ -954,6 +1017,7 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
     cudaGetDevice(&h->device);
     cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
     h->norm_threads = std::max(32, std::min(1024, round_up(cfg->hidden / 4, 32)));
+
     h->H = cfg->hidden;
     h->nq = cfg->n_q_heads;
     h->nkv = cfg->n_kv_heads;
@@ -1078,12 +1142,11 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
         (rc = dalloc(h, &h->hc, R * H)) || (rc = dalloc(h, &h->hexit, R * H)) ||
         (rc = dalloc(h, &h->qkv, R * h->n_qkv)) || (rc = dalloc(h, &h->xn, R * H)) ||
         (rc = dalloc(h, &h->qb, R * qd)) || (rc = dalloc(h, &h->attn_out, R * qd)) ||
-        (rc = dalloc(h, &h->act, R * h->I)) || (rc = dalloc(h, &h->ws, SPLITK_WS_FLOATS)) ||
-        (rc = dalloc(h, &h->aws_o, ATTN_WS_FLOATS)) ||
-        (rc = dalloc(h, &h->aws_ml, ATTN_WS_FLOATS / 16)) || (rc = dalloc(h, &h->sk_counters, SK_COUNTERS)) ||
-        (rc = dalloc(h, &h->attn_counters, ATTN_COUNTERS)))
+        (rc = dalloc(h, &h->act, R * h->I)) || (rc = dalloc(h, &h->aws_o, ATTN_WS_FLOATS)) ||
+        (rc = dalloc(h, &h->aws_ml, ATTN_WS_FLOATS / 16)) || (rc = dalloc(h, &h->attn_counters, ATTN_COUNTERS)))
         return cleanup(rc);
-    cudaMemsetAsync(h->sk_counters, 0, SK_COUNTERS * sizeof(int), h->stream);
+    h->ss_cap = cdiv(H, 16);
+    if ((rc = dalloc(h, &h->ss, R * h->ss_cap))) return cleanup(rc);
     cudaMemsetAsync(h->attn_counters, 0, ATTN_COUNTERS * sizeof(int), h->stream);
     // zero the activation buffers once so rows past the live ones never hold NaN patterns
     cudaMemsetAsync(h->xn, 0, R * H * 2, h->stream);
@@ -1258,10 +1321,9 @@ int alodlm_sync(alodlm_t *h) {
     e = cudaMemcpy(&dev_err, h->d_err, sizeof(int), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(h, e, "sync: read error word");
     if (dev_err) {
-        // A kernel that gave up may have left a split tile's arrival counter part-way (its
-        // epilogue skipped the increment): re-arm every counter, so that the next launch does
-        // not take a CTA for the last arriver too early.
-        cudaMemsetAsync(h->sk_counters, 0, SK_COUNTERS * sizeof(int), h->stream);
+        // A kernel that gave up may have left a split's arrival counter part-way (its epilogue
+        // skipped the increment): re-arm the counters, so that the next launch does not take a
+        // CTA for the last arriver too early.
         cudaMemsetAsync(h->attn_counters, 0, ATTN_COUNTERS * sizeof(int), h->stream);
         cudaMemsetAsync(h->d_err, 0, sizeof(int), h->stream);
         e = cudaStreamSynchronize(h->stream);
@@ -1287,6 +1349,7 @@ namespace {
 // k_max everywhere (then n_depths = k_max and every row runs every depth).
 int build_prefix_rows(alodlm *h, const int32_t *ids, int b0, int nb, int n, int pos0, const int *exit,
                       const std::vector<int> &e_host, int n_depths) {
+    h->fold_layer = -1;  // the stream's contents come from elsewhere
     const alodlm_cfg &c = h->cfg;
     const int M = nb * n, kv_len = pos0 + n;
     RowMap full_map{h->iota + b0, n, pos0};
@@ -1514,6 +1577,7 @@ int denoise_step_impl(alodlm *h, const int32_t *block_ids, int B, int N, float t
     float *x = h->hbuf[hi];
     LAUNCH(KC_OTHER, 6.0 * M * H, 0.0,
            (klaunch(k::embed_kernel, M, 256, 0, h->stream, block_ids, N, map, h->embed, h->V, H, x, h->d_err)));
+    h->fold_layer = -1;
     for (int l = 0; l < c.n_prelude; ++l)
         if ((rc = run_layer(h, l, slot_prelude(h, l), M, map, n_act, P + N, 0, x, nullptr))) return rc;
 
@@ -1525,6 +1589,9 @@ int denoise_step_impl(alodlm *h, const int32_t *block_ids, int B, int N, float t
     auto enqueue_loop = [&](int s, int n_act_, int cur_, int hi_) -> int {
         RowMap mp{h->seq_of[cur_], N, P};
         const int Ml = n_act_ * N;
+        // loop 1 continues the Prelude's rows; later loops start from the merged (and possibly
+        // compacted) states
+        if (s > 1) h->fold_layer = -1;
         float *xl = h->hbuf[hi_];
         const long long dbg_off = (long long)(s - 1) * c.max_batch * c.max_block * H;
         int r;
@@ -1543,6 +1610,7 @@ int denoise_step_impl(alodlm *h, const int32_t *block_ids, int B, int N, float t
             LAUNCH(KC_OTHER, 0.0, 0.0,
                    (klaunch(k::dump_rows_kernel, Ml, 256, 0, h->stream, xl, mp, H, h->dbg[1] + dbg_off)));
         cudaMemcpyAsync(h->hc, xl, (size_t)Ml * H * sizeof(float), cudaMemcpyDeviceToDevice, h->stream);
+        if (h->fold_x == xl) h->fold_x = h->hc;  // the Coda runs on a copy of the same rows
         for (int j = 0; j < c.n_coda; ++j)
             if ((r = run_layer(h, c.n_prelude + c.n_core + j, slot_coda(h, j), Ml, mp, n_act_, P + N, 0, h->hc,
                                nullptr)))
@@ -1719,29 +1787,15 @@ int alodlm_gemm_bf16(const void *A, const void *W, float *C, int M, int N, int K
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // workspace: [status word | 63 spare floats | tile counters | partials]
-    const size_t total_floats = workspace_bytes / sizeof(float);
-    const int n_tiles = cdiv(N, gemm::BM);
-    const size_t counter_floats = (size_t)cdiv(std::max(n_tiles, sms), 64) * 64;
+    // workspace: the status word (split-K reduces inside a cluster; nothing else is needed)
     GemmEnv env{};
     env.err = reinterpret_cast<int *>(workspace);
     env.st = static_cast<cudaStream_t>(stream);
     env.num_sms = sms;
-    if (total_floats >= 64 + counter_floats) {
-        env.counters = reinterpret_cast<int *>(workspace + 64);
-        env.n_counters = (int)counter_floats;
-        env.ws = workspace + 64 + counter_floats;
-        env.ws_floats = total_floats - 64 - counter_floats;
-    } else {
-        env.counters = nullptr;
-        env.n_counters = 0;
-        env.ws = workspace + 64;
-        env.ws_floats = 0;
-    }
     CUtensorMap tW, tA;
     if (!make_tmap(&tW, W, K, N, gemm::BM)) return ALODLM_ECUDA;
     auto map_for_bn = [&](int bn) -> const CUtensorMap * { return make_tmap(&tA, A, K, M, bn) ? &tA : nullptr; };
-    if (run_gemm(env, tW, N, map_for_bn, M, K, gemm::EPI_F32, C, N, nullptr, 0, ALODLM_STEP_STREAM_K != 0, 0) < 0)
+    if (run_gemm(env, tW, N, map_for_bn, M, K, gemm::EPI_F32, C, N, nullptr, 0, 0) < 0)
         return ALODLM_ECUDA;
     return cudaGetLastError() == cudaSuccess ? ALODLM_OK : ALODLM_ECUDA;
 }

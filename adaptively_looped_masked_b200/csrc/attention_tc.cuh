@@ -53,6 +53,10 @@ struct Params {
     int m_rows;
     float scale_log2;
     int *err;
+    // keys [0, static_keys) are not written by the kernels this launch depends on (the cached
+    // prefix during a step): their first K/V stages are requested before griddepcontrol.wait.
+    // 0: every key waits.
+    int static_keys;
 };
 
 // K-major operand, 128-byte swizzle (8-row atoms of 128 B, 1024 B apart)
@@ -116,6 +120,7 @@ __global__ void __launch_bounds__(192, 1)
     const int kend = min(p.kv_len, kstart + p.keys_per_split);
     const int n_tiles = kend > kstart ? (kend - kstart + BKV - 1) / BKV : 0;
 
+    int pre = 0;  // K/V stages requested before the wait (thread 0, the producer)
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         for (int s = 0; s < 2; ++s) {
@@ -131,6 +136,19 @@ __global__ void __launch_bounds__(192, 1)
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
+        if (n_tiles > 0 && kstart + BKV <= p.static_keys) {
+            const int b0 = p.seq_of[j];
+            const int kvrow0 = (int)((((long long)p.slot * p.max_batch + b0) * p.nkv + kvh) * p.pos_stride);
+            for (; pre < min(n_tiles, KV_STAGES) && kstart + (pre + 1) * BKV <= p.static_keys; ++pre) {
+                const int row = kvrow0 + kstart + pre * BKV;
+                mbar_arrive_expect_tx(k_full + pre, KV_BYTES);
+                tma_load_2d(sK + pre * KV_BYTES, &tmK, k_full + pre, 0, row);
+                tma_load_2d(sK + pre * KV_BYTES + HALF, &tmK, k_full + pre, 64, row);
+                mbar_arrive_expect_tx(v_full + pre, KV_BYTES);
+                tma_load_2d(sV + pre * KV_BYTES, &tmV, v_full + pre, 0, row);
+                tma_load_2d(sV + pre * KV_BYTES + HALF, &tmV, v_full + pre, 64, row);
+            }
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -153,8 +171,8 @@ __global__ void __launch_bounds__(192, 1)
             tma_load_2d(sQ, &tmQ, q_full, 0, qrow);
             tma_load_2d(sQ + HALF, &tmQ, q_full, 64, qrow);
             const int kvrow0 = (int)((((long long)p.slot * p.max_batch + b) * p.nkv + kvh) * p.pos_stride);
-            int issued = 0;
-            for (int i = 0; i < n_tiles; ++i) {
+            int issued = pre;
+            for (int i = pre; i < n_tiles; ++i) {
                 const int s = i & 1;
                 if (!mbar_wait(kv_empty + s, ((uint32_t)(i >> 1) & 1u) ^ 1u, p.err)) break;
                 issued = i + 1;

@@ -47,7 +47,74 @@ struct EpiParams {
     const SampleParams *samp;
     const int *rr_b, *rr_i;
     int N, loop;
+    // RMSNorm folded into the linear layers around it (y = x / rms(x) * g feeds a projection
+    // W: y W^T = (1 / rms(x)) * ((x * g) W^T), the scale being one number per activation row).
+    // Residual-add epilogue (EPI_ADD) with xg set: besides x it writes xg[b * ldo + f] =
+    // bf16(x[b, f] * g_next[f]) -- the next projection's operand -- and partial sums of x[b, f]^2
+    // over groups of features, ss[b * ss_ld + f / G]: G = 32 (per-tile kernel), 16 (split-K
+    // owners), 128 (staged epilogue of the persistent and pair kernels).
+    bf16 *xg;
+    const float *g_next;
+    float *ss;
+    int ss_ld;
+    // Projection after a folded RMSNorm (EPI_F32 / EPI_SWIGLU) with ss_in set: every output of
+    // activation row b is scaled by 1 / sqrt(sum_{i < ss_n} ss_in[b * ss_ld + i] / norm_h + eps)
+    // before the epilogue (SwiGLU: gate and up both).
+    const float *ss_in;
+    int ss_n;
+    float norm_h, norm_eps;
 };
+
+// 1 / rms of activation rows b0 .. b0 + n - 1 (n a power of two, 32 .. 256) from their partial
+// sums of squares, into rb[0, n), by the 128 epilogue threads (tid = 0 .. 127).  Every thread's
+// loads are issued before its additions, so the whole computation costs about one L2 round
+// trip: with n < 128 each row is shared by 128 / n consecutive threads, each summing a
+// contiguous share of the partials in index order, then combined by a fixed butterfly; with
+// n >= 128 each thread sums whole rows.  Deterministic.
+__device__ __forceinline__ float sum_partials(const float *p, int cnt) {
+    float acc = 0.f;
+    int k = 0;
+    for (; k + 16 <= cnt; k += 16) {
+        float v[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = p[k + e];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc += v[e];
+    }
+    for (; k < cnt; ++k) acc += p[k];
+    return acc;
+}
+__device__ __forceinline__ void fold_scales(const EpiParams &ep, int b0, int n, int rowsB, float *rb, int tid) {
+    if (n >= 128) {
+        for (int i = tid; i < n; i += 128) {
+            const int b = b0 + i;
+            const float sq = b < rowsB ? sum_partials(ep.ss_in + (long long)b * ep.ss_ld, ep.ss_n) : 0.f;
+            rb[i] = rsqrtf(sq / ep.norm_h + ep.norm_eps);
+        }
+    } else {
+        const int tpr = 128 / n, i = tid / tpr, part = tid % tpr;  // tpr in {1, 2, 4}
+        const int b = b0 + i;
+        const int chunk = (ep.ss_n + tpr - 1) / tpr, k0 = min(ep.ss_n, part * chunk);
+        const int cnt = min(ep.ss_n, k0 + chunk) - k0;
+        float sq = b < rowsB ? sum_partials(ep.ss_in + (long long)b * ep.ss_ld + k0, cnt) : 0.f;
+        for (int o = 1; o < tpr; o <<= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        if (part == 0) rb[i] = rsqrtf(sq / ep.norm_h + ep.norm_eps);
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    uint32_t u;
+    memcpy(&u, &v, 4);
+    return u;
+}
+
+// sum over the 16 lanes of an aligned half-warp
+__device__ __forceinline__ float half_warp_sum(float v) {
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
 
 // Write (EPI_F32) or add to (EPI_ADD) 16 consecutive rows of one output column: p points at
 // row 0, rows `ld` floats apart, only the first `n_rows` exist.  For the residual add every
@@ -143,7 +210,11 @@ struct Cfg {
     // epilogue columns per TMEM round trip: a narrow tile's whole row at once
     static constexpr int EC = (BN <= 64) ? BN : 16;
     static constexpr uint32_t TMEM_COLS = BN * NACC;  // power of two >= 32
-    static constexpr size_t SMEM = 1024 /*align slack*/ + (size_t)STAGES * STAGE_BYTES + 256;
+    // behind the ring: 256 bytes of barriers, then 1 KB of per-activation-row scales (folded
+    // RMSNorm), then the kernel's own extra buffer
+    static constexpr uint32_t RB_OFF = STAGES * STAGE_BYTES + 256;
+    static constexpr uint32_t EXTRA_OFF = RB_OFF + 1024;
+    static constexpr size_t SMEM = 1024 /*align slack*/ + (size_t)EXTRA_OFF;
     // split-K receive buffer: [split][owned row][BN + 4] f32.  Narrow tiles get a buffer of their own behind the barriers (a partial can then be
     // pushed while the owner is still streaming); wide tiles reuse the stage ring once every CTA
     // of the cluster is done with its own.
@@ -219,7 +290,8 @@ __global__ void __launch_bounds__(192, 1)
     pdl_trigger();
     constexpr bool SPLIT_EPI = EPI == EPI_F32 || EPI == EPI_ADD || EPI == EPI_SWIGLU;
     const bool split_k = SPLIT_EPI && gridDim.z > 1;
-    float *recv = reinterpret_cast<float *>(C::RECV_SEPARATE ? smem + STAGES * C::STAGE_BYTES + 256 : smem);
+    float *recv = reinterpret_cast<float *>(C::RECV_SEPARATE ? smem + C::EXTRA_OFF : smem);
+    float *rbuf = reinterpret_cast<float *>(smem + C::RB_OFF);  // 1 / rms per column (folded RMSNorm)
     // phase 0 of the cluster barrier: "every CTA of the cluster has started" (separate receive
     // buffer) or "every CTA is done with its stage ring" (receive buffer in the ring, arrived below)
     if (split_k && C::RECV_SEPARATE) cluster_arrive_relaxed();
@@ -271,6 +343,12 @@ __global__ void __launch_bounds__(192, 1)
         // ---------------- epilogue (warps 2..5) ----------------
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         pdl_wait();
+        if constexpr (EPI == EPI_F32 || EPI == EPI_SWIGLU) {
+            if (ep.ss_in) {  // the folded RMSNorm's row scales, while the MMAs run
+                fold_scales(ep, b_tile * BN, BN, rowsB, rbuf, q * 32 + lane);
+                epilogue_bar();
+            }
+        }
         const bool ready = mbar_wait(accum, 0, err);
         ep_ready = ready;
         tc_fence_after();
@@ -279,8 +357,18 @@ __global__ void __launch_bounds__(192, 1)
         const int b0 = b_tile * BN;
         if (ready) {
             if constexpr (EPI == EPI_F32 || EPI == EPI_ADD || EPI == EPI_SWIGLU) {
-                // final epilogue of one 16-column chunk (warp-uniform: SwiGLU shuffles lanes)
-                auto apply = [&](int c0, const float (&v)[16]) {
+                // final epilogue of one 16-column chunk (warp-uniform: SwiGLU and the folded
+                // RMSNorm's sums of squares shuffle lanes)
+                auto apply = [&](int c0, const float (&v_in)[16]) {
+                    float v[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[j] = v_in[j];
+                    if constexpr (EPI != EPI_ADD) {
+                        if (ep.ss_in) {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) v[j] *= rbuf[c0 + j];
+                        }
+                    }
                     if constexpr (EPI == EPI_SWIGLU) {
                         // weight rows interleaved in groups of 32: 16 gate rows then the 16 up rows
                         // of the same features, so lane l < 16 holds gate and lane l + 16 holds up
@@ -291,6 +379,32 @@ __global__ void __launch_bounds__(192, 1)
                             const int br = b0 + c0 + j;
                             if (lane < 16 && a_row < rowsA && br < rowsB)
                                 ep.act[(long long)br * ep.ld_act + feat] = __float2bfloat16_rn(silu_f(v[j]) * up);
+                        }
+                    } else if (EPI == EPI_ADD && ep.xg) {
+                        // residual add feeding a folded RMSNorm: x, bf16(x * g), and per column the
+                        // sum of x^2 over this warp's 32 features
+                        const bool fv = a_row < rowsA;
+                        const int nr = rowsB - (b0 + c0);
+                        float *p = ep.out + (long long)(b0 + c0) * ep.ldo + a_row;
+                        bf16 *px = ep.xg + (long long)(b0 + c0) * ep.ldo + a_row;
+                        const float gf = fv ? ep.g_next[a_row] : 0.f;
+                        float nv[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) nv[j] = (fv && j < nr) ? p[(long long)j * ep.ldo] : 0.f;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            nv[j] += v[j];
+                            if (fv && j < nr) {
+                                p[(long long)j * ep.ldo] = nv[j];
+                                px[(long long)j * ep.ldo] = __float2bfloat16_rn(nv[j] * gf);
+                            }
+                        }
+                        const int f0 = a_tile * BM + q * 32;  // first feature of this warp
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float sq = warp_sum((fv && j < nr) ? nv[j] * nv[j] : 0.f);
+                            if (lane == 0 && j < nr && f0 < rowsA)
+                                ep.ss[(long long)(b0 + c0 + j) * ep.ss_ld + f0 / 32] = sq;
                         }
                     } else if (a_row < rowsA) {
                         store_chunk<EPI>(v, ep.out + (long long)(b0 + c0) * ep.ldo + a_row, ep.ldo, rowsB - (b0 + c0));
@@ -359,6 +473,10 @@ __global__ void __launch_bounds__(192, 1)
                         g += recv[(rr * rs + fl) * LD + col];
                         u += recv[(rr * rs + fs + fl) * LD + col];
                     }
+                    if (ep.ss_in) {
+                        g *= rbuf[col];
+                        u *= rbuf[col];
+                    }
                     const int ft = r * fs + fl, grow = (ft >> 4) * 32 + (ft & 15);
                     const int br = b_tile * BN + col;
                     if (a_tile * BM + grow < rowsA && br < rowsB)
@@ -366,22 +484,28 @@ __global__ void __launch_bounds__(192, 1)
                 }
             } else {
                 // consecutive threads take consecutive rows of one output column (coalesced);
-                // eight elements per thread at a time so that the residual loads overlap
+                // eight elements per thread at a time so that the residual loads overlap.  rs * BN
+                // and NT are multiples of 32, so each warp's lanes enter every round together, and
+                // an aligned half-warp holds 16 consecutive features of one column.
                 const int total = rs * BN;
                 for (int base = threadIdx.x; base < total; base += 8 * NT) {
                     float acc[8], old[8];
                     long long off[8];
                     bool ok[8];
+                    int ars[8], brs[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const int e = base + i * NT;
                         const int lrow = e & (rs - 1), col = e >> lg_rs;
                         const int ar = a_tile * BM + r * rs + lrow, br = b_tile * BN + col;
+                        ars[i] = ar;
+                        brs[i] = br;
                         ok[i] = e < total && ar < rowsA && br < rowsB;
                         off[i] = (long long)br * ep.ldo + ar;
                         float a = 0.f;
                         if (e < total)
                             for (int rr = 0; rr < S; ++rr) a += recv[(rr * rs + lrow) * LD + col];
+                        if (EPI == EPI_F32 && ep.ss_in && e < total) a *= rbuf[col];
                         acc[i] = a;
                         old[i] = 0.f;
                     }
@@ -393,6 +517,18 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
                         if (ok[i]) ep.out[off[i]] = old[i] + acc[i];
+                    if constexpr (EPI == EPI_ADD) {
+                        if (ep.xg) {  // folded RMSNorm: bf16(x * g) and sums of x^2 over 16 features
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float nv = old[i] + acc[i];
+                                if (ok[i]) ep.xg[off[i]] = __float2bfloat16_rn(nv * ep.g_next[ars[i]]);
+                                const float sq = half_warp_sum(ok[i] ? nv * nv : 0.f);
+                                if ((lane & 15) == 0 && base + i * NT < total && ars[i] < rowsA && brs[i] < rowsB)
+                                    ep.ss[(long long)brs[i] * ep.ss_ld + ars[i] / 16] = sq;
+                            }
+                        }
+                    }
                 }
             }
         }
@@ -765,7 +901,59 @@ __device__ __forceinline__ void staged_cols(float *stg, const float (&v)[64], in
         float4 val[PER];
 #pragma unroll
         for (int i = 0; i < PER; ++i) val[i] = *reinterpret_cast<const float4 *>(stg + (w + 4 * i) * LD + r0);
-        if (vec) {
+        if (EPI == EPI_ADD && ep.xg) {
+            // residual add feeding a folded RMSNorm: x, bf16(x * g), and per output row the sum
+            // of x^2 over the tile's 128 features (one warp covers them)
+            float gg[4];
+            bool fin[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                fin[e] = a * BM + r0 + e < rowsA;
+                gg[e] = fin[e] ? ep.g_next[a * BM + r0 + e] : 0.f;
+            }
+            float4 old[PER];
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {  // every old value in flight before any store
+                const int br = b_first + w + 4 * i;
+                const float *src = ep.out + (long long)br * ep.ldo + a * BM + r0;
+                if (br >= rowsB) {
+                    old[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                } else if (vec) {
+                    old[i] = *reinterpret_cast<const float4 *>(src);
+                } else {
+                    old[i].x = fin[0] ? src[0] : 0.f;
+                    old[i].y = fin[1] ? src[1] : 0.f;
+                    old[i].z = fin[2] ? src[2] : 0.f;
+                    old[i].w = fin[3] ? src[3] : 0.f;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int br = b_first + w + 4 * i;
+                if (br >= rowsB) break;  // uniform across the warp
+                float *dst = ep.out + (long long)br * ep.ldo + a * BM + r0;
+                bf16 *dx = ep.xg + (long long)br * ep.ldo + a * BM + r0;
+                float nv[4] = {old[i].x + val[i].x, old[i].y + val[i].y, old[i].z + val[i].z, old[i].w + val[i].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) nv[e] = fin[e] ? nv[e] : 0.f;
+                if (vec) {
+                    *reinterpret_cast<float4 *>(dst) = make_float4(nv[0], nv[1], nv[2], nv[3]);
+                    uint2 pk;
+                    pk.x = pack_bf16x2(nv[0] * gg[0], nv[1] * gg[1]);
+                    pk.y = pack_bf16x2(nv[2] * gg[2], nv[3] * gg[3]);
+                    *reinterpret_cast<uint2 *>(dx) = pk;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (fin[e]) {
+                            dst[e] = nv[e];
+                            dx[e] = __float2bfloat16_rn(nv[e] * gg[e]);
+                        }
+                }
+                const float sq = warp_sum(nv[0] * nv[0] + nv[1] * nv[1] + nv[2] * nv[2] + nv[3] * nv[3]);
+                if (lane == 0) ep.ss[(long long)br * ep.ss_ld + a] = sq;
+            }
+        } else if (vec) {
             float4 old[PER];
             if constexpr (EPI == EPI_ADD) {
 #pragma unroll
@@ -829,7 +1017,8 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
-    float *stg = reinterpret_cast<float *>(smem + STAGES * C::STAGE_BYTES + 256);  // epilogue staging
+    float *stg = reinterpret_cast<float *>(smem + C::EXTRA_OFF);  // epilogue staging
+    float *rbuf = reinterpret_cast<float *>(smem + C::RB_OFF);     // 1 / rms per column (folded RMSNorm)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -944,6 +1133,9 @@ __global__ void __launch_bounds__(192, 1)
             int a, b;
             tile_of(t, a, b);
             const int buf = li & 1;
+            if constexpr (EPI == EPI_F32 || EPI == EPI_SWIGLU) {
+                if (ep.ss_in) fold_scales(ep, b * BN, BN, rowsB, rbuf, row);  // ordered by the barrier below
+            }
             // one verdict for all epilogue threads (they take named barriers below)
             const bool ready = epilogue_all(mbar_wait(tfull + buf, (uint32_t)(li >> 1) & 1u, err));
             tc_fence_after();
@@ -959,6 +1151,12 @@ __global__ void __launch_bounds__(192, 1)
                         if (b0 + c0 >= rowsB) break;  // uniform across the epilogue warps
                         float v[64];
                         acc_ld<1, BN, 64>(taddr, c0, v);
+                        if constexpr (EPI == EPI_F32 || EPI == EPI_SWIGLU) {
+                            if (ep.ss_in) {
+#pragma unroll
+                                for (int j = 0; j < 64; ++j) v[j] *= rbuf[c0 + j];
+                            }
+                        }
                         staged_cols<EPI>(stg, v, row, a, b0 + c0, rowsA, rowsB, ep);
                     }
                 }
@@ -1002,7 +1200,9 @@ struct PairCfg {
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr uint32_t TMEM_COLS = 2 * TN;         // two 128 x 256 f32 accumulators
     static constexpr size_t STG_BYTES = 64 * BM * 4;
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + STG_BYTES;
+    static constexpr uint32_t RB_OFF = STAGES * STAGE_BYTES + 256;  // 1 KB of per-row scales
+    static constexpr uint32_t EXTRA_OFF = RB_OFF + 1024;             // staging tile
+    static constexpr size_t SMEM = 1024 + (size_t)EXTRA_OFF + STG_BYTES;
 };
 
 __device__ __forceinline__ void tma_operand_pair(void *dst, const CUtensorMap *map, uint32_t bar, bool tiled, int tile,
@@ -1028,7 +1228,8 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t *tempty = tfull + 2;    // used in the even CTA: 4 epilogue warps of each CTA arrive
     uint64_t *mma_done = tempty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
-    float *stg = reinterpret_cast<float *>(smem + STAGES * C::STAGE_BYTES + 256);
+    float *stg = reinterpret_cast<float *>(smem + C::EXTRA_OFF);
+    float *rbuf = reinterpret_cast<float *>(smem + C::RB_OFF);  // 1 / rms per column (folded RMSNorm)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank() & 1u;  // 0: the CTA whose thread issues the pair's MMAs
@@ -1150,6 +1351,9 @@ __global__ void __launch_bounds__(192, 1)
         for (int t = pair; t < total; t += n_pairs, ++li) {
             const int a = t / n_b, b = t % n_b;
             const int buf = li & 1;
+            if constexpr (EPI == EPI_F32 || EPI == EPI_SWIGLU) {
+                if (ep.ss_in) fold_scales(ep, b * C::TN, C::TN, rowsB, rbuf, row);  // ordered by the barrier below
+            }
             const bool ready = epilogue_all(mbar_wait(tfull + buf, (uint32_t)(li >> 1) & 1u, err));
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * C::TN;
@@ -1159,6 +1363,12 @@ __global__ void __launch_bounds__(192, 1)
                     if (b * C::TN + c0 >= rowsB) break;  // uniform across the epilogue warps
                     float v[64];
                     acc_ld<1, C::TN, 64>(taddr, c0, v);
+                    if constexpr (EPI == EPI_F32 || EPI == EPI_SWIGLU) {
+                        if (ep.ss_in) {
+#pragma unroll
+                            for (int j = 0; j < 64; ++j) v[j] *= rbuf[c0 + j];
+                        }
+                    }
                     staged_cols<EPI>(stg, v, row, a128, b * C::TN + c0, rowsA, rowsB, ep);
                 }
             }

@@ -265,15 +265,11 @@ ALODLM_API const char *alodlm_kernel_class_name(int k);
  * A device bf16 [M, K], W device bf16 [N, K] (both row-major, K-major), C device float32
  * [M, N].  K a multiple of 8 (16-byte rows for TMA), M, N >= 1, all pointers 16-byte aligned.
  * workspace: caller-owned device scratch of workspace_bytes >= 256 bytes, zeroed by the caller
- * before its first use (calls leave it ready for the next one).  Its first 4 bytes are the
- * device status word (non-zero after a call means a bounded wait inside the kernel timed out
- * and C is invalid; the caller clears it); then come per-tile counters and split partials.
- * With too little room for the split the heuristic picks, fewer splits are used (and no
- * stream-K balancing, which needs one 128 x BN f32 tile per SM).  After a call that left the
- * status word non-zero, zero the whole workspace again (a timed-out split may have left its
- * tile counter part-way).  Partial sums are added in a fixed order, so results are
- * deterministic.  Runs on `stream` of the
- * current device and allocates nothing.  For kernel-level tests and benchmarks.
+ * before its first use.  Its first 4 bytes are the device status word (non-zero after a call
+ * means a bounded wait inside the kernel timed out and C is invalid; the caller clears it);
+ * the rest is reserved.  Split-K partial sums meet inside a thread-block cluster and are
+ * added in a fixed order, so results are deterministic.  Runs on `stream` of the current
+ * device and allocates nothing.  For kernel-level tests and benchmarks.
  * Errors: EINVAL, ECUDA. */
 ALODLM_API int alodlm_gemm_bf16(const void *A, const void *W, float *C, int M, int N, int K, float *workspace,
                      size_t workspace_bytes, void *stream);
