@@ -23,7 +23,7 @@ DTYPE_BF16 = 0
 DTYPE_F32 = 1
 
 STATUS = {0: "OK", -1: "EINVAL", -2: "ENOMEM", -3: "ECUDA", -4: "EDEVICE", -5: "ETIMEOUT", -6: "ESTATE"}
-N_KCLASS = 8
+N_KCLASS = 9
 
 
 class AlodlmError(RuntimeError):

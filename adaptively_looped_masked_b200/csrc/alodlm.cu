@@ -112,9 +112,11 @@ constexpr int PREFILL_ROWS = 16384;         // rows of one prefill group (sequen
 constexpr size_t ATTN_WS_FLOATS = 16u << 20;    // split-KV partials (64 MB)
 constexpr int ATTN_COUNTERS = 16384;            // split-KV merge counters
 
-enum KClass { KC_GEMM = 0, KC_ATTN, KC_RGEMM, KC_RCOMB, KC_NORM, KC_QKV, KC_COMMIT, KC_OTHER };
+// KC_GEMM: linear layers on the pair and persistent kernels (many rows, tensor-bound);
+// KC_GEMM_TILE: linear layers on the per-tile split-K kernel (few rows, weight streaming)
+enum KClass { KC_GEMM = 0, KC_ATTN, KC_RGEMM, KC_RCOMB, KC_NORM, KC_QKV, KC_COMMIT, KC_OTHER, KC_GEMM_TILE };
 const char *kclass_names[ALODLM_N_KCLASS] = {"gemm", "attention", "readout_gemm", "readout_combine",
-                                             "norm", "qkv_rope", "commit", "other"};
+                                             "norm", "qkv_rope", "commit", "other", "gemm_tile"};
 
 std::mutex g_err_mu;
 std::string g_create_err;
@@ -399,10 +401,13 @@ struct Fold {
 // inside a cluster when the tiles do not fill the SMs; otherwise the pair or the persistent
 // kernel.  map_for_bn(bn) returns the activation's tensor map with BN-row boxes.  `ss_group`
 // (if set) receives the number of features per partial sum a folding residual add writes on
-// the path taken.  Returns the number of kernels launched, or -1 (tensor map failure).
+// the path taken; `per_tile` (if set) whether the per-tile kernel ran.  Returns the number of
+// kernels launched, or -1 (tensor map failure).
 template <typename MapFn>
 int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_bn, int M, int K, int epi, float *out,
-             int ldo, bf16 *act_out, int ld_act, int w_tiled, const Fold &fold = Fold{}, int *ss_group = nullptr) {
+             int ldo, bf16 *act_out, int ld_act, int w_tiled, const Fold &fold = Fold{}, int *ss_group = nullptr,
+             bool *per_tile = nullptr) {
+    if (per_tile) *per_tile = false;
     gemm::EpiParams ep{};
     ep.out = out;
     ep.ldo = ldo;
@@ -464,6 +469,7 @@ int run_gemm(const GemmEnv &env, const CUtensorMap &tmW, int Nw, MapFn map_for_b
         return 1;
     }
     group = g.splits > 1 ? 16 : 32;  // split-K owners: half-warps; one CTA per tile: warps
+    if (per_tile) *per_tile = true;
     if (epi == gemm::EPI_F32)
         launch_gemm_epi<gemm::EPI_F32>(g.bn, tmW, *tB, Nw, M, g.k_tiles, g.kps, g.splits, 0, ep, env.err, env.st, w_tiled);
     else if (epi == gemm::EPI_ADD)
@@ -699,8 +705,10 @@ int linear(alodlm *h, const CUtensorMap &tmW, int Nw, const bf16 *actp, int M, i
     const GemmEnv env{nullptr, 0, nullptr, 0, h->d_err, h->stream, h->num_sms};
     auto map_for_bn = [&](int bn) { return act_map(h, actp, K, h->rows_cap, bn); };
     int n = 0;
-    LAUNCH(KC_GEMM, bytes, flops,
-           n = run_gemm(env, tmW, Nw, map_for_bn, M, K, epi, out, ldo, act_out, ld_act, 1, fold, ss_group));
+    bool per_tile = false;
+    kbegin(h);
+    n = run_gemm(env, tmW, Nw, map_for_bn, M, K, epi, out, ldo, act_out, ld_act, 1, fold, ss_group, &per_tile);
+    kend(h, per_tile ? KC_GEMM_TILE : KC_GEMM, bytes, flops);
     if (n < 0) return fail(h, ALODLM_ECUDA, "cuTensorMapEncodeTiled failed (activation)");
     h->launches += n - 1;
     return ALODLM_OK;

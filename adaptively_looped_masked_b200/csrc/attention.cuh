@@ -75,8 +75,7 @@ __global__ void __launch_bounds__(128) attn_kernel(Params p) {
     bf16 *sK = sQ + 64 * HD;
     bf16 *sV = sK + 2 * 64 * HD;
 
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g8 = lane >> 2, t4 = lane & 3;
     const int j = blockIdx.z;

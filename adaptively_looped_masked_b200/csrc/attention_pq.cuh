@@ -88,8 +88,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const int b = p.seq_of[j];
     if (warp == 0) {
         if (lane == 0 && n_tiles > 0) {

@@ -158,8 +158,7 @@ __global__ void __launch_bounds__(192, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const int b = p.seq_of[j];
     float m_ref = -INFINITY, l = 0.f;  // softmax thread: running reference max and sum
     bool have_partial = false;         // split partial ready in TMEM

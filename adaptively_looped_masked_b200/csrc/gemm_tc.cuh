@@ -187,9 +187,9 @@ __device__ __forceinline__ void acc_ld16(uint32_t taddr, int c0, float (&v)[16])
     acc_ld<NACC, BN, 16>(taddr, c0, v);
 }
 
-// Compile-time tuning of the few-row tiles (BN <= 64): ring depth (4 keeps two CTAs per SM,
-// which the 192-tile gate/up launch at 32 rows needs) and TMEM accumulators per tile (1: the
-// MMAs of a stage chain on one accumulator; more measured no faster).
+// Compile-time tuning of the few-row tiles: ring depth of the 32-wide tiles (4 keeps two CTAs
+// per SM, which the 192-tile gate/up launch at 32 rows needs) and TMEM accumulators per tile
+// for BN <= 64 (1: the MMAs of a stage chain on one accumulator; more measured no faster).
 #ifndef ALODLM_STAGES_SMALL
 #define ALODLM_STAGES_SMALL 4
 #endif
@@ -199,7 +199,10 @@ __device__ __forceinline__ void acc_ld16(uint32_t taddr, int c0, float (&v)[16])
 
 template <int BN>
 struct Cfg {
-    static constexpr int STAGES = (BN <= 64) ? ALODLM_STAGES_SMALL : (BN == 128 ? 5 : 4);
+    // 64-wide tiles take three stages so that two CTAs with their split-K receive buffer still
+    // share an SM (four made it 131 KB: one CTA per SM, and the planner's 256-CTA split-K grids
+    // ran in two waves)
+    static constexpr int STAGES = (BN <= 32) ? ALODLM_STAGES_SMALL : (BN == 64 ? 3 : (BN == 128 ? 5 : 4));
     static constexpr uint32_t A_BYTES = BM * BK * 2;
     static constexpr uint32_t B_BYTES = BN * BK * 2;
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;

@@ -75,8 +75,7 @@ __global__ void rope_table_kernel(float2 *rope, int n_pos, int half, double base
 // h[m, :] = Emb[ids[b, t], :] (bf16 -> f32)
 __global__ void embed_kernel(const int *ids, int ids_ld, RowMap map, const bf16 *emb, int vocab, int H, float *h,
                              int *err) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const int m = blockIdx.x;
     const int jj = m / map.rows_per_seq, t = m % map.rows_per_seq;
     const int b = map.seq_of[jj];
@@ -95,8 +94,7 @@ __global__ void embed_kernel(const int *ids, int ids_ld, RowMap map, const bf16 
 
 // y[m, :] = bf16(x[m, :] / sqrt(mean(x^2) + eps) * g)
 __global__ void rmsnorm_kernel(const float *x, const float *g, bf16 *y, int H, float eps) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     __shared__ float red[32];
     const long long m = blockIdx.x;
     const float4 *xr = reinterpret_cast<const float4 *>(x + m * H);
@@ -120,8 +118,7 @@ __global__ void rmsnorm_kernel(const float *x, const float *g, bf16 *y, int H, f
 // keeps eight float4 loads in flight, the sum of squares is a fixed per-lane order and a fixed
 // butterfly, and the second pass re-reads the row (from L1).  H a multiple of 128.
 __global__ void rmsnorm_warp_kernel(const float *x, const float *g, bf16 *y, int M, int H, float eps) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const int lane = threadIdx.x & 31;
     const long long m = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (m >= M) return;
@@ -155,8 +152,7 @@ __global__ void rmsnorm_warp_kernel(const float *x, const float *g, bf16 *y, int
 __global__ void qkv_post_kernel(const float *qkv, int nq, int nkv, int hd, const float *qn, const float *kn,
                                 int qk_norm, float eps, const float2 *rope, RowMap map, bf16 *q_out, bf16 *kc,
                                 bf16 *vc, long long seq_stride, long long head_stride) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const int m = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     int jj, u, t;
@@ -230,8 +226,7 @@ __global__ void qkv_post_kernel(const float *qkv, int nq, int nkv, int hd, const
 __global__ void qkv_post128_kernel(const float *qkv, int nq, int nkv, int hpw, const float *qn, const float *kn,
                                    int qk_norm, float eps, const float2 *rope, RowMap map, bf16 *q_out, bf16 *kc,
                                    bf16 *vc, long long seq_stride, long long head_stride) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     constexpr int HD = 128, MAXH = 8;
     const int m = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -276,8 +271,7 @@ __global__ void qkv_post128_kernel(const float *qkv, int nq, int nkv, int hpw, c
 __global__ void kv_fallback_kernel(const int *exit_depth, int n, int pos0, int b0, int depth, const bf16 *src_k,
                                    const bf16 *src_v, bf16 *dst_k, bf16 *dst_v, long long seq_stride,
                                    long long head_stride, int hd) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const int b = b0 + blockIdx.x, kvh = blockIdx.y;
     const long long base = (long long)b * seq_stride + (long long)kvh * head_stride;
     const int chunks = hd / 8;
@@ -292,8 +286,7 @@ __global__ void kv_fallback_kernel(const int *exit_depth, int n, int pos0, int b
 
 // Raise DEVERR_BOUNDS if any of v[0, n) lies outside [lo, hi]
 __global__ void check_range_kernel(const int *v, long long n, int lo, int hi, int *err) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
         if (v[i] < lo || v[i] > hi) atomicOr(err, DEVERR_BOUNDS);
 }
@@ -301,8 +294,7 @@ __global__ void check_range_kernel(const int *v, long long n, int lo, int hi, in
 // h_exit[m] = h[m] for prefix rows whose exit depth equals `depth`
 __global__ void capture_exit_kernel(const int *exit_depth, int P, int b0, int depth, const float *h, float *h_exit,
                                     int H) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const int m = blockIdx.x;
     const int b = b0 + m / P, pos = m % P;
     if (exit_depth[(long long)b * P + pos] != depth) return;
@@ -316,8 +308,7 @@ __global__ void capture_exit_kernel(const int *exit_depth, int P, int b0, int de
 // h_exit[orig] = h[m] for the rows whose exit depth equals d
 __global__ void scatter_exit_kernel(const int *exit_depth, int n, int b0, int depth, const int *row_seq,
                                     const int *row_t, const float *h, float *h_exit, int H) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const int m = blockIdx.x;
     const int jj = row_seq[m], t = row_t[m];
     if (exit_depth[(long long)(b0 + jj) * n + t] != depth) return;
@@ -328,8 +319,7 @@ __global__ void scatter_exit_kernel(const int *exit_depth, int n, int b0, int de
 
 // dst[m] = src[idx[m]] (rows of H floats)
 __global__ void gather_idx_rows_kernel(const float *src, float *dst, const int *idx, int H) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const int m = blockIdx.x;
     const float4 *s = reinterpret_cast<const float4 *>(src + (long long)idx[m] * H);
     float4 *d = reinterpret_cast<float4 *>(dst + (long long)m * H);
@@ -340,8 +330,7 @@ __global__ void gather_idx_rows_kernel(const float *src, float *dst, const int *
 // Fills a Core depth that no position had reached yet from the deepest one built.
 __global__ void copy_positions_kernel(const bf16 *src_k, const bf16 *src_v, bf16 *dst_k, bf16 *dst_v, int n_pos,
                                       long long seq_stride, long long head_stride, int hd) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const int b = blockIdx.x, kvh = blockIdx.y;
     const long long base = (long long)b * seq_stride + (long long)kvh * head_stride;
     const long long n = (long long)n_pos * hd / 8;
@@ -360,8 +349,7 @@ __global__ void copy_positions_kernel(const bf16 *src_k, const bf16 *src_v, bf16
 // r is also stored at [b, i].
 __global__ void final_norm_kernel(const float *hc, const float *g, const float *exit_w, float exit_b, int H, float eps,
                                   RowMap map, const int *ridx, bf16 *rb, float *lam_rr, float *dbg_r) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     __shared__ float red[32];
     const int m = blockIdx.x;
     const int rr = ridx[m];
@@ -410,8 +398,7 @@ __global__ void readout_combine_kernel(const float4 *part, const double2 *spart,
                                        const int *R_dev, const int *rr_b, const int *rr_i, const float *lam_rr, int N,
                                        int Kstep, int s, float *a_state, float *cur_H, int *cur_y, float *tr_H,
                                        float *tr_lam, float *tr_a) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const int rr = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (rr >= *R_dev) return;
@@ -499,8 +486,7 @@ struct StepState {
 
 __global__ void step_init_kernel(const int *block_ids, int B, int N, int Kstep, int mask_id, StepState st,
                                  SampleParams sp, SampleParams *samp) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     if (blockIdx.x == 0 && threadIdx.x == 0) *samp = sp;
     const long long total = (long long)B * N;
     const float qnan = __int_as_float(0x7fc00000);
@@ -533,8 +519,7 @@ __global__ void step_init_kernel(const int *block_ids, int B, int N, int Kstep, 
 
 // *left = 1 if any of ids[0, total) is the mask id (*left cleared by the caller)
 __global__ void any_mask_kernel(const int *ids, long long total, int mask_id, int *left) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
          idx += (long long)gridDim.x * blockDim.x)
         if (ids[idx] == mask_id) *left = 1;
@@ -546,8 +531,7 @@ __global__ void any_mask_kernel(const int *ids, long long total, int mask_id, in
 __global__ void decode_update_kernel(const int *in_ids, const int *tokens, const int *exit_depth, int t, int B,
                                      int N, int mask_id, int *commit_step, int *commit_depth, int *steps_run,
                                      int *left) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const long long total = (long long)B * N;
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
          idx += (long long)gridDim.x * blockDim.x) {
@@ -565,8 +549,7 @@ __global__ void decode_update_kernel(const int *in_ids, const int *tokens, const
 // commit, and the Eq. 3 merge of committed rows into the loop state h.
 __global__ void commit_kernel(RowMap map, int s, int Kstep, int rule, float tau, float lam, const bf16 *emb, int H,
                               float *h, StepState st) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     __shared__ float red[32];
     __shared__ int red_i[32];
     const int jj = blockIdx.x;
@@ -670,8 +653,7 @@ __global__ void commit_kernel(RowMap map, int s, int Kstep, int rule, float tau,
 __global__ void plan_kernel(int n_cur, const int *seq_cur, int N, const int *cont, const unsigned char *U,
                             int *seq_next, int *old_slot, int *ridx, int *rr_b, int *rr_i, int *counts, int s_next,
                             int Kstep, int *active_rows, int *readout_rows, const int *err) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     __shared__ int n_next;
     __shared__ int scan[1024];
     __shared__ int carry;
@@ -731,8 +713,7 @@ __global__ void plan_kernel(int n_cur, const int *seq_cur, int N, const int *con
 
 // dst rows of the next loop's compact layout from the current layout
 __global__ void gather_rows_kernel(const float *src, float *dst, const int *old_slot, int N, int H) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const int m = blockIdx.x;
     const int jn = m / N, i = m % N;
     const float4 *s = reinterpret_cast<const float4 *>(src + ((long long)old_slot[jn] * N + i) * H);
@@ -742,8 +723,7 @@ __global__ void gather_rows_kernel(const float *src, float *dst, const int *old_
 
 // debug copy of compact rows to [b, i] order
 __global__ void dump_rows_kernel(const float *src, RowMap map, int H, float *dst) {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter();
     const int m = blockIdx.x;
     const int N = map.rows_per_seq;
     const int b = map.seq_of[m / N], i = m % N;

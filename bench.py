@@ -191,14 +191,11 @@ def step_roofline(m, B, P, N, active_rows, readout_rows, peaks):
     return t, total_f, total_b
 
 
-# DRAM traffic of the GEMM class per launch, from an ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum over every GEMM launch of one step), keyed by workload and by a hash of
-# the GEMM kernel source it was taken on: a changed kernel reports null until captured again.
-GEMM_TRAFFIC = {
-    # one bs32 step: 768 linear-layer launches, 102.56 GB read + written
-    # (profiles/gemm_traffic_qwen3-8b-bs32.md)
-    "qwen3-8b-bs32": dict(source="bb9ab5e82b70b75e", bytes_per_launch=102.56e9 / 768),
-}
+# DRAM traffic per launch of each linear-layer kernel class, from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum over every GEMM launch of one step), keyed by
+# workload and by a hash of the GEMM kernel source it was taken on: a changed kernel reports
+# null until captured again.  {workload: {"source": hash, "gemm": bytes, "gemm_tile": bytes}}
+GEMM_TRAFFIC = {}
 
 
 def gemm_source_hash():
@@ -210,11 +207,11 @@ def gemm_source_hash():
     return h.hexdigest()[:16]
 
 
-def gemm_traffic_per_launch(workload, launches):
+def gemm_traffic_per_launch(workload, kernel_class):
     rec = GEMM_TRAFFIC.get(workload)
     if rec is None or rec["source"] != gemm_source_hash():
         return None
-    return rec["bytes_per_launch"]
+    return rec.get(kernel_class)
 
 
 # ------------------------------------------------------------------------------------
@@ -477,25 +474,36 @@ def run_ours(args, world, rank, local):
     e2e_value = total_commits / (max_e2e / 1e3)
     ms_step = max_ms / args.steps
 
-    # roofline of the dominant kernel class (the tcgen05 linear layers)
+    # roofline of the dominant linear-layer kernel class: "gemm" (CTA-pair and persistent
+    # kernels, many rows: tensor-bound, against the sustained bf16 peak) or "gemm_tile" (per-tile
+    # split-K kernel, few rows: weight streaming, against HBM bandwidth)
     cls = r["classes"]
     dom = max(cls, key=lambda k_: cls[k_]["ms"])
-    g = cls["gemm"]
     tensor_bound = r["tensor_bound"]
-    if tensor_bound:
-        achieved = g["flops"] / (g["ms"] / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        roof = dict(bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s", frac=achieved / peak)
-    else:
-        achieved = g["bytes"] / (g["ms"] / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = dict(bound="hbm", achieved=achieved, peak=peak, unit="GB/s", frac=achieved / peak)
-    roof["traffic"] = gemm_traffic_per_launch(args.workload, g["launches"])
-    roof.update(kernel="gemm (tcgen05 linear layers, incl. split-K reduce)", peak_source=peaks_src,
-                launches_per_step=g["launches"], ms_per_step=g["ms"],
-                algorithmic_per_launch=(g["flops"] / g["launches"] if tensor_bound else g["bytes"] / g["launches"]),
-                algorithmic_unit=("flop" if tensor_bound else "byte"),
-                algorithmic_bytes_per_launch=g["bytes"] / g["launches"])
+
+    def class_roofline(name):
+        g = cls[name]
+        if name == "gemm":
+            achieved = g["flops"] / (g["ms"] / 1e3) / 1e12
+            peak = peaks["bf16_tflops_sustained"]
+            ro = dict(bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s", frac=achieved / peak)
+        else:
+            achieved = g["bytes"] / (g["ms"] / 1e3) / 1e9
+            peak = peaks["hbm_gbs"]
+            ro = dict(bound="hbm", achieved=achieved, peak=peak, unit="GB/s", frac=achieved / peak)
+        ro["traffic"] = gemm_traffic_per_launch(args.workload, name)
+        ro.update(kernel={"gemm": "gemm_pair_kernel / gemm_persist_kernel (tcgen05 linear layers, many rows)",
+                          "gemm_tile": "gemm_tc_kernel (tcgen05 linear layers, few rows, split-K in a cluster)"}[name],
+                  kernel_class=name, peak_source=peaks_src, launches_per_step=g["launches"], ms_per_step=g["ms"],
+                  algorithmic_per_launch=(g["flops"] if name == "gemm" else g["bytes"]) / g["launches"],
+                  algorithmic_unit="flop" if name == "gemm" else "byte",
+                  algorithmic_bytes_per_launch=g["bytes"] / g["launches"])
+        return ro
+
+    gemm_names = [k_ for k_ in ("gemm", "gemm_tile") if k_ in cls and cls[k_]["launches"] > 0]
+    gdom = max(gemm_names, key=lambda k_: cls[k_]["ms"])
+    roof = class_roofline(gdom)
+    gemm_rooflines = {k_: class_roofline(k_) for k_ in gemm_names}
     kernel_share = {k_: round(v["ms"] / max(sum(c["ms"] for c in cls.values()), 1e-9), 4) for k_, v in cls.items()}
 
     line = {
@@ -508,6 +516,7 @@ def run_ours(args, world, rank, local):
                    "rule": ["paper", "per_token"][rule], "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (weights 16 GB + KV arena)"},
         "roofline": roof,
+        "gemm_rooflines": gemm_rooflines,
         "step_roofline": {"t_roof_ms": r["t_roof"] * 1e3, "frac": r["t_roof"] * 1e3 / ms_step,
                           "bound": "tensor" if tensor_bound else "hbm", "flops": r["F"], "bytes": r["B"],
                           "peak_source": peaks_src},

@@ -245,7 +245,7 @@ ALODLM_API int alodlm_kv_slot(alodlm_t *h, int which, int slot, int b, int n_pos
  * if timing was enabled, per kernel class the summed device time (ms) and launch count and the
  * algorithmic bytes and flops (see alodlm_kernel_class_name).  times/launches/bytes/flops may be
  * NULL; each is an array of ALODLM_N_KCLASS entries. */
-#define ALODLM_N_KCLASS 8
+#define ALODLM_N_KCLASS 9
 ALODLM_API int alodlm_step_stats(const alodlm_t *h, int *kernel_launches, double *times_ms, int *launches,
                       double *bytes, double *flops);
 /* 1: time every kernel class with CUDA events on the handle's stream during the next steps
@@ -256,8 +256,10 @@ ALODLM_API int alodlm_set_timing(alodlm_t *h, int on);
  * 0: launch every kernel directly and drop the recorded graphs. */
 ALODLM_API int alodlm_set_graphs(alodlm_t *h, int on);
 
-/* Name of kernel class k (0 <= k < ALODLM_N_KCLASS): "gemm", "attention", "readout_gemm",
- * "readout_combine", "norm", "qkv_rope", "commit", "other". */
+/* Name of kernel class k (0 <= k < ALODLM_N_KCLASS): "gemm" (linear layers on the CTA-pair and
+ * persistent kernels: many activation rows), "attention", "readout_gemm", "readout_combine",
+ * "norm", "qkv_rope", "commit", "other", "gemm_tile" (linear layers on the per-tile split-K
+ * kernel: few activation rows). */
 ALODLM_API const char *alodlm_kernel_class_name(int k);
 
 /* Plain bf16 GEMM through the library's tcgen05 kernels (the ones the step's linear layers use,

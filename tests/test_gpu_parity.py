@@ -45,9 +45,11 @@ def _gemm_ref(A, W):
                                    (128, 256, 4096), (300, 640, 768), (2048, 512, 1024), (20, 6144, 4096),
                                    (512, 4096, 1024), (2048, 6144, 4096), (1000, 3000, 880),
                                    (832, 6144, 4096), (1536, 4096, 4096), (32, 4096, 2112),
-                                   (1000, 6016, 880), (300, 19072, 256), (2048, 24576, 4096)])
+                                   (1000, 6016, 880), (300, 19072, 256), (2048, 24576, 4096),
+                                   (64, 4096, 12288), (48, 24576, 4096)])
 def test_gemm_tcgen05_against_fp64(M, N, K):
-    """The shapes cover every GEMM path: split-K clusters of 2-8 CTAs (few rows), the persistent
+    """The shapes cover every GEMM path: split-K clusters of 2-8 CTAs (few rows; 64-row tiles with
+    their three-stage ring split and unsplit), the persistent
     kernel with 128- and 256-wide tiles, and the CTA-pair kernel (256 x 256 tiles; ragged
     edges in M, N and K, and an odd number of 128-row weight tiles, whose last pair half reads
     past the matrix).  K = 2112 (33 k-tiles) cannot be cut into 8 equal non-empty ranges: the
