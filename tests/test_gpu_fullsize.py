@@ -23,7 +23,7 @@ import torch
 
 from oracle import Oracle
 from synth import MODELS, WORKLOADS, make_exit_depths, make_weights, weights_to_numpy
-from tests.gpu_util import STATE_REL_TOL, Case, row_rel_err, step_parity
+from tests.gpu_util import STATE_REL_TOL, Case, e2e_tolerances, row_rel_err, step_parity
 from tests.helpers import oracle_cfg
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
@@ -90,18 +90,23 @@ def test_fullsize_end_to_end_with_oracle_prefill(name):
     of.prefill(case.prefix_ids, e)
     ob = Oracle(oracle_cfg(case.m, wl.k_max), case.w_host, precision="bf16", dtype=np.float32)
     stats = step_parity(case, gpu, tau, lam, wl.k_max, rule, case.block_ids, oracle=of, ob=ob)
-    # the prefix KV cache against the oracle's own, on the first and the deepest slots
+    # the prefix KV cache against the oracle's own, on the first and the deepest slots.  A slot
+    # of Core depth d holds projections of the prefix states after the Prelude and d Core
+    # passes, which carry the bf16 drift of that depth: each is held to the state tolerance of
+    # loop d (the Prelude's to loop 1's, the Coda's to loop K's; R20)
     m, K = case.m, wl.k_max
-    slots = [(("prelude", 0), 0), (("core", 0, 1), m.n_prelude), (("core", m.n_core - 1, K), m.n_prelude + K * m.n_core - 1),
-             (("coda", m.n_coda - 1), m.n_prelude + K * m.n_core + m.n_coda - 1)]
+    state_tol = e2e_tolerances(wl.model, K)["state"]
+    slots = [(("prelude", 0), 0, 1), (("core", 0, 1), m.n_prelude, 1),
+             (("core", m.n_core - 1, K), m.n_prelude + K * m.n_core - 1, K),
+             (("coda", m.n_coda - 1), m.n_prelude + K * m.n_core + m.n_coda - 1, K)]
     worst_kv = 0.0
-    for key, slot in slots:
+    for key, slot, depth in slots:
         for which in (0, 1):
             got = case.handle.kv_slot(which, slot, 0, wl.prefix).float().cpu().numpy()  # [nkv, P, hd]
             ref = of.kv[0][key][which].transpose(1, 0, 2)
             rel = row_rel_err(got, ref)
             worst_kv = max(worst_kv, float(rel.max()))
-            assert rel.max() <= STATE_REL_TOL, (key, which, rel.max())
+            assert rel.max() <= state_tol[depth - 1], (key, which, rel.max(), state_tol[depth - 1])
     print(f"{name}: loops {gpu['loops_run'].tolist()} commits {int((gpu['exit_depth'] > 0).sum())} "
           f"kv rel {worst_kv:.2e} {stats}")
     _free(case)
