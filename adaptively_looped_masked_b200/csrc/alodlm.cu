@@ -33,6 +33,10 @@ namespace {
 #ifndef ALODLM_MAX_SPLITS
 #define ALODLM_MAX_SPLITS 8
 #endif
+// step attention may split keys over 16-CTA clusters (non-portable size) when they all fit
+#ifndef ALODLM_ATTN_CLUSTER16
+#define ALODLM_ATTN_CLUSTER16 1
+#endif
 // RMSNorm folded into the residual-add and projection epilogues (1) or a norm kernel before
 // every projection (0, the default: on a B200 the folded epilogues cost more than the norm
 // launches they replace -- Qwen3-8B shape bs 1 10.24 vs 9.86 ms per step, bs 32 114.5 vs
@@ -207,6 +211,36 @@ int pair_slots() {
     return cached[dev];
 }
 
+// How many 16-CTA clusters of the step attention can be resident at once (0: the
+// non-portable cluster size is not available).  Looked up once per device, outside captures.
+int attn_clusters16() {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 0;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaFuncSetAttribute(attn_tc::attn_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+            cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(1, 16 * 8, 1);
+            cfg.blockDim = dim3(192);
+            cfg.dynamicSmemBytes = attn_tc::SMEM;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 1;
+            attr[0].val.clusterDim.y = 16;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&n, attn_tc::attn_tc_kernel, &cfg) != cudaSuccess) n = 0;
+        }
+        cudaGetLastError();
+        cached[dev] = n > 0 ? n : -1;
+    }
+    return std::max(cached[dev], 0);
+}
+
 bool init_kernel_attrs() {
     static bool done[64] = {false};
     int dev = 0;
@@ -246,10 +280,11 @@ bool init_kernel_attrs() {
     cudaFuncSetAttribute(attn_pq::attn_pq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_pq::SMEM);
     cudaFuncSetAttribute(attn::attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 5 * 64 * 128 * 2);
     done[dev] = cudaGetLastError() == cudaSuccess;
-    if (done[dev]) {  // the pair kernel's occupancy, looked up here (never during a graph capture)
+    if (done[dev]) {  // occupancies, looked up here (never during a graph capture)
         pair_slots<gemm::EPI_F32>();
         pair_slots<gemm::EPI_ADD>();
         pair_slots<gemm::EPI_SWIGLU>();
+        attn_clusters16();
     }
     return done[dev];
 }
@@ -750,10 +785,15 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
                            h->stream, h->tm_q, h->tm_kv_k, h->tm_kv_v, p));
             return ALODLM_OK;
         }
-        // splits of a query tile form one cluster (<= 8 CTAs, a power of two so that they
-        // share the 128 rows evenly); enough CTAs to cover the SMs
-        int splits = std::max(1, std::min(std::min(ktiles, cdiv(h->num_sms, base)), 8));
-        while (splits & (splits - 1)) --splits;
+        // splits of a query tile form one cluster (a power of two so that they share the 128
+        // rows evenly; 8 CTAs, or 16 where that many 16-CTA clusters fit at once): enough CTAs
+        // to cover the SMs, rounded up to the next power of two while the grid still fits in
+        // one wave, so that a latency-bound launch walks one key tile per CTA
+        const int cap = (ALODLM_ATTN_CLUSTER16 && attn_clusters16() >= base) ? 16 : 8;
+        const int want = std::max(1, std::min(std::min(ktiles, cdiv(h->num_sms, base)), cap));
+        int splits = 1;
+        while (splits < want) splits <<= 1;
+        if (splits > cap || (splits > 1 && (long long)splits * base > h->num_sms)) splits >>= 1;
         const int kps = cdiv(ktiles, splits);  // trailing ranks may get no keys (empty partials)
         p.n_splits = splits;
         p.keys_per_split = kps * attn_tc::BKV;

@@ -236,3 +236,15 @@ def test_step_parity_two_query_tiles_per_cta(rule):
     case.prefill()
     print("two query tiles per CTA", rule, _step_parity(case, 0.6, 0.5, rule))
     case.handle.close()
+
+
+def test_step_parity_key_split_over_sixteen_ctas():
+    """One sequence of the Qwen3-8B attention geometry (32 q / 8 kv heads, head_dim 128, block
+    32) against a 1040-position prefix: 9 key tiles, the last ragged, for each of the 8 query
+    tiles.  The step attention then splits the keys over a 16-CTA cluster where the device holds
+    eight such clusters at once (one key tile per CTA, seven ranks without keys whose empty
+    partials the merge skips), else over 8."""
+    case = Case("attn-probe", 1, 1040, 32, 2)
+    case.prefill()
+    print("16-way key split", _step_parity(case, 0.6, 0.5, 0))
+    case.handle.close()
