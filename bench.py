@@ -195,7 +195,11 @@ def step_roofline(m, B, P, N, active_rows, readout_rows, peaks):
 # (dram__bytes_read.sum + dram__bytes_write.sum over every GEMM launch of one step), keyed by
 # workload and by a hash of the GEMM kernel source it was taken on: a changed kernel reports
 # null until captured again.  {workload: {"source": hash, "gemm": bytes, "gemm_tile": bytes}}
-GEMM_TRAFFIC = {}
+GEMM_TRAFFIC = {
+    # profiles/gemm_traffic_qwen3-8b-bs32.md, profiles/step_launches_qwen3-8b-bs1.md
+    "qwen3-8b-bs32": {"source": "b3df654e15822bdf", "gemm": 87.225e9 / 586, "gemm_tile": 15.254e9 / 182},
+    "qwen3-8b-bs1": {"source": "b3df654e15822bdf", "gemm_tile": 34.249e9 / 352},
+}
 
 
 def gemm_source_hash():
