@@ -84,6 +84,7 @@ def lib() -> ctypes.CDLL:
         L.alodlm_decode_block_sampled.argtypes = [vp, vp, ci, ci, cf, cf, ci, ci, ci, u64, ctypes.POINTER(DecodeOut),
                                                   ctypes.POINTER(ci)]
         L.alodlm_sync.argtypes = [vp]
+        L.alodlm_inject_wait_timeout.argtypes = [vp]
         L.alodlm_destroy.argtypes = [vp]
         L.alodlm_destroy.restype = None
         L.alodlm_last_error.argtypes = [vp]
@@ -304,6 +305,11 @@ class Handle:
 
     def sync(self):
         self._check(lib().alodlm_sync(self._h), "sync")
+
+    def inject_wait_timeout(self):
+        """Queue the error-path probe (a bounded wait that expires after about 2 s); the next
+        sync() raises AlodlmError with ALODLM_ETIMEOUT."""
+        self._check(lib().alodlm_inject_wait_timeout(self._h), "inject_wait_timeout")
 
     def debug_state(self, which: int, loop: int) -> torch.Tensor:
         dst = torch.empty((self.B, self.N, self.shape.hidden), dtype=torch.float32, device="cuda")

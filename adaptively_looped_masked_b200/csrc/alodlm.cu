@@ -1361,6 +1361,13 @@ int alodlm_set_timing(alodlm_t *h, int on) {
     return ALODLM_OK;
 }
 
+int alodlm_inject_wait_timeout(alodlm_t *h) {
+    if (!h) return ALODLM_EINVAL;
+    k::wait_expiry_kernel<<<1, 32, 0, h->stream>>>(h->d_err);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ALODLM_OK : cuda_fail(h, e, "wait_expiry_kernel");
+}
+
 int alodlm_sync(alodlm_t *h) {
     if (!h) return ALODLM_EINVAL;
     cudaError_t e = cudaStreamSynchronize(h->stream);

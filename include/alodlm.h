@@ -219,6 +219,13 @@ ALODLM_API int alodlm_decode_block_sampled(alodlm_t *h, const int32_t *block_ids
  * word since the last call (the word is then cleared), ECUDA on a CUDA error. */
 ALODLM_API int alodlm_sync(alodlm_t *h);
 
+/* Test hook for the error path (no counterpart in the paper): enqueue on the handle's stream a
+ * kernel whose one bounded wait (on an mbarrier nothing arrives on) expires after the library's
+ * wait limit (about 2 s), raising the device error word exactly as a timed-out wait inside a
+ * step would.  The next alodlm_sync then returns ETIMEOUT and re-arms the handle's counters;
+ * the handle stays usable.  No GPU fault is involved.  Errors: EINVAL (null handle), ECUDA. */
+ALODLM_API int alodlm_inject_wait_timeout(alodlm_t *h);
+
 /* Free everything the handle owns (synchronises first).  NULL is a no-op. */
 ALODLM_API void alodlm_destroy(alodlm_t *h);
 

@@ -116,8 +116,10 @@ def test_null_arguments_are_rejected(L):
     assert lib.alodlm_denoise_step(None, None, 1, 1, 0.5, 0.5, 1, 0, None) == -1
     assert lib.alodlm_decode_block(None, None, 1, 1, 0.5, 0.5, 1, 0, 1, None, None) == -1
     assert lib.alodlm_sync(None) == -1
+    assert lib.alodlm_inject_wait_timeout(None) == -1
     lib.alodlm_destroy(None)
     assert lib.alodlm_kernel_class_name(0) == b"gemm"
+    assert lib.alodlm_kernel_class_name(8) == b"gemm_tile"
     assert lib.alodlm_gemm_bf16(None, None, None, 1, 1, 8, None, 0, None) == -1
 
 

@@ -213,6 +213,27 @@ def test_state_and_argument_errors():
     assert (out["exit_depth"] >= 0).all()
 
 
+def test_expired_wait_reports_timeout_and_the_next_step_is_unchanged(mid):
+    """The error path of every bounded device wait, without a GPU fault: a probe kernel waits on
+    an mbarrier that nothing arrives on until the library's wait limit expires.  sync() reports
+    ALODLM_ETIMEOUT, re-arms the handle's counters and clears the error word; the next step on
+    the same handle is bit-identical to the one before the timeout and matches the oracle."""
+    import time
+    import adaptively_looped_masked_b200 as alo
+    before = mid.step(0.6, 0.5, rule=0)
+    t0 = time.time()
+    mid.handle.inject_wait_timeout()
+    with pytest.raises(alo.AlodlmError) as e:
+        mid.handle.sync()
+    assert e.value.code == -5  # ALODLM_ETIMEOUT
+    assert time.time() - t0 > 1.0  # the wait ran to its limit
+    mid.handle.sync()  # cleared: the handle is usable
+    after = mid.step(0.6, 0.5, rule=0)
+    for k in before:
+        np.testing.assert_array_equal(np.nan_to_num(before[k], nan=-7.0), np.nan_to_num(after[k], nan=-7.0))
+    print("after an expired wait", _step_parity(mid, 0.6, 0.5, 0))
+
+
 def test_memory_limit_gives_enomem():
     import adaptively_looped_masked_b200 as alo
     from synth import MODELS
