@@ -232,8 +232,11 @@ struct Cfg {
     static_assert(RECV_SEPARATE || RECV_BYTES <= (size_t)STAGES * STAGE_BYTES, "split-K partials must fit the ring");
 };
 
+// Two CTAs per SM (the split-K planner counts on it for tiles up to 64 wide): registers are
+// capped at 170 per thread (the 64-wide residual-add instance otherwise took 196, leaving one
+// CTA per SM and its 256-CTA grids in two waves).
 template <int BN, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, 2)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int rowsA,
                    int rowsB, const int *rowsA_dyn, int k_tiles, int kt_per_split, int a_fastest, int tiled,
                    EpiParams ep, int *err) {
