@@ -883,7 +883,11 @@ struct Fallback {
 // (the whole GPU works on each), one warp per row once the rows alone fill it
 int rmsnorm(alodlm *h, const float *x, const float *g, bf16 *xn, int M) {
     const int H = h->H;
-    if (M >= 256 && H % 128 == 0)
+    if (M >= 256 && H % 128 == 0 && H <= 128 * 32)
+        LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
+               (klaunch(k::rmsnorm_row_regs_kernel<32>, cdiv(M, 4), 128, 0, h->stream, x, g, xn, M, H,
+                        h->cfg.rms_eps)));
+    else if (M >= 256 && H % 128 == 0)
         LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
                (klaunch(k::rmsnorm_warp_kernel, cdiv(M, 8), 256, 0, h->stream, x, g, xn, M, H, h->cfg.rms_eps)));
     else

@@ -146,6 +146,42 @@ __global__ void rmsnorm_warp_kernel(const float *x, const float *g, bf16 *y, int
     }
 }
 
+// One warp per row with the whole row in registers (H a multiple of 128, at most 128 * MAXV):
+// every lane issues all of its float4 loads before the first use, so a row costs one memory
+// round trip instead of one per batch, and the second pass needs no re-read.  The sum of
+// squares is a fixed per-lane order and a fixed butterfly.
+template <int MAXV>
+__global__ void __launch_bounds__(128) rmsnorm_row_regs_kernel(const float *x, const float *g, bf16 *y, int M, int H,
+                                                                float eps) {
+    pdl_enter();
+    const int lane = threadIdx.x & 31;
+    const long long m = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (m >= M) return;
+    const float4 *xr = reinterpret_cast<const float4 *>(x + m * H);
+    const int nv = H / 128;  // float4 per lane
+    float4 v[MAXV];
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) v[i] = i < nv ? xr[i * 32 + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+    float ss[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) ss[i & 3] += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+    const float r = rsqrtf(warp_sum((ss[0] + ss[1]) + (ss[2] + ss[3])) / H + eps);
+    const float4 *gr = reinterpret_cast<const float4 *>(g);
+    uint2 *yr = reinterpret_cast<uint2 *>(y + m * H);
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+        if (i < nv) {
+            const float4 w = gr[i * 32 + lane];
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(v[i].x * r * w.x, v[i].y * r * w.y);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(v[i].z * r * w.z, v[i].w * r * w.w);
+            uint2 pk;
+            memcpy(&pk.x, &lo, 4);
+            memcpy(&pk.y, &hi, 4);
+            yr[i * 32 + lane] = pk;
+        }
+    }
+}
+
 // Per row m and head: optional per-head RMSNorm of q and k, rotate-half RoPE at the row's
 // position, then q -> q_out (bf16, packed: [slot j][kv head][position * G + head-in-group][hd],
 // so the G query heads of a KV head are consecutive rows) and k, v -> the KV arena slot (bf16).

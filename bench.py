@@ -226,8 +226,8 @@ def gemm_traffic_per_launch(workload, kernel_class):
 # measured it: loops run per sequence and tokens committed per step.  The reference arm runs
 # without the GPU arm's results and scales its per-layer timing by this profile.
 GPU_LOOP_PROFILE = {
-    "qwen3-8b-bs32": dict(loops=[3, 3, 2, 4, 2, 6, 4, 3, 3, 4, 3, 5, 3, 2, 3, 2, 2, 3, 2, 5, 4, 4, 2, 7, 5, 3, 2,
-                                 4, 2, 5, 4, 4], commits=1652),
+    "qwen3-8b-bs32": dict(loops=[3, 3, 2, 3, 2, 5, 4, 3, 3, 4, 3, 6, 3, 2, 3, 2, 2, 3, 2, 7, 4, 4, 2, 5, 5, 3, 3,
+                                 3, 2, 5, 3, 4], commits=1635),
 }
 
 
