@@ -37,6 +37,11 @@ namespace {
 #ifndef ALODLM_ATTN_CLUSTER16
 #define ALODLM_ATTN_CLUSTER16 1
 #endif
+// row count from which RMSNorm runs one warp per row (row in registers) instead of one block
+// per row
+#ifndef ALODLM_NORM_WARP_ROWS
+#define ALODLM_NORM_WARP_ROWS 256
+#endif
 // RMSNorm folded into the residual-add and projection epilogues (1) or a norm kernel before
 // every projection (0, the default: on a B200 the folded epilogues cost more than the norm
 // launches they replace -- Qwen3-8B shape bs 1 10.24 vs 9.86 ms per step, bs 32 114.5 vs
@@ -883,7 +888,7 @@ struct Fallback {
 // (the whole GPU works on each), one warp per row once the rows alone fill it
 int rmsnorm(alodlm *h, const float *x, const float *g, bf16 *xn, int M) {
     const int H = h->H;
-    if (M >= 256 && H % 128 == 0 && H <= 128 * 32)
+    if (M >= ALODLM_NORM_WARP_ROWS && H % 128 == 0 && H <= 128 * 32)
         LAUNCH(KC_NORM, 6.0 * M * H, 0.0,
                (klaunch(k::rmsnorm_row_regs_kernel<32>, cdiv(M, 4), 128, 0, h->stream, x, g, xn, M, H,
                         h->cfg.rms_eps)));
