@@ -197,8 +197,8 @@ def step_roofline(m, B, P, N, active_rows, readout_rows, peaks):
 # null until captured again.  {workload: {"source": hash, "gemm": bytes, "gemm_tile": bytes}}
 GEMM_TRAFFIC = {
     # profiles/gemm_traffic_qwen3-8b-bs32.md, profiles/step_launches_qwen3-8b-bs1.md
-    "qwen3-8b-bs32": {"source": "b3df654e15822bdf", "gemm": 87.225e9 / 586, "gemm_tile": 15.254e9 / 182},
-    "qwen3-8b-bs1": {"source": "b3df654e15822bdf", "gemm_tile": 34.249e9 / 352},
+    "qwen3-8b-bs32": {"source": "967b1f20f09d80f8", "gemm": 86.858e9 / 586, "gemm_tile": 15.243e9 / 182},
+    "qwen3-8b-bs1": {"source": "967b1f20f09d80f8", "gemm_tile": 34.253e9 / 352},
 }
 
 
