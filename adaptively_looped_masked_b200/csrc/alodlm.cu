@@ -799,7 +799,16 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
         int splits = 1;
         while (splits < want) splits <<= 1;
         if (splits > cap || (splits > 1 && (long long)splits * base > h->num_sms)) splits >>= 1;
-        const int kps = cdiv(ktiles, splits);  // trailing ranks may get no keys (empty partials)
+        int kps = cdiv(ktiles, splits);  // trailing ranks may get no keys (empty partials)
+        // a remainder shorter than a key tile rides on the last rank when that saves every other
+        // rank a tile: e.g. 8 full tiles + 32 keys over 8 ranks -> one tile each, the last two
+        const int full = kv_len / attn_tc::BKV, kps_full = std::max(1, cdiv(full, splits));
+        p.last_to_end = 0;
+        if (splits > 1 && kps_full < kps && (long long)splits * kps_full * attn_tc::BKV >= (long long)full * attn_tc::BKV &&
+            kv_len - (long long)splits * kps_full * attn_tc::BKV < attn_tc::BKV) {
+            kps = kps_full;
+            p.last_to_end = 1;
+        }
         p.n_splits = splits;
         p.keys_per_split = kps * attn_tc::BKV;
         if (splits > 1) {

@@ -57,6 +57,9 @@ struct Params {
     // prefix during a step): their first K/V stages are requested before griddepcontrol.wait.
     // 0: every key waits.
     int static_keys;
+    // 1: the last key split runs to kv_len even past keys_per_split (a remainder shorter than
+    // a key tile rides on the last rank instead of costing every rank a second tile)
+    int last_to_end;
 };
 
 // K-major operand, 128-byte swizzle (8-row atoms of 128 B, 1024 B apart)
@@ -117,7 +120,8 @@ __global__ void __launch_bounds__(192, 1)
     const int kvh = blockIdx.y / p.n_splits, split = blockIdx.y % p.n_splits;
     const int j = blockIdx.z;
     const int kstart = split * p.keys_per_split;
-    const int kend = min(p.kv_len, kstart + p.keys_per_split);
+    // the last rank may also take a ragged remainder past its range (last_to_end)
+    const int kend = (p.last_to_end && split == p.n_splits - 1) ? p.kv_len : min(p.kv_len, kstart + p.keys_per_split);
     const int n_tiles = kend > kstart ? (kend - kstart + BKV - 1) / BKV : 0;
 
     int pre = 0;  // K/V stages requested before the wait (thread 0, the producer)
@@ -277,15 +281,24 @@ __global__ void __launch_bounds__(192, 1)
             const bool resc = mt > m_ref + RESCALE_THRESHOLD;
             const float f = (resc && i > 0) ? exp2f(m_ref - mt) : 1.f;
             if (resc) m_ref = mt;
-            // p = 2^(s * scale - m_ref), summed as eight independent chains
+            // p = 2^(s * scale - m_ref), summed as eight independent chains; 32-key chunks that
+            // lie wholly past the range (a ragged last tile) are zero without exponentials
             const float neg_m = -m_ref;
             float sm[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) sm[c] = 0.f;
 #pragma unroll
-            for (int c = 0; c < BKV; ++c) {
-                sv[c] = ex2_approx(fmaf(sv[c], p.scale_log2, neg_m));
-                sm[c & 7] += sv[c];
+            for (int c0 = 0; c0 < BKV; c0 += 32) {
+                if (key0 + c0 < kend) {  // uniform across the CTA
+#pragma unroll
+                    for (int c = c0; c < c0 + 32; ++c) {
+                        sv[c] = ex2_approx(fmaf(sv[c], p.scale_log2, neg_m));
+                        sm[c & 7] += sv[c];
+                    }
+                } else {
+#pragma unroll
+                    for (int c = c0; c < c0 + 32; ++c) sv[c] = 0.f;
+                }
             }
             const float lt = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
             l = l * f + lt;
