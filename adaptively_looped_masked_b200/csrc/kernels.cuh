@@ -258,10 +258,12 @@ __global__ void qkv_post_kernel(const float *qkv, int nq, int nkv, int hd, const
 
 // The same for head_dim 128 with one block per row and each warp taking `hpw` (<= 8) heads of
 // it: every head's load and the row's RoPE table entries are issued before any arithmetic, so
-// a warp waits for one memory round trip instead of one per head.
-__global__ void qkv_post128_kernel(const float *qkv, int nq, int nkv, int hpw, const float *qn, const float *kn,
-                                   int qk_norm, float eps, const float2 *rope, RowMap map, bf16 *q_out, bf16 *kc,
-                                   bf16 *vc, long long seq_stride, long long head_stride) {
+// a warp waits for one memory round trip instead of one per head.  At 64 registers four blocks
+// share an SM (80 left three).
+__global__ void __launch_bounds__(256, 4)
+    qkv_post128_kernel(const float *qkv, int nq, int nkv, int hpw, const float *qn, const float *kn, int qk_norm,
+                       float eps, const float2 *rope, RowMap map, bf16 *q_out, bf16 *kc, bf16 *vc,
+                       long long seq_stride, long long head_stride) {
     pdl_enter();
     constexpr int HD = 128, MAXH = 8;
     const int m = blockIdx.x;
