@@ -458,19 +458,11 @@ def make_handle(alo, m, wl, w, stream, rank):
     return handle, time.time() - t0
 
 
-def run_ours(args, world, rank, local):
-    import adaptively_looped_masked_b200 as alo
-    wl = WORKLOADS[args.workload]
-    m = MODELS[wl.model]
-    peaks, peaks_src = load_peaks()
-    stream = torch.cuda.Stream()
-    w = make_weights(m, seed=0, device="cuda")
-    handle, prefill_s = make_handle(alo, m, wl, w, stream, rank)
-    torch.cuda.empty_cache()
-    block_np = make_block_ids(m, wl.batch, wl.block)
+def assemble_line(args, wl, world, r, peaks, peaks_src, prefill_s):
+    """The bench line of the GPU arm from one rank's measurement `r` (measure_step's dict): the
+    whole-job throughput over the max-over-ranks time, the roofline of the dominant
+    linear-layer kernel class and of each class, the step roofline, e2e and clocks."""
     tau, lam, rule = args.tau, args.lam, args.rule
-    r = measure_step(handle, m, wl, block_np, tau, lam, rule, args.steps, args.warmup, world, local, peaks, stream)
-
     max_ms = all_max(r["ms"], world)
     max_e2e = all_max(r["e2e_ms"], world)
     total_commits = all_sum(float(r["commits"]) * args.steps, world)
@@ -531,6 +523,24 @@ def run_ours(args, world, rank, local):
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "clocks": r["clocks"],
     }
+
+    return line
+
+
+def run_ours(args, world, rank, local):
+    import adaptively_looped_masked_b200 as alo
+    wl = WORKLOADS[args.workload]
+    m = MODELS[wl.model]
+    peaks, peaks_src = load_peaks()
+    stream = torch.cuda.Stream()
+    w = make_weights(m, seed=0, device="cuda")
+    handle, prefill_s = make_handle(alo, m, wl, w, stream, rank)
+    torch.cuda.empty_cache()
+    block_np = make_block_ids(m, wl.batch, wl.block)
+    tau, lam, rule = args.tau, args.lam, args.rule
+    r = measure_step(handle, m, wl, block_np, tau, lam, rule, args.steps, args.warmup, world, local, peaks, stream)
+
+    line = assemble_line(args, wl, world, r, peaks, peaks_src, prefill_s)
 
     if world == 1 and not args.no_extras:
         # the pages' sweep: tau x lambda on the same workload, active-row fraction per loop

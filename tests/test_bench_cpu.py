@@ -106,3 +106,45 @@ def test_reference_arm_under_two_ranks():
     assert out.returncode == 0, out.stderr[-3000:]
     lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1 and json.loads(lines[0])["impl"] == "reference"
+
+
+def test_gpu_arm_line_from_a_measurement():
+    """The GPU arm's JSON line, assembled from a synthetic measurement (no GPU): whole-job
+    throughput over the time, the roofline of whichever linear-layer class takes longer (the
+    many-row class against the sustained bf16 peak, the few-row class against HBM), both
+    classes under gemm_rooflines, traffic only for a recorded source hash, the step roofline."""
+    import argparse
+    import bench
+    from synth import WORKLOADS
+    wl = WORKLOADS["qwen3-8b-bs32"]
+    args = argparse.Namespace(tau=0.6, lam=0.5, rule=0, steps=10, warmup=3, workload="qwen3-8b-bs32",
+                              no_extras=True)
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops_sustained": 1400.0, "bf16_tflops": 1600.0}
+    classes = {
+        "gemm": {"ms": 70.0, "launches": 586, "bytes": 586 * 150e6, "flops": 7.0e13},
+        "gemm_tile": {"ms": 6.0, "launches": 182, "bytes": 182 * 85e6, "flops": 1.0e12},
+        "attention": {"ms": 16.0, "launches": 200, "bytes": 1e9, "flops": 1e12},
+    }
+    r = {"ms": 1050.0, "e2e_ms": 1070.0, "commits": 1635, "classes": classes, "tensor_bound": True,
+         "t_roof": 0.0655, "F": 9.0e13, "B": 1.1e11, "loops": [3] * 32, "active_rows": [2048, 0],
+         "readout_rows": [2048, 0], "launches_per_step": 1500, "h2d": 8192, "d2h": 1000, "clocks": None}
+    line = bench.assemble_line(args, wl, 1, r, peaks, "test", 1.0)
+    assert abs(line["ms_per_step"] - 105.0) < 1e-9
+    assert abs(line["value"] - 1635 * 10 / 1.05) < 1e-6
+    roof = line["roofline"]
+    assert roof["kernel_class"] == "gemm" and roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s"
+    assert abs(roof["achieved"] - 7.0e13 / 0.070 / 1e12) < 1e-6 and abs(roof["frac"] - roof["achieved"] / 1400.0) < 1e-12
+    tile = line["gemm_rooflines"]["gemm_tile"]
+    assert tile["bound"] == "hbm" and abs(tile["achieved"] - 182 * 85e6 / 0.006 / 1e9) < 1e-6
+    recorded = bench.GEMM_TRAFFIC.get("qwen3-8b-bs32")
+    if recorded and recorded["source"] == bench.gemm_source_hash():
+        assert roof["traffic"] == recorded["gemm"]
+    else:
+        assert roof["traffic"] is None
+    assert abs(line["step_roofline"]["frac"] - 65.5 / 105.0) < 1e-9
+    assert line["dominant_kernel_class"] == "gemm" and line["gpu_launches"] == 15000
+    assert line["e2e"]["h2d_bytes_per_step"] == 8192
+    # few rows: the per-tile class dominates and is held against HBM
+    classes["gemm"]["ms"] = 1.0
+    line = bench.assemble_line(args, wl, 1, r, peaks, "test", 1.0)
+    assert line["roofline"]["kernel_class"] == "gemm_tile" and line["roofline"]["bound"] == "hbm"
