@@ -575,7 +575,7 @@ struct alodlm {
     int n_slots = 0, pos_stride = 0;
     long long head_stride = 0, seq_stride = 0, slot_elems = 0;
     float2 *rope = nullptr;
-    bool tc_attn = false;            // tcgen05 attention for the step (head_dim 128)
+    bool tc_attn = false;            // tcgen05 attention (head_dim 128): steps, prefills, appends
     CUtensorMap tm_q, tm_kv_k, tm_kv_v;
 
     // prefill state
@@ -756,9 +756,15 @@ int linear(alodlm *h, const CUtensorMap &tmW, int Nw, const bf16 *actp, int M, i
 
 // attention of M rows (n_seq sequences x rows_per_seq) against slot `slot`, keys [0, kv_len)
 int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_len, int causal) {
-    if (!causal && h->tc_attn) {
+    if (h->tc_attn) {
         attn_tc::Params p{};
-        p.static_keys = std::max(0, kv_len - map.rows_per_seq);  // the step's cached prefix
+        // keys before the rows' own: the step's cached prefix, or the positions an append extends
+        p.static_keys = std::max(0, kv_len - map.rows_per_seq);
+        p.causal = causal;
+        p.pos0 = map.pos0;
+        p.row_t = map.row_t;
+        p.seq_off = map.seq_off;
+        p.seq_cnt = map.seq_cnt;
         p.G = h->nq / h->nkv;
         p.RP = p.G * map.rows_per_seq;
         p.nkv = h->nkv;
@@ -778,11 +784,11 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
         const int base = qtiles * h->nkv * n_seq;
         const int ktiles = cdiv(kv_len, attn_tc::BKV);
         const double bytes = 4.0 * n_seq * h->nkv * (double)kv_len * h->hd + 4.0 * M * h->nq * h->hd;
-        const double flops = 4.0 * M * h->nq * (double)kv_len * h->hd;
+        const double flops = 4.0 * M * h->nq * (double)kv_len * h->hd * (causal ? 0.5 : 1.0);
         // two query tiles per CTA (K/V loaded once for both, softmax warpgroups in turn) where a
         // (sequence, KV head) has two and the pairs still cover half the SMs without a key split
         const int qpairs = cdiv(qtiles, 2);
-        if (ALODLM_ATTN_PQ && qtiles >= 2 && 2 * qpairs * h->nkv * n_seq >= h->num_sms) {
+        if (!causal && !map.seq_cnt && ALODLM_ATTN_PQ && qtiles >= 2 && 2 * qpairs * h->nkv * n_seq >= h->num_sms) {
             p.n_splits = 1;
             p.keys_per_split = ktiles * attn_tc::BKV;
             LAUNCH(KC_ATTN, bytes, flops,
@@ -794,8 +800,10 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
         // rows evenly; 8 CTAs, or 16 where that many 16-CTA clusters fit at once): enough CTAs
         // to cover the SMs, rounded up to the next power of two while the grid still fits in
         // one wave, so that a latency-bound launch walks one key tile per CTA
+        // causal rows: no key split (each query tile walks keys [0, its last position]; a
+        // prefill's query tiles alone fill the SMs)
         const int cap = (ALODLM_ATTN_CLUSTER16 && attn_clusters16() >= base) ? 16 : 8;
-        const int want = std::max(1, std::min(std::min(ktiles, cdiv(h->num_sms, base)), cap));
+        const int want = causal ? 1 : std::max(1, std::min(std::min(ktiles, cdiv(h->num_sms, base)), cap));
         int splits = 1;
         while (splits < want) splits <<= 1;
         if (splits > cap || (splits > 1 && (long long)splits * base > h->num_sms)) splits >>= 1;

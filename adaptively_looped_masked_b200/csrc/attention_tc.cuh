@@ -2,8 +2,11 @@
 //
 // One CTA serves 128 packed query rows of one (sequence, KV head): packed row r is query head
 // kvh*G + r % G at block position r / G (q is stored in that packed order), so the G query
-// heads of a KV head share every K/V tile.  head_dim 128.  The block attends every prefix key
-// and every block key (no mask inside [0, kv_len)).
+// heads of a KV head share every K/V tile.  head_dim 128.  A denoising step's block attends
+// every prefix key and every block key (no mask inside [0, kv_len)); causal rows (a prefill or
+// an append, possibly compacted to the positions that run a Core depth) attend keys up to their
+// own position: the CTA's key range ends at its last row's position, and the key tiles that
+// cross the tile's first row's position mask each row at its own.
 //
 //   warp 0      TMA: Q once; K and V tiles of 128 keys (two 64-wide halves each, 128-byte
 //               swizzle) into a 2-stage ring, straight from the depth-aware KV arena
@@ -60,6 +63,12 @@ struct Params {
     // 1: the last key split runs to kv_len even past keys_per_split (a remainder shorter than
     // a key tile rides on the last rank instead of costing every rank a second tile)
     int last_to_end;
+    // 1: row u of sequence slot j sits at position pos0 + (row_t ? row_t[row_off + u] : u) and
+    // sees keys [0, that position] (n_splits must be 1).  Row tables (compacted rows, null
+    // otherwise, causal or not): slot j owns output rows [seq_off[j], seq_off[j] + seq_cnt[j]),
+    // in position order; without them its rows are j * Tq + u, u < Tq.
+    int causal, pos0;
+    const int *row_t, *seq_off, *seq_cnt;
 };
 
 // K-major operand, 128-byte swizzle (8-row atoms of 128 B, 1024 B apart)
@@ -116,12 +125,27 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 12);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qtile = blockIdx.x;
+    // causal: the last query tiles (the longest key ranges) are scheduled first
+    const int qtile = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
     const int kvh = blockIdx.y / p.n_splits, split = blockIdx.y % p.n_splits;
     const int j = blockIdx.z;
+    // this slot's query rows (fewer than Tq when compacted; the row tables were copied in before
+    // the layer's first kernel started, so they are read before griddepcontrol.wait)
+    const int seq_rows = p.seq_cnt ? p.seq_cnt[j] : p.Tq;
+    const int row_off = p.seq_off ? p.seq_off[j] : j * p.Tq;
+    const int rows_packed = p.G * seq_rows;
+    auto pos_of = [&](int u) { return p.pos0 + (p.row_t ? p.row_t[row_off + u] : u); };
     const int kstart = split * p.keys_per_split;
     // the last rank may also take a ragged remainder past its range (last_to_end)
-    const int kend = (p.last_to_end && split == p.n_splits - 1) ? p.kv_len : min(p.kv_len, kstart + p.keys_per_split);
+    int kend = (p.last_to_end && split == p.n_splits - 1) ? p.kv_len : min(p.kv_len, kstart + p.keys_per_split);
+    int mask_from = kend;  // the first key that some row of the tile does not see
+    if (qtile * BQ >= rows_packed) {
+        kend = kstart;  // no query rows in this tile
+    } else if (p.causal) {
+        // rows are in position order: the last row sees the most keys, the first the fewest
+        kend = min(kend, pos_of(min(qtile * BQ + BQ - 1, rows_packed - 1) / p.G) + 1);
+        mask_from = min(kend, pos_of(qtile * BQ / p.G) + 1);
+    }
     const int n_tiles = kend > kstart ? (kend - kstart + BKV - 1) / BKV : 0;
 
     int pre = 0;  // K/V stages requested before the wait (thread 0, the producer)
@@ -242,6 +266,10 @@ __global__ void __launch_bounds__(192, 1)
         const int q = warp & 3;
         const int t = q * 32 + lane;  // TMEM lane = row of the tile
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        // keys [0, row_end) of this row; every row sees key 0, so the first tile of an
+        // unsplit range sets a finite reference max
+        const int rp_t = qtile * BQ + t;
+        const int row_end = (p.causal && rp_t < rows_packed) ? min(kend, pos_of(rp_t / p.G) + 1) : kend;
         bool ok = n_tiles > 0;
         for (int i = 0; i < n_tiles && ok; ++i) {
             const int s = i & 1;
@@ -263,10 +291,10 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             const int key0 = kstart + i * BKV;
-            if (key0 + BKV > kend) {  // ragged last tile (uniform across the CTA)
+            if (key0 + BKV > mask_from) {  // ragged last tile or causal diagonal (uniform across the CTA)
 #pragma unroll
                 for (int c = 0; c < BKV; ++c)
-                    if (key0 + c >= kend) sv[c] = -INFINITY;
+                    if (key0 + c >= row_end) sv[c] = -INFINITY;
             }
             // row max of the raw scores (the scale is positive), as eight independent chains
             float mx[8];
@@ -283,7 +311,7 @@ __global__ void __launch_bounds__(192, 1)
             if (resc) m_ref = mt;
             // p = 2^(s * scale - m_ref), summed as eight independent chains; 32-key chunks that
             // lie wholly past the range (a ragged last tile) are zero without exponentials
-            const float neg_m = -m_ref;
+            const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;  // a row with no key yet: p = 0
             float sm[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) sm[c] = 0.f;
@@ -345,9 +373,9 @@ __global__ void __launch_bounds__(192, 1)
             mbar_wait(pv_done + ((n_tiles - 1) & 1), ((uint32_t)((n_tiles - 1) >> 1)) & 1u, p.err)) {
             tc_fence_after();
             const int rp = qtile * BQ + t;
-            const bool valid = rp < p.RP;
+            const bool valid = rp < rows_packed;
             const int tt = rp / p.G, h = kvh * p.G + rp % p.G;
-            const int m = j * p.Tq + tt;
+            const int m = row_off + tt;
             if (p.n_splits == 1) {
                 const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
@@ -419,7 +447,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int e = threadIdx.x; e < rs * CH; e += blockDim.x) {
             const int lr = e / CH, c8 = (e % CH) * 8;
             const int rp = qtile * BQ + split * rs + lr;
-            if (rp >= p.RP) continue;
+            if (rp >= rows_packed) continue;
             float M = -INFINITY;
             for (int rr = 0; rr < S; ++rr) {
                 const float *ml = recv_ml + 2 * (rr * rs + lr);
@@ -451,7 +479,7 @@ __global__ void __launch_bounds__(192, 1)
             pk.y = pack2_bf16(acc[2] * inv, acc[3] * inv);
             pk.z = pack2_bf16(acc[4] * inv, acc[5] * inv);
             pk.w = pack2_bf16(acc[6] * inv, acc[7] * inv);
-            *reinterpret_cast<uint4 *>(p.out + (long long)(j * p.Tq + tt) * p.out_ld + h * HD + c8) = pk;
+            *reinterpret_cast<uint4 *>(p.out + (long long)(row_off + tt) * p.out_ld + h * HD + c8) = pk;
         }
     }
     tc_fence_before();

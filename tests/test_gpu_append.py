@@ -39,12 +39,23 @@ def _prefill_append(case, P0, e):
     case.handle.sync()
 
 
-@pytest.mark.parametrize("name", ["tiny", "mid"])
-def test_append_matches_oracle_and_one_long_prefill(name):
+def _append_shape(name):
+    """(model, batch, P0, N, k_max): the tiny and mid workloads, and "attn-probe": the Qwen3-8B
+    attention geometry (32 q / 8 kv heads, head_dim 128) on 300 + 37 positions.  Its causal rows
+    run on the tensor-core attention: 32 positions per 128-row query tile, three key tiles (the
+    last ragged), rows compacted to the positions that reach depths 2 and 3, and an append that
+    starts at position 300, inside a query tile's span of positions."""
+    if name == "attn-probe":
+        return "attn-probe", 2, 300, 37, 3
     wl = WORKLOADS[name]
-    m, K, B = MODELS[wl.model], wl.k_max, wl.batch
-    P0, N = wl.prefix, wl.block
-    case = Case(wl.model, B, P0 + N, N, K, debug=True)
+    return wl.model, wl.batch, wl.prefix, wl.block, wl.k_max
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid", "attn-probe"])
+def test_append_matches_oracle_and_one_long_prefill(name):
+    model, B, P0, N, K = _append_shape(name)
+    m = MODELS[model]
+    case = Case(model, B, P0 + N, N, K, debug=True)
     e = make_exit_depths(B, P0 + N, K, seed=5)
     _prefill_append(case, P0, e)
     o = case.oracle("bf16")
