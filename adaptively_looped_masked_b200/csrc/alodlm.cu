@@ -225,7 +225,7 @@ int attn_clusters16() {
     if (dev < 0 || dev >= 64) return 0;
     if (!cached[dev]) {
         int n = 0;
-        if (cudaFuncSetAttribute(attn_tc::attn_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+        if (cudaFuncSetAttribute(attn_tc::attn_tc_kernel<128>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
             cudaSuccess) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(1, 16 * 8, 1);
@@ -238,7 +238,7 @@ int attn_clusters16() {
             attr[0].val.clusterDim.z = 1;
             cfg.attrs = attr;
             cfg.numAttrs = 1;
-            if (cudaOccupancyMaxActiveClusters(&n, attn_tc::attn_tc_kernel, &cfg) != cudaSuccess) n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, attn_tc::attn_tc_kernel<128>, &cfg) != cudaSuccess) n = 0;
         }
         cudaGetLastError();
         cached[dev] = n > 0 ? n : -1;
@@ -281,7 +281,10 @@ bool init_kernel_attrs() {
     set_sk_attr<64, gemm::EPI_ADD>();
     set_sk_attr<64, gemm::EPI_SWIGLU>();
     cudaFuncSetAttribute(attn::attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 5 * 64 * 64 * 2);
-    cudaFuncSetAttribute(attn_tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_tc::SMEM);
+    cudaFuncSetAttribute(attn_tc::attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)attn_tc::smem_bytes<128>());
+    cudaFuncSetAttribute(attn_tc::attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)attn_tc::smem_bytes<64>());
     cudaFuncSetAttribute(attn_pq::attn_pq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_pq::SMEM);
     cudaFuncSetAttribute(attn::attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 5 * 64 * 128 * 2);
     done[dev] = cudaGetLastError() == cudaSuccess;
@@ -575,7 +578,7 @@ struct alodlm {
     int n_slots = 0, pos_stride = 0;
     long long head_stride = 0, seq_stride = 0, slot_elems = 0;
     float2 *rope = nullptr;
-    bool tc_attn = false;            // tcgen05 attention (head_dim 128): steps, prefills, appends
+    bool tc_attn = false;            // tcgen05 attention (head_dim 64 or 128): steps, prefills, appends
     CUtensorMap tm_q, tm_kv_k, tm_kv_v;
 
     // prefill state
@@ -788,7 +791,8 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
         // two query tiles per CTA (K/V loaded once for both, softmax warpgroups in turn) where a
         // (sequence, KV head) has two and the pairs still cover half the SMs without a key split
         const int qpairs = cdiv(qtiles, 2);
-        if (!causal && !map.seq_cnt && ALODLM_ATTN_PQ && qtiles >= 2 && 2 * qpairs * h->nkv * n_seq >= h->num_sms) {
+        if (h->hd == attn_tc::HD && !causal && !map.seq_cnt && ALODLM_ATTN_PQ && qtiles >= 2 &&
+            2 * qpairs * h->nkv * n_seq >= h->num_sms) {
             p.n_splits = 1;
             p.keys_per_split = ktiles * attn_tc::BKV;
             LAUNCH(KC_ATTN, bytes, flops,
@@ -802,7 +806,7 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
         // one wave, so that a latency-bound launch walks one key tile per CTA
         // causal rows: no key split (each query tile walks keys [0, its last position]; a
         // prefill's query tiles alone fill the SMs)
-        const int cap = (ALODLM_ATTN_CLUSTER16 && attn_clusters16() >= base) ? 16 : 8;
+        const int cap = (h->hd == 128 && ALODLM_ATTN_CLUSTER16 && attn_clusters16() >= base) ? 16 : 8;
         const int want = causal ? 1 : std::max(1, std::min(std::min(ktiles, cdiv(h->num_sms, base)), cap));
         int splits = 1;
         while (splits < want) splits <<= 1;
@@ -819,12 +823,15 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
         }
         p.n_splits = splits;
         p.keys_per_split = kps * attn_tc::BKV;
+        // one instance per head_dim (one or two 64-wide halves per head vector)
+        auto *const kern = h->hd == 128 ? attn_tc::attn_tc_kernel<128> : attn_tc::attn_tc_kernel<64>;
+        const size_t smem = h->hd == 128 ? attn_tc::smem_bytes<128>() : attn_tc::smem_bytes<64>();
         if (splits > 1) {
             // cluster along y: the `splits` consecutive y indices of one kv head
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(qtiles, h->nkv * splits, n_seq);
             cfg.blockDim = dim3(192);
-            cfg.dynamicSmemBytes = attn_tc::SMEM;
+            cfg.dynamicSmemBytes = smem;
             cfg.stream = h->stream;
             cudaLaunchAttribute attr[2];
             attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -836,11 +843,11 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
             cfg.attrs = attr;
             cfg.numAttrs = ALODLM_PDL ? 2 : 1;
             LAUNCH(KC_ATTN, bytes, flops,
-                   cudaLaunchKernelEx(&cfg, attn_tc::attn_tc_kernel, h->tm_q, h->tm_kv_k, h->tm_kv_v, p));
+                   cudaLaunchKernelEx(&cfg, kern, h->tm_q, h->tm_kv_k, h->tm_kv_v, p));
         } else {
             LAUNCH(KC_ATTN, bytes, flops,
-                   klaunch(attn_tc::attn_tc_kernel, dim3(qtiles, h->nkv, n_seq), 192, attn_tc::SMEM, h->stream,
-                           h->tm_q, h->tm_kv_k, h->tm_kv_v, p));
+                   klaunch(kern, dim3(qtiles, h->nkv, n_seq), 192, smem, h->stream, h->tm_q, h->tm_kv_k, h->tm_kv_v,
+                           p));
         }
         return ALODLM_OK;
     }
@@ -1232,7 +1239,8 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
     cudaMemsetAsync(h->kv_v, 0, (size_t)h->slot_elems * h->n_slots * 2, h->stream);
     {
         const long long arena_rows = (long long)h->n_slots * cfg->max_batch * h->nkv * h->pos_stride;
-        h->tc_attn = h->hd == 128 && arena_rows + 256 < (1ll << 31) && (long long)R * h->nq < (1ll << 31);
+        h->tc_attn = (h->hd == 128 || h->hd == 64) && arena_rows + 256 < (1ll << 31) &&
+                     (long long)R * h->nq < (1ll << 31);
         if (h->tc_attn)
             h->tc_attn = make_tmap(&h->tm_q, h->qb, h->hd, (int)(R * h->nq), attn_tc::BQ) &&
                          make_tmap(&h->tm_kv_k, h->kv_k, h->hd, (int)arena_rows, attn_tc::BKV) &&

@@ -2,14 +2,15 @@
 //
 // One CTA serves 128 packed query rows of one (sequence, KV head): packed row r is query head
 // kvh*G + r % G at block position r / G (q is stored in that packed order), so the G query
-// heads of a KV head share every K/V tile.  head_dim 128.  A denoising step's block attends
+// heads of a KV head share every K/V tile.  head_dim 64 or 128 (a template argument: one or two
+// 64-wide, 128-byte-swizzled halves per head vector).  A denoising step's block attends
 // every prefix key and every block key (no mask inside [0, kv_len)); causal rows (a prefill or
 // an append, possibly compacted to the positions that run a Core depth) attend keys up to their
 // own position: the CTA's key range ends at its last row's position, and the key tiles that
 // cross the tile's first row's position mask each row at its own.
 //
-//   warp 0      TMA: Q once; K and V tiles of 128 keys (two 64-wide halves each, 128-byte
-//               swizzle) into a 2-stage ring, straight from the depth-aware KV arena
+//   warp 0      TMA: Q once; K and V tiles of 128 keys (64-wide halves, 128-byte swizzle)
+//               into a 2-stage ring, straight from the depth-aware KV arena
 //   warp 1      tcgen05.mma: S_i = Q K_i^T into a double-buffered TMEM tile (M=128, N=128),
 //               then O += P_i V_i into the TMEM accumulator (V read MN-major)
 //   warps 2-5   softmax, one thread per query row: tcgen05.ld its S row, exp2 with a running
@@ -31,7 +32,7 @@ namespace attn_tc {
 
 namespace cg = cooperative_groups;
 
-constexpr int HD = 128;
+constexpr int HD = 128;        // head_dim of the two-tile kernel (attention_pq.cuh)
 constexpr int BQ = 128;        // query rows per CTA
 constexpr int BKV = 128;       // keys per tile
 constexpr int KV_STAGES = 2;
@@ -42,7 +43,12 @@ constexpr uint32_t P_BYTES = 2 * HALF;
 constexpr uint32_t TMEM_COLS = 512;      // S0 [0,128) S1 [128,256) O [256,384)
 constexpr uint32_t O_COL = 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
-constexpr size_t SMEM = 1024 + Q_BYTES + 2 * KV_STAGES * KV_BYTES + 2 * P_BYTES + 256;  // P double-buffered
+// shared memory at head_dim D: Q, the K and V rings, P double-buffered, barriers
+template <int D>
+constexpr size_t smem_bytes() {
+    return 1024 + (D / 64) * HALF + 2 * KV_STAGES * (D / 64) * HALF + 2 * P_BYTES + 256;
+}
+constexpr size_t SMEM = smem_bytes<HD>();
 
 struct Params {
     int RP;            // packed query rows per (sequence, kv head) = G * rows_per_seq
@@ -105,15 +111,20 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+template <int D>
 __global__ void __launch_bounds__(192, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, Params p) {
+    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    constexpr int NH = D / 64;              // 64-wide halves of a head vector
+    constexpr uint32_t QB = NH * HALF;      // the Q tile
+    constexpr uint32_t KVB = NH * HALF;     // one K (or V) tile
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem;
-    uint8_t *sK = sQ + Q_BYTES;                       // [stage] K tiles
-    uint8_t *sV = sK + KV_STAGES * KV_BYTES;          // [stage] V tiles
-    uint8_t *sP = sV + KV_STAGES * KV_BYTES;
+    uint8_t *sK = sQ + QB;                       // [stage] K tiles
+    uint8_t *sV = sK + KV_STAGES * KVB;          // [stage] V tiles
+    uint8_t *sP = sV + KV_STAGES * KVB;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sP + 2 * P_BYTES);
     uint64_t *q_full = bars;
     uint64_t *k_full = bars + 1;                      // [2]
@@ -169,12 +180,10 @@ __global__ void __launch_bounds__(192, 1)
             const int kvrow0 = (int)((((long long)p.slot * p.max_batch + b0) * p.nkv + kvh) * p.pos_stride);
             for (; pre < min(n_tiles, KV_STAGES) && kstart + (pre + 1) * BKV <= p.static_keys; ++pre) {
                 const int row = kvrow0 + kstart + pre * BKV;
-                mbar_arrive_expect_tx(k_full + pre, KV_BYTES);
-                tma_load_2d(sK + pre * KV_BYTES, &tmK, k_full + pre, 0, row);
-                tma_load_2d(sK + pre * KV_BYTES + HALF, &tmK, k_full + pre, 64, row);
-                mbar_arrive_expect_tx(v_full + pre, KV_BYTES);
-                tma_load_2d(sV + pre * KV_BYTES, &tmV, v_full + pre, 0, row);
-                tma_load_2d(sV + pre * KV_BYTES + HALF, &tmV, v_full + pre, 64, row);
+                mbar_arrive_expect_tx(k_full + pre, KVB);
+                for (int hh = 0; hh < NH; ++hh) tma_load_2d(sK + pre * KVB + hh * HALF, &tmK, k_full + pre, 64 * hh, row);
+                mbar_arrive_expect_tx(v_full + pre, KVB);
+                for (int hh = 0; hh < NH; ++hh) tma_load_2d(sV + pre * KVB + hh * HALF, &tmV, v_full + pre, 64 * hh, row);
             }
         }
     }
@@ -194,9 +203,8 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 0) {
         if (lane == 0 && n_tiles > 0) {
             const int qrow = (j * p.nkv + kvh) * p.RP + qtile * BQ;
-            mbar_arrive_expect_tx(q_full, Q_BYTES);
-            tma_load_2d(sQ, &tmQ, q_full, 0, qrow);
-            tma_load_2d(sQ + HALF, &tmQ, q_full, 64, qrow);
+            mbar_arrive_expect_tx(q_full, QB);
+            for (int hh = 0; hh < NH; ++hh) tma_load_2d(sQ + hh * HALF, &tmQ, q_full, 64 * hh, qrow);
             const int kvrow0 = (int)((((long long)p.slot * p.max_batch + b) * p.nkv + kvh) * p.pos_stride);
             int issued = pre;
             for (int i = pre; i < n_tiles; ++i) {
@@ -204,12 +212,10 @@ __global__ void __launch_bounds__(192, 1)
                 if (!mbar_wait(kv_empty + s, ((uint32_t)(i >> 1) & 1u) ^ 1u, p.err)) break;
                 issued = i + 1;
                 const int row = kvrow0 + kstart + i * BKV;
-                mbar_arrive_expect_tx(k_full + s, KV_BYTES);
-                tma_load_2d(sK + s * KV_BYTES, &tmK, k_full + s, 0, row);
-                tma_load_2d(sK + s * KV_BYTES + HALF, &tmK, k_full + s, 64, row);
-                mbar_arrive_expect_tx(v_full + s, KV_BYTES);
-                tma_load_2d(sV + s * KV_BYTES, &tmV, v_full + s, 0, row);
-                tma_load_2d(sV + s * KV_BYTES + HALF, &tmV, v_full + s, 64, row);
+                mbar_arrive_expect_tx(k_full + s, KVB);
+                for (int hh = 0; hh < NH; ++hh) tma_load_2d(sK + s * KVB + hh * HALF, &tmK, k_full + s, 64 * hh, row);
+                mbar_arrive_expect_tx(v_full + s, KVB);
+                for (int hh = 0; hh < NH; ++hh) tma_load_2d(sV + s * KVB + hh * HALF, &tmV, v_full + s, 64 * hh, row);
             }
             // no copy into shared memory may still be in flight when the CTA exits
             mbar_wait(q_full, 0, p.err);
@@ -221,13 +227,13 @@ __global__ void __launch_bounds__(192, 1)
     } else if (warp == 1) {
         if (lane == 0 && n_tiles > 0) {
             constexpr uint32_t idesc_s = umma_idesc_bf16(BQ, BKV);
-            constexpr uint32_t idesc_o = umma_idesc_bf16(BQ, HD) | (1u << 16);  // B (V) MN-major
+            constexpr uint32_t idesc_o = umma_idesc_bf16(BQ, D) | (1u << 16);  // B (V) MN-major
             const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
             auto issue_s = [&](int i) {
                 const int s = i & 1;
-                const uint32_t k_addr = smem_u32(sK + s * KV_BYTES);
+                const uint32_t k_addr = smem_u32(sK + s * KVB);
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
+                for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
                     umma_f16(tmem + s * BKV, sdesc_k(q_addr + off), sdesc_k(k_addr + off), idesc_s, kk > 0 ? 1u : 0u);
                 }
@@ -248,7 +254,7 @@ __global__ void __launch_bounds__(192, 1)
                 if (!mbar_wait(p_full, (uint32_t)i & 1u, p.err)) break;
                 if (!mbar_wait(v_full + s, ((uint32_t)(i >> 1)) & 1u, p.err)) break;
                 tc_fence_after();
-                const uint32_t v_addr = smem_u32(sV + s * KV_BYTES);
+                const uint32_t v_addr = smem_u32(sV + s * KVB);
                 const uint32_t pb_addr = p_addr + (i & 1) * P_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < BKV / 16; ++kk) {
@@ -342,7 +348,7 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 tc_fence_after();
 #pragma unroll 1
-                for (int c0 = 0; c0 < HD; c0 += 16) {
+                for (int c0 = 0; c0 < D; c0 += 16) {
                     float v[16];
                     tmem_ld16(tmem + lane_base + O_COL + c0, v);
 #pragma unroll
@@ -379,7 +385,7 @@ __global__ void __launch_bounds__(192, 1)
             if (p.n_splits == 1) {
                 const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
-                for (int c0 = 0; c0 < HD; c0 += 16) {
+                for (int c0 = 0; c0 < D; c0 += 16) {
                     float v[16];
                     tmem_ld16(tmem + lane_base + O_COL + c0, v);
                     if (valid) {
@@ -392,7 +398,7 @@ __global__ void __launch_bounds__(192, 1)
                         w1.y = pack2_bf16(v[10] * inv, v[11] * inv);
                         w1.z = pack2_bf16(v[12] * inv, v[13] * inv);
                         w1.w = pack2_bf16(v[14] * inv, v[15] * inv);
-                        bf16 *dst = p.out + (long long)m * p.out_ld + h * HD + c0;
+                        bf16 *dst = p.out + (long long)m * p.out_ld + h * D + c0;
                         *reinterpret_cast<uint4 *>(dst) = w0;
                         *reinterpret_cast<uint4 *>(dst + 8) = w1;
                     }
@@ -407,12 +413,12 @@ __global__ void __launch_bounds__(192, 1)
         // The splits of this (sequence, kv head, query tile) form one cluster (rank = split).
         // Phase 0: every CTA is done with its K/V ring and P tiles (a softmax thread gets here
         // after the last PV product completed, or with no keys at all), which become receive
-        // buffers: [source rank][owned row][HD + 4] f32 partial O rows in the K/V ring (66 KB) and
+        // buffers: [source rank][owned row][D + 4] f32 partial O rows in the K/V ring (66 KB at D = 128) and
         // (reference max, l) pairs in the P tiles.
         const int S = p.n_splits, rs = BQ / S;
         float *recv_o = reinterpret_cast<float *>(sK);
         float *recv_ml = reinterpret_cast<float *>(sP);
-        constexpr int LDO = HD + 4;
+        constexpr int LDO = D + 4;
         cluster_arrive_relaxed();
         cluster_wait_acquire();
         if (warp >= 2) {
@@ -425,7 +431,7 @@ __global__ void __launch_bounds__(192, 1)
                 const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
                 const uint32_t dst = cluster_map(smem_u32(recv_o + (size_t)slot * LDO), owner);
 #pragma unroll 1
-                for (int c0 = 0; c0 < HD; c0 += 32) {
+                for (int c0 = 0; c0 < D; c0 += 32) {
                     uint32_t r[32];
                     tmem_ld16_async(tmem + lane_base + O_COL + c0, &r[0]);
                     tmem_ld16_async(tmem + lane_base + O_COL + c0 + 16, &r[16]);
@@ -443,7 +449,7 @@ __global__ void __launch_bounds__(192, 1)
         cluster_wait_acquire();  // every partial of the rows owned here has landed
         // merge, in rank order: O = sum_r 2^(m_r - M) O_r / sum_r 2^(m_r - M) l_r over the ranks
         // that saw keys (l_r > 0); thread = (owned row, 8 columns)
-        constexpr int CH = HD / 8;
+        constexpr int CH = D / 8;
         for (int e = threadIdx.x; e < rs * CH; e += blockDim.x) {
             const int lr = e / CH, c8 = (e % CH) * 8;
             const int rp = qtile * BQ + split * rs + lr;
@@ -479,7 +485,7 @@ __global__ void __launch_bounds__(192, 1)
             pk.y = pack2_bf16(acc[2] * inv, acc[3] * inv);
             pk.z = pack2_bf16(acc[4] * inv, acc[5] * inv);
             pk.w = pack2_bf16(acc[6] * inv, acc[7] * inv);
-            *reinterpret_cast<uint4 *>(p.out + (long long)(row_off + tt) * p.out_ld + h * HD + c8) = pk;
+            *reinterpret_cast<uint4 *>(p.out + (long long)(row_off + tt) * p.out_ld + h * D + c8) = pk;
         }
     }
     tc_fence_before();

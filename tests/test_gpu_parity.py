@@ -1,17 +1,19 @@
 """GPU parity: the CUDA library (through the C ABI) against the CPU oracle on the same
-seeded inputs.  Three checks per step:
+seeded inputs.  Three checks per step (tests/gpu_util.py, ``step_parity``):
 
 1. readout stage: the oracle's LM head, entropy, argmax and ExitGate applied to the GPU's
    own readout states r^(s) (kernel precision, r rounded to bf16 as the kernel does) match
-   the GPU's traces: entropy within 1e-2 nats, lambda within 1e-2, argmax exact except
+   the GPU's traces: entropy within 1e-2 nats, lambda within 1e-3, argmax exact except
    where the top-two logit gap is below 1e-3;
 2. decisions: every commit, exit depth, token and halt is re-taken from the GPU's traces by
    the oracle's rules (float32 thresholds) and must match bit-exactly;
-3. end to end: the float64 oracle, taking the GPU's decisions, runs the whole step; loop
-   inputs, Core outputs and readout states (and the logits they give) match within 2e-2
-   relative per row, and each entropy within 1e-2 nats plus the first-order effect of its
-   logit deviation.  The decisions the float64 oracle would have taken differently from
-   its own values are counted and printed.
+3. end to end: the float64 oracle runs the whole step from the same ids and weights and
+   takes its own decisions; only where a deciding value lies inside a fixed band around its
+   threshold (per loop, three times the oracle's own bf16-vs-float64 spread, written by
+   tests/golden/make_oracle_spread.py from the oracle alone, never below 1e-2 nats and 1e-3)
+   does it take the GPU's decision.  Tokens, exit depths, loops and row counts must then be
+   equal, and states, logits, entropies and halts lie within that loop's fixed tolerance.
+   The followed decisions whose own choice differed are counted and printed with margins.
 """
 import numpy as np
 import pytest
@@ -268,4 +270,20 @@ def test_step_parity_key_split_over_sixteen_ctas():
     case = Case("attn-probe", 1, 1040, 32, 2)
     case.prefill()
     print("16-way key split", _step_parity(case, 0.6, 0.5, 0))
+    case.handle.close()
+
+
+def test_head_dim_64_over_several_tiles():
+    """The tiny model (head_dim 64: one 64-wide half per head vector) against a 300-position
+    prefix, two sequences.  The causal prefill runs 5 query tiles of 2 x 300 packed rows (the
+    last ragged) over up to 3 key tiles, checked slot by slot against the oracle's prefill; the
+    step's 316 keys (3 tiles, the last ragged) are split over a 4-CTA cluster whose last rank
+    gets no keys, checked under both commit rules."""
+    case = Case("tiny", 2, 300, 16, 4)
+    case.prefill()
+    o = case.oracle("bf16")
+    o.prefill(case.prefix_ids)
+    _check_prefill_kv(case, o, range(2), _slots(case))
+    for rule in (0, 1):
+        print("head_dim 64, several tiles", rule, _step_parity(case, 0.6, 0.9, rule))
     case.handle.close()
