@@ -17,7 +17,6 @@
 #include <type_traits>
 #include <vector>
 
-#include "attention.cuh"
 #include "attention_pq.cuh"
 #include "attention_tc.cuh"
 #include "common.cuh"
@@ -118,8 +117,6 @@ void klaunch_cluster_x(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     cudaLaunchKernelEx(&cfg, kern, args...);
 }
 constexpr int PREFILL_ROWS = 16384;         // rows of one prefill group (sequences x P)
-constexpr size_t ATTN_WS_FLOATS = 16u << 20;    // split-KV partials (64 MB)
-constexpr int ATTN_COUNTERS = 16384;            // split-KV merge counters
 
 // KC_GEMM: linear layers on the pair and persistent kernels (many rows, tensor-bound);
 // KC_GEMM_TILE: linear layers on the per-tile split-K kernel (few rows, weight streaming)
@@ -280,13 +277,11 @@ bool init_kernel_attrs() {
     set_sk_attr<64, gemm::EPI_F32>();
     set_sk_attr<64, gemm::EPI_ADD>();
     set_sk_attr<64, gemm::EPI_SWIGLU>();
-    cudaFuncSetAttribute(attn::attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 5 * 64 * 64 * 2);
     cudaFuncSetAttribute(attn_tc::attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)attn_tc::smem_bytes<128>());
     cudaFuncSetAttribute(attn_tc::attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)attn_tc::smem_bytes<64>());
     cudaFuncSetAttribute(attn_pq::attn_pq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_pq::SMEM);
-    cudaFuncSetAttribute(attn::attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 5 * 64 * 128 * 2);
     done[dev] = cudaGetLastError() == cudaSuccess;
     if (done[dev]) {  // occupancies, looked up here (never during a graph capture)
         pair_slots<gemm::EPI_F32>();
@@ -578,7 +573,6 @@ struct alodlm {
     int n_slots = 0, pos_stride = 0;
     long long head_stride = 0, seq_stride = 0, slot_elems = 0;
     float2 *rope = nullptr;
-    bool tc_attn = false;            // tcgen05 attention (head_dim 64 or 128): steps, prefills, appends
     CUtensorMap tm_q, tm_kv_k, tm_kv_v;
 
     // prefill state
@@ -596,14 +590,12 @@ struct alodlm {
     int rows_cap = 0, step_rows_cap = 0;
     float *hbuf[2] = {nullptr, nullptr}, *hc = nullptr, *hexit = nullptr, *qkv = nullptr;
     bf16 *xn = nullptr, *qb = nullptr, *attn_out = nullptr, *act = nullptr;
-    float *aws_o = nullptr, *aws_ml = nullptr;  // split-KV partials of the mma.sync attention
     // folded RMSNorm: per-row partial sums of squares [rows_cap][ss_cap] (ss_cap = H / 16 rounded
     // up), and which layer's first norm the last residual add already prepared: layer fold_layer
     // over the M = fold_M rows of residual stream fold_x, with fold_n partials per row (-1: none)
     float *ss = nullptr;
     int ss_cap = 0, fold_layer = -1, fold_M = 0, fold_n = 0;
     const float *fold_x = nullptr;
-    int *attn_counters = nullptr;
     int norm_threads = 256;  // one float4 per thread per row where possible
     int num_sms = 148;
 
@@ -759,141 +751,95 @@ int linear(alodlm *h, const CUtensorMap &tmW, int Nw, const bf16 *actp, int M, i
 
 // attention of M rows (n_seq sequences x rows_per_seq) against slot `slot`, keys [0, kv_len)
 int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_len, int causal) {
-    if (h->tc_attn) {
-        attn_tc::Params p{};
-        // keys before the rows' own: the step's cached prefix, or the positions an append extends
-        p.static_keys = std::max(0, kv_len - map.rows_per_seq);
-        p.causal = causal;
-        p.pos0 = map.pos0;
-        p.row_t = map.row_t;
-        p.seq_off = map.seq_off;
-        p.seq_cnt = map.seq_cnt;
-        p.G = h->nq / h->nkv;
-        p.RP = p.G * map.rows_per_seq;
-        p.nkv = h->nkv;
-        p.nq = h->nq;
-        p.Tq = map.rows_per_seq;
-        p.kv_len = kv_len;
-        p.slot = slot;
-        p.max_batch = h->cfg.max_batch;
-        p.pos_stride = h->pos_stride;
-        p.seq_of = map.seq_of;
-        p.out = h->attn_out;
-        p.out_ld = h->nq * h->hd;
-        p.m_rows = M;
-        p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)h->hd));
-        p.err = h->d_err;
-        const int qtiles = cdiv(p.RP, attn_tc::BQ);
-        const int base = qtiles * h->nkv * n_seq;
-        const int ktiles = cdiv(kv_len, attn_tc::BKV);
-        const double bytes = 4.0 * n_seq * h->nkv * (double)kv_len * h->hd + 4.0 * M * h->nq * h->hd;
-        const double flops = 4.0 * M * h->nq * (double)kv_len * h->hd * (causal ? 0.5 : 1.0);
-        // two query tiles per CTA (K/V loaded once for both, softmax warpgroups in turn) where a
-        // (sequence, KV head) has two and the pairs still cover half the SMs without a key split
-        const int qpairs = cdiv(qtiles, 2);
-        if (h->hd == attn_tc::HD && !causal && !map.seq_cnt && ALODLM_ATTN_PQ && qtiles >= 2 &&
-            2 * qpairs * h->nkv * n_seq >= h->num_sms) {
-            p.n_splits = 1;
-            p.keys_per_split = ktiles * attn_tc::BKV;
-            LAUNCH(KC_ATTN, bytes, flops,
-                   klaunch(attn_pq::attn_pq_kernel, dim3(qpairs, h->nkv, n_seq), attn_pq::THREADS, attn_pq::SMEM,
-                           h->stream, h->tm_q, h->tm_kv_k, h->tm_kv_v, p));
-            return ALODLM_OK;
-        }
-        // splits of a query tile form one cluster (a power of two so that they share the 128
-        // rows evenly; 8 CTAs, or 16 where that many 16-CTA clusters fit at once): enough CTAs
-        // to cover the SMs, rounded up to the next power of two while the grid still fits in
-        // one wave, so that a latency-bound launch walks one key tile per CTA
-        // causal rows: no key split (each query tile walks keys [0, its last position]; a
-        // prefill's query tiles alone fill the SMs)
-        const int cap = (h->hd == 128 && ALODLM_ATTN_CLUSTER16 && attn_clusters16() >= base) ? 16 : 8;
-        const int want = causal ? 1 : std::max(1, std::min(std::min(ktiles, cdiv(h->num_sms, base)), cap));
-        int splits = 1;
-        while (splits < want) splits <<= 1;
-        if (splits > cap || (splits > 1 && (long long)splits * base > h->num_sms)) splits >>= 1;
-        int kps = cdiv(ktiles, splits);  // trailing ranks may get no keys (empty partials)
-        // a remainder shorter than a key tile rides on the last rank when that saves every other
-        // rank a tile: e.g. 8 full tiles + 32 keys over 8 ranks -> one tile each, the last two
-        const int full = kv_len / attn_tc::BKV, kps_full = std::max(1, cdiv(full, splits));
-        p.last_to_end = 0;
-        if (splits > 1 && kps_full < kps && (long long)splits * kps_full * attn_tc::BKV >= (long long)full * attn_tc::BKV &&
-            kv_len - (long long)splits * kps_full * attn_tc::BKV < attn_tc::BKV) {
-            kps = kps_full;
-            p.last_to_end = 1;
-        }
-        p.n_splits = splits;
-        p.keys_per_split = kps * attn_tc::BKV;
-        // one instance per head_dim (one or two 64-wide halves per head vector)
-        auto *const kern = h->hd == 128 ? attn_tc::attn_tc_kernel<128> : attn_tc::attn_tc_kernel<64>;
-        const size_t smem = h->hd == 128 ? attn_tc::smem_bytes<128>() : attn_tc::smem_bytes<64>();
-        if (splits > 1) {
-            // cluster along y: the `splits` consecutive y indices of one kv head
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3(qtiles, h->nkv * splits, n_seq);
-            cfg.blockDim = dim3(192);
-            cfg.dynamicSmemBytes = smem;
-            cfg.stream = h->stream;
-            cudaLaunchAttribute attr[2];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = 1;
-            attr[0].val.clusterDim.y = splits;
-            attr[0].val.clusterDim.z = 1;
-            attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-            attr[1].val.programmaticStreamSerializationAllowed = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = ALODLM_PDL ? 2 : 1;
-            LAUNCH(KC_ATTN, bytes, flops,
-                   cudaLaunchKernelEx(&cfg, kern, h->tm_q, h->tm_kv_k, h->tm_kv_v, p));
-        } else {
-            LAUNCH(KC_ATTN, bytes, flops,
-                   klaunch(kern, dim3(qtiles, h->nkv, n_seq), 192, smem, h->stream, h->tm_q, h->tm_kv_k, h->tm_kv_v,
-                           p));
-        }
-        return ALODLM_OK;
-    }
-    attn::Params p{};
-    p.q = h->qb;
-    p.q_ld = h->nq * h->hd;
-    p.kc = h->kv_k + (long long)slot * h->slot_elems;
-    p.vc = h->kv_v + (long long)slot * h->slot_elems;
-    p.seq_stride = h->seq_stride;
-    p.head_stride = h->head_stride;
-    p.map = map;
-    p.G = h->nq / h->nkv;
-    p.nq = h->nq;
-    p.kv_len = kv_len;
+    attn_tc::Params p{};
+    // keys before the rows' own: the step's cached prefix, or the positions an append extends
+    p.static_keys = std::max(0, kv_len - map.rows_per_seq);
     p.causal = causal;
+    p.pos0 = map.pos0;
+    p.row_t = map.row_t;
+    p.seq_off = map.seq_off;
+    p.seq_cnt = map.seq_cnt;
+    p.G = h->nq / h->nkv;
+    p.RP = p.G * map.rows_per_seq;
+    p.nkv = h->nkv;
+    p.nq = h->nq;
+    p.Tq = map.rows_per_seq;
+    p.kv_len = kv_len;
+    p.slot = slot;
+    p.max_batch = h->cfg.max_batch;
+    p.pos_stride = h->pos_stride;
+    p.seq_of = map.seq_of;
     p.out = h->attn_out;
     p.out_ld = h->nq * h->hd;
-    p.ws_o = h->aws_o;
-    p.ws_ml = h->aws_ml;
-    p.counters = h->attn_counters;
     p.m_rows = M;
     p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)h->hd));
-    const int Tq = map.rows_per_seq;
-    const int qtiles = cdiv(p.G * Tq, 64);
+    p.err = h->d_err;
+    const int qtiles = cdiv(p.RP, attn_tc::BQ);
     const int base = qtiles * h->nkv * n_seq;
-    const int ktiles = cdiv(kv_len, 64);
-    int splits = 1;
-    if (!causal) {
-        // enough CTAs to cover the SMs, but at least 4 key tiles per split
-        splits = std::max(1, std::min(ktiles / 4, cdiv(h->num_sms, base)));
-        while (splits > 1 && ((size_t)splits * M * h->nq * (h->hd + 2) > ATTN_WS_FLOATS ||
-                              (size_t)base > ATTN_COUNTERS))
-            --splits;
-    }
-    const int kps_tiles = cdiv(ktiles, splits);
-    splits = cdiv(ktiles, kps_tiles);
-    p.n_splits = splits;
-    p.keys_per_split = kps_tiles * 64;
-    dim3 grid(qtiles, h->nkv * splits, n_seq);
-    const double kvb = 4.0 * n_seq * h->nkv * (double)kv_len * h->hd;
-    const double bytes = kvb + 4.0 * M * h->nq * h->hd;
+    const int ktiles = cdiv(kv_len, attn_tc::BKV);
+    const double bytes = 4.0 * n_seq * h->nkv * (double)kv_len * h->hd + 4.0 * M * h->nq * h->hd;
     const double flops = 4.0 * M * h->nq * (double)kv_len * h->hd * (causal ? 0.5 : 1.0);
-    if (h->hd == 128)
-        LAUNCH(KC_ATTN, bytes, flops, (klaunch(attn::attn_kernel<128>, grid, 128, 5 * 64 * 128 * 2, h->stream, p)));
-    else
-        LAUNCH(KC_ATTN, bytes, flops, (klaunch(attn::attn_kernel<64>, grid, 128, 5 * 64 * 64 * 2, h->stream, p)));
+    // two query tiles per CTA (K/V loaded once for both, softmax warpgroups in turn) where a
+    // (sequence, KV head) has two and the pairs still cover half the SMs without a key split
+    const int qpairs = cdiv(qtiles, 2);
+    if (h->hd == attn_tc::HD && !causal && !map.seq_cnt && ALODLM_ATTN_PQ && qtiles >= 2 &&
+        2 * qpairs * h->nkv * n_seq >= h->num_sms) {
+        p.n_splits = 1;
+        p.keys_per_split = ktiles * attn_tc::BKV;
+        LAUNCH(KC_ATTN, bytes, flops,
+               klaunch(attn_pq::attn_pq_kernel, dim3(qpairs, h->nkv, n_seq), attn_pq::THREADS, attn_pq::SMEM,
+                       h->stream, h->tm_q, h->tm_kv_k, h->tm_kv_v, p));
+        return ALODLM_OK;
+    }
+    // splits of a query tile form one cluster (a power of two so that they share the 128
+    // rows evenly; 8 CTAs, or 16 where that many 16-CTA clusters fit at once): enough CTAs
+    // to cover the SMs, rounded up to the next power of two while the grid still fits in
+    // one wave, so that a latency-bound launch walks one key tile per CTA
+    // causal rows: no key split (each query tile walks keys [0, its last position]; a
+    // prefill's query tiles alone fill the SMs)
+    const int cap = (h->hd == 128 && ALODLM_ATTN_CLUSTER16 && attn_clusters16() >= base) ? 16 : 8;
+    const int want = causal ? 1 : std::max(1, std::min(std::min(ktiles, cdiv(h->num_sms, base)), cap));
+    int splits = 1;
+    while (splits < want) splits <<= 1;
+    if (splits > cap || (splits > 1 && (long long)splits * base > h->num_sms)) splits >>= 1;
+    int kps = cdiv(ktiles, splits);  // trailing ranks may get no keys (empty partials)
+    // a remainder shorter than a key tile rides on the last rank when that saves every other
+    // rank a tile: e.g. 8 full tiles + 32 keys over 8 ranks -> one tile each, the last two
+    const int full = kv_len / attn_tc::BKV, kps_full = std::max(1, cdiv(full, splits));
+    p.last_to_end = 0;
+    if (splits > 1 && kps_full < kps && (long long)splits * kps_full * attn_tc::BKV >= (long long)full * attn_tc::BKV &&
+        kv_len - (long long)splits * kps_full * attn_tc::BKV < attn_tc::BKV) {
+        kps = kps_full;
+        p.last_to_end = 1;
+    }
+    p.n_splits = splits;
+    p.keys_per_split = kps * attn_tc::BKV;
+    // one instance per head_dim (one or two 64-wide halves per head vector)
+    auto *const kern = h->hd == 128 ? attn_tc::attn_tc_kernel<128> : attn_tc::attn_tc_kernel<64>;
+    const size_t smem = h->hd == 128 ? attn_tc::smem_bytes<128>() : attn_tc::smem_bytes<64>();
+    if (splits > 1) {
+        // cluster along y: the `splits` consecutive y indices of one kv head
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(qtiles, h->nkv * splits, n_seq);
+        cfg.blockDim = dim3(192);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = h->stream;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 1;
+        attr[0].val.clusterDim.y = splits;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = ALODLM_PDL ? 2 : 1;
+        LAUNCH(KC_ATTN, bytes, flops,
+               cudaLaunchKernelEx(&cfg, kern, h->tm_q, h->tm_kv_k, h->tm_kv_v, p));
+    } else {
+        LAUNCH(KC_ATTN, bytes, flops,
+               klaunch(kern, dim3(qtiles, h->nkv, n_seq), 192, smem, h->stream, h->tm_q, h->tm_kv_k, h->tm_kv_v,
+                       p));
+    }
     return ALODLM_OK;
 }
 
@@ -1223,12 +1169,10 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
         (rc = dalloc(h, &h->hc, R * H)) || (rc = dalloc(h, &h->hexit, R * H)) ||
         (rc = dalloc(h, &h->qkv, R * h->n_qkv)) || (rc = dalloc(h, &h->xn, R * H)) ||
         (rc = dalloc(h, &h->qb, R * qd)) || (rc = dalloc(h, &h->attn_out, R * qd)) ||
-        (rc = dalloc(h, &h->act, R * h->I)) || (rc = dalloc(h, &h->aws_o, ATTN_WS_FLOATS)) ||
-        (rc = dalloc(h, &h->aws_ml, ATTN_WS_FLOATS / 16)) || (rc = dalloc(h, &h->attn_counters, ATTN_COUNTERS)))
+        (rc = dalloc(h, &h->act, R * h->I)))
         return cleanup(rc);
     h->ss_cap = cdiv(H, 16);
     if ((rc = dalloc(h, &h->ss, R * h->ss_cap))) return cleanup(rc);
-    cudaMemsetAsync(h->attn_counters, 0, ATTN_COUNTERS * sizeof(int), h->stream);
     // zero the activation buffers once so rows past the live ones never hold NaN patterns
     cudaMemsetAsync(h->xn, 0, R * H * 2, h->stream);
     cudaMemsetAsync(h->attn_out, 0, R * qd * 2, h->stream);
@@ -1238,13 +1182,18 @@ int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *w, void *stream, 
     cudaMemsetAsync(h->kv_k, 0, (size_t)h->slot_elems * h->n_slots * 2, h->stream);
     cudaMemsetAsync(h->kv_v, 0, (size_t)h->slot_elems * h->n_slots * 2, h->stream);
     {
+        // the attention's tensor maps address head vectors by 32-bit row coordinates
         const long long arena_rows = (long long)h->n_slots * cfg->max_batch * h->nkv * h->pos_stride;
-        h->tc_attn = (h->hd == 128 || h->hd == 64) && arena_rows + 256 < (1ll << 31) &&
-                     (long long)R * h->nq < (1ll << 31);
-        if (h->tc_attn)
-            h->tc_attn = make_tmap(&h->tm_q, h->qb, h->hd, (int)(R * h->nq), attn_tc::BQ) &&
-                         make_tmap(&h->tm_kv_k, h->kv_k, h->hd, (int)arena_rows, attn_tc::BKV) &&
-                         make_tmap(&h->tm_kv_v, h->kv_v, h->hd, (int)arena_rows, attn_tc::BKV);
+        if (arena_rows + 256 >= (1ll << 31) || (long long)R * h->nq >= (1ll << 31)) {
+            h->err = "KV arena or query rows beyond 2^31 head vectors";
+            return cleanup(ALODLM_EINVAL);
+        }
+        if (!make_tmap(&h->tm_q, h->qb, h->hd, (int)(R * h->nq), attn_tc::BQ) ||
+            !make_tmap(&h->tm_kv_k, h->kv_k, h->hd, (int)arena_rows, attn_tc::BKV) ||
+            !make_tmap(&h->tm_kv_v, h->kv_v, h->hd, (int)arena_rows, attn_tc::BKV)) {
+            h->err = "cuTensorMapEncodeTiled failed (attention)";
+            return cleanup(ALODLM_ECUDA);
+        }
     }
 
     h->R_cap = round_up(h->step_rows_cap, 128);
@@ -1410,13 +1359,11 @@ int alodlm_sync(alodlm_t *h) {
     e = cudaMemcpy(&dev_err, h->d_err, sizeof(int), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(h, e, "sync: read error word");
     if (dev_err) {
-        // A kernel that gave up may have left a split's arrival counter part-way (its epilogue
-        // skipped the increment): re-arm the counters, so that the next launch does not take a
-        // CTA for the last arriver too early.
-        cudaMemsetAsync(h->attn_counters, 0, ATTN_COUNTERS * sizeof(int), h->stream);
+        // no kernel of a step keeps state across launches that a kernel giving up could leave
+        // part-way (cluster merges only): clearing the error word re-arms the handle
         cudaMemsetAsync(h->d_err, 0, sizeof(int), h->stream);
         e = cudaStreamSynchronize(h->stream);
-        if (e != cudaSuccess) return cuda_fail(h, e, "sync: re-arm counters");
+        if (e != cudaSuccess) return cuda_fail(h, e, "sync: clear the error word");
         if (dev_err & DEVERR_TIMEOUT) return fail(h, ALODLM_ETIMEOUT, "a bounded device wait timed out");
         return fail(h, ALODLM_EDEVICE, "a kernel flagged an out-of-range value (token id or exit depth)");
     }

@@ -111,8 +111,9 @@ typedef struct {
  * Allocates the depth-aware KV arena: (n_prelude + k_max*n_core + n_coda) slots of
  * max_batch x n_kv_heads x (max_prefix + max_block) x head_dim, K and V, bf16.
  * stream: a cudaStream_t (NULL = legacy default stream).
- * Errors: EINVAL (shape/null), ENOMEM, ECUDA.  On error *out is NULL and the text is in
- * alodlm_last_error(NULL). */
+ * Errors: EINVAL (shape/null, or a KV arena of 2^31 head vectors or more, which the
+ * attention's 32-bit tensor-map coordinates cannot address), ENOMEM, ECUDA.  On error *out is
+ * NULL and the text is in alodlm_last_error(NULL). */
 ALODLM_API int alodlm_create(const alodlm_cfg *cfg, const alodlm_weights *weights, void *stream, alodlm_t **out);
 
 /* Build the depth-aware KV cache of the prefix.
@@ -222,8 +223,9 @@ ALODLM_API int alodlm_sync(alodlm_t *h);
 /* Test hook for the error path (no counterpart in the paper): enqueue on the handle's stream a
  * kernel whose one bounded wait (on an mbarrier nothing arrives on) expires after the library's
  * wait limit (about 2 s), raising the device error word exactly as a timed-out wait inside a
- * step would.  The next alodlm_sync then returns ETIMEOUT and re-arms the handle's counters;
- * the handle stays usable.  No GPU fault is involved.  Errors: EINVAL (null handle), ECUDA. */
+ * step would.  The next alodlm_sync then returns ETIMEOUT and clears the word; the handle
+ * stays usable (no step kernel keeps state across launches that an expired wait could leave
+ * part-way).  No GPU fault is involved.  Errors: EINVAL (null handle), ECUDA. */
 ALODLM_API int alodlm_inject_wait_timeout(alodlm_t *h);
 
 /* Free everything the handle owns (synchronises first).  NULL is a no-op. */

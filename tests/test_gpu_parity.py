@@ -218,7 +218,7 @@ def test_state_and_argument_errors():
 def test_expired_wait_reports_timeout_and_the_next_step_is_unchanged(mid):
     """The error path of every bounded device wait, without a GPU fault: a probe kernel waits on
     an mbarrier that nothing arrives on until the library's wait limit expires.  sync() reports
-    ALODLM_ETIMEOUT, re-arms the handle's counters and clears the error word; the next step on
+    ALODLM_ETIMEOUT and clears the error word; the next step on
     the same handle is bit-identical to the one before the timeout and matches the oracle."""
     import time
     import adaptively_looped_masked_b200 as alo
