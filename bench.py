@@ -544,18 +544,23 @@ def run_ours(args, world, rank, local):
 
     if world == 1 and not args.no_extras:
         # the pages' sweep: tau x lambda on the same workload, active-row fraction per loop
+        # (an extra that fails is recorded in the line; the headline above stands)
         sweep = []
-        for t_ in wl.taus:
-            for l_ in wl.lambdas:
-                rs = measure_step(handle, m, wl, block_np, t_, l_, rule, 5, 3, world, local, peaks, stream,
-                                  classes=False, e2e=False, clocks=False)
-                ms_s = rs["ms"] / 5
-                BN = wl.batch * wl.block
-                sweep.append({"tau_H": t_, "lambda": l_, "value": rs["commits"] / (ms_s / 1e3), "ms_per_step": ms_s,
-                              "committed_per_step": rs["commits"], "mean_loops": float(np.mean(rs["loops"])),
-                              "active_row_fraction": [round(x / BN, 4) for x in rs["active_rows"]],
-                              "readout_row_fraction": [round(x / BN, 4) for x in rs["readout_rows"]],
-                              "step_roofline_frac": rs["t_roof"] * 1e3 / ms_s})
+        try:
+            for t_ in wl.taus:
+                for l_ in wl.lambdas:
+                    rs = measure_step(handle, m, wl, block_np, t_, l_, rule, 5, 3, world, local, peaks, stream,
+                                      classes=False, e2e=False, clocks=False)
+                    ms_s = rs["ms"] / 5
+                    BN = wl.batch * wl.block
+                    sweep.append({"tau_H": t_, "lambda": l_, "value": rs["commits"] / (ms_s / 1e3),
+                                  "ms_per_step": ms_s, "committed_per_step": rs["commits"],
+                                  "mean_loops": float(np.mean(rs["loops"])),
+                                  "active_row_fraction": [round(x / BN, 4) for x in rs["active_rows"]],
+                                  "readout_row_fraction": [round(x / BN, 4) for x in rs["readout_rows"]],
+                                  "step_roofline_frac": rs["t_roof"] * 1e3 / ms_s})
+        except Exception as exc:  # noqa: BLE001
+            sweep.append({"error": f"{type(exc).__name__}: {exc}"[:300]})
         line["sweep"] = sweep
     handle.close()
     del handle
@@ -568,16 +573,21 @@ def run_ours(args, world, rank, local):
         for name in [n for n in ("qwen3-8b-bs1", "qwen3-1.7b-bs1", "qwen3-8b-long") if n != args.workload]:
             wl2 = WORKLOADS[name]
             m2 = MODELS[wl2.model]
-            w2 = w if wl2.model == wl.model else make_weights(m2, seed=0, device="cuda")
-            h2, p2 = make_handle(alo, m2, wl2, w2, stream, rank)
-            r2 = measure_step(h2, m2, wl2, make_block_ids(m2, wl2.batch, wl2.block), tau,
-                              wl2.lambdas[-1] if wl2.mixed_exit_depths else lam, rule, args.steps, args.warmup,
-                              world, local, peaks, stream)
-            secondary[name] = step_summary(name, wl2, r2, args.steps, world)
-            secondary[name]["prefill_s"] = p2
-            if name == "qwen3-1.7b-bs1" and rank == 0 and not args.no_cpu_baseline:
+            h2 = None
+            try:
+                w2 = w if wl2.model == wl.model else make_weights(m2, seed=0, device="cuda")
+                h2, p2 = make_handle(alo, m2, wl2, w2, stream, rank)
+                r2 = measure_step(h2, m2, wl2, make_block_ids(m2, wl2.batch, wl2.block), tau,
+                                  wl2.lambdas[-1] if wl2.mixed_exit_depths else lam, rule, args.steps, args.warmup,
+                                  world, local, peaks, stream)
+                secondary[name] = step_summary(name, wl2, r2, args.steps, world)
+                secondary[name]["prefill_s"] = p2
+            except Exception as exc:  # noqa: BLE001
+                secondary[name] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+            if h2 is not None and name == "qwen3-1.7b-bs1" and rank == 0 and not args.no_cpu_baseline \
+                    and "error" not in secondary[name]:
                 handle_17, w_17 = h2, w2
-            else:
+            elif h2 is not None:
                 h2.close()
             torch.cuda.empty_cache()
         line["secondary"] = secondary
