@@ -100,13 +100,47 @@ def lib() -> ctypes.CDLL:
         L.alodlm_kernel_class_name.restype = ctypes.c_char_p
         L.alodlm_gemm_bf16.argtypes = [vp, vp, vp, ci, ci, ci, vp, csz, vp]
         L.alodlm_gemm_bf16_noalloc.argtypes = [vp, vp, vp, ci, ci, ci, vp, vp]
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        L.alodlm_plan_gemm.argtypes = [ci, ci, ci, i32p]
+        L.alodlm_plan_gemm_noalloc.argtypes = [ci, ci, ci, ci, i32p]
+        L.alodlm_plan_attention.argtypes = [ci, ci, ci, ci, ci, ci, ci, ci, i32p]
         for f in ("alodlm_create", "alodlm_prefill", "alodlm_append", "alodlm_denoise_step",
                   "alodlm_denoise_step_sampled", "alodlm_decode_block_sampled", "alodlm_decode_block", "alodlm_sync", "alodlm_debug_state",
                   "alodlm_kv_slot", "alodlm_step_stats", "alodlm_set_timing", "alodlm_set_graphs",
-                  "alodlm_gemm_bf16", "alodlm_gemm_bf16_noalloc"):
+                  "alodlm_gemm_bf16", "alodlm_gemm_bf16_noalloc", "alodlm_plan_gemm", "alodlm_plan_gemm_noalloc",
+                  "alodlm_plan_attention"):
             getattr(L, f).restype = ci
         _lib = L
     return _lib
+
+
+def _plan(fn: str, n_out: int, *args) -> tuple:
+    out = (ctypes.c_int32 * n_out)()
+    rc = getattr(lib(), fn)(*args, out)
+    if rc != 0:
+        raise AlodlmError(rc, lib().alodlm_last_error(None).decode())
+    return tuple(out)
+
+
+def plan_gemm(M: int, N: int, K: int) -> dict:
+    """The per-tile linear-layer kernel's partition (alodlm_plan_gemm); no device work."""
+    bn, splits, kps, k_tiles = _plan("alodlm_plan_gemm", 4, M, N, K)
+    return dict(bn=bn, splits=splits, kps=kps, k_tiles=k_tiles)
+
+
+def plan_gemm_noalloc(M: int, N: int, K: int, num_sms: int) -> dict:
+    """The allocation-free GEMM's stream-K partition (alodlm_plan_gemm_noalloc); no device work."""
+    bn, grid, upc, max_seg, n_tiles, k_tiles = _plan("alodlm_plan_gemm_noalloc", 6, M, N, K, num_sms)
+    return dict(bn=bn, grid=grid, upc=upc, max_seg=max_seg, n_tiles=n_tiles, k_tiles=k_tiles)
+
+
+def plan_attention(packed_rows: int, n_kv_heads: int, n_seq: int, kv_len: int, causal: bool, num_sms: int,
+                   two_tile_ok: bool, cluster16_ok: bool) -> dict:
+    """One attention launch's partition (alodlm_plan_attention); no device work."""
+    qtiles, two_tile, splits, kps, last_to_end = _plan("alodlm_plan_attention", 5, packed_rows, n_kv_heads, n_seq,
+                                                       kv_len, int(causal), num_sms, int(two_tile_ok),
+                                                       int(cluster16_ok))
+    return dict(qtiles=qtiles, two_tile=two_tile, splits=splits, keys_per_split=kps, last_to_end=last_to_end)
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:

@@ -749,6 +749,56 @@ int linear(alodlm *h, const CUtensorMap &tmW, int Nw, const bf16 *actp, int M, i
     return ALODLM_OK;
 }
 
+// Work partition of one attention launch: RP packed query rows per (sequence, KV head), n_seq
+// sequences, keys [0, kv_len).  pq_ok: the two-tile kernel may serve this launch (head_dim 128,
+// unmasked rows without row tables); cap16: 16-CTA clusters fit for the one-tile grid.
+struct AttnPlan {
+    int qtiles;          // 128-row query tiles per (sequence, KV head)
+    int two_tile;        // 1: the two-tile kernel, ceil(qtiles / 2) CTAs per (sequence, KV head)
+    int splits;          // key splits per query tile (one cluster); a power of two
+    int keys_per_split;  // a multiple of the 128-key tile
+    int last_to_end;     // the last split also takes the keys past splits * keys_per_split
+};
+
+AttnPlan plan_attention(int RP, int nkv, int n_seq, int kv_len, int causal, int num_sms, int pq_ok, int cap16) {
+    AttnPlan a{};
+    a.qtiles = cdiv(RP, attn_tc::BQ);
+    const int base = a.qtiles * nkv * n_seq;
+    const int ktiles = cdiv(kv_len, attn_tc::BKV);
+    // two query tiles per CTA (K/V loaded once for both, softmax warpgroups in turn) where a
+    // (sequence, KV head) has two and the pairs still cover half the SMs without a key split
+    const int qpairs = cdiv(a.qtiles, 2);
+    if (pq_ok && !causal && ALODLM_ATTN_PQ && a.qtiles >= 2 && 2 * qpairs * nkv * n_seq >= num_sms) {
+        a.two_tile = 1;
+        a.splits = 1;
+        a.keys_per_split = ktiles * attn_tc::BKV;
+        return a;
+    }
+    // splits of a query tile form one cluster (a power of two so that they share the 128
+    // rows evenly; 8 CTAs, or 16 where that many 16-CTA clusters fit at once): enough CTAs
+    // to cover the SMs, rounded up to the next power of two while the grid still fits in
+    // one wave, so that a latency-bound launch walks one key tile per CTA
+    // causal rows: no key split (each query tile walks keys [0, its last position]; a
+    // prefill's query tiles alone fill the SMs)
+    const int cap = cap16 ? 16 : 8;
+    const int want = causal ? 1 : std::max(1, std::min(std::min(ktiles, cdiv(num_sms, base)), cap));
+    int splits = 1;
+    while (splits < want) splits <<= 1;
+    if (splits > cap || (splits > 1 && (long long)splits * base > num_sms)) splits >>= 1;
+    int kps = cdiv(ktiles, splits);  // trailing ranks may get no keys (empty partials)
+    // a remainder shorter than a key tile rides on the last rank when that saves every other
+    // rank a tile: e.g. 8 full tiles + 32 keys over 8 ranks -> one tile each, the last two
+    const int full = kv_len / attn_tc::BKV, kps_full = std::max(1, cdiv(full, splits));
+    if (splits > 1 && kps_full < kps && (long long)splits * kps_full * attn_tc::BKV >= (long long)full * attn_tc::BKV &&
+        kv_len - (long long)splits * kps_full * attn_tc::BKV < attn_tc::BKV) {
+        kps = kps_full;
+        a.last_to_end = 1;
+    }
+    a.splits = splits;
+    a.keys_per_split = kps * attn_tc::BKV;
+    return a;
+}
+
 // attention of M rows (n_seq sequences x rows_per_seq) against slot `slot`, keys [0, kv_len)
 int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_len, int causal) {
     attn_tc::Params p{};
@@ -776,44 +826,21 @@ int attention(alodlm *h, int slot, int M, const RowMap &map, int n_seq, int kv_l
     p.err = h->d_err;
     const int qtiles = cdiv(p.RP, attn_tc::BQ);
     const int base = qtiles * h->nkv * n_seq;
-    const int ktiles = cdiv(kv_len, attn_tc::BKV);
     const double bytes = 4.0 * n_seq * h->nkv * (double)kv_len * h->hd + 4.0 * M * h->nq * h->hd;
     const double flops = 4.0 * M * h->nq * (double)kv_len * h->hd * (causal ? 0.5 : 1.0);
-    // two query tiles per CTA (K/V loaded once for both, softmax warpgroups in turn) where a
-    // (sequence, KV head) has two and the pairs still cover half the SMs without a key split
-    const int qpairs = cdiv(qtiles, 2);
-    if (h->hd == attn_tc::HD && !causal && !map.seq_cnt && ALODLM_ATTN_PQ && qtiles >= 2 &&
-        2 * qpairs * h->nkv * n_seq >= h->num_sms) {
-        p.n_splits = 1;
-        p.keys_per_split = ktiles * attn_tc::BKV;
+    const AttnPlan plan =
+        plan_attention(p.RP, h->nkv, n_seq, kv_len, causal, h->num_sms, h->hd == attn_tc::HD && !map.seq_cnt,
+                       h->hd == 128 && ALODLM_ATTN_CLUSTER16 && attn_clusters16() >= base);
+    p.n_splits = plan.splits;
+    p.keys_per_split = plan.keys_per_split;
+    p.last_to_end = plan.last_to_end;
+    if (plan.two_tile) {
         LAUNCH(KC_ATTN, bytes, flops,
-               klaunch(attn_pq::attn_pq_kernel, dim3(qpairs, h->nkv, n_seq), attn_pq::THREADS, attn_pq::SMEM,
-                       h->stream, h->tm_q, h->tm_kv_k, h->tm_kv_v, p));
+               klaunch(attn_pq::attn_pq_kernel, dim3(cdiv(qtiles, 2), h->nkv, n_seq), attn_pq::THREADS,
+                       attn_pq::SMEM, h->stream, h->tm_q, h->tm_kv_k, h->tm_kv_v, p));
         return ALODLM_OK;
     }
-    // splits of a query tile form one cluster (a power of two so that they share the 128
-    // rows evenly; 8 CTAs, or 16 where that many 16-CTA clusters fit at once): enough CTAs
-    // to cover the SMs, rounded up to the next power of two while the grid still fits in
-    // one wave, so that a latency-bound launch walks one key tile per CTA
-    // causal rows: no key split (each query tile walks keys [0, its last position]; a
-    // prefill's query tiles alone fill the SMs)
-    const int cap = (h->hd == 128 && ALODLM_ATTN_CLUSTER16 && attn_clusters16() >= base) ? 16 : 8;
-    const int want = causal ? 1 : std::max(1, std::min(std::min(ktiles, cdiv(h->num_sms, base)), cap));
-    int splits = 1;
-    while (splits < want) splits <<= 1;
-    if (splits > cap || (splits > 1 && (long long)splits * base > h->num_sms)) splits >>= 1;
-    int kps = cdiv(ktiles, splits);  // trailing ranks may get no keys (empty partials)
-    // a remainder shorter than a key tile rides on the last rank when that saves every other
-    // rank a tile: e.g. 8 full tiles + 32 keys over 8 ranks -> one tile each, the last two
-    const int full = kv_len / attn_tc::BKV, kps_full = std::max(1, cdiv(full, splits));
-    p.last_to_end = 0;
-    if (splits > 1 && kps_full < kps && (long long)splits * kps_full * attn_tc::BKV >= (long long)full * attn_tc::BKV &&
-        kv_len - (long long)splits * kps_full * attn_tc::BKV < attn_tc::BKV) {
-        kps = kps_full;
-        p.last_to_end = 1;
-    }
-    p.n_splits = splits;
-    p.keys_per_split = kps * attn_tc::BKV;
+    const int splits = plan.splits;
     // one instance per head_dim (one or two 64-wide halves per head vector)
     auto *const kern = h->hd == 128 ? attn_tc::attn_tc_kernel<128> : attn_tc::attn_tc_kernel<64>;
     const size_t smem = h->hd == 128 ? attn_tc::smem_bytes<128>() : attn_tc::smem_bytes<64>();
@@ -1349,6 +1376,42 @@ int alodlm_inject_wait_timeout(alodlm_t *h) {
     k::wait_expiry_kernel<<<1, 32, 0, h->stream>>>(h->d_err);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? ALODLM_OK : cuda_fail(h, e, "wait_expiry_kernel");
+}
+
+int alodlm_plan_gemm(int M, int N, int K, int32_t *out) {
+    if (!out || M < 1 || N < 1 || K < 1) return fail(nullptr, ALODLM_EINVAL, "plan_gemm: bad argument");
+    const GemmShape g = plan_gemm(M, N, K);
+    out[0] = g.bn;
+    out[1] = g.splits;
+    out[2] = g.kps;
+    out[3] = g.k_tiles;
+    return ALODLM_OK;
+}
+
+int alodlm_plan_gemm_noalloc(int M, int N, int K, int num_sms, int32_t *out) {
+    if (!out || M < 1 || M > 64 || N < 1 || K < 1 || num_sms < 1)
+        return fail(nullptr, ALODLM_EINVAL, "plan_gemm_noalloc: bad argument");
+    const SkPlan p = plan_sk(M, N, K, num_sms);
+    out[0] = p.bn;
+    out[1] = p.grid;
+    out[2] = p.upc;
+    out[3] = p.max_seg;
+    out[4] = p.n_tiles;
+    out[5] = p.k_tiles;
+    return ALODLM_OK;
+}
+
+int alodlm_plan_attention(int packed_rows, int n_kv_heads, int n_seq, int kv_len, int causal, int num_sms,
+                          int two_tile_ok, int cluster16_ok, int32_t *out) {
+    if (!out || packed_rows < 1 || n_kv_heads < 1 || n_seq < 1 || kv_len < 1 || num_sms < 1)
+        return fail(nullptr, ALODLM_EINVAL, "plan_attention: bad argument");
+    const AttnPlan a = plan_attention(packed_rows, n_kv_heads, n_seq, kv_len, causal, num_sms, two_tile_ok, cluster16_ok);
+    out[0] = a.qtiles;
+    out[1] = a.two_tile;
+    out[2] = a.splits;
+    out[3] = a.keys_per_split;
+    out[4] = a.last_to_end;
+    return ALODLM_OK;
 }
 
 int alodlm_sync(alodlm_t *h) {

@@ -228,6 +228,32 @@ ALODLM_API int alodlm_sync(alodlm_t *h);
  * part-way).  No GPU fault is involved.  Errors: EINVAL (null handle), ECUDA. */
 ALODLM_API int alodlm_inject_wait_timeout(alodlm_t *h);
 
+/* Work partitions of the kernels' launches, for host-side tests (no counterpart in the paper:
+ * they state how the library cuts a GEMM or an attention launch into CTAs).  Pure functions:
+ * no handle, no device work, callable without a GPU.  `out` is a caller-owned int32 array.
+ * Errors: EINVAL on a null `out` or a size below 1 (text in alodlm_last_error(NULL)).
+ *
+ * alodlm_plan_gemm: the per-tile linear-layer kernel for out[M, N] = act[M, K] W[N, K]^T:
+ * out[0] activation rows per tile (32/64/128/256), out[1] split-K ranks per tile (one cluster,
+ * a power of two), out[2] 64-wide k-tiles per rank, out[3] k-tiles in all (4 ints). */
+ALODLM_API int alodlm_plan_gemm(int M, int N, int K, int32_t *out);
+
+/* alodlm_plan_gemm_noalloc: the stream-K partition of alodlm_gemm_bf16_noalloc (M <= 64) on
+ * num_sms SMs: out[0] activation rows per tile, out[1] CTAs, out[2] (weight tile, k-tile) units
+ * per CTA, out[3] the most CTAs that share one weight tile (split partials kept per tile),
+ * out[4] 128-row weight tiles, out[5] k-tiles per weight tile (6 ints). */
+ALODLM_API int alodlm_plan_gemm_noalloc(int M, int N, int K, int num_sms, int32_t *out);
+
+/* alodlm_plan_attention: one attention launch over packed_rows (= query heads per KV head x
+ * rows per sequence) query rows per (sequence, KV head), keys [0, kv_len); causal rows, the
+ * SM count, whether the two-query-tile kernel may serve it (head_dim 128, rows without row
+ * tables) and whether 16-CTA clusters fit: out[0] 128-row query tiles, out[1] 1 if two query
+ * tiles share a CTA, out[2] key splits per query tile (one cluster, a power of two), out[3]
+ * keys per split (a multiple of 128), out[4] 1 if the last split also takes the keys past
+ * out[2] x out[3] (5 ints). */
+ALODLM_API int alodlm_plan_attention(int packed_rows, int n_kv_heads, int n_seq, int kv_len, int causal, int num_sms,
+                                     int two_tile_ok, int cluster16_ok, int32_t *out);
+
 /* Free everything the handle owns (synchronises first).  NULL is a no-op. */
 ALODLM_API void alodlm_destroy(alodlm_t *h);
 
