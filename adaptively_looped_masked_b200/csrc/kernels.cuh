@@ -322,7 +322,6 @@ __global__ void kv_fallback_kernel(const int *exit_depth, int n, int pos0, int b
     }
 }
 
-// Raise DEVERR_BOUNDS if any of v[0, n) lies outside [lo, hi]
 // Error-path probe: one thread waits, bounded, on an mbarrier that nothing ever arrives on, so
 // the wait expires and the device error word records a timeout -- the path every bounded wait
 // of the library takes, exercised without a GPU fault (no trap, no endless loop).
@@ -333,12 +332,6 @@ __global__ void wait_expiry_kernel(int *err) {
         fence_mbarrier_init();
         mbar_wait(&bar, 0, err);
     }
-}
-
-__global__ void check_range_kernel(const int *v, long long n, int lo, int hi, int *err) {
-    pdl_enter();
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
-        if (v[i] < lo || v[i] > hi) atomicOr(err, DEVERR_BOUNDS);
 }
 
 // h_exit[m] = h[m] for prefix rows whose exit depth equals `depth`
