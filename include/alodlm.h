@@ -41,7 +41,8 @@ extern "C" {
 #define ALODLM_ETIMEOUT (-5) /* a bounded device-side wait gave up; the step's outputs are invalid */
 #define ALODLM_ESTATE (-6)   /* call out of order (step before prefill, batch differs from prefill) */
 
-/* commit rules (the pages and the benchmark spec differ on the halting threshold) */
+/* commit rules: two readings of the halting threshold (a mean over the unresolved positions,
+   as the paper states it, or each position's own cumulative halt) */
 #define ALODLM_RULE_PAPER 0     /* commit H <= tau; stop when mean a over U >= lambda (the pages' q),
                                    or U empty, or s = K; if nothing committed in the step, commit
                                    the lowest-entropy position of the last loop */

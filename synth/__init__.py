@@ -7,7 +7,7 @@ CUDA library consume what it produces, and neither depends on the other.
 Model shapes follow the Qwen3 conversions named by the paper digest "ALoDLM: Adaptively
 Looped Diffusion Language Models" (section "Core method": 8B = Prelude layers [0,10),
 Recurrent Core [10,26), Coda [26,36)), plus two small shapes that the oracle finishes in
-seconds.  There are no trained weights and no datasets in this build: weights are drawn
+seconds.  No trained weights or datasets are used here: weights are drawn
 from seeded normals, prefix ids are uniform random ids, and the decoded block is all
 [MASK], standing in for the GSM8K prompts the paper decodes with a 16-token window.
 
