@@ -54,6 +54,15 @@ probabilities, attention output, SwiGLU output, the readout state fed to the LM 
 is rounded to bfloat16 (nearest, ties to even) at the point where the kernels round it;
 accumulation stays float64.  ``dtype=np.float32`` trades accuracy for speed at the
 Qwen3 shapes.
+
+Pins (tests/test_oracle_pins.py, CPU): brute-force primitives, entropy and sigmoid closed
+forms, the commit-disabled step against an unrolled non-shared stack, K = 1 against a plain
+masked-DLM step, the depth fallback against a position-by-position recursion, the layer and
+KV-buffer counts the pages print, halting and rule traces built by hand, Eq. 3 on the loop
+inputs, block decoding's step counts, append against one longer prefill, the sampler against
+numpy's Philox generator and a chi-square test, and planted mistakes that each fail a pin.
+The pages print no worked example with values, so absolute values on random weights are
+parity unpinned beyond these structural pins.
 """
 from __future__ import annotations
 
