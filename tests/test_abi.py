@@ -133,6 +133,12 @@ int main(void) {
   printf("%d %d %s\n", rc, h == NULL, alodlm_last_error(NULL) ? "msg" : "none");
   printf("%d\n", alodlm_denoise_step(NULL, NULL, 1, 1, 0.5f, 0.5f, 1, ALODLM_RULE_PAPER, NULL));
   printf("%s\n", alodlm_kernel_class_name(1));
+  int32_t g[4], a[5];          /* launch partitions: pure queries, callable without a GPU */
+  rc = alodlm_plan_gemm(32, 4096, 2112, g);
+  printf("%d %d %d %d %d\n", rc, g[0], g[1], g[2], g[3]);
+  rc = alodlm_plan_attention(128, 8, 1, 1056, 0, 148, 1, 0, a);
+  printf("%d %d %d %d %d\n", rc, a[0], a[2], a[3], a[4]);
+  printf("%d\n", alodlm_plan_gemm(32, 4096, 2112, NULL));
   alodlm_destroy(NULL);
   return 0;
 }
@@ -152,3 +158,6 @@ def test_plain_c_program_links_and_calls_the_library(L):
     assert out[0] == "-1 1 msg"
     assert out[1] == "-1"
     assert out[2] == "attention"
+    assert out[3] == "0 32 4 9 33"   # 33 k-tiles over 4 ranks of 9
+    assert out[4] == "0 1 8 128 1"   # one query tile, 8 key splits of one tile, remainder on the last
+    assert out[5] == "-1"
