@@ -81,6 +81,18 @@ def test_noalloc_stream_k_units_and_partials(sms):
         assert p["max_seg"] == segs, (M, N, K, sms, p, segs)
 
 
+def test_noalloc_limits_fit_its_fixed_scratch_on_a_b200():
+    """Every shape within the allocation-free GEMM's documented limits (M <= 64, N <= 32768,
+    K <= 32768) fits its fixed array on a 148-SM B200: at most 1024 tile counters and at most
+    4 Mi floats of split partials (a weight tile's partials are 128 x bn floats per segment)."""
+    Ns = sorted(set([1, 128, 129, 1000, 4096, 6144, 12288, 24576, 32640, 32768] + list(range(128, 32769, 1280))))
+    Ks = sorted(set([8, 64, 72, 880, 2112, 4096, 12288, 32760, 32768] + list(range(64, 32769, 2048))))
+    for M, N, K in itertools.product((1, 32, 33, 64), Ns, Ks):
+        p = alo.plan_gemm_noalloc(M, N, K, SMS)
+        assert p["n_tiles"] <= 1024
+        assert p["n_tiles"] * p["max_seg"] * 128 * p["bn"] <= 4 << 20, (M, N, K, p)
+
+
 def _key_cover(kv_len, a):
     s, kps = a["splits"], a["keys_per_split"]
     cover = np.zeros(kv_len, dtype=int)
