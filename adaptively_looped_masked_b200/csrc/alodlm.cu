@@ -5,6 +5,7 @@
 #include "../../include/alodlm.h"
 
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -24,6 +25,28 @@
 #include "kernels.cuh"
 
 namespace {
+
+// A named range on the host timeline (NVTX) around each phase of the library -- prefill,
+// append, denoising step, loop s of a step (payload s), block decode -- so that a profiler
+// which records NVTX (ncu --nvtx --nvtx-include) can pick out one phase's launches.  With no
+// profiler attached each push and pop is a call that returns at once.
+struct NvtxRange {
+    explicit NvtxRange(const char *name, int payload = -1) {
+        nvtxEventAttributes_t a = {};
+        a.version = NVTX_VERSION;
+        a.size = NVTX_EVENT_ATTRIB_STRUCT_SIZE;
+        a.messageType = NVTX_MESSAGE_TYPE_ASCII;
+        a.message.ascii = name;
+        if (payload >= 0) {
+            a.payloadType = NVTX_PAYLOAD_TYPE_INT32;
+            a.payload.iValue = payload;
+        }
+        nvtxRangePushEx(&a);
+    }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 // The step's linear layers and alodlm_gemm_bf16 use the per-tile kernel for few rows: on
 // B200 it streams the weights faster than the stream-K kernel at 32-64 rows (0.77 vs 0.65 of
@@ -1285,6 +1308,7 @@ int denoise_step_impl(alodlm *h, const int32_t *block_ids, int B, int N, float t
 int decode_block_impl(alodlm *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda, int k_max,
                       int rule, int max_steps, bool sampled, uint64_t seed, const alodlm_decode_out *out,
                       int *steps_taken) {
+    const NvtxRange range("alodlm decode_block");
     if (steps_taken) *steps_taken = 0;
     if (!h || !block_ids || !out || !out->tokens || !out->commit_step || !out->commit_depth || !out->steps_run ||
         !out->loops || !out->rows)
@@ -1571,6 +1595,7 @@ int exit_depths_to_host(alodlm *h, const int *exit, long long n, std::vector<int
 extern "C" {
 
 int alodlm_prefill(alodlm_t *h, const int32_t *prefix_ids, int B, int P, const int32_t *exit_depth) {
+    const NvtxRange range("alodlm prefill");
     if (!h || !prefix_ids) return fail(h, ALODLM_EINVAL, "null argument");
     const alodlm_cfg &c = h->cfg;
     if (B < 1 || B > c.max_batch || P < 1 || P > c.max_prefix)
@@ -1598,6 +1623,7 @@ int alodlm_prefill(alodlm_t *h, const int32_t *prefix_ids, int B, int P, const i
 }
 
 int alodlm_append(alodlm_t *h, const int32_t *ids, int B, int N, const int32_t *exit_depth) {
+    const NvtxRange range("alodlm append");
     if (!h || !ids) return fail(h, ALODLM_EINVAL, "null argument");
     const alodlm_cfg &c = h->cfg;
     if (!h->prefilled) return fail(h, ALODLM_ESTATE, "append before prefill");
@@ -1631,6 +1657,7 @@ namespace {
 
 int denoise_step_impl(alodlm *h, const int32_t *block_ids, int B, int N, float tau_H, float lambda, int k_max,
                       int rule, const SampleParams &sp, const alodlm_step_out *out) {
+    const NvtxRange range("alodlm step");
     if (!h || !block_ids || !out || !out->tokens || !out->exit_depth || !out->entropy || !out->halt ||
         !out->cum_halt || !out->loops_run || !out->active_rows || !out->readout_rows)
         return fail(h, ALODLM_EINVAL, "null argument");
@@ -1754,6 +1781,7 @@ int denoise_step_impl(alodlm *h, const int32_t *block_ids, int B, int N, float t
     const bool graphs = h->use_graphs && !h->timing && h->stream != nullptr && h->stream != cudaStreamLegacy &&
                         h->stream != cudaStreamPerThread;
     for (int s = 1; s <= K; ++s) {
+        const NvtxRange loop_range("alodlm loop", s);
         if (graphs) {
             const GraphKey key{s, n_act, cur, hi, N, K, rule, P, h->depth_built, tau_H, lambda, out->tokens, out->exit_depth,
                                out->entropy, out->halt, out->cum_halt, out->loops_run, out->active_rows,
